@@ -1,0 +1,343 @@
+"""Benchmark of one decoupled sparse attention step on B200: Reassign Cache + fused attention.
+
+    python bench.py [--gpus N --steps K --warmup W] [--workload wan14b] [--impl reference]
+
+A step is one pass of the whole hot path over one batch of synthetic input: da_reassign
+(reassign every key to its cached centroid, refresh the per-(block, cluster) statistics and
+the per-head totals) followed by da_attention (exact attention on the fixed blocks plus the
+cluster compensation, one fused kernel).  The metric is effective TFLOP/s, where effective
+FLOPs = sum over heads and q-blocks of 4 * |q-block| * (kept keys + C) * d; the reassignment
+is inside the timed step but its FLOPs are not counted.
+
+Under torchrun every rank runs its own copy of the workload with its own seed (heads are
+independent: weak scaling, no collective on the data path); the step time is the maximum
+over ranks of CUDA-event time.  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+import workloads as W
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+METRIC = "effective TFLOP/s & ms/call of reassign+fused sparse attn; % of bf16 TC peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# DRAM bytes per launch of the attention kernel from the last ncu capture of the current kernel
+# (None until a capture of this kernel version exists).
+ATTENTION_TRAFFIC_BYTES = None
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.dev = device_index
+
+    def __enter__(self):
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
+            sel = ["-i", uuid if uuid.startswith("GPU-") else "GPU-" + uuid]
+        except Exception:
+            sel = []
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                                          "-lms", "200", *sel], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out = ""
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in self.lines:
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    if ws > 1 and not torch.distributed.is_initialized():
+        import datetime
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def _max_over_ranks(x: float, ws: int, device) -> float:
+    if ws == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _barrier(ws: int):
+    if ws > 1:
+        torch.distributed.barrier()
+
+
+# ---------------------------------------------------------------------------
+# the fp64 oracle timed on host cores (cpu_baseline and the reference arm)
+
+def oracle_item_sampler(w: W.Workload, seed: int):
+    """Per work item (head h, q-block i): the oracle's reassignment of key block i of that head and
+    its decoupled attention for q-block i.  The complement statistics need an assignment of every
+    key of the head; the generator's own cluster labels stand in for it (the timing does not depend
+    on which valid assignment is used)."""
+    import oracle
+    b, h = 0, 0
+    q, k, v, mu = W.head_qkv(w, seed, b, h)
+    plan = W.head_plan(w, seed, b, h)
+    labels = W.head_labels(w, seed, b, h).numpy()
+    Qf, Kf, Vf, Cf = (x.float().numpy().astype(np.float64) for x in (q, k, v, mu))
+    blk_len = [min(w.block, w.N - i * w.block) for i in range(w.nB)]
+    rng = np.random.default_rng(seed)
+
+    def run(n_items: int):
+        flops = 0.0
+        t0 = time.perf_counter()
+        for _ in range(n_items):
+            i = int(rng.integers(0, w.nB))
+            s0, s1 = i * w.block, min(w.N, (i + 1) * w.block)
+            oracle.reassign(Kf[s0:s1], Cf)
+            oracle.attention_qblock(Qf, Kf, Vf, Cf, plan[i], labels, i, w.block)
+            kept = sum(blk_len[j] for j in plan[i])
+            flops += 4.0 * blk_len[i] * (kept + w.C) * w.d
+        return flops, time.perf_counter() - t0
+
+    return run
+
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        return 1
+
+
+def cpu_baseline(w: W.Workload, seed: int, budget_s: float = 12.0):
+    run = oracle_item_sampler(w, seed)
+    run(1)  # warm caches
+    flops, t, items = 0.0, 0.0, 0
+    while t < budget_s and items < 400:
+        f, dt = run(4)
+        flops += f
+        t += dt
+        items += 4
+    return {"value": flops / t / 1e12, "unit": "TFLOP/s", "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"{items} work items of head 0 (reassign of one key block + decoupled attention of one "
+                      f"q-block each, random q-blocks), fp64 numpy, {t:.1f} s"}
+
+
+def run_reference(args, w: W.Workload, ws: int, rank: int):
+    if rank != 0:
+        return
+    run = oracle_item_sampler(w, args.seed)
+    per_step = max(1, args.ref_items)
+    for _ in range(args.warmup):
+        run(per_step)
+    flops, t = 0.0, 0.0
+    for _ in range(args.steps):
+        f, dt = run(per_step)
+        flops += f
+        t += dt
+    value = flops / t / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": _config(w, args),
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": _blas_threads(), "kind": "oracle",
+                             "sample": f"{per_step} random work items of head 0 per step (reassign of one key "
+                                       f"block + decoupled attention of one q-block each), fp64 numpy"},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def _config(w: W.Workload, args):
+    return {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} ({w.T}x{w.Hs}x{w.Ws} latent) d={w.d} block={w.block} "
+                        f"C={w.C} density={w.density}",
+            "B": w.B, "H": w.H, "N": w.N, "d": w.d, "block": w.block, "C": w.C, "density": w.density,
+            "seed": args.seed, "parallelism": "independent heads per rank (weak)",
+            "l2": "inputs (Q,K,V 2.3 GB at wan14b) exceed the 126 MB L2; no flush between steps"}
+
+
+# ---------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="wan14b", choices=list(W.WORKLOADS))
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--ref-items", type=int, default=8)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    ws, rank, local = _dist()
+    w = W.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w, ws, rank)
+        if ws > 1:
+            torch.distributed.destroy_process_group()
+        return
+
+    import block_sparse_cluster_b200 as da
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    seed = args.seed + 1000 * rank
+    inp = W.make_inputs(w, seed=seed)
+    dims = da.Dims(w.B, w.H, w.N, w.d, w.C, w.block, w.torch_dtype)
+    eff = W.effective_flops(w, inp.kv_cnt, inp.kv_idx)
+
+    stream = torch.cuda.current_stream(dev)
+    eng = da.DecoupledAttention(dims, dev)
+    Q, K, V, cent = (x.to(dev) for x in (inp.Q, inp.K, inp.V, inp.centroids))
+    eng.prepare(inp.kv_idx.to(dev), inp.kv_cnt.to(dev))
+    O = torch.empty_like(Q)
+    torch.cuda.synchronize(dev)
+
+    def step(ev_pair=None):
+        da.da_reassign(dims, K, V, cent, eng.stats, eng.ws)
+        if ev_pair is not None:
+            ev_pair[0].record(stream)
+        da.da_attention(dims, Q, K, V, eng.mask, cent, eng.stats, 0.0, O, None, eng.ws)
+        if ev_pair is not None:
+            ev_pair[1].record(stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    if eng.status() != 0:
+        raise RuntimeError("device status after warm-up: " + da.da_status_string(eng.status()))
+
+    K_steps = args.steps
+    att_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K_steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    _barrier(ws)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for k in range(K_steps):
+            step(att_ev[k])
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+    _barrier(ws)
+    st = eng.status()
+    if st != 0:
+        raise RuntimeError("device status after timing: " + da.da_status_string(st))
+    ms_local = start.elapsed_time(end) / K_steps
+    att_ms_local = sum(a.elapsed_time(b) for a, b in att_ev) / K_steps
+    ms = _max_over_ranks(ms_local, ws, dev)
+    att_ms = _max_over_ranks(att_ms_local, ws, dev)
+    value = ws * eff / (ms * 1e-3) / 1e12
+
+    # end to end through the same public calls: pinned host inputs in, O back to the host
+    pinned = [x.pin_memory() for x in (inp.Q, inp.K, inp.V, inp.centroids)]
+    O_host = torch.empty(O.shape, dtype=O.dtype, pin_memory=True)
+    h2d = sum(x.numel() * x.element_size() for x in pinned)
+    d2h = O_host.numel() * O_host.element_size()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    _barrier(ws)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        for dst, src in zip((Q, K, V, cent), pinned):
+            dst.copy_(src, non_blocking=True)
+        eng.step(Q, K, V, cent, O)
+        O_host.copy_(O, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = _max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, ws, dev)
+    e2e_value = ws * eff / (e2e_ms * 1e-3) / 1e12
+
+    if rank == 0:
+        peaks, kind = _peaks()
+        peak = float(peaks["bf16_tflops"])
+        att_tflops = eff / (att_ms * 1e-3) / 1e12
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws, "steps": K_steps,
+            "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
+            "config": _config(w, args),
+            "pct_of_bf16_peak": 100.0 * (value / ws) / peak,
+            "breakdown_ms": {"reassign": ms_local - att_ms_local, "attention": att_ms_local},
+            "effective_flop_per_step_per_gpu": eff,
+            "roofline": {"bound": "tensor", "kernel": "fused decoupled attention", "achieved": att_tflops,
+                         "peak": peak, "unit": "TFLOP/s", "frac": att_tflops / peak,
+                         "peak_source": f"{kind} bf16 dense (burst)",
+                         "frac_of_sustained": att_tflops / float(peaks.get("bf16_tflops_sustained", peak)),
+                         "traffic": ATTENTION_TRAFFIC_BYTES},
+            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": K_steps * LAUNCHES_PER_STEP,
+            "clocks": clk.summary(),
+        }
+        if ws == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(w, args.seed, args.cpu_budget)
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        _barrier(ws)
+        torch.distributed.destroy_process_group()
+
+
+# kernels of ours per timed step: reassign (assignment, block statistics, totals) + attention
+LAUNCHES_PER_STEP = 4
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,184 @@
+// C ABI of libda.so: argument checks, workspace layout and kernel launches.
+// Every check happens before the first launch, so a call that returns an error launched nothing.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "da.h"
+#include "da_internal.h"
+
+using namespace da;
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+da_status check_dims(const da_dims* dims, Dims* g) {
+  if (!dims) return DA_ERR_INVALID_ARG;
+  if (dims->B <= 0 || dims->H <= 0 || dims->N <= 0 || dims->d <= 0 || dims->C <= 0 || dims->block <= 0)
+    return DA_ERR_INVALID_ARG;
+  if (dims->dtype != DA_BF16 && dims->dtype != DA_F32) return DA_ERR_DTYPE;
+  if (dims->d != 64 && dims->d != 128) return DA_ERR_UNSUPPORTED;
+  if (dims->block != 64 && dims->block != 128) return DA_ERR_UNSUPPORTED;
+  if (dims->C % 32 != 0 || dims->C > 1024) return DA_ERR_UNSUPPORTED;
+  g->B = dims->B;
+  g->H = dims->H;
+  g->N = dims->N;
+  g->d = dims->d;
+  g->C = dims->C;
+  g->block = dims->block;
+  g->nB = (dims->N + dims->block - 1) / dims->block;
+  g->bf16 = dims->dtype == DA_BF16;
+  const long long BH = (long long)dims->B * dims->H;
+  // work items and block-row indices are int32 on the device
+  if (BH * g->nB >= (1LL << 31) || BH * dims->N >= (1LL << 31)) return DA_ERR_SHAPE;
+  return DA_OK;
+}
+
+da_status check_stats(const da_cluster_stats* st, StatsPtrs* p) {
+  if (!st) return DA_ERR_INVALID_ARG;
+  if (!st->assign || !st->blk_hist || !st->seg_idx || !st->seg_n || !st->seg_c || !st->seg_cnt ||
+      !st->seg_vsum || !st->n_tot || !st->S_tot)
+    return DA_ERR_INVALID_ARG;
+  if (!aligned16(st->assign) || !aligned16(st->blk_hist) || !aligned16(st->seg_idx) || !aligned16(st->seg_n) ||
+      !aligned16(st->seg_c) || !aligned16(st->seg_cnt) || !aligned16(st->seg_vsum) || !aligned16(st->n_tot) ||
+      !aligned16(st->S_tot))
+    return DA_ERR_ALIGNMENT;
+  *p = StatsPtrs{st->assign, st->blk_hist, st->seg_idx, st->seg_n, st->seg_c,
+                 st->seg_cnt, st->seg_vsum, st->n_tot, st->S_tot};
+  return DA_OK;
+}
+
+da_status check_ws(const Dims& g, void* ws, size_t ws_bytes) {
+  if (!ws) return DA_ERR_INVALID_ARG;
+  if (!aligned16(ws)) return DA_ERR_ALIGNMENT;
+  if (ws_bytes < ws_layout(g).total) return DA_ERR_WORKSPACE;
+  return DA_OK;
+}
+
+da_status check_mask(const Dims& g, const da_block_mask* mask) {
+  if (!mask || !mask->kv_idx || !mask->kv_cnt) return DA_ERR_INVALID_ARG;
+  if (mask->max_sel < 1) return DA_ERR_SHAPE;
+  if ((long long)g.B * g.H * g.nB * mask->max_sel >= (1LL << 40)) return DA_ERR_SHAPE;
+  if (!aligned16(mask->kv_idx) || !aligned16(mask->kv_cnt)) return DA_ERR_ALIGNMENT;
+  if (mask->schedule && !aligned16(mask->schedule)) return DA_ERR_ALIGNMENT;
+  return DA_OK;
+}
+
+da_status cuda_status(cudaError_t e) { return e == cudaSuccess ? DA_OK : DA_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+int da_version(void) { return 100; }
+
+size_t da_workspace_bytes(const da_dims* dims) {
+  Dims g;
+  if (check_dims(dims, &g) != DA_OK) return 0;
+  return ws_layout(g).total;
+}
+
+size_t da_schedule_bytes(const da_dims* dims) {
+  Dims g;
+  if (check_dims(dims, &g) != DA_OK) return 0;
+  return (size_t)g.B * g.H * g.nB * sizeof(int32_t);
+}
+
+da_status da_reassign(const da_dims* dims, const void* K, const void* V, const void* centroids,
+                      const da_cluster_stats* out, void* ws, size_t ws_bytes, da_stream stream) {
+  Dims g;
+  da_status st = check_dims(dims, &g);
+  if (st != DA_OK) return st;
+  if (!K || !V || !centroids) return DA_ERR_INVALID_ARG;
+  if (!aligned16(K) || !aligned16(V) || !aligned16(centroids)) return DA_ERR_ALIGNMENT;
+  StatsPtrs sp;
+  if ((st = check_stats(out, &sp)) != DA_OK) return st;
+  if ((st = check_ws(g, ws, ws_bytes)) != DA_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = g.bf16 ? launch_assign_simt_bf16(g, K, centroids, sp.assign, s)
+                         : launch_assign_simt_f32(g, K, centroids, sp.assign, s);
+  if (e == cudaSuccess) e = launch_block_stats(g, V, sp, s);
+  if (e == cudaSuccess) e = launch_totals(g, sp, s);
+  return cuda_status(e);
+}
+
+da_status da_mask_prepare(const da_dims* dims, const da_block_mask* mask, int32_t* schedule,
+                          size_t schedule_bytes, void* ws, size_t ws_bytes, da_stream stream) {
+  Dims g;
+  da_status st = check_dims(dims, &g);
+  if (st != DA_OK) return st;
+  if ((st = check_mask(g, mask)) != DA_OK) return st;
+  if (!schedule) return DA_ERR_INVALID_ARG;
+  if (!aligned16(schedule)) return DA_ERR_ALIGNMENT;
+  if (schedule_bytes < (size_t)g.B * g.H * g.nB * sizeof(int32_t)) return DA_ERR_WORKSPACE;
+  if ((st = check_ws(g, ws, ws_bytes)) != DA_OK) return st;
+  const WsLayout L = ws_layout(g);
+  int* status = reinterpret_cast<int*>(static_cast<char*>(ws) + L.status);
+  return cuda_status(launch_schedule(g, mask->kv_idx, mask->kv_cnt, mask->max_sel, schedule, status,
+                                     reinterpret_cast<cudaStream_t>(stream)));
+}
+
+da_status da_attention(const da_dims* dims, const void* Q, const void* K, const void* V,
+                       const da_block_mask* mask, const void* centroids, const da_cluster_stats* stats,
+                       float scale, void* O, float* lse, void* ws, size_t ws_bytes, da_stream stream) {
+  Dims g;
+  da_status st = check_dims(dims, &g);
+  if (st != DA_OK) return st;
+  if (!Q || !K || !V || !centroids || !O) return DA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(centroids) || !aligned16(O) ||
+      (lse && !aligned16(lse)))
+    return DA_ERR_ALIGNMENT;
+  if ((st = check_mask(g, mask)) != DA_OK) return st;
+  StatsPtrs sp;
+  if ((st = check_stats(stats, &sp)) != DA_OK) return st;
+  if ((st = check_ws(g, ws, ws_bytes)) != DA_OK) return st;
+  if (!(scale > 0.f)) scale = 1.0f / sqrtf((float)g.d);
+  const WsLayout L = ws_layout(g);
+  int* status = reinterpret_cast<int*>(static_cast<char*>(ws) + L.status);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int32_t* sched = mask->schedule;
+  cudaError_t e = cudaSuccess;
+  if (!sched) {
+    int32_t* own = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + L.sched);
+    e = launch_schedule(g, mask->kv_idx, mask->kv_cnt, mask->max_sel, own, status, s);
+    sched = own;
+  }
+  if (e == cudaSuccess)
+    e = (g.bf16 ? launch_attention_simt_bf16 : launch_attention_simt_f32)(
+        g, Q, K, V, mask->kv_idx, mask->kv_cnt, mask->max_sel, sched, centroids, sp, scale, O, lse, status, s);
+  return cuda_status(e);
+}
+
+da_status da_device_status(void* ws, da_stream stream) {
+  if (!ws) return DA_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int word = 0;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return DA_ERR_CUDA;
+  if (cudaMemcpyAsync(&word, ws, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess) return DA_ERR_CUDA;
+  if (cudaMemsetAsync(ws, 0, sizeof(int), s) != cudaSuccess) return DA_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return DA_ERR_CUDA;
+  switch (word) {
+    case 0: return DA_OK;
+    case DA_ERR_TIMEOUT: return DA_ERR_TIMEOUT;
+    case DA_ERR_DEVICE_INDEX: return DA_ERR_DEVICE_INDEX;
+    default: return DA_ERR_CUDA;
+  }
+}
+
+const char* da_status_string(da_status s) {
+  switch (s) {
+    case DA_OK: return "ok";
+    case DA_ERR_INVALID_ARG: return "invalid argument (NULL pointer or non-positive size)";
+    case DA_ERR_SHAPE: return "inconsistent or too large shape";
+    case DA_ERR_DTYPE: return "unknown dtype";
+    case DA_ERR_ALIGNMENT: return "tensor base pointer not 16-byte aligned";
+    case DA_ERR_UNSUPPORTED: return "sizes not supported by this build (d, block or C)";
+    case DA_ERR_CUDA: return "CUDA runtime or driver call failed";
+    case DA_ERR_TIMEOUT: return "a bounded device wait gave up";
+    case DA_ERR_DEVICE_INDEX: return "malformed block plan seen on the device";
+    case DA_ERR_WORKSPACE: return "workspace or schedule buffer too small";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

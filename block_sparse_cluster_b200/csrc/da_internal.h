@@ -1,0 +1,53 @@
+// Internal launch interface between the C ABI (da_api.cu) and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "da.h"
+
+namespace da {
+
+struct StatsPtrs {
+  int32_t* assign;
+  int32_t* blk_hist;
+  uint8_t* seg_idx;
+  int32_t* seg_n;
+  int32_t* seg_c;
+  int32_t* seg_cnt;
+  float* seg_vsum;
+  int32_t* n_tot;
+  float* S_tot;
+};
+
+struct Dims {
+  int B, H, N, d, C, block, nB;
+  bool bf16;
+};
+
+// Workspace layout (byte offsets), shared by every call.
+struct WsLayout {
+  size_t status, norms, sched, total;
+};
+WsLayout ws_layout(const Dims& g);
+
+// stats.cu
+cudaError_t launch_centroid_norms(const Dims& g, const void* cent, float* norms, cudaStream_t s);
+cudaError_t launch_block_stats(const Dims& g, const void* V, const StatsPtrs& st, cudaStream_t s);
+cudaError_t launch_totals(const Dims& g, const StatsPtrs& st, cudaStream_t s);
+cudaError_t launch_schedule(const Dims& g, const int32_t* kv_idx, const int32_t* kv_cnt, int max_sel,
+                            int32_t* schedule, int* status, cudaStream_t s);
+
+// simt_f32.cu / simt_bf16.cu
+#define DA_SIMT_DECL(SUFFIX)                                                                                 \
+  cudaError_t launch_assign_simt_##SUFFIX(const Dims& g, const void* K, const void* cent, int32_t* assign,    \
+                                          cudaStream_t s);                                                    \
+  cudaError_t launch_attention_simt_##SUFFIX(const Dims& g, const void* Q, const void* K, const void* V,      \
+                                             const int32_t* kv_idx, const int32_t* kv_cnt, int max_sel,       \
+                                             const int32_t* schedule, const void* cent, const StatsPtrs& st,  \
+                                             float scale, void* O, float* lse, int* status, cudaStream_t s);
+DA_SIMT_DECL(f32)
+DA_SIMT_DECL(bf16)
+#undef DA_SIMT_DECL
+
+}  // namespace da

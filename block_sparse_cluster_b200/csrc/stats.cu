@@ -1,0 +1,183 @@
+// Reassign Cache statistics and plan kernels shared by the fp32 and bf16 paths: centroid norms,
+// per-block statistics, per-head totals, plan validation and work order.
+#include <math.h>
+
+#include "block_stats.cuh"
+#include "da_common.cuh"
+#include "da_internal.h"
+
+namespace da {
+
+WsLayout ws_layout(const Dims& g) {
+  auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  WsLayout L;
+  const size_t BH = (size_t)g.B * g.H;
+  L.status = 0;
+  L.norms = 256;
+  L.sched = L.norms + up(BH * g.C * sizeof(float));
+  L.total = L.sched + up(BH * g.nB * sizeof(int32_t));
+  return L;
+}
+
+// ||cbar_c||^2 in fp32 from the stored centroids; one warp per centroid, fixed reduction order.
+template <typename T>
+__global__ void centroid_norms_kernel(const T* __restrict__ cent, float* __restrict__ norms, long long rows, int d) {
+  const long long r = (long long)blockIdx.x * 4 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (r >= rows) return;
+  const T* c = cent + r * d;
+  float s = 0.f;
+  for (int t = lane; t < d; t += 32) {
+    const float x = to_f32(c[t]);
+    s = fmaf(x, x, s);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (lane == 0) norms[r] = s;
+}
+
+// Per-block statistics from an existing assignment: one CTA of 128 threads per (head, block).
+template <typename T, int D>
+__global__ void __launch_bounds__(128) block_stats_kernel(const T* __restrict__ V, StatsPtrs st, int N, int C,
+                                                          int block, int nB) {
+  __shared__ StatsSmem sm;
+  __shared__ int s_assign[128];
+  const int bh = blockIdx.y, j = blockIdx.x;
+  const int k0 = j * block;
+  const int nk = min(block, N - k0);
+  const int t = threadIdx.x;
+  if (t < nk) s_assign[t] = st.assign[(size_t)bh * N + k0 + t];
+  __syncthreads();
+  const size_t bj = (size_t)bh * nB + j;
+  block_stats_group<T, D>(t, 1, s_assign, nk, V + ((size_t)bh * N + k0) * D, C, st.blk_hist + bj * C,
+                          st.seg_idx + bj * C, st.seg_n + bj, st.seg_c + bj * block, st.seg_cnt + bj * block,
+                          st.seg_vsum + bj * block * D, sm);
+}
+
+// Per-head totals n_c, S_c = sum over blocks of the block entries, in a fixed order.
+// CTA (head, 32 clusters); warp w walks blocks j = w, w+4, ...; partial sums per warp are
+// combined in warp order.
+template <int D>
+__global__ void __launch_bounds__(128) totals_kernel(StatsPtrs st, int C, int block, int nB) {
+  extern __shared__ float part[];   // [4][32][D]
+  __shared__ int cnt[4][32];
+  const int bh = blockIdx.x, c0 = blockIdx.y * 32;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int NE = D / 32;
+  float* mine = part + (size_t)warp * 32 * D;
+  for (int x = lane; x < 32 * D; x += 32) mine[x] = 0.f;
+  __syncwarp();
+  int my_n = 0;
+  for (int j = warp; j < nB; j += 4) {
+    const size_t bj = (size_t)bh * nB + j;
+    const int e = st.seg_idx[bj * C + c0 + lane];
+    unsigned m = __ballot_sync(0xffffffffu, e != 0xFF);
+    if (e != 0xFF) my_n += st.seg_cnt[bj * block + e];
+    while (m) {
+      const int L = __ffs(m) - 1;
+      m &= m - 1;
+      const int eL = __shfl_sync(0xffffffffu, e, L);
+      const float* src = st.seg_vsum + (bj * block + eL) * D + lane * NE;
+      float* dst = mine + L * D + lane * NE;
+#pragma unroll
+      for (int i = 0; i < NE; ++i) dst[i] += src[i];
+    }
+  }
+  cnt[warp][lane] = my_n;
+  __syncthreads();
+  for (int x = threadIdx.x; x < 32 * D; x += 128) {
+    const float s = ((part[x] + part[32 * D + x]) + part[2 * 32 * D + x]) + part[3 * 32 * D + x];
+    st.S_tot[((size_t)bh * C + c0) * D + x] = s;
+  }
+  if (threadIdx.x < 32) {
+    const int l = threadIdx.x;
+    st.n_tot[(size_t)bh * C + c0 + l] = cnt[0][l] + cnt[1][l] + cnt[2][l] + cnt[3][l];
+  }
+}
+
+// Plan validation and work order: items of a head ordered by descending row length
+// (ties by q-block index); heads in order.  A malformed row is reported and scheduled with
+// cost 0 (the attention kernels skip its invalid entries).
+__global__ void schedule_kernel(const int32_t* __restrict__ kv_idx, const int32_t* __restrict__ kv_cnt,
+                                int max_sel, int nB, int32_t* __restrict__ schedule, int* status) {
+  extern __shared__ int cost[];
+  const int bh = blockIdx.x;
+  for (int i = threadIdx.x; i < nB; i += blockDim.x) {
+    const size_t item = (size_t)bh * nB + i;
+    const int cnt = kv_cnt[item];
+    bool ok = cnt >= 0 && cnt <= max_sel;
+    if (ok) {
+      int prev = -1;
+      const int32_t* row = kv_idx + item * max_sel;
+      for (int s = 0; s < cnt; ++s) {
+        const int j = row[s];
+        if (j <= prev || j >= nB) { ok = false; break; }
+        prev = j;
+      }
+    }
+    if (!ok) set_status(status, DA_ERR_DEVICE_INDEX);
+    cost[i] = ok ? cnt : 0;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < nB; i += blockDim.x) {
+    const int ci = cost[i];
+    int rank = 0;
+    for (int i2 = 0; i2 < nB; ++i2) {
+      const int c2 = cost[i2];
+      rank += (c2 > ci) || (c2 == ci && i2 < i);
+    }
+    schedule[(size_t)bh * nB + rank] = bh * nB + i;
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// launches
+
+cudaError_t launch_centroid_norms(const Dims& g, const void* cent, float* norms, cudaStream_t s) {
+  const long long rows = (long long)g.B * g.H * g.C;
+  const unsigned grid = (unsigned)((rows + 3) / 4);
+  if (g.bf16)
+    centroid_norms_kernel<<<grid, 128, 0, s>>>((const __nv_bfloat16*)cent, norms, rows, g.d);
+  else
+    centroid_norms_kernel<<<grid, 128, 0, s>>>((const float*)cent, norms, rows, g.d);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_block_stats(const Dims& g, const void* V, const StatsPtrs& st, cudaStream_t s) {
+  dim3 grid(g.nB, g.B * g.H);
+#define DA_STATS(T, DD) block_stats_kernel<T, DD><<<grid, 128, 0, s>>>((const T*)V, st, g.N, g.C, g.block, g.nB)
+  if (g.bf16) {
+    if (g.d == 128) DA_STATS(__nv_bfloat16, 128); else DA_STATS(__nv_bfloat16, 64);
+  } else {
+    if (g.d == 128) DA_STATS(float, 128); else DA_STATS(float, 64);
+  }
+#undef DA_STATS
+  return cudaGetLastError();
+}
+
+cudaError_t launch_totals(const Dims& g, const StatsPtrs& st, cudaStream_t s) {
+  dim3 grid(g.B * g.H, g.C / 32);
+  const size_t smem = (size_t)4 * 32 * g.d * sizeof(float);
+  cudaError_t e;
+  if (g.d == 128) {
+    e = cudaFuncSetAttribute(totals_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    totals_kernel<128><<<grid, 128, smem, s>>>(st, g.C, g.block, g.nB);
+  } else {
+    totals_kernel<64><<<grid, 128, smem, s>>>(st, g.C, g.block, g.nB);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_schedule(const Dims& g, const int32_t* kv_idx, const int32_t* kv_cnt, int max_sel,
+                            int32_t* schedule, int* status, cudaStream_t s) {
+  const size_t smem = (size_t)g.nB * sizeof(int);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(schedule_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  schedule_kernel<<<g.B * g.H, 256, smem, s>>>(kv_idx, kv_cnt, max_sel, g.nB, schedule, status);
+  return cudaGetLastError();
+}
+
+}  // namespace da

@@ -1,0 +1,175 @@
+/*
+ * da.h -- C ABI of the decoupled sparse attention library (libda.so).
+ *
+ * The method ("DecoupAttn: Decoupled Sparse Attention for Training-Free
+ * Acceleration of Video Diffusion", abstract) runs exact softmax attention on
+ * a few key blocks per query block, fixed once offline by position, and
+ * compensates every other key through a semantic cluster.  Each denoising
+ * step first runs Reassign Cache: the drifting keys are reassigned to cached
+ * centroids and the compensation statistics are refreshed while the planned
+ * blocks stay fixed.  Inference then runs block-sparse attention with one
+ * fused compensation.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Tensors are dense, row-major, on the current CUDA device, owned by the
+ *   caller.  The library allocates no memory and keeps no state between calls.
+ * - Q, K, V are [B, H, N, d] with d contiguous; centroids are [B, H, C, d].
+ *   Element type: dims.dtype (bf16 or fp32); every base pointer must be
+ *   16-byte aligned.
+ * - Key block j of a head holds tokens [j*block, min((j+1)*block, N)); the
+ *   last block may be short; nB = ceil(N / block).  Query blocks use the same
+ *   partition.
+ * - Calls are asynchronous on the given stream (NULL = legacy default
+ *   stream).  Argument checks are synchronous: a call that returns an error
+ *   code launched nothing.  Problems found on the device (an out-of-range or
+ *   unsorted block index, a bounded wait that gave up) are recorded in a
+ *   status word inside the workspace; da_device_status() reports them.
+ * - Supported sizes: d in {64, 128}; block in {64, 128}; C a multiple of 32,
+ *   32 <= C <= 1024; N >= 1.  The bf16 tensor-core path needs d = 128 and
+ *   block = 128; fp32 runs d in {64, 128}, block in {64, 128}.
+ */
+#ifndef DA_H
+#define DA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define DA_API __attribute__((visibility("default")))
+#else
+#define DA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream (cudaStream_t); NULL is the legacy default stream. */
+typedef struct CUstream_st* da_stream;
+
+typedef enum {
+  DA_OK = 0,
+  DA_ERR_INVALID_ARG = 1,   /* a required pointer is NULL, or a size is not positive */
+  DA_ERR_SHAPE = 2,         /* sizes that contradict each other (max_sel < 1, ...) */
+  DA_ERR_DTYPE = 3,         /* dtype not one of da_dtype */
+  DA_ERR_ALIGNMENT = 4,     /* a tensor base pointer is not 16-byte aligned */
+  DA_ERR_UNSUPPORTED = 5,   /* valid sizes this build has no kernel for (d, block, C) */
+  DA_ERR_CUDA = 6,          /* a CUDA runtime or driver call failed (launch, tensor map) */
+  DA_ERR_TIMEOUT = 7,       /* a bounded device-side wait gave up (from da_device_status) */
+  DA_ERR_DEVICE_INDEX = 8,  /* the device found a block index out of range, unsorted or repeated,
+                               or kv_cnt outside [0, max_sel] (from da_device_status) */
+  DA_ERR_WORKSPACE = 9      /* workspace or schedule buffer too small */
+} da_status;
+
+typedef enum { DA_BF16 = 0, DA_F32 = 1 } da_dtype;
+
+typedef struct {
+  int B, H;        /* batch, heads (each (b, h) has its own centroids, plan and statistics) */
+  int N;           /* tokens per head (queries = keys) */
+  int d;           /* head dimension */
+  int C;           /* cached centroids (clusters) per head */
+  int block;       /* block size Bs of the q/kv partition */
+  da_dtype dtype;  /* element type of Q, K, V, centroids and O */
+} da_dims;
+
+/*
+ * Reassign Cache output (DecoupAttn abstract: "reassigns the drifting keys to
+ * cached centroids and refreshes compensation").  All buffers are caller
+ * owned and written in full by da_reassign; nB = ceil(N / block).
+ */
+typedef struct {
+  int32_t* assign;    /* [B,H,N]          nearest centroid of every key (ties -> lowest index) */
+  int32_t* blk_hist;  /* [B,H,nB,C]       n_{c,j}: keys of block j in cluster c */
+  uint8_t* seg_idx;   /* [B,H,nB,C]       entry of cluster c in block j's list, 0xFF if absent */
+  int32_t* seg_n;     /* [B,H,nB]         number of entries (distinct clusters) of block j */
+  int32_t* seg_c;     /* [B,H,nB,block]   cluster of each entry, ascending; first seg_n valid */
+  int32_t* seg_cnt;   /* [B,H,nB,block]   keys per entry */
+  float*   seg_vsum;  /* [B,H,nB,block,d] fp32 sum of the entry's value rows */
+  int32_t* n_tot;     /* [B,H,C]          n_c = sum_j n_{c,j} */
+  float*   S_tot;     /* [B,H,C,d]        S_c = sum of the value rows of cluster c (fp32) */
+} da_cluster_stats;
+
+/*
+ * Fixed block plan ("a few blocks fixed once offline by position",
+ * DecoupAttn abstract).  Row (b, h, i) lists the kv blocks q-block i attends
+ * exactly: kv_idx[b][h][i][0 .. kv_cnt[b][h][i]-1], strictly increasing, each
+ * in [0, nB).  A row may be empty (pure compensation) or hold every block
+ * (dense attention).  `schedule` is optional: the work order written by
+ * da_mask_prepare for this plan (the plan is fixed across steps), or NULL to
+ * let da_attention build it in its workspace on every call.
+ */
+typedef struct {
+  const int32_t* kv_idx;    /* [B,H,nB,max_sel] device int32 */
+  const int32_t* kv_cnt;    /* [B,H,nB] device int32 */
+  int max_sel;              /* row capacity of kv_idx, >= 1 */
+  const int32_t* schedule;  /* [B*H*nB] device int32 from da_mask_prepare, or NULL */
+} da_block_mask;
+
+/* Version of this ABI (major*100 + minor). */
+DA_API int da_version(void);
+
+/* Bytes of device workspace da_reassign and da_attention need for these dims
+ * (status word, centroid norms, work order).  Returns 0 for invalid dims.
+ * The workspace must be zero-filled once before its first use; afterwards
+ * the library keeps it consistent itself. */
+DA_API size_t da_workspace_bytes(const da_dims* dims);
+
+/* Bytes of the schedule buffer da_mask_prepare writes (B*H*nB int32). */
+DA_API size_t da_schedule_bytes(const da_dims* dims);
+
+/*
+ * Reassign Cache.  For every key k of every head: assign[k] = argmin_c
+ * ||k - cbar_c||^2 (squared Euclidean, as in Lloyd's least-squares
+ * quantisation; ties to the lowest index), then the per-(block, cluster)
+ * counts, the sorted per-block entry lists with their fp32 value sums, and
+ * the per-head totals n_c and S_c.  bf16 inputs: distances from a bf16
+ * tensor-core contraction with fp32 accumulation, ||cbar||^2 in fp32.
+ * K, V: [B,H,N,d]; centroids: [B,H,C,d]; out: every pointer non-NULL.
+ * The totals are reduced in a fixed order (no floating-point atomics), so
+ * the call is deterministic.
+ */
+DA_API da_status da_reassign(const da_dims* dims, const void* K, const void* V, const void* centroids,
+                      const da_cluster_stats* out, void* ws, size_t ws_bytes, da_stream stream);
+
+/*
+ * Validate a fixed block plan on the device and write its work order:
+ * items (b, h, i) head-major, and within a head longest row first.  Call it
+ * once per plan; pass the buffer as da_block_mask.schedule afterwards.
+ * A malformed row sets DA_ERR_DEVICE_INDEX in the workspace status word.
+ */
+DA_API da_status da_mask_prepare(const da_dims* dims, const da_block_mask* mask, int32_t* schedule,
+                          size_t schedule_bytes, void* ws, size_t ws_bytes, da_stream stream);
+
+/*
+ * Decoupled sparse attention (DecoupAttn abstract: exact attention on the
+ * fixed blocks, every other key compensated through its cluster, in one
+ * fused pass).  For query q of q-block i with selected blocks sel(i):
+ *   exact logits     s * q.k            for keys k in the selected blocks,
+ *   cluster logits   s * q.cbar_c + ln n^U_c   for clusters with n^U_c > 0,
+ * where n^U_c = n_c - sum_{j in sel(i)} n_{c,j} counts the cluster's keys
+ * outside the selected blocks and its value is the mean of their values,
+ * vbar^U_c = (S_c - sum_{j in sel(i)} S_{c,j}) / n^U_c.  One online softmax
+ * runs over both kinds of logits with fp32 accumulation; O = [B,H,N,d] in
+ * dims.dtype; lse (nullable) = [B,H,N] fp32 natural-log sum of exponentials.
+ * scale <= 0 selects 1/sqrt(d).  stats must come from da_reassign on the
+ * same K, V, centroids.
+ */
+DA_API da_status da_attention(const da_dims* dims, const void* Q, const void* K, const void* V,
+                       const da_block_mask* mask, const void* centroids,
+                       const da_cluster_stats* stats, float scale, void* O, float* lse,
+                       void* ws, size_t ws_bytes, da_stream stream);
+
+/* Synchronise `stream`, then report and clear the workspace status word:
+ * DA_OK, DA_ERR_TIMEOUT or DA_ERR_DEVICE_INDEX (or DA_ERR_CUDA if the
+ * synchronisation itself failed). */
+DA_API da_status da_device_status(void* ws, da_stream stream);
+
+/* Static description of a status code. */
+DA_API const char* da_status_string(da_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DA_H */

@@ -1,0 +1,194 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle on the same seeded inputs."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+from tests import parity as P
+
+pytestmark = pytest.mark.gpu
+
+# Small cases the oracle finishes in seconds; each spans several tiles and ends in a ragged block.
+SMALL = {
+    # fp32, d=64, block 64, 16 full blocks, C=32 (the tiny workload itself)
+    "tiny": W.WORKLOADS["tiny"],
+    # fp32, d=128, block 128: N = 5*15*16 = 1200 -> 10 blocks, last one 48 keys
+    "f32_d128_ragged": W.scaled(W.WORKLOADS["tiny"], d=128, block=128, T=5, Hs=15, C=64),
+    # bf16 Wan2.1-1.3B shape cut to 3 frames: N = 4680, 37 blocks, last one 72 keys, C=256
+    "wan13b_3f": W.scaled(W.WORKLOADS["wan13b"], H=2, T=3),
+    # bf16 Wan2.1-14B shape cut to 2 frames: N = 7200, 57 blocks, last one 32 keys, C=512
+    "wan14b_2f": W.scaled(W.WORKLOADS["wan14b"], H=2, T=2),
+    # bf16 HunyuanVideo shape cut to 3 frames: N = 10800, 85 blocks, last one 48 keys, C=1024
+    "hunyuan_3f": W.scaled(W.WORKLOADS["hunyuan"], H=1, T=3),
+}
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_small_case_full_parity(name):
+    w = SMALL[name]
+    inp = W.make_inputs(w, seed=7)
+    eng, O, lse = P.run_gpu(inp)
+    assert eng.status() == 0
+    st = eng.stats
+    assign = st.assign.cpu().numpy()
+    for b in range(w.B):
+        for h in range(w.H):
+            a = assign[b, h].astype(np.int64)
+            P.check_assignment(inp, b, h, a)
+            P.check_block_stats(inp, b, h, st, a)
+            P.check_totals(inp, b, h, st, a)
+            P.check_attention(inp, b, h, O, lse, a)
+
+
+def _edge_plan(w, rows):
+    kv_idx, kv_cnt = W.pack_plan([[rows] * w.H] * w.B, w.nB)
+    return kv_idx, kv_cnt
+
+
+@pytest.mark.parametrize("name", ["tiny", "wan13b_3f"])
+def test_empty_full_and_offset_rows(name):
+    """Rows with no block (pure compensation), every block (dense), and plans without the own block."""
+    w = SMALL[name]
+    inp = W.make_inputs(w, seed=8)
+    nB = w.nB
+    rows = []
+    for i in range(nB):
+        if i % 3 == 0:
+            rows.append(np.zeros(0, np.int32))
+        elif i % 3 == 1:
+            rows.append(np.arange(nB, dtype=np.int32))
+        else:
+            rows.append(np.array(sorted({(i + 5) % nB, (i + 9) % nB}), np.int32))
+    inp.plans = [[rows] * w.H] * w.B
+    inp.kv_idx, inp.kv_cnt = _edge_plan(w, rows)
+    eng, O, lse = P.run_gpu(inp)
+    assert eng.status() == 0
+    a = eng.stats.assign.cpu().numpy()
+    for h in range(w.H):
+        P.check_attention(inp, 0, h, O, lse, a[0, h].astype(np.int64))
+
+
+def test_full_plan_equals_dense_attention():
+    w = SMALL["wan13b_3f"]
+    inp = W.make_inputs(w, seed=9)
+    rows = [np.arange(w.nB, dtype=np.int32)] * w.nB
+    inp.kv_idx, inp.kv_cnt = _edge_plan(w, rows)
+    _, O, _ = P.run_gpu(inp)
+    q, k, v = (x.cuda().float() for x in (inp.Q, inp.K, inp.V))
+    dense = torch.nn.functional.scaled_dot_product_attention(q, k, v)
+    assert (O.float() - dense).abs().max().item() <= P.ATT_TOL["bf16"]
+
+
+def test_singleton_clusters_equal_dense_attention():
+    """C = N and the centroids are the keys: every cluster holds one key, so the result is dense."""
+    w = W.scaled(W.WORKLOADS["tiny"], T=1, Hs=16, Ws=16, C=256, block=64)
+    inp = W.make_inputs(w, seed=10)
+    inp.centroids = inp.K.clone()
+    eng, O, _ = P.run_gpu(inp)
+    a = eng.stats.assign.cpu().numpy()
+    assert np.array_equal(a[0, 0], np.arange(256))
+    q, k, v = (x.double() for x in (inp.Q, inp.K, inp.V))
+    dense = torch.nn.functional.scaled_dot_product_attention(q, k, v)
+    assert (O.cpu().double() - dense).abs().max().item() <= P.ATT_TOL["f32"]
+
+
+def test_explicit_scale_and_no_lse():
+    import block_sparse_cluster_b200 as da
+    w = SMALL["tiny"]
+    inp = W.make_inputs(w, seed=11)
+    dims = P.dims_of(w)
+    eng = da.DecoupledAttention(dims)
+    Q, K, V, cent = (x.cuda() for x in (inp.Q, inp.K, inp.V, inp.centroids))
+    eng.prepare(inp.kv_idx.cuda(), inp.kv_cnt.cuda())
+    O = torch.empty_like(Q)
+    eng.step(Q, K, V, cent, O, None, scale=0.05)
+    assert eng.status() == 0
+    a = eng.stats.assign.cpu().numpy()
+    for h in range(w.H):
+        ref = oracle.attention(inp.Q[0, h], inp.K[0, h], inp.V[0, h], inp.centroids[0, h], inp.plans[0][h],
+                               a[0, h], w.block, scale=0.05)
+        assert np.abs(O[0, h].cpu().numpy() - ref).max() <= P.ATT_TOL["f32"]
+
+
+def test_short_sequence_single_partial_block():
+    w = W.scaled(W.WORKLOADS["tiny"], T=1, Hs=10, Ws=10, C=32)      # N = 100: blocks of 64 and 36
+    inp = W.make_inputs(w, seed=12)
+    eng, O, lse = P.run_gpu(inp)
+    a = eng.stats.assign.cpu().numpy()
+    for h in range(w.H):
+        ah = a[0, h].astype(np.int64)
+        P.check_assignment(inp, 0, h, ah)
+        P.check_block_stats(inp, 0, h, eng.stats, ah)
+        P.check_attention(inp, 0, h, O, lse, ah)
+
+
+def test_repeat_calls_are_bitwise_identical():
+    w = SMALL["wan13b_3f"]
+    inp = W.make_inputs(w, seed=13)
+    eng, O1, l1 = P.run_gpu(inp)
+    s1 = {k: getattr(eng.stats, k).clone() for k in ("assign", "blk_hist", "seg_vsum", "S_tot", "n_tot")}
+    Q, K, V, cent = (x.cuda() for x in (inp.Q, inp.K, inp.V, inp.centroids))
+    O2 = torch.empty_like(O1)
+    l2 = torch.empty_like(l1)
+    eng.step(Q, K, V, cent, O2, l2)
+    torch.cuda.synchronize()
+    assert torch.equal(O1, O2) and torch.equal(l1, l2)
+    for k, v in s1.items():
+        assert torch.equal(v, getattr(eng.stats, k)), k
+
+
+def test_malformed_plan_is_reported_without_fault():
+    import block_sparse_cluster_b200 as da
+    w = SMALL["tiny"]
+    inp = W.make_inputs(w, seed=14)
+    ki = inp.kv_idx.clone()
+    kc = inp.kv_cnt.clone()
+    ki[0, 0, 3, 0] = 10_000          # out of range
+    ki[0, 1, 5, :2] = torch.tensor([7, 2], dtype=torch.int32)   # unsorted
+    eng, O, _ = P.run_gpu(inp, kv_idx=ki, kv_cnt=kc)
+    assert eng.status() == da.STATUS_NAMES.index("DA_ERR_DEVICE_INDEX")
+    assert eng.status() == 0           # cleared by the read
+    kc2 = inp.kv_cnt.clone()
+    kc2[0, 0, 0] = 99                  # more than max_sel
+    eng, _, _ = P.run_gpu(inp, kv_cnt=kc2)
+    assert eng.status() == da.STATUS_NAMES.index("DA_ERR_DEVICE_INDEX")
+    # the same plan without da_mask_prepare: da_attention validates it itself
+    eng, _, _ = P.run_gpu(inp, kv_idx=ki, kv_cnt=kc, prepare=False)
+    assert eng.status() == da.STATUS_NAMES.index("DA_ERR_DEVICE_INDEX")
+
+
+# ---------------------------------------------------------------------------
+# full-size workloads, in the launch configuration the benchmark times: sampled outputs
+
+FULL = ["wan13b", "wan14b", "hunyuan"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_sampled(name):
+    w = W.WORKLOADS[name]
+    inp = W.make_inputs(w, seed=0)
+    eng, O, lse = P.run_gpu(inp)
+    assert eng.status() == 0
+    st = eng.stats
+    rng = np.random.default_rng(1)
+    # properties over every head
+    sizes = torch.full((w.nB,), w.block, dtype=torch.int64, device="cuda")
+    sizes[-1] = w.N - (w.nB - 1) * w.block
+    assert torch.equal(st.blk_hist.sum(-1).long(), sizes.expand(w.B, w.H, -1))
+    assert torch.equal(st.blk_hist.sum(2), st.n_tot)
+    assert (st.n_tot.sum(-1) == w.N).all()
+    assert torch.isfinite(O.float()).all() and torch.isfinite(lse).all()
+    assign = st.assign.cpu().numpy()
+    heads = sorted(set([0, w.H - 1] + rng.choice(w.H, size=2, replace=False).tolist()))
+    for h in heads:
+        a = assign[0, h].astype(np.int64)
+        keys = np.concatenate([rng.choice(w.N, size=512, replace=False), np.arange(w.N - 16, w.N)])
+        P.check_assignment(inp, 0, h, a, keys=keys)
+        blocks = sorted(set(rng.choice(w.nB, size=12, replace=False).tolist() + [w.nB - 1]))
+        P.check_block_stats(inp, 0, h, st, a, blocks=blocks)
+        P.check_totals(inp, 0, h, st, a)
+        qbs = sorted(set(rng.choice(w.nB, size=6, replace=False).tolist() + [0, w.nB - 1]))
+        P.check_attention(inp, 0, h, O, lse, a, q_blocks=qbs)
