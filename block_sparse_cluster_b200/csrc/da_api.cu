@@ -95,9 +95,18 @@ da_status da_reassign(const da_dims* dims, const void* K, const void* V, const v
   if ((st = check_stats(out, &sp)) != DA_OK) return st;
   if ((st = check_ws(g, ws, ws_bytes)) != DA_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = g.bf16 ? launch_assign_simt_bf16(g, K, centroids, sp.assign, s)
-                         : launch_assign_simt_f32(g, K, centroids, sp.assign, s);
-  if (e == cudaSuccess) e = launch_block_stats(g, V, sp, s);
+  const WsLayout L = ws_layout(g);
+  int* status = reinterpret_cast<int*>(static_cast<char*>(ws) + L.status);
+  float* norms = reinterpret_cast<float*>(static_cast<char*>(ws) + L.norms);
+  cudaError_t e;
+  if (reassign_tc_supported(g)) {
+    e = launch_centroid_norms(g, centroids, norms, s);
+    if (e == cudaSuccess) e = launch_reassign_tc(g, K, V, centroids, norms, sp, status, s);
+  } else {
+    e = g.bf16 ? launch_assign_simt_bf16(g, K, centroids, sp.assign, s)
+               : launch_assign_simt_f32(g, K, centroids, sp.assign, s);
+    if (e == cudaSuccess) e = launch_block_stats(g, V, sp, s);
+  }
   if (e == cudaSuccess) e = launch_totals(g, sp, s);
   return cuda_status(e);
 }
@@ -143,9 +152,14 @@ da_status da_attention(const da_dims* dims, const void* Q, const void* K, const 
     e = launch_schedule(g, mask->kv_idx, mask->kv_cnt, mask->max_sel, own, status, s);
     sched = own;
   }
-  if (e == cudaSuccess)
-    e = (g.bf16 ? launch_attention_simt_bf16 : launch_attention_simt_f32)(
-        g, Q, K, V, mask->kv_idx, mask->kv_cnt, mask->max_sel, sched, centroids, sp, scale, O, lse, status, s);
+  if (e == cudaSuccess) {
+    if (attention_tc_supported(g))
+      e = launch_attention_tc(g, Q, K, V, mask->kv_idx, mask->kv_cnt, mask->max_sel, sched, centroids, sp, scale,
+                              O, lse, status, s);
+    else
+      e = (g.bf16 ? launch_attention_simt_bf16 : launch_attention_simt_f32)(
+          g, Q, K, V, mask->kv_idx, mask->kv_cnt, mask->max_sel, sched, centroids, sp, scale, O, lse, status, s);
+  }
   return cuda_status(e);
 }
 

@@ -121,6 +121,21 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   return false;
 }
 
+// Wait for the tensor core or the TMA unit to finish work already issued, whether or not the
+// CTA aborted (so that no copy or MMA is still in flight when the CTA frees its memory).
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+  unsigned long long t0 = 0;
+  for (unsigned int it = 0; it < kWaitPolls; ++it) {
+    if (mbar_test(bar, parity)) return true;
+    if ((it & 255u) == 255u) {
+      unsigned long long now = global_ns();
+      if (t0 == 0) t0 = now;
+      else if (now - t0 > kWaitNs) break;
+    }
+  }
+  return false;
+}
+
 // TMA --------------------------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

@@ -38,6 +38,18 @@ cudaError_t launch_totals(const Dims& g, const StatsPtrs& st, cudaStream_t s);
 cudaError_t launch_schedule(const Dims& g, const int32_t* kv_idx, const int32_t* kv_cnt, int max_sel,
                             int32_t* schedule, int* status, cudaStream_t s);
 
+// reassign_tc.cu
+bool reassign_tc_supported(const Dims& g);
+cudaError_t launch_reassign_tc(const Dims& g, const void* K, const void* V, const void* cent, const float* norms,
+                               const StatsPtrs& st, int* status, cudaStream_t s);
+
+// attention_tc.cu
+bool attention_tc_supported(const Dims& g);
+cudaError_t launch_attention_tc(const Dims& g, const void* Q, const void* K, const void* V,
+                                const int32_t* kv_idx, const int32_t* kv_cnt, int max_sel,
+                                const int32_t* schedule, const void* cent, const StatsPtrs& st, float scale,
+                                void* O, float* lse, int* status, cudaStream_t s);
+
 // simt_f32.cu / simt_bf16.cu
 #define DA_SIMT_DECL(SUFFIX)                                                                                 \
   cudaError_t launch_assign_simt_##SUFFIX(const Dims& g, const void* K, const void* cent, int32_t* assign,    \

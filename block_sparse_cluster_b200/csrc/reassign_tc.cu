@@ -1,0 +1,186 @@
+// Reassign Cache on the tensor cores (bf16, d = 128, block = 128).
+//
+// "each step reassigns the drifting keys to cached centroids and refreshes compensation"
+// (DecoupAttn abstract).  One CTA per (head, key block of 128 keys):
+//   1. TMA loads the key tile (128 x 128 bf16, 128-byte swizzle) and the centroid chunks
+//      (256 x 128 bf16 each, double buffered).
+//   2. One thread issues tcgen05.mma: D[key, c] = k . cbar_c into TMEM (fp32, 256 columns per
+//      chunk, two TMEM buffers so the next chunk's contraction overlaps this chunk's epilogue).
+//   3. Every thread owns one key (= one TMEM lane) and keeps the running argmin of
+//      ||cbar_c||^2 - 2 k.cbar_c (ties to the lowest c; the key's own norm is the same for
+//      every c and is dropped).
+//   4. The same 128 threads refresh the block's statistics (block_stats.cuh): sorted entry list,
+//      histogram row, entry index row and fp32 value sums.
+#include "block_stats.cuh"
+#include "da_common.cuh"
+#include "da_internal.h"
+#include "tma_host.h"
+
+namespace da {
+
+namespace {
+
+constexpr int kKeys = 128;           // keys per tile (= block)
+constexpr int kD = 128;              // head dimension
+constexpr int kChunk = 256;          // centroids per MMA chunk (N of the MMA)
+constexpr int kKTileBytes = kKeys * kD * 2;        // 32 KB
+constexpr int kCTileBytes = kChunk * kD * 2;       // 64 KB
+constexpr int kPanelK = kKeys * 128;               // one 64-column panel of the key tile
+constexpr int kPanelC = kChunk * 128;              // one 64-column panel of a centroid chunk
+
+struct __align__(8) Bars {
+  uint64_t kfull;
+  uint64_t cfull[2];
+  uint64_t mdone[2];
+  uint32_t tmem_base;
+  int abort;
+};
+
+constexpr size_t kSmemBytes = 1024 /*align slack*/ + kKTileBytes + 2 * kCTileBytes + 4096 /*norms*/ +
+                              sizeof(StatsSmem) + 512 /*assign*/ + 128 /*bars*/;
+
+__global__ void __launch_bounds__(128, 1)
+reassign_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_c,
+                   const __nv_bfloat16* __restrict__ V, const float* __restrict__ norms, StatsPtrs st, int N, int C,
+                   int nB, int* status) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint8_t* sK = base;
+  uint8_t* sC0 = sK + kKTileBytes;
+  float* s_norm = reinterpret_cast<float*>(sC0 + 2 * kCTileBytes);
+  StatsSmem* ssm = reinterpret_cast<StatsSmem*>(s_norm + 1024);
+  int* s_assign = reinterpret_cast<int*>(ssm + 1);
+  Bars* bars = reinterpret_cast<Bars*>(s_assign + 128);
+
+  const int t = threadIdx.x;
+  const int warp = t >> 5;
+  const int j = blockIdx.x;
+  const int bh = blockIdx.y;
+  const int k0 = j * kKeys;
+  const int nk = min(kKeys, N - k0);
+  const int nchunks = (C + kChunk - 1) / kChunk;
+
+  if (t == 0) {
+    mbar_init(&bars->kfull, 1);
+    mbar_init(&bars->cfull[0], 1);
+    mbar_init(&bars->cfull[1], 1);
+    mbar_init(&bars->mdone[0], 1);
+    mbar_init(&bars->mdone[1], 1);
+    bars->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&bars->tmem_base, 512);
+    tmem_relinquish();
+  }
+  for (int c = t; c < C; c += 128) s_norm[c] = norms[(size_t)bh * C + c];
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  volatile int* abort = &bars->abort;
+
+  auto load_chunk = [&](int c) {
+    uint8_t* dst = sC0 + (c & 1) * kCTileBytes;
+    mbar_expect_tx(&bars->cfull[c & 1], kCTileBytes);
+    tma_load_3d(dst, &tm_c, &bars->cfull[c & 1], 0, c * kChunk, bh);
+    tma_load_3d(dst + kPanelC, &tm_c, &bars->cfull[c & 1], 64, c * kChunk, bh);
+  };
+  auto issue_mma = [&](int c) -> bool {
+    if (!mbar_wait(&bars->cfull[c & 1], (c >> 1) & 1, abort, status)) return false;
+    tc_fence_after();
+    const int n = min(kChunk, C - c * kChunk);
+    const uint32_t idesc = idesc_bf16(128, n, 0, 0);
+    const uint32_t a0 = smem_u32(sK), b0 = smem_u32(sC0 + (c & 1) * kCTileBytes);
+#pragma unroll
+    for (int ks = 0; ks < kD / 16; ++ks) {
+      const uint32_t koff = (ks & 3) * 32;
+      const uint64_t ad = sdesc_sw128(a0 + (ks >> 2) * kPanelK + koff, 16, 1024);
+      const uint64_t bd = sdesc_sw128(b0 + (ks >> 2) * kPanelC + koff, 16, 1024);
+      umma_ss(tmem + (c & 1) * kChunk, ad, bd, idesc, ks > 0 ? 1u : 0u);
+    }
+    umma_commit(&bars->mdone[c & 1]);
+    return true;
+  };
+
+  if (t == 0) {
+    tma_prefetch(&tm_k);
+    tma_prefetch(&tm_c);
+    mbar_expect_tx(&bars->kfull, kKTileBytes);
+    tma_load_3d(sK, &tm_k, &bars->kfull, 0, k0, bh);
+    tma_load_3d(sK + kPanelK, &tm_k, &bars->kfull, 64, k0, bh);
+    load_chunk(0);
+    if (nchunks > 1) load_chunk(1);
+    if (mbar_wait(&bars->kfull, 0, abort, status)) issue_mma(0);
+  }
+
+  float best = INFINITY;
+  int arg = 0;
+  const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+  for (int c = 0; c < nchunks; ++c) {
+    if (t == 0 && c + 1 < nchunks && !*abort) issue_mma(c + 1);
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(&bars->mdone[c & 1], (c >> 1) & 1, abort, status));
+    tc_fence_after();
+    const int n = ok ? min(kChunk, C - c * kChunk) : 0;
+    for (int col = 0; col < n; col += 32) {
+      uint32_t r[32];
+      tmem_ld32(lane_base + (c & 1) * kChunk + col, r);
+      tmem_wait_ld();
+#pragma unroll
+      for (int q = 0; q < 32; ++q) {
+        const int cc = c * kChunk + col + q;
+        const float dist = fmaf(-2.f, __uint_as_float(r[q]), s_norm[cc]);
+        if (dist < best) {
+          best = dist;
+          arg = cc;
+        }
+      }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (t == 0 && c + 2 < nchunks && !*abort) load_chunk(c + 2);
+  }
+  __syncthreads();
+
+  if (!*abort) {
+    if (t < nk) {
+      s_assign[t] = arg;
+      st.assign[(size_t)bh * N + k0 + t] = arg;
+    }
+    __syncthreads();
+    const size_t bj = (size_t)bh * nB + j;
+    block_stats_group<__nv_bfloat16, kD>(t, 1, s_assign, nk, V + ((size_t)bh * N + k0) * kD, C,
+                                         st.blk_hist + bj * C, st.seg_idx + bj * C, st.seg_n + bj,
+                                         st.seg_c + bj * kKeys, st.seg_cnt + bj * kKeys,
+                                         st.seg_vsum + bj * kKeys * kD, *ssm);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+
+bool reassign_tc_supported(const Dims& g) { return g.bf16 && g.d == kD && g.block == kKeys; }
+
+cudaError_t launch_reassign_tc(const Dims& g, const void* K, const void* V, const void* cent, const float* norms,
+                               const StatsPtrs& st, int* status, cudaStream_t s) {
+  CUtensorMap tk, tc;
+  const unsigned long long BH = (unsigned long long)g.B * g.H;
+  if (!make_tmap_bf16_3d(&tk, K, kD, g.N, BH, 64, kKeys)) return cudaErrorInvalidValue;
+  if (!make_tmap_bf16_3d(&tc, cent, kD, g.C, BH, 64, kChunk)) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(reassign_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)kSmemBytes);
+  if (e != cudaSuccess) return e;
+  dim3 grid(g.nB, (unsigned)BH);
+  reassign_tc_kernel<<<grid, 128, kSmemBytes, s>>>(tk, tc, (const __nv_bfloat16*)V, norms, st, g.N, g.C, g.nB,
+                                                   status);
+  return cudaGetLastError();
+}
+
+}  // namespace da
