@@ -43,7 +43,7 @@ constexpr int kWarpMMA = 7;
 
 struct __align__(8) Bars {
   uint64_t q_full, q_empty;
-  uint64_t k_full[kStages], v_full[kStages], st_empty[kStages];
+  uint64_t k_full[kStages], v_full[kStages], st_empty[kStages], bfree[kStages];
   uint64_t s_full[2], p_ready[2];
   uint64_t o_done, o_free, drain;
   uint32_t tmem_base;
@@ -53,6 +53,7 @@ struct __align__(8) Bars {
 
 constexpr size_t kSmemBytes =
     1024 + kTile /*Q*/ + 2 * kStages * kTile /*K,V*/ + kStages * kBN * sizeof(float) /*beta*/ + sizeof(Bars);
+static_assert(kSmemBytes <= 232448, "shared memory above the 227 KB per-block limit");
 
 struct Params {
   const int32_t* kv_idx;
@@ -178,6 +179,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       mbar_init(&bars->k_full[s], 1);
       mbar_init(&bars->v_full[s], 1);
       mbar_init(&bars->st_empty[s], 1);
+      mbar_init(&bars->bfree[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars->s_full[b], 1);
@@ -208,10 +210,12 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       tma_prefetch(&tm_v);
       tma_prefetch(&tm_c);
       uint32_t g = 0;
-      int n = 0;
+      uint32_t exact_bits = 0;           // bit x: the last load into slot x carried a value block
+      int n = 0, nq = 0;                 // items walked, query tiles loaded
       for (int k = blockIdx.x; k < p.n_items && !*abort; k += gridDim.x, ++n) {
         const Item it = item_at(p, k);
         if (!mbar_wait(&bars->q_empty, (n & 1) ^ 1, abort, status)) break;
+        ++nq;
         mbar_expect_tx(&bars->q_full, kTile);
         tma_load_3d(sQ, &tm_q, &bars->q_full, 0, it.q0, it.bh);
         tma_load_3d(sQ + kPanel, &tm_q, &bars->q_full, 64, it.q0, it.bh);
@@ -231,14 +235,25 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             mbar_expect_tx(&bars->v_full[slot], kTile);
             tma_load_3d(dv, &tm_v, &bars->v_full[slot], 0, j * kBN, it.bh);
             tma_load_3d(dv + kPanel, &tm_v, &bars->v_full[slot], 64, j * kBN, it.bh);
+            exact_bits |= 1u << slot;
           } else {
+            exact_bits &= ~(1u << slot);
             const int c = s - it.nsel;
+            mbar_arrive(&bars->bfree[slot]);        // hand the value half of the slot to the builder
             mbar_expect_tx(&bars->k_full[slot], kTile);
             tma_load_3d(dk, &tm_c, &bars->k_full[slot], 0, c * kBN, it.bh);
             tma_load_3d(dk + kPanel, &tm_c, &bars->k_full[slot], 64, c * kBN, it.bh);
           }
         }
         if (!ok) break;
+      }
+      // no copy may still be in flight when the CTA leaves (this matters only after an abort:
+      // otherwise the MMA issuer has consumed every load)
+      if (nq > 0) mbar_wait_drain(&bars->q_full, (nq - 1) & 1);
+      for (uint32_t gd = g >= kStages ? g - kStages : 0; gd < g; ++gd) {
+        const int slot = gd % kStages;
+        mbar_wait_drain(&bars->k_full[slot], (gd / kStages) & 1);
+        if ((exact_bits >> slot) & 1u) mbar_wait_drain(&bars->v_full[slot], (gd / kStages) & 1);
       }
     }
   } else if (warp == kWarpMMA) {
@@ -302,7 +317,9 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     // ------------------------------------------------------------------ builder
     const int t = tid - 128;                  // rows t and t + 64 of every chunk
     uint32_t g = 0, nb = 0;                   // global step, chunks built so far
-    for (int k = blockIdx.x; k < p.n_items && !*abort; k += gridDim.x) {
+    uint32_t use_par = 0;                     // bit x: parity of the chunks built into slot x so far
+    // (no abort test in the loop condition: the builders leave together, on bld_ok)
+    for (int k = blockIdx.x; k < p.n_items; k += gridDim.x) {
       const Item it = item_at(p, k);
       g += it.nsel;
       bool ok = true;
@@ -312,10 +329,13 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         build_row(p, it, c * kBN + t, packed[0], &beta[0]);
         build_row(p, it, c * kBN + t + 64, packed[1], &beta[1]);
         const int slot = g % kStages;
-        const uint32_t u = g / kStages;
-        // one thread waits for the slot; the decision reaches both builder warps through a
-        // named barrier so that they leave (or go on) together
-        if (t == 0) bars->bld_ok[nb & 1] = mbar_wait(&bars->st_empty[slot], (u & 1) ^ 1, abort, status);
+        // The producer, which follows every phase of the ring, releases the slot's value half
+        // through bfree[slot] once the slot is empty; its phases are this builder's uses of the
+        // slot, in order.  One thread waits; the decision reaches both builder warps through a
+        // named barrier so that they leave (or go on) together.
+        const uint32_t use = (use_par >> slot) & 1u;
+        use_par ^= 1u << slot;
+        if (t == 0) bars->bld_ok[nb & 1] = mbar_wait(&bars->bfree[slot], use, abort, status);
         asm volatile("bar.sync 2, 64;" ::: "memory");
         if (!bars->bld_ok[(nb++) & 1]) { ok = false; break; }
 #pragma unroll
@@ -343,7 +363,8 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const int r = tid;                                        // query row = TMEM lane
     const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
     uint32_t g = 0;
-    for (int k = blockIdx.x; k < p.n_items && !*abort; k += gridDim.x) {
+    // (no abort test in the loop condition: a warp leaves as a whole, on its __all_sync'd waits)
+    for (int k = blockIdx.x; k < p.n_items; k += gridDim.x) {
       const Item it = item_at(p, k);
       float m = -INFINITY, l = 0.f;
       bool ok = true;
@@ -357,7 +378,9 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           const int j = block_of(p, it, s, &valid);
           ncol = valid ? min(kBN, p.N - j * kBN) : 0;
         }
-        bool w_ok = !comp || mbar_wait(&bars->v_full[slot], (g / kStages) & 1, abort, status);
+        // every phase of v_full and s_full is waited, in order (the value half of a compensation
+        // step carries the chunk's log2 n^U in sBeta)
+        bool w_ok = mbar_wait(&bars->v_full[slot], (g / kStages) & 1, abort, status);
         w_ok = w_ok && mbar_wait(&bars->s_full[b], (g >> 1) & 1, abort, status);
         if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
         tc_fence_after();
@@ -385,29 +408,11 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             mx = fmaxf(mx, x[c]);
           }
         }
-        // lazy rescaling: the running max moves only when it grows by more than 2^8; O is then
-        // rescaled in TMEM once PV(g-1) has landed (warp-uniform, as tcgen05.ld/st are)
+        // lazy rescaling: the running max moves only when it grows by more than 2^8
         const bool grow = mx > m + kRescaleLog2 || (m == -INFINITY && mx > -INFINITY);
         const bool need_o = grow && s > 0 && m > -INFINITY;
-        if (__any_sync(0xffffffffu, need_o)) {
-          const bool d_ok = mbar_wait(&bars->o_done, (g - 1) & 1, abort, status);
-          if (!__all_sync(0xffffffffu, d_ok)) { ok = false; break; }
-          tc_fence_after();
-          const float alpha = need_o ? ex2(m - mx) : 1.f;
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint32_t rr[32];
-            tmem_ld32(lane_addr + 2 * kBN + q * 32, rr);
-            tmem_wait_ld();
-#pragma unroll
-            for (int v = 0; v < 32; ++v) rr[v] = __float_as_uint(__uint_as_float(rr[v]) * alpha);
-            tmem_st32(lane_addr + 2 * kBN + q * 32, rr);
-          }
-          tmem_wait_st();
-          if (need_o) l *= alpha;
-        }
-        if (grow) m = mx;
-        const float mu = (m == -INFINITY) ? 0.f : m;
+        const float m_new = grow ? mx : m;
+        const float mu = (m_new == -INFINITY) ? 0.f : m_new;
         float rs = 0.f;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -421,6 +426,27 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           }
           tmem_st16(lane_addr + b * kBN + q * 16, pk);
         }
+        if (s > 0) {
+          // PV(g-1) has landed in O: every phase of o_done is waited, in order; a row whose max
+          // moved rescales its O (warp-uniform, as tcgen05.ld/st are)
+          const bool d_ok = mbar_wait(&bars->o_done, (g - 1) & 1, abort, status);
+          if (!__all_sync(0xffffffffu, d_ok)) { ok = false; break; }
+          tc_fence_after();
+          if (__any_sync(0xffffffffu, need_o)) {
+            const float alpha = need_o ? ex2(m - m_new) : 1.f;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              uint32_t rr[32];
+              tmem_ld32(lane_addr + 2 * kBN + q * 32, rr);
+              tmem_wait_ld();
+#pragma unroll
+              for (int v = 0; v < 32; ++v) rr[v] = __float_as_uint(__uint_as_float(rr[v]) * alpha);
+              tmem_st32(lane_addr + 2 * kBN + q * 32, rr);
+            }
+            if (need_o) l *= alpha;
+          }
+        }
+        m = m_new;
         l += rs;
         tmem_wait_st();
         tc_fence_before();

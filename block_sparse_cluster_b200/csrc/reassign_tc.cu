@@ -38,6 +38,8 @@ struct __align__(8) Bars {
 
 constexpr size_t kSmemBytes = 1024 /*align slack*/ + kKTileBytes + 2 * kCTileBytes + 4096 /*norms*/ +
                               sizeof(StatsSmem) + 512 /*assign*/ + 128 /*bars*/;
+static_assert(sizeof(Bars) <= 128, "barrier block");
+static_assert(kSmemBytes <= 232448, "shared memory above the 227 KB per-block limit");
 
 __global__ void __launch_bounds__(128, 1)
 reassign_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_c,

@@ -1,0 +1,265 @@
+"""Host-side model of the fused attention kernel's synchronisation protocol.
+
+The kernel's roles (TMA producer, MMA issuer, compensation builder, softmax
+warpgroup) talk only through mbarriers.  An mbarrier wait names a phase by its
+parity alone, so a wait is only meaningful while the barrier is within one
+phase of the awaited one; a role that falls two phases behind (or waits one
+phase early) reads the wrong phase.  This model replays the roles' exact
+sequence of arrivals and waits, with the tensor core executing its queue in
+order and the TMA unit completing loads in any order, under many random
+interleavings, and checks that
+
+* every parity wait is evaluated only while the barrier is at the awaited
+  phase or one past it;
+* no phase receives more arrivals than its count, and the transaction count
+  never goes negative;
+* no shared-memory slot, TMEM buffer or the query tile is overwritten while an
+  operation that reads it is still in flight;
+* every role finishes (no deadlock).
+
+It mirrors the step structure of attention_tc.cu: per work item, one step per
+selected block followed by one step per 128-cluster chunk, a 3-stage K/V ring,
+S double-buffered in TMEM, P in the S buffer, O accumulated across the item.
+"""
+import random
+
+import pytest
+
+STAGES = 3
+
+
+class Barrier:
+    def __init__(self, name, count):
+        self.name, self.count = name, count
+        self.pending = count
+        self.tx = 0
+        self.phase = 0          # number of completed phases
+
+    def _maybe_complete(self):
+        if self.pending == 0 and self.tx == 0:
+            self.phase += 1
+            self.pending = self.count
+
+    def arrive(self):
+        assert self.pending > 0, f"{self.name}: arrival beyond the count"
+        self.pending -= 1
+        self._maybe_complete()
+
+    def expect_tx(self, n):
+        self.tx += n
+        self.arrive()
+
+    def complete_tx(self, n):
+        self.tx -= n
+        assert self.tx >= 0, f"{self.name}: transaction count below zero"
+        self._maybe_complete()
+
+    def test(self, target):
+        """Wait for completion of phase `target` (-1: the phase before the first)."""
+        assert self.phase in (target, target + 1) or (target == -1 and self.phase == 0), (
+            f"{self.name}: parity wait for phase {target} while at phase {self.phase}")
+        return self.phase > target
+
+
+class Machine:
+    def __init__(self, items, nchunk, rng, old_builder=False):
+        self.items = items                     # list of nsel per item of one CTA
+        self.nchunk = nchunk
+        self.rng = rng
+        self.old_builder = old_builder
+        B = Barrier
+        self.q_full, self.q_empty = B("q_full", 1), B("q_empty", 1)
+        self.k_full = [B(f"k_full{i}", 1) for i in range(STAGES)]
+        self.v_full = [B(f"v_full{i}", 1) for i in range(STAGES)]
+        self.st_empty = [B(f"st_empty{i}", 1) for i in range(STAGES)]
+        self.bfree = [B(f"bfree{i}", 1) for i in range(STAGES)]
+        self.s_full = [B(f"s_full{i}", 1) for i in range(2)]
+        self.p_ready = [B(f"p_ready{i}", 1) for i in range(2)]
+        self.o_done, self.o_free = B("o_done", 1), B("o_free", 1)
+        self.tc_queue = []                     # in-order tensor core: ("mma", reads, writes) / ("commit", bar)
+        self.tma = []                          # in flight: (bar, bytes, slot_tag)
+        self.readers = {}                      # resource -> units with an operation in flight on it
+
+    # ---- resources: in-flight users of each buffer, tagged by unit
+    def _start_read(self, res, unit):
+        self.readers.setdefault(res, []).append(unit)
+
+    def _end_read(self, res, unit):
+        self.readers[res].remove(unit)
+
+    def _write(self, res, who, unit=None):
+        """A write by `unit`; the tensor core executes its own queue in issue order, so its earlier
+        operations on the same buffer are not a hazard for its later ones."""
+        busy = [u for u in self.readers.get(res, []) if not (unit == "tc" and u == "tc")]
+        assert not busy, f"{who} overwrites {res} while {busy} use it"
+
+    # ---- asynchronous units
+    def tc_issue_mma(self, reads, writes):
+        for w in writes:
+            self._write(w, "tensor core", unit="tc")
+        for r in reads + writes:     # the destination is busy until the MMA completes
+            self._start_read(r, "tc")
+        self.tc_queue.append(("mma", reads + writes))
+
+    def tc_commit(self, bar):
+        self.tc_queue.append(("commit", bar))
+
+    def step_units(self):
+        progressed = False
+        if self.tc_queue and self.rng.random() < 0.5:
+            kind, x = self.tc_queue.pop(0)
+            if kind == "mma":
+                for r in x:
+                    self._end_read(r, "tc")
+            else:
+                x.arrive()
+            progressed = True
+        if self.tma and self.rng.random() < 0.5:
+            i = self.rng.randrange(len(self.tma))
+            bar, n, res = self.tma.pop(i)
+            self._end_read(res, "tma")
+            bar.complete_tx(n)
+            progressed = True
+        return progressed
+
+    def tma_load(self, bar, res):
+        self._write(res, "TMA", unit="tma")
+        self._start_read(res, "tma")  # busy until the copy lands
+        self.tma.append((bar, 1, res))
+
+    # ---- roles (generators yield a predicate to wait on)
+    def producer(self):
+        g = 0
+        for n, nsel in enumerate(self.items):
+            T = nsel + self.nchunk
+            yield lambda: self.q_empty.test(n - 1)
+            self.q_full.expect_tx(1)
+            self.tma_load(self.q_full, "Q")
+            for s in range(T):
+                slot, u = g % STAGES, g // STAGES
+                yield lambda: self.st_empty[slot].test(u - 1)
+                if s < nsel:
+                    self.k_full[slot].expect_tx(1)
+                    self.tma_load(self.k_full[slot], f"K{slot}")
+                    self.v_full[slot].expect_tx(1)
+                    self.tma_load(self.v_full[slot], f"V{slot}")
+                else:
+                    if not self.old_builder:
+                        self.bfree[slot].arrive()
+                    self.k_full[slot].expect_tx(1)
+                    self.tma_load(self.k_full[slot], f"K{slot}")
+                g += 1
+
+    def mma(self):
+        g = 0
+        for n, nsel in enumerate(self.items):
+            T = nsel + self.nchunk
+            yield lambda: self.q_full.test(n)
+            yield lambda: self.k_full[g % STAGES].test(g // STAGES)
+            self.tc_issue_mma(["Q", f"K{g % STAGES}"], [f"S{g & 1}"])
+            self.tc_commit(self.s_full[g & 1])
+            for s in range(T):
+                if s + 1 < T:
+                    gn = g + 1
+                    yield lambda: self.k_full[gn % STAGES].test(gn // STAGES)
+                    self.tc_issue_mma(["Q", f"K{gn % STAGES}"], [f"S{gn & 1}"])
+                    self.tc_commit(self.s_full[gn & 1])
+                else:
+                    self.tc_commit(self.q_empty)
+                yield lambda: self.p_ready[g & 1].test(g >> 1)
+                yield lambda: self.v_full[g % STAGES].test(g // STAGES)
+                if s == 0:
+                    yield lambda: self.o_free.test(n - 1)
+                self.tc_issue_mma([f"S{g & 1}", f"V{g % STAGES}"], ["O"])
+                self.tc_commit(self.st_empty[g % STAGES])
+                self.tc_commit(self.o_done)
+                g += 1
+
+    def builder(self):
+        g = 0
+        uses = [0] * STAGES
+        for n, nsel in enumerate(self.items):
+            g += nsel
+            for c in range(self.nchunk):
+                slot = g % STAGES
+                if self.old_builder:
+                    u = g // STAGES
+                    yield lambda: self.st_empty[slot].test(u - 1)
+                else:
+                    use = uses[slot]
+                    uses[slot] += 1
+                    yield lambda: self.bfree[slot].test(use)
+                self._write(f"V{slot}", "builder")
+                self.v_full[slot].arrive()
+                g += 1
+
+    def softmax(self):
+        g = 0
+        for n, nsel in enumerate(self.items):
+            T = nsel + self.nchunk
+            for s in range(T):
+                b, slot = g & 1, g % STAGES
+                yield lambda: self.v_full[slot].test(g // STAGES)
+                yield lambda: self.s_full[b].test(g >> 1)
+                assert not self.readers.get(f"S{b}"), "S read before its MMA completed"
+                self._write(f"S{b}", "softmax (P)")
+                if s > 0:
+                    yield lambda: self.o_done.test(g - 1)
+                    self._write("O", "softmax (rescale)")
+                self.p_ready[b].arrive()
+                g += 1
+            yield lambda: self.o_done.test(g - 1)
+            self._write("O", "epilogue")
+            self.o_free.arrive()
+
+    def run(self, max_iters=200000):
+        roles = [self.producer(), self.mma(), self.builder(), self.softmax()]
+        waits = [None] * len(roles)
+        done = [False] * len(roles)
+        for _ in range(max_iters):
+            if all(done) and not self.tc_queue and not self.tma:
+                return True
+            order = list(range(len(roles)))
+            self.rng.shuffle(order)
+            progressed = False
+            for r in order:
+                if done[r]:
+                    continue
+                if waits[r] is not None and not waits[r]():
+                    continue
+                try:
+                    waits[r] = next(roles[r])
+                except StopIteration:
+                    done[r] = True
+                    waits[r] = None
+                progressed = True
+                if self.rng.random() < 0.5:
+                    break
+            progressed = self.step_units() or progressed
+            if not progressed and not self.tc_queue and not self.tma:
+                raise AssertionError("deadlock: no role can progress")
+        raise AssertionError("did not finish")
+
+
+CASES = [
+    ([4], 2), ([37], 2), ([0], 2), ([0, 37, 2, 0, 5], 2), ([30, 30, 30], 4), ([1, 0, 0, 1], 1),
+    ([9, 3, 0, 12], 8), ([2], 1), ([0, 0, 0], 3), ([40, 1], 4),
+]
+
+
+@pytest.mark.parametrize("items,nchunk", CASES)
+def test_protocol_random_interleavings(items, nchunk):
+    for seed in range(60):
+        Machine(items, nchunk, random.Random(seed)).run()
+
+
+def test_model_catches_a_builder_that_skips_ring_phases():
+    """The builder waiting on the ring's empty barrier only at its own steps falls behind
+    the ring by several phases when many exact steps precede a chunk."""
+    caught = 0
+    for seed in range(40):
+        try:
+            Machine([37], 2, random.Random(seed), old_builder=True).run()
+        except AssertionError:
+            caught += 1
+    assert caught > 0
