@@ -13,14 +13,15 @@
 // block, then one per 128-cluster chunk.  Every step is a 128 x 128 score tile S = Q K^T (K a
 // key block or a centroid chunk) and a P V product (V a value block or the chunk's vbar^U rows).
 //
-// Roles (256 threads):
+// Roles (384 threads, three warpgroups):
 //   warps 0-3  softmax: thread t owns query row t = TMEM lane t; online softmax with lazy
 //              rescaling (the running max only moves when it grows by more than 2^8), P written
 //              back to TMEM as bf16, final normalisation and store of O;
-//   warps 4-5  builder: thread t owns cluster rows t and t + 64 of a chunk; builds vbar^U (bf16,
-//              in the swizzled operand layout) and log2 n^U in shared memory;
-//   warp 6     producer: TMA loads of Q, K / V blocks and centroid chunks into a 3-stage ring;
-//   warp 7     MMA: allocates TMEM, issues tcgen05.mma S(g+1) = Q K^T ahead of O += P(g) V(g).
+//   warps 4-7  builder: thread t owns cluster row t of a chunk; builds vbar^U (bf16, in the
+//              swizzled operand layout) and log2 n^U in shared memory;
+//   warp 8     producer: TMA loads of Q, K / V blocks and centroid chunks into a 3-stage ring;
+//   warp 9     MMA: allocates TMEM, issues tcgen05.mma S(g+1) = Q K^T ahead of O += P(g) V(g);
+//   warps 10-11 idle.
 // TMEM columns: S double buffer [0,128) and [128,256), O [256,384).
 #include "da_common.cuh"
 #include "da_internal.h"
@@ -37,9 +38,14 @@ constexpr int kStages = 3;
 constexpr int kTile = kBN * kD * 2;      // 32 KB bf16 tile
 constexpr int kPanel = kBN * 128;        // one 64-column panel (128 rows x 128 B)
 constexpr float kRescaleLog2 = 8.0f;     // lazy rescale threshold (factor 256)
-constexpr int kThreads = 256;
-constexpr int kWarpProducer = 6;
-constexpr int kWarpMMA = 7;
+constexpr int kThreads = 384;            // three warpgroups
+constexpr int kWarpProducer = 8;
+constexpr int kWarpMMA = 9;
+// Register split (setmaxnreg): the launch holds 384 x 168 registers; the softmax and builder
+// warpgroups grow, the producer / MMA warpgroup shrinks.
+constexpr int kRegSoftmax = 240, kRegBuilder = 200, kRegIssue = 56;
+static_assert(128 * (kRegSoftmax + kRegBuilder + kRegIssue) <= kThreads * 168, "register split above the launch");
+constexpr int kBatch = 16;               // selected blocks looked up per round by the builder
 
 struct __align__(8) Bars {
   uint64_t q_full, q_empty;
@@ -105,7 +111,9 @@ __device__ __forceinline__ int block_of(const Params& p, const Item& it, int s, 
 
 // One row of a compensation chunk: cluster cl of the item's head.  Packs
 // vbar^U = (S_c - sum_{j in sel} S_{c,j}) / n^U_c as bf16 pairs and returns log2 n^U_c
-// (-inf when the cluster has no key outside the selected blocks or cl >= C).
+// (-inf when the cluster has no key outside the selected blocks or cl >= C).  The selected
+// blocks are looked up kBatch at a time with independent loads (the entry index of cluster cl in
+// block j is seg_idx[j][cl]); a hit subtracts that entry's value sum and count.
 __device__ __forceinline__ void build_row(const Params& p, const Item& it, int cl, uint32_t (&packed)[64],
                                           float* beta) {
   if (cl >= p.C) {
@@ -115,45 +123,45 @@ __device__ __forceinline__ void build_row(const Params& p, const Item& it, int c
     return;
   }
   const size_t hc = (size_t)it.bh * p.C + cl;
-  int nU = p.st.n_tot[hc];
-  for (int s = 0; s < it.nsel; ++s) {
-    bool valid;
-    const int j = block_of(p, it, s, &valid);
-    if (!valid) continue;
-    const size_t bj = (size_t)it.bh * p.nB + j;
-    const int e = p.st.seg_idx[bj * p.C + cl];
-    if (e != 0xFF) nU -= p.st.seg_cnt[bj * kBN + e];
-  }
-  const float inv = nU > 0 ? 1.f / (float)nU : 0.f;
-  *beta = nU > 0 ? log2f((float)nU) : -INFINITY;
+  float acc[kD];
+  {
+    const float4* tot = reinterpret_cast<const float4*>(p.st.S_tot + hc * kD);
 #pragma unroll
-  for (int qd = 0; qd < 4; ++qd) {
-    float acc[32];
-    const float4* tot = reinterpret_cast<const float4*>(p.st.S_tot + hc * kD + qd * 32);
-#pragma unroll
-    for (int v = 0; v < 8; ++v) {
+    for (int v = 0; v < kD / 4; ++v) {
       const float4 x = tot[v];
       acc[4 * v] = x.x; acc[4 * v + 1] = x.y; acc[4 * v + 2] = x.z; acc[4 * v + 3] = x.w;
     }
-    if (nU > 0) {
-      for (int s = 0; s < it.nsel; ++s) {
-        bool valid;
-        const int j = block_of(p, it, s, &valid);
-        if (!valid) continue;
-        const size_t bj = (size_t)it.bh * p.nB + j;
-        const int e = p.st.seg_idx[bj * p.C + cl];
-        if (e == 0xFF) continue;
-        const float4* sv = reinterpret_cast<const float4*>(p.st.seg_vsum + (bj * kBN + e) * kD + qd * 32);
+  }
+  int nU = p.st.n_tot[hc];
+  const size_t head_blk = (size_t)it.bh * p.nB;
+  for (int s0 = 0; s0 < it.nsel; s0 += kBatch) {
+    int jb[kBatch];
 #pragma unroll
-        for (int v = 0; v < 8; ++v) {
+    for (int u = 0; u < kBatch; ++u) {
+      const int j = s0 + u < it.nsel ? it.row[s0 + u] : -1;
+      jb[u] = (j >= 0 && j < p.nB) ? j : -1;
+    }
+    int eb[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) eb[u] = jb[u] >= 0 ? (int)p.st.seg_idx[(head_blk + jb[u]) * p.C + cl] : 0xFF;
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      if (eb[u] != 0xFF) {
+        const size_t ent = (head_blk + jb[u]) * kBN + eb[u];
+        nU -= p.st.seg_cnt[ent];
+        const float4* sv = reinterpret_cast<const float4*>(p.st.seg_vsum + ent * kD);
+#pragma unroll
+        for (int v = 0; v < kD / 4; ++v) {
           const float4 x = sv[v];
           acc[4 * v] -= x.x; acc[4 * v + 1] -= x.y; acc[4 * v + 2] -= x.z; acc[4 * v + 3] -= x.w;
         }
       }
     }
-#pragma unroll
-    for (int v = 0; v < 16; ++v) packed[qd * 16 + v] = pack_bf16x2(acc[2 * v] * inv, acc[2 * v + 1] * inv);
   }
+  const float inv = nU > 0 ? 1.f / (float)nU : 0.f;
+  *beta = nU > 0 ? log2f((float)nU) : -INFINITY;
+#pragma unroll
+  for (int v = 0; v < 64; ++v) packed[v] = pack_bf16x2(acc[2 * v] * inv, acc[2 * v + 1] * inv);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -202,6 +210,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   volatile int* abort = &bars->abort;
   int* status = p.status;
 
+  if (warp >= 8) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegIssue));
   if (warp == kWarpProducer) {
     // ------------------------------------------------------------------ producer
     if (lane == 0) {
@@ -313,9 +322,12 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       umma_commit(&bars->drain);
       mbar_wait_drain(&bars->drain, 0);
     }
+  } else if (warp >= 8) {
+    // warps 10-11: idle
   } else if (warp >= 4) {
     // ------------------------------------------------------------------ builder
-    const int t = tid - 128;                  // rows t and t + 64 of every chunk
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegBuilder));
+    const int t = tid - 128;                  // row t of every chunk
     uint32_t g = 0, nb = 0;                   // global step, chunks built so far
     uint32_t use_par = 0;                     // bit x: parity of the chunks built into slot x so far
     // (no abort test in the loop condition: the builders leave together, on bld_ok)
@@ -324,42 +336,37 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       g += it.nsel;
       bool ok = true;
       for (int c = 0; c < p.nchunk; ++c, ++g) {
-        uint32_t packed[2][64];
-        float beta[2];
-        build_row(p, it, c * kBN + t, packed[0], &beta[0]);
-        build_row(p, it, c * kBN + t + 64, packed[1], &beta[1]);
+        uint32_t packed[64];
+        float beta;
+        build_row(p, it, c * kBN + t, packed, &beta);
         const int slot = g % kStages;
         // The producer, which follows every phase of the ring, releases the slot's value half
         // through bfree[slot] once the slot is empty; its phases are this builder's uses of the
-        // slot, in order.  One thread waits; the decision reaches both builder warps through a
+        // slot, in order.  One thread waits; the decision reaches every builder warp through a
         // named barrier so that they leave (or go on) together.
         const uint32_t use = (use_par >> slot) & 1u;
         use_par ^= 1u << slot;
         if (t == 0) bars->bld_ok[nb & 1] = mbar_wait(&bars->bfree[slot], use, abort, status);
-        asm volatile("bar.sync 2, 64;" ::: "memory");
+        asm volatile("bar.sync 2, 128;" ::: "memory");
         if (!bars->bld_ok[(nb++) & 1]) { ok = false; break; }
+        // row t of the value operand: panel d / 64, 16-byte chunk (d % 64) / 8, 128-byte swizzle
+        uint8_t* rowp = sV + slot * kTile + t * 128;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int r = t + 64 * h;
-          // row r of the value operand: panel d / 64, 16-byte chunk (d % 64) / 8, 128-byte swizzle
-          uint8_t* rowp = sV + slot * kTile + r * 128;
-#pragma unroll
-          for (int ch = 0; ch < 16; ++ch) {
-            const int panel = ch >> 3, cc = ch & 7;
-            const uint4 v = make_uint4(packed[h][4 * ch], packed[h][4 * ch + 1], packed[h][4 * ch + 2],
-                                       packed[h][4 * ch + 3]);
-            *reinterpret_cast<uint4*>(rowp + panel * kPanel + ((cc ^ (r & 7)) << 4)) = v;
-          }
-          sBeta[slot * kBN + r] = beta[h];
+        for (int ch = 0; ch < 16; ++ch) {
+          const int panel = ch >> 3, cc = ch & 7;
+          const uint4 v = make_uint4(packed[4 * ch], packed[4 * ch + 1], packed[4 * ch + 2], packed[4 * ch + 3]);
+          *reinterpret_cast<uint4*>(rowp + panel * kPanel + ((cc ^ (t & 7)) << 4)) = v;
         }
+        sBeta[slot * kBN + t] = beta;
         fence_async_smem();
-        asm volatile("bar.sync 2, 64;" ::: "memory");
+        asm volatile("bar.sync 2, 128;" ::: "memory");
         if (t == 0) mbar_arrive(&bars->v_full[slot]);
       }
       if (!ok) break;
     }
   } else {
     // ------------------------------------------------------------------ softmax (warps 0-3)
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegSoftmax));
     const int r = tid;                                        // query row = TMEM lane
     const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
     uint32_t g = 0;

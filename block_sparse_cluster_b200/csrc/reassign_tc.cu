@@ -10,7 +10,8 @@
 //      ||cbar_c||^2 - 2 k.cbar_c (ties to the lowest c; the key's own norm is the same for
 //      every c and is dropped).
 //   4. The same 128 threads refresh the block's statistics (block_stats.cuh): sorted entry list,
-//      histogram row, entry index row and fp32 value sums.
+//      histogram row, entry index row and fp32 value sums, reading the block's value rows from a
+//      shared-memory copy (TMA, loaded with the key tile).
 #include "block_stats.cuh"
 #include "da_common.cuh"
 #include "da_internal.h"
@@ -36,20 +37,21 @@ struct __align__(8) Bars {
   int abort;
 };
 
-constexpr size_t kSmemBytes = 1024 /*align slack*/ + kKTileBytes + 2 * kCTileBytes + 4096 /*norms*/ +
+constexpr size_t kSmemBytes = 1024 /*align slack*/ + 2 * kKTileBytes /*K, V*/ + 2 * kCTileBytes + 4096 /*norms*/ +
                               sizeof(StatsSmem) + 512 /*assign*/ + 128 /*bars*/;
 static_assert(sizeof(Bars) <= 128, "barrier block");
 static_assert(kSmemBytes <= 232448, "shared memory above the 227 KB per-block limit");
 
 __global__ void __launch_bounds__(128, 1)
 reassign_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_c,
-                   const __nv_bfloat16* __restrict__ V, const float* __restrict__ norms, StatsPtrs st, int N, int C,
-                   int nB, int* status) {
+                   const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ norms, StatsPtrs st, int N,
+                   int C, int nB, int* status) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   uint8_t* sK = base;
-  uint8_t* sC0 = sK + kKTileBytes;
+  uint8_t* sVt = sK + kKTileBytes;                 // value rows of the block, [128][128] bf16, unswizzled
+  uint8_t* sC0 = sVt + kKTileBytes;
   float* s_norm = reinterpret_cast<float*>(sC0 + 2 * kCTileBytes);
   StatsSmem* ssm = reinterpret_cast<StatsSmem*>(s_norm + 1024);
   int* s_assign = reinterpret_cast<int*>(ssm + 1);
@@ -109,9 +111,11 @@ reassign_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
   if (t == 0) {
     tma_prefetch(&tm_k);
     tma_prefetch(&tm_c);
-    mbar_expect_tx(&bars->kfull, kKTileBytes);
+    tma_prefetch(&tm_v);
+    mbar_expect_tx(&bars->kfull, 2 * kKTileBytes);
     tma_load_3d(sK, &tm_k, &bars->kfull, 0, k0, bh);
     tma_load_3d(sK + kPanelK, &tm_k, &bars->kfull, 64, k0, bh);
+    tma_load_3d(sVt, &tm_v, &bars->kfull, 0, k0, bh);
     load_chunk(0);
     if (nchunks > 1) load_chunk(1);
     if (mbar_wait(&bars->kfull, 0, abort, status)) issue_mma(0);
@@ -153,7 +157,7 @@ reassign_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     }
     __syncthreads();
     const size_t bj = (size_t)bh * nB + j;
-    block_stats_group<__nv_bfloat16, kD>(t, 1, s_assign, nk, V + ((size_t)bh * N + k0) * kD, C,
+    block_stats_group<__nv_bfloat16, kD>(t, 1, s_assign, nk, reinterpret_cast<const __nv_bfloat16*>(sVt), C,
                                          st.blk_hist + bj * C, st.seg_idx + bj * C, st.seg_n + bj,
                                          st.seg_c + bj * kKeys, st.seg_cnt + bj * kKeys,
                                          st.seg_vsum + bj * kKeys * kD, *ssm);
@@ -172,16 +176,16 @@ bool reassign_tc_supported(const Dims& g) { return g.bf16 && g.d == kD && g.bloc
 
 cudaError_t launch_reassign_tc(const Dims& g, const void* K, const void* V, const void* cent, const float* norms,
                                const StatsPtrs& st, int* status, cudaStream_t s) {
-  CUtensorMap tk, tc;
+  CUtensorMap tk, tc, tv;
   const unsigned long long BH = (unsigned long long)g.B * g.H;
   if (!make_tmap_bf16_3d(&tk, K, kD, g.N, BH, 64, kKeys)) return cudaErrorInvalidValue;
   if (!make_tmap_bf16_3d(&tc, cent, kD, g.C, BH, 64, kChunk)) return cudaErrorInvalidValue;
+  if (!make_tmap_bf16_3d(&tv, V, kD, g.N, BH, kD, kKeys, false)) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(reassign_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid(g.nB, (unsigned)BH);
-  reassign_tc_kernel<<<grid, 128, kSmemBytes, s>>>(tk, tc, (const __nv_bfloat16*)V, norms, st, g.N, g.C, g.nB,
-                                                   status);
+  reassign_tc_kernel<<<grid, 128, kSmemBytes, s>>>(tk, tc, tv, norms, st, g.N, g.C, g.nB, status);
   return cudaGetLastError();
 }
 
