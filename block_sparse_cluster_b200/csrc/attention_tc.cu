@@ -13,16 +13,24 @@
 // block, then one per 128-cluster chunk.  Every step is a 128 x 128 score tile S = Q K^T (K a
 // key block or a centroid chunk) and a P V product (V a value block or the chunk's vbar^U rows).
 //
-// Roles (384 threads, three warpgroups):
+// Roles (384 threads, three warpgroups; registers rebalanced with setmaxnreg):
 //   warps 0-3  softmax: thread t owns query row t = TMEM lane t; online softmax with lazy
 //              rescaling (the running max only moves when it grows by more than 2^8), P written
 //              back to TMEM as bf16, final normalisation and store of O;
-//   warps 4-7  builder: thread t owns cluster row t of a chunk; builds vbar^U (bf16, in the
-//              swizzled operand layout) and log2 n^U in shared memory;
-//   warp 8     producer: TMA loads of Q, K / V blocks and centroid chunks into a 3-stage ring;
+//   warps 4-7  builder: one work item ahead of the tensor cores, writes the item's vbar^U rows
+//              (bf16) and log2 n^U to a per-CTA, double-buffered global scratch (L2-resident):
+//              one batch of independent lookups per chunk finds, for each cluster row, the
+//              selected blocks holding that cluster; then each warp gathers 32 rows with
+//              coalesced loads (lanes over d);
+//   warp 8     producer: TMA loads of Q, K / V blocks, centroid chunks and the scratch chunks
+//              into a 3-stage ring;
 //   warp 9     MMA: allocates TMEM, issues tcgen05.mma S(g+1) = Q K^T ahead of O += P(g) V(g);
 //   warps 10-11 idle.
 // TMEM columns: S double buffer [0,128) and [128,256), O [256,384).
+//
+// Every mbarrier is waited at every phase, in order, by each role that waits on it (a parity
+// wait is only meaningful within one phase); the host-side protocol model in the tests replays
+// this schedule.
 #include "da_common.cuh"
 #include "da_internal.h"
 #include "tma_host.h"
@@ -43,15 +51,18 @@ constexpr int kWarpProducer = 8;
 constexpr int kWarpMMA = 9;
 // Register split (setmaxnreg): the launch holds 384 x 168 registers; the softmax and builder
 // warpgroups grow, the producer / MMA warpgroup shrinks.
-constexpr int kRegSoftmax = 240, kRegBuilder = 200, kRegIssue = 56;
+constexpr int kRegSoftmax = 240, kRegBuilder = 200, kRegIssue = 64;
 static_assert(128 * (kRegSoftmax + kRegBuilder + kRegIssue) <= kThreads * 168, "register split above the launch");
-constexpr int kBatch = 16;               // selected blocks looked up per round by the builder
+constexpr int kMaxCtas = 160;            // scratch is sized for this many persistent CTAs
+constexpr int kChunkBytes = kTile + kBN * 4;   // scratch chunk: vbar^U rows, then log2 n^U
+constexpr int kSlots = 4;                // matches per cluster row handled on the fast path
 
 struct __align__(8) Bars {
   uint64_t q_full, q_empty;
-  uint64_t k_full[kStages], v_full[kStages], st_empty[kStages], bfree[kStages];
+  uint64_t k_full[kStages], v_full[kStages], st_empty[kStages];
   uint64_t s_full[2], p_ready[2];
   uint64_t o_done, o_free, drain;
+  uint64_t bready[2], sfree[2];          // scratch buffer b: built (builder -> producer), free (softmax -> builder)
   uint32_t tmem_base;
   int abort;
   volatile int bld_ok[2];
@@ -70,6 +81,7 @@ struct Params {
   __nv_bfloat16* O;
   float* lse;
   int* status;
+  uint8_t* scratch;                      // kMaxCtas x 2 x nchunk chunks of kChunkBytes
   int N, C, nB, n_items, nchunk;
   float scale_log2;
 };
@@ -79,6 +91,8 @@ __device__ __forceinline__ float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+
+__device__ __forceinline__ float4 ldg4(const float* p) { return __ldg(reinterpret_cast<const float4*>(p)); }
 
 // Item geometry shared by every role.
 struct Item {
@@ -109,65 +123,109 @@ __device__ __forceinline__ int block_of(const Params& p, const Item& it, int s, 
   return *valid ? j : 0;
 }
 
-// One row of a compensation chunk: cluster cl of the item's head.  Packs
-// vbar^U = (S_c - sum_{j in sel} S_{c,j}) / n^U_c as bf16 pairs and returns log2 n^U_c
-// (-inf when the cluster has no key outside the selected blocks or cl >= C).  The selected
-// blocks are looked up kBatch at a time with independent loads (the entry index of cluster cl in
-// block j is seg_idx[j][cl]); a hit subtracts that entry's value sum and count.
-__device__ __forceinline__ void build_row(const Params& p, const Item& it, int cl, uint32_t (&packed)[64],
-                                          float* beta) {
-  if (cl >= p.C) {
-#pragma unroll
-    for (int v = 0; v < 64; ++v) packed[v] = 0u;
-    *beta = -INFINITY;
-    return;
-  }
-  const size_t hc = (size_t)it.bh * p.C + cl;
-  float acc[kD];
-  {
-    const float4* tot = reinterpret_cast<const float4*>(p.st.S_tot + hc * kD);
-#pragma unroll
-    for (int v = 0; v < kD / 4; ++v) {
-      const float4 x = tot[v];
-      acc[4 * v] = x.x; acc[4 * v + 1] = x.y; acc[4 * v + 2] = x.z; acc[4 * v + 3] = x.w;
+__device__ __forceinline__ uint8_t* scratch_chunk(const Params& p, int buf, int c) {
+  return p.scratch + (((size_t)blockIdx.x * 2 + buf) * p.nchunk + c) * kChunkBytes;
+}
+
+// Builder: the compensation chunks of one item into scratch buffer `buf` (t: 0..127).
+__device__ __forceinline__ void build_item(const Params& p, const Item& it, int buf, int t) {
+  const int bw = t >> 5, lane = t & 31;
+  const size_t hb = (size_t)it.bh * p.nB;      // first block row of the head
+  const size_t hc = (size_t)it.bh * p.C;       // first cluster row of the head
+  for (int c = 0; c < p.nchunk; ++c) {
+    uint8_t* tile = scratch_chunk(p, buf, c);
+    // (1) lookups, thread t <-> cluster row r: the entry of r in each selected block (0xFF: none),
+    // the selected count n^sel_r, and the first kSlots entry rows in block order
+    const int r = c * kBN + t;
+    const bool rl = r < p.C;
+    int nm = 0, csel = 0;
+    uint32_t m0 = 0, m1 = 0, m2 = 0, m3 = 0;
+#pragma unroll 8
+    for (int s = 0; s < it.nsel; ++s) {
+      const int jr = it.row[s];
+      const bool ok = rl && jr >= 0 && jr < p.nB;
+      const size_t cell = (hb + (ok ? jr : 0)) * p.C + (rl ? r : 0);
+      const int e = ok ? (int)p.st.seg_idx[cell] : 0xFF;
+      csel += ok ? p.st.blk_hist[cell] : 0;
+      const bool hit = e != 0xFF;
+      const uint32_t ptr = (uint32_t)((hb + (ok ? jr : 0)) * kBN + (hit ? e : 0));
+      m0 = (hit && nm == 0) ? ptr : m0;
+      m1 = (hit && nm == 1) ? ptr : m1;
+      m2 = (hit && nm == 2) ? ptr : m2;
+      m3 = (hit && nm == 3) ? ptr : m3;
+      nm += hit ? 1 : 0;
     }
-  }
-  int nU = p.st.n_tot[hc];
-  const size_t head_blk = (size_t)it.bh * p.nB;
-  for (int s0 = 0; s0 < it.nsel; s0 += kBatch) {
-    int jb[kBatch];
+    const int nU = rl ? p.st.n_tot[hc + r] - csel : 0;
+    reinterpret_cast<float*>(tile + kTile)[t] = nU > 0 ? log2f((float)nU) : -INFINITY;
+    const float inv = nU > 0 ? 1.f / (float)nU : 0.f;
+    // (2) gather: warp bw writes rows 32*bw .. 32*bw+31; lane l holds d = 4l .. 4l+3
+    for (int i0 = 0; i0 < 32; i0 += 4) {
+      float4 a[4], x[4][kSlots];
+      int nmi[4];
+      float invi[4];
 #pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const int j = s0 + u < it.nsel ? it.row[s0 + u] : -1;
-      jb[u] = (j >= 0 && j < p.nB) ? j : -1;
-    }
-    int eb[kBatch];
+      for (int q = 0; q < 4; ++q) {
+        const int i = i0 + q;
+        const int rr = c * kBN + 32 * bw + i;
+        nmi[q] = __shfl_sync(0xffffffffu, nm, i);
+        invi[q] = __shfl_sync(0xffffffffu, inv, i);
+        const uint32_t p0 = __shfl_sync(0xffffffffu, m0, i), p1 = __shfl_sync(0xffffffffu, m1, i);
+        const uint32_t p2 = __shfl_sync(0xffffffffu, m2, i), p3 = __shfl_sync(0xffffffffu, m3, i);
+        const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+        a[q] = rr < p.C ? ldg4(p.st.S_tot + (hc + rr) * kD + 4 * lane) : z;
+        x[q][0] = nmi[q] > 0 ? ldg4(p.st.seg_vsum + (size_t)p0 * kD + 4 * lane) : z;
+        x[q][1] = nmi[q] > 1 ? ldg4(p.st.seg_vsum + (size_t)p1 * kD + 4 * lane) : z;
+        x[q][2] = nmi[q] > 2 ? ldg4(p.st.seg_vsum + (size_t)p2 * kD + 4 * lane) : z;
+        x[q][3] = nmi[q] > 3 ? ldg4(p.st.seg_vsum + (size_t)p3 * kD + 4 * lane) : z;
+      }
 #pragma unroll
-    for (int u = 0; u < kBatch; ++u) eb[u] = jb[u] >= 0 ? (int)p.st.seg_idx[(head_blk + jb[u]) * p.C + cl] : 0xFF;
+      for (int q = 0; q < 4; ++q) {
+        float4 v = a[q];
 #pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      if (eb[u] != 0xFF) {
-        const size_t ent = (head_blk + jb[u]) * kBN + eb[u];
-        nU -= p.st.seg_cnt[ent];
-        const float4* sv = reinterpret_cast<const float4*>(p.st.seg_vsum + ent * kD);
-#pragma unroll
-        for (int v = 0; v < kD / 4; ++v) {
-          const float4 x = sv[v];
-          acc[4 * v] -= x.x; acc[4 * v + 1] -= x.y; acc[4 * v + 2] -= x.z; acc[4 * v + 3] -= x.w;
+        for (int k = 0; k < kSlots; ++k) {
+          v.x -= x[q][k].x; v.y -= x[q][k].y; v.z -= x[q][k].z; v.w -= x[q][k].w;
         }
+        if (nmi[q] > kSlots) {
+          // rare: the row's cluster sits in more than kSlots selected blocks; the remaining
+          // entries, again in block order
+          const int rr = c * kBN + 32 * bw + i0 + q;
+          int seen = 0;
+          for (int s0 = 0; s0 < it.nsel; s0 += 8) {
+            int e8[8];
+            size_t b8[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const int jr = s0 + u < it.nsel ? it.row[s0 + u] : -1;
+              const bool ok = jr >= 0 && jr < p.nB;
+              b8[u] = hb + (ok ? jr : 0);
+              e8[u] = ok ? (int)p.st.seg_idx[b8[u] * p.C + rr] : 0xFF;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              if (e8[u] != 0xFF) {
+                if (seen >= kSlots) {
+                  const float4 y = ldg4(p.st.seg_vsum + (b8[u] * kBN + e8[u]) * kD + 4 * lane);
+                  v.x -= y.x; v.y -= y.y; v.z -= y.z; v.w -= y.w;
+                }
+                ++seen;
+              }
+            }
+          }
+        }
+        const float iv = invi[q];
+        uint2 o;
+        o.x = pack_bf16x2(v.x * iv, v.y * iv);
+        o.y = pack_bf16x2(v.z * iv, v.w * iv);
+        *reinterpret_cast<uint2*>(tile + (size_t)(32 * bw + i0 + q) * (kD * 2) + lane * 8) = o;
       }
     }
   }
-  const float inv = nU > 0 ? 1.f / (float)nU : 0.f;
-  *beta = nU > 0 ? log2f((float)nU) : -INFINITY;
-#pragma unroll
-  for (int v = 0; v < 64; ++v) packed[v] = pack_bf16x2(acc[2 * v] * inv, acc[2 * v + 1] * inv);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
 attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_c,
-                    const Params p) {
+                    const __grid_constant__ CUtensorMap tm_s, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -187,11 +245,12 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       mbar_init(&bars->k_full[s], 1);
       mbar_init(&bars->v_full[s], 1);
       mbar_init(&bars->st_empty[s], 1);
-      mbar_init(&bars->bfree[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars->s_full[b], 1);
       mbar_init(&bars->p_ready[b], 128);
+      mbar_init(&bars->bready[b], 1);
+      mbar_init(&bars->sfree[b], 128);
     }
     mbar_init(&bars->o_done, 1);
     mbar_init(&bars->o_free, 128);
@@ -218,8 +277,8 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       tma_prefetch(&tm_k);
       tma_prefetch(&tm_v);
       tma_prefetch(&tm_c);
+      tma_prefetch(&tm_s);
       uint32_t g = 0;
-      uint32_t exact_bits = 0;           // bit x: the last load into slot x carried a value block
       int n = 0, nq = 0;                 // items walked, query tiles loaded
       for (int k = blockIdx.x; k < p.n_items && !*abort; k += gridDim.x, ++n) {
         const Item it = item_at(p, k);
@@ -234,24 +293,29 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           const uint32_t u = g / kStages;
           if (!mbar_wait(&bars->st_empty[slot], (u & 1) ^ 1, abort, status)) { ok = false; break; }
           uint8_t* dk = sK + slot * kTile;
+          uint8_t* dv = sV + slot * kTile;
           if (s < it.nsel) {
             bool valid;
             const int j = block_of(p, it, s, &valid);
-            uint8_t* dv = sV + slot * kTile;
             mbar_expect_tx(&bars->k_full[slot], kTile);
             tma_load_3d(dk, &tm_k, &bars->k_full[slot], 0, j * kBN, it.bh);
             tma_load_3d(dk + kPanel, &tm_k, &bars->k_full[slot], 64, j * kBN, it.bh);
             mbar_expect_tx(&bars->v_full[slot], kTile);
             tma_load_3d(dv, &tm_v, &bars->v_full[slot], 0, j * kBN, it.bh);
             tma_load_3d(dv + kPanel, &tm_v, &bars->v_full[slot], 64, j * kBN, it.bh);
-            exact_bits |= 1u << slot;
           } else {
-            exact_bits &= ~(1u << slot);
             const int c = s - it.nsel;
-            mbar_arrive(&bars->bfree[slot]);        // hand the value half of the slot to the builder
+            const int buf = n & 1;
+            // the builder has finished this item's scratch chunks (once per item, in order)
+            if (c == 0 && !mbar_wait(&bars->bready[buf], (n >> 1) & 1, abort, status)) { ok = false; break; }
             mbar_expect_tx(&bars->k_full[slot], kTile);
             tma_load_3d(dk, &tm_c, &bars->k_full[slot], 0, c * kBN, it.bh);
             tma_load_3d(dk + kPanel, &tm_c, &bars->k_full[slot], 64, c * kBN, it.bh);
+            const int z = ((int)blockIdx.x * 2 + buf) * p.nchunk + c;
+            mbar_expect_tx(&bars->v_full[slot], kTile + kBN * 4);
+            tma_load_3d(dv, &tm_s, &bars->v_full[slot], 0, 0, z);
+            tma_load_3d(dv + kPanel, &tm_s, &bars->v_full[slot], 64, 0, z);
+            bulk_load(sBeta + slot * kBN, scratch_chunk(p, buf, c) + kTile, kBN * 4, &bars->v_full[slot]);
           }
         }
         if (!ok) break;
@@ -260,9 +324,8 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       // otherwise the MMA issuer has consumed every load)
       if (nq > 0) mbar_wait_drain(&bars->q_full, (nq - 1) & 1);
       for (uint32_t gd = g >= kStages ? g - kStages : 0; gd < g; ++gd) {
-        const int slot = gd % kStages;
-        mbar_wait_drain(&bars->k_full[slot], (gd / kStages) & 1);
-        if ((exact_bits >> slot) & 1u) mbar_wait_drain(&bars->v_full[slot], (gd / kStages) & 1);
+        mbar_wait_drain(&bars->k_full[gd % kStages], (gd / kStages) & 1);
+        mbar_wait_drain(&bars->v_full[gd % kStages], (gd / kStages) & 1);
       }
     }
   } else if (warp == kWarpMMA) {
@@ -327,42 +390,21 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   } else if (warp >= 4) {
     // ------------------------------------------------------------------ builder
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegBuilder));
-    const int t = tid - 128;                  // row t of every chunk
-    uint32_t g = 0, nb = 0;                   // global step, chunks built so far
-    uint32_t use_par = 0;                     // bit x: parity of the chunks built into slot x so far
+    const int t = tid - 128;
+    int n = 0;
     // (no abort test in the loop condition: the builders leave together, on bld_ok)
-    for (int k = blockIdx.x; k < p.n_items; k += gridDim.x) {
+    for (int k = blockIdx.x; k < p.n_items; k += gridDim.x, ++n) {
       const Item it = item_at(p, k);
-      g += it.nsel;
-      bool ok = true;
-      for (int c = 0; c < p.nchunk; ++c, ++g) {
-        uint32_t packed[64];
-        float beta;
-        build_row(p, it, c * kBN + t, packed, &beta);
-        const int slot = g % kStages;
-        // The producer, which follows every phase of the ring, releases the slot's value half
-        // through bfree[slot] once the slot is empty; its phases are this builder's uses of the
-        // slot, in order.  One thread waits; the decision reaches every builder warp through a
-        // named barrier so that they leave (or go on) together.
-        const uint32_t use = (use_par >> slot) & 1u;
-        use_par ^= 1u << slot;
-        if (t == 0) bars->bld_ok[nb & 1] = mbar_wait(&bars->bfree[slot], use, abort, status);
-        asm volatile("bar.sync 2, 128;" ::: "memory");
-        if (!bars->bld_ok[(nb++) & 1]) { ok = false; break; }
-        // row t of the value operand: panel d / 64, 16-byte chunk (d % 64) / 8, 128-byte swizzle
-        uint8_t* rowp = sV + slot * kTile + t * 128;
-#pragma unroll
-        for (int ch = 0; ch < 16; ++ch) {
-          const int panel = ch >> 3, cc = ch & 7;
-          const uint4 v = make_uint4(packed[4 * ch], packed[4 * ch + 1], packed[4 * ch + 2], packed[4 * ch + 3]);
-          *reinterpret_cast<uint4*>(rowp + panel * kPanel + ((cc ^ (t & 7)) << 4)) = v;
-        }
-        sBeta[slot * kBN + t] = beta;
-        fence_async_smem();
-        asm volatile("bar.sync 2, 128;" ::: "memory");
-        if (t == 0) mbar_arrive(&bars->v_full[slot]);
-      }
-      if (!ok) break;
+      const int buf = n & 1;
+      // scratch buffer `buf` was last read for item n-2: wait until that item has finished.
+      // One thread waits; the decision reaches every builder warp through a named barrier.
+      if (t == 0) bars->bld_ok[n & 1] = n < 2 || mbar_wait(&bars->sfree[buf], ((n >> 1) - 1) & 1, abort, status);
+      asm volatile("bar.sync 2, 128;" ::: "memory");
+      if (!bars->bld_ok[n & 1]) break;
+      build_item(p, it, buf, t);
+      fence_async_global();
+      asm volatile("bar.sync 2, 128;" ::: "memory");
+      if (t == 0) mbar_arrive(&bars->bready[buf]);
     }
   } else {
     // ------------------------------------------------------------------ softmax (warps 0-3)
@@ -370,8 +412,9 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const int r = tid;                                        // query row = TMEM lane
     const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
     uint32_t g = 0;
+    int n = 0;
     // (no abort test in the loop condition: a warp leaves as a whole, on its __all_sync'd waits)
-    for (int k = blockIdx.x; k < p.n_items; k += gridDim.x) {
+    for (int k = blockIdx.x; k < p.n_items; k += gridDim.x, ++n) {
       const Item it = item_at(p, k);
       float m = -INFINITY, l = 0.f;
       bool ok = true;
@@ -392,35 +435,43 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
         tc_fence_after();
         float x[kBN];
+        {
+          uint32_t rr[4][32];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint32_t rr[32];
-          tmem_ld32(lane_addr + b * kBN + q * 32, rr);
+          for (int q = 0; q < 4; ++q) tmem_ld32(lane_addr + b * kBN + q * 32, rr[q]);
           tmem_wait_ld();
 #pragma unroll
-          for (int v = 0; v < 32; ++v) x[q * 32 + v] = __uint_as_float(rr[v]);
+          for (int q = 0; q < 4; ++q)
+#pragma unroll
+            for (int v = 0; v < 32; ++v) x[q * 32 + v] = __uint_as_float(rr[q][v]);
         }
-        float mx = -INFINITY;
+        float mx8[8];
+#pragma unroll
+        for (int v = 0; v < 8; ++v) mx8[v] = -INFINITY;
         if (comp) {
           const float* bt = sBeta + slot * kBN;
 #pragma unroll
           for (int c = 0; c < kBN; ++c) {
             x[c] = fmaf(x[c], p.scale_log2, bt[c]);
-            mx = fmaxf(mx, x[c]);
+            mx8[c & 7] = fmaxf(mx8[c & 7], x[c]);
           }
         } else {
 #pragma unroll
           for (int c = 0; c < kBN; ++c) {
             x[c] = c < ncol ? x[c] * p.scale_log2 : -INFINITY;
-            mx = fmaxf(mx, x[c]);
+            mx8[c & 7] = fmaxf(mx8[c & 7], x[c]);
           }
         }
+        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
         // lazy rescaling: the running max moves only when it grows by more than 2^8
         const bool grow = mx > m + kRescaleLog2 || (m == -INFINITY && mx > -INFINITY);
         const bool need_o = grow && s > 0 && m > -INFINITY;
         const float m_new = grow ? mx : m;
         const float mu = (m_new == -INFINITY) ? 0.f : m_new;
-        float rs = 0.f;
+        float rs8[8];
+#pragma unroll
+        for (int v = 0; v < 8; ++v) rs8[v] = 0.f;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           uint32_t pk[16];
@@ -428,11 +479,12 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           for (int v = 0; v < 16; ++v) {
             const float p0 = ex2(x[q * 32 + 2 * v] - mu);
             const float p1 = ex2(x[q * 32 + 2 * v + 1] - mu);
-            rs += p0 + p1;
+            rs8[v & 7] += p0 + p1;
             pk[v] = pack_bf16x2(p0, p1);
           }
           tmem_st16(lane_addr + b * kBN + q * 16, pk);
         }
+        const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
         if (s > 0) {
           // PV(g-1) has landed in O: every phase of o_done is waited, in order; a row whose max
           // moved rescales its O (warp-uniform, as tcgen05.ld/st are)
@@ -488,6 +540,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       if (live && p.lse) p.lse[(size_t)it.bh * p.N + it.q0 + r] = (m + __log2f(l)) * 0.69314718055994531f;
       tc_fence_before();
       mbar_arrive(&bars->o_free);
+      mbar_arrive(&bars->sfree[n & 1]);
     }
   }
 
@@ -503,14 +556,21 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 
 bool attention_tc_supported(const Dims& g) { return g.bf16 && g.d == kD && g.block == kBN; }
 
+size_t attention_tc_scratch_bytes(const Dims& g) {
+  if (!attention_tc_supported(g)) return 0;
+  return (size_t)kMaxCtas * 2 * ((g.C + kBN - 1) / kBN) * kChunkBytes;
+}
+
 cudaError_t launch_attention_tc(const Dims& g, const void* Q, const void* K, const void* V,
                                 const int32_t* kv_idx, const int32_t* kv_cnt, int max_sel,
                                 const int32_t* schedule, const void* cent, const StatsPtrs& st, float scale,
-                                void* O, float* lse, int* status, cudaStream_t s) {
-  CUtensorMap tq, tk, tv, tc;
+                                void* O, float* lse, int* status, void* scratch, cudaStream_t s) {
+  CUtensorMap tq, tk, tv, tc, ts;
   const unsigned long long BH = (unsigned long long)g.B * g.H;
+  const int nchunk = (g.C + kBN - 1) / kBN;
   if (!make_tmap_bf16_3d(&tq, Q, kD, g.N, BH, 64, kBM) || !make_tmap_bf16_3d(&tk, K, kD, g.N, BH, 64, kBN) ||
-      !make_tmap_bf16_3d(&tv, V, kD, g.N, BH, 64, kBN) || !make_tmap_bf16_3d(&tc, cent, kD, g.C, BH, 64, kBN))
+      !make_tmap_bf16_3d(&tv, V, kD, g.N, BH, 64, kBN) || !make_tmap_bf16_3d(&tc, cent, kD, g.C, BH, 64, kBN) ||
+      !make_tmap_bf16_tiles(&ts, scratch, kD, kBN, (uint64_t)kMaxCtas * 2 * nchunk, kChunkBytes, kBN))
     return cudaErrorInvalidValue;
   Params p;
   p.kv_idx = kv_idx;
@@ -521,11 +581,12 @@ cudaError_t launch_attention_tc(const Dims& g, const void* Q, const void* K, con
   p.O = (__nv_bfloat16*)O;
   p.lse = lse;
   p.status = status;
+  p.scratch = static_cast<uint8_t*>(scratch);
   p.N = g.N;
   p.C = g.C;
   p.nB = g.nB;
   p.n_items = (int)(BH * g.nB);
-  p.nchunk = (g.C + kBN - 1) / kBN;
+  p.nchunk = nchunk;
   p.scale_log2 = scale * 1.4426950408889634f;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
@@ -533,8 +594,8 @@ cudaError_t launch_attention_tc(const Dims& g, const void* Q, const void* K, con
   cudaError_t e = cudaFuncSetAttribute(attention_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kSmemBytes);
   if (e != cudaSuccess) return e;
-  const int grid = min(sms, p.n_items);
-  attention_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, tc, p);
+  const int grid = min(min(sms, kMaxCtas), p.n_items);
+  attention_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, tc, ts, p);
   return cudaGetLastError();
 }
 

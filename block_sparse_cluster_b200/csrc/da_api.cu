@@ -31,6 +31,8 @@ da_status check_dims(const da_dims* dims, Dims* g) {
   const long long BH = (long long)dims->B * dims->H;
   // work items and block-row indices are int32 on the device
   if (BH * g->nB >= (1LL << 31) || BH * dims->N >= (1LL << 31)) return DA_ERR_SHAPE;
+  // the tensor-core path addresses block entries (block row x block + entry) in 32 bits
+  if (g->bf16 && BH * g->nB * g->block >= (1LL << 32)) return DA_ERR_SHAPE;
   return DA_OK;
 }
 
@@ -155,7 +157,7 @@ da_status da_attention(const da_dims* dims, const void* Q, const void* K, const 
   if (e == cudaSuccess) {
     if (attention_tc_supported(g))
       e = launch_attention_tc(g, Q, K, V, mask->kv_idx, mask->kv_cnt, mask->max_sel, sched, centroids, sp, scale,
-                              O, lse, status, s);
+                              O, lse, status, static_cast<char*>(ws) + L.comp, s);
     else
       e = (g.bf16 ? launch_attention_simt_bf16 : launch_attention_simt_f32)(
           g, Q, K, V, mask->kv_idx, mask->kv_cnt, mask->max_sel, sched, centroids, sp, scale, O, lse, status, s);

@@ -27,7 +27,7 @@ struct Dims {
 
 // Workspace layout (byte offsets), shared by every call.
 struct WsLayout {
-  size_t status, norms, sched, total;
+  size_t status, norms, sched, comp, total;
 };
 WsLayout ws_layout(const Dims& g);
 
@@ -45,10 +45,11 @@ cudaError_t launch_reassign_tc(const Dims& g, const void* K, const void* V, cons
 
 // attention_tc.cu
 bool attention_tc_supported(const Dims& g);
+size_t attention_tc_scratch_bytes(const Dims& g);   // per-CTA compensation scratch, all CTAs
 cudaError_t launch_attention_tc(const Dims& g, const void* Q, const void* K, const void* V,
                                 const int32_t* kv_idx, const int32_t* kv_cnt, int max_sel,
                                 const int32_t* schedule, const void* cent, const StatsPtrs& st, float scale,
-                                void* O, float* lse, int* status, cudaStream_t s);
+                                void* O, float* lse, int* status, void* scratch, cudaStream_t s);
 
 // simt_f32.cu / simt_bf16.cu
 #define DA_SIMT_DECL(SUFFIX)                                                                                 \

@@ -15,7 +15,8 @@ WsLayout ws_layout(const Dims& g) {
   L.status = 0;
   L.norms = 256;
   L.sched = L.norms + up(BH * g.C * sizeof(float));
-  L.total = L.sched + up(BH * g.nB * sizeof(int32_t));
+  L.comp = L.sched + up(BH * g.nB * sizeof(int32_t));
+  L.total = L.comp + up(attention_tc_scratch_bytes(g));
   return L;
 }
 

@@ -30,4 +30,19 @@ inline bool make_tmap_bf16_3d(CUtensorMap* m, const void* ptr, uint64_t inner, u
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// A bf16 tensor of `depth` tiles, each `rows` x `inner` (inner contiguous, rows `inner`*2 bytes
+// apart), tiles `tile_stride` bytes apart; boxes of box_rows x 64 elements, 128-byte swizzle.
+inline bool make_tmap_bf16_tiles(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows, uint64_t depth,
+                                 uint64_t tile_stride, uint32_t box_rows) {
+  EncodeTiledFn fn = get_encode_tiled();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {inner, rows, depth};
+  cuuint64_t strides[2] = {inner * 2, tile_stride};
+  cuuint32_t box[3] = {64, box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace da

@@ -19,7 +19,9 @@ interleavings, and checks that
 
 It mirrors the step structure of attention_tc.cu: per work item, one step per
 selected block followed by one step per 128-cluster chunk, a 3-stage K/V ring,
-S double-buffered in TMEM, P in the S buffer, O accumulated across the item.
+S double-buffered in TMEM, P in the S buffer, O accumulated across the item,
+and the compensation builder one item ahead, writing a double-buffered scratch
+that the producer copies into the ring.
 """
 import random
 
@@ -62,22 +64,25 @@ class Barrier:
 
 
 class Machine:
-    def __init__(self, items, nchunk, rng, old_builder=False):
+    def __init__(self, items, nchunk, rng, old_builder=False, skip_sfree=False):
         self.items = items                     # list of nsel per item of one CTA
         self.nchunk = nchunk
         self.rng = rng
         self.old_builder = old_builder
+        self.skip_sfree = skip_sfree
         B = Barrier
         self.q_full, self.q_empty = B("q_full", 1), B("q_empty", 1)
         self.k_full = [B(f"k_full{i}", 1) for i in range(STAGES)]
         self.v_full = [B(f"v_full{i}", 1) for i in range(STAGES)]
         self.st_empty = [B(f"st_empty{i}", 1) for i in range(STAGES)]
-        self.bfree = [B(f"bfree{i}", 1) for i in range(STAGES)]
+        self.bready = [B(f"bready{i}", 1) for i in range(2)]     # scratch buffer built
+        self.sfree = [B(f"sfree{i}", 1) for i in range(2)]       # scratch buffer released
+        self.scratch_version = [None, None]
         self.s_full = [B(f"s_full{i}", 1) for i in range(2)]
         self.p_ready = [B(f"p_ready{i}", 1) for i in range(2)]
         self.o_done, self.o_free = B("o_done", 1), B("o_free", 1)
         self.tc_queue = []                     # in-order tensor core: ("mma", reads, writes) / ("commit", bar)
-        self.tma = []                          # in flight: (bar, bytes, slot_tag)
+        self.tma = []                          # in flight: (bar, buffer written, buffers read)
         self.readers = {}                      # resource -> units with an operation in flight on it
 
     # ---- resources: in-flight users of each buffer, tagged by unit
@@ -116,16 +121,19 @@ class Machine:
             progressed = True
         if self.tma and self.rng.random() < 0.5:
             i = self.rng.randrange(len(self.tma))
-            bar, n, res = self.tma.pop(i)
-            self._end_read(res, "tma")
-            bar.complete_tx(n)
+            bar, dst, srcs = self.tma.pop(i)
+            for r in [dst] + srcs:
+                self._end_read(r, "tma")
+            bar.complete_tx(1)
             progressed = True
         return progressed
 
-    def tma_load(self, bar, res):
+    def tma_load(self, bar, res, srcs=()):
+        """A copy into buffer `res` (busy until it lands) that reads the buffers `srcs`."""
         self._write(res, "TMA", unit="tma")
-        self._start_read(res, "tma")  # busy until the copy lands
-        self.tma.append((bar, 1, res))
+        for r in [res, *srcs]:
+            self._start_read(r, "tma")
+        self.tma.append((bar, res, list(srcs)))
 
     # ---- roles (generators yield a predicate to wait on)
     def producer(self):
@@ -144,10 +152,18 @@ class Machine:
                     self.v_full[slot].expect_tx(1)
                     self.tma_load(self.v_full[slot], f"V{slot}")
                 else:
-                    if not self.old_builder:
-                        self.bfree[slot].arrive()
-                    self.k_full[slot].expect_tx(1)
-                    self.tma_load(self.k_full[slot], f"K{slot}")
+                    c, buf = s - nsel, n & 1
+                    if self.old_builder:
+                        self.k_full[slot].expect_tx(1)
+                        self.tma_load(self.k_full[slot], f"K{slot}")
+                    else:
+                        if c == 0:
+                            yield lambda: self.bready[buf].test(n >> 1)
+                        assert self.scratch_version[buf] == n, "scratch chunk read before it was built"
+                        self.k_full[slot].expect_tx(1)
+                        self.tma_load(self.k_full[slot], f"K{slot}")
+                        self.v_full[slot].expect_tx(1)
+                        self.tma_load(self.v_full[slot], f"V{slot}", srcs=[f"SCR{buf}"])
                 g += 1
 
     def mma(self):
@@ -176,19 +192,26 @@ class Machine:
                 g += 1
 
     def builder(self):
+        if self.old_builder:
+            yield from self.old_builder_role()
+            return
+        for n, nsel in enumerate(self.items):
+            buf = n & 1
+            if n >= 2 and not self.skip_sfree:
+                yield lambda: self.sfree[buf].test((n >> 1) - 1)
+            self._write(f"SCR{buf}", "builder", unit="builder")
+            self.scratch_version[buf] = n
+            self.bready[buf].arrive()
+
+    def old_builder_role(self):
+        """The first design: the builder wrote the ring's value slot itself, waiting on the ring's
+        empty barrier only at its own (compensation) steps."""
         g = 0
-        uses = [0] * STAGES
         for n, nsel in enumerate(self.items):
             g += nsel
             for c in range(self.nchunk):
-                slot = g % STAGES
-                if self.old_builder:
-                    u = g // STAGES
-                    yield lambda: self.st_empty[slot].test(u - 1)
-                else:
-                    use = uses[slot]
-                    uses[slot] += 1
-                    yield lambda: self.bfree[slot].test(use)
+                slot, u = g % STAGES, g // STAGES
+                yield lambda: self.st_empty[slot].test(u - 1)
                 self._write(f"V{slot}", "builder")
                 self.v_full[slot].arrive()
                 g += 1
@@ -211,6 +234,8 @@ class Machine:
             yield lambda: self.o_done.test(g - 1)
             self._write("O", "epilogue")
             self.o_free.arrive()
+            if not self.old_builder:
+                self.sfree[n & 1].arrive()
 
     def run(self, max_iters=200000):
         roles = [self.producer(), self.mma(), self.builder(), self.softmax()]
@@ -260,6 +285,16 @@ def test_model_catches_a_builder_that_skips_ring_phases():
     for seed in range(40):
         try:
             Machine([37], 2, random.Random(seed), old_builder=True).run()
+        except AssertionError:
+            caught += 1
+    assert caught > 0
+
+
+def test_model_catches_a_builder_that_does_not_wait_for_its_buffer():
+    caught = 0
+    for seed in range(40):
+        try:
+            Machine([3, 3, 3, 3, 3], 2, random.Random(seed), skip_sfree=True).run()
         except AssertionError:
             caught += 1
     assert caught > 0
