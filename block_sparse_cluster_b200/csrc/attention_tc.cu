@@ -127,6 +127,25 @@ __device__ __forceinline__ uint8_t* scratch_chunk(const Params& p, int buf, int 
   return p.scratch + (((size_t)blockIdx.x * 2 + buf) * p.nchunk + c) * kChunkBytes;
 }
 
+// Rare path of the builder: cluster row rr sits in more than kSlots selected blocks; subtract the
+// entries after the first kSlots, again in block order (lane l: d = 4l .. 4l+3).
+__device__ __noinline__ void subtract_overflow(const Params& p, const Item& it, size_t hb, int rr, int lane,
+                                               float4& v) {
+  int seen = 0;
+  for (int s = 0; s < it.nsel; ++s) {
+    const int jr = it.row[s];
+    if (jr < 0 || jr >= p.nB) continue;
+    const size_t bj = hb + jr;
+    const int e = p.st.seg_idx[bj * p.C + rr];
+    if (e == 0xFF) continue;
+    if (seen >= kSlots) {
+      const float4 y = ldg4(p.st.seg_vsum + (bj * kBN + e) * kD + 4 * lane);
+      v.x -= y.x; v.y -= y.y; v.z -= y.z; v.w -= y.w;
+    }
+    ++seen;
+  }
+}
+
 // Builder: the compensation chunks of one item into scratch buffer `buf` (t: 0..127).
 __device__ __forceinline__ void build_item(const Params& p, const Item& it, int buf, int t) {
   const int bw = t >> 5, lane = t & 31;
@@ -140,7 +159,7 @@ __device__ __forceinline__ void build_item(const Params& p, const Item& it, int 
     const bool rl = r < p.C;
     int nm = 0, csel = 0;
     uint32_t m0 = 0, m1 = 0, m2 = 0, m3 = 0;
-#pragma unroll 8
+#pragma unroll 4
     for (int s = 0; s < it.nsel; ++s) {
       const int jr = it.row[s];
       const bool ok = rl && jr >= 0 && jr < p.nB;
@@ -185,33 +204,7 @@ __device__ __forceinline__ void build_item(const Params& p, const Item& it, int 
         for (int k = 0; k < kSlots; ++k) {
           v.x -= x[q][k].x; v.y -= x[q][k].y; v.z -= x[q][k].z; v.w -= x[q][k].w;
         }
-        if (nmi[q] > kSlots) {
-          // rare: the row's cluster sits in more than kSlots selected blocks; the remaining
-          // entries, again in block order
-          const int rr = c * kBN + 32 * bw + i0 + q;
-          int seen = 0;
-          for (int s0 = 0; s0 < it.nsel; s0 += 8) {
-            int e8[8];
-            size_t b8[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              const int jr = s0 + u < it.nsel ? it.row[s0 + u] : -1;
-              const bool ok = jr >= 0 && jr < p.nB;
-              b8[u] = hb + (ok ? jr : 0);
-              e8[u] = ok ? (int)p.st.seg_idx[b8[u] * p.C + rr] : 0xFF;
-            }
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              if (e8[u] != 0xFF) {
-                if (seen >= kSlots) {
-                  const float4 y = ldg4(p.st.seg_vsum + (b8[u] * kBN + e8[u]) * kD + 4 * lane);
-                  v.x -= y.x; v.y -= y.y; v.z -= y.z; v.w -= y.w;
-                }
-                ++seen;
-              }
-            }
-          }
-        }
+        if (nmi[q] > kSlots) subtract_overflow(p, it, hb, c * kBN + 32 * bw + i0 + q, lane, v);
         const float iv = invi[q];
         uint2 o;
         o.x = pack_bf16x2(v.x * iv, v.y * iv);
@@ -434,57 +427,74 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         w_ok = w_ok && mbar_wait(&bars->s_full[b], (g >> 1) & 1, abort, status);
         if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
         tc_fence_after();
-        float x[kBN];
-        {
-          uint32_t rr[4][32];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) tmem_ld32(lane_addr + b * kBN + q * 32, rr[q]);
+        // Two compact passes over the S row in TMEM (32 columns at a time): the row max, then
+        // p = 2^(x - m), the row sum and the bf16 P written back over S.  Column c's logit is
+        // x_c * s*log2(e) + bias_c: bias = log2 n^U_c on a compensation step, 0 on a key block
+        // (-inf past the end of a short last block).
+        const uint32_t sbase = lane_addr + b * kBN;
+        const float* bt = sBeta + slot * kBN;
+        const float sl2 = p.scale_log2;
+        const int mode = comp ? 0 : (ncol == kBN ? 1 : 2);      // warp-uniform
+        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll 1
+        for (int q = 0; q < 4; ++q) {
+          uint32_t rr[32];
+          tmem_ld32(sbase + q * 32, rr);
           tmem_wait_ld();
+          if (mode == 0) {
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
+            for (int v = 0; v < 32; ++v) mx4[v & 3] = fmaxf(mx4[v & 3], fmaf(__uint_as_float(rr[v]), sl2, bt[q * 32 + v]));
+          } else if (mode == 1) {
 #pragma unroll
-            for (int v = 0; v < 32; ++v) x[q * 32 + v] = __uint_as_float(rr[q][v]);
-        }
-        float mx8[8];
+            for (int v = 0; v < 32; ++v) mx4[v & 3] = fmaxf(mx4[v & 3], __uint_as_float(rr[v]));
+          } else {
 #pragma unroll
-        for (int v = 0; v < 8; ++v) mx8[v] = -INFINITY;
-        if (comp) {
-          const float* bt = sBeta + slot * kBN;
-#pragma unroll
-          for (int c = 0; c < kBN; ++c) {
-            x[c] = fmaf(x[c], p.scale_log2, bt[c]);
-            mx8[c & 7] = fmaxf(mx8[c & 7], x[c]);
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < kBN; ++c) {
-            x[c] = c < ncol ? x[c] * p.scale_log2 : -INFINITY;
-            mx8[c & 7] = fmaxf(mx8[c & 7], x[c]);
+            for (int v = 0; v < 32; ++v)
+              mx4[v & 3] = fmaxf(mx4[v & 3], q * 32 + v < ncol ? __uint_as_float(rr[v]) : -INFINITY);
           }
         }
-        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+        if (mode != 0 && mx > -INFINITY) mx *= sl2;           // s*log2(e) > 0 commutes with max
         // lazy rescaling: the running max moves only when it grows by more than 2^8
         const bool grow = mx > m + kRescaleLog2 || (m == -INFINITY && mx > -INFINITY);
         const bool need_o = grow && s > 0 && m > -INFINITY;
         const float m_new = grow ? mx : m;
         const float mu = (m_new == -INFINITY) ? 0.f : m_new;
-        float rs8[8];
-#pragma unroll
-        for (int v = 0; v < 8; ++v) rs8[v] = 0.f;
-#pragma unroll
+        float rs4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
         for (int q = 0; q < 4; ++q) {
-          uint32_t pk[16];
+          uint32_t rr[32], pk[16];
+          tmem_ld32(sbase + q * 32, rr);
+          tmem_wait_ld();
+          if (mode == 0) {
 #pragma unroll
-          for (int v = 0; v < 16; ++v) {
-            const float p0 = ex2(x[q * 32 + 2 * v] - mu);
-            const float p1 = ex2(x[q * 32 + 2 * v + 1] - mu);
-            rs8[v & 7] += p0 + p1;
-            pk[v] = pack_bf16x2(p0, p1);
+            for (int v = 0; v < 16; ++v) {
+              const float p0 = ex2(fmaf(__uint_as_float(rr[2 * v]), sl2, bt[q * 32 + 2 * v]) - mu);
+              const float p1 = ex2(fmaf(__uint_as_float(rr[2 * v + 1]), sl2, bt[q * 32 + 2 * v + 1]) - mu);
+              rs4[v & 3] += p0 + p1;
+              pk[v] = pack_bf16x2(p0, p1);
+            }
+          } else if (mode == 1) {
+#pragma unroll
+            for (int v = 0; v < 16; ++v) {
+              const float p0 = ex2(fmaf(__uint_as_float(rr[2 * v]), sl2, -mu));
+              const float p1 = ex2(fmaf(__uint_as_float(rr[2 * v + 1]), sl2, -mu));
+              rs4[v & 3] += p0 + p1;
+              pk[v] = pack_bf16x2(p0, p1);
+            }
+          } else {
+#pragma unroll
+            for (int v = 0; v < 16; ++v) {
+              const int c0 = q * 32 + 2 * v;
+              const float p0 = c0 < ncol ? ex2(fmaf(__uint_as_float(rr[2 * v]), sl2, -mu)) : 0.f;
+              const float p1 = c0 + 1 < ncol ? ex2(fmaf(__uint_as_float(rr[2 * v + 1]), sl2, -mu)) : 0.f;
+              rs4[v & 3] += p0 + p1;
+              pk[v] = pack_bf16x2(p0, p1);
+            }
           }
-          tmem_st16(lane_addr + b * kBN + q * 16, pk);
+          tmem_st16(sbase + q * 16, pk);
         }
-        const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
+        const float rs = (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
         if (s > 0) {
           // PV(g-1) has landed in O: every phase of o_done is waited, in order; a row whose max
           // moved rescales its O (warp-uniform, as tcgen05.ld/st are)
@@ -493,7 +503,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           tc_fence_after();
           if (__any_sync(0xffffffffu, need_o)) {
             const float alpha = need_o ? ex2(m - m_new) : 1.f;
-#pragma unroll
+#pragma unroll 1
             for (int q = 0; q < 4; ++q) {
               uint32_t rr[32];
               tmem_ld32(lane_addr + 2 * kBN + q * 32, rr);
@@ -520,7 +530,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       const float inv = l > 0.f ? 1.f / l : 0.f;
       const bool live = r < it.qlen;
       __nv_bfloat16* op = p.O + ((size_t)it.bh * p.N + it.q0 + r) * kD;
-#pragma unroll
+#pragma unroll 1
       for (int q = 0; q < 4; ++q) {
         uint32_t rr[32];
         tmem_ld32(lane_addr + 2 * kBN + q * 32, rr);
