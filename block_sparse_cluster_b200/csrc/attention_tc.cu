@@ -42,7 +42,8 @@ namespace {
 constexpr int kD = 128;
 constexpr int kBM = 128;                 // query rows per item
 constexpr int kBN = 128;                 // keys per block / clusters per chunk
-constexpr int kStages = 3;
+constexpr int kKStages = 3;             // key / centroid tiles (freed as soon as S is computed)
+constexpr int kVStages = 2;             // value / vbar^U tiles (freed after P V)
 constexpr int kTile = kBN * kD * 2;      // 32 KB bf16 tile
 constexpr int kPanel = kBN * 128;        // one 64-column panel (128 rows x 128 B)
 constexpr float kRescaleLog2 = 8.0f;     // lazy rescale threshold (factor 256)
@@ -51,7 +52,7 @@ constexpr int kWarpProducer = 8;
 constexpr int kWarpMMA = 9;
 // Register split (setmaxnreg): the launch holds 384 x 168 registers; the softmax and builder
 // warpgroups grow, the producer / MMA warpgroup shrinks.
-constexpr int kRegSoftmax = 240, kRegBuilder = 200, kRegIssue = 64;
+constexpr int kRegSoftmax = 200, kRegBuilder = 240, kRegIssue = 64;
 static_assert(128 * (kRegSoftmax + kRegBuilder + kRegIssue) <= kThreads * 168, "register split above the launch");
 constexpr int kMaxCtas = 160;            // scratch is sized for this many persistent CTAs
 constexpr int kChunkBytes = kTile + kBN * 4;   // scratch chunk: vbar^U rows, then log2 n^U
@@ -59,7 +60,7 @@ constexpr int kSlots = 4;                // matches per cluster row handled on t
 
 struct __align__(8) Bars {
   uint64_t q_full, q_empty;
-  uint64_t k_full[kStages], v_full[kStages], st_empty[kStages];
+  uint64_t k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
   uint64_t s_full[2], p_ready[2];
   uint64_t o_done, o_free, drain;
   uint64_t bready[2], sfree[2];          // scratch buffer b: built (builder -> producer), free (softmax -> builder)
@@ -68,8 +69,10 @@ struct __align__(8) Bars {
   volatile int bld_ok[2];
 };
 
-constexpr size_t kSmemBytes =
-    1024 + kTile /*Q*/ + 2 * kStages * kTile /*K,V*/ + kStages * kBN * sizeof(float) /*beta*/ + sizeof(Bars);
+constexpr int kStageRows = 8;           // builder: S_c rows staged per warp and group
+constexpr int kStageFloats = 4 * 2 * kStageRows * kD;   // 4 builder warps x double buffer
+constexpr size_t kSmemBytes = 1024 + kTile /*Q*/ + (kKStages + kVStages) * kTile /*K,V*/ +
+                              kVStages * kBN * sizeof(float) /*beta*/ + kStageFloats * sizeof(float) + sizeof(Bars);
 static_assert(kSmemBytes <= 232448, "shared memory above the 227 KB per-block limit");
 
 struct Params {
@@ -146,71 +149,116 @@ __device__ __noinline__ void subtract_overflow(const Params& p, const Item& it, 
   }
 }
 
-// Builder: the compensation chunks of one item into scratch buffer `buf` (t: 0..127).
-__device__ __forceinline__ void build_item(const Params& p, const Item& it, int buf, int t) {
-  const int bw = t >> 5, lane = t & 31;
+// Builder: the compensation chunks of one item into scratch buffer `buf` (t: 0..127).  Warp w
+// builds chunks w, w+4, ...  For a chunk, lane l first looks up cluster rows 4l .. 4l+3 in every
+// selected block (one 32-bit load of the entry-index row and one 16-byte load of the histogram row
+// per block): the first kSlots entries of each row, in block order, and its selected count.  The
+// warp then builds the rows in groups of kStageRows: the fp32 totals S_c of the next group are
+// copied to shared memory with cp.async while the current group's entry sums are gathered with
+// coalesced loads (lanes over d) and subtracted; rows are scaled by 1 / n^U_c, rounded to bf16 and
+// written to the scratch chunk, whose log2 n^U_c row the lookup lanes write.
+__device__ __forceinline__ void build_item(const Params& p, const Item& it, int buf, int t, float* stage_all) {
+  const int w = t >> 5, lane = t & 31;
+  float* stage = stage_all + w * (2 * kStageRows * kD);
   const size_t hb = (size_t)it.bh * p.nB;      // first block row of the head
   const size_t hc = (size_t)it.bh * p.C;       // first cluster row of the head
-  for (int c = 0; c < p.nchunk; ++c) {
+  for (int c = w; c < p.nchunk; c += 4) {
     uint8_t* tile = scratch_chunk(p, buf, c);
-    // (1) lookups, thread t <-> cluster row r: the entry of r in each selected block (0xFF: none),
-    // the selected count n^sel_r, and the first kSlots entry rows in block order
-    const int r = c * kBN + t;
-    const bool rl = r < p.C;
-    int nm = 0, csel = 0;
-    uint32_t m0 = 0, m1 = 0, m2 = 0, m3 = 0;
+    const int rbase = c * kBN;
+    // (1) lookups: lane <-> rows r0 .. r0+3 (C is a multiple of 32: the four are valid together)
+    const int r0 = rbase + 4 * lane;
+    const bool rl = r0 < p.C;
+    int nm[4] = {0, 0, 0, 0};
+    int4 cs = make_int4(0, 0, 0, 0);
+    uint32_t mp[4][kSlots];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+      for (int k = 0; k < kSlots; ++k) mp[q][k] = 0;
 #pragma unroll 4
     for (int s = 0; s < it.nsel; ++s) {
       const int jr = it.row[s];
       const bool ok = rl && jr >= 0 && jr < p.nB;
-      const size_t cell = (hb + (ok ? jr : 0)) * p.C + (rl ? r : 0);
-      const int e = ok ? (int)p.st.seg_idx[cell] : 0xFF;
-      csel += ok ? p.st.blk_hist[cell] : 0;
-      const bool hit = e != 0xFF;
-      const uint32_t ptr = (uint32_t)((hb + (ok ? jr : 0)) * kBN + (hit ? e : 0));
-      m0 = (hit && nm == 0) ? ptr : m0;
-      m1 = (hit && nm == 1) ? ptr : m1;
-      m2 = (hit && nm == 2) ? ptr : m2;
-      m3 = (hit && nm == 3) ? ptr : m3;
-      nm += hit ? 1 : 0;
-    }
-    const int nU = rl ? p.st.n_tot[hc + r] - csel : 0;
-    reinterpret_cast<float*>(tile + kTile)[t] = nU > 0 ? log2f((float)nU) : -INFINITY;
-    const float inv = nU > 0 ? 1.f / (float)nU : 0.f;
-    // (2) gather: warp bw writes rows 32*bw .. 32*bw+31; lane l holds d = 4l .. 4l+3
-    for (int i0 = 0; i0 < 32; i0 += 4) {
-      float4 a[4], x[4][kSlots];
-      int nmi[4];
-      float invi[4];
+      const size_t bj = hb + (ok ? jr : 0);
+      const size_t cell = bj * p.C + (rl ? r0 : 0);
+      const uint32_t e4 = ok ? __ldg(reinterpret_cast<const unsigned int*>(p.st.seg_idx + cell)) : 0xFFFFFFFFu;
+      const int4 h4 = ok ? __ldg(reinterpret_cast<const int4*>(p.st.blk_hist + cell)) : make_int4(0, 0, 0, 0);
+      cs.x += h4.x; cs.y += h4.y; cs.z += h4.z; cs.w += h4.w;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const int i = i0 + q;
-        const int rr = c * kBN + 32 * bw + i;
-        nmi[q] = __shfl_sync(0xffffffffu, nm, i);
-        invi[q] = __shfl_sync(0xffffffffu, inv, i);
-        const uint32_t p0 = __shfl_sync(0xffffffffu, m0, i), p1 = __shfl_sync(0xffffffffu, m1, i);
-        const uint32_t p2 = __shfl_sync(0xffffffffu, m2, i), p3 = __shfl_sync(0xffffffffu, m3, i);
-        const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-        a[q] = rr < p.C ? ldg4(p.st.S_tot + (hc + rr) * kD + 4 * lane) : z;
-        x[q][0] = nmi[q] > 0 ? ldg4(p.st.seg_vsum + (size_t)p0 * kD + 4 * lane) : z;
-        x[q][1] = nmi[q] > 1 ? ldg4(p.st.seg_vsum + (size_t)p1 * kD + 4 * lane) : z;
-        x[q][2] = nmi[q] > 2 ? ldg4(p.st.seg_vsum + (size_t)p2 * kD + 4 * lane) : z;
-        x[q][3] = nmi[q] > 3 ? ldg4(p.st.seg_vsum + (size_t)p3 * kD + 4 * lane) : z;
+        const uint32_t e = (e4 >> (8 * q)) & 0xFFu;
+        const bool hit = e != 0xFFu;
+        const uint32_t ptr = (uint32_t)(bj * kBN + e);
+#pragma unroll
+        for (int k = 0; k < kSlots; ++k) mp[q][k] = (hit && nm[q] == k) ? ptr : mp[q][k];
+        nm[q] += hit ? 1 : 0;
       }
+    }
+    float inv4[4];
+    {
+      const int4 nt = rl ? __ldg(reinterpret_cast<const int4*>(p.st.n_tot + hc + r0)) : make_int4(0, 0, 0, 0);
+      const int nu[4] = {nt.x - cs.x, nt.y - cs.y, nt.z - cs.z, nt.w - cs.w};
+      float4 bt;
+      float* btp = &bt.x;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        float4 v = a[q];
+        inv4[q] = nu[q] > 0 ? 1.f / (float)nu[q] : 0.f;
+        btp[q] = nu[q] > 0 ? log2f((float)nu[q]) : -INFINITY;
+      }
+      reinterpret_cast<float4*>(tile + kTile)[lane] = bt;
+    }
+    // (2) rows in groups of kStageRows (= lanes 2G and 2G+1 of the lookups)
+    auto prefetch = [&](int G) {
+      const int rg = rbase + G * kStageRows;
+      if (rg < p.C) {
+        const float* src = p.st.S_tot + (hc + rg) * kD;
+        float* dst = stage + (G & 1) * kStageRows * kD;
+#pragma unroll
+        for (int i = 0; i < kStageRows * kD / 128; ++i) cp_async16(dst + (i * 32 + lane) * 4, src + (i * 32 + lane) * 4);
+      }
+      cp_async_commit();
+    };
+    constexpr int kGroups = kBN / kStageRows;
+    prefetch(0);
+    for (int G = 0; G < kGroups; ++G) {
+      if (G + 1 < kGroups) prefetch(G + 1); else cp_async_commit();
+      float4 xm[kStageRows][kSlots];
+      int nmr[kStageRows];
+      float invr[kStageRows];
+#pragma unroll
+      for (int i = 0; i < kStageRows; ++i) {
+        const int src = 2 * G + (i >> 2);           // lookup lane holding row i of the group
+        const int q = i & 3;
+        nmr[i] = __shfl_sync(0xffffffffu, nm[q], src);
+        invr[i] = __shfl_sync(0xffffffffu, inv4[q], src);
 #pragma unroll
         for (int k = 0; k < kSlots; ++k) {
-          v.x -= x[q][k].x; v.y -= x[q][k].y; v.z -= x[q][k].z; v.w -= x[q][k].w;
+          const uint32_t pk = __shfl_sync(0xffffffffu, mp[q][k], src);
+          xm[i][k] = nmr[i] > k ? ldg4(p.st.seg_vsum + (size_t)pk * kD + 4 * lane) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        if (nmi[q] > kSlots) subtract_overflow(p, it, hb, c * kBN + 32 * bw + i0 + q, lane, v);
-        const float iv = invi[q];
+      }
+      cp_async_wait<1>();
+      __syncwarp();
+      const float* sg = stage + (G & 1) * kStageRows * kD;
+#pragma unroll
+      for (int i = 0; i < kStageRows; ++i) {
+        const int rr = rbase + G * kStageRows + i;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (rr < p.C) {
+          v = *reinterpret_cast<const float4*>(sg + i * kD + 4 * lane);
+#pragma unroll
+          for (int k = 0; k < kSlots; ++k) {
+            v.x -= xm[i][k].x; v.y -= xm[i][k].y; v.z -= xm[i][k].z; v.w -= xm[i][k].w;
+          }
+          if (nmr[i] > kSlots) subtract_overflow(p, it, hb, rr, lane, v);
+        }
+        const float iv = invr[i];
         uint2 o;
         o.x = pack_bf16x2(v.x * iv, v.y * iv);
         o.y = pack_bf16x2(v.z * iv, v.w * iv);
-        *reinterpret_cast<uint2*>(tile + (size_t)(32 * bw + i0 + q) * (kD * 2) + lane * 8) = o;
+        *reinterpret_cast<uint2*>(tile + (size_t)(G * kStageRows + i) * (kD * 2) + lane * 8) = o;
       }
+      __syncwarp();     // the staging buffer of this group is refilled two groups later
     }
   }
 }
@@ -223,10 +271,11 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   uint8_t* sQ = base;
-  uint8_t* sK = sQ + kTile;                       // kStages tiles
-  uint8_t* sV = sK + kStages * kTile;             // kStages tiles
-  float* sBeta = reinterpret_cast<float*>(sV + kStages * kTile);   // [kStages][kBN]
-  Bars* bars = reinterpret_cast<Bars*>(sBeta + kStages * kBN);
+  uint8_t* sK = sQ + kTile;                       // kKStages tiles
+  uint8_t* sV = sK + kKStages * kTile;            // kVStages tiles
+  float* sBeta = reinterpret_cast<float*>(sV + kVStages * kTile);   // [kVStages][kBN]
+  float* sStage = sBeta + kVStages * kBN;         // builder staging
+  Bars* bars = reinterpret_cast<Bars*>(sStage + kStageFloats);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -234,10 +283,13 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   if (tid == 0) {
     mbar_init(&bars->q_full, 1);
     mbar_init(&bars->q_empty, 1);
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kKStages; ++s) {
       mbar_init(&bars->k_full[s], 1);
+      mbar_init(&bars->k_empty[s], 1);
+    }
+    for (int s = 0; s < kVStages; ++s) {
       mbar_init(&bars->v_full[s], 1);
-      mbar_init(&bars->st_empty[s], 1);
+      mbar_init(&bars->v_empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars->s_full[b], 1);
@@ -282,33 +334,33 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         tma_load_3d(sQ + kPanel, &tm_q, &bars->q_full, 64, it.q0, it.bh);
         bool ok = true;
         for (int s = 0; s < it.T; ++s, ++g) {
-          const int slot = g % kStages;
-          const uint32_t u = g / kStages;
-          if (!mbar_wait(&bars->st_empty[slot], (u & 1) ^ 1, abort, status)) { ok = false; break; }
-          uint8_t* dk = sK + slot * kTile;
-          uint8_t* dv = sV + slot * kTile;
+          const int ks = g % kKStages, vs = g % kVStages;
+          if (!mbar_wait(&bars->k_empty[ks], ((g / kKStages) & 1) ^ 1, abort, status)) { ok = false; break; }
+          if (!mbar_wait(&bars->v_empty[vs], ((g / kVStages) & 1) ^ 1, abort, status)) { ok = false; break; }
+          uint8_t* dk = sK + ks * kTile;
+          uint8_t* dv = sV + vs * kTile;
           if (s < it.nsel) {
             bool valid;
             const int j = block_of(p, it, s, &valid);
-            mbar_expect_tx(&bars->k_full[slot], kTile);
-            tma_load_3d(dk, &tm_k, &bars->k_full[slot], 0, j * kBN, it.bh);
-            tma_load_3d(dk + kPanel, &tm_k, &bars->k_full[slot], 64, j * kBN, it.bh);
-            mbar_expect_tx(&bars->v_full[slot], kTile);
-            tma_load_3d(dv, &tm_v, &bars->v_full[slot], 0, j * kBN, it.bh);
-            tma_load_3d(dv + kPanel, &tm_v, &bars->v_full[slot], 64, j * kBN, it.bh);
+            mbar_expect_tx(&bars->k_full[ks], kTile);
+            tma_load_3d(dk, &tm_k, &bars->k_full[ks], 0, j * kBN, it.bh);
+            tma_load_3d(dk + kPanel, &tm_k, &bars->k_full[ks], 64, j * kBN, it.bh);
+            mbar_expect_tx(&bars->v_full[vs], kTile);
+            tma_load_3d(dv, &tm_v, &bars->v_full[vs], 0, j * kBN, it.bh);
+            tma_load_3d(dv + kPanel, &tm_v, &bars->v_full[vs], 64, j * kBN, it.bh);
           } else {
             const int c = s - it.nsel;
             const int buf = n & 1;
             // the builder has finished this item's scratch chunks (once per item, in order)
             if (c == 0 && !mbar_wait(&bars->bready[buf], (n >> 1) & 1, abort, status)) { ok = false; break; }
-            mbar_expect_tx(&bars->k_full[slot], kTile);
-            tma_load_3d(dk, &tm_c, &bars->k_full[slot], 0, c * kBN, it.bh);
-            tma_load_3d(dk + kPanel, &tm_c, &bars->k_full[slot], 64, c * kBN, it.bh);
+            mbar_expect_tx(&bars->k_full[ks], kTile);
+            tma_load_3d(dk, &tm_c, &bars->k_full[ks], 0, c * kBN, it.bh);
+            tma_load_3d(dk + kPanel, &tm_c, &bars->k_full[ks], 64, c * kBN, it.bh);
             const int z = ((int)blockIdx.x * 2 + buf) * p.nchunk + c;
-            mbar_expect_tx(&bars->v_full[slot], kTile + kBN * 4);
-            tma_load_3d(dv, &tm_s, &bars->v_full[slot], 0, 0, z);
-            tma_load_3d(dv + kPanel, &tm_s, &bars->v_full[slot], 64, 0, z);
-            bulk_load(sBeta + slot * kBN, scratch_chunk(p, buf, c) + kTile, kBN * 4, &bars->v_full[slot]);
+            mbar_expect_tx(&bars->v_full[vs], kTile + kBN * 4);
+            tma_load_3d(dv, &tm_s, &bars->v_full[vs], 0, 0, z);
+            tma_load_3d(dv + kPanel, &tm_s, &bars->v_full[vs], 64, 0, z);
+            bulk_load(sBeta + vs * kBN, scratch_chunk(p, buf, c) + kTile, kBN * 4, &bars->v_full[vs]);
           }
         }
         if (!ok) break;
@@ -316,10 +368,10 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       // no copy may still be in flight when the CTA leaves (this matters only after an abort:
       // otherwise the MMA issuer has consumed every load)
       if (nq > 0) mbar_wait_drain(&bars->q_full, (nq - 1) & 1);
-      for (uint32_t gd = g >= kStages ? g - kStages : 0; gd < g; ++gd) {
-        mbar_wait_drain(&bars->k_full[gd % kStages], (gd / kStages) & 1);
-        mbar_wait_drain(&bars->v_full[gd % kStages], (gd / kStages) & 1);
-      }
+      for (uint32_t gd = g >= kKStages ? g - kKStages : 0; gd < g; ++gd)
+        mbar_wait_drain(&bars->k_full[gd % kKStages], (gd / kKStages) & 1);
+      for (uint32_t gd = g >= kVStages ? g - kVStages : 0; gd < g; ++gd)
+        mbar_wait_drain(&bars->v_full[gd % kVStages], (gd / kVStages) & 1);
     }
   } else if (warp == kWarpMMA) {
     // ------------------------------------------------------------------ MMA issuer
@@ -330,8 +382,8 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       uint32_t g = 0;
       int n = 0;
       auto issue_s = [&](uint32_t gs) {
-        const int slot = gs % kStages;
-        const uint32_t kb = smem_u32(sK + slot * kTile);
+        const int ks = gs % kKStages;
+        const uint32_t kb = smem_u32(sK + ks * kTile);
         const uint32_t d = tmem + (gs & 1) * kBN;
 #pragma unroll
         for (int ks = 0; ks < kD / 16; ++ks) {
@@ -339,6 +391,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           umma_ss(d, sdesc_sw128(q0 + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), idesc_qk, ks > 0);
         }
         umma_commit(&bars->s_full[gs & 1]);
+        umma_commit(&bars->k_empty[ks]);
       };
       bool ok = true;
       for (int k = blockIdx.x; k < p.n_items && ok; k += gridDim.x, ++n) {
@@ -346,24 +399,24 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         if (!mbar_wait(&bars->q_full, n & 1, abort, status)) break;
         tc_fence_after();
         const uint32_t g0 = g;
-        if (!mbar_wait(&bars->k_full[g0 % kStages], (g0 / kStages) & 1, abort, status)) break;
+        if (!mbar_wait(&bars->k_full[g0 % kKStages], (g0 / kKStages) & 1, abort, status)) break;
         tc_fence_after();
         issue_s(g0);
         for (int s = 0; s < it.T; ++s, ++g) {
           if (s + 1 < it.T) {
             const uint32_t gn = g + 1;
-            if (!mbar_wait(&bars->k_full[gn % kStages], (gn / kStages) & 1, abort, status)) { ok = false; break; }
+            if (!mbar_wait(&bars->k_full[gn % kKStages], (gn / kKStages) & 1, abort, status)) { ok = false; break; }
             tc_fence_after();
             issue_s(gn);
           } else {
             umma_commit(&bars->q_empty);
           }
-          const int slot = g % kStages;
+          const int vs = g % kVStages;
           if (!mbar_wait(&bars->p_ready[g & 1], (g >> 1) & 1, abort, status)) { ok = false; break; }
-          if (!mbar_wait(&bars->v_full[slot], (g / kStages) & 1, abort, status)) { ok = false; break; }
+          if (!mbar_wait(&bars->v_full[vs], (g / kVStages) & 1, abort, status)) { ok = false; break; }
           if (s == 0 && !mbar_wait(&bars->o_free, (n & 1) ^ 1, abort, status)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t vb = smem_u32(sV + slot * kTile);
+          const uint32_t vb = smem_u32(sV + vs * kTile);
           const uint32_t pt = tmem + (g & 1) * kBN;       // P: bf16 pairs in the S buffer's first 64 columns
 #pragma unroll
           for (int ks = 0; ks < kBN / 16; ++ks) {
@@ -371,7 +424,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             umma_ts(tmem + 2 * kBN, pt + ks * 8, sdesc_sw128(vb + ks * 2048, kPanel, 1024), idesc_pv,
                     (s > 0 || ks > 0) ? 1u : 0u);
           }
-          umma_commit(&bars->st_empty[slot]);
+          umma_commit(&bars->v_empty[vs]);
           umma_commit(&bars->o_done);
         }
       }
@@ -394,7 +447,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       if (t == 0) bars->bld_ok[n & 1] = n < 2 || mbar_wait(&bars->sfree[buf], ((n >> 1) - 1) & 1, abort, status);
       asm volatile("bar.sync 2, 128;" ::: "memory");
       if (!bars->bld_ok[n & 1]) break;
-      build_item(p, it, buf, t);
+      build_item(p, it, buf, t, sStage);
       fence_async_global();
       asm volatile("bar.sync 2, 128;" ::: "memory");
       if (t == 0) mbar_arrive(&bars->bready[buf]);
@@ -413,7 +466,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       bool ok = true;
       for (int s = 0; s < it.T; ++s, ++g) {
         const int b = g & 1;
-        const int slot = g % kStages;
+        const int vs = g % kVStages;
         const bool comp = s >= it.nsel;
         int ncol = kBN;                       // valid columns of this tile
         if (!comp) {
@@ -423,7 +476,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
         // every phase of v_full and s_full is waited, in order (the value half of a compensation
         // step carries the chunk's log2 n^U in sBeta)
-        bool w_ok = mbar_wait(&bars->v_full[slot], (g / kStages) & 1, abort, status);
+        bool w_ok = mbar_wait(&bars->v_full[vs], (g / kVStages) & 1, abort, status);
         w_ok = w_ok && mbar_wait(&bars->s_full[b], (g >> 1) & 1, abort, status);
         if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
         tc_fence_after();
@@ -432,7 +485,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         // x_c * s*log2(e) + bias_c: bias = log2 n^U_c on a compensation step, 0 on a key block
         // (-inf past the end of a short last block).
         const uint32_t sbase = lane_addr + b * kBN;
-        const float* bt = sBeta + slot * kBN;
+        const float* bt = sBeta + vs * kBN;
         const float sl2 = p.scale_log2;
         const int mode = comp ? 0 : (ncol == kBN ? 1 : 2);      // warp-uniform
         float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};

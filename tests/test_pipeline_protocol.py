@@ -27,7 +27,8 @@ import random
 
 import pytest
 
-STAGES = 3
+KSTAGES = 3   # key / centroid tiles, freed when S is computed
+VSTAGES = 2   # value / vbar^U tiles, freed after P V
 
 
 class Barrier:
@@ -72,9 +73,10 @@ class Machine:
         self.skip_sfree = skip_sfree
         B = Barrier
         self.q_full, self.q_empty = B("q_full", 1), B("q_empty", 1)
-        self.k_full = [B(f"k_full{i}", 1) for i in range(STAGES)]
-        self.v_full = [B(f"v_full{i}", 1) for i in range(STAGES)]
-        self.st_empty = [B(f"st_empty{i}", 1) for i in range(STAGES)]
+        self.k_full = [B(f"k_full{i}", 1) for i in range(KSTAGES)]
+        self.k_empty = [B(f"k_empty{i}", 1) for i in range(KSTAGES)]
+        self.v_full = [B(f"v_full{i}", 1) for i in range(VSTAGES)]
+        self.v_empty = [B(f"v_empty{i}", 1) for i in range(VSTAGES)]
         self.bready = [B(f"bready{i}", 1) for i in range(2)]     # scratch buffer built
         self.sfree = [B(f"sfree{i}", 1) for i in range(2)]       # scratch buffer released
         self.scratch_version = [None, None]
@@ -144,26 +146,20 @@ class Machine:
             self.q_full.expect_tx(1)
             self.tma_load(self.q_full, "Q")
             for s in range(T):
-                slot, u = g % STAGES, g // STAGES
-                yield lambda: self.st_empty[slot].test(u - 1)
-                if s < nsel:
-                    self.k_full[slot].expect_tx(1)
-                    self.tma_load(self.k_full[slot], f"K{slot}")
-                    self.v_full[slot].expect_tx(1)
-                    self.tma_load(self.v_full[slot], f"V{slot}")
-                else:
-                    c, buf = s - nsel, n & 1
-                    if self.old_builder:
-                        self.k_full[slot].expect_tx(1)
-                        self.tma_load(self.k_full[slot], f"K{slot}")
-                    else:
-                        if c == 0:
-                            yield lambda: self.bready[buf].test(n >> 1)
-                        assert self.scratch_version[buf] == n, "scratch chunk read before it was built"
-                        self.k_full[slot].expect_tx(1)
-                        self.tma_load(self.k_full[slot], f"K{slot}")
-                        self.v_full[slot].expect_tx(1)
-                        self.tma_load(self.v_full[slot], f"V{slot}", srcs=[f"SCR{buf}"])
+                ks, vs = g % KSTAGES, g % VSTAGES
+                yield lambda: self.k_empty[ks].test(g // KSTAGES - 1)
+                yield lambda: self.v_empty[vs].test(g // VSTAGES - 1)
+                comp = s >= nsel
+                if comp and not self.old_builder:
+                    if s == nsel:
+                        buf = n & 1
+                        yield lambda: self.bready[buf].test(n >> 1)
+                    assert self.scratch_version[n & 1] == n, "scratch chunk read before it was built"
+                self.k_full[ks].expect_tx(1)
+                self.tma_load(self.k_full[ks], f"K{ks}")
+                if not (comp and self.old_builder):      # the old builder filled the value slot itself
+                    self.v_full[vs].expect_tx(1)
+                    self.tma_load(self.v_full[vs], f"V{vs}", srcs=[f"SCR{n & 1}"] if comp else [])
                 g += 1
 
     def mma(self):
@@ -171,23 +167,25 @@ class Machine:
         for n, nsel in enumerate(self.items):
             T = nsel + self.nchunk
             yield lambda: self.q_full.test(n)
-            yield lambda: self.k_full[g % STAGES].test(g // STAGES)
-            self.tc_issue_mma(["Q", f"K{g % STAGES}"], [f"S{g & 1}"])
+            yield lambda: self.k_full[g % KSTAGES].test(g // KSTAGES)
+            self.tc_issue_mma(["Q", f"K{g % KSTAGES}"], [f"S{g & 1}"])
             self.tc_commit(self.s_full[g & 1])
+            self.tc_commit(self.k_empty[g % KSTAGES])
             for s in range(T):
                 if s + 1 < T:
                     gn = g + 1
-                    yield lambda: self.k_full[gn % STAGES].test(gn // STAGES)
-                    self.tc_issue_mma(["Q", f"K{gn % STAGES}"], [f"S{gn & 1}"])
+                    yield lambda: self.k_full[gn % KSTAGES].test(gn // KSTAGES)
+                    self.tc_issue_mma(["Q", f"K{gn % KSTAGES}"], [f"S{gn & 1}"])
                     self.tc_commit(self.s_full[gn & 1])
+                    self.tc_commit(self.k_empty[gn % KSTAGES])
                 else:
                     self.tc_commit(self.q_empty)
                 yield lambda: self.p_ready[g & 1].test(g >> 1)
-                yield lambda: self.v_full[g % STAGES].test(g // STAGES)
+                yield lambda: self.v_full[g % VSTAGES].test(g // VSTAGES)
                 if s == 0:
                     yield lambda: self.o_free.test(n - 1)
-                self.tc_issue_mma([f"S{g & 1}", f"V{g % STAGES}"], ["O"])
-                self.tc_commit(self.st_empty[g % STAGES])
+                self.tc_issue_mma([f"S{g & 1}", f"V{g % VSTAGES}"], ["O"])
+                self.tc_commit(self.v_empty[g % VSTAGES])
                 self.tc_commit(self.o_done)
                 g += 1
 
@@ -210,10 +208,10 @@ class Machine:
         for n, nsel in enumerate(self.items):
             g += nsel
             for c in range(self.nchunk):
-                slot, u = g % STAGES, g // STAGES
-                yield lambda: self.st_empty[slot].test(u - 1)
-                self._write(f"V{slot}", "builder")
-                self.v_full[slot].arrive()
+                vs, u = g % VSTAGES, g // VSTAGES
+                yield lambda: self.v_empty[vs].test(u - 1)
+                self._write(f"V{vs}", "builder")
+                self.v_full[vs].arrive()
                 g += 1
 
     def softmax(self):
@@ -221,8 +219,8 @@ class Machine:
         for n, nsel in enumerate(self.items):
             T = nsel + self.nchunk
             for s in range(T):
-                b, slot = g & 1, g % STAGES
-                yield lambda: self.v_full[slot].test(g // STAGES)
+                b, vs = g & 1, g % VSTAGES
+                yield lambda: self.v_full[vs].test(g // VSTAGES)
                 yield lambda: self.s_full[b].test(g >> 1)
                 assert not self.readers.get(f"S{b}"), "S read before its MMA completed"
                 self._write(f"S{b}", "softmax (P)")
