@@ -52,11 +52,12 @@ constexpr int kWarpProducer = 8;
 constexpr int kWarpMMA = 9;
 // Register split (setmaxnreg): the launch holds 384 x 168 registers; the softmax and builder
 // warpgroups grow, the producer / MMA warpgroup shrinks.
-constexpr int kRegSoftmax = 200, kRegBuilder = 240, kRegIssue = 64;
+constexpr int kRegSoftmax = 192, kRegBuilder = 248, kRegIssue = 64;
 static_assert(128 * (kRegSoftmax + kRegBuilder + kRegIssue) <= kThreads * 168, "register split above the launch");
 constexpr int kMaxCtas = 160;            // scratch is sized for this many persistent CTAs
 constexpr int kChunkBytes = kTile + kBN * 4;   // scratch chunk: vbar^U rows, then log2 n^U
-constexpr int kSlots = 4;                // matches per cluster row handled on the fast path
+constexpr int kSlots = 8;                // matches per cluster row gathered on the fast path
+constexpr int kRound = 4;                // matches per row loaded in one round of the gather
 
 struct __align__(8) Bars {
   uint64_t q_full, q_empty;
@@ -130,22 +131,31 @@ __device__ __forceinline__ uint8_t* scratch_chunk(const Params& p, int buf, int 
   return p.scratch + (((size_t)blockIdx.x * 2 + buf) * p.nchunk + c) * kChunkBytes;
 }
 
-// Rare path of the builder: cluster row rr sits in more than kSlots selected blocks; subtract the
-// entries after the first kSlots, again in block order (lane l: d = 4l .. 4l+3).
+// Rare path of the builder: cluster row rr sits in more than kSlots selected blocks; add the
+// entries after the first kSlots, in block order, to acc (lane l: d = 4l .. 4l+3).
 __device__ __noinline__ void subtract_overflow(const Params& p, const Item& it, size_t hb, int rr, int lane,
-                                               float4& v) {
+                                               float4& acc) {
   int seen = 0;
-  for (int s = 0; s < it.nsel; ++s) {
-    const int jr = it.row[s];
-    if (jr < 0 || jr >= p.nB) continue;
-    const size_t bj = hb + jr;
-    const int e = p.st.seg_idx[bj * p.C + rr];
-    if (e == 0xFF) continue;
-    if (seen >= kSlots) {
-      const float4 y = ldg4(p.st.seg_vsum + (bj * kBN + e) * kD + 4 * lane);
-      v.x -= y.x; v.y -= y.y; v.z -= y.z; v.w -= y.w;
+  for (int s0 = 0; s0 < it.nsel; s0 += 8) {
+    int e8[8];
+    size_t b8[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int jr = s0 + u < it.nsel ? it.row[s0 + u] : -1;
+      const bool ok = jr >= 0 && jr < p.nB;
+      b8[u] = hb + (ok ? jr : 0);
+      e8[u] = ok ? (int)p.st.seg_idx[b8[u] * p.C + rr] : 0xFF;
     }
-    ++seen;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (e8[u] != 0xFF) {
+        if (seen >= kSlots) {
+          const float4 y = ldg4(p.st.seg_vsum + (b8[u] * kBN + e8[u]) * kD + 4 * lane);
+          acc.x += y.x; acc.y += y.y; acc.z += y.z; acc.w += y.w;
+        }
+        ++seen;
+      }
+    }
   }
 }
 
@@ -222,20 +232,39 @@ __device__ __forceinline__ void build_item(const Params& p, const Item& it, int 
     prefetch(0);
     for (int G = 0; G < kGroups; ++G) {
       if (G + 1 < kGroups) prefetch(G + 1); else cp_async_commit();
-      float4 xm[kStageRows][kSlots];
       int nmr[kStageRows];
       float invr[kStageRows];
 #pragma unroll
       for (int i = 0; i < kStageRows; ++i) {
-        const int src = 2 * G + (i >> 2);           // lookup lane holding row i of the group
-        const int q = i & 3;
-        nmr[i] = __shfl_sync(0xffffffffu, nm[q], src);
-        invr[i] = __shfl_sync(0xffffffffu, inv4[q], src);
+        nmr[i] = __shfl_sync(0xffffffffu, nm[i & 3], 2 * G + (i >> 2));
+        invr[i] = __shfl_sync(0xffffffffu, inv4[i & 3], 2 * G + (i >> 2));
+      }
+      float4 acc[kStageRows];
 #pragma unroll
-        for (int k = 0; k < kSlots; ++k) {
-          const uint32_t pk = __shfl_sync(0xffffffffu, mp[q][k], src);
-          xm[i][k] = nmr[i] > k ? ldg4(p.st.seg_vsum + (size_t)pk * kD + 4 * lane) : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
+      for (int i = 0; i < kStageRows; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      // entry sums, kRound slots per row per round (a second round only when a row of the group
+      // has more than kRound entries); summed in block order
+#pragma unroll
+      for (int k0 = 0; k0 < kSlots; k0 += kRound) {
+        int need = 0;
+#pragma unroll
+        for (int i = 0; i < kStageRows; ++i) need |= nmr[i] > k0;
+        if (!need) break;                                    // warp-uniform
+        float4 xm[kStageRows][kRound];
+#pragma unroll
+        for (int i = 0; i < kStageRows; ++i)
+#pragma unroll
+          for (int k = 0; k < kRound; ++k) {
+            const uint32_t pk = __shfl_sync(0xffffffffu, mp[i & 3][k0 + k], 2 * G + (i >> 2));
+            xm[i][k] = nmr[i] > k0 + k ? ldg4(p.st.seg_vsum + (size_t)pk * kD + 4 * lane)
+                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+#pragma unroll
+        for (int i = 0; i < kStageRows; ++i)
+#pragma unroll
+          for (int k = 0; k < kRound; ++k) {
+            acc[i].x += xm[i][k].x; acc[i].y += xm[i][k].y; acc[i].z += xm[i][k].z; acc[i].w += xm[i][k].w;
+          }
       }
       cp_async_wait<1>();
       __syncwarp();
@@ -246,11 +275,8 @@ __device__ __forceinline__ void build_item(const Params& p, const Item& it, int 
         float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
         if (rr < p.C) {
           v = *reinterpret_cast<const float4*>(sg + i * kD + 4 * lane);
-#pragma unroll
-          for (int k = 0; k < kSlots; ++k) {
-            v.x -= xm[i][k].x; v.y -= xm[i][k].y; v.z -= xm[i][k].z; v.w -= xm[i][k].w;
-          }
-          if (nmr[i] > kSlots) subtract_overflow(p, it, hb, rr, lane, v);
+          if (nmr[i] > kSlots) subtract_overflow(p, it, hb, rr, lane, acc[i]);
+          v.x -= acc[i].x; v.y -= acc[i].y; v.z -= acc[i].z; v.w -= acc[i].w;
         }
         const float iv = invr[i];
         uint2 o;
@@ -260,6 +286,43 @@ __device__ __forceinline__ void build_item(const Params& p, const Item& it, int 
       }
       __syncwarp();     // the staging buffer of this group is refilled two groups later
     }
+  }
+}
+
+// Softmax helpers over 32 columns of S (raw bits in r): logits y = x * s*log2(e) + bias.
+__device__ __forceinline__ float chunk_max(const uint32_t (&r)[32], const float* bias, uint64_t sl2x2) {
+  float m0 = -INFINITY, m1 = -INFINITY;
+#pragma unroll
+  for (int v = 0; v < 8; ++v) {
+    const float4 bb = *reinterpret_cast<const float4*>(bias + 4 * v);
+    const uint64_t y0 = f2_fma(f2_pack(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1])), sl2x2, f2_pack(bb.x, bb.y));
+    const uint64_t y1 = f2_fma(f2_pack(__uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3])), sl2x2, f2_pack(bb.z, bb.w));
+    float a, c, d, e;
+    f2_unpack(y0, a, c);
+    f2_unpack(y1, d, e);
+    m0 = fmax3(m0, a, c);
+    m1 = fmax3(m1, d, e);
+  }
+  return fmaxf(m0, m1);
+}
+// p = 2^(y - m) for 32 columns: packed to bf16 pairs in pk, summed (fp32 pairs) into rsum.
+__device__ __forceinline__ void chunk_exp(const uint32_t (&r)[32], const float* bias, uint64_t sl2x2, uint64_t negmu,
+                                          uint32_t (&pk)[16], uint64_t& rsum) {
+#pragma unroll
+  for (int v = 0; v < 8; ++v) {
+    const float4 bb = *reinterpret_cast<const float4*>(bias + 4 * v);
+    const uint64_t y0 = f2_add(f2_fma(f2_pack(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1])), sl2x2,
+                                      f2_pack(bb.x, bb.y)), negmu);
+    const uint64_t y1 = f2_add(f2_fma(f2_pack(__uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3])), sl2x2,
+                                      f2_pack(bb.z, bb.w)), negmu);
+    float a, c, d, e;
+    f2_unpack(y0, a, c);
+    f2_unpack(y1, d, e);
+    const float pa = ex2(a), pc = ex2(c), pd = ex2(d), pe = ex2(e);
+    rsum = f2_add(rsum, f2_pack(pa, pc));
+    rsum = f2_add(rsum, f2_pack(pd, pe));
+    pk[2 * v] = pack_bf16x2(pa, pc);
+    pk[2 * v + 1] = pack_bf16x2(pd, pe);
   }
 }
 
@@ -342,6 +405,16 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           if (s < it.nsel) {
             bool valid;
             const int j = block_of(p, it, s, &valid);
+            // bias row of a key block: 0 for its keys, -inf past the end of a short last block
+            // (generic stores, published to the softmax by the arrive on v_full below)
+            const int ncol = valid ? min(kBN, p.N - j * kBN) : 0;
+            float4* bb = reinterpret_cast<float4*>(sBeta + vs * kBN);
+#pragma unroll 4
+            for (int c4 = 0; c4 < kBN / 4; ++c4) {
+              const int c = 4 * c4;
+              bb[c4] = make_float4(c < ncol ? 0.f : -INFINITY, c + 1 < ncol ? 0.f : -INFINITY,
+                                   c + 2 < ncol ? 0.f : -INFINITY, c + 3 < ncol ? 0.f : -INFINITY);
+            }
             mbar_expect_tx(&bars->k_full[ks], kTile);
             tma_load_3d(dk, &tm_k, &bars->k_full[ks], 0, j * kBN, it.bh);
             tma_load_3d(dk + kPanel, &tm_k, &bars->k_full[ks], 64, j * kBN, it.bh);
@@ -467,87 +540,59 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       for (int s = 0; s < it.T; ++s, ++g) {
         const int b = g & 1;
         const int vs = g % kVStages;
-        const bool comp = s >= it.nsel;
-        int ncol = kBN;                       // valid columns of this tile
-        if (!comp) {
-          bool valid;
-          const int j = block_of(p, it, s, &valid);
-          ncol = valid ? min(kBN, p.N - j * kBN) : 0;
-        }
         // every phase of v_full and s_full is waited, in order (the value half of a compensation
         // step carries the chunk's log2 n^U in sBeta)
         bool w_ok = mbar_wait(&bars->v_full[vs], (g / kVStages) & 1, abort, status);
         w_ok = w_ok && mbar_wait(&bars->s_full[b], (g >> 1) & 1, abort, status);
         if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
         tc_fence_after();
-        // Two compact passes over the S row in TMEM (32 columns at a time): the row max, then
-        // p = 2^(x - m), the row sum and the bf16 P written back over S.  Column c's logit is
-        // x_c * s*log2(e) + bias_c: bias = log2 n^U_c on a compensation step, 0 on a key block
-        // (-inf past the end of a short last block).
+        // Two passes over the S row in TMEM, 32 columns at a time with the next load in flight: the
+        // row max, then p = 2^(x - m), the row sum and the bf16 P written back over S.  Column c's
+        // logit is x_c * s*log2(e) + bias_c, the bias row in shared memory: log2 n^U_c on a
+        // compensation step, 0 on a key block (-inf past the end of a short last block).
         const uint32_t sbase = lane_addr + b * kBN;
         const float* bt = sBeta + vs * kBN;
-        const float sl2 = p.scale_log2;
-        const int mode = comp ? 0 : (ncol == kBN ? 1 : 2);      // warp-uniform
-        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        const uint64_t sl2x2 = f2_pack(p.scale_log2, p.scale_log2);
+        float mx = -INFINITY;
+        {
+          uint32_t ra[32], rb[32];
+          tmem_ld32(sbase, ra);
 #pragma unroll 1
-        for (int q = 0; q < 4; ++q) {
-          uint32_t rr[32];
-          tmem_ld32(sbase + q * 32, rr);
-          tmem_wait_ld();
-          if (mode == 0) {
-#pragma unroll
-            for (int v = 0; v < 32; ++v) mx4[v & 3] = fmaxf(mx4[v & 3], fmaf(__uint_as_float(rr[v]), sl2, bt[q * 32 + v]));
-          } else if (mode == 1) {
-#pragma unroll
-            for (int v = 0; v < 32; ++v) mx4[v & 3] = fmaxf(mx4[v & 3], __uint_as_float(rr[v]));
-          } else {
-#pragma unroll
-            for (int v = 0; v < 32; ++v)
-              mx4[v & 3] = fmaxf(mx4[v & 3], q * 32 + v < ncol ? __uint_as_float(rr[v]) : -INFINITY);
+          for (int q = 0; q < 4; q += 2) {
+            tmem_wait_ld_into(ra);
+            tmem_ld32(sbase + (q + 1) * 32, rb);
+            mx = fmaxf(mx, chunk_max(ra, bt + q * 32, sl2x2));
+            tmem_wait_ld_into(rb);
+            if (q + 2 < 4) tmem_ld32(sbase + (q + 2) * 32, ra);
+            mx = fmaxf(mx, chunk_max(rb, bt + (q + 1) * 32, sl2x2));
           }
         }
-        float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-        if (mode != 0 && mx > -INFINITY) mx *= sl2;           // s*log2(e) > 0 commutes with max
         // lazy rescaling: the running max moves only when it grows by more than 2^8
         const bool grow = mx > m + kRescaleLog2 || (m == -INFINITY && mx > -INFINITY);
         const bool need_o = grow && s > 0 && m > -INFINITY;
         const float m_new = grow ? mx : m;
         const float mu = (m_new == -INFINITY) ? 0.f : m_new;
-        float rs4[4] = {0.f, 0.f, 0.f, 0.f};
+        uint64_t rsum = 0;
+        {
+          const uint64_t negmu = f2_pack(-mu, -mu);
+          uint32_t ra[32], rb[32];
+          tmem_ld32(sbase, ra);
 #pragma unroll 1
-        for (int q = 0; q < 4; ++q) {
-          uint32_t rr[32], pk[16];
-          tmem_ld32(sbase + q * 32, rr);
-          tmem_wait_ld();
-          if (mode == 0) {
-#pragma unroll
-            for (int v = 0; v < 16; ++v) {
-              const float p0 = ex2(fmaf(__uint_as_float(rr[2 * v]), sl2, bt[q * 32 + 2 * v]) - mu);
-              const float p1 = ex2(fmaf(__uint_as_float(rr[2 * v + 1]), sl2, bt[q * 32 + 2 * v + 1]) - mu);
-              rs4[v & 3] += p0 + p1;
-              pk[v] = pack_bf16x2(p0, p1);
-            }
-          } else if (mode == 1) {
-#pragma unroll
-            for (int v = 0; v < 16; ++v) {
-              const float p0 = ex2(fmaf(__uint_as_float(rr[2 * v]), sl2, -mu));
-              const float p1 = ex2(fmaf(__uint_as_float(rr[2 * v + 1]), sl2, -mu));
-              rs4[v & 3] += p0 + p1;
-              pk[v] = pack_bf16x2(p0, p1);
-            }
-          } else {
-#pragma unroll
-            for (int v = 0; v < 16; ++v) {
-              const int c0 = q * 32 + 2 * v;
-              const float p0 = c0 < ncol ? ex2(fmaf(__uint_as_float(rr[2 * v]), sl2, -mu)) : 0.f;
-              const float p1 = c0 + 1 < ncol ? ex2(fmaf(__uint_as_float(rr[2 * v + 1]), sl2, -mu)) : 0.f;
-              rs4[v & 3] += p0 + p1;
-              pk[v] = pack_bf16x2(p0, p1);
-            }
+          for (int q = 0; q < 4; q += 2) {
+            uint32_t pk[16];
+            tmem_wait_ld_into(ra);
+            tmem_ld32(sbase + (q + 1) * 32, rb);
+            chunk_exp(ra, bt + q * 32, sl2x2, negmu, pk, rsum);
+            tmem_st16(sbase + q * 16, pk);
+            tmem_wait_ld_into(rb);
+            if (q + 2 < 4) tmem_ld32(sbase + (q + 2) * 32, ra);
+            chunk_exp(rb, bt + (q + 1) * 32, sl2x2, negmu, pk, rsum);
+            tmem_st16(sbase + (q + 1) * 16, pk);
           }
-          tmem_st16(sbase + q * 16, pk);
         }
-        const float rs = (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
+        float rs_lo, rs_hi;
+        f2_unpack(rsum, rs_lo, rs_hi);
+        const float rs = rs_lo + rs_hi;
         if (s > 0) {
           // PV(g-1) has landed in O: every phase of o_done is waited, in order; a row whose max
           // moved rescales its O (warp-uniform, as tcgen05.ld/st are)
