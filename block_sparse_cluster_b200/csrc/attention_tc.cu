@@ -44,6 +44,7 @@ constexpr int kBM = 128;                 // query rows per item
 constexpr int kBN = 128;                 // keys per block / clusters per chunk
 constexpr int kKStages = 3;             // key / centroid tiles (freed as soon as S is computed)
 constexpr int kVStages = 2;             // value / vbar^U tiles (freed after P V)
+constexpr int kBStages = 3;             // bias rows of the softmax (freed after the softmax pass)
 constexpr int kTile = kBN * kD * 2;      // 32 KB bf16 tile
 constexpr int kPanel = kBN * 128;        // one 64-column panel (128 rows x 128 B)
 constexpr float kRescaleLog2 = 8.0f;     // lazy rescale threshold (factor 256)
@@ -62,6 +63,7 @@ constexpr int kRound = 4;                // matches per row loaded in one round 
 struct __align__(8) Bars {
   uint64_t q_full, q_empty;
   uint64_t k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
+  uint64_t b_full[kBStages], b_empty[kBStages];
   uint64_t s_full[2], p_ready[2];
   uint64_t o_done, o_free, drain;
   uint64_t bready[2], sfree[2];          // scratch buffer b: built (builder -> producer), free (softmax -> builder)
@@ -73,7 +75,7 @@ struct __align__(8) Bars {
 constexpr int kStageRows = 8;           // builder: S_c rows staged per warp and group
 constexpr int kStageFloats = 4 * 2 * kStageRows * kD;   // 4 builder warps x double buffer
 constexpr size_t kSmemBytes = 1024 + kTile /*Q*/ + (kKStages + kVStages) * kTile /*K,V*/ +
-                              kVStages * kBN * sizeof(float) /*beta*/ + kStageFloats * sizeof(float) + sizeof(Bars);
+                              kBStages * kBN * sizeof(float) /*bias*/ + kStageFloats * sizeof(float) + sizeof(Bars);
 static_assert(kSmemBytes <= 232448, "shared memory above the 227 KB per-block limit");
 
 struct Params {
@@ -336,8 +338,8 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   uint8_t* sQ = base;
   uint8_t* sK = sQ + kTile;                       // kKStages tiles
   uint8_t* sV = sK + kKStages * kTile;            // kVStages tiles
-  float* sBeta = reinterpret_cast<float*>(sV + kVStages * kTile);   // [kVStages][kBN]
-  float* sStage = sBeta + kVStages * kBN;         // builder staging
+  float* sBias = reinterpret_cast<float*>(sV + kVStages * kTile);   // [kBStages][kBN]
+  float* sStage = sBias + kBStages * kBN;         // builder staging
   Bars* bars = reinterpret_cast<Bars*>(sStage + kStageFloats);
 
   const int tid = threadIdx.x;
@@ -353,6 +355,10 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     for (int s = 0; s < kVStages; ++s) {
       mbar_init(&bars->v_full[s], 1);
       mbar_init(&bars->v_empty[s], 1);
+    }
+    for (int s = 0; s < kBStages; ++s) {
+      mbar_init(&bars->b_full[s], 1);
+      mbar_init(&bars->b_empty[s], 128);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars->s_full[b], 1);
@@ -380,10 +386,12 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   if (warp >= 8) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegIssue));
   if (warp == kWarpProducer) {
     // ------------------------------------------------------------------ producer
+    // lane 0: query tiles, key / centroid tiles and the softmax bias rows; lane 1: value tiles.
+    // The two streams wait on separate barriers, so a value slot still in use never holds back
+    // the next key tile.
     if (lane == 0) {
       tma_prefetch(&tm_q);
       tma_prefetch(&tm_k);
-      tma_prefetch(&tm_v);
       tma_prefetch(&tm_c);
       tma_prefetch(&tm_s);
       uint32_t g = 0;
@@ -397,52 +405,78 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         tma_load_3d(sQ + kPanel, &tm_q, &bars->q_full, 64, it.q0, it.bh);
         bool ok = true;
         for (int s = 0; s < it.T; ++s, ++g) {
-          const int ks = g % kKStages, vs = g % kVStages;
+          const int ks = g % kKStages, bs = g % kBStages;
+          const int buf = n & 1;
           if (!mbar_wait(&bars->k_empty[ks], ((g / kKStages) & 1) ^ 1, abort, status)) { ok = false; break; }
-          if (!mbar_wait(&bars->v_empty[vs], ((g / kVStages) & 1) ^ 1, abort, status)) { ok = false; break; }
           uint8_t* dk = sK + ks * kTile;
-          uint8_t* dv = sV + vs * kTile;
           if (s < it.nsel) {
             bool valid;
             const int j = block_of(p, it, s, &valid);
+            mbar_expect_tx(&bars->k_full[ks], kTile);
+            tma_load_3d(dk, &tm_k, &bars->k_full[ks], 0, j * kBN, it.bh);
+            tma_load_3d(dk + kPanel, &tm_k, &bars->k_full[ks], 64, j * kBN, it.bh);
             // bias row of a key block: 0 for its keys, -inf past the end of a short last block
-            // (generic stores, published to the softmax by the arrive on v_full below)
+            // (generic stores, published to the softmax by the arrive on b_full)
+            if (!mbar_wait(&bars->b_empty[bs], ((g / kBStages) & 1) ^ 1, abort, status)) { ok = false; break; }
             const int ncol = valid ? min(kBN, p.N - j * kBN) : 0;
-            float4* bb = reinterpret_cast<float4*>(sBeta + vs * kBN);
+            float4* bb = reinterpret_cast<float4*>(sBias + bs * kBN);
 #pragma unroll 4
             for (int c4 = 0; c4 < kBN / 4; ++c4) {
               const int c = 4 * c4;
               bb[c4] = make_float4(c < ncol ? 0.f : -INFINITY, c + 1 < ncol ? 0.f : -INFINITY,
                                    c + 2 < ncol ? 0.f : -INFINITY, c + 3 < ncol ? 0.f : -INFINITY);
             }
-            mbar_expect_tx(&bars->k_full[ks], kTile);
-            tma_load_3d(dk, &tm_k, &bars->k_full[ks], 0, j * kBN, it.bh);
-            tma_load_3d(dk + kPanel, &tm_k, &bars->k_full[ks], 64, j * kBN, it.bh);
-            mbar_expect_tx(&bars->v_full[vs], kTile);
-            tma_load_3d(dv, &tm_v, &bars->v_full[vs], 0, j * kBN, it.bh);
-            tma_load_3d(dv + kPanel, &tm_v, &bars->v_full[vs], 64, j * kBN, it.bh);
+            mbar_arrive(&bars->b_full[bs]);
           } else {
             const int c = s - it.nsel;
-            const int buf = n & 1;
             // the builder has finished this item's scratch chunks (once per item, in order)
             if (c == 0 && !mbar_wait(&bars->bready[buf], (n >> 1) & 1, abort, status)) { ok = false; break; }
             mbar_expect_tx(&bars->k_full[ks], kTile);
             tma_load_3d(dk, &tm_c, &bars->k_full[ks], 0, c * kBN, it.bh);
             tma_load_3d(dk + kPanel, &tm_c, &bars->k_full[ks], 64, c * kBN, it.bh);
-            const int z = ((int)blockIdx.x * 2 + buf) * p.nchunk + c;
-            mbar_expect_tx(&bars->v_full[vs], kTile + kBN * 4);
-            tma_load_3d(dv, &tm_s, &bars->v_full[vs], 0, 0, z);
-            tma_load_3d(dv + kPanel, &tm_s, &bars->v_full[vs], 64, 0, z);
-            bulk_load(sBeta + vs * kBN, scratch_chunk(p, buf, c) + kTile, kBN * 4, &bars->v_full[vs]);
+            if (!mbar_wait(&bars->b_empty[bs], ((g / kBStages) & 1) ^ 1, abort, status)) { ok = false; break; }
+            mbar_expect_tx(&bars->b_full[bs], kBN * 4);
+            bulk_load(sBias + bs * kBN, scratch_chunk(p, buf, c) + kTile, kBN * 4, &bars->b_full[bs]);
           }
         }
         if (!ok) break;
       }
       // no copy may still be in flight when the CTA leaves (this matters only after an abort:
-      // otherwise the MMA issuer has consumed every load)
+      // otherwise the consumers have waited for every load)
       if (nq > 0) mbar_wait_drain(&bars->q_full, (nq - 1) & 1);
       for (uint32_t gd = g >= kKStages ? g - kKStages : 0; gd < g; ++gd)
         mbar_wait_drain(&bars->k_full[gd % kKStages], (gd / kKStages) & 1);
+      for (uint32_t gd = g >= kBStages ? g - kBStages : 0; gd < g; ++gd)
+        mbar_wait_drain(&bars->b_full[gd % kBStages], (gd / kBStages) & 1);
+    } else if (lane == 1) {
+      tma_prefetch(&tm_v);
+      uint32_t g = 0;
+      int n = 0;
+      for (int k = blockIdx.x; k < p.n_items && !*abort; k += gridDim.x, ++n) {
+        const Item it = item_at(p, k);
+        bool ok = true;
+        for (int s = 0; s < it.T; ++s, ++g) {
+          const int vs = g % kVStages;
+          const int buf = n & 1;
+          if (!mbar_wait(&bars->v_empty[vs], ((g / kVStages) & 1) ^ 1, abort, status)) { ok = false; break; }
+          uint8_t* dv = sV + vs * kTile;
+          if (s < it.nsel) {
+            bool valid;
+            const int j = block_of(p, it, s, &valid);
+            mbar_expect_tx(&bars->v_full[vs], kTile);
+            tma_load_3d(dv, &tm_v, &bars->v_full[vs], 0, j * kBN, it.bh);
+            tma_load_3d(dv + kPanel, &tm_v, &bars->v_full[vs], 64, j * kBN, it.bh);
+          } else {
+            const int c = s - it.nsel;
+            if (c == 0 && !mbar_wait(&bars->bready[buf], (n >> 1) & 1, abort, status)) { ok = false; break; }
+            const int z = ((int)blockIdx.x * 2 + buf) * p.nchunk + c;
+            mbar_expect_tx(&bars->v_full[vs], kTile);
+            tma_load_3d(dv, &tm_s, &bars->v_full[vs], 0, 0, z);
+            tma_load_3d(dv + kPanel, &tm_s, &bars->v_full[vs], 64, 0, z);
+          }
+        }
+        if (!ok) break;
+      }
       for (uint32_t gd = g >= kVStages ? g - kVStages : 0; gd < g; ++gd)
         mbar_wait_drain(&bars->v_full[gd % kVStages], (gd / kVStages) & 1);
     }
@@ -539,10 +573,9 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       bool ok = true;
       for (int s = 0; s < it.T; ++s, ++g) {
         const int b = g & 1;
-        const int vs = g % kVStages;
-        // every phase of v_full and s_full is waited, in order (the value half of a compensation
-        // step carries the chunk's log2 n^U in sBeta)
-        bool w_ok = mbar_wait(&bars->v_full[vs], (g / kVStages) & 1, abort, status);
+        // every phase of b_full and s_full is waited, in order (b_full: the step's bias row)
+        const int bs = g % kBStages;
+        bool w_ok = mbar_wait(&bars->b_full[bs], (g / kBStages) & 1, abort, status);
         w_ok = w_ok && mbar_wait(&bars->s_full[b], (g >> 1) & 1, abort, status);
         if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
         tc_fence_after();
@@ -551,7 +584,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         // logit is x_c * s*log2(e) + bias_c, the bias row in shared memory: log2 n^U_c on a
         // compensation step, 0 on a key block (-inf past the end of a short last block).
         const uint32_t sbase = lane_addr + b * kBN;
-        const float* bt = sBeta + vs * kBN;
+        const float* bt = sBias + bs * kBN;
         const uint64_t sl2x2 = f2_pack(p.scale_log2, p.scale_log2);
         float mx = -INFINITY;
         {
@@ -590,6 +623,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             tmem_st16(sbase + (q + 1) * 16, pk);
           }
         }
+        mbar_arrive(&bars->b_empty[bs]);          // this thread has read the bias row
         float rs_lo, rs_hi;
         f2_unpack(rsum, rs_lo, rs_hi);
         const float rs = rs_lo + rs_hi;

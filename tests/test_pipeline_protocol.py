@@ -29,6 +29,7 @@ import pytest
 
 KSTAGES = 3   # key / centroid tiles, freed when S is computed
 VSTAGES = 2   # value / vbar^U tiles, freed after P V
+BSTAGES = 3   # softmax bias rows, freed after the softmax has read them
 
 
 class Barrier:
@@ -77,6 +78,8 @@ class Machine:
         self.k_empty = [B(f"k_empty{i}", 1) for i in range(KSTAGES)]
         self.v_full = [B(f"v_full{i}", 1) for i in range(VSTAGES)]
         self.v_empty = [B(f"v_empty{i}", 1) for i in range(VSTAGES)]
+        self.b_full = [B(f"b_full{i}", 1) for i in range(BSTAGES)]
+        self.b_empty = [B(f"b_empty{i}", 1) for i in range(BSTAGES)]
         self.bready = [B(f"bready{i}", 1) for i in range(2)]     # scratch buffer built
         self.sfree = [B(f"sfree{i}", 1) for i in range(2)]       # scratch buffer released
         self.scratch_version = [None, None]
@@ -139,6 +142,7 @@ class Machine:
 
     # ---- roles (generators yield a predicate to wait on)
     def producer(self):
+        """Lane 0 of the producer warp: query tiles, key / centroid tiles, bias rows."""
         g = 0
         for n, nsel in enumerate(self.items):
             T = nsel + self.nchunk
@@ -146,17 +150,38 @@ class Machine:
             self.q_full.expect_tx(1)
             self.tma_load(self.q_full, "Q")
             for s in range(T):
-                ks, vs = g % KSTAGES, g % VSTAGES
-                yield lambda: self.k_empty[ks].test(g // KSTAGES - 1)
-                yield lambda: self.v_empty[vs].test(g // VSTAGES - 1)
+                ks, bs = g % KSTAGES, g % BSTAGES
                 comp = s >= nsel
+                yield lambda: self.k_empty[ks].test(g // KSTAGES - 1)
+                if comp and s == nsel and not self.old_builder:
+                    buf = n & 1
+                    yield lambda: self.bready[buf].test(n >> 1)
+                self.k_full[ks].expect_tx(1)
+                self.tma_load(self.k_full[ks], f"K{ks}")
+                yield lambda: self.b_empty[bs].test(g // BSTAGES - 1)
+                if comp and not self.old_builder:
+                    assert self.scratch_version[n & 1] == n, "scratch chunk read before it was built"
+                    self.b_full[bs].expect_tx(1)
+                    self.tma_load(self.b_full[bs], f"BIAS{bs}", srcs=[f"SCR{n & 1}"])
+                else:
+                    self._write(f"BIAS{bs}", "producer")
+                    self.b_full[bs].arrive()
+                g += 1
+
+    def producer_v(self):
+        """Lane 1 of the producer warp: value / vbar^U tiles."""
+        g = 0
+        for n, nsel in enumerate(self.items):
+            T = nsel + self.nchunk
+            for s in range(T):
+                vs = g % VSTAGES
+                comp = s >= nsel
+                yield lambda: self.v_empty[vs].test(g // VSTAGES - 1)
                 if comp and not self.old_builder:
                     if s == nsel:
                         buf = n & 1
                         yield lambda: self.bready[buf].test(n >> 1)
                     assert self.scratch_version[n & 1] == n, "scratch chunk read before it was built"
-                self.k_full[ks].expect_tx(1)
-                self.tma_load(self.k_full[ks], f"K{ks}")
                 if not (comp and self.old_builder):      # the old builder filled the value slot itself
                     self.v_full[vs].expect_tx(1)
                     self.tma_load(self.v_full[vs], f"V{vs}", srcs=[f"SCR{n & 1}"] if comp else [])
@@ -219,11 +244,13 @@ class Machine:
         for n, nsel in enumerate(self.items):
             T = nsel + self.nchunk
             for s in range(T):
-                b, vs = g & 1, g % VSTAGES
-                yield lambda: self.v_full[vs].test(g // VSTAGES)
+                b, bs = g & 1, g % BSTAGES
+                yield lambda: self.b_full[bs].test(g // BSTAGES)
                 yield lambda: self.s_full[b].test(g >> 1)
                 assert not self.readers.get(f"S{b}"), "S read before its MMA completed"
+                assert not self.readers.get(f"BIAS{bs}"), "bias row read before it landed"
                 self._write(f"S{b}", "softmax (P)")
+                self.b_empty[bs].arrive()
                 if s > 0:
                     yield lambda: self.o_done.test(g - 1)
                     self._write("O", "softmax (rescale)")
@@ -236,7 +263,7 @@ class Machine:
                 self.sfree[n & 1].arrive()
 
     def run(self, max_iters=200000):
-        roles = [self.producer(), self.mma(), self.builder(), self.softmax()]
+        roles = [self.producer(), self.producer_v(), self.mma(), self.builder(), self.softmax()]
         waits = [None] * len(roles)
         done = [False] * len(roles)
         for _ in range(max_iters):
