@@ -1,6 +1,8 @@
 """Build libda.so in-tree with nvcc for sm_100a (one nvcc per source file, in parallel).
 
-    python -m block_sparse_cluster_b200.build
+    python block_sparse_cluster_b200/build.py [--force]
+
+(Run it by path: importing the package loads libda.so, which this script produces.)
 """
 import concurrent.futures as cf
 import glob
