@@ -159,24 +159,23 @@ def oracle_item_sampler(w: W.Workload, seed: int):
     return run
 
 
-def _blas_threads():
-    try:
-        from threadpoolctl import threadpool_info
-        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    except Exception:
-        return 1
+def _single_thread():
+    """Run the oracle on one host core (BLAS pools limited to one thread), so `cores` is exact."""
+    from threadpoolctl import threadpool_limits
+    return threadpool_limits(limits=1)
 
 
 def cpu_baseline(w: W.Workload, seed: int, budget_s: float = 12.0):
     run = oracle_item_sampler(w, seed)
-    run(1)  # warm caches
     flops, t, items = 0.0, 0.0, 0
-    while t < budget_s and items < 400:
-        f, dt = run(4)
-        flops += f
-        t += dt
-        items += 4
-    return {"value": flops / t / 1e12, "unit": "TFLOP/s", "cores": _blas_threads(), "kind": "oracle",
+    with _single_thread():
+        run(1)  # warm caches
+        while t < budget_s and items < 400:
+            f, dt = run(4)
+            flops += f
+            t += dt
+            items += 4
+    return {"value": flops / t / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
             "sample": f"{items} work items of head 0 (reassign of one key block + decoupled attention of one "
                       f"q-block each, random q-blocks), fp64 numpy, {t:.1f} s"}
 
@@ -186,19 +185,20 @@ def run_reference(args, w: W.Workload, ws: int, rank: int):
         return
     run = oracle_item_sampler(w, args.seed)
     per_step = max(1, args.ref_items)
-    for _ in range(args.warmup):
-        run(per_step)
     flops, t = 0.0, 0.0
-    for _ in range(args.steps):
-        f, dt = run(per_step)
-        flops += f
-        t += dt
+    with _single_thread():
+        for _ in range(args.warmup):
+            run(per_step)
+        for _ in range(args.steps):
+            f, dt = run(per_step)
+            flops += f
+            t += dt
     value = flops / t / 1e12
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": _config(w, args),
-            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": _blas_threads(), "kind": "oracle",
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
                              "sample": f"{per_step} random work items of head 0 per step (reassign of one key "
                                        f"block + decoupled attention of one q-block each), fp64 numpy"},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
