@@ -4,7 +4,7 @@ Argument marshalling only: every step of the computation runs in the CUDA
 kernels of libda.so.  The functions carry the names of the C ABI in
 include/da.h and take torch CUDA tensors; they raise DAError when the library
 returns a status other than DA_OK.  Importing this module loads libda.so and
-fails loudly if it has not been built (``python -m block_sparse_cluster_b200.build``).
+fails loudly if it has not been built (``python block_sparse_cluster_b200/build.py``).
 """
 from __future__ import annotations
 
@@ -19,7 +19,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libda.so")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"libda.so is not built ({LIB_PATH}); run python -m block_sparse_cluster_b200.build")
+    raise ImportError(f"libda.so is not built ({LIB_PATH}); run python block_sparse_cluster_b200/build.py")
 _lib = ctypes.CDLL(LIB_PATH)
 
 DA_BF16, DA_F32 = 0, 1
@@ -27,7 +27,7 @@ STATUS_NAMES = ["DA_OK", "DA_ERR_INVALID_ARG", "DA_ERR_SHAPE", "DA_ERR_DTYPE", "
                 "DA_ERR_UNSUPPORTED", "DA_ERR_CUDA", "DA_ERR_TIMEOUT", "DA_ERR_DEVICE_INDEX",
                 "DA_ERR_WORKSPACE"]
 EXPORTS = ["da_version", "da_workspace_bytes", "da_schedule_bytes", "da_reassign", "da_mask_prepare",
-           "da_attention", "da_device_status", "da_status_string"]
+           "da_attention", "da_device_status", "da_status_string", "da_reassign_noalloc"]
 
 
 class DAError(RuntimeError):
@@ -66,6 +66,8 @@ _lib.da_mask_prepare.argtypes = [ctypes.POINTER(_Dims), ctypes.POINTER(_Mask), _
 _lib.da_attention.restype = ctypes.c_int
 _lib.da_attention.argtypes = [ctypes.POINTER(_Dims), _P, _P, _P, ctypes.POINTER(_Mask), _P,
                               ctypes.POINTER(_Stats), ctypes.c_float, _P, _P, _P, ctypes.c_size_t, _P]
+_lib.da_reassign_noalloc.restype = ctypes.c_int
+_lib.da_reassign_noalloc.argtypes = [ctypes.POINTER(_Dims), _P, _P, _P, ctypes.POINTER(_Stats), _P]
 _lib.da_device_status.restype = ctypes.c_int
 _lib.da_device_status.argtypes = [_P, _P]
 _lib.da_status_string.restype = ctypes.c_char_p
@@ -174,6 +176,15 @@ def da_reassign(dims: Dims, K: torch.Tensor, V: torch.Tensor, centroids: torch.T
                 ws: torch.Tensor, stream=None) -> ClusterStats:
     _check(_lib.da_reassign(ctypes.byref(dims.c()), K.data_ptr(), V.data_ptr(), centroids.data_ptr(),
                             ctypes.byref(stats.c()), ws.data_ptr(), ws.numel(), _stream(stream)), "da_reassign")
+    return stats
+
+
+def da_reassign_noalloc(dims: Dims, K: torch.Tensor, V: torch.Tensor, centroids: torch.Tensor,
+                        stats: ClusterStats, stream=None) -> ClusterStats:
+    """da_reassign for callers that cannot allocate device memory: no workspace argument; the
+    library's own fixed device scratch (about 1 MiB, B*H*C <= 262144) is used instead."""
+    _check(_lib.da_reassign_noalloc(ctypes.byref(dims.c()), K.data_ptr(), V.data_ptr(), centroids.data_ptr(),
+                                    ctypes.byref(stats.c()), _stream(stream)), "da_reassign_noalloc")
     return stats
 
 

@@ -160,6 +160,25 @@ DA_API da_status da_attention(const da_dims* dims, const void* Q, const void* K,
                        const da_cluster_stats* stats, float scale, void* O, float* lse,
                        void* ws, size_t ws_bytes, da_stream stream);
 
+/*
+ * Reassign Cache without a caller workspace (the paper has no counterpart: this is a calling
+ * convention of this library).  Some callers cannot call cudaMalloc when they run a step: a
+ * runtime whose device memory is planned once at start-up, a host application whose pool owns all
+ * device memory, or a path where an allocation would synchronise the device.  This call computes
+ * exactly what da_reassign computes, with the same kernels, but keeps its scratch (centroid norms
+ * and a status word) in a fixed file-scope device array of the library, about 1 MiB, held by every
+ * GPU that loads libda.so until the process exits.  It allocates nothing.
+ *   - Limit: B*H*C <= 262144; larger dims return DA_ERR_WORKSPACE before any launch.
+ *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
+ *     that device current; make that first call before any stream capture.
+ *   - Every call on a device shares the array and leaves its contents behind; the status word is
+ *     cleared at the start of each call.  Calls whose kernels overlap on the GPU (for instance on
+ *     two streams) race on the array.
+ *   - Device-side problems (a bounded wait that gave up) are not reported by this call.
+ */
+DA_API da_status da_reassign_noalloc(const da_dims* dims, const void* K, const void* V, const void* centroids,
+                                     const da_cluster_stats* out, da_stream stream);
+
 /* Synchronise `stream`, then report and clear the workspace status word:
  * DA_OK, DA_ERR_TIMEOUT or DA_ERR_DEVICE_INDEX (or DA_ERR_CUDA if the
  * synchronisation itself failed). */
