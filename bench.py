@@ -325,7 +325,7 @@ def main():
             "pct_of_bf16_peak": 100.0 * (value / ws) / peak,
             "breakdown_ms": {"reassign": ms_local - att_ms_local, "attention": att_ms_local},
             "effective_flop_per_step_per_gpu": eff,
-            "roofline": {"bound": "tensor", "kernel": "fused decoupled attention", "achieved": att_tflops,
+            "roofline": {"bound": "tensor", "kernel": "da_attention (compensation chunks + fused attention)", "achieved": att_tflops,
                          "peak": peak, "unit": "TFLOP/s", "frac": att_tflops / peak,
                          "peak_source": f"{kind} bf16 dense (burst)",
                          "frac_of_sustained": att_tflops / float(peaks.get("bf16_tflops_sustained", peak)),
@@ -342,8 +342,9 @@ def main():
         torch.distributed.destroy_process_group()
 
 
-# kernels of ours per timed step: reassign (assignment, block statistics, totals) + attention
-LAUNCHES_PER_STEP = 4
+# kernels of ours per timed step: reassign (centroid norms, assignment with block statistics,
+# totals) + attention (compensation chunks, fused attention)
+LAUNCHES_PER_STEP = 5
 
 if __name__ == "__main__":
     main()

@@ -13,19 +13,17 @@
 // block, then one per 128-cluster chunk.  Every step is a 128 x 128 score tile S = Q K^T (K a
 // key block or a centroid chunk) and a P V product (V a value block or the chunk's vbar^U rows).
 //
-// Roles (384 threads, three warpgroups; registers rebalanced with setmaxnreg):
+// The compensation chunks (vbar^U rows in bf16 and log2 n^U per cluster) of every item are
+// written beforehand by comp_build.cu; here they are loaded like value blocks.
+//
+// Roles (192 threads):
 //   warps 0-3  softmax: thread t owns query row t = TMEM lane t; online softmax with lazy
 //              rescaling (the running max only moves when it grows by more than 2^8), P written
 //              back to TMEM as bf16, final normalisation and store of O;
-//   warps 4-7  builder: one work item ahead of the tensor cores, writes the item's vbar^U rows
-//              (bf16) and log2 n^U to a per-CTA, double-buffered global scratch (L2-resident):
-//              one batch of independent lookups per chunk finds, for each cluster row, the
-//              selected blocks holding that cluster; then each warp gathers 32 rows with
-//              coalesced loads (lanes over d);
-//   warp 8     producer: TMA loads of Q, K / V blocks, centroid chunks and the scratch chunks
-//              into a 3-stage ring;
-//   warp 9     MMA: allocates TMEM, issues tcgen05.mma S(g+1) = Q K^T ahead of O += P(g) V(g);
-//   warps 10-11 idle.
+//   warp 4     producer: lane 0 loads Q, key tiles / centroid chunks (3-stage ring) and the
+//              softmax bias rows (3-stage ring); lane 1 loads value tiles / compensation chunks
+//              (3-stage ring);
+//   warp 5     MMA: allocates TMEM, issues tcgen05.mma S(g+1) = Q K^T ahead of O += P(g) V(g).
 // TMEM columns: S double buffer [0,128) and [128,256), O [256,384).
 //
 // Every mbarrier is waited at every phase, in order, by each role that waits on it (a parity
@@ -43,22 +41,15 @@ constexpr int kD = 128;
 constexpr int kBM = 128;                 // query rows per item
 constexpr int kBN = 128;                 // keys per block / clusters per chunk
 constexpr int kKStages = 3;             // key / centroid tiles (freed as soon as S is computed)
-constexpr int kVStages = 2;             // value / vbar^U tiles (freed after P V)
+constexpr int kVStages = 3;             // value / vbar^U tiles (freed after P V)
 constexpr int kBStages = 3;             // bias rows of the softmax (freed after the softmax pass)
 constexpr int kTile = kBN * kD * 2;      // 32 KB bf16 tile
 constexpr int kPanel = kBN * 128;        // one 64-column panel (128 rows x 128 B)
 constexpr float kRescaleLog2 = 8.0f;     // lazy rescale threshold (factor 256)
-constexpr int kThreads = 384;            // three warpgroups
-constexpr int kWarpProducer = 8;
-constexpr int kWarpMMA = 9;
-// Register split (setmaxnreg): the launch holds 384 x 168 registers; the softmax and builder
-// warpgroups grow, the producer / MMA warpgroup shrinks.
-constexpr int kRegSoftmax = 192, kRegBuilder = 248, kRegIssue = 64;
-static_assert(128 * (kRegSoftmax + kRegBuilder + kRegIssue) <= kThreads * 168, "register split above the launch");
-constexpr int kMaxCtas = 160;            // scratch is sized for this many persistent CTAs
-constexpr int kChunkBytes = kTile + kBN * 4;   // scratch chunk: vbar^U rows, then log2 n^U
-constexpr int kSlots = 8;                // matches per cluster row gathered on the fast path
-constexpr int kRound = 4;                // matches per row loaded in one round of the gather
+constexpr int kThreads = 192;
+constexpr int kWarpProducer = 4;
+constexpr int kWarpMMA = 5;
+constexpr int kChunkBytes = kTile + kBN * 4;   // compensation chunk: vbar^U rows, then log2 n^U
 
 struct __align__(8) Bars {
   uint64_t q_full, q_empty;
@@ -66,16 +57,12 @@ struct __align__(8) Bars {
   uint64_t b_full[kBStages], b_empty[kBStages];
   uint64_t s_full[2], p_ready[2];
   uint64_t o_done, o_free, drain;
-  uint64_t bready[2], sfree[2];          // scratch buffer b: built (builder -> producer), free (softmax -> builder)
   uint32_t tmem_base;
   int abort;
-  volatile int bld_ok[2];
 };
 
-constexpr int kStageRows = 8;           // builder: S_c rows staged per warp and group
-constexpr int kStageFloats = 4 * 2 * kStageRows * kD;   // 4 builder warps x double buffer
 constexpr size_t kSmemBytes = 1024 + kTile /*Q*/ + (kKStages + kVStages) * kTile /*K,V*/ +
-                              kBStages * kBN * sizeof(float) /*bias*/ + kStageFloats * sizeof(float) + sizeof(Bars);
+                              kBStages * kBN * sizeof(float) /*bias*/ + sizeof(Bars);
 static_assert(kSmemBytes <= 232448, "shared memory above the 227 KB per-block limit");
 
 struct Params {
@@ -87,7 +74,7 @@ struct Params {
   __nv_bfloat16* O;
   float* lse;
   int* status;
-  uint8_t* scratch;                      // kMaxCtas x 2 x nchunk chunks of kChunkBytes
+  const uint8_t* comp;                   // [items][nchunk] compensation chunks of kChunkBytes
   int N, C, nB, n_items, nchunk;
   float scale_log2;
 };
@@ -129,166 +116,8 @@ __device__ __forceinline__ int block_of(const Params& p, const Item& it, int s, 
   return *valid ? j : 0;
 }
 
-__device__ __forceinline__ uint8_t* scratch_chunk(const Params& p, int buf, int c) {
-  return p.scratch + (((size_t)blockIdx.x * 2 + buf) * p.nchunk + c) * kChunkBytes;
-}
-
-// Rare path of the builder: cluster row rr sits in more than kSlots selected blocks; add the
-// entries after the first kSlots, in block order, to acc (lane l: d = 4l .. 4l+3).
-__device__ __noinline__ void subtract_overflow(const Params& p, const Item& it, size_t hb, int rr, int lane,
-                                               float4& acc) {
-  int seen = 0;
-  for (int s0 = 0; s0 < it.nsel; s0 += 8) {
-    int e8[8];
-    size_t b8[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int jr = s0 + u < it.nsel ? it.row[s0 + u] : -1;
-      const bool ok = jr >= 0 && jr < p.nB;
-      b8[u] = hb + (ok ? jr : 0);
-      e8[u] = ok ? (int)p.st.seg_idx[b8[u] * p.C + rr] : 0xFF;
-    }
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      if (e8[u] != 0xFF) {
-        if (seen >= kSlots) {
-          const float4 y = ldg4(p.st.seg_vsum + (b8[u] * kBN + e8[u]) * kD + 4 * lane);
-          acc.x += y.x; acc.y += y.y; acc.z += y.z; acc.w += y.w;
-        }
-        ++seen;
-      }
-    }
-  }
-}
-
-// Builder: the compensation chunks of one item into scratch buffer `buf` (t: 0..127).  Warp w
-// builds chunks w, w+4, ...  For a chunk, lane l first looks up cluster rows 4l .. 4l+3 in every
-// selected block (one 32-bit load of the entry-index row and one 16-byte load of the histogram row
-// per block): the first kSlots entries of each row, in block order, and its selected count.  The
-// warp then builds the rows in groups of kStageRows: the fp32 totals S_c of the next group are
-// copied to shared memory with cp.async while the current group's entry sums are gathered with
-// coalesced loads (lanes over d) and subtracted; rows are scaled by 1 / n^U_c, rounded to bf16 and
-// written to the scratch chunk, whose log2 n^U_c row the lookup lanes write.
-__device__ __forceinline__ void build_item(const Params& p, const Item& it, int buf, int t, float* stage_all) {
-  const int w = t >> 5, lane = t & 31;
-  float* stage = stage_all + w * (2 * kStageRows * kD);
-  const size_t hb = (size_t)it.bh * p.nB;      // first block row of the head
-  const size_t hc = (size_t)it.bh * p.C;       // first cluster row of the head
-  for (int c = w; c < p.nchunk; c += 4) {
-    uint8_t* tile = scratch_chunk(p, buf, c);
-    const int rbase = c * kBN;
-    // (1) lookups: lane <-> rows r0 .. r0+3 (C is a multiple of 32: the four are valid together)
-    const int r0 = rbase + 4 * lane;
-    const bool rl = r0 < p.C;
-    int nm[4] = {0, 0, 0, 0};
-    int4 cs = make_int4(0, 0, 0, 0);
-    uint32_t mp[4][kSlots];
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-#pragma unroll
-      for (int k = 0; k < kSlots; ++k) mp[q][k] = 0;
-#pragma unroll 4
-    for (int s = 0; s < it.nsel; ++s) {
-      const int jr = it.row[s];
-      const bool ok = rl && jr >= 0 && jr < p.nB;
-      const size_t bj = hb + (ok ? jr : 0);
-      const size_t cell = bj * p.C + (rl ? r0 : 0);
-      const uint32_t e4 = ok ? __ldg(reinterpret_cast<const unsigned int*>(p.st.seg_idx + cell)) : 0xFFFFFFFFu;
-      const int4 h4 = ok ? __ldg(reinterpret_cast<const int4*>(p.st.blk_hist + cell)) : make_int4(0, 0, 0, 0);
-      cs.x += h4.x; cs.y += h4.y; cs.z += h4.z; cs.w += h4.w;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint32_t e = (e4 >> (8 * q)) & 0xFFu;
-        const bool hit = e != 0xFFu;
-        const uint32_t ptr = (uint32_t)(bj * kBN + e);
-#pragma unroll
-        for (int k = 0; k < kSlots; ++k) mp[q][k] = (hit && nm[q] == k) ? ptr : mp[q][k];
-        nm[q] += hit ? 1 : 0;
-      }
-    }
-    float inv4[4];
-    {
-      const int4 nt = rl ? __ldg(reinterpret_cast<const int4*>(p.st.n_tot + hc + r0)) : make_int4(0, 0, 0, 0);
-      const int nu[4] = {nt.x - cs.x, nt.y - cs.y, nt.z - cs.z, nt.w - cs.w};
-      float4 bt;
-      float* btp = &bt.x;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        inv4[q] = nu[q] > 0 ? 1.f / (float)nu[q] : 0.f;
-        btp[q] = nu[q] > 0 ? log2f((float)nu[q]) : -INFINITY;
-      }
-      reinterpret_cast<float4*>(tile + kTile)[lane] = bt;
-    }
-    // (2) rows in groups of kStageRows (= lanes 2G and 2G+1 of the lookups)
-    auto prefetch = [&](int G) {
-      const int rg = rbase + G * kStageRows;
-      if (rg < p.C) {
-        const float* src = p.st.S_tot + (hc + rg) * kD;
-        float* dst = stage + (G & 1) * kStageRows * kD;
-#pragma unroll
-        for (int i = 0; i < kStageRows * kD / 128; ++i) cp_async16(dst + (i * 32 + lane) * 4, src + (i * 32 + lane) * 4);
-      }
-      cp_async_commit();
-    };
-    constexpr int kGroups = kBN / kStageRows;
-    prefetch(0);
-    for (int G = 0; G < kGroups; ++G) {
-      if (G + 1 < kGroups) prefetch(G + 1); else cp_async_commit();
-      int nmr[kStageRows];
-      float invr[kStageRows];
-#pragma unroll
-      for (int i = 0; i < kStageRows; ++i) {
-        nmr[i] = __shfl_sync(0xffffffffu, nm[i & 3], 2 * G + (i >> 2));
-        invr[i] = __shfl_sync(0xffffffffu, inv4[i & 3], 2 * G + (i >> 2));
-      }
-      float4 acc[kStageRows];
-#pragma unroll
-      for (int i = 0; i < kStageRows; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-      // entry sums, kRound slots per row per round (a second round only when a row of the group
-      // has more than kRound entries); summed in block order
-#pragma unroll
-      for (int k0 = 0; k0 < kSlots; k0 += kRound) {
-        int need = 0;
-#pragma unroll
-        for (int i = 0; i < kStageRows; ++i) need |= nmr[i] > k0;
-        if (!need) break;                                    // warp-uniform
-        float4 xm[kStageRows][kRound];
-#pragma unroll
-        for (int i = 0; i < kStageRows; ++i)
-#pragma unroll
-          for (int k = 0; k < kRound; ++k) {
-            const uint32_t pk = __shfl_sync(0xffffffffu, mp[i & 3][k0 + k], 2 * G + (i >> 2));
-            xm[i][k] = nmr[i] > k0 + k ? ldg4(p.st.seg_vsum + (size_t)pk * kD + 4 * lane)
-                                       : make_float4(0.f, 0.f, 0.f, 0.f);
-          }
-#pragma unroll
-        for (int i = 0; i < kStageRows; ++i)
-#pragma unroll
-          for (int k = 0; k < kRound; ++k) {
-            acc[i].x += xm[i][k].x; acc[i].y += xm[i][k].y; acc[i].z += xm[i][k].z; acc[i].w += xm[i][k].w;
-          }
-      }
-      cp_async_wait<1>();
-      __syncwarp();
-      const float* sg = stage + (G & 1) * kStageRows * kD;
-#pragma unroll
-      for (int i = 0; i < kStageRows; ++i) {
-        const int rr = rbase + G * kStageRows + i;
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (rr < p.C) {
-          v = *reinterpret_cast<const float4*>(sg + i * kD + 4 * lane);
-          if (nmr[i] > kSlots) subtract_overflow(p, it, hb, rr, lane, acc[i]);
-          v.x -= acc[i].x; v.y -= acc[i].y; v.z -= acc[i].z; v.w -= acc[i].w;
-        }
-        const float iv = invr[i];
-        uint2 o;
-        o.x = pack_bf16x2(v.x * iv, v.y * iv);
-        o.y = pack_bf16x2(v.z * iv, v.w * iv);
-        *reinterpret_cast<uint2*>(tile + (size_t)(G * kStageRows + i) * (kD * 2) + lane * 8) = o;
-      }
-      __syncwarp();     // the staging buffer of this group is refilled two groups later
-    }
-  }
+__device__ __forceinline__ const uint8_t* comp_chunk(const Params& p, const Item& it, int c) {
+  return p.comp + ((size_t)(it.bh * p.nB + it.i) * p.nchunk + c) * kChunkBytes;
 }
 
 // Softmax helpers over 32 columns of S (raw bits in r): logits y = x * s*log2(e) + bias.
@@ -331,7 +160,7 @@ __device__ __forceinline__ void chunk_exp(const uint32_t (&r)[32], const float* 
 __global__ void __launch_bounds__(kThreads, 1)
 attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_c,
-                    const __grid_constant__ CUtensorMap tm_s, const Params p) {
+                    const __grid_constant__ CUtensorMap tm_p, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -339,8 +168,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   uint8_t* sK = sQ + kTile;                       // kKStages tiles
   uint8_t* sV = sK + kKStages * kTile;            // kVStages tiles
   float* sBias = reinterpret_cast<float*>(sV + kVStages * kTile);   // [kBStages][kBN]
-  float* sStage = sBias + kBStages * kBN;         // builder staging
-  Bars* bars = reinterpret_cast<Bars*>(sStage + kStageFloats);
+  Bars* bars = reinterpret_cast<Bars*>(sBias + kBStages * kBN);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -363,8 +191,6 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars->s_full[b], 1);
       mbar_init(&bars->p_ready[b], 128);
-      mbar_init(&bars->bready[b], 1);
-      mbar_init(&bars->sfree[b], 128);
     }
     mbar_init(&bars->o_done, 1);
     mbar_init(&bars->o_free, 128);
@@ -383,7 +209,6 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   volatile int* abort = &bars->abort;
   int* status = p.status;
 
-  if (warp >= 8) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegIssue));
   if (warp == kWarpProducer) {
     // ------------------------------------------------------------------ producer
     // lane 0: query tiles, key / centroid tiles and the softmax bias rows; lane 1: value tiles.
@@ -393,7 +218,6 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       tma_prefetch(&tm_q);
       tma_prefetch(&tm_k);
       tma_prefetch(&tm_c);
-      tma_prefetch(&tm_s);
       uint32_t g = 0;
       int n = 0, nq = 0;                 // items walked, query tiles loaded
       for (int k = blockIdx.x; k < p.n_items && !*abort; k += gridDim.x, ++n) {
@@ -406,7 +230,6 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         bool ok = true;
         for (int s = 0; s < it.T; ++s, ++g) {
           const int ks = g % kKStages, bs = g % kBStages;
-          const int buf = n & 1;
           if (!mbar_wait(&bars->k_empty[ks], ((g / kKStages) & 1) ^ 1, abort, status)) { ok = false; break; }
           uint8_t* dk = sK + ks * kTile;
           if (s < it.nsel) {
@@ -429,14 +252,12 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             mbar_arrive(&bars->b_full[bs]);
           } else {
             const int c = s - it.nsel;
-            // the builder has finished this item's scratch chunks (once per item, in order)
-            if (c == 0 && !mbar_wait(&bars->bready[buf], (n >> 1) & 1, abort, status)) { ok = false; break; }
             mbar_expect_tx(&bars->k_full[ks], kTile);
             tma_load_3d(dk, &tm_c, &bars->k_full[ks], 0, c * kBN, it.bh);
             tma_load_3d(dk + kPanel, &tm_c, &bars->k_full[ks], 64, c * kBN, it.bh);
             if (!mbar_wait(&bars->b_empty[bs], ((g / kBStages) & 1) ^ 1, abort, status)) { ok = false; break; }
             mbar_expect_tx(&bars->b_full[bs], kBN * 4);
-            bulk_load(sBias + bs * kBN, scratch_chunk(p, buf, c) + kTile, kBN * 4, &bars->b_full[bs]);
+            bulk_load(sBias + bs * kBN, comp_chunk(p, it, c) + kTile, kBN * 4, &bars->b_full[bs]);
           }
         }
         if (!ok) break;
@@ -450,6 +271,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         mbar_wait_drain(&bars->b_full[gd % kBStages], (gd / kBStages) & 1);
     } else if (lane == 1) {
       tma_prefetch(&tm_v);
+      tma_prefetch(&tm_p);
       uint32_t g = 0;
       int n = 0;
       for (int k = blockIdx.x; k < p.n_items && !*abort; k += gridDim.x, ++n) {
@@ -457,7 +279,6 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         bool ok = true;
         for (int s = 0; s < it.T; ++s, ++g) {
           const int vs = g % kVStages;
-          const int buf = n & 1;
           if (!mbar_wait(&bars->v_empty[vs], ((g / kVStages) & 1) ^ 1, abort, status)) { ok = false; break; }
           uint8_t* dv = sV + vs * kTile;
           if (s < it.nsel) {
@@ -467,12 +288,10 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             tma_load_3d(dv, &tm_v, &bars->v_full[vs], 0, j * kBN, it.bh);
             tma_load_3d(dv + kPanel, &tm_v, &bars->v_full[vs], 64, j * kBN, it.bh);
           } else {
-            const int c = s - it.nsel;
-            if (c == 0 && !mbar_wait(&bars->bready[buf], (n >> 1) & 1, abort, status)) { ok = false; break; }
-            const int z = ((int)blockIdx.x * 2 + buf) * p.nchunk + c;
+            const int z = (it.bh * p.nB + it.i) * p.nchunk + (s - it.nsel);
             mbar_expect_tx(&bars->v_full[vs], kTile);
-            tma_load_3d(dv, &tm_s, &bars->v_full[vs], 0, 0, z);
-            tma_load_3d(dv + kPanel, &tm_s, &bars->v_full[vs], 64, 0, z);
+            tma_load_3d(dv, &tm_p, &bars->v_full[vs], 0, 0, z);
+            tma_load_3d(dv + kPanel, &tm_p, &bars->v_full[vs], 64, 0, z);
           }
         }
         if (!ok) break;
@@ -538,30 +357,8 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       umma_commit(&bars->drain);
       mbar_wait_drain(&bars->drain, 0);
     }
-  } else if (warp >= 8) {
-    // warps 10-11: idle
-  } else if (warp >= 4) {
-    // ------------------------------------------------------------------ builder
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegBuilder));
-    const int t = tid - 128;
-    int n = 0;
-    // (no abort test in the loop condition: the builders leave together, on bld_ok)
-    for (int k = blockIdx.x; k < p.n_items; k += gridDim.x, ++n) {
-      const Item it = item_at(p, k);
-      const int buf = n & 1;
-      // scratch buffer `buf` was last read for item n-2: wait until that item has finished.
-      // One thread waits; the decision reaches every builder warp through a named barrier.
-      if (t == 0) bars->bld_ok[n & 1] = n < 2 || mbar_wait(&bars->sfree[buf], ((n >> 1) - 1) & 1, abort, status);
-      asm volatile("bar.sync 2, 128;" ::: "memory");
-      if (!bars->bld_ok[n & 1]) break;
-      build_item(p, it, buf, t, sStage);
-      fence_async_global();
-      asm volatile("bar.sync 2, 128;" ::: "memory");
-      if (t == 0) mbar_arrive(&bars->bready[buf]);
-    }
   } else {
     // ------------------------------------------------------------------ softmax (warps 0-3)
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegSoftmax));
     const int r = tid;                                        // query row = TMEM lane
     const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
     uint32_t g = 0;
@@ -682,7 +479,6 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       if (live && p.lse) p.lse[(size_t)it.bh * p.N + it.q0 + r] = (m + __log2f(l)) * 0.69314718055994531f;
       tc_fence_before();
       mbar_arrive(&bars->o_free);
-      mbar_arrive(&bars->sfree[n & 1]);
     }
   }
 
@@ -700,19 +496,19 @@ bool attention_tc_supported(const Dims& g) { return g.bf16 && g.d == kD && g.blo
 
 size_t attention_tc_scratch_bytes(const Dims& g) {
   if (!attention_tc_supported(g)) return 0;
-  return (size_t)kMaxCtas * 2 * ((g.C + kBN - 1) / kBN) * kChunkBytes;
+  return (size_t)g.B * g.H * g.nB * ((g.C + kBN - 1) / kBN) * kChunkBytes;
 }
 
 cudaError_t launch_attention_tc(const Dims& g, const void* Q, const void* K, const void* V,
                                 const int32_t* kv_idx, const int32_t* kv_cnt, int max_sel,
                                 const int32_t* schedule, const void* cent, const StatsPtrs& st, float scale,
-                                void* O, float* lse, int* status, void* scratch, cudaStream_t s) {
-  CUtensorMap tq, tk, tv, tc, ts;
+                                void* O, float* lse, int* status, void* comp, cudaStream_t s) {
+  CUtensorMap tq, tk, tv, tc, tp;
   const unsigned long long BH = (unsigned long long)g.B * g.H;
   const int nchunk = (g.C + kBN - 1) / kBN;
   if (!make_tmap_bf16_3d(&tq, Q, kD, g.N, BH, 64, kBM) || !make_tmap_bf16_3d(&tk, K, kD, g.N, BH, 64, kBN) ||
       !make_tmap_bf16_3d(&tv, V, kD, g.N, BH, 64, kBN) || !make_tmap_bf16_3d(&tc, cent, kD, g.C, BH, 64, kBN) ||
-      !make_tmap_bf16_tiles(&ts, scratch, kD, kBN, (uint64_t)kMaxCtas * 2 * nchunk, kChunkBytes, kBN))
+      !make_tmap_bf16_tiles(&tp, comp, kD, kBN, BH * g.nB * nchunk, kChunkBytes, kBN))
     return cudaErrorInvalidValue;
   Params p;
   p.kv_idx = kv_idx;
@@ -723,7 +519,7 @@ cudaError_t launch_attention_tc(const Dims& g, const void* Q, const void* K, con
   p.O = (__nv_bfloat16*)O;
   p.lse = lse;
   p.status = status;
-  p.scratch = static_cast<uint8_t*>(scratch);
+  p.comp = static_cast<const uint8_t*>(comp);
   p.N = g.N;
   p.C = g.C;
   p.nB = g.nB;
@@ -736,8 +532,8 @@ cudaError_t launch_attention_tc(const Dims& g, const void* Q, const void* K, con
   cudaError_t e = cudaFuncSetAttribute(attention_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kSmemBytes);
   if (e != cudaSuccess) return e;
-  const int grid = min(min(sms, kMaxCtas), p.n_items);
-  attention_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, tc, ts, p);
+  const int grid = min(sms, p.n_items);
+  attention_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, tc, tp, p);
   return cudaGetLastError();
 }
 

@@ -155,9 +155,13 @@ da_status da_attention(const da_dims* dims, const void* Q, const void* K, const 
     sched = own;
   }
   if (e == cudaSuccess) {
-    if (attention_tc_supported(g))
-      e = launch_attention_tc(g, Q, K, V, mask->kv_idx, mask->kv_cnt, mask->max_sel, sched, centroids, sp, scale,
-                              O, lse, status, static_cast<char*>(ws) + L.comp, s);
+    if (attention_tc_supported(g)) {
+      void* comp = static_cast<char*>(ws) + L.comp;
+      e = launch_comp_build(g, mask->kv_idx, mask->kv_cnt, mask->max_sel, sp, comp, s);
+      if (e == cudaSuccess)
+        e = launch_attention_tc(g, Q, K, V, mask->kv_idx, mask->kv_cnt, mask->max_sel, sched, centroids, sp,
+                                scale, O, lse, status, comp, s);
+    }
     else
       e = (g.bf16 ? launch_attention_simt_bf16 : launch_attention_simt_f32)(
           g, Q, K, V, mask->kv_idx, mask->kv_cnt, mask->max_sel, sched, centroids, sp, scale, O, lse, status, s);

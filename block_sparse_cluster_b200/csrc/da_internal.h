@@ -45,11 +45,15 @@ cudaError_t launch_reassign_tc(const Dims& g, const void* K, const void* V, cons
 
 // attention_tc.cu
 bool attention_tc_supported(const Dims& g);
-size_t attention_tc_scratch_bytes(const Dims& g);   // per-CTA compensation scratch, all CTAs
+size_t attention_tc_scratch_bytes(const Dims& g);   // compensation chunks of every item
 cudaError_t launch_attention_tc(const Dims& g, const void* Q, const void* K, const void* V,
                                 const int32_t* kv_idx, const int32_t* kv_cnt, int max_sel,
                                 const int32_t* schedule, const void* cent, const StatsPtrs& st, float scale,
-                                void* O, float* lse, int* status, void* scratch, cudaStream_t s);
+                                void* O, float* lse, int* status, void* comp, cudaStream_t s);
+
+// comp_build.cu
+cudaError_t launch_comp_build(const Dims& g, const int32_t* kv_idx, const int32_t* kv_cnt, int max_sel,
+                              const StatsPtrs& st, void* out, cudaStream_t s);
 
 // simt_f32.cu / simt_bf16.cu
 #define DA_SIMT_DECL(SUFFIX)                                                                                 \

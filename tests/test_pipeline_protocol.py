@@ -1,7 +1,7 @@
 """Host-side model of the fused attention kernel's synchronisation protocol.
 
-The kernel's roles (TMA producer, MMA issuer, compensation builder, softmax
-warpgroup) talk only through mbarriers.  An mbarrier wait names a phase by its
+The kernel's roles (TMA producer lanes, MMA issuer, softmax warpgroup) talk
+only through mbarriers.  An mbarrier wait names a phase by its
 parity alone, so a wait is only meaningful while the barrier is within one
 phase of the awaited one; a role that falls two phases behind (or waits one
 phase early) reads the wrong phase.  This model replays the roles' exact
@@ -14,21 +14,22 @@ interleavings, and checks that
 * no phase receives more arrivals than its count, and the transaction count
   never goes negative;
 * no shared-memory slot, TMEM buffer or the query tile is overwritten while an
-  operation that reads it is still in flight;
+  operation that reads it is still in flight, and every consumer reads the
+  tile of its own step;
 * every role finishes (no deadlock).
 
 It mirrors the step structure of attention_tc.cu: per work item, one step per
-selected block followed by one step per 128-cluster chunk, a 3-stage K/V ring,
-S double-buffered in TMEM, P in the S buffer, O accumulated across the item,
-and the compensation builder one item ahead, writing a double-buffered scratch
-that the producer copies into the ring.
+selected block followed by one step per 128-cluster chunk, 3-stage key, value
+and bias-row rings, S double-buffered in TMEM, P in the S buffer and O
+accumulated across the item.  The compensation chunks are written by an earlier
+kernel, so they are plain inputs here.
 """
 import random
 
 import pytest
 
 KSTAGES = 3   # key / centroid tiles, freed when S is computed
-VSTAGES = 2   # value / vbar^U tiles, freed after P V
+VSTAGES = 3   # value / vbar^U tiles, freed after P V
 BSTAGES = 3   # softmax bias rows, freed after the softmax has read them
 
 
@@ -66,12 +67,12 @@ class Barrier:
 
 
 class Machine:
-    def __init__(self, items, nchunk, rng, old_builder=False, skip_sfree=False):
+    def __init__(self, items, nchunk, rng, lazy_v_wait=False, skip_b_empty=False):
         self.items = items                     # list of nsel per item of one CTA
         self.nchunk = nchunk
         self.rng = rng
-        self.old_builder = old_builder
-        self.skip_sfree = skip_sfree
+        self.lazy_v_wait = lazy_v_wait         # planted: value lane waits for a free slot only at chunk steps
+        self.skip_b_empty = skip_b_empty       # planted: bias rows loaded without waiting for a free slot
         B = Barrier
         self.q_full, self.q_empty = B("q_full", 1), B("q_empty", 1)
         self.k_full = [B(f"k_full{i}", 1) for i in range(KSTAGES)]
@@ -80,9 +81,7 @@ class Machine:
         self.v_empty = [B(f"v_empty{i}", 1) for i in range(VSTAGES)]
         self.b_full = [B(f"b_full{i}", 1) for i in range(BSTAGES)]
         self.b_empty = [B(f"b_empty{i}", 1) for i in range(BSTAGES)]
-        self.bready = [B(f"bready{i}", 1) for i in range(2)]     # scratch buffer built
-        self.sfree = [B(f"sfree{i}", 1) for i in range(2)]       # scratch buffer released
-        self.scratch_version = [None, None]
+        self.version = {}                      # buffer -> step whose tile it holds
         self.s_full = [B(f"s_full{i}", 1) for i in range(2)]
         self.p_ready = [B(f"p_ready{i}", 1) for i in range(2)]
         self.o_done, self.o_free = B("o_done", 1), B("o_free", 1)
@@ -133,12 +132,16 @@ class Machine:
             progressed = True
         return progressed
 
-    def tma_load(self, bar, res, srcs=()):
-        """A copy into buffer `res` (busy until it lands) that reads the buffers `srcs`."""
+    def tma_load(self, bar, res, step, srcs=()):
+        """A copy of step `step`'s tile into buffer `res` (busy until it lands) that reads `srcs`."""
         self._write(res, "TMA", unit="tma")
         for r in [res, *srcs]:
             self._start_read(r, "tma")
+        self.version[res] = step
         self.tma.append((bar, res, list(srcs)))
+
+    def holds(self, res, step):
+        assert self.version.get(res) == step, f"{res} holds step {self.version.get(res)}, read at step {step}"
 
     # ---- roles (generators yield a predicate to wait on)
     def producer(self):
@@ -148,24 +151,18 @@ class Machine:
             T = nsel + self.nchunk
             yield lambda: self.q_empty.test(n - 1)
             self.q_full.expect_tx(1)
-            self.tma_load(self.q_full, "Q")
+            self.tma_load(self.q_full, "Q", n)
             for s in range(T):
                 ks, bs = g % KSTAGES, g % BSTAGES
-                comp = s >= nsel
                 yield lambda: self.k_empty[ks].test(g // KSTAGES - 1)
-                if comp and s == nsel and not self.old_builder:
-                    buf = n & 1
-                    yield lambda: self.bready[buf].test(n >> 1)
                 self.k_full[ks].expect_tx(1)
-                self.tma_load(self.k_full[ks], f"K{ks}")
-                yield lambda: self.b_empty[bs].test(g // BSTAGES - 1)
-                if comp and not self.old_builder:
-                    assert self.scratch_version[n & 1] == n, "scratch chunk read before it was built"
+                self.tma_load(self.k_full[ks], f"K{ks}", g)
+                if not self.skip_b_empty:
+                    yield lambda: self.b_empty[bs].test(g // BSTAGES - 1)
                     self.b_full[bs].expect_tx(1)
-                    self.tma_load(self.b_full[bs], f"BIAS{bs}", srcs=[f"SCR{n & 1}"])
                 else:
-                    self._write(f"BIAS{bs}", "producer")
-                    self.b_full[bs].arrive()
+                    self.b_full[bs].tx += 1          # the planted variant: no free-slot wait
+                self.tma_load(self.b_full[bs], f"BIAS{bs}", g)
                 g += 1
 
     def producer_v(self):
@@ -175,16 +172,10 @@ class Machine:
             T = nsel + self.nchunk
             for s in range(T):
                 vs = g % VSTAGES
-                comp = s >= nsel
-                yield lambda: self.v_empty[vs].test(g // VSTAGES - 1)
-                if comp and not self.old_builder:
-                    if s == nsel:
-                        buf = n & 1
-                        yield lambda: self.bready[buf].test(n >> 1)
-                    assert self.scratch_version[n & 1] == n, "scratch chunk read before it was built"
-                if not (comp and self.old_builder):      # the old builder filled the value slot itself
-                    self.v_full[vs].expect_tx(1)
-                    self.tma_load(self.v_full[vs], f"V{vs}", srcs=[f"SCR{n & 1}"] if comp else [])
+                if not self.lazy_v_wait or s >= nsel:
+                    yield lambda: self.v_empty[vs].test(g // VSTAGES - 1)
+                self.v_full[vs].expect_tx(1)
+                self.tma_load(self.v_full[vs], f"V{vs}", g)
                 g += 1
 
     def mma(self):
@@ -193,6 +184,8 @@ class Machine:
             T = nsel + self.nchunk
             yield lambda: self.q_full.test(n)
             yield lambda: self.k_full[g % KSTAGES].test(g // KSTAGES)
+            self.holds("Q", n)
+            self.holds(f"K{g % KSTAGES}", g)
             self.tc_issue_mma(["Q", f"K{g % KSTAGES}"], [f"S{g & 1}"])
             self.tc_commit(self.s_full[g & 1])
             self.tc_commit(self.k_empty[g % KSTAGES])
@@ -200,6 +193,7 @@ class Machine:
                 if s + 1 < T:
                     gn = g + 1
                     yield lambda: self.k_full[gn % KSTAGES].test(gn // KSTAGES)
+                    self.holds(f"K{gn % KSTAGES}", gn)
                     self.tc_issue_mma(["Q", f"K{gn % KSTAGES}"], [f"S{gn & 1}"])
                     self.tc_commit(self.s_full[gn & 1])
                     self.tc_commit(self.k_empty[gn % KSTAGES])
@@ -209,34 +203,10 @@ class Machine:
                 yield lambda: self.v_full[g % VSTAGES].test(g // VSTAGES)
                 if s == 0:
                     yield lambda: self.o_free.test(n - 1)
+                self.holds(f"V{g % VSTAGES}", g)
                 self.tc_issue_mma([f"S{g & 1}", f"V{g % VSTAGES}"], ["O"])
                 self.tc_commit(self.v_empty[g % VSTAGES])
                 self.tc_commit(self.o_done)
-                g += 1
-
-    def builder(self):
-        if self.old_builder:
-            yield from self.old_builder_role()
-            return
-        for n, nsel in enumerate(self.items):
-            buf = n & 1
-            if n >= 2 and not self.skip_sfree:
-                yield lambda: self.sfree[buf].test((n >> 1) - 1)
-            self._write(f"SCR{buf}", "builder", unit="builder")
-            self.scratch_version[buf] = n
-            self.bready[buf].arrive()
-
-    def old_builder_role(self):
-        """The first design: the builder wrote the ring's value slot itself, waiting on the ring's
-        empty barrier only at its own (compensation) steps."""
-        g = 0
-        for n, nsel in enumerate(self.items):
-            g += nsel
-            for c in range(self.nchunk):
-                vs, u = g % VSTAGES, g // VSTAGES
-                yield lambda: self.v_empty[vs].test(u - 1)
-                self._write(f"V{vs}", "builder")
-                self.v_full[vs].arrive()
                 g += 1
 
     def softmax(self):
@@ -249,6 +219,7 @@ class Machine:
                 yield lambda: self.s_full[b].test(g >> 1)
                 assert not self.readers.get(f"S{b}"), "S read before its MMA completed"
                 assert not self.readers.get(f"BIAS{bs}"), "bias row read before it landed"
+                self.holds(f"BIAS{bs}", g)
                 self._write(f"S{b}", "softmax (P)")
                 self.b_empty[bs].arrive()
                 if s > 0:
@@ -259,11 +230,9 @@ class Machine:
             yield lambda: self.o_done.test(g - 1)
             self._write("O", "epilogue")
             self.o_free.arrive()
-            if not self.old_builder:
-                self.sfree[n & 1].arrive()
 
     def run(self, max_iters=200000):
-        roles = [self.producer(), self.producer_v(), self.mma(), self.builder(), self.softmax()]
+        roles = [self.producer(), self.producer_v(), self.mma(), self.softmax()]
         waits = [None] * len(roles)
         done = [False] * len(roles)
         for _ in range(max_iters):
@@ -303,23 +272,21 @@ def test_protocol_random_interleavings(items, nchunk):
         Machine(items, nchunk, random.Random(seed)).run()
 
 
-def test_model_catches_a_builder_that_skips_ring_phases():
-    """The builder waiting on the ring's empty barrier only at its own steps falls behind
-    the ring by several phases when many exact steps precede a chunk."""
+def _caught(items, nchunk, **planted):
     caught = 0
     for seed in range(40):
         try:
-            Machine([37], 2, random.Random(seed), old_builder=True).run()
+            Machine(items, nchunk, random.Random(seed), **planted).run()
         except AssertionError:
             caught += 1
-    assert caught > 0
+    return caught
 
 
-def test_model_catches_a_builder_that_does_not_wait_for_its_buffer():
-    caught = 0
-    for seed in range(40):
-        try:
-            Machine([3, 3, 3, 3, 3], 2, random.Random(seed), skip_sfree=True).run()
-        except AssertionError:
-            caught += 1
-    assert caught > 0
+def test_model_catches_a_lane_that_skips_ring_phases():
+    """A value lane waiting for a free slot only at its chunk steps runs ahead of the ring by
+    several phases when many exact steps precede a chunk."""
+    assert _caught([37], 2, lazy_v_wait=True) > 0
+
+
+def test_model_catches_bias_rows_loaded_without_a_free_slot():
+    assert _caught([3, 3, 3, 3, 3], 2, skip_b_empty=True) > 0
