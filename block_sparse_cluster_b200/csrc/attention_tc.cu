@@ -16,15 +16,21 @@
 // The compensation chunks (vbar^U rows in bf16 and log2 n^U per cluster) of every item are
 // written beforehand by comp_build.cu; here they are loaded like value blocks.
 //
-// Roles (192 threads):
-//   warps 0-3  softmax: thread t owns query row t = TMEM lane t; online softmax with lazy
-//              rescaling (the running max only moves when it grows by more than 2^8), P written
-//              back to TMEM as bf16, final normalisation and store of O;
-//   warp 4     producer: lane 0 loads Q, key tiles / centroid chunks (3-stage ring) and the
-//              softmax bias rows (3-stage ring); lane 1 loads value tiles / compensation chunks
-//              (3-stage ring);
-//   warp 5     MMA: allocates TMEM, issues tcgen05.mma S(g+1) = Q K^T ahead of O += P(g) V(g).
-// TMEM columns: S double buffer [0,128) and [128,256), O [256,384).
+// Roles (384 threads):
+//   warps 0-3, 4-7  two softmax warpgroups X = 0, 1; warpgroup X takes the steps g with g & 1 = X
+//              of every item, so the two overlap each other and the tensor core.  Thread t of a
+//              warpgroup owns query row t = TMEM lane t: online softmax with lazy rescaling (the
+//              running max only moves when it grows by more than 2^8) of its own accumulator O_X,
+//              P written back to TMEM as bf16.  At the end of the item the two exchange their
+//              (max, sum) per row and each normalises and stores half of the columns of
+//              O = O_0 2^(m_0 - m) + O_1 2^(m_1 - m);
+//   warp 8     producer: loads Q, key tiles / centroid chunks (3-stage ring) and the softmax bias
+//              rows (4-stage ring, so a slot always serves the same warpgroup);
+//   warp 9     MMA: allocates TMEM, issues tcgen05.mma S(g+1) = Q K^T ahead of O_X += P(g) V(g);
+//   warp 10    producer of value tiles / compensation chunks (2-stage ring); a warp of its own,
+//              since divergent lanes of one warp waiting on different barriers hold each other up;
+//   warp 11    idle (it completes the third warpgroup, whose registers go to the softmax).
+// TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,384), O_1 [384,512).
 //
 // Every mbarrier is waited at every phase, in order, by each role that waits on it (a parity
 // wait is only meaningful within one phase); the host-side protocol model in the tests replays
@@ -41,14 +47,20 @@ constexpr int kD = 128;
 constexpr int kBM = 128;                 // query rows per item
 constexpr int kBN = 128;                 // keys per block / clusters per chunk
 constexpr int kKStages = 3;             // key / centroid tiles (freed as soon as S is computed)
-constexpr int kVStages = 3;             // value / vbar^U tiles (freed after P V)
-constexpr int kBStages = 3;             // bias rows of the softmax (freed after the softmax pass)
+constexpr int kVStages = 2;             // value / vbar^U tiles (freed after P V)
+constexpr int kBStages = 4;             // bias rows of the softmax (even: a slot serves one warpgroup)
 constexpr int kTile = kBN * kD * 2;      // 32 KB bf16 tile
 constexpr int kPanel = kBN * 128;        // one 64-column panel (128 rows x 128 B)
 constexpr float kRescaleLog2 = 8.0f;     // lazy rescale threshold (factor 256)
-constexpr int kThreads = 192;
-constexpr int kWarpProducer = 4;
-constexpr int kWarpMMA = 5;
+constexpr int kThreads = 384;           // three warpgroups; warp 11 idle
+constexpr int kWarpProducer = 8;
+constexpr int kWarpMMA = 9;
+constexpr int kWarpProducerV = 10;
+// Register split (setmaxnreg): the launch holds 384 x 168 registers; the softmax warpgroups grow,
+// the producer / MMA warpgroup shrinks.
+constexpr int kRegSoftmax = 216, kRegIssue = 72;
+static_assert(128 * (2 * kRegSoftmax + kRegIssue) <= kThreads * 168, "register split above the launch");
+static_assert(kBStages % 2 == 0, "a bias slot must always serve the same softmax warpgroup");
 constexpr int kChunkBytes = kTile + kBN * 4;   // compensation chunk: vbar^U rows, then log2 n^U
 
 struct __align__(8) Bars {
@@ -56,9 +68,14 @@ struct __align__(8) Bars {
   uint64_t k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
   uint64_t b_full[kBStages], b_empty[kBStages];
   uint64_t s_full[2], p_ready[2];
-  uint64_t o_done, o_free, drain;
+  uint64_t o_done[2], o_free, drain;
+  // (max, sum) published: [item parity][warpgroup].  One barrier per item parity: a warpgroup
+  // without steps in an item could otherwise complete a barrier twice before the other
+  // warpgroup's parity wait on it runs.
+  uint64_t xch_full[2][2];
   uint32_t tmem_base;
   int abort;
+  float2 xch[2][2][kBM];                 // [item parity][warpgroup][row] = (max, sum)
 };
 
 constexpr size_t kSmemBytes = 1024 + kTile /*Q*/ + (kKStages + kVStages) * kTile /*K,V*/ +
@@ -84,8 +101,6 @@ __device__ __forceinline__ float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
-
-__device__ __forceinline__ float4 ldg4(const float* p) { return __ldg(reinterpret_cast<const float4*>(p)); }
 
 // Item geometry shared by every role.
 struct Item {
@@ -191,9 +206,11 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars->s_full[b], 1);
       mbar_init(&bars->p_ready[b], 128);
+      mbar_init(&bars->o_done[b], 1);
+      mbar_init(&bars->xch_full[b][0], 128);
+      mbar_init(&bars->xch_full[b][1], 128);
     }
-    mbar_init(&bars->o_done, 1);
-    mbar_init(&bars->o_free, 128);
+    mbar_init(&bars->o_free, 256);
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
     fence_mbar_init();
@@ -209,11 +226,12 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   volatile int* abort = &bars->abort;
   int* status = p.status;
 
+  // the whole third warpgroup gives registers up at one instruction (setmaxnreg is warpgroup-wide)
+  if (warp >= 8) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegIssue));
+
   if (warp == kWarpProducer) {
-    // ------------------------------------------------------------------ producer
-    // lane 0: query tiles, key / centroid tiles and the softmax bias rows; lane 1: value tiles.
-    // The two streams wait on separate barriers, so a value slot still in use never holds back
-    // the next key tile.
+    // ------------------------------------------------------------------ producer (keys)
+    // query tiles, key / centroid tiles and the softmax bias rows
     if (lane == 0) {
       tma_prefetch(&tm_q);
       tma_prefetch(&tm_k);
@@ -269,7 +287,10 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         mbar_wait_drain(&bars->k_full[gd % kKStages], (gd / kKStages) & 1);
       for (uint32_t gd = g >= kBStages ? g - kBStages : 0; gd < g; ++gd)
         mbar_wait_drain(&bars->b_full[gd % kBStages], (gd / kBStages) & 1);
-    } else if (lane == 1) {
+    }
+  } else if (warp == kWarpProducerV) {
+    // ------------------------------------------------------------------ producer (values)
+    if (lane == 0) {
       tma_prefetch(&tm_v);
       tma_prefetch(&tm_p);
       uint32_t g = 0;
@@ -344,43 +365,49 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           tc_fence_after();
           const uint32_t vb = smem_u32(sV + vs * kTile);
           const uint32_t pt = tmem + (g & 1) * kBN;       // P: bf16 pairs in the S buffer's first 64 columns
+          const uint32_t ot = tmem + (2 + (g & 1)) * kBN;  // O_X of the step's warpgroup
 #pragma unroll
           for (int ks = 0; ks < kBN / 16; ++ks) {
-            // V rows (keys) 16*ks .. 16*ks+15: two 8-row groups of 1024 B
-            umma_ts(tmem + 2 * kBN, pt + ks * 8, sdesc_sw128(vb + ks * 2048, kPanel, 1024), idesc_pv,
-                    (s > 0 || ks > 0) ? 1u : 0u);
+            // V rows (keys) 16*ks .. 16*ks+15: two 8-row groups of 1024 B; the first product of each
+            // accumulator in the item (steps 0 and 1) overwrites it
+            umma_ts(ot, pt + ks * 8, sdesc_sw128(vb + ks * 2048, kPanel, 1024), idesc_pv,
+                    (s > 1 || ks > 0) ? 1u : 0u);
           }
           umma_commit(&bars->v_empty[vs]);
-          umma_commit(&bars->o_done);
+          umma_commit(&bars->o_done[g & 1]);
         }
       }
       umma_commit(&bars->drain);
       mbar_wait_drain(&bars->drain, 0);
     }
-  } else {
-    // ------------------------------------------------------------------ softmax (warps 0-3)
-    const int r = tid;                                        // query row = TMEM lane
-    const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
-    uint32_t g = 0;
+  } else if (warp < 8) {
+    // ------------------------------------------------------------------ softmax (warps 0-7)
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegSoftmax));
+    const int X = warp >> 2;                                  // warpgroup: steps g with g & 1 == X
+    const int r = tid & 127;                                  // query row = TMEM lane
+    const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    const uint32_t o_own = lane_addr + (2 + X) * kBN;
+    uint32_t g0 = 0;                                          // first step of the item
+    uint32_t u = 0;                                           // products into O_X issued so far
     int n = 0;
     // (no abort test in the loop condition: a warp leaves as a whole, on its __all_sync'd waits)
     for (int k = blockIdx.x; k < p.n_items; k += gridDim.x, ++n) {
       const Item it = item_at(p, k);
       float m = -INFINITY, l = 0.f;
-      bool ok = true;
-      for (int s = 0; s < it.T; ++s, ++g) {
-        const int b = g & 1;
-        // every phase of b_full and s_full is waited, in order (b_full: the step's bias row)
+      bool ok = true, first = true;
+      for (int s = (int)((X - g0) & 1u); s < it.T; s += 2) {
+        const uint32_t g = g0 + s;
+        // every phase of this warpgroup's b_full slots and of s_full[X] is waited, in order
         const int bs = g % kBStages;
         bool w_ok = mbar_wait(&bars->b_full[bs], (g / kBStages) & 1, abort, status);
-        w_ok = w_ok && mbar_wait(&bars->s_full[b], (g >> 1) & 1, abort, status);
+        w_ok = w_ok && mbar_wait(&bars->s_full[X], (g >> 1) & 1, abort, status);
         if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
         tc_fence_after();
         // Two passes over the S row in TMEM, 32 columns at a time with the next load in flight: the
         // row max, then p = 2^(x - m), the row sum and the bf16 P written back over S.  Column c's
         // logit is x_c * s*log2(e) + bias_c, the bias row in shared memory: log2 n^U_c on a
         // compensation step, 0 on a key block (-inf past the end of a short last block).
-        const uint32_t sbase = lane_addr + b * kBN;
+        const uint32_t sbase = lane_addr + X * kBN;
         const float* bt = sBias + bs * kBN;
         const uint64_t sl2x2 = f2_pack(p.scale_log2, p.scale_log2);
         float mx = -INFINITY;
@@ -399,7 +426,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
         // lazy rescaling: the running max moves only when it grows by more than 2^8
         const bool grow = mx > m + kRescaleLog2 || (m == -INFINITY && mx > -INFINITY);
-        const bool need_o = grow && s > 0 && m > -INFINITY;
+        const bool need_o = grow && !first && m > -INFINITY;
         const float m_new = grow ? mx : m;
         const float mu = (m_new == -INFINITY) ? 0.f : m_new;
         uint64_t rsum = 0;
@@ -424,10 +451,11 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         float rs_lo, rs_hi;
         f2_unpack(rsum, rs_lo, rs_hi);
         const float rs = rs_lo + rs_hi;
-        if (s > 0) {
-          // PV(g-1) has landed in O: every phase of o_done is waited, in order; a row whose max
-          // moved rescales its O (warp-uniform, as tcgen05.ld/st are)
-          const bool d_ok = mbar_wait(&bars->o_done, (g - 1) & 1, abort, status);
+        if (!first) {
+          // this warpgroup's previous product has landed in O_X: every phase of o_done[X] is
+          // waited, in order; a row whose max moved rescales its O_X (warp-uniform, as
+          // tcgen05.ld/st are)
+          const bool d_ok = mbar_wait(&bars->o_done[X], (u - 1) & 1, abort, status);
           if (!__all_sync(0xffffffffu, d_ok)) { ok = false; break; }
           tc_fence_after();
           if (__any_sync(0xffffffffu, need_o)) {
@@ -435,50 +463,72 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 #pragma unroll 1
             for (int q = 0; q < 4; ++q) {
               uint32_t rr[32];
-              tmem_ld32(lane_addr + 2 * kBN + q * 32, rr);
+              tmem_ld32(o_own + q * 32, rr);
               tmem_wait_ld();
 #pragma unroll
               for (int v = 0; v < 32; ++v) rr[v] = __float_as_uint(__uint_as_float(rr[v]) * alpha);
-              tmem_st32(lane_addr + 2 * kBN + q * 32, rr);
+              tmem_st32(o_own + q * 32, rr);
             }
             if (need_o) l *= alpha;
           }
         }
         m = m_new;
         l += rs;
+        first = false;
+        ++u;
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&bars->p_ready[b]);
+        mbar_arrive(&bars->p_ready[X]);
       }
       if (!ok) break;
-      // epilogue: O / l once the item's last PV has landed
-      const uint32_t glast = g - 1;
-      const bool e_ok = mbar_wait(&bars->o_done, glast & 1, abort, status);
+      // epilogue: once this warpgroup's last product has landed, exchange (max, sum) per row with
+      // the other warpgroup; warpgroup X normalises and stores columns [64X, 64X + 64) of
+      // O = (O_0 2^(m_0 - M) + O_1 2^(m_1 - M)) / (l_0 2^(m_0 - M) + l_1 2^(m_1 - M)).
+      // A warpgroup without a step in the item (a one-step item) has an unwritten O_X: skipped.
+      const bool had0 = it.T >= 2 || (g0 & 1u) == 0u;
+      const bool had1 = it.T >= 2 || (g0 & 1u) == 1u;
+      bool e_ok = first || mbar_wait(&bars->o_done[X], (u - 1) & 1, abort, status);
+      bars->xch[n & 1][X][r] = make_float2(m, l);
+      mbar_arrive(&bars->xch_full[n & 1][X]);
+      e_ok = e_ok && mbar_wait(&bars->xch_full[n & 1][X ^ 1], (n >> 1) & 1, abort, status);
       if (!__all_sync(0xffffffffu, e_ok)) break;
       tc_fence_after();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const float2 e0 = bars->xch[n & 1][0][r], e1 = bars->xch[n & 1][1][r];
+      const float M = fmaxf(e0.x, e1.x);
+      const float f0 = (had0 && e0.x > -INFINITY) ? ex2(e0.x - M) : 0.f;
+      const float f1 = (had1 && e1.x > -INFINITY) ? ex2(e1.x - M) : 0.f;
+      const float L = e0.y * f0 + e1.y * f1;
+      const float inv = L > 0.f ? 1.f / L : 0.f;
+      const float c0 = f0 * inv, c1 = f1 * inv;
       const bool live = r < it.qlen;
-      __nv_bfloat16* op = p.O + ((size_t)it.bh * p.N + it.q0 + r) * kD;
+      __nv_bfloat16* op = p.O + ((size_t)it.bh * p.N + it.q0 + r) * kD + 64 * X;
 #pragma unroll 1
-      for (int q = 0; q < 4; ++q) {
-        uint32_t rr[32];
-        tmem_ld32(lane_addr + 2 * kBN + q * 32, rr);
+      for (int q = 0; q < 2; ++q) {
+        const uint32_t col = 64 * X + 32 * q;
+        uint32_t ra[32], rb[32];
+        if (had0) tmem_ld32(lane_addr + 2 * kBN + col, ra);
+        if (had1) tmem_ld32(lane_addr + 3 * kBN + col, rb);
         tmem_wait_ld();
         if (live) {
+          auto o = [&](int v) {
+            const float a = had0 ? __uint_as_float(ra[v]) * c0 : 0.f;
+            return had1 ? fmaf(__uint_as_float(rb[v]), c1, a) : a;
+          };
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
             uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(rr[8 * v + 0]) * inv, __uint_as_float(rr[8 * v + 1]) * inv);
-            w.y = pack_bf16x2(__uint_as_float(rr[8 * v + 2]) * inv, __uint_as_float(rr[8 * v + 3]) * inv);
-            w.z = pack_bf16x2(__uint_as_float(rr[8 * v + 4]) * inv, __uint_as_float(rr[8 * v + 5]) * inv);
-            w.w = pack_bf16x2(__uint_as_float(rr[8 * v + 6]) * inv, __uint_as_float(rr[8 * v + 7]) * inv);
+            w.x = pack_bf16x2(o(8 * v + 0), o(8 * v + 1));
+            w.y = pack_bf16x2(o(8 * v + 2), o(8 * v + 3));
+            w.z = pack_bf16x2(o(8 * v + 4), o(8 * v + 5));
+            w.w = pack_bf16x2(o(8 * v + 6), o(8 * v + 7));
             *reinterpret_cast<uint4*>(op + q * 32 + v * 8) = w;
           }
         }
       }
-      if (live && p.lse) p.lse[(size_t)it.bh * p.N + it.q0 + r] = (m + __log2f(l)) * 0.69314718055994531f;
+      if (X == 0 && live && p.lse) p.lse[(size_t)it.bh * p.N + it.q0 + r] = (M + __log2f(L)) * 0.69314718055994531f;
       tc_fence_before();
       mbar_arrive(&bars->o_free);
+      g0 += it.T;
     }
   }
 

@@ -1,7 +1,7 @@
 """Host-side model of the fused attention kernel's synchronisation protocol.
 
-The kernel's roles (TMA producer lanes, MMA issuer, softmax warpgroup) talk
-only through mbarriers.  An mbarrier wait names a phase by its
+The kernel's roles (TMA producer lanes, MMA issuer, two softmax warpgroups)
+talk only through mbarriers.  An mbarrier wait names a phase by its
 parity alone, so a wait is only meaningful while the barrier is within one
 phase of the awaited one; a role that falls two phases behind (or waits one
 phase early) reads the wrong phase.  This model replays the roles' exact
@@ -19,18 +19,20 @@ interleavings, and checks that
 * every role finishes (no deadlock).
 
 It mirrors the step structure of attention_tc.cu: per work item, one step per
-selected block followed by one step per 128-cluster chunk, 3-stage key, value
-and bias-row rings, S double-buffered in TMEM, P in the S buffer and O
-accumulated across the item.  The compensation chunks are written by an earlier
-kernel, so they are plain inputs here.
+selected block followed by one step per 128-cluster chunk; key, value and
+bias-row rings; softmax warpgroup X taking the steps g with g & 1 == X, with its
+own S buffer (P written over it) and accumulator O_X; at the end of an item the
+two warpgroups exchange (max, sum) through a double-buffered shared array and
+each reads both accumulators.  The compensation chunks are written by an
+earlier kernel, so they are plain inputs here.
 """
 import random
 
 import pytest
 
 KSTAGES = 3   # key / centroid tiles, freed when S is computed
-VSTAGES = 3   # value / vbar^U tiles, freed after P V
-BSTAGES = 3   # softmax bias rows, freed after the softmax has read them
+VSTAGES = 2   # value / vbar^U tiles, freed after P V
+BSTAGES = 4   # softmax bias rows, freed after the softmax has read them (even: one warpgroup per slot)
 
 
 class Barrier:
@@ -67,12 +69,16 @@ class Barrier:
 
 
 class Machine:
-    def __init__(self, items, nchunk, rng, lazy_v_wait=False, skip_b_empty=False):
+    def __init__(self, items, nchunk, rng, lazy_v_wait=False, skip_b_empty=False, single_xch=False,
+                 no_final_wait=False, single_xch_barrier=False):
         self.items = items                     # list of nsel per item of one CTA
         self.nchunk = nchunk
         self.rng = rng
         self.lazy_v_wait = lazy_v_wait         # planted: value lane waits for a free slot only at chunk steps
         self.skip_b_empty = skip_b_empty       # planted: bias rows loaded without waiting for a free slot
+        self.single_xch = single_xch           # planted: one (max, sum) exchange buffer for all items
+        self.no_final_wait = no_final_wait     # planted: epilogue without waiting for the last product
+        self.single_xch_barrier = single_xch_barrier   # planted: one exchange barrier per warpgroup
         B = Barrier
         self.q_full, self.q_empty = B("q_full", 1), B("q_empty", 1)
         self.k_full = [B(f"k_full{i}", 1) for i in range(KSTAGES)]
@@ -84,7 +90,13 @@ class Machine:
         self.version = {}                      # buffer -> step whose tile it holds
         self.s_full = [B(f"s_full{i}", 1) for i in range(2)]
         self.p_ready = [B(f"p_ready{i}", 1) for i in range(2)]
-        self.o_done, self.o_free = B("o_done", 1), B("o_free", 1)
+        self.o_done = [B(f"o_done{i}", 1) for i in range(2)]
+        self.o_free = B("o_free", 2)           # one arrival per warpgroup (128 threads each)
+        # exchange published: [item parity][warpgroup]; one barrier per item parity, so a warpgroup
+        # without steps cannot complete a barrier twice before the other has waited on it once
+        self.xch_full = [[B(f"xch_full{j}{i}", 1) for i in range(2)] for j in range(2)]
+        self.xch = [[None, None], [None, None]]   # [item parity][warpgroup] -> item whose (max, sum) it holds
+        self.o_content = [None, None]          # accumulator -> (item, products accumulated), at issue
         self.tc_queue = []                     # in-order tensor core: ("mma", reads, writes) / ("commit", bar)
         self.tma = []                          # in flight: (bar, buffer written, buffers read)
         self.readers = {}                      # resource -> units with an operation in flight on it
@@ -204,35 +216,57 @@ class Machine:
                 if s == 0:
                     yield lambda: self.o_free.test(n - 1)
                 self.holds(f"V{g % VSTAGES}", g)
-                self.tc_issue_mma([f"S{g & 1}", f"V{g % VSTAGES}"], ["O"])
+                x = g & 1
+                self.tc_issue_mma([f"S{x}", f"V{g % VSTAGES}"], [f"O{x}"])
+                self.o_content[x] = (n, 1) if s <= 1 else (n, self.o_content[x][1] + 1)
                 self.tc_commit(self.v_empty[g % VSTAGES])
-                self.tc_commit(self.o_done)
+                self.tc_commit(self.o_done[x])
                 g += 1
 
-    def softmax(self):
-        g = 0
+    def softmax(self, X):
+        g0 = 0
+        u = 0                                   # products into O_X issued so far
         for n, nsel in enumerate(self.items):
             T = nsel + self.nchunk
-            for s in range(T):
-                b, bs = g & 1, g % BSTAGES
+            first = True
+            for s in range((X - g0) & 1, T, 2):
+                g = g0 + s
+                bs = g % BSTAGES
                 yield lambda: self.b_full[bs].test(g // BSTAGES)
-                yield lambda: self.s_full[b].test(g >> 1)
-                assert not self.readers.get(f"S{b}"), "S read before its MMA completed"
+                yield lambda: self.s_full[X].test(g >> 1)
+                assert not self.readers.get(f"S{X}"), "S read before its MMA completed"
                 assert not self.readers.get(f"BIAS{bs}"), "bias row read before it landed"
                 self.holds(f"BIAS{bs}", g)
-                self._write(f"S{b}", "softmax (P)")
+                self._write(f"S{X}", "softmax (P)")
                 self.b_empty[bs].arrive()
-                if s > 0:
-                    yield lambda: self.o_done.test(g - 1)
-                    self._write("O", "softmax (rescale)")
-                self.p_ready[b].arrive()
-                g += 1
-            yield lambda: self.o_done.test(g - 1)
-            self._write("O", "epilogue")
+                if not first:
+                    yield lambda: self.o_done[X].test(u - 1)
+                    self._write(f"O{X}", "softmax (rescale)")
+                self.p_ready[X].arrive()
+                first = False
+                u += 1
+            # epilogue
+            if not first and not self.no_final_wait:
+                yield lambda: self.o_done[X].test(u - 1)
+            slot = 0 if self.single_xch else n & 1
+            self.xch[slot][X] = n
+            if self.single_xch_barrier:
+                self.xch_full[0][X].arrive()
+                yield lambda: self.xch_full[0][X ^ 1].test(n)
+            else:
+                self.xch_full[n & 1][X].arrive()
+                yield lambda: self.xch_full[n & 1][X ^ 1].test(n >> 1)
+            assert self.xch[slot][X ^ 1] == n, f"exchange slot holds item {self.xch[slot][X ^ 1]}, read for item {n}"
+            for Y in (0, 1):
+                steps = len(range((Y - g0) & 1, T, 2))
+                if steps:
+                    assert not self.readers.get(f"O{Y}"), f"O{Y} read while a product into it is in flight"
+                    assert self.o_content[Y] == (n, steps), f"O{Y} holds {self.o_content[Y]} at the end of item {n}"
             self.o_free.arrive()
+            g0 += T
 
     def run(self, max_iters=200000):
-        roles = [self.producer(), self.producer_v(), self.mma(), self.softmax()]
+        roles = [self.producer(), self.producer_v(), self.mma(), self.softmax(0), self.softmax(1)]
         waits = [None] * len(roles)
         done = [False] * len(roles)
         for _ in range(max_iters):
@@ -290,3 +324,19 @@ def test_model_catches_a_lane_that_skips_ring_phases():
 
 def test_model_catches_bias_rows_loaded_without_a_free_slot():
     assert _caught([3, 3, 3, 3, 3], 2, skip_b_empty=True) > 0
+
+
+def test_model_catches_a_single_exchange_buffer():
+    """With one-step items a warpgroup without steps reaches the next exchange while the other
+    still reads the previous one."""
+    assert _caught([0, 0, 0, 0, 0, 0], 1, single_xch=True) > 0
+
+
+def test_model_catches_an_epilogue_that_does_not_wait_for_the_last_product():
+    assert _caught([3, 4, 1], 2, no_final_wait=True) > 0
+
+
+def test_model_catches_one_exchange_barrier_per_warpgroup():
+    """A warpgroup without steps in an item can complete a single exchange barrier twice before
+    the other warpgroup's parity wait on it runs."""
+    assert _caught([1, 0, 0, 1], 1, single_xch_barrier=True) > 0
