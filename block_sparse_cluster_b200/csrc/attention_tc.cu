@@ -46,8 +46,8 @@ namespace {
 constexpr int kD = 128;
 constexpr int kBM = 128;                 // query rows per item
 constexpr int kBN = 128;                 // keys per block / clusters per chunk
-constexpr int kKStages = 3;             // key / centroid tiles (freed as soon as S is computed)
-constexpr int kVStages = 2;             // value / vbar^U tiles (freed after P V)
+constexpr int kKStages = 2;             // key / centroid tiles (freed as soon as S is computed)
+constexpr int kVStages = 3;             // value / vbar^U tiles (freed after P V)
 constexpr int kBStages = 4;             // bias rows of the softmax (even: a slot serves one warpgroup)
 constexpr int kTile = kBN * kD * 2;      // 32 KB bf16 tile
 constexpr int kPanel = kBN * 128;        // one 64-column panel (128 rows x 128 B)
@@ -58,7 +58,7 @@ constexpr int kWarpMMA = 9;
 constexpr int kWarpProducerV = 10;
 // Register split (setmaxnreg): the launch holds 384 x 168 registers; the softmax warpgroups grow,
 // the producer / MMA warpgroup shrinks.
-constexpr int kRegSoftmax = 216, kRegIssue = 72;
+constexpr int kRegSoftmax = 232, kRegIssue = 40;
 static_assert(128 * (2 * kRegSoftmax + kRegIssue) <= kThreads * 168, "register split above the launch");
 static_assert(kBStages % 2 == 0, "a bias slot must always serve the same softmax warpgroup");
 constexpr int kChunkBytes = kTile + kBN * 4;   // compensation chunk: vbar^U rows, then log2 n^U
@@ -75,6 +75,7 @@ struct __align__(8) Bars {
   uint64_t xch_full[2][2];
   uint32_t tmem_base;
   int abort;
+  int bflag[kBStages];                   // 1: the slot's bias row is all zero (a full key block)
   float2 xch[2][2][kBM];                 // [item parity][warpgroup][row] = (max, sum)
 };
 
@@ -135,41 +136,69 @@ __device__ __forceinline__ const uint8_t* comp_chunk(const Params& p, const Item
   return p.comp + ((size_t)(it.bh * p.nB + it.i) * p.nchunk + c) * kChunkBytes;
 }
 
-// Softmax helpers over 32 columns of S (raw bits in r): logits y = x * s*log2(e) + bias.
-__device__ __forceinline__ float chunk_max(const uint32_t (&r)[32], const float* bias, uint64_t sl2x2) {
-  float m0 = -INFINITY, m1 = -INFINITY;
-#pragma unroll
-  for (int v = 0; v < 8; ++v) {
-    const float4 bb = *reinterpret_cast<const float4*>(bias + 4 * v);
-    const uint64_t y0 = f2_fma(f2_pack(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1])), sl2x2, f2_pack(bb.x, bb.y));
-    const uint64_t y1 = f2_fma(f2_pack(__uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3])), sl2x2, f2_pack(bb.z, bb.w));
-    float a, c, d, e;
-    f2_unpack(y0, a, c);
-    f2_unpack(y1, d, e);
-    m0 = fmax3(m0, a, c);
-    m1 = fmax3(m1, d, e);
-  }
-  return fmaxf(m0, m1);
+// Orders later uses of r after a tcgen05.wait::ld already issued (emits no instruction).
+__device__ __forceinline__ void reg_fence32(uint32_t (&r)[32]) {
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                 "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
+                 "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),
+                 "+r"(r[29]), "+r"(r[30]), "+r"(r[31]));
 }
-// p = 2^(y - m) for 32 columns: packed to bf16 pairs in pk, summed (fp32 pairs) into rsum.
-__device__ __forceinline__ void chunk_exp(const uint32_t (&r)[32], const float* bias, uint64_t sl2x2, uint64_t negmu,
-                                          uint32_t (&pk)[16], uint64_t& rsum) {
+
+// Softmax of one S row held in registers (128 columns as raw fp32 bits).  A column's logit in
+// log2 units is y_c = x_c * s*log2(e) + bias_c.  On a full key block the bias row is zero and
+// the row max is taken on the raw scores (the scale is positive); otherwise y is formed in
+// place first.  Returns the row max of y.
+__device__ __forceinline__ float row_logits_max(uint32_t (&x)[4][32], const float* bias, bool plain, float sl2) {
+  if (!plain) {
+    const uint64_t sl2x2 = f2_pack(sl2, sl2);
 #pragma unroll
-  for (int v = 0; v < 8; ++v) {
-    const float4 bb = *reinterpret_cast<const float4*>(bias + 4 * v);
-    const uint64_t y0 = f2_add(f2_fma(f2_pack(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1])), sl2x2,
-                                      f2_pack(bb.x, bb.y)), negmu);
-    const uint64_t y1 = f2_add(f2_fma(f2_pack(__uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3])), sl2x2,
-                                      f2_pack(bb.z, bb.w)), negmu);
-    float a, c, d, e;
-    f2_unpack(y0, a, c);
-    f2_unpack(y1, d, e);
-    const float pa = ex2(a), pc = ex2(c), pd = ex2(d), pe = ex2(e);
-    rsum = f2_add(rsum, f2_pack(pa, pc));
-    rsum = f2_add(rsum, f2_pack(pd, pe));
-    pk[2 * v] = pack_bf16x2(pa, pc);
-    pk[2 * v + 1] = pack_bf16x2(pd, pe);
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+      for (int v = 0; v < 32; v += 4) {
+        const float4 bb = *reinterpret_cast<const float4*>(bias + 32 * q + v);
+        const uint64_t y0 = f2_fma(f2_pack(__uint_as_float(x[q][v]), __uint_as_float(x[q][v + 1])), sl2x2, f2_pack(bb.x, bb.y));
+        const uint64_t y1 = f2_fma(f2_pack(__uint_as_float(x[q][v + 2]), __uint_as_float(x[q][v + 3])), sl2x2, f2_pack(bb.z, bb.w));
+        float a, c, d, e;
+        f2_unpack(y0, a, c);
+        f2_unpack(y1, d, e);
+        x[q][v] = __float_as_uint(a);
+        x[q][v + 1] = __float_as_uint(c);
+        x[q][v + 2] = __float_as_uint(d);
+        x[q][v + 3] = __float_as_uint(e);
+      }
   }
+  float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+#pragma unroll
+    for (int v = 0; v < 32; v += 8) {
+      m0 = fmax3(m0, __uint_as_float(x[q][v]), __uint_as_float(x[q][v + 1]));
+      m1 = fmax3(m1, __uint_as_float(x[q][v + 2]), __uint_as_float(x[q][v + 3]));
+      m2 = fmax3(m2, __uint_as_float(x[q][v + 4]), __uint_as_float(x[q][v + 5]));
+      m3 = fmax3(m3, __uint_as_float(x[q][v + 6]), __uint_as_float(x[q][v + 7]));
+    }
+  const float mr = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+  return plain ? mr * sl2 : mr;
+}
+
+// p = 2^(x * coef - mu) for the 32 columns of chunk q: packed to bf16 pairs in pk, summed (fp32
+// pairs) into rsum.  coef is s*log2(e) on a full key block and 1 when x already holds y.
+__device__ __forceinline__ void chunk_exp(const uint32_t (&x)[32], uint64_t coef, uint64_t negmu, uint32_t (&pk)[16],
+                                          uint64_t& rsum) {
+  uint64_t s0 = 0, s1 = 0;                // two accumulators: shorter dependency chains
+#pragma unroll
+  for (int v = 0; v < 16; ++v) {
+    const uint64_t y = f2_fma(f2_pack(__uint_as_float(x[2 * v]), __uint_as_float(x[2 * v + 1])), coef, negmu);
+    float a, c;
+    f2_unpack(y, a, c);
+    const float pa = ex2(a), pc = ex2(c);
+    if (v & 1) s1 = f2_add(s1, f2_pack(pa, pc));
+    else s0 = f2_add(s0, f2_pack(pa, pc));
+    pk[v] = pack_bf16x2(pa, pc);
+  }
+  rsum = f2_add(rsum, f2_add(s0, s1));
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -260,6 +289,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             // (generic stores, published to the softmax by the arrive on b_full)
             if (!mbar_wait(&bars->b_empty[bs], ((g / kBStages) & 1) ^ 1, abort, status)) { ok = false; break; }
             const int ncol = valid ? min(kBN, p.N - j * kBN) : 0;
+            bars->bflag[bs] = ncol == kBN ? 1 : 0;
             float4* bb = reinterpret_cast<float4*>(sBias + bs * kBN);
 #pragma unroll 4
             for (int c4 = 0; c4 < kBN / 4; ++c4) {
@@ -274,6 +304,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             tma_load_3d(dk, &tm_c, &bars->k_full[ks], 0, c * kBN, it.bh);
             tma_load_3d(dk + kPanel, &tm_c, &bars->k_full[ks], 64, c * kBN, it.bh);
             if (!mbar_wait(&bars->b_empty[bs], ((g / kBStages) & 1) ^ 1, abort, status)) { ok = false; break; }
+            bars->bflag[bs] = 0;
             mbar_expect_tx(&bars->b_full[bs], kBN * 4);
             bulk_load(sBias + bs * kBN, comp_chunk(p, it, c) + kTile, kBN * 4, &bars->b_full[bs]);
           }
@@ -403,27 +434,23 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         w_ok = w_ok && mbar_wait(&bars->s_full[X], (g >> 1) & 1, abort, status);
         if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
         tc_fence_after();
-        // Two passes over the S row in TMEM, 32 columns at a time with the next load in flight: the
-        // row max, then p = 2^(x - m), the row sum and the bf16 P written back over S.  Column c's
-        // logit is x_c * s*log2(e) + bias_c, the bias row in shared memory: log2 n^U_c on a
-        // compensation step, 0 on a key block (-inf past the end of a short last block).
+        // The S row is loaded from TMEM once (128 registers): the row max, then p = 2^(y - m), the
+        // row sum and the bf16 P written back over S.  Column c's logit is y_c = x_c * s*log2(e) +
+        // bias_c, the bias row in shared memory: log2 n^U_c on a compensation step, 0 on a key
+        // block (-inf past the end of a short last block).
         const uint32_t sbase = lane_addr + X * kBN;
         const float* bt = sBias + bs * kBN;
-        const uint64_t sl2x2 = f2_pack(p.scale_log2, p.scale_log2);
-        float mx = -INFINITY;
-        {
-          uint32_t ra[32], rb[32];
-          tmem_ld32(sbase, ra);
-#pragma unroll 1
-          for (int q = 0; q < 4; q += 2) {
-            tmem_wait_ld_into(ra);
-            tmem_ld32(sbase + (q + 1) * 32, rb);
-            mx = fmaxf(mx, chunk_max(ra, bt + q * 32, sl2x2));
-            tmem_wait_ld_into(rb);
-            if (q + 2 < 4) tmem_ld32(sbase + (q + 2) * 32, ra);
-            mx = fmaxf(mx, chunk_max(rb, bt + (q + 1) * 32, sl2x2));
-          }
-        }
+        const bool plain = bars->bflag[bs] != 0 && p.scale_log2 > 0.f;
+        uint32_t x[4][32];
+        tmem_ld32(sbase, x[0]);
+        tmem_ld32(sbase + 32, x[1]);
+        tmem_ld32(sbase + 64, x[2]);
+        tmem_ld32(sbase + 96, x[3]);
+        tmem_wait_ld_into(x[0]);
+        reg_fence32(x[1]);
+        reg_fence32(x[2]);
+        reg_fence32(x[3]);
+        const float mx = row_logits_max(x, bt, plain, p.scale_log2);
         // lazy rescaling: the running max moves only when it grows by more than 2^8
         const bool grow = mx > m + kRescaleLog2 || (m == -INFINITY && mx > -INFINITY);
         const bool need_o = grow && !first && m > -INFINITY;
@@ -432,19 +459,12 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         uint64_t rsum = 0;
         {
           const uint64_t negmu = f2_pack(-mu, -mu);
-          uint32_t ra[32], rb[32];
-          tmem_ld32(sbase, ra);
-#pragma unroll 1
-          for (int q = 0; q < 4; q += 2) {
+          const uint64_t coef = plain ? f2_pack(p.scale_log2, p.scale_log2) : f2_pack(1.f, 1.f);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
             uint32_t pk[16];
-            tmem_wait_ld_into(ra);
-            tmem_ld32(sbase + (q + 1) * 32, rb);
-            chunk_exp(ra, bt + q * 32, sl2x2, negmu, pk, rsum);
+            chunk_exp(x[q], coef, negmu, pk, rsum);
             tmem_st16(sbase + q * 16, pk);
-            tmem_wait_ld_into(rb);
-            if (q + 2 < 4) tmem_ld32(sbase + (q + 2) * 32, ra);
-            chunk_exp(rb, bt + (q + 1) * 32, sl2x2, negmu, pk, rsum);
-            tmem_st16(sbase + (q + 1) * 16, pk);
           }
         }
         mbar_arrive(&bars->b_empty[bs]);          // this thread has read the bias row

@@ -30,8 +30,8 @@ import random
 
 import pytest
 
-KSTAGES = 3   # key / centroid tiles, freed when S is computed
-VSTAGES = 2   # value / vbar^U tiles, freed after P V
+KSTAGES = 2   # key / centroid tiles, freed when S is computed
+VSTAGES = 3   # value / vbar^U tiles, freed after P V
 BSTAGES = 4   # softmax bias rows, freed after the softmax has read them (even: one warpgroup per slot)
 
 
