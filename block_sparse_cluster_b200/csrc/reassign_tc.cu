@@ -3,15 +3,17 @@
 // "each step reassigns the drifting keys to cached centroids and refreshes compensation"
 // (DecoupAttn abstract).  One CTA per (head, key block of 128 keys):
 //   1. TMA loads the key tile (128 x 128 bf16, 128-byte swizzle) and the centroid chunks
-//      (256 x 128 bf16 each, double buffered).
-//   2. One thread issues tcgen05.mma: D[key, c] = k . cbar_c into TMEM (fp32, 256 columns per
+//      (128 x 128 bf16 each, double buffered).
+//   2. One thread issues tcgen05.mma: D[key, c] = k . cbar_c into TMEM (fp32, 128 columns per
 //      chunk, two TMEM buffers so the next chunk's contraction overlaps this chunk's epilogue).
 //   3. Every thread owns one key (= one TMEM lane) and keeps the running argmin of
 //      ||cbar_c||^2 - 2 k.cbar_c (ties to the lowest c; the key's own norm is the same for
 //      every c and is dropped).
 //   4. The same 128 threads refresh the block's statistics (block_stats.cuh): sorted entry list,
-//      histogram row, entry index row and fp32 value sums, reading the block's value rows from a
-//      shared-memory copy (TMA, loaded with the key tile).
+//      histogram row, entry index row and fp32 value sums, reading the block's value rows from
+//      shared memory (copied with cp.async into the centroid buffer, free once the last MMA is done).
+// The CTA takes about 109 KB of shared memory and 256 TMEM columns, so two CTAs share an SM and
+// one's contraction overlaps the other's argmin and statistics.
 #include "block_stats.cuh"
 #include "da_common.cuh"
 #include "da_internal.h"
@@ -23,7 +25,8 @@ namespace {
 
 constexpr int kKeys = 128;           // keys per tile (= block)
 constexpr int kD = 128;              // head dimension
-constexpr int kChunk = 256;          // centroids per MMA chunk (N of the MMA)
+constexpr int kChunk = 128;          // centroids per MMA chunk (N of the MMA)
+constexpr int kMaxC = 1024;          // centroid norms staged in shared memory
 constexpr int kKTileBytes = kKeys * kD * 2;        // 32 KB
 constexpr int kCTileBytes = kChunk * kD * 2;       // 64 KB
 constexpr int kPanelK = kKeys * 128;               // one 64-column panel of the key tile
@@ -37,23 +40,22 @@ struct __align__(8) Bars {
   int abort;
 };
 
-constexpr size_t kSmemBytes = 1024 /*align slack*/ + 2 * kKTileBytes /*K, V*/ + 2 * kCTileBytes + 4096 /*norms*/ +
+constexpr size_t kSmemBytes = 1024 /*align slack*/ + kKTileBytes /*K*/ + 2 * kCTileBytes + kMaxC * 4 /*norms*/ +
                               sizeof(StatsSmem) + 512 /*assign*/ + 128 /*bars*/;
 static_assert(sizeof(Bars) <= 128, "barrier block");
-static_assert(kSmemBytes <= 232448, "shared memory above the 227 KB per-block limit");
+static_assert(2 * (kSmemBytes + 1024) <= 233472, "two CTAs per SM");
 
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(128, 2)
 reassign_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_c,
-                   const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ norms, StatsPtrs st, int N,
+                   const __nv_bfloat16* __restrict__ V, const float* __restrict__ norms, StatsPtrs st, int N,
                    int C, int nB, int* status) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   uint8_t* sK = base;
-  uint8_t* sVt = sK + kKTileBytes;                 // value rows of the block, [128][128] bf16, unswizzled
-  uint8_t* sC0 = sVt + kKTileBytes;
+  uint8_t* sC0 = sK + kKTileBytes;
   float* s_norm = reinterpret_cast<float*>(sC0 + 2 * kCTileBytes);
-  StatsSmem* ssm = reinterpret_cast<StatsSmem*>(s_norm + 1024);
+  StatsSmem* ssm = reinterpret_cast<StatsSmem*>(s_norm + kMaxC);
   int* s_assign = reinterpret_cast<int*>(ssm + 1);
   Bars* bars = reinterpret_cast<Bars*>(s_assign + 128);
 
@@ -75,7 +77,7 @@ reassign_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     fence_mbar_init();
   }
   if (warp == 0) {
-    tmem_alloc(&bars->tmem_base, 512);
+    tmem_alloc(&bars->tmem_base, 2 * kChunk);
     tmem_relinquish();
   }
   for (int c = t; c < C; c += 128) s_norm[c] = norms[(size_t)bh * C + c];
@@ -111,11 +113,9 @@ reassign_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
   if (t == 0) {
     tma_prefetch(&tm_k);
     tma_prefetch(&tm_c);
-    tma_prefetch(&tm_v);
-    mbar_expect_tx(&bars->kfull, 2 * kKTileBytes);
+    mbar_expect_tx(&bars->kfull, kKTileBytes);
     tma_load_3d(sK, &tm_k, &bars->kfull, 0, k0, bh);
     tma_load_3d(sK + kPanelK, &tm_k, &bars->kfull, 64, k0, bh);
-    tma_load_3d(sVt, &tm_v, &bars->kfull, 0, k0, bh);
     load_chunk(0);
     if (nchunks > 1) load_chunk(1);
     if (mbar_wait(&bars->kfull, 0, abort, status)) issue_mma(0);
@@ -133,13 +133,19 @@ reassign_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
       uint32_t r[32];
       tmem_ld32(lane_base + (c & 1) * kChunk + col, r);
       tmem_wait_ld();
+      const float4* nv = reinterpret_cast<const float4*>(s_norm + c * kChunk + col);
 #pragma unroll
-      for (int q = 0; q < 32; ++q) {
-        const int cc = c * kChunk + col + q;
-        const float dist = fmaf(-2.f, __uint_as_float(r[q]), s_norm[cc]);
-        if (dist < best) {
-          best = dist;
-          arg = cc;
+      for (int q4 = 0; q4 < 8; ++q4) {
+        const float4 nn = nv[q4];
+        const float nq[4] = {nn.x, nn.y, nn.z, nn.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int q = 4 * q4 + u;
+          const float dist = fmaf(-2.f, __uint_as_float(r[q]), nq[u]);
+          if (col + q < n && dist < best) {   // ascending c: ties keep the lowest index
+            best = dist;
+            arg = c * kChunk + col + q;
+          }
         }
       }
     }
@@ -151,13 +157,18 @@ reassign_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
   __syncthreads();
 
   if (!*abort) {
+    // every MMA has completed (the last chunk's mdone was waited): the centroid buffer is free
+    const __nv_bfloat16* Vg = V + ((size_t)bh * N + k0) * kD;
+    for (int i = t; i < nk * kD / 8; i += 128) cp_async16(sC0 + (size_t)i * 16, Vg + (size_t)i * 8);
+    cp_async_commit();
     if (t < nk) {
       s_assign[t] = arg;
       st.assign[(size_t)bh * N + k0 + t] = arg;
     }
+    cp_async_wait<0>();
     __syncthreads();
     const size_t bj = (size_t)bh * nB + j;
-    block_stats_group<__nv_bfloat16, kD>(t, 1, s_assign, nk, reinterpret_cast<const __nv_bfloat16*>(sVt), C,
+    block_stats_group<__nv_bfloat16, kD>(t, 1, s_assign, nk, reinterpret_cast<const __nv_bfloat16*>(sC0), C,
                                          st.blk_hist + bj * C, st.seg_idx + bj * C, st.seg_n + bj,
                                          st.seg_c + bj * kKeys, st.seg_cnt + bj * kKeys,
                                          st.seg_vsum + bj * kKeys * kD, *ssm);
@@ -166,26 +177,26 @@ reassign_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, 2 * kChunk);
   }
 }
 
 }  // namespace
 
-bool reassign_tc_supported(const Dims& g) { return g.bf16 && g.d == kD && g.block == kKeys; }
+bool reassign_tc_supported(const Dims& g) { return g.bf16 && g.d == kD && g.block == kKeys && g.C <= kMaxC; }
 
 cudaError_t launch_reassign_tc(const Dims& g, const void* K, const void* V, const void* cent, const float* norms,
                                const StatsPtrs& st, int* status, cudaStream_t s) {
-  CUtensorMap tk, tc, tv;
+  CUtensorMap tk, tc;
   const unsigned long long BH = (unsigned long long)g.B * g.H;
   if (!make_tmap_bf16_3d(&tk, K, kD, g.N, BH, 64, kKeys)) return cudaErrorInvalidValue;
   if (!make_tmap_bf16_3d(&tc, cent, kD, g.C, BH, 64, kChunk)) return cudaErrorInvalidValue;
-  if (!make_tmap_bf16_3d(&tv, V, kD, g.N, BH, kD, kKeys, false)) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(reassign_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid(g.nB, (unsigned)BH);
-  reassign_tc_kernel<<<grid, 128, kSmemBytes, s>>>(tk, tc, tv, norms, st, g.N, g.C, g.nB, status);
+  reassign_tc_kernel<<<grid, 128, kSmemBytes, s>>>(tk, tc, static_cast<const __nv_bfloat16*>(V), norms, st, g.N,
+                                                   g.C, g.nB, status);
   return cudaGetLastError();
 }
 

@@ -60,40 +60,42 @@ __global__ void __launch_bounds__(128) block_stats_kernel(const T* __restrict__ 
 // combined in warp order.
 template <int D>
 __global__ void __launch_bounds__(128) totals_kernel(StatsPtrs st, int C, int block, int nB) {
-  extern __shared__ float part[];   // [4][32][D]
-  __shared__ int cnt[4][32];
-  const int bh = blockIdx.x, c0 = blockIdx.y * 32;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  constexpr int NE = D / 32;
-  float* mine = part + (size_t)warp * 32 * D;
-  for (int x = lane; x < 32 * D; x += 32) mine[x] = 0.f;
-  __syncwarp();
-  int my_n = 0;
-  for (int j = warp; j < nB; j += 4) {
-    const size_t bj = (size_t)bh * nB + j;
-    const int e = st.seg_idx[bj * C + c0 + lane];
-    unsigned m = __ballot_sync(0xffffffffu, e != 0xFF);
-    if (e != 0xFF) my_n += st.seg_cnt[bj * block + e];
-    while (m) {
-      const int L = __ffs(m) - 1;
-      m &= m - 1;
-      const int eL = __shfl_sync(0xffffffffu, e, L);
-      const float* src = st.seg_vsum + (bj * block + eL) * D + lane * NE;
-      float* dst = mine + L * D + lane * NE;
+  // thread t: cluster c0 + t/4, value columns [(t%4) * D/4, (t%4+1) * D/4); the cluster's entries
+  // are summed over the blocks in block order (registers, a fixed order: deterministic bits)
+  constexpr int NS = D / 4;               // columns per thread
+  const int bh = blockIdx.x;
+  const int c = blockIdx.y * 32 + (threadIdx.x >> 2);
+  const int q = threadIdx.x & 3;
+  float acc[NS];
 #pragma unroll
-      for (int i = 0; i < NE; ++i) dst[i] += src[i];
+  for (int i = 0; i < NS; ++i) acc[i] = 0.f;
+  int n = 0;
+  const size_t hb = (size_t)bh * nB;
+  constexpr int kB = 8;                   // blocks looked up per batch
+  for (int j0 = 0; j0 < nB; j0 += kB) {
+    int e[kB];
+#pragma unroll
+    for (int u = 0; u < kB; ++u) e[u] = j0 + u < nB ? (int)st.seg_idx[(hb + j0 + u) * C + c] : 0xFF;
+#pragma unroll
+    for (int u = 0; u < kB; ++u) {
+      if (e[u] == 0xFF) continue;
+      const size_t row = (hb + j0 + u) * block + e[u];
+      if (q == 0) n += st.seg_cnt[row];
+      const float4* src = reinterpret_cast<const float4*>(st.seg_vsum + row * D + q * NS);
+#pragma unroll
+      for (int i = 0; i < NS / 4; ++i) {
+        const float4 y = __ldg(src + i);
+        acc[4 * i] += y.x;
+        acc[4 * i + 1] += y.y;
+        acc[4 * i + 2] += y.z;
+        acc[4 * i + 3] += y.w;
+      }
     }
   }
-  cnt[warp][lane] = my_n;
-  __syncthreads();
-  for (int x = threadIdx.x; x < 32 * D; x += 128) {
-    const float s = ((part[x] + part[32 * D + x]) + part[2 * 32 * D + x]) + part[3 * 32 * D + x];
-    st.S_tot[((size_t)bh * C + c0) * D + x] = s;
-  }
-  if (threadIdx.x < 32) {
-    const int l = threadIdx.x;
-    st.n_tot[(size_t)bh * C + c0 + l] = cnt[0][l] + cnt[1][l] + cnt[2][l] + cnt[3][l];
-  }
+  float4* dst = reinterpret_cast<float4*>(st.S_tot + ((size_t)bh * C + c) * D + q * NS);
+#pragma unroll
+  for (int i = 0; i < NS / 4; ++i) dst[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
+  if (q == 0) st.n_tot[(size_t)bh * C + c] = n;
 }
 
 // Plan validation and work order: items of a head ordered by descending row length
@@ -158,15 +160,8 @@ cudaError_t launch_block_stats(const Dims& g, const void* V, const StatsPtrs& st
 
 cudaError_t launch_totals(const Dims& g, const StatsPtrs& st, cudaStream_t s) {
   dim3 grid(g.B * g.H, g.C / 32);
-  const size_t smem = (size_t)4 * 32 * g.d * sizeof(float);
-  cudaError_t e;
-  if (g.d == 128) {
-    e = cudaFuncSetAttribute(totals_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    totals_kernel<128><<<grid, 128, smem, s>>>(st, g.C, g.block, g.nB);
-  } else {
-    totals_kernel<64><<<grid, 128, smem, s>>>(st, g.C, g.block, g.nB);
-  }
+  if (g.d == 128) totals_kernel<128><<<grid, 128, 0, s>>>(st, g.C, g.block, g.nB);
+  else totals_kernel<64><<<grid, 128, 0, s>>>(st, g.C, g.block, g.nB);
   return cudaGetLastError();
 }
 
