@@ -8,11 +8,11 @@
 // One CTA per (item, 128-cluster chunk) writes the chunk as 128 bf16 rows of d = 128 (the layout a
 // TMA tile load reads) followed by the 128 fp32 beta values.
 //
-// Phase 1: thread t <-> cluster row t of the chunk looks the row up in every selected block
-// (seg_idx: the entry of the cluster in the block, or 0xFF) with independent loads, keeping the
-// first kSlots entries in block order and the selected count.  Phase 2: each warp builds 16 rows
-// with lanes over d (coalesced 512-byte rows): S_c minus the entries' value sums, summed in block
-// order, times 1 / n^U_c.
+// Phase 1: thread (row, h) looks the row up in half h of the selected blocks (seg_idx: the entry
+// of the cluster in the block, or 0xFF) with batches of independent loads, keeping the first
+// kSlots entries of its half in block order and the half's selected count.  Phase 2: each warp
+// builds 16 rows with lanes over d (coalesced 512-byte rows): S_c minus the entries' value sums
+// (slot k of both halves before slot k + 1: a fixed order), times 1 / n^U_c.
 #include "da_common.cuh"
 #include "da_internal.h"
 
@@ -22,13 +22,15 @@ namespace {
 
 constexpr int kD = 128;
 constexpr int kRows = 128;               // clusters per chunk
-constexpr int kSlots = 8;                // entries per row kept from phase 1
-constexpr int kThreads = 256;            // 8 warps: 16 rows each in phase 2
+constexpr int kSlots = 4;                // entries per (row, half) kept from phase 1
+constexpr int kThreads = 256;            // phase 1: (row, half); phase 2: 8 warps x 16 rows
+constexpr int kBatch = 16;               // lookups in flight per thread
 constexpr int kChunkBytes = kRows * kD * 2 + kRows * 4;
 
 struct Smem {
-  uint32_t ptr[kRows][kSlots];           // entry rows (block row * block + entry), block order
-  int nm[kRows];                         // entries of the row in the selected blocks
+  uint32_t ptr[2][kRows][kSlots];        // entry rows (block row * block + entry), block order
+  int nm[2][kRows];                      // entries of the row in each half of the selected blocks
+  int csel[2][kRows];                    // selected keys of the cluster in each half
   float inv[kRows];                      // 1 / n^U (0 when n^U = 0)
 };
 
@@ -49,30 +51,42 @@ comp_build_kernel(StatsPtrs st, const int32_t* __restrict__ kv_idx, const int32_
   const size_t hc = (size_t)bh * C;                    // first cluster row of the head
   uint8_t* chunk = out + (size_t)blockIdx.x * kChunkBytes;
 
+  {
+    const int rr = t & (kRows - 1), h = t / kRows;
+    const int r = c * kRows + rr;
+    const bool rl = r < C;
+    const int mid = (nsel + 1) >> 1;
+    const int sb = h ? mid : 0, se = h ? nsel : mid;
+    int nm = 0, cs = 0;
+    for (int s0 = sb; s0 < se; s0 += kBatch) {
+      int e[kBatch], hv[kBatch];
+      uint32_t bb[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int sidx = s0 + u;
+        const int jr = sidx < se ? __ldg(row + sidx) : -1;
+        const bool ok = rl && jr >= 0 && jr < nB;
+        const size_t bj = hb + (ok ? jr : 0);
+        bb[u] = (uint32_t)(bj * block);
+        e[u] = ok ? (int)__ldg(st.seg_idx + bj * C + r) : 0xFF;
+        hv[u] = ok ? __ldg(st.blk_hist + bj * C + r) : 0;
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        if (e[u] != 0xFF) {
+          if (nm < kSlots) sm.ptr[h][rr][nm] = bb[u] + (uint32_t)e[u];
+          ++nm;
+        }
+        cs += hv[u];                                     // zero where the cluster is absent
+      }
+    }
+    sm.nm[h][rr] = nm;
+    sm.csel[h][rr] = cs;
+  }
+  __syncthreads();
   if (t < kRows) {
     const int r = c * kRows + t;
-    const bool rl = r < C;
-    int nm = 0, csel = 0;
-    uint32_t mp[kSlots];
-#pragma unroll
-    for (int k = 0; k < kSlots; ++k) mp[k] = 0;
-#pragma unroll 8
-    for (int s = 0; s < nsel; ++s) {
-      const int jr = row[s];
-      const bool ok = rl && jr >= 0 && jr < nB;
-      const size_t bj = hb + (ok ? jr : 0);
-      const int e = ok ? (int)st.seg_idx[bj * C + r] : 0xFF;
-      const bool hit = e != 0xFF;
-      csel += hit ? st.blk_hist[bj * C + r] : 0;
-      const uint32_t ptr = (uint32_t)(bj * block + (hit ? e : 0));
-#pragma unroll
-      for (int k = 0; k < kSlots; ++k) mp[k] = (hit && nm == k) ? ptr : mp[k];
-      nm += hit ? 1 : 0;
-    }
-    const int nU = rl ? st.n_tot[hc + r] - csel : 0;
-#pragma unroll
-    for (int k = 0; k < kSlots; ++k) sm.ptr[t][k] = mp[k];
-    sm.nm[t] = nm;
+    const int nU = r < C ? st.n_tot[hc + r] - sm.csel[0][t] - sm.csel[1][t] : 0;
     sm.inv[t] = nU > 0 ? 1.f / (float)nU : 0.f;
     reinterpret_cast<float*>(chunk + kRows * kD * 2)[t] = nU > 0 ? log2f((float)nU) : -INFINITY;
   }
@@ -81,12 +95,13 @@ comp_build_kernel(StatsPtrs st, const int32_t* __restrict__ kv_idx, const int32_
   const int w = t >> 5, lane = t & 31;
   for (int i0 = 0; i0 < 16; i0 += 4) {
     float4 a[4];
-    int nmq[4];
+    int nmq[2][4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const int i = 16 * w + i0 + q;
       const int r = c * kRows + i;
-      nmq[q] = sm.nm[i];
+      nmq[0][q] = sm.nm[0][i];
+      nmq[1][q] = sm.nm[1][i];
       a[q] = r < C ? ldg4(st.S_tot + (hc + r) * kD + 4 * lane) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
     float4 acc[4];
@@ -95,10 +110,13 @@ comp_build_kernel(StatsPtrs st, const int32_t* __restrict__ kv_idx, const int32_
 #pragma unroll
     for (int k = 0; k < kSlots; ++k) {
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        if (nmq[q] > k) {                               // warp-uniform
-          const float4 y = ldg4(st.seg_vsum + (size_t)sm.ptr[16 * w + i0 + q][k] * kD + 4 * lane);
-          acc[q].x += y.x; acc[q].y += y.y; acc[q].z += y.z; acc[q].w += y.w;
+      for (int h = 0; h < 2; ++h) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          if (nmq[h][q] > k) {                           // warp-uniform
+            const float4 y = ldg4(st.seg_vsum + (size_t)sm.ptr[h][16 * w + i0 + q][k] * kD + 4 * lane);
+            acc[q].x += y.x; acc[q].y += y.y; acc[q].z += y.z; acc[q].w += y.w;
+          }
         }
       }
     }
@@ -106,12 +124,15 @@ comp_build_kernel(StatsPtrs st, const int32_t* __restrict__ kv_idx, const int32_
     for (int q = 0; q < 4; ++q) {
       const int i = 16 * w + i0 + q;
       const int r = c * kRows + i;
-      if (nmq[q] > kSlots) {
-        // rare: the cluster sits in more than kSlots selected blocks; the remaining entries, in
-        // block order
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        if (nmq[h][q] <= kSlots) continue;               // warp-uniform
+        // rare: the cluster sits in more than kSlots blocks of this half; the rest, in block order
+        const int mid = (nsel + 1) >> 1;
+        const int sb = h ? mid : 0, se = h ? nsel : mid;
         int seen = 0;
-        for (int s = 0; s < nsel; ++s) {
-          const int jr = row[s];
+        for (int sidx = sb; sidx < se; ++sidx) {
+          const int jr = row[sidx];
           if (jr < 0 || jr >= nB) continue;
           const size_t bj = hb + jr;
           const int e = st.seg_idx[bj * C + r];
