@@ -24,7 +24,8 @@ constexpr int kD = 128;
 constexpr int kRows = 128;               // clusters per chunk
 constexpr int kSlots = 4;                // entries per (row, half) kept from phase 1
 constexpr int kThreads = 256;            // phase 1: (row, half); phase 2: 8 warps x 16 rows
-constexpr int kBatch = 16;               // lookups in flight per thread
+constexpr int kBatch = 4;                // lookups in flight per thread
+constexpr int kGroup = 2;                // rows whose loads a warp issues together in phase 2
 constexpr int kChunkBytes = kRows * kD * 2 + kRows * 4;
 
 struct Smem {
@@ -36,7 +37,7 @@ struct Smem {
 
 __device__ __forceinline__ float4 ldg4(const float* p) { return __ldg(reinterpret_cast<const float4*>(p)); }
 
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 5)
 comp_build_kernel(StatsPtrs st, const int32_t* __restrict__ kv_idx, const int32_t* __restrict__ kv_cnt,
                   int max_sel, int N, int C, int nB, int block, int nchunk, uint8_t* __restrict__ out) {
   __shared__ Smem sm;
@@ -93,26 +94,26 @@ comp_build_kernel(StatsPtrs st, const int32_t* __restrict__ kv_idx, const int32_
   __syncthreads();
 
   const int w = t >> 5, lane = t & 31;
-  for (int i0 = 0; i0 < 16; i0 += 4) {
-    float4 a[4];
-    int nmq[2][4];
+  for (int i0 = 0; i0 < 16; i0 += kGroup) {
+    float4 a[kGroup];
+    int nmq[2][kGroup];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 0; q < kGroup; ++q) {
       const int i = 16 * w + i0 + q;
       const int r = c * kRows + i;
       nmq[0][q] = sm.nm[0][i];
       nmq[1][q] = sm.nm[1][i];
       a[q] = r < C ? ldg4(st.S_tot + (hc + r) * kD + 4 * lane) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    float4 acc[4];
+    float4 acc[kGroup];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int q = 0; q < kGroup; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int k = 0; k < kSlots; ++k) {
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < kGroup; ++q) {
           if (nmq[h][q] > k) {                           // warp-uniform
             const float4 y = ldg4(st.seg_vsum + (size_t)sm.ptr[h][16 * w + i0 + q][k] * kD + 4 * lane);
             acc[q].x += y.x; acc[q].y += y.y; acc[q].z += y.z; acc[q].w += y.w;
@@ -121,7 +122,7 @@ comp_build_kernel(StatsPtrs st, const int32_t* __restrict__ kv_idx, const int32_
       }
     }
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 0; q < kGroup; ++q) {
       const int i = 16 * w + i0 + q;
       const int r = c * kRows + i;
 #pragma unroll
