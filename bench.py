@@ -32,9 +32,10 @@ import workloads as W
 ROOT = os.path.dirname(os.path.abspath(__file__))
 METRIC = "effective TFLOP/s & ms/call of reassign+fused sparse attn; % of bf16 TC peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# DRAM bytes per launch of the attention kernel from the last ncu capture of the current kernel
-# (None until a capture of this kernel version exists).
-ATTENTION_TRAFFIC_BYTES = None
+# DRAM bytes (read + write) per launch of attention_tc_kernel at the 40-head workload: an ncu
+# capture of this kernel version on a 4-head cut of the same workload (695.9 MB), times 10 (work
+# and bytes are per head).  Set back to None whenever the kernel changes until it is re-captured.
+ATTENTION_TRAFFIC_BYTES = 6.959e9
 
 
 def _peaks():
@@ -256,13 +257,19 @@ def main():
     O = torch.empty_like(Q)
     torch.cuda.synchronize(dev)
 
-    def step(ev_pair=None):
+    def step(evs=None):
+        # the three calls of da_attention's public halves; events between them time each kernel
+        if evs is not None:
+            evs[0].record(stream)
         da.da_reassign(dims, K, V, cent, eng.stats, eng.ws)
-        if ev_pair is not None:
-            ev_pair[0].record(stream)
-        da.da_attention(dims, Q, K, V, eng.mask, cent, eng.stats, 0.0, O, None, eng.ws)
-        if ev_pair is not None:
-            ev_pair[1].record(stream)
+        if evs is not None:
+            evs[1].record(stream)
+        da.da_compensation(dims, eng.mask, eng.stats, eng.ws)
+        if evs is not None:
+            evs[2].record(stream)
+        da.da_attention_prebuilt(dims, Q, K, V, eng.mask, cent, eng.stats, 0.0, O, None, eng.ws)
+        if evs is not None:
+            evs[3].record(stream)
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -271,7 +278,7 @@ def main():
         raise RuntimeError("device status after warm-up: " + da.da_status_string(eng.status()))
 
     K_steps = args.steps
-    att_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K_steps)]
+    att_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K_steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     _barrier(ws)
     torch.cuda.synchronize(dev)
@@ -286,7 +293,9 @@ def main():
     if st != 0:
         raise RuntimeError("device status after timing: " + da.da_status_string(st))
     ms_local = start.elapsed_time(end) / K_steps
-    att_ms_local = sum(a.elapsed_time(b) for a, b in att_ev) / K_steps
+    reas_ms_local = sum(e[0].elapsed_time(e[1]) for e in att_ev) / K_steps
+    comp_ms_local = sum(e[1].elapsed_time(e[2]) for e in att_ev) / K_steps
+    att_ms_local = sum(e[2].elapsed_time(e[3]) for e in att_ev) / K_steps
     ms = _max_over_ranks(ms_local, ws, dev)
     att_ms = _max_over_ranks(att_ms_local, ws, dev)
     value = ws * eff / (ms * 1e-3) / 1e12
@@ -323,9 +332,9 @@ def main():
             "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
             "config": _config(w, args),
             "pct_of_bf16_peak": 100.0 * (value / ws) / peak,
-            "breakdown_ms": {"reassign": ms_local - att_ms_local, "attention": att_ms_local},
+            "breakdown_ms": {"reassign": reas_ms_local, "compensation": comp_ms_local, "attention": att_ms_local},
             "effective_flop_per_step_per_gpu": eff,
-            "roofline": {"bound": "tensor", "kernel": "da_attention (compensation chunks + fused attention)", "achieved": att_tflops,
+            "roofline": {"bound": "tensor", "kernel": "attention_tc_kernel (fused exact + compensation attention)", "achieved": att_tflops,
                          "peak": peak, "unit": "TFLOP/s", "frac": att_tflops / peak,
                          "peak_source": f"{kind} bf16 dense (burst)",
                          "frac_of_sustained": att_tflops / float(peaks.get("bf16_tflops_sustained", peak)),

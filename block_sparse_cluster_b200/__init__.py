@@ -27,7 +27,8 @@ STATUS_NAMES = ["DA_OK", "DA_ERR_INVALID_ARG", "DA_ERR_SHAPE", "DA_ERR_DTYPE", "
                 "DA_ERR_UNSUPPORTED", "DA_ERR_CUDA", "DA_ERR_TIMEOUT", "DA_ERR_DEVICE_INDEX",
                 "DA_ERR_WORKSPACE"]
 EXPORTS = ["da_version", "da_workspace_bytes", "da_schedule_bytes", "da_reassign", "da_mask_prepare",
-           "da_attention", "da_device_status", "da_status_string", "da_reassign_noalloc"]
+           "da_attention", "da_device_status", "da_status_string", "da_reassign_noalloc", "da_compensation",
+           "da_attention_prebuilt"]
 
 
 class DAError(RuntimeError):
@@ -66,6 +67,11 @@ _lib.da_mask_prepare.argtypes = [ctypes.POINTER(_Dims), ctypes.POINTER(_Mask), _
 _lib.da_attention.restype = ctypes.c_int
 _lib.da_attention.argtypes = [ctypes.POINTER(_Dims), _P, _P, _P, ctypes.POINTER(_Mask), _P,
                               ctypes.POINTER(_Stats), ctypes.c_float, _P, _P, _P, ctypes.c_size_t, _P]
+_lib.da_attention_prebuilt.restype = ctypes.c_int
+_lib.da_attention_prebuilt.argtypes = _lib.da_attention.argtypes
+_lib.da_compensation.restype = ctypes.c_int
+_lib.da_compensation.argtypes = [ctypes.POINTER(_Dims), ctypes.POINTER(_Mask), ctypes.POINTER(_Stats), _P,
+                                 ctypes.c_size_t, _P]
 _lib.da_reassign_noalloc.restype = ctypes.c_int
 _lib.da_reassign_noalloc.argtypes = [ctypes.POINTER(_Dims), _P, _P, _P, ctypes.POINTER(_Stats), _P]
 _lib.da_device_status.restype = ctypes.c_int
@@ -202,6 +208,23 @@ def da_attention(dims: Dims, Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, 
                              ctypes.byref(mask.c()), centroids.data_ptr(), ctypes.byref(stats.c()),
                              float(scale), O.data_ptr(), lse.data_ptr() if lse is not None else None,
                              ws.data_ptr(), ws.numel(), _stream(stream)), "da_attention")
+    return O
+
+
+def da_compensation(dims: Dims, mask: BlockMask, stats: ClusterStats, ws: torch.Tensor, stream=None) -> None:
+    """First half of da_attention: the compensation values of every q-block, into ws."""
+    _check(_lib.da_compensation(ctypes.byref(dims.c()), ctypes.byref(mask.c()), ctypes.byref(stats.c()),
+                                ws.data_ptr(), ws.numel(), _stream(stream)), "da_compensation")
+
+
+def da_attention_prebuilt(dims: Dims, Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, mask: BlockMask,
+                          centroids: torch.Tensor, stats: ClusterStats, scale: float, O: torch.Tensor,
+                          lse: Optional[torch.Tensor], ws: torch.Tensor, stream=None) -> torch.Tensor:
+    """Second half of da_attention: the fused kernel on the values da_compensation left in ws."""
+    _check(_lib.da_attention_prebuilt(ctypes.byref(dims.c()), Q.data_ptr(), K.data_ptr(), V.data_ptr(),
+                                      ctypes.byref(mask.c()), centroids.data_ptr(), ctypes.byref(stats.c()),
+                                      float(scale), O.data_ptr(), lse.data_ptr() if lse is not None else None,
+                                      ws.data_ptr(), ws.numel(), _stream(stream)), "da_attention_prebuilt")
     return O
 
 

@@ -72,7 +72,7 @@ da_status cuda_status(cudaError_t e) { return e == cudaSuccess ? DA_OK : DA_ERR_
 
 extern "C" {
 
-int da_version(void) { return 100; }
+int da_version(void) { return 101; }
 
 size_t da_workspace_bytes(const da_dims* dims) {
   Dims g;
@@ -129,24 +129,40 @@ da_status da_mask_prepare(const da_dims* dims, const da_block_mask* mask, int32_
                                      reinterpret_cast<cudaStream_t>(stream)));
 }
 
-da_status da_attention(const da_dims* dims, const void* Q, const void* K, const void* V,
-                       const da_block_mask* mask, const void* centroids, const da_cluster_stats* stats,
-                       float scale, void* O, float* lse, void* ws, size_t ws_bytes, da_stream stream) {
-  Dims g;
-  da_status st = check_dims(dims, &g);
+// Validation shared by da_compensation, da_attention_prebuilt and da_attention.
+static da_status attention_common(const da_dims* dims, const da_block_mask* mask, const da_cluster_stats* stats,
+                                  void* ws, size_t ws_bytes, Dims* g, StatsPtrs* sp) {
+  da_status st = check_dims(dims, g);
   if (st != DA_OK) return st;
+  if ((st = check_mask(*g, mask)) != DA_OK) return st;
+  if ((st = check_stats(stats, sp)) != DA_OK) return st;
+  return check_ws(*g, ws, ws_bytes);
+}
+
+static da_status check_attention_ptrs(const void* Q, const void* K, const void* V, const void* centroids,
+                                      const void* O, const float* lse) {
   if (!Q || !K || !V || !centroids || !O) return DA_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(centroids) || !aligned16(O) ||
       (lse && !aligned16(lse)))
     return DA_ERR_ALIGNMENT;
-  if ((st = check_mask(g, mask)) != DA_OK) return st;
-  StatsPtrs sp;
-  if ((st = check_stats(stats, &sp)) != DA_OK) return st;
-  if ((st = check_ws(g, ws, ws_bytes)) != DA_OK) return st;
+  return DA_OK;
+}
+
+static cudaError_t compensation_launch(const Dims& g, const da_block_mask* mask, const StatsPtrs& sp, void* ws,
+                                       cudaStream_t s) {
+  if (!attention_tc_supported(g)) return cudaSuccess;   // the CUDA-core path compensates in-kernel
+  const WsLayout L = ws_layout(g);
+  return launch_comp_build(g, mask->kv_idx, mask->kv_cnt, mask->max_sel, sp, static_cast<char*>(ws) + L.comp, s);
+}
+
+static da_status attention_launch(const Dims& g, const void* Q, const void* K, const void* V,
+                                  const da_block_mask* mask, const void* centroids, const StatsPtrs& sp, float scale,
+                                  void* O, float* lse, void* ws, cudaStream_t s) {
+  const da_status pst = check_attention_ptrs(Q, K, V, centroids, O, lse);
+  if (pst != DA_OK) return pst;
   if (!(scale > 0.f)) scale = 1.0f / sqrtf((float)g.d);
   const WsLayout L = ws_layout(g);
   int* status = reinterpret_cast<int*>(static_cast<char*>(ws) + L.status);
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int32_t* sched = mask->schedule;
   cudaError_t e = cudaSuccess;
   if (!sched) {
@@ -155,18 +171,47 @@ da_status da_attention(const da_dims* dims, const void* Q, const void* K, const 
     sched = own;
   }
   if (e == cudaSuccess) {
-    if (attention_tc_supported(g)) {
-      void* comp = static_cast<char*>(ws) + L.comp;
-      e = launch_comp_build(g, mask->kv_idx, mask->kv_cnt, mask->max_sel, sp, comp, s);
-      if (e == cudaSuccess)
-        e = launch_attention_tc(g, Q, K, V, mask->kv_idx, mask->kv_cnt, mask->max_sel, sched, centroids, sp,
-                                scale, O, lse, status, comp, s);
-    }
+    if (attention_tc_supported(g))
+      e = launch_attention_tc(g, Q, K, V, mask->kv_idx, mask->kv_cnt, mask->max_sel, sched, centroids, sp, scale, O,
+                              lse, status, static_cast<char*>(ws) + L.comp, s);
     else
       e = (g.bf16 ? launch_attention_simt_bf16 : launch_attention_simt_f32)(
           g, Q, K, V, mask->kv_idx, mask->kv_cnt, mask->max_sel, sched, centroids, sp, scale, O, lse, status, s);
   }
   return cuda_status(e);
+}
+
+da_status da_compensation(const da_dims* dims, const da_block_mask* mask, const da_cluster_stats* stats, void* ws,
+                          size_t ws_bytes, da_stream stream) {
+  Dims g;
+  StatsPtrs sp;
+  da_status st = attention_common(dims, mask, stats, ws, ws_bytes, &g, &sp);
+  if (st != DA_OK) return st;
+  return cuda_status(compensation_launch(g, mask, sp, ws, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+da_status da_attention_prebuilt(const da_dims* dims, const void* Q, const void* K, const void* V,
+                                const da_block_mask* mask, const void* centroids, const da_cluster_stats* stats,
+                                float scale, void* O, float* lse, void* ws, size_t ws_bytes, da_stream stream) {
+  Dims g;
+  StatsPtrs sp;
+  da_status st = attention_common(dims, mask, stats, ws, ws_bytes, &g, &sp);
+  if (st != DA_OK) return st;
+  return attention_launch(g, Q, K, V, mask, centroids, sp, scale, O, lse, ws, reinterpret_cast<cudaStream_t>(stream));
+}
+
+da_status da_attention(const da_dims* dims, const void* Q, const void* K, const void* V,
+                       const da_block_mask* mask, const void* centroids, const da_cluster_stats* stats,
+                       float scale, void* O, float* lse, void* ws, size_t ws_bytes, da_stream stream) {
+  Dims g;
+  StatsPtrs sp;
+  da_status st = attention_common(dims, mask, stats, ws, ws_bytes, &g, &sp);
+  if (st != DA_OK) return st;
+  if ((st = check_attention_ptrs(Q, K, V, centroids, O, lse)) != DA_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const cudaError_t e = compensation_launch(g, mask, sp, ws, s);
+  if (e != cudaSuccess) return cuda_status(e);
+  return attention_launch(g, Q, K, V, mask, centroids, sp, scale, O, lse, ws, s);
 }
 
 da_status da_device_status(void* ws, da_stream stream) {

@@ -161,6 +161,33 @@ DA_API da_status da_attention(const da_dims* dims, const void* Q, const void* K,
                        void* ws, size_t ws_bytes, da_stream stream);
 
 /*
+ * The two halves of da_attention, for callers that time or schedule them
+ * apart; da_attention(...) is da_compensation(...) followed by
+ * da_attention_prebuilt(...) with the same arguments.
+ *
+ * da_compensation: the per-q-block compensation statistics (DecoupAttn
+ * abstract: every key outside the fixed blocks is compensated through its
+ * cluster).  For every q-block i and cluster c it writes, into the workspace,
+ *   n^U_c = n_c - sum_{j in sel(i)} n_{c,j}   (as log2 n^U_c, -inf when 0)
+ *   vbar^U_c = (S_c - sum_{j in sel(i)} S_{c,j}) / n^U_c   (bf16),
+ * the fp32 subtraction summed in a fixed order.  bf16 inputs with d = 128 and
+ * block = 128 only; for other dims it launches nothing and returns DA_OK (the
+ * CUDA-core attention path forms these values itself).
+ *
+ * da_attention_prebuilt: the fused attention of da_attention, reading the
+ * compensation values da_compensation left in the same workspace.  Those
+ * values belong to the stats and mask they were built from: after
+ * da_reassign refreshes stats, or with another mask, call da_compensation
+ * again first.  Arguments, layouts and errors as in da_attention.
+ */
+DA_API da_status da_compensation(const da_dims* dims, const da_block_mask* mask, const da_cluster_stats* stats,
+                          void* ws, size_t ws_bytes, da_stream stream);
+DA_API da_status da_attention_prebuilt(const da_dims* dims, const void* Q, const void* K, const void* V,
+                                const da_block_mask* mask, const void* centroids,
+                                const da_cluster_stats* stats, float scale, void* O, float* lse,
+                                void* ws, size_t ws_bytes, da_stream stream);
+
+/*
  * Reassign Cache without a caller workspace (the paper has no counterpart: this is a calling
  * convention of this library).  Some callers cannot call cudaMalloc when they run a step: a
  * runtime whose device memory is planned once at start-up, a host application whose pool owns all

@@ -32,7 +32,7 @@ def test_every_declared_symbol_is_exported():
 
 
 def test_version_and_strings():
-    assert da.da_version() == 100
+    assert da.da_version() == 101
     for code in range(10):
         assert da.da_status_string(code) and da.da_status_string(code) != "unknown status"
 
@@ -103,3 +103,16 @@ def test_mask_prepare_rejects_small_schedule():
 
 def test_shape_overflow_rejected():
     assert _call_reassign(_dims(B=64, H=1024, N=1 << 20)) == 2
+
+
+def test_split_attention_calls_reject_arguments():
+    d = _dims()
+    st = da._Stats(*([0x1000] * 9))
+    m = da._Mask(0x1000, 0x1000, 4, None)
+    assert da._lib.da_compensation(ctypes.byref(d.c()), ctypes.byref(m), ctypes.byref(st), 0x1000, 0, None) == 9
+    assert da._lib.da_compensation(ctypes.byref(d.c()), ctypes.byref(da._Mask(None, 0x1000, 4, None)),
+                                   ctypes.byref(st), 0x1000, 1 << 30, None) == 1
+    assert da._lib.da_attention_prebuilt(ctypes.byref(d.c()), 0x1000, 0x1000, 0x1000, ctypes.byref(m), 0x1000,
+                                         ctypes.byref(st), 0.0, None, None, 0x1000, 1 << 30, None) == 1
+    assert da._lib.da_attention_prebuilt(ctypes.byref(d.c()), 0x1000, 0x1000, 0x1000, ctypes.byref(m), 0x1000,
+                                         ctypes.byref(st), 0.0, 0x1002, None, 0x1000, 1 << 30, None) == 4

@@ -140,6 +140,22 @@ def test_repeat_calls_are_bitwise_identical():
         assert torch.equal(v, getattr(eng.stats, k)), k
 
 
+def test_split_calls_equal_da_attention():
+    """da_compensation followed by da_attention_prebuilt is da_attention, bit for bit."""
+    import block_sparse_cluster_b200 as da
+    w = SMALL["wan14b_2f"]
+    inp = W.make_inputs(w, seed=17)
+    eng, O1, l1 = P.run_gpu(inp)
+    Q, K, V, cent = (x.cuda() for x in (inp.Q, inp.K, inp.V, inp.centroids))
+    O2 = torch.empty_like(O1)
+    l2 = torch.empty_like(l1)
+    da.da_compensation(eng.dims, eng.mask, eng.stats, eng.ws)
+    da.da_attention_prebuilt(eng.dims, Q, K, V, eng.mask, cent, eng.stats, 0.0, O2, l2, eng.ws)
+    torch.cuda.synchronize()
+    assert eng.status() == 0
+    assert torch.equal(O1, O2) and torch.equal(l1, l2)
+
+
 def test_malformed_plan_is_reported_without_fault():
     import block_sparse_cluster_b200 as da
     w = SMALL["tiny"]
