@@ -215,6 +215,62 @@ def _config(w: W.Workload, args):
 
 
 # ---------------------------------------------------------------------------
+# Reassign-cache loop: the plan is prepared once and the keys drift from step to step; each step
+# reassigns them to the cached centroids.  Reported per step: the device time of reassign +
+# attention, and the error against dense attention with the cached centroids and with fresh ones
+# (20 GPU Lloyd iterations on that step's keys, untimed), with both k-means objectives.
+
+def run_loop(args):
+    import block_sparse_cluster_b200 as da
+    import torch.nn.functional as F
+
+    w = W.WORKLOADS["loop"]
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    dims = da.Dims(w.B, w.H, w.N, w.d, w.C, w.block, w.torch_dtype)
+    eng = da.DecoupledAttention(dims, dev)
+    fresh = da.DecoupledAttention(dims, dev)
+    rows = []
+    for step in range(w.steps):
+        inp = W.make_inputs(w, seed=args.seed, step=step)
+        Q, K, V, cent = (x.to(dev) for x in (inp.Q, inp.K, inp.V, inp.centroids))
+        if step == 0:
+            eng.prepare(inp.kv_idx.to(dev), inp.kv_cnt.to(dev))     # the plan is fixed across steps
+            fresh.mask = eng.mask
+        O = torch.empty_like(Q)
+        for _ in range(max(3, args.warmup)):
+            eng.step(Q, K, V, cent, O)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        eng.step(Q, K, V, cent, O)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = e0.elapsed_time(e1)
+        a_cached = eng.stats.assign.long()
+        # fresh clusters for comparison: Lloyd from the cached centroids on this step's keys
+        cent_f = cent.clone()
+        da.kmeans(dims, K, cent_f, 20, fresh.stats, fresh.ws)
+        O_f = torch.empty_like(Q)
+        fresh.step(Q, K, V, cent_f, O_f)
+        from torch.nn.attention import SDPBackend, sdpa_kernel
+        with sdpa_kernel(SDPBackend.EFFICIENT_ATTENTION):           # fp32, no score matrix in memory
+            dense = F.scaled_dot_product_attention(Q.float(), K.float(), V.float())
+        nrm = dense.norm()
+
+        def obj(c, a):
+            return float(((K.float() - torch.gather(c.float(), 2, a[..., None].expand(-1, -1, -1, w.d))) ** 2).sum())
+
+        rows.append({"step": step, "ms": ms, "err_cached": float((O.float() - dense).norm() / nrm),
+                     "err_fresh": float((O_f.float() - dense).norm() / nrm),
+                     "sse_cached": obj(cent, a_cached), "sse_fresh": obj(cent_f, fresh.stats.assign.long())})
+    if eng.status() != 0 or fresh.status() != 0:
+        raise RuntimeError("device status after the loop")
+    print(json.dumps({"metric": "reassign-cache loop: ms per step (reassign + attention) and drift error",
+                      "workload": f"{w.name}: B={w.B} H={w.H} N={w.N} d={w.d} C={w.C} steps={w.steps} "
+                                  f"drift={w.drift} per-head density in {list(w.density_range)}",
+                      "data": "synthetic", "steps": rows}), flush=True)
+
 
 def main():
     ap = argparse.ArgumentParser()
@@ -230,7 +286,11 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--heads", type=int, default=0, help="override the head count (profiling runs)")
+    ap.add_argument("--loop", action="store_true", help="run the reassign-cache loop workload instead")
     args = ap.parse_args()
+    if args.loop:
+        run_loop(args)
+        return
     ws, rank, local = _dist()
     w = W.WORKLOADS[args.workload]
     if args.heads > 0:

@@ -28,7 +28,7 @@ STATUS_NAMES = ["DA_OK", "DA_ERR_INVALID_ARG", "DA_ERR_SHAPE", "DA_ERR_DTYPE", "
                 "DA_ERR_WORKSPACE"]
 EXPORTS = ["da_version", "da_workspace_bytes", "da_schedule_bytes", "da_reassign", "da_mask_prepare",
            "da_attention", "da_device_status", "da_status_string", "da_reassign_noalloc", "da_compensation",
-           "da_attention_prebuilt"]
+           "da_attention_prebuilt", "da_centroid_update"]
 
 
 class DAError(RuntimeError):
@@ -72,6 +72,8 @@ _lib.da_attention_prebuilt.argtypes = _lib.da_attention.argtypes
 _lib.da_compensation.restype = ctypes.c_int
 _lib.da_compensation.argtypes = [ctypes.POINTER(_Dims), ctypes.POINTER(_Mask), ctypes.POINTER(_Stats), _P,
                                  ctypes.c_size_t, _P]
+_lib.da_centroid_update.restype = ctypes.c_int
+_lib.da_centroid_update.argtypes = [ctypes.POINTER(_Dims), ctypes.POINTER(_Stats), _P, _P]
 _lib.da_reassign_noalloc.restype = ctypes.c_int
 _lib.da_reassign_noalloc.argtypes = [ctypes.POINTER(_Dims), _P, _P, _P, ctypes.POINTER(_Stats), _P]
 _lib.da_device_status.restype = ctypes.c_int
@@ -226,6 +228,24 @@ def da_attention_prebuilt(dims: Dims, Q: torch.Tensor, K: torch.Tensor, V: torch
                                       float(scale), O.data_ptr(), lse.data_ptr() if lse is not None else None,
                                       ws.data_ptr(), ws.numel(), _stream(stream)), "da_attention_prebuilt")
     return O
+
+
+def da_centroid_update(dims: Dims, stats: ClusterStats, centroids: torch.Tensor, stream=None) -> torch.Tensor:
+    """Lloyd update: centroids <- S_c / n_c from stats taken with the keys as the values."""
+    _check(_lib.da_centroid_update(ctypes.byref(dims.c()), ctypes.byref(stats.c()), centroids.data_ptr(),
+                                   _stream(stream)), "da_centroid_update")
+    return centroids
+
+
+def kmeans(dims: Dims, K: torch.Tensor, centroids: torch.Tensor, iters: int, stats: ClusterStats,
+           ws: torch.Tensor, stream=None) -> torch.Tensor:
+    """`iters` Lloyd iterations on the GPU, updating `centroids` in place.  Each iteration is
+    da_reassign with the keys as the values (so S_c sums the keys of cluster c) followed by
+    da_centroid_update; `stats` holds the last iteration's assignment afterwards."""
+    for _ in range(iters):
+        da_reassign(dims, K, K, centroids, stats, ws, stream)
+        da_centroid_update(dims, stats, centroids, stream)
+    return centroids
 
 
 def da_device_status(ws: torch.Tensor, stream=None) -> int:

@@ -72,7 +72,7 @@ da_status cuda_status(cudaError_t e) { return e == cudaSuccess ? DA_OK : DA_ERR_
 
 extern "C" {
 
-int da_version(void) { return 101; }
+int da_version(void) { return 102; }
 
 size_t da_workspace_bytes(const da_dims* dims) {
   Dims g;
@@ -212,6 +212,18 @@ da_status da_attention(const da_dims* dims, const void* Q, const void* K, const 
   const cudaError_t e = compensation_launch(g, mask, sp, ws, s);
   if (e != cudaSuccess) return cuda_status(e);
   return attention_launch(g, Q, K, V, mask, centroids, sp, scale, O, lse, ws, s);
+}
+
+da_status da_centroid_update(const da_dims* dims, const da_cluster_stats* stats, void* centroids,
+                             da_stream stream) {
+  Dims g;
+  da_status st = check_dims(dims, &g);
+  if (st != DA_OK) return st;
+  if (!centroids) return DA_ERR_INVALID_ARG;
+  if (!aligned16(centroids)) return DA_ERR_ALIGNMENT;
+  StatsPtrs sp;
+  if ((st = check_stats(stats, &sp)) != DA_OK) return st;
+  return cuda_status(launch_centroid_update(g, sp, centroids, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 da_status da_device_status(void* ws, da_stream stream) {

@@ -35,6 +35,7 @@ WsLayout ws_layout(const Dims& g);
 cudaError_t launch_centroid_norms(const Dims& g, const void* cent, float* norms, cudaStream_t s);
 cudaError_t launch_block_stats(const Dims& g, const void* V, const StatsPtrs& st, cudaStream_t s);
 cudaError_t launch_totals(const Dims& g, const StatsPtrs& st, cudaStream_t s);
+cudaError_t launch_centroid_update(const Dims& g, const StatsPtrs& st, void* cent, cudaStream_t s);
 cudaError_t launch_schedule(const Dims& g, const int32_t* kv_idx, const int32_t* kv_cnt, int max_sel,
                             int32_t* schedule, int* status, cudaStream_t s);
 

@@ -6,6 +6,8 @@
 #include "da_common.cuh"
 #include "da_internal.h"
 
+#include <type_traits>
+
 namespace da {
 
 WsLayout ws_layout(const Dims& g) {
@@ -155,6 +157,32 @@ cudaError_t launch_block_stats(const Dims& g, const void* V, const StatsPtrs& st
     if (g.d == 128) DA_STATS(float, 128); else DA_STATS(float, 64);
   }
 #undef DA_STATS
+  return cudaGetLastError();
+}
+
+// Lloyd update (least-squares quantisation): centroid c <- S_c / n_c, where the totals were taken
+// with the keys as values; a centroid without keys stays where it is.  One thread per (row, column).
+template <typename T>
+__global__ void centroid_update_kernel(const float* __restrict__ S, const int32_t* __restrict__ n, T* cent,
+                                       long long rows, int d) {
+  const long long x = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (x >= rows * d) return;
+  const long long r = x / d;
+  const int cnt = n[r];
+  if (cnt <= 0) return;
+  const float v = S[x] / (float)cnt;
+  if constexpr (std::is_same<T, float>::value) cent[x] = v;
+  else cent[x] = __float2bfloat16_rn(v);
+}
+
+cudaError_t launch_centroid_update(const Dims& g, const StatsPtrs& st, void* cent, cudaStream_t s) {
+  const long long rows = (long long)g.B * g.H * g.C;
+  const long long total = rows * g.d;
+  const unsigned grid = (unsigned)((total + 255) / 256);
+  if (g.bf16)
+    centroid_update_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(st.S_tot, st.n_tot, (__nv_bfloat16*)cent, rows, g.d);
+  else
+    centroid_update_kernel<float><<<grid, 256, 0, s>>>(st.S_tot, st.n_tot, (float*)cent, rows, g.d);
   return cudaGetLastError();
 }
 

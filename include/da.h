@@ -188,6 +188,20 @@ DA_API da_status da_attention_prebuilt(const da_dims* dims, const void* Q, const
                                 void* ws, size_t ws_bytes, da_stream stream);
 
 /*
+ * Lloyd update step (the clustering the pages build on: "Least squares
+ * quantization in PCM", listed on the DecoupAttn paper page among the works it
+ * builds on).  With stats from da_reassign(dims, K, K, centroids, stats, ...)
+ * -- the keys passed as the values, so S_c is the sum of the keys assigned to
+ * centroid c -- this moves every centroid to the mean of its keys:
+ * centroids[b,h,c,:] = S_c / n_c, rounded to the dims' dtype; a centroid with
+ * n_c = 0 is left unchanged.  One da_reassign + da_centroid_update pair is one
+ * Lloyd iteration (initial clustering, or a refresh of the cached centroids).
+ * centroids: [B,H,C,d] device, updated in place.  Same errors as da_reassign.
+ */
+DA_API da_status da_centroid_update(const da_dims* dims, const da_cluster_stats* stats, void* centroids,
+                             da_stream stream);
+
+/*
  * Reassign Cache without a caller workspace (the paper has no counterpart: this is a calling
  * convention of this library).  Some callers cannot call cudaMalloc when they run a step: a
  * runtime whose device memory is planned once at start-up, a host application whose pool owns all

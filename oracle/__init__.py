@@ -52,7 +52,7 @@ import numpy as np
 
 __all__ = [
     "reassign", "block_ranges", "block_histogram", "block_entries", "cluster_totals",
-    "complement_stats", "attention_qblock", "attention",
+    "complement_stats", "attention_qblock", "attention", "lloyd_step", "kmeans", "sse",
 ]
 
 
@@ -226,3 +226,39 @@ def attention(Q, K, V, centroids, plan: Sequence[Sequence[int]], assign, block: 
         s, e = rng[i]
         out[s:e] = attention_qblock(Qf, K, V, centroids, plan[i], assign, i, block, scale)
     return out
+
+
+# ---------------------------------------------------------------------------------------------
+# Lloyd's algorithm (the clustering the pages build on: "Least squares quantization in PCM"), used
+# for the initial centroids and for the comparison with fresh clusters in the reassign-cache loop.
+
+def sse(K, centroids, assign) -> float:
+    """Sum of squared distances of every key to its assigned centroid (the k-means objective)."""
+    Kf, Cf = _f64(K), _f64(centroids)
+    a = _i64(assign)
+    return float(((Kf - Cf[a]) ** 2).sum())
+
+
+def lloyd_step(K, centroids) -> Tuple[np.ndarray, np.ndarray]:
+    """One Lloyd iteration: assign every key to its nearest centroid (reassign, reading R1), then
+    move each centroid to the mean of its keys; a centroid without keys stays where it is.
+    Returns (new centroids float64 [C, d], assignment int64 [N])."""
+    Kf, Cf = _f64(K), _f64(centroids)
+    a, _ = reassign(Kf, Cf)
+    C = Cf.shape[0]
+    n = np.bincount(a, minlength=C)
+    S = np.zeros_like(Cf)
+    np.add.at(S, a, Kf)
+    new = Cf.copy()
+    live = n > 0
+    new[live] = S[live] / n[live][:, None]
+    return new, a
+
+
+def kmeans(K, init, iters: int) -> Tuple[np.ndarray, np.ndarray]:
+    """`iters` Lloyd iterations from `init`; returns (centroids, assignment of the last step)."""
+    c = _f64(init)
+    a = None
+    for _ in range(iters):
+        c, a = lloyd_step(K, c)
+    return c, a

@@ -32,7 +32,7 @@ def test_every_declared_symbol_is_exported():
 
 
 def test_version_and_strings():
-    assert da.da_version() == 101
+    assert da.da_version() == 102
     for code in range(10):
         assert da.da_status_string(code) and da.da_status_string(code) != "unknown status"
 
@@ -116,3 +116,12 @@ def test_split_attention_calls_reject_arguments():
                                          ctypes.byref(st), 0.0, None, None, 0x1000, 1 << 30, None) == 1
     assert da._lib.da_attention_prebuilt(ctypes.byref(d.c()), 0x1000, 0x1000, 0x1000, ctypes.byref(m), 0x1000,
                                          ctypes.byref(st), 0.0, 0x1002, None, 0x1000, 1 << 30, None) == 4
+
+
+def test_centroid_update_rejects_arguments():
+    d = _dims()
+    st = da._Stats(*([0x1000] * 9))
+    assert da._lib.da_centroid_update(ctypes.byref(d.c()), ctypes.byref(st), None, None) == 1
+    assert da._lib.da_centroid_update(ctypes.byref(d.c()), ctypes.byref(st), 0x1004, None) == 4
+    bad = da._Stats(*([0x1000] * 7 + [0x1004, 0x1000]))
+    assert da._lib.da_centroid_update(ctypes.byref(d.c()), ctypes.byref(bad), 0x1000, None) == 4
