@@ -55,3 +55,8 @@ def test_objective_never_increases():
         assert cur <= prev + 1e-9
         prev = cur
         c, _ = oracle.lloyd_step(K, c)
+
+
+def test_objective_hand_value():
+    # keys (0, 0) and (3, 4) on one centroid at the origin: 0 + 3^2 + 4^2 = 25
+    assert oracle.sse(np.array([[0.0, 0.0], [3.0, 4.0]]), np.array([[0.0, 0.0]]), np.array([0, 0])) == 25.0

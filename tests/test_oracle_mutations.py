@@ -10,6 +10,7 @@ import types
 import pytest
 
 import oracle
+from tests import test_oracle_lloyd as lloyd_pins
 from tests import test_oracle_pins as pins
 
 MUTATIONS = {
@@ -32,6 +33,10 @@ MUTATIONS = {
     "centroid term missing from denominator": ("den = pe.sum(axis=1) + pl.sum(axis=1)", "den = pe.sum(axis=1)"),
     "exact term missing from numerator": ("num = pe @ Vf[in_sel] + pl @ vbar[live]", "num = pl @ vbar[live]"),
     "values of the wrong keys": ("num = pe @ Vf[in_sel]", "num = pe @ Vf[in_sel][::-1]"),
+    "Lloyd: sum instead of mean": ("new[live] = S[live] / n[live][:, None]", "new[live] = S[live]"),
+    "Lloyd: empty cluster sent to the origin": ("new = Cf.copy()", "new = np.zeros_like(Cf)"),
+    "Lloyd: mean of the wrong keys": ("np.add.at(S, a, Kf)", "np.add.at(S, a, Kf[::-1])"),
+    "k-means objective without the square": ("((Kf - Cf[a]) ** 2).sum()", "np.abs(Kf - Cf[a]).sum()"),
 }
 
 PINS = [
@@ -49,6 +54,12 @@ PINS = [
     (pins.test_zero_queries_give_mean_value_for_any_plan, {}),
     (pins.test_per_key_correction_form, {}),
     (pins.test_brute_force_tiny, {}),
+    (lloyd_pins.test_hand_example_one_step, {}),
+    (lloyd_pins.test_matches_scikit_learn_lloyd, {}),
+    (lloyd_pins.test_means_are_a_fixed_point, {}),
+    (lloyd_pins.test_empty_cluster_keeps_its_centroid, {}),
+    (lloyd_pins.test_objective_never_increases, {}),
+    (lloyd_pins.test_objective_hand_value, {}),
 ]
 
 
@@ -65,6 +76,7 @@ def test_pins_catch_planted_mistake(name, monkeypatch):
     old, new = MUTATIONS[name]
     mutant = _mutant(old, new)
     monkeypatch.setattr(pins, "oracle", mutant)
+    monkeypatch.setattr(lloyd_pins, "oracle", mutant)
     caught = []
     for fn, kw in PINS:
         try:
