@@ -11,7 +11,8 @@
 //      every c and is dropped).
 //   4. The same 128 threads refresh the block's statistics (block_stats.cuh): sorted entry list,
 //      histogram row, entry index row and fp32 value sums, reading the block's value rows from
-//      shared memory (copied with cp.async into the centroid buffer, free once the last MMA is done).
+//      shared memory (copied with cp.async into centroid buffer 0 once the last MMA reading it is
+//      done, overlapping the remaining epilogues).
 // The CTA takes about 109 KB of shared memory and 256 TMEM columns, so two CTAs share an SM and
 // one's contraction overlaps the other's argmin and statistics.
 #include "block_stats.cuh"
@@ -128,6 +129,14 @@ reassign_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     if (t == 0 && c + 1 < nchunks && !*abort) issue_mma(c + 1);
     const bool ok = __all_sync(0xffffffffu, mbar_wait(&bars->mdone[c & 1], (c >> 1) & 1, abort, status));
     tc_fence_after();
+    // MMA(c) is done, so its centroid buffer is free: the next chunk for it loads during this epilogue
+    if (t == 0 && c + 2 < nchunks && !*abort) load_chunk(c + 2);
+    // buffer 0 after its last chunk: the block's value rows for the statistics
+    if ((c & 1) == 0 && c + 2 >= nchunks && ok) {
+      const __nv_bfloat16* Vg = V + ((size_t)bh * N + k0) * kD;
+      for (int i = t; i < nk * kD / 8; i += 128) cp_async16(sC0 + (size_t)i * 16, Vg + (size_t)i * 8);
+      cp_async_commit();
+    }
     const int n = ok ? min(kChunk, C - c * kChunk) : 0;
     for (int col = 0; col < n; col += 32) {
       uint32_t r[32];
@@ -152,15 +161,10 @@ reassign_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (t == 0 && c + 2 < nchunks && !*abort) load_chunk(c + 2);
   }
   __syncthreads();
 
   if (!*abort) {
-    // every MMA has completed (the last chunk's mdone was waited): the centroid buffer is free
-    const __nv_bfloat16* Vg = V + ((size_t)bh * N + k0) * kD;
-    for (int i = t; i < nk * kD / 8; i += 128) cp_async16(sC0 + (size_t)i * 16, Vg + (size_t)i * 8);
-    cp_async_commit();
     if (t < nk) {
       s_assign[t] = arg;
       st.assign[(size_t)bh * N + k0 + t] = arg;
