@@ -23,6 +23,8 @@ SMALL = {
     "wan14b_2f": W.scaled(W.WORKLOADS["wan14b"], H=2, T=2),
     # bf16 HunyuanVideo shape cut to 3 frames: N = 10800, 85 blocks, last one 48 keys, C=1024
     "hunyuan_3f": W.scaled(W.WORKLOADS["hunyuan"], H=1, T=3),
+    # two batch entries: (batch, head) slices are flattened in every kernel
+    "wan13b_b2": W.scaled(W.WORKLOADS["wan13b"], B=2, H=2, T=2),
 }
 
 
@@ -41,6 +43,24 @@ def test_small_case_full_parity(name):
             P.check_block_stats(inp, b, h, st, a)
             P.check_totals(inp, b, h, st, a)
             P.check_attention(inp, b, h, O, lse, a)
+
+
+def test_drifted_keys_with_the_step0_plan():
+    """Reassign-cache loop: step 3 of drifting keys, the plan prepared once from step 0 and the
+    cached step-0 centroids; full parity on the drifted step."""
+    w = W.scaled(W.WORKLOADS["loop"], H=2, T=3)
+    inp0 = W.make_inputs(w, seed=31, step=0)
+    inp = W.make_inputs(w, seed=31, step=3)
+    assert torch.equal(inp.kv_idx, inp0.kv_idx) and not torch.equal(inp.K, inp0.K)
+    eng, O, lse = P.run_gpu(inp)
+    assert eng.status() == 0
+    assign = eng.stats.assign.cpu().numpy()
+    for h in range(w.H):
+        a = assign[0, h].astype(np.int64)
+        P.check_assignment(inp, 0, h, a)
+        P.check_block_stats(inp, 0, h, eng.stats, a)
+        P.check_totals(inp, 0, h, eng.stats, a)
+        P.check_attention(inp, 0, h, O, lse, a)
 
 
 def _edge_plan(w, rows):
