@@ -281,6 +281,7 @@ def main():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-groups", type=int, default=8, help="head groups pipelined in the end-to-end leg")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--ref-items", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -372,27 +373,66 @@ def main():
     del flush
     median_ms = _max_over_ranks(median_ms_local, ws, dev)
 
-    # end to end through the same public calls: pinned host inputs in, O back to the host
+    # End to end through the same public calls: pinned host inputs in, O back to the host.  The
+    # heads go in groups on three streams, so that group g+1's inputs cross PCIe while group g
+    # computes and group g-1's output returns (each group is a head slice with its own buffers).
     e2e = None
     if not args.no_e2e:
+        groups = max(d for d in range(1, min(args.e2e_groups, w.H) + 1) if w.H % d == 0) if w.B == 1 else 1
+        hg = w.H // groups
+        gdims = da.Dims(w.B, hg, w.N, w.d, w.C, w.block, w.torch_dtype)
+        sl = lambda t, g: t[:, g * hg:(g + 1) * hg]
+        engs = []
+        for g in range(groups):
+            e = da.DecoupledAttention(gdims, dev)
+            e.prepare(sl(inp.kv_idx, g).contiguous().to(dev), sl(inp.kv_cnt, g).contiguous().to(dev))
+            engs.append(e)
         pinned = [x.pin_memory() for x in (inp.Q, inp.K, inp.V, inp.centroids)]
         O_host = torch.empty(O.shape, dtype=O.dtype, pin_memory=True)
         h2d = sum(x.numel() * x.element_size() for x in pinned)
         d2h = O_host.numel() * O_host.element_size()
+        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev_in = [torch.cuda.Event() for _ in range(groups)]
+        ev_done = [torch.cuda.Event() for _ in range(groups)]
+        ev_out = [torch.cuda.Event() for _ in range(groups)]
+        dev_bufs = (Q, K, V, cent)
+
+        def e2e_step(first):
+            for g in range(groups):
+                if not first:
+                    s_in.wait_event(ev_done[g])            # the group's inputs are free again
+                with torch.cuda.stream(s_in):
+                    for dst, src in zip(dev_bufs, pinned):
+                        sl(dst, g).copy_(sl(src, g), non_blocking=True)
+                ev_in[g].record(s_in)
+                stream.wait_event(ev_in[g])
+                if not first:
+                    stream.wait_event(ev_out[g])            # the group's output has left the GPU
+                engs[g].step(sl(Q, g), sl(K, g), sl(V, g), sl(cent, g), sl(O, g), stream=stream)
+                ev_done[g].record(stream)
+                s_out.wait_event(ev_done[g])
+                with torch.cuda.stream(s_out):
+                    sl(O_host, g).copy_(sl(O, g), non_blocking=True)
+                ev_out[g].record(s_out)
+
+        e2e_step(True)                                  # untimed warm-up of the three streams
+        torch.cuda.synchronize(dev)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         _barrier(ws)
         torch.cuda.synchronize(dev)
         e0.record(stream)
-        for _ in range(args.e2e_steps):
-            for dst, src in zip((Q, K, V, cent), pinned):
-                dst.copy_(src, non_blocking=True)
-            eng.step(Q, K, V, cent, O)
-            O_host.copy_(O, non_blocking=True)
+        s_in.wait_stream(stream)
+        for k in range(args.e2e_steps):
+            e2e_step(False)
+        stream.wait_stream(s_out)
         e1.record(stream)
         torch.cuda.synchronize(dev)
+        for e in engs:
+            if e.status() != 0:
+                raise RuntimeError("device status after the end-to-end steps")
         e2e_ms = _max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, ws, dev)
         e2e = {"value": ws * eff / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "head_groups": groups}
 
     if rank == 0:
         peaks, kind = _peaks()
