@@ -249,7 +249,7 @@ const char* da_status_string(da_status s) {
     case DA_ERR_SHAPE: return "inconsistent or too large shape";
     case DA_ERR_DTYPE: return "unknown dtype";
     case DA_ERR_ALIGNMENT: return "tensor base pointer not 16-byte aligned";
-    case DA_ERR_UNSUPPORTED: return "sizes not supported by this build (d, block or C)";
+    case DA_ERR_UNSUPPORTED: return "sizes not supported by this library (d, block or C)";
     case DA_ERR_CUDA: return "CUDA runtime or driver call failed";
     case DA_ERR_TIMEOUT: return "a bounded device wait gave up";
     case DA_ERR_DEVICE_INDEX: return "malformed block plan seen on the device";

@@ -54,7 +54,7 @@ typedef enum {
   DA_ERR_SHAPE = 2,         /* sizes that contradict each other (max_sel < 1, ...) */
   DA_ERR_DTYPE = 3,         /* dtype not one of da_dtype */
   DA_ERR_ALIGNMENT = 4,     /* a tensor base pointer is not 16-byte aligned */
-  DA_ERR_UNSUPPORTED = 5,   /* valid sizes this build has no kernel for (d, block, C) */
+  DA_ERR_UNSUPPORTED = 5,   /* valid sizes this library has no kernel for (d, block, C) */
   DA_ERR_CUDA = 6,          /* a CUDA runtime or driver call failed (launch, tensor map) */
   DA_ERR_TIMEOUT = 7,       /* a bounded device-side wait gave up (from da_device_status) */
   DA_ERR_DEVICE_INDEX = 8,  /* the device found a block index out of range, unsorted or repeated,
