@@ -5,8 +5,8 @@
 //   n^U_c    = n_c - sum_{j in sel} n_{c,j}                      (keys of c outside sel(i))
 //   vbar^U_c = (S_c - sum_{j in sel} S_{c,j}) / n^U_c            (their mean value, fp32 -> bf16)
 //   beta_c   = log2 n^U_c  (-inf when n^U_c = 0)                 (the count weight, log2 units)
-// One CTA per (item, 128-cluster chunk) writes the chunk as 128 bf16 rows of d = 128 (the layout a
-// TMA tile load reads) followed by the 128 fp32 beta values.
+// One CTA per (item, 128-cluster chunk), in chunk-major order, writes the chunk as 128 bf16 rows
+// of d = 128 (the layout a TMA tile load reads) followed by the 128 fp32 beta values.
 //
 // Phase 1: thread (row, h) looks the row up in half h of the selected blocks (seg_idx: the entry
 // of the cluster in the block, or 0xFF) with batches of independent loads, keeping the first
@@ -41,8 +41,11 @@ __global__ void __launch_bounds__(kThreads, 5)
 comp_build_kernel(StatsPtrs st, const int32_t* __restrict__ kv_idx, const int32_t* __restrict__ kv_cnt,
                   int max_sel, int N, int C, int nB, int block, int nchunk, uint8_t* __restrict__ out) {
   __shared__ Smem sm;
-  const int item = blockIdx.x / nchunk;
-  const int c = blockIdx.x - item * nchunk;
+  // chunk-major order: the CTAs resident at one time share the chunk, so its S_c rows and the
+  // blocks' lookup rows are served from L1
+  const int n_items = gridDim.x / nchunk;
+  const int c = blockIdx.x / n_items;
+  const int item = blockIdx.x - c * n_items;
   const int bh = item / nB;
   const int t = threadIdx.x;
   int nsel = kv_cnt[item];
@@ -50,7 +53,7 @@ comp_build_kernel(StatsPtrs st, const int32_t* __restrict__ kv_idx, const int32_
   const int32_t* row = kv_idx + (size_t)item * max_sel;
   const size_t hb = (size_t)bh * nB;                   // first block row of the head
   const size_t hc = (size_t)bh * C;                    // first cluster row of the head
-  uint8_t* chunk = out + (size_t)blockIdx.x * kChunkBytes;
+  uint8_t* chunk = out + ((size_t)item * nchunk + c) * kChunkBytes;
 
   {
     const int rr = t & (kRows - 1), h = t / kRows;
