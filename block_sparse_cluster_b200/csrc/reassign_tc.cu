@@ -29,7 +29,7 @@ constexpr int kD = 128;              // head dimension
 constexpr int kChunk = 128;          // centroids per MMA chunk (N of the MMA)
 constexpr int kMaxC = 1024;          // centroid norms staged in shared memory
 constexpr int kKTileBytes = kKeys * kD * 2;        // 32 KB
-constexpr int kCTileBytes = kChunk * kD * 2;       // 64 KB
+constexpr int kCTileBytes = kChunk * kD * 2;       // 32 KB
 constexpr int kPanelK = kKeys * 128;               // one 64-column panel of the key tile
 constexpr int kPanelC = kChunk * 128;              // one 64-column panel of a centroid chunk
 
@@ -122,8 +122,15 @@ reassign_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     if (mbar_wait(&bars->kfull, 0, abort, status)) issue_mma(0);
   }
 
-  float best = INFINITY;
-  int arg = 0;
+  // eight running minima over disjoint column groups (shorter dependency chains), merged at the
+  // end; each visits its columns in ascending c and keeps the first of equal distances
+  float best[8];
+  int arg[8];
+#pragma unroll
+  for (int a = 0; a < 8; ++a) {
+    best[a] = INFINITY;
+    arg[a] = 0;
+  }
   const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
   for (int c = 0; c < nchunks; ++c) {
     if (t == 0 && c + 1 < nchunks && !*abort) issue_mma(c + 1);
@@ -137,24 +144,35 @@ reassign_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
       for (int i = t; i < nk * kD / 8; i += 128) cp_async16(sC0 + (size_t)i * 16, Vg + (size_t)i * 8);
       cp_async_commit();
     }
-    const int n = ok ? min(kChunk, C - c * kChunk) : 0;
-    for (int col = 0; col < n; col += 32) {
-      uint32_t r[32];
-      tmem_ld32(lane_base + (c & 1) * kChunk + col, r);
+    // C is a multiple of 32: the chunk has n / 32 full groups of 32 columns
+    const int ngroups = ok ? min(kChunk, C - c * kChunk) >> 5 : 0;
+    if (ngroups > 0) {
+      uint32_t r[4][32];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) tmem_ld32(lane_base + (c & 1) * kChunk + 32 * q, r[q]);
       tmem_wait_ld();
-      const float4* nv = reinterpret_cast<const float4*>(s_norm + c * kChunk + col);
+      const float4* nv = reinterpret_cast<const float4*>(s_norm + c * kChunk);
 #pragma unroll
-      for (int q4 = 0; q4 < 8; ++q4) {
-        const float4 nn = nv[q4];
-        const float nq[4] = {nn.x, nn.y, nn.z, nn.w};
+      for (int q = 0; q < 4; ++q) {
+        if (q < ngroups) {                            // warp-uniform
+          int loc[2] = {-1, -1};                      // column (in the chunk) of a new minimum
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int q = 4 * q4 + u;
-          const float dist = fmaf(-2.f, __uint_as_float(r[q]), nq[u]);
-          if (col + q < n && dist < best) {   // ascending c: ties keep the lowest index
-            best = dist;
-            arg = c * kChunk + col + q;
+          for (int q4 = 0; q4 < 8; ++q4) {
+            const float4 nn = nv[8 * q + q4];
+            const float nq[4] = {nn.x, nn.y, nn.z, nn.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int h = q4 >> 2;
+              const float dist = fmaf(-2.f, __uint_as_float(r[q][4 * q4 + u]), nq[u]);
+              if (dist < best[2 * q + h]) {
+                best[2 * q + h] = dist;
+                loc[h] = 32 * q + 4 * q4 + u;
+              }
+            }
           }
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            if (loc[h] >= 0) arg[2 * q + h] = c * kChunk + loc[h];
         }
       }
     }
@@ -164,10 +182,20 @@ reassign_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
   }
   __syncthreads();
 
+  // merge: the smallest distance, the lowest cluster among equal ones
+  float bd = best[0];
+  int ba = arg[0];
+#pragma unroll
+  for (int a = 1; a < 8; ++a) {
+    if (best[a] < bd || (best[a] == bd && arg[a] < ba)) {
+      bd = best[a];
+      ba = arg[a];
+    }
+  }
   if (!*abort) {
     if (t < nk) {
-      s_assign[t] = arg;
-      st.assign[(size_t)bh * N + k0 + t] = arg;
+      s_assign[t] = ba;
+      st.assign[(size_t)bh * N + k0 + t] = ba;
     }
     cp_async_wait<0>();
     __syncthreads();
