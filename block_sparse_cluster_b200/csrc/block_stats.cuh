@@ -18,17 +18,19 @@ namespace da {
 struct StatsSmem {
   int sorted_key[128];     // the block's keys ranked by (cluster, key index)
   int start_pos[132];      // first rank of each entry; start_pos[E] = nk
-  int scan_c[4], scan_f[4];
+  int scan_c[8], scan_f[8];
   int hist_row[1024];      // n_{c,j}; then, for a cluster present in the block, its first rank
   uint8_t idx_row[1024];
 };
 
-// Synchronise the 128 threads of named barrier `bar_id` (1..15).
+// Synchronise the NT threads of named barrier `bar_id` (1..15).
+template <int NT>
 __device__ __forceinline__ void group_sync(int bar_id) {
-  asm volatile("bar.sync %0, 128;" ::"r"(bar_id) : "memory");
+  asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "n"(NT) : "memory");
 }
 
-// t: thread index within the group (0..127); every thread of the group must call this.
+// t: thread index within the group of NT = 128 or 256 threads; every thread of the group must
+// call this.
 // s_assign: the block's clusters in shared memory (nk <= 128 entries, each in [0, C)).
 // Vblk: value rows of the block (row k at Vblk + k*D).  Output pointers are already offset to
 // this block.
@@ -37,7 +39,7 @@ __device__ __forceinline__ void group_sync(int bar_id) {
 //      rank, without atomics.
 //   2. One scan over the clusters gives each present cluster its entry index and its first rank.
 //   3. A warp per entry sums the run's value rows in rank order, lanes over the columns.
-template <typename T, int D>
+template <typename T, int D, int NT = 128>
 __device__ void block_stats_group(int t, int bar_id, const int* s_assign, int nk, const T* __restrict__ Vblk,
                                   int C, int32_t* __restrict__ hist_out, uint8_t* __restrict__ idx_out,
                                   int32_t* __restrict__ segn_out, int32_t* __restrict__ segc_out,
@@ -45,12 +47,13 @@ __device__ void block_stats_group(int t, int bar_id, const int* s_assign, int nk
                                   StatsSmem& sm) {
   const int warp = t >> 5, lane = t & 31;
   const unsigned below = (1u << lane) - 1u;
-  const int a_t = t < nk ? s_assign[t] : C;          // C: no key
+  static_assert(NT == 128 || NT == 256, "a group of 4 or 8 warps");
+  const int a_t = t < nk ? s_assign[t] : C;          // C: no key (also every thread t >= 128)
   const unsigned peers = __match_any_sync(0xffffffffu, a_t);
   const int r_in = __popc(peers & below);
   const bool leader = (peers & below) == 0u;
-  for (int c = t; c < C; c += 128) sm.hist_row[c] = 0;
-  group_sync(bar_id);
+  for (int c = t; c < C; c += NT) sm.hist_row[c] = 0;
+  group_sync<NT>(bar_id);
   int before = 0;                                     // keys of the cluster in earlier warps
 #pragma unroll 1
   for (int w = 0; w < 4; ++w) {
@@ -58,12 +61,12 @@ __device__ void block_stats_group(int t, int bar_id, const int* s_assign, int nk
       before = sm.hist_row[a_t];
       sm.hist_row[a_t] = before + __popc(peers);
     }
-    group_sync(bar_id);
+    group_sync<NT>(bar_id);
   }
   before = __shfl_sync(0xffffffffu, before, __ffs(peers) - 1);
 
   // exclusive scan over the clusters of (count, present): thread t owns clusters [t*cp, t*cp + cp)
-  const int cp = (C + 127) >> 7;
+  const int cp = (C + NT - 1) / NT;
   const int c0 = t * cp;
   int cnt = 0, flg = 0;
   for (int i = 0; i < cp; ++i) {
@@ -88,10 +91,10 @@ __device__ void block_stats_group(int t, int bar_id, const int* s_assign, int nk
     sm.scan_c[warp] = ic;
     sm.scan_f[warp] = ifl;
   }
-  group_sync(bar_id);
+  group_sync<NT>(bar_id);
   int run_c = ic - cnt, run_f = ifl - flg, E = 0;
 #pragma unroll
-  for (int w = 0; w < 4; ++w) {
+  for (int w = 0; w < NT / 32; ++w) {
     run_c += w < warp ? sm.scan_c[w] : 0;
     run_f += w < warp ? sm.scan_f[w] : 0;
     E += sm.scan_f[w];
@@ -118,20 +121,20 @@ __device__ void block_stats_group(int t, int bar_id, const int* s_assign, int nk
     *segn_out = E;
     sm.start_pos[E] = nk;
   }
-  group_sync(bar_id);
+  group_sync<NT>(bar_id);
 
   if (t < nk) sm.sorted_key[sm.hist_row[a_t] + before + r_in] = t;
   {
     uint32_t* dst = reinterpret_cast<uint32_t*>(idx_out);
     const uint32_t* src = reinterpret_cast<const uint32_t*>(sm.idx_row);
-    for (int w4 = t; w4 < C / 4; w4 += 128) dst[w4] = src[w4];
+    for (int w4 = t; w4 < C / 4; w4 += NT) dst[w4] = src[w4];
   }
-  group_sync(bar_id);
+  group_sync<NT>(bar_id);
 
-  // value sums: warp w takes entries w, w + 4, ...; lane l holds columns [l*D/32, (l+1)*D/32);
+  // value sums: warp w takes entries w, w + NT/32, ...; lane l holds columns [l*D/32, (l+1)*D/32);
   // the run's keys are added in rank order, two rows in flight at a time
   constexpr int NE = D / 32;
-  for (int ee = warp; ee < E; ee += 4) {
+  for (int ee = warp; ee < E; ee += NT / 32) {
     const int p0 = sm.start_pos[ee], p1 = sm.start_pos[ee + 1];
     float acc[NE];
 #pragma unroll
@@ -161,7 +164,7 @@ __device__ void block_stats_group(int t, int bar_id, const int* s_assign, int nk
       for (int i = 0; i < NE; ++i) dst[i] = acc[i];
     }
   }
-  group_sync(bar_id);
+  group_sync<NT>(bar_id);
 }
 
 }  // namespace da

@@ -32,6 +32,7 @@ constexpr int kKTileBytes = kKeys * kD * 2;        // 32 KB
 constexpr int kCTileBytes = kChunk * kD * 2;       // 32 KB
 constexpr int kPanelK = kKeys * 128;               // one 64-column panel of the key tile
 constexpr int kPanelC = kChunk * 128;              // one 64-column panel of a centroid chunk
+constexpr int kThreads = 256;                      // two warpgroups: each half of every chunk's columns
 
 struct __align__(8) Bars {
   uint64_t kfull;
@@ -42,11 +43,11 @@ struct __align__(8) Bars {
 };
 
 constexpr size_t kSmemBytes = 1024 /*align slack*/ + kKTileBytes /*K*/ + 2 * kCTileBytes + kMaxC * 4 /*norms*/ +
-                              sizeof(StatsSmem) + 512 /*assign*/ + 128 /*bars*/;
+                              sizeof(StatsSmem) + 512 /*assign*/ + 1024 /*second half's minima*/ + 128 /*bars*/;
 static_assert(sizeof(Bars) <= 128, "barrier block");
 static_assert(2 * (kSmemBytes + 1024) <= 233472, "two CTAs per SM");
 
-__global__ void __launch_bounds__(128, 2)
+__global__ void __launch_bounds__(kThreads, 2)
 reassign_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_c,
                    const __nv_bfloat16* __restrict__ V, const float* __restrict__ norms, StatsPtrs st, int N,
                    int C, int nB, int* status) {
@@ -58,10 +59,14 @@ reassign_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
   float* s_norm = reinterpret_cast<float*>(sC0 + 2 * kCTileBytes);
   StatsSmem* ssm = reinterpret_cast<StatsSmem*>(s_norm + kMaxC);
   int* s_assign = reinterpret_cast<int*>(ssm + 1);
-  Bars* bars = reinterpret_cast<Bars*>(s_assign + 128);
+  float* s_hbest = reinterpret_cast<float*>(s_assign + 128);   // warpgroup 1's (distance, cluster)
+  int* s_harg = reinterpret_cast<int*>(s_hbest + 128);
+  Bars* bars = reinterpret_cast<Bars*>(s_harg + 128);
 
   const int t = threadIdx.x;
   const int warp = t >> 5;
+  const int half = t >> 7;                           // columns [64 half, 64 half + 64) of each chunk
+  const int row = t & 127;                           // key = TMEM lane
   const int j = blockIdx.x;
   const int bh = blockIdx.y;
   const int k0 = j * kKeys;
@@ -81,7 +86,7 @@ reassign_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     tmem_alloc(&bars->tmem_base, 2 * kChunk);
     tmem_relinquish();
   }
-  for (int c = t; c < C; c += 128) s_norm[c] = norms[(size_t)bh * C + c];
+  for (int c = t; c < C; c += kThreads) s_norm[c] = norms[(size_t)bh * C + c];
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -122,16 +127,16 @@ reassign_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     if (mbar_wait(&bars->kfull, 0, abort, status)) issue_mma(0);
   }
 
-  // eight running minima over disjoint column groups (shorter dependency chains), merged at the
-  // end; each visits its columns in ascending c and keeps the first of equal distances
-  float best[8];
-  int arg[8];
+  // four running minima per thread over disjoint groups of 16 columns (shorter dependency
+  // chains); each visits its columns in ascending c and keeps the first of equal distances
+  float best[4];
+  int arg[4];
 #pragma unroll
-  for (int a = 0; a < 8; ++a) {
+  for (int a = 0; a < 4; ++a) {
     best[a] = INFINITY;
     arg[a] = 0;
   }
-  const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+  const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
   for (int c = 0; c < nchunks; ++c) {
     if (t == 0 && c + 1 < nchunks && !*abort) issue_mma(c + 1);
     const bool ok = __all_sync(0xffffffffu, mbar_wait(&bars->mdone[c & 1], (c >> 1) & 1, abort, status));
@@ -141,20 +146,20 @@ reassign_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     // buffer 0 after its last chunk: the block's value rows for the statistics
     if ((c & 1) == 0 && c + 2 >= nchunks && ok) {
       const __nv_bfloat16* Vg = V + ((size_t)bh * N + k0) * kD;
-      for (int i = t; i < nk * kD / 8; i += 128) cp_async16(sC0 + (size_t)i * 16, Vg + (size_t)i * 8);
+      for (int i = t; i < nk * kD / 8; i += kThreads) cp_async16(sC0 + (size_t)i * 16, Vg + (size_t)i * 8);
       cp_async_commit();
     }
     // C is a multiple of 32: the chunk has n / 32 full groups of 32 columns
     const int ngroups = ok ? min(kChunk, C - c * kChunk) >> 5 : 0;
-    if (ngroups > 0) {
-      uint32_t r[4][32];
+    if (ngroups > 2 * half) {                         // warp-uniform
+      uint32_t r[2][32];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) tmem_ld32(lane_base + (c & 1) * kChunk + 32 * q, r[q]);
+      for (int q = 0; q < 2; ++q) tmem_ld32(lane_base + (c & 1) * kChunk + 64 * half + 32 * q, r[q]);
       tmem_wait_ld();
-      const float4* nv = reinterpret_cast<const float4*>(s_norm + c * kChunk);
+      const float4* nv = reinterpret_cast<const float4*>(s_norm + c * kChunk + 64 * half);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        if (q < ngroups) {                            // warp-uniform
+      for (int q = 0; q < 2; ++q) {
+        if (2 * half + q < ngroups) {                 // warp-uniform
           int loc[2] = {-1, -1};                      // column (in the chunk) of a new minimum
 #pragma unroll
           for (int q4 = 0; q4 < 8; ++q4) {
@@ -172,7 +177,7 @@ reassign_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
           }
 #pragma unroll
           for (int h = 0; h < 2; ++h)
-            if (loc[h] >= 0) arg[2 * q + h] = c * kChunk + loc[h];
+            if (loc[h] >= 0) arg[2 * q + h] = c * kChunk + 64 * half + loc[h];
         }
       }
     }
@@ -180,16 +185,28 @@ reassign_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     __syncthreads();
     tc_fence_after();
   }
-  __syncthreads();
-
-  // merge: the smallest distance, the lowest cluster among equal ones
+  // merge: the smallest distance, the lowest cluster among equal ones; warpgroup 1 hands its
+  // minimum to warpgroup 0 through shared memory
   float bd = best[0];
   int ba = arg[0];
 #pragma unroll
-  for (int a = 1; a < 8; ++a) {
+  for (int a = 1; a < 4; ++a) {
     if (best[a] < bd || (best[a] == bd && arg[a] < ba)) {
       bd = best[a];
       ba = arg[a];
+    }
+  }
+  if (half == 1) {
+    s_hbest[row] = bd;
+    s_harg[row] = ba;
+  }
+  __syncthreads();
+  if (half == 0) {
+    const float b1 = s_hbest[row];
+    const int a1 = s_harg[row];
+    if (b1 < bd || (b1 == bd && a1 < ba)) {
+      bd = b1;
+      ba = a1;
     }
   }
   if (!*abort) {
@@ -200,10 +217,10 @@ reassign_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     cp_async_wait<0>();
     __syncthreads();
     const size_t bj = (size_t)bh * nB + j;
-    block_stats_group<__nv_bfloat16, kD>(t, 1, s_assign, nk, reinterpret_cast<const __nv_bfloat16*>(sC0), C,
-                                         st.blk_hist + bj * C, st.seg_idx + bj * C, st.seg_n + bj,
-                                         st.seg_c + bj * kKeys, st.seg_cnt + bj * kKeys,
-                                         st.seg_vsum + bj * kKeys * kD, *ssm);
+    block_stats_group<__nv_bfloat16, kD, kThreads>(t, 1, s_assign, nk, reinterpret_cast<const __nv_bfloat16*>(sC0), C,
+                                                   st.blk_hist + bj * C, st.seg_idx + bj * C, st.seg_n + bj,
+                                                   st.seg_c + bj * kKeys, st.seg_cnt + bj * kKeys,
+                                                   st.seg_vsum + bj * kKeys * kD, *ssm);
   }
   tc_fence_before();
   __syncthreads();
@@ -227,7 +244,7 @@ cudaError_t launch_reassign_tc(const Dims& g, const void* K, const void* V, cons
                                        (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid(g.nB, (unsigned)BH);
-  reassign_tc_kernel<<<grid, 128, kSmemBytes, s>>>(tk, tc, static_cast<const __nv_bfloat16*>(V), norms, st, g.N,
+  reassign_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(tk, tc, static_cast<const __nv_bfloat16*>(V), norms, st, g.N,
                                                    g.C, g.nB, status);
   return cudaGetLastError();
 }
