@@ -58,16 +58,16 @@ __global__ void __launch_bounds__(128) block_stats_kernel(const T* __restrict__ 
 }
 
 // Per-head totals n_c, S_c = sum over blocks of the block entries, in a fixed order.
-// CTA (head, 32 clusters); warp w walks blocks j = w, w+4, ...; partial sums per warp are
-// combined in warp order.
+// A warp per (head, cluster): it walks the blocks in order, finds the cluster's entry through
+// seg_idx (eight blocks looked up at a time) and adds the entry row, lanes over the value columns
+// (coalesced rows; registers; blocks in order: deterministic bits).
 template <int D>
 __global__ void __launch_bounds__(128) totals_kernel(StatsPtrs st, int C, int block, int nB) {
-  // thread t: cluster c0 + t/4, value columns [(t%4) * D/4, (t%4+1) * D/4); the cluster's entries
-  // are summed over the blocks in block order (registers, a fixed order: deterministic bits)
-  constexpr int NS = D / 4;               // columns per thread
+  constexpr int NS = D / 32;              // columns per lane
   const int bh = blockIdx.x;
-  const int c = blockIdx.y * 32 + (threadIdx.x >> 2);
-  const int q = threadIdx.x & 3;
+  const int c = blockIdx.y * 4 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (c >= C) return;                     // (C is a multiple of 32)
   float acc[NS];
 #pragma unroll
   for (int i = 0; i < NS; ++i) acc[i] = 0.f;
@@ -80,24 +80,23 @@ __global__ void __launch_bounds__(128) totals_kernel(StatsPtrs st, int C, int bl
     for (int u = 0; u < kB; ++u) e[u] = j0 + u < nB ? (int)st.seg_idx[(hb + j0 + u) * C + c] : 0xFF;
 #pragma unroll
     for (int u = 0; u < kB; ++u) {
-      if (e[u] == 0xFF) continue;
+      if (e[u] == 0xFF) continue;         // warp-uniform
       const size_t row = (hb + j0 + u) * block + e[u];
-      if (q == 0) n += st.seg_cnt[row];
-      const float4* src = reinterpret_cast<const float4*>(st.seg_vsum + row * D + q * NS);
+      if (lane == 0) n += st.seg_cnt[row];
+      float y[NS];
+      load_vec(st.seg_vsum + row * D + lane * NS, y, NS);
 #pragma unroll
-      for (int i = 0; i < NS / 4; ++i) {
-        const float4 y = __ldg(src + i);
-        acc[4 * i] += y.x;
-        acc[4 * i + 1] += y.y;
-        acc[4 * i + 2] += y.z;
-        acc[4 * i + 3] += y.w;
-      }
+      for (int i = 0; i < NS; ++i) acc[i] += y[i];
     }
   }
-  float4* dst = reinterpret_cast<float4*>(st.S_tot + ((size_t)bh * C + c) * D + q * NS);
+  float* dst = st.S_tot + ((size_t)bh * C + c) * D + lane * NS;
+  if constexpr (NS == 4) {
+    *reinterpret_cast<float4*>(dst) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+  } else {
 #pragma unroll
-  for (int i = 0; i < NS / 4; ++i) dst[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
-  if (q == 0) st.n_tot[(size_t)bh * C + c] = n;
+    for (int i = 0; i < NS; ++i) dst[i] = acc[i];
+  }
+  if (lane == 0) st.n_tot[(size_t)bh * C + c] = n;
 }
 
 // Plan validation and work order: items of a head ordered by descending row length
@@ -187,7 +186,7 @@ cudaError_t launch_centroid_update(const Dims& g, const StatsPtrs& st, void* cen
 }
 
 cudaError_t launch_totals(const Dims& g, const StatsPtrs& st, cudaStream_t s) {
-  dim3 grid(g.B * g.H, g.C / 32);
+  dim3 grid(g.B * g.H, (g.C + 3) / 4);                  // 4 clusters (warps) per CTA
   if (g.d == 128) totals_kernel<128><<<grid, 128, 0, s>>>(st, g.C, g.block, g.nB);
   else totals_kernel<64><<<grid, 128, 0, s>>>(st, g.C, g.block, g.nB);
   return cudaGetLastError();
