@@ -34,6 +34,13 @@ Readings taken where the pages are silent (each is listed in the design notes):
 * R4 the cached centroid is used as given; it is not re-estimated from the
   keys assigned to it.
 * R5 scale s = 1/sqrt(d) unless given.
+* R6 (variance correction, optional) the pages' ESTRA abstract refines the
+  weights of the cluster representatives with "a variance-based correction"
+  and prints no formula.  Reading: the cluster's keys are treated as Gaussian
+  about the representative with a diagonal second moment D_c (per dimension,
+  the mean of (k_t - cbar_{c,t})^2 over all keys assigned to c), so that
+  mean_k exp(s q.k) = exp(s q.cbar_c + s^2/2 sum_t q_t^2 D_{c,t}) up to higher
+  cumulants; the cluster logit gains the term s^2/2 sum_t q_t^2 D_{c,t}.
 
 Parity status: reassignment, block statistics and attention are each pinned
 by tests that do not call this module's formulas again (library routines,
@@ -53,6 +60,7 @@ import numpy as np
 __all__ = [
     "reassign", "block_ranges", "block_histogram", "block_entries", "cluster_totals",
     "complement_stats", "attention_qblock", "attention", "lloyd_step", "kmeans", "sse",
+    "cluster_spread",
 ]
 
 
@@ -154,6 +162,22 @@ def cluster_totals(assign, V, C: int) -> Tuple[np.ndarray, np.ndarray]:
     return n, S
 
 
+def cluster_spread(K, centroids, assign, C: int) -> np.ndarray:
+    """Second moment of each cluster's keys about its representative (reading R6):
+    D[c, t] = mean over the keys k with a(k) = c of (k_t - cbar_{c,t})^2; zero for an empty
+    cluster.  float64 [C, d]."""
+    a = _i64(assign)
+    Kf = _f64(K)
+    Cf = _f64(centroids)
+    dev2 = (Kf - Cf[a]) ** 2
+    n = np.bincount(a, minlength=C).astype(np.float64)
+    tot = np.stack([np.bincount(a, weights=dev2[:, t], minlength=C) for t in range(Kf.shape[1])], axis=1)
+    D = np.zeros_like(tot)
+    nz = n > 0
+    D[nz] = tot[nz] / n[nz, None]
+    return D
+
+
 # ---------------------------------------------------------------------------
 # Decoupled attention for one q-block
 
@@ -177,13 +201,15 @@ def complement_stats(assign, V, C: int, in_sel: np.ndarray):
 
 
 def attention_qblock(Q, K, V, centroids, sel_blocks: Sequence[int], assign, i: int,
-                     block: int, scale: Optional[float] = None, return_lse: bool = False):
+                     block: int, scale: Optional[float] = None, return_lse: bool = False,
+                     spread=None):
     """Output rows of q-block i (DecoupAttn abstract: exact attention on the
     fixed blocks, every other key compensated through its cluster).
 
     Logits: s*q.k for keys in the selected blocks, s*q.cbar_c + ln n^U_c for
     the clusters with n^U_c > 0; one softmax over both; the clusters carry the
-    mean complement value vbar^U_c.
+    mean complement value vbar^U_c.  With `spread` (D of cluster_spread, reading
+    R6) each cluster logit gains s^2/2 sum_t q_t^2 D_{c,t}.
     """
     Qf = _f64(Q)
     Kf = _f64(K)
@@ -203,6 +229,8 @@ def attention_qblock(Q, K, V, centroids, sel_blocks: Sequence[int], assign, i: i
     q = Qf[qs:qe]
     ell = s * (q @ Kf[in_sel].T)                               # [nq, |Sel|]
     lam = s * (q @ Cf[live].T) + np.log(nU[live])[None, :]    # [nq, #live]
+    if spread is not None:
+        lam = lam + 0.5 * s * s * ((q * q) @ _f64(spread)[live].T)
     m = np.maximum(ell.max(axis=1, initial=-np.inf), lam.max(axis=1, initial=-np.inf))
     pe = np.exp(ell - m[:, None])
     pl = np.exp(lam - m[:, None])
@@ -215,7 +243,7 @@ def attention_qblock(Q, K, V, centroids, sel_blocks: Sequence[int], assign, i: i
 
 
 def attention(Q, K, V, centroids, plan: Sequence[Sequence[int]], assign, block: int,
-              scale: Optional[float] = None, q_blocks: Optional[Iterable[int]] = None):
+              scale: Optional[float] = None, q_blocks: Optional[Iterable[int]] = None, spread=None):
     """Output [N, d] of one head (rows of q-blocks not requested stay NaN)."""
     Qf = _f64(Q)
     N, d = Qf.shape
@@ -224,7 +252,7 @@ def attention(Q, K, V, centroids, plan: Sequence[Sequence[int]], assign, block: 
     qb = range(len(rng)) if q_blocks is None else q_blocks
     for i in qb:
         s, e = rng[i]
-        out[s:e] = attention_qblock(Qf, K, V, centroids, plan[i], assign, i, block, scale)
+        out[s:e] = attention_qblock(Qf, K, V, centroids, plan[i], assign, i, block, scale, spread=spread)
     return out
 
 

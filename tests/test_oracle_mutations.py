@@ -12,6 +12,7 @@ import pytest
 import oracle
 from tests import test_oracle_lloyd as lloyd_pins
 from tests import test_oracle_pins as pins
+from tests import test_oracle_spread as spread_pins
 
 MUTATIONS = {
     "wrong distance sign": ("diff = K[s:e, None, :] - Cn[None, :, :]", "diff = K[s:e, None, :] + Cn[None, :, :]"),
@@ -37,6 +38,11 @@ MUTATIONS = {
     "Lloyd: empty cluster sent to the origin": ("new = Cf.copy()", "new = np.zeros_like(Cf)"),
     "Lloyd: mean of the wrong keys": ("np.add.at(S, a, Kf)", "np.add.at(S, a, Kf[::-1])"),
     "k-means objective without the square": ("((Kf - Cf[a]) ** 2).sum()", "np.abs(Kf - Cf[a]).sum()"),
+    "spread: factor 1 instead of 1/2": ("lam = lam + 0.5 * s * s *", "lam = lam + 1.0 * s * s *"),
+    "spread: s instead of s^2": ("lam = lam + 0.5 * s * s *", "lam = lam + 0.5 * s *"),
+    "spread: wrong sign": ("lam = lam + 0.5 * s * s *", "lam = lam - 0.5 * s * s *"),
+    "spread about the mean of all keys": ("dev2 = (Kf - Cf[a]) ** 2", "dev2 = (Kf - Kf.mean(axis=0)) ** 2"),
+    "spread: sum instead of mean": ("D[nz] = tot[nz] / n[nz, None]", "D[nz] = tot[nz]"),
 }
 
 PINS = [
@@ -60,6 +66,8 @@ PINS = [
     (lloyd_pins.test_empty_cluster_keeps_its_centroid, {}),
     (lloyd_pins.test_objective_never_increases, {}),
     (lloyd_pins.test_objective_hand_value, {}),
+    (spread_pins.test_offset_keys_give_the_squared_offset, {}),
+    (spread_pins.test_corrected_logit_matches_the_cluster_log_sum_exp_to_fourth_order, {"seed": 0}),
 ]
 
 
@@ -77,6 +85,7 @@ def test_pins_catch_planted_mistake(name, monkeypatch):
     mutant = _mutant(old, new)
     monkeypatch.setattr(pins, "oracle", mutant)
     monkeypatch.setattr(lloyd_pins, "oracle", mutant)
+    monkeypatch.setattr(spread_pins, "oracle", mutant)
     caught = []
     for fn, kw in PINS:
         try:
