@@ -272,6 +272,59 @@ def run_loop(args):
                       "data": "synthetic", "steps": rows}), flush=True)
 
 
+def run_spread(args):
+    """The variance-corrected cluster logits (ESTRA abstract's correction, read as a diagonal
+    Gaussian about each representative): da_reassign + da_cluster_spread + da_attention_spread,
+    which runs on the CUDA cores.  One JSON line with the step time and its split."""
+    import block_sparse_cluster_b200 as da
+    w = W.WORKLOADS[args.workload]
+    if args.heads > 0:
+        w = W.scaled(w, H=args.heads)
+    dev = torch.device("cuda", 0)
+    inp = W.make_inputs(w, seed=args.seed)
+    dims = da.Dims(w.B, w.H, w.N, w.d, w.C, w.block, w.torch_dtype)
+    eff = W.effective_flops(w, inp.kv_cnt, inp.kv_idx)
+    eng = da.DecoupledAttention(dims, dev)
+    Q, K, V, cent = (x.to(dev) for x in (inp.Q, inp.K, inp.V, inp.centroids))
+    eng.prepare(inp.kv_idx.to(dev), inp.kv_cnt.to(dev))
+    O = torch.empty_like(Q)
+    spread = torch.empty(w.B, w.H, w.C, w.d, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(evs=None):
+        if evs is not None:
+            evs[0].record(stream)
+        da.da_reassign(dims, K, V, cent, eng.stats, eng.ws)
+        if evs is not None:
+            evs[1].record(stream)
+        da.da_cluster_spread(dims, K, cent, eng.stats, spread)
+        if evs is not None:
+            evs[2].record(stream)
+        da.da_attention_spread(dims, Q, K, V, eng.mask, cent, eng.stats, spread, 0.0, O, None, eng.ws)
+        if evs is not None:
+            evs[3].record(stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    for k in range(args.steps):
+        step(evs[k])
+    torch.cuda.synchronize(dev)
+    if eng.status() != 0:
+        raise RuntimeError("device status: " + da.da_status_string(eng.status()))
+    ms = sum(e[0].elapsed_time(e[3]) for e in evs) / args.steps
+    split = {name: sum(e[i].elapsed_time(e[i + 1]) for e in evs) / args.steps
+             for i, name in enumerate(("reassign", "cluster_spread", "attention_spread"))}
+    print(json.dumps({
+        "metric": "effective TFLOP/s & ms/call of reassign + cluster spread + variance-corrected attention "
+                  "(CUDA-core path)",
+        "value": eff / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms, "steps": args.steps,
+        "warmup": args.warmup, "higher_is_better": True, "dtype": {"bf16": "bf16", "f32": "f32"}[w.dtype],
+        "data": "synthetic", "breakdown_ms": split, "effective_flop_per_step": eff,
+        "config": _config(w, args)}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -288,9 +341,14 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--heads", type=int, default=0, help="override the head count (profiling runs)")
     ap.add_argument("--loop", action="store_true", help="run the reassign-cache loop workload instead")
+    ap.add_argument("--spread", action="store_true",
+                    help="time the variance-corrected path (reassign + cluster spread + corrected attention)")
     args = ap.parse_args()
     if args.loop:
         run_loop(args)
+        return
+    if args.spread:
+        run_spread(args)
         return
     ws, rank, local = _dist()
     w = W.WORKLOADS[args.workload]

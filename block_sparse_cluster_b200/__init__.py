@@ -28,7 +28,7 @@ STATUS_NAMES = ["DA_OK", "DA_ERR_INVALID_ARG", "DA_ERR_SHAPE", "DA_ERR_DTYPE", "
                 "DA_ERR_WORKSPACE"]
 EXPORTS = ["da_version", "da_workspace_bytes", "da_schedule_bytes", "da_reassign", "da_mask_prepare",
            "da_attention", "da_device_status", "da_status_string", "da_reassign_noalloc", "da_compensation",
-           "da_attention_prebuilt", "da_centroid_update"]
+           "da_attention_prebuilt", "da_centroid_update", "da_cluster_spread", "da_attention_spread"]
 
 
 class DAError(RuntimeError):
@@ -74,6 +74,11 @@ _lib.da_compensation.argtypes = [ctypes.POINTER(_Dims), ctypes.POINTER(_Mask), c
                                  ctypes.c_size_t, _P]
 _lib.da_centroid_update.restype = ctypes.c_int
 _lib.da_centroid_update.argtypes = [ctypes.POINTER(_Dims), ctypes.POINTER(_Stats), _P, _P]
+_lib.da_cluster_spread.restype = ctypes.c_int
+_lib.da_cluster_spread.argtypes = [ctypes.POINTER(_Dims), _P, _P, ctypes.POINTER(_Stats), _P, _P]
+_lib.da_attention_spread.restype = ctypes.c_int
+_lib.da_attention_spread.argtypes = [ctypes.POINTER(_Dims), _P, _P, _P, ctypes.POINTER(_Mask), _P,
+                                     ctypes.POINTER(_Stats), _P, ctypes.c_float, _P, _P, _P, ctypes.c_size_t, _P]
 _lib.da_reassign_noalloc.restype = ctypes.c_int
 _lib.da_reassign_noalloc.argtypes = [ctypes.POINTER(_Dims), _P, _P, _P, ctypes.POINTER(_Stats), _P]
 _lib.da_device_status.restype = ctypes.c_int
@@ -235,6 +240,27 @@ def da_centroid_update(dims: Dims, stats: ClusterStats, centroids: torch.Tensor,
     _check(_lib.da_centroid_update(ctypes.byref(dims.c()), ctypes.byref(stats.c()), centroids.data_ptr(),
                                    _stream(stream)), "da_centroid_update")
     return centroids
+
+
+def da_cluster_spread(dims: Dims, K: torch.Tensor, centroids: torch.Tensor, stats: ClusterStats,
+                      spread: torch.Tensor, stream=None) -> torch.Tensor:
+    """Second moment of each cluster's keys about its centroid, [B,H,C,d] fp32 (variance
+    correction); stats from da_reassign on the same keys and centroids."""
+    _check(_lib.da_cluster_spread(ctypes.byref(dims.c()), K.data_ptr(), centroids.data_ptr(),
+                                  ctypes.byref(stats.c()), spread.data_ptr(), _stream(stream)), "da_cluster_spread")
+    return spread
+
+
+def da_attention_spread(dims: Dims, Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, mask: BlockMask,
+                        centroids: torch.Tensor, stats: ClusterStats, spread: torch.Tensor, scale: float,
+                        O: torch.Tensor, lse: Optional[torch.Tensor], ws: torch.Tensor, stream=None) -> torch.Tensor:
+    """da_attention with the variance-corrected cluster logits (CUDA-core path)."""
+    _check(_lib.da_attention_spread(ctypes.byref(dims.c()), Q.data_ptr(), K.data_ptr(), V.data_ptr(),
+                                    ctypes.byref(mask.c()), centroids.data_ptr(), ctypes.byref(stats.c()),
+                                    spread.data_ptr(), float(scale), O.data_ptr(),
+                                    lse.data_ptr() if lse is not None else None, ws.data_ptr(), ws.numel(),
+                                    _stream(stream)), "da_attention_spread")
+    return O
 
 
 def kmeans(dims: Dims, K: torch.Tensor, centroids: torch.Tensor, iters: int, stats: ClusterStats,

@@ -72,7 +72,7 @@ da_status cuda_status(cudaError_t e) { return e == cudaSuccess ? DA_OK : DA_ERR_
 
 extern "C" {
 
-int da_version(void) { return 102; }
+int da_version(void) { return 103; }
 
 size_t da_workspace_bytes(const da_dims* dims) {
   Dims g;
@@ -176,7 +176,8 @@ static da_status attention_launch(const Dims& g, const void* Q, const void* K, c
                               lse, status, static_cast<char*>(ws) + L.comp, s);
     else
       e = (g.bf16 ? launch_attention_simt_bf16 : launch_attention_simt_f32)(
-          g, Q, K, V, mask->kv_idx, mask->kv_cnt, mask->max_sel, sched, centroids, sp, scale, O, lse, status, s);
+          g, Q, K, V, mask->kv_idx, mask->kv_cnt, mask->max_sel, sched, centroids, sp, nullptr, scale, O, lse, status,
+          s);
   }
   return cuda_status(e);
 }
@@ -224,6 +225,47 @@ da_status da_centroid_update(const da_dims* dims, const da_cluster_stats* stats,
   StatsPtrs sp;
   if ((st = check_stats(stats, &sp)) != DA_OK) return st;
   return cuda_status(launch_centroid_update(g, sp, centroids, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+da_status da_cluster_spread(const da_dims* dims, const void* K, const void* centroids, const da_cluster_stats* stats,
+                            float* spread, da_stream stream) {
+  Dims g;
+  da_status st = check_dims(dims, &g);
+  if (st != DA_OK) return st;
+  if (!K || !centroids || !spread) return DA_ERR_INVALID_ARG;
+  if (!aligned16(K) || !aligned16(centroids) || !aligned16(spread)) return DA_ERR_ALIGNMENT;
+  StatsPtrs sp;
+  if ((st = check_stats(stats, &sp)) != DA_OK) return st;
+  return cuda_status(launch_cluster_spread(g, K, centroids, sp, spread, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+da_status da_attention_spread(const da_dims* dims, const void* Q, const void* K, const void* V,
+                              const da_block_mask* mask, const void* centroids, const da_cluster_stats* stats,
+                              const float* spread, float scale, void* O, float* lse, void* ws, size_t ws_bytes,
+                              da_stream stream) {
+  Dims g;
+  StatsPtrs sp;
+  da_status st = attention_common(dims, mask, stats, ws, ws_bytes, &g, &sp);
+  if (st != DA_OK) return st;
+  if ((st = check_attention_ptrs(Q, K, V, centroids, O, lse)) != DA_OK) return st;
+  if (!spread) return DA_ERR_INVALID_ARG;
+  if (!aligned16(spread)) return DA_ERR_ALIGNMENT;
+  if (!(scale > 0.f)) scale = 1.0f / sqrtf((float)g.d);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const WsLayout L = ws_layout(g);
+  int* status = reinterpret_cast<int*>(static_cast<char*>(ws) + L.status);
+  const int32_t* sched = mask->schedule;
+  cudaError_t e = cudaSuccess;
+  if (!sched) {
+    int32_t* own = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + L.sched);
+    e = launch_schedule(g, mask->kv_idx, mask->kv_cnt, mask->max_sel, own, status, s);
+    sched = own;
+  }
+  if (e == cudaSuccess)
+    e = (g.bf16 ? launch_attention_simt_bf16 : launch_attention_simt_f32)(
+        g, Q, K, V, mask->kv_idx, mask->kv_cnt, mask->max_sel, sched, centroids, sp, spread, scale, O, lse, status,
+        s);
+  return cuda_status(e);
 }
 
 da_status da_device_status(void* ws, da_stream stream) {

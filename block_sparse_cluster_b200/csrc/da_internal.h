@@ -36,6 +36,8 @@ cudaError_t launch_centroid_norms(const Dims& g, const void* cent, float* norms,
 cudaError_t launch_block_stats(const Dims& g, const void* V, const StatsPtrs& st, cudaStream_t s);
 cudaError_t launch_totals(const Dims& g, const StatsPtrs& st, cudaStream_t s);
 cudaError_t launch_centroid_update(const Dims& g, const StatsPtrs& st, void* cent, cudaStream_t s);
+cudaError_t launch_cluster_spread(const Dims& g, const void* K, const void* cent, const StatsPtrs& st, float* spread,
+                                  cudaStream_t s);
 cudaError_t launch_schedule(const Dims& g, const int32_t* kv_idx, const int32_t* kv_cnt, int max_sel,
                             int32_t* schedule, int* status, cudaStream_t s);
 
@@ -63,7 +65,8 @@ cudaError_t launch_comp_build(const Dims& g, const int32_t* kv_idx, const int32_
   cudaError_t launch_attention_simt_##SUFFIX(const Dims& g, const void* Q, const void* K, const void* V,      \
                                              const int32_t* kv_idx, const int32_t* kv_cnt, int max_sel,       \
                                              const int32_t* schedule, const void* cent, const StatsPtrs& st,  \
-                                             float scale, void* O, float* lse, int* status, cudaStream_t s);
+                                             const float* spread, float scale, void* O, float* lse,           \
+                                             int* status, cudaStream_t s);
 DA_SIMT_DECL(f32)
 DA_SIMT_DECL(bf16)
 #undef DA_SIMT_DECL

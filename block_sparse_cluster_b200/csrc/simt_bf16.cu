@@ -13,8 +13,10 @@ cudaError_t launch_assign_simt_bf16(const Dims& g, const void* K, const void* ce
 cudaError_t launch_attention_simt_bf16(const Dims& g, const void* Q, const void* K, const void* V,
                                       const int32_t* kv_idx, const int32_t* kv_cnt, int max_sel,
                                       const int32_t* schedule, const void* cent, const StatsPtrs& st,
-                                      float scale, void* O, float* lse, int* status, cudaStream_t s) {
-  return launch_attention_simt_t(g, Q, K, V, kv_idx, kv_cnt, max_sel, schedule, cent, st, scale, O, lse, status, s);
+                                      const float* spread, float scale, void* O, float* lse, int* status,
+                                      cudaStream_t s) {
+  return launch_attention_simt_t(g, Q, K, V, kv_idx, kv_cnt, max_sel, schedule, cent, st, spread, scale, O, lse,
+                                 status, s);
 }
 
 }  // namespace da

@@ -54,13 +54,17 @@ __global__ void __launch_bounds__(128) assign_simt_kernel(const T* __restrict__ 
 // complement statistics built in shared memory:
 //   n^U_c = n_c - sum_{j in sel} n_{c,j},  vbar^U_c = (S_c - sum_{j in sel} S_{c,j}) / n^U_c,
 //   logit = s q.cbar_c + ln n^U_c  (left out when n^U_c = 0).
-// Logits are kept in log2 units (q pre-scaled by s*log2(e), bias log2 n^U_c).
+// With `spread` (the second moment D_c of each cluster's keys about its representative), the
+// variance-corrected logit of the ESTRA abstract's reading: + s^2/2 sum_t q_t^2 D_{c,t}; the
+// clusters then go in chunks of 16, their D rows in the upper half of ks.
+// Logits are kept in log2 units (q pre-scaled by s*log2(e), bias log2 n^U_c; the correction is
+// then ln(2)/2 sum_t q_t^2 D_{c,t} in those units).
 template <typename T, int D>
 __global__ void __launch_bounds__(128) attention_simt_kernel(
     const T* __restrict__ Q, const T* __restrict__ K, const T* __restrict__ V, const int32_t* __restrict__ kv_idx,
     const int32_t* __restrict__ kv_cnt, int max_sel, const int32_t* __restrict__ schedule,
-    const T* __restrict__ cent, StatsPtrs st, float scale_log2, T* __restrict__ O, float* __restrict__ lse,
-    int* status, int N, int C, int block, int nB) {
+    const T* __restrict__ cent, StatsPtrs st, const float* __restrict__ spread, float scale_log2,
+    T* __restrict__ O, float* __restrict__ lse, int* status, int N, int C, int block, int nB) {
   __shared__ float ks[32][D];
   __shared__ float vs[32][D];
   __shared__ float beta[32];
@@ -91,8 +95,9 @@ __global__ void __launch_bounds__(128) attention_simt_kernel(
   if (cnt < 0 || cnt > max_sel) cnt = 0;   // reported by the schedule pass
   const int32_t* row = kv_idx + (size_t)item * max_sel;
 
-  // online softmax over shared rows [r0, r0 + 16) of ks/vs, of which the first `valid` are real
-  auto absorb16 = [&](int r0, int valid) {
+  // online softmax over shared rows [r0, r0 + 16) of ks/vs, of which the first `valid` are real;
+  // `corr`: rows 16.. of ks hold the clusters' second moments (variance correction, r0 = 0)
+  auto absorb16 = [&](int r0, int valid, bool corr) {
     float x[16];
     float cm = -INFINITY;
 #pragma unroll
@@ -103,6 +108,12 @@ __global__ void __launch_bounds__(128) attention_simt_kernel(
 #pragma unroll 16
         for (int u = 0; u < D; ++u) dot = fmaf(q[u], ks[r0 + kk][u], dot);
         dot += beta[r0 + kk];
+        if (corr) {
+          float c2 = 0.f;
+#pragma unroll 16
+          for (int u = 0; u < D; ++u) c2 = fmaf(q[u] * q[u], ks[16 + kk][u], c2);
+          dot = fmaf(0.34657359027997264f, c2, dot);   // ln(2) / 2
+        }
       }
       x[kk] = dot;
       cm = fmaxf(cm, dot);
@@ -123,8 +134,8 @@ __global__ void __launch_bounds__(128) attention_simt_kernel(
     }
   };
   auto absorb = [&](int valid) {   // rows [0, valid) of the 32 staged
-    absorb16(0, min(valid, 16));
-    if (valid > 16) absorb16(16, valid - 16);
+    absorb16(0, min(valid, 16), false);
+    if (valid > 16) absorb16(16, valid - 16, false);
   };
 
   // exact attention on the selected blocks
@@ -156,10 +167,11 @@ __global__ void __launch_bounds__(128) attention_simt_kernel(
     }
   }
 
-  // compensation: clusters in chunks of 32
-  for (int c0 = 0; c0 < C; c0 += 32) {
+  // compensation: clusters in chunks of 32 (16 with the variance correction)
+  const int CH = spread ? 16 : 32;
+  for (int c0 = 0; c0 < C; c0 += CH) {
     __syncthreads();
-    {
+    if ((t >> 2) < CH) {
       const int cl = t >> 2, part = t & 3;
       const int c = c0 + cl;
       constexpr int W = D / 4;
@@ -183,10 +195,15 @@ __global__ void __launch_bounds__(128) attention_simt_kernel(
 #pragma unroll
       for (int u = 0; u < W; ++u) vs[cl][part * W + u] = acc[u] * inv;
       if (part == 0) beta[cl] = nU > 0 ? log2f((float)nU) : -INFINITY;
-      for (int x = t; x < 32 * D; x += 128) ks[x / D][x % D] = to_f32(cent[((size_t)bh * C + c0) * D + x]);
     }
+    for (int x = t; x < CH * D; x += 128) ks[x / D][x % D] = to_f32(cent[((size_t)bh * C + c0) * D + x]);
+    if (spread)
+      for (int x = t; x < 16 * D; x += 128) ks[16 + x / D][x % D] = spread[((size_t)bh * C + c0) * D + x];
     __syncthreads();
-    if (active) absorb(32);
+    if (active) {
+      if (spread) absorb16(0, 16, true);
+      else absorb(32);
+    }
   }
 
   if (active) {

@@ -99,6 +99,54 @@ __global__ void __launch_bounds__(128) totals_kernel(StatsPtrs st, int C, int bl
   if (lane == 0) st.n_tot[(size_t)bh * C + c] = n;
 }
 
+// Second moment of each cluster's keys about its representative (the variance correction of
+// the ESTRA abstract, read as a diagonal Gaussian about cbar_c):
+//   D[c, t] = (1 / n_c) sum over the keys k with a(k) = c of (k_t - cbar_{c,t})^2  (0 when n_c = 0).
+// A warp per (head, cluster), lanes over the columns: it walks the blocks that hold the cluster
+// (seg_idx) in order and, in each, the block's keys of the cluster in index order (a ballot over
+// the assignments), so the sums are taken in a fixed order: deterministic bits.
+template <typename T, int D>
+__global__ void __launch_bounds__(128) cluster_spread_kernel(const T* __restrict__ K, const T* __restrict__ cent,
+                                                             StatsPtrs st, float* __restrict__ spread, int N, int C,
+                                                             int block, int nB) {
+  constexpr int NS = D / 32;              // columns per lane
+  const int bh = blockIdx.x;
+  const int c = blockIdx.y * 4 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (c >= C) return;                     // (C is a multiple of 32)
+  float cb[NS], acc[NS];
+  load_vec(cent + ((size_t)bh * C + c) * D + lane * NS, cb, NS);
+#pragma unroll
+  for (int i = 0; i < NS; ++i) acc[i] = 0.f;
+  const size_t hb = (size_t)bh * nB;
+  for (int j = 0; j < nB; ++j) {
+    if (st.seg_idx[(hb + j) * C + c] == 0xFF) continue;      // warp-uniform
+    const int k0 = j * block;
+    const int nk = min(block, N - k0);
+    for (int kb = 0; kb < nk; kb += 32) {
+      const int kk = kb + lane;
+      const bool mine = kk < nk && st.assign[(size_t)bh * N + k0 + kk] == c;
+      unsigned msk = __ballot_sync(0xffffffffu, mine);
+      while (msk) {
+        const int b = __ffs(msk) - 1;
+        msk &= msk - 1u;
+        float kv[NS];
+        load_vec(K + ((size_t)bh * N + k0 + kb + b) * D + lane * NS, kv, NS);
+#pragma unroll
+        for (int i = 0; i < NS; ++i) {
+          const float dv = kv[i] - cb[i];
+          acc[i] = fmaf(dv, dv, acc[i]);
+        }
+      }
+    }
+  }
+  const int n = st.n_tot[(size_t)bh * C + c];
+  const float inv = n > 0 ? 1.f / (float)n : 0.f;
+  float* dst = spread + ((size_t)bh * C + c) * D + lane * NS;
+#pragma unroll
+  for (int i = 0; i < NS; ++i) dst[i] = acc[i] * inv;
+}
+
 // Plan validation and work order: items of a head ordered by descending row length
 // (ties by q-block index); heads in order.  A malformed row is reported and scheduled with
 // cost 0 (the attention kernels skip its invalid entries).
@@ -189,6 +237,20 @@ cudaError_t launch_totals(const Dims& g, const StatsPtrs& st, cudaStream_t s) {
   dim3 grid(g.B * g.H, (g.C + 3) / 4);                  // 4 clusters (warps) per CTA
   if (g.d == 128) totals_kernel<128><<<grid, 128, 0, s>>>(st, g.C, g.block, g.nB);
   else totals_kernel<64><<<grid, 128, 0, s>>>(st, g.C, g.block, g.nB);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_cluster_spread(const Dims& g, const void* K, const void* cent, const StatsPtrs& st, float* spread,
+                                  cudaStream_t s) {
+  dim3 grid(g.B * g.H, (g.C + 3) / 4);                  // 4 clusters (warps) per CTA
+#define DA_SPREAD(T, DD) \
+  cluster_spread_kernel<T, DD><<<grid, 128, 0, s>>>((const T*)K, (const T*)cent, st, spread, g.N, g.C, g.block, g.nB)
+  if (g.bf16) {
+    if (g.d == 128) DA_SPREAD(__nv_bfloat16, 128); else DA_SPREAD(__nv_bfloat16, 64);
+  } else {
+    if (g.d == 128) DA_SPREAD(float, 128); else DA_SPREAD(float, 64);
+  }
+#undef DA_SPREAD
   return cudaGetLastError();
 }
 

@@ -202,6 +202,36 @@ DA_API da_status da_centroid_update(const da_dims* dims, const da_cluster_stats*
                              da_stream stream);
 
 /*
+ * Variance-corrected cluster logits ("ESTRA: Extreme Sparsity Through Refined
+ * Attention", abstract: "a variance-based correction further refines the
+ * attention weights of the cluster representatives").  The page prints no
+ * formula; the reading here treats the keys of cluster c as Gaussian about
+ * the representative cbar_c with a diagonal second moment D_c, so that
+ * mean_k exp(s q.k) ~ exp(s q.cbar_c + s^2/2 sum_t q_t^2 D_{c,t}).
+ *
+ * da_cluster_spread: with stats from da_reassign on these keys and centroids,
+ *   spread[b,h,c,t] = (1/n_c) sum_{k: a(k)=c} (k_t - cbar_{c,t})^2
+ * (fp32, 0 for a cluster without keys), summed in a fixed order (blocks, then
+ * keys in index order).  K, centroids: as given to da_reassign.  spread:
+ * [B,H,C,d] fp32 device, written, 16-byte aligned.  Errors: those of
+ * da_reassign's arguments; DA_ERR_INVALID_ARG for a NULL spread.
+ *
+ * da_attention_spread: da_attention with every cluster logit corrected,
+ *   s q.cbar_c + ln n^U_c + s^2/2 sum_t q_t^2 D_{c,t},
+ * D = spread.  It runs on the CUDA cores for both dtypes (fp32 arithmetic,
+ * the bf16 inputs upcast): a reference-grade path, not the tensor-core one.
+ * It does not use da_compensation's values.  Arguments, layouts and errors as
+ * in da_attention, plus spread ([B,H,C,d] fp32, read; DA_ERR_INVALID_ARG if
+ * NULL).
+ */
+DA_API da_status da_cluster_spread(const da_dims* dims, const void* K, const void* centroids,
+                                   const da_cluster_stats* stats, float* spread, da_stream stream);
+DA_API da_status da_attention_spread(const da_dims* dims, const void* Q, const void* K, const void* V,
+                                     const da_block_mask* mask, const void* centroids,
+                                     const da_cluster_stats* stats, const float* spread, float scale, void* O,
+                                     float* lse, void* ws, size_t ws_bytes, da_stream stream);
+
+/*
  * Reassign Cache without a caller workspace (the paper has no counterpart: this is a calling
  * convention of this library).  Some callers cannot call cudaMalloc when they run a step: a
  * runtime whose device memory is planned once at start-up, a host application whose pool owns all

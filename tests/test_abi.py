@@ -32,7 +32,7 @@ def test_every_declared_symbol_is_exported():
 
 
 def test_version_and_strings():
-    assert da.da_version() == 102
+    assert da.da_version() == 103
     for code in range(10):
         assert da.da_status_string(code) and da.da_status_string(code) != "unknown status"
 
@@ -125,3 +125,21 @@ def test_centroid_update_rejects_arguments():
     assert da._lib.da_centroid_update(ctypes.byref(d.c()), ctypes.byref(st), 0x1004, None) == 4
     bad = da._Stats(*([0x1000] * 7 + [0x1004, 0x1000]))
     assert da._lib.da_centroid_update(ctypes.byref(d.c()), ctypes.byref(bad), 0x1000, None) == 4
+
+
+def test_spread_calls_reject_arguments():
+    d = _dims()
+    st = da._Stats(*([0x1000] * 9))
+    m = da._Mask(0x1000, 0x1000, 4, None)
+    sp = da._lib.da_cluster_spread
+    assert sp(ctypes.byref(d.c()), 0x1000, 0x1000, ctypes.byref(st), None, None) == 1
+    assert sp(ctypes.byref(d.c()), None, 0x1000, ctypes.byref(st), 0x1000, None) == 1
+    assert sp(ctypes.byref(d.c()), 0x1000, 0x1000, ctypes.byref(st), 0x1008, None) == 4
+    bad = da._Stats(*([0x1000] * 7 + [0x1004, 0x1000]))
+    assert sp(ctypes.byref(d.c()), 0x1000, 0x1000, ctypes.byref(bad), 0x1000, None) == 4
+    at = da._lib.da_attention_spread
+    ok = (0x1000, 0x1000, 0x1000, ctypes.byref(m), 0x1000, ctypes.byref(st))
+    assert at(ctypes.byref(d.c()), *ok, None, 0.0, 0x1000, None, 0x1000, 1 << 30, None) == 1
+    assert at(ctypes.byref(d.c()), *ok, 0x1004, 0.0, 0x1000, None, 0x1000, 1 << 30, None) == 4
+    assert at(ctypes.byref(d.c()), *ok, 0x1000, 0.0, None, None, 0x1000, 1 << 30, None) == 1
+    assert at(ctypes.byref(d.c()), *ok, 0x1000, 0.0, 0x1000, None, 0x1000, 0, None) == 9
