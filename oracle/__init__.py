@@ -41,6 +41,13 @@ Readings taken where the pages are silent (each is listed in the design notes):
   the mean of (k_t - cbar_{c,t})^2 over all keys assigned to c), so that
   mean_k exp(s q.k) = exp(s q.cbar_c + s^2/2 sum_t q_t^2 D_{c,t}) up to higher
   cumulants; the cluster logit gains the term s^2/2 sum_t q_t^2 D_{c,t}.
+* R7 (inclusion-probability reweighting, optional) the AB-Attention abstract
+  samples blocks and "reweights them by inverse inclusion probability, so that
+  one pass estimates dense attention".  Reading: the q-block's selected blocks
+  carry inclusion probabilities pi_j in (0, 1]; numerator and denominator of
+  the softmax each sum (1 / pi_j) times the block's exact terms (Horvitz-
+  Thompson), with no cluster compensation; a row without selected blocks
+  gives O = 0 and LSE = -inf.
 
 Parity status: reassignment, block statistics and attention are each pinned
 by tests that do not call this module's formulas again (library routines,
@@ -60,7 +67,7 @@ import numpy as np
 __all__ = [
     "reassign", "block_ranges", "block_histogram", "block_entries", "cluster_totals",
     "complement_stats", "attention_qblock", "attention", "lloyd_step", "kmeans", "sse",
-    "cluster_spread",
+    "cluster_spread", "attention_sip_qblock",
 ]
 
 
@@ -237,6 +244,39 @@ def attention_qblock(Q, K, V, centroids, sel_blocks: Sequence[int], assign, i: i
     num = pe @ Vf[in_sel] + pl @ vbar[live]
     den = pe.sum(axis=1) + pl.sum(axis=1)
     out = num / den[:, None]
+    if return_lse:
+        return out, m + np.log(den)
+    return out
+
+
+def attention_sip_qblock(Q, K, V, sel_blocks: Sequence[int], incl: Sequence[float], i: int, block: int,
+                         scale: Optional[float] = None, return_lse: bool = False):
+    """Output rows of q-block i under inclusion-probability reweighting (reading R7): block j of
+    the selection, included with probability incl[j], enters numerator and denominator with the
+    weight 1 / incl[j]."""
+    Qf = _f64(Q)
+    Kf = _f64(K)
+    Vf = _f64(V)
+    N, d = Kf.shape
+    s = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    rng = block_ranges(N, block)
+    qs, qe = rng[i]
+    q = Qf[qs:qe]
+    nq = qe - qs
+    if len(sel_blocks) == 0:
+        out = np.zeros((nq, d))
+        return (out, np.full(nq, -np.inf)) if return_lse else out
+    logits, vals = [], []
+    for j, p in zip(sel_blocks, incl):
+        bs, be = rng[int(j)]
+        logits.append(s * (q @ Kf[bs:be].T) - math.log(float(p)))   # weight 1/p as a log
+        vals.append(Vf[bs:be])
+    ell = np.concatenate(logits, axis=1)
+    vv = np.concatenate(vals, axis=0)
+    m = ell.max(axis=1)
+    pe = np.exp(ell - m[:, None])
+    den = pe.sum(axis=1)
+    out = (pe @ vv) / den[:, None]
     if return_lse:
         return out, m + np.log(den)
     return out

@@ -12,6 +12,7 @@ import pytest
 import oracle
 from tests import test_oracle_lloyd as lloyd_pins
 from tests import test_oracle_pins as pins
+from tests import test_oracle_sip as sip_pins
 from tests import test_oracle_spread as spread_pins
 
 MUTATIONS = {
@@ -43,6 +44,11 @@ MUTATIONS = {
     "spread: wrong sign": ("lam = lam + 0.5 * s * s *", "lam = lam - 0.5 * s * s *"),
     "spread about the mean of all keys": ("dev2 = (Kf - Cf[a]) ** 2", "dev2 = (Kf - Kf.mean(axis=0)) ** 2"),
     "spread: sum instead of mean": ("D[nz] = tot[nz] / n[nz, None]", "D[nz] = tot[nz]"),
+    "inclusion weight pi instead of 1/pi": ("s * (q @ Kf[bs:be].T) - math.log(float(p))",
+                                             "s * (q @ Kf[bs:be].T) + math.log(float(p))"),
+    "inclusion weight dropped": ("s * (q @ Kf[bs:be].T) - math.log(float(p))", "s * (q @ Kf[bs:be].T)"),
+    "inclusion weights replaced by one common weight": ("s * (q @ Kf[bs:be].T) - math.log(float(p))",
+                                                        "s * (q @ Kf[bs:be].T) - math.log(float(sum(incl)))"),
 }
 
 PINS = [
@@ -68,6 +74,9 @@ PINS = [
     (lloyd_pins.test_objective_hand_value, {}),
     (spread_pins.test_offset_keys_give_the_squared_offset, {}),
     (spread_pins.test_corrected_logit_matches_the_cluster_log_sum_exp_to_fourth_order, {"seed": 0}),
+    (sip_pins.test_certain_inclusion_of_every_block_is_dense_attention, {}),
+    (sip_pins.test_sums_are_unbiased_over_all_subsets, {"seed": 1}),
+    (sip_pins.test_equal_weights_cancel, {}),
 ]
 
 
@@ -86,6 +95,7 @@ def test_pins_catch_planted_mistake(name, monkeypatch):
     monkeypatch.setattr(pins, "oracle", mutant)
     monkeypatch.setattr(lloyd_pins, "oracle", mutant)
     monkeypatch.setattr(spread_pins, "oracle", mutant)
+    monkeypatch.setattr(sip_pins, "oracle", mutant)
     caught = []
     for fn, kw in PINS:
         try:
