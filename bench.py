@@ -325,6 +325,45 @@ def run_spread(args):
         "config": _config(w, args)}))
 
 
+def run_sip(args):
+    """Inclusion-probability reweighting (AB-Attention abstract's estimator): one call of
+    da_attention_sip per step on the plan's blocks with seeded inclusion probabilities; the fused
+    tensor-core kernel with the weights as bias rows.  Effective FLOPs count the kept keys only."""
+    import block_sparse_cluster_b200 as da
+    w = W.WORKLOADS[args.workload]
+    if args.heads > 0:
+        w = W.scaled(w, H=args.heads)
+    dev = torch.device("cuda", 0)
+    inp = W.make_inputs(w, seed=args.seed)
+    dims = da.Dims(w.B, w.H, w.N, w.d, w.C, w.block, w.torch_dtype)
+    flops_all = W.effective_flops(w, inp.kv_cnt, inp.kv_idx)
+    eff = flops_all - float(w.B * w.H * 4 * w.N * w.C * w.d)       # drop the cluster columns
+    incl = W.inclusion_probabilities(w, args.seed, inp.kv_idx.shape[-1]).to(dev)
+    ws = da.workspace(dims, dev)
+    Q, K, V = (x.to(dev) for x in (inp.Q, inp.K, inp.V))
+    sched = torch.empty(w.B * w.H * w.nB, dtype=torch.int32, device=dev)
+    mask = da.da_mask_prepare(dims, da.BlockMask(inp.kv_idx.to(dev), inp.kv_cnt.to(dev)), sched, ws)
+    O = torch.empty_like(Q)
+    for _ in range(max(3, args.warmup)):
+        da.da_attention_sip(dims, Q, K, V, mask, incl, 0.0, O, None, ws)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        da.da_attention_sip(dims, Q, K, V, mask, incl, 0.0, O, None, ws)
+    e1.record()
+    torch.cuda.synchronize(dev)
+    if da.da_device_status(ws) != 0:
+        raise RuntimeError("device status after the timed calls")
+    ms = e0.elapsed_time(e1) / args.steps
+    print(json.dumps({
+        "metric": "effective TFLOP/s & ms/call of inclusion-probability reweighted block-sparse attention",
+        "value": eff / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms, "steps": args.steps,
+        "warmup": args.warmup, "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+        "pct_of_bf16_peak": 100.0 * eff / (ms * 1e-3) / 1e12 / _peaks()[0]["bf16_tflops"],
+        "effective_flop_per_step": eff, "config": _config(w, args)}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -343,12 +382,17 @@ def main():
     ap.add_argument("--loop", action="store_true", help="run the reassign-cache loop workload instead")
     ap.add_argument("--spread", action="store_true",
                     help="time the variance-corrected path (reassign + cluster spread + corrected attention)")
+    ap.add_argument("--sip", action="store_true",
+                    help="time the inclusion-probability reweighted attention (no compensation)")
     args = ap.parse_args()
     if args.loop:
         run_loop(args)
         return
     if args.spread:
         run_spread(args)
+        return
+    if args.sip:
+        run_sip(args)
         return
     ws, rank, local = _dist()
     w = W.WORKLOADS[args.workload]

@@ -28,7 +28,8 @@ STATUS_NAMES = ["DA_OK", "DA_ERR_INVALID_ARG", "DA_ERR_SHAPE", "DA_ERR_DTYPE", "
                 "DA_ERR_WORKSPACE"]
 EXPORTS = ["da_version", "da_workspace_bytes", "da_schedule_bytes", "da_reassign", "da_mask_prepare",
            "da_attention", "da_device_status", "da_status_string", "da_reassign_noalloc", "da_compensation",
-           "da_attention_prebuilt", "da_centroid_update", "da_cluster_spread", "da_attention_spread"]
+           "da_attention_prebuilt", "da_centroid_update", "da_cluster_spread", "da_attention_spread",
+           "da_attention_sip"]
 
 
 class DAError(RuntimeError):
@@ -79,6 +80,9 @@ _lib.da_cluster_spread.argtypes = [ctypes.POINTER(_Dims), _P, _P, ctypes.POINTER
 _lib.da_attention_spread.restype = ctypes.c_int
 _lib.da_attention_spread.argtypes = [ctypes.POINTER(_Dims), _P, _P, _P, ctypes.POINTER(_Mask), _P,
                                      ctypes.POINTER(_Stats), _P, ctypes.c_float, _P, _P, _P, ctypes.c_size_t, _P]
+_lib.da_attention_sip.restype = ctypes.c_int
+_lib.da_attention_sip.argtypes = [ctypes.POINTER(_Dims), _P, _P, _P, ctypes.POINTER(_Mask), _P, ctypes.c_float, _P,
+                                  _P, _P, ctypes.c_size_t, _P]
 _lib.da_reassign_noalloc.restype = ctypes.c_int
 _lib.da_reassign_noalloc.argtypes = [ctypes.POINTER(_Dims), _P, _P, _P, ctypes.POINTER(_Stats), _P]
 _lib.da_device_status.restype = ctypes.c_int
@@ -260,6 +264,18 @@ def da_attention_spread(dims: Dims, Q: torch.Tensor, K: torch.Tensor, V: torch.T
                                     spread.data_ptr(), float(scale), O.data_ptr(),
                                     lse.data_ptr() if lse is not None else None, ws.data_ptr(), ws.numel(),
                                     _stream(stream)), "da_attention_spread")
+    return O
+
+
+def da_attention_sip(dims: Dims, Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, mask: BlockMask,
+                     incl: torch.Tensor, scale: float, O: torch.Tensor, lse: Optional[torch.Tensor], ws: torch.Tensor,
+                     stream=None) -> torch.Tensor:
+    """Block-sparse attention with every selected block weighted by 1 / its inclusion probability
+    (incl [B,H,nB,max_sel] fp32, aligned with the plan's slots); no cluster compensation."""
+    _check(_lib.da_attention_sip(ctypes.byref(dims.c()), Q.data_ptr(), K.data_ptr(), V.data_ptr(),
+                                 ctypes.byref(mask.c()), incl.data_ptr(), float(scale), O.data_ptr(),
+                                 lse.data_ptr() if lse is not None else None, ws.data_ptr(), ws.numel(),
+                                 _stream(stream)), "da_attention_sip")
     return O
 
 

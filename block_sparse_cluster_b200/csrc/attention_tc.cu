@@ -16,6 +16,11 @@
 // The compensation chunks (vbar^U rows in bf16 and log2 n^U per cluster) of every item are
 // written beforehand by comp_build.cu; here they are loaded like value blocks.
 //
+// Inclusion-probability mode (AB-Attention abstract: sampled blocks "reweighted by inverse
+// inclusion probability"): with p.incl, an item's steps are its selected blocks only (one fully
+// masked step if it has none), and block j's logits carry the bias -log2 pi_j, i.e. the weight
+// 1 / pi_j in both sums of the softmax; no cluster columns.
+//
 // Roles (384 threads):
 //   warps 0-3, 4-7  two softmax warpgroups X = 0, 1; warpgroup X takes the steps g with g & 1 = X
 //              of every item, so the two overlap each other and the tensor core.  Thread t of a
@@ -93,6 +98,7 @@ struct Params {
   float* lse;
   int* status;
   const uint8_t* comp;                   // [items][nchunk] compensation chunks of kChunkBytes
+  const float* incl;                     // [items][max_sel] inclusion probabilities, or NULL
   int N, C, nB, n_items, nchunk;
   float scale_log2;
 };
@@ -120,14 +126,14 @@ __device__ __forceinline__ Item item_at(const Params& p, int k) {
   int cnt = p.kv_cnt[item];
   if (cnt < 0 || cnt > p.max_sel) cnt = 0;
   it.nsel = cnt;
-  it.T = cnt + p.nchunk;
+  it.T = p.incl ? max(cnt, 1) : cnt + p.nchunk;
   it.row = p.kv_idx + (size_t)item * p.max_sel;
   return it;
 }
 
 // Key block of exact step s; an out-of-range index becomes a fully masked block 0.
 __device__ __forceinline__ int block_of(const Params& p, const Item& it, int s, bool* valid) {
-  const int j = it.row[s];
+  const int j = s < it.nsel ? it.row[s] : -1;
   *valid = (j >= 0 && j < p.nB);
   return *valid ? j : 0;
 }
@@ -279,7 +285,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           const int ks = g % kKStages, bs = g % kBStages;
           if (!mbar_wait(&bars->k_empty[ks], ((g / kKStages) & 1) ^ 1, abort, status)) { ok = false; break; }
           uint8_t* dk = sK + ks * kTile;
-          if (s < it.nsel) {
+          if (s < it.nsel || p.incl) {
             bool valid;
             const int j = block_of(p, it, s, &valid);
             mbar_expect_tx(&bars->k_full[ks], kTile);
@@ -288,14 +294,20 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             // bias row of a key block: 0 for its keys, -inf past the end of a short last block
             // (generic stores, published to the softmax by the arrive on b_full)
             if (!mbar_wait(&bars->b_empty[bs], ((g / kBStages) & 1) ^ 1, abort, status)) { ok = false; break; }
-            const int ncol = valid ? min(kBN, p.N - j * kBN) : 0;
-            bars->bflag[bs] = ncol == kBN ? 1 : 0;
+            int ncol = valid ? min(kBN, p.N - j * kBN) : 0;
+            float w = 0.f;                 // log2 weight of the block's columns
+            if (p.incl && ncol > 0) {
+              const float pi = p.incl[(size_t)(it.bh * p.nB + it.i) * p.max_sel + s];
+              if (pi > 0.f) w = -__log2f(pi);
+              else ncol = 0;               // a block that is never included: left out
+            }
+            bars->bflag[bs] = (ncol == kBN && !p.incl) ? 1 : 0;
             float4* bb = reinterpret_cast<float4*>(sBias + bs * kBN);
 #pragma unroll 4
             for (int c4 = 0; c4 < kBN / 4; ++c4) {
               const int c = 4 * c4;
-              bb[c4] = make_float4(c < ncol ? 0.f : -INFINITY, c + 1 < ncol ? 0.f : -INFINITY,
-                                   c + 2 < ncol ? 0.f : -INFINITY, c + 3 < ncol ? 0.f : -INFINITY);
+              bb[c4] = make_float4(c < ncol ? w : -INFINITY, c + 1 < ncol ? w : -INFINITY,
+                                   c + 2 < ncol ? w : -INFINITY, c + 3 < ncol ? w : -INFINITY);
             }
             mbar_arrive(&bars->b_full[bs]);
           } else {
@@ -333,7 +345,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           const int vs = g % kVStages;
           if (!mbar_wait(&bars->v_empty[vs], ((g / kVStages) & 1) ^ 1, abort, status)) { ok = false; break; }
           uint8_t* dv = sV + vs * kTile;
-          if (s < it.nsel) {
+          if (s < it.nsel || p.incl) {
             bool valid;
             const int j = block_of(p, it, s, &valid);
             mbar_expect_tx(&bars->v_full[vs], kTile);
@@ -572,7 +584,7 @@ size_t attention_tc_scratch_bytes(const Dims& g) {
 cudaError_t launch_attention_tc(const Dims& g, const void* Q, const void* K, const void* V,
                                 const int32_t* kv_idx, const int32_t* kv_cnt, int max_sel,
                                 const int32_t* schedule, const void* cent, const StatsPtrs& st, float scale,
-                                void* O, float* lse, int* status, void* comp, cudaStream_t s) {
+                                void* O, float* lse, int* status, void* comp, const float* incl, cudaStream_t s) {
   CUtensorMap tq, tk, tv, tc, tp;
   const unsigned long long BH = (unsigned long long)g.B * g.H;
   const int nchunk = (g.C + kBN - 1) / kBN;
@@ -590,6 +602,7 @@ cudaError_t launch_attention_tc(const Dims& g, const void* Q, const void* K, con
   p.lse = lse;
   p.status = status;
   p.comp = static_cast<const uint8_t*>(comp);
+  p.incl = incl;
   p.N = g.N;
   p.C = g.C;
   p.nB = g.nB;

@@ -173,7 +173,7 @@ static da_status attention_launch(const Dims& g, const void* Q, const void* K, c
   if (e == cudaSuccess) {
     if (attention_tc_supported(g))
       e = launch_attention_tc(g, Q, K, V, mask->kv_idx, mask->kv_cnt, mask->max_sel, sched, centroids, sp, scale, O,
-                              lse, status, static_cast<char*>(ws) + L.comp, s);
+                              lse, status, static_cast<char*>(ws) + L.comp, nullptr, s);
     else
       e = (g.bf16 ? launch_attention_simt_bf16 : launch_attention_simt_f32)(
           g, Q, K, V, mask->kv_idx, mask->kv_cnt, mask->max_sel, sched, centroids, sp, nullptr, scale, O, lse, status,
@@ -265,6 +265,36 @@ da_status da_attention_spread(const da_dims* dims, const void* Q, const void* K,
     e = (g.bf16 ? launch_attention_simt_bf16 : launch_attention_simt_f32)(
         g, Q, K, V, mask->kv_idx, mask->kv_cnt, mask->max_sel, sched, centroids, sp, spread, scale, O, lse, status,
         s);
+  return cuda_status(e);
+}
+
+da_status da_attention_sip(const da_dims* dims, const void* Q, const void* K, const void* V,
+                           const da_block_mask* mask, const float* incl, float scale, void* O, float* lse, void* ws,
+                           size_t ws_bytes, da_stream stream) {
+  Dims g;
+  da_status st = check_dims(dims, &g);
+  if (st != DA_OK) return st;
+  if (!attention_tc_supported(g)) return DA_ERR_UNSUPPORTED;
+  if ((st = check_mask(g, mask)) != DA_OK) return st;
+  if ((st = check_ws(g, ws, ws_bytes)) != DA_OK) return st;
+  if ((st = check_attention_ptrs(Q, K, V, K, O, lse)) != DA_OK) return st;
+  if (!incl) return DA_ERR_INVALID_ARG;
+  if (!aligned16(incl)) return DA_ERR_ALIGNMENT;
+  if (!(scale > 0.f)) scale = 1.0f / sqrtf((float)g.d);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const WsLayout L = ws_layout(g);
+  int* status = reinterpret_cast<int*>(static_cast<char*>(ws) + L.status);
+  const int32_t* sched = mask->schedule;
+  cudaError_t e = cudaSuccess;
+  if (!sched) {
+    int32_t* own = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + L.sched);
+    e = launch_schedule(g, mask->kv_idx, mask->kv_cnt, mask->max_sel, own, status, s);
+    sched = own;
+  }
+  // no cluster steps: the centroid map is never read (K stands in for it), nor are the statistics
+  if (e == cudaSuccess)
+    e = launch_attention_tc(g, Q, K, V, mask->kv_idx, mask->kv_cnt, mask->max_sel, sched, K, StatsPtrs{}, scale, O,
+                            lse, status, static_cast<char*>(ws) + L.comp, incl, s);
   return cuda_status(e);
 }
 

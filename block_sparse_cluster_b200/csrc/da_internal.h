@@ -52,7 +52,8 @@ size_t attention_tc_scratch_bytes(const Dims& g);   // compensation chunks of ev
 cudaError_t launch_attention_tc(const Dims& g, const void* Q, const void* K, const void* V,
                                 const int32_t* kv_idx, const int32_t* kv_cnt, int max_sel,
                                 const int32_t* schedule, const void* cent, const StatsPtrs& st, float scale,
-                                void* O, float* lse, int* status, void* comp, cudaStream_t s);
+                                void* O, float* lse, int* status, void* comp, const float* incl,
+                                cudaStream_t s);
 
 // comp_build.cu
 cudaError_t launch_comp_build(const Dims& g, const int32_t* kv_idx, const int32_t* kv_cnt, int max_sel,

@@ -224,6 +224,27 @@ DA_API da_status da_centroid_update(const da_dims* dims, const da_cluster_stats*
  * in da_attention, plus spread ([B,H,C,d] fp32, read; DA_ERR_INVALID_ARG if
  * NULL).
  */
+/*
+ * Inclusion-probability reweighting ("AB-Attention", abstract: sampled blocks
+ * are "reweighted by inverse inclusion probability, so that one pass estimates
+ * dense attention").  Reading: block j of q-block i's selection, included with
+ * probability pi = incl[b,h,i,s] for its slot s in kv_idx, enters both sums of
+ * the softmax with the weight 1 / pi (Horvitz-Thompson), with no cluster
+ * compensation:
+ *   O_q = sum_s (1/pi_s) sum_{k in block s} e^{s q.k} v_k
+ *         / sum_s (1/pi_s) sum_{k in block s} e^{s q.k};
+ * a q-block without selected blocks gets O = 0 (LSE = -inf), and a slot with
+ * pi <= 0 leaves its block out.  The fused tensor-core kernel with the weights
+ * as its bias rows: bf16 inputs, d = 128, block = 128 only (else
+ * DA_ERR_UNSUPPORTED).  No reassignment or statistics are needed.
+ * incl: [B,H,nB,max_sel] fp32 device, read for the filled slots only,
+ * 16-byte aligned.  Other arguments, layouts and errors as in da_attention;
+ * DA_ERR_INVALID_ARG for a NULL incl.
+ */
+DA_API da_status da_attention_sip(const da_dims* dims, const void* Q, const void* K, const void* V,
+                                  const da_block_mask* mask, const float* incl, float scale, void* O, float* lse,
+                                  void* ws, size_t ws_bytes, da_stream stream);
+
 DA_API da_status da_cluster_spread(const da_dims* dims, const void* K, const void* centroids,
                                    const da_cluster_stats* stats, float* spread, da_stream stream);
 DA_API da_status da_attention_spread(const da_dims* dims, const void* Q, const void* K, const void* V,

@@ -143,3 +143,15 @@ def test_spread_calls_reject_arguments():
     assert at(ctypes.byref(d.c()), *ok, 0x1004, 0.0, 0x1000, None, 0x1000, 1 << 30, None) == 4
     assert at(ctypes.byref(d.c()), *ok, 0x1000, 0.0, None, None, 0x1000, 1 << 30, None) == 1
     assert at(ctypes.byref(d.c()), *ok, 0x1000, 0.0, 0x1000, None, 0x1000, 0, None) == 9
+
+
+def test_sip_call_rejects_arguments():
+    d = _dims()
+    m = da._Mask(0x1000, 0x1000, 4, None)
+    f = da._lib.da_attention_sip
+    ok = (0x1000, 0x1000, 0x1000, ctypes.byref(m))
+    assert f(ctypes.byref(d.c()), *ok, None, 0.0, 0x1000, None, 0x1000, 1 << 30, None) == 1
+    assert f(ctypes.byref(d.c()), *ok, 0x1004, 0.0, 0x1000, None, 0x1000, 1 << 30, None) == 4
+    assert f(ctypes.byref(d.c()), *ok, 0x1000, 0.0, 0x1000, None, 0x1000, 0, None) == 9
+    f32 = _dims(dtype=torch.float32)
+    assert f(ctypes.byref(f32.c()), *ok, 0x1000, 0.0, 0x1000, None, 0x1000, 1 << 30, None) == 5

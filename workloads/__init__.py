@@ -94,7 +94,7 @@ def scaled(w: Workload, **kw) -> Workload:
 # seeding
 
 _TAGS = {"q": 1, "k": 2, "v": 3, "mu": 4, "label": 5, "mask": 6, "density": 7, "drift": 8,
-         "perm": 9}
+         "perm": 9, "incl": 10}
 
 
 def _seed(seed: int, tag: str, *idx: int) -> int:
@@ -254,3 +254,14 @@ def effective_flops(w: Workload, kv_cnt: torch.Tensor, kv_idx: torch.Tensor) -> 
     kept = np.where(valid, blk_len[np.clip(idx, 0, nB - 1)], 0).sum(-1)      # [B,H,nB]
     qlen = blk_len[None, None, :]
     return float((4 * qlen * (kept + C) * d).sum())
+
+
+def inclusion_probabilities(w: Workload, seed: int, max_sel: int, lo: float = 0.2) -> torch.Tensor:
+    """Seeded inclusion probabilities for the plan's slots, [B,H,nB,max_sel] fp32 drawn uniformly
+    from [lo, 1) per (batch, head); numbers only (the reweighting itself lives elsewhere)."""
+    out = torch.empty(w.B, w.H, w.nB, max_sel, dtype=torch.float32)
+    for b in range(w.B):
+        for h in range(w.H):
+            u = torch.rand(w.nB, max_sel, generator=_gen(seed, "incl", b, h))
+            out[b, h] = lo + (1.0 - lo) * u
+    return out
