@@ -102,10 +102,24 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// Non-blocking test of phase `parity` (test_wait returns at once; try_wait may first suspend).
+__device__ __forceinline__ bool mbar_peek(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 // Wait for phase `parity` of `bar`.  Returns false (and raises *abort) when the wait gave up
-// or another role of the CTA already aborted.
+// or another role of the CTA already aborted.  A phase that has already completed is seen by
+// the non-blocking test; otherwise the thread waits in try_wait.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           int* status) {
+  if (mbar_peek(bar, parity)) return true;
   unsigned long long t0 = 0;
   for (unsigned int it = 0; it < kWaitPolls; ++it) {
     if (mbar_test(bar, parity)) return true;
