@@ -8,11 +8,13 @@
 // One CTA per (item, 128-cluster chunk), in chunk-major order, writes the chunk as 128 bf16 rows
 // of d = 128 (the layout a TMA tile load reads) followed by the 128 fp32 beta values.
 //
+// Phase 0: the item's selected blocks are validated once into shared memory (tiles of kThreads).
 // Phase 1: thread (row, h) looks the row up in half h of the selected blocks (seg_idx: the entry
 // of the cluster in the block, or 0xFF) with batches of independent loads, keeping the first
-// kSlots entries of its half in block order and the half's selected count.  Phase 2: each warp
-// builds 16 rows with lanes over d (coalesced 512-byte rows): S_c minus the entries' value sums
-// (slot k of both halves before slot k + 1: a fixed order), times 1 / n^U_c.
+// kSlots entries of its half in block order and the half's selected count.  The two halves'
+// entries are then merged per row, slot k of both halves before slot k + 1 (a fixed order).
+// Phase 2: each warp builds 16 rows with lanes over d (coalesced 512-byte rows): S_c minus the
+// entries' value sums in merged order, times 1 / n^U_c.
 #include "da_common.cuh"
 #include "da_internal.h"
 
@@ -30,14 +32,21 @@ constexpr int kChunkBytes = kRows * kD * 2 + kRows * 4;
 
 struct Smem {
   uint32_t ptr[2][kRows][kSlots];        // entry rows (block row * block + entry), block order
+  uint32_t lst[kRows][2 * kSlots];       // both halves' kept entries, merged slot-major
   int nm[2][kRows];                      // entries of the row in each half of the selected blocks
   int csel[2][kRows];                    // selected keys of the cluster in each half
+  int ne[kRows];                         // merged entries of the row
   float inv[kRows];                      // 1 / n^U (0 when n^U = 0)
+  int jsel[kThreads];                    // a tile of the selected blocks, -1 where out of range
 };
 
 __device__ __forceinline__ float4 ldg4(const float* p) { return __ldg(reinterpret_cast<const float4*>(p)); }
 
-__global__ void __launch_bounds__(kThreads, 5)
+__device__ __forceinline__ void add4(float4& a, const float4& y) {
+  a.x += y.x; a.y += y.y; a.z += y.z; a.w += y.w;
+}
+
+__global__ void __launch_bounds__(kThreads, 4)
 comp_build_kernel(StatsPtrs st, const int32_t* __restrict__ kv_idx, const int32_t* __restrict__ kv_cnt,
                   int max_sel, int N, int C, int nB, int block, int nchunk, uint8_t* __restrict__ out) {
   __shared__ Smem sm;
@@ -53,27 +62,37 @@ comp_build_kernel(StatsPtrs st, const int32_t* __restrict__ kv_idx, const int32_
   const int32_t* row = kv_idx + (size_t)item * max_sel;
   const size_t hb = (size_t)bh * nB;                   // first block row of the head
   const size_t hc = (size_t)bh * C;                    // first cluster row of the head
+  const uint8_t* seg_idx_h = st.seg_idx + hb * C;      // the head's lookup rows (nB * C < 2^31)
+  const int32_t* blk_hist_h = st.blk_hist + hb * C;
+  const uint32_t eb = (uint32_t)(hb * block);          // first entry row of the head
   uint8_t* chunk = out + ((size_t)item * nchunk + c) * kChunkBytes;
 
-  {
-    const int rr = t & (kRows - 1), h = t / kRows;
-    const int r = c * kRows + rr;
-    const bool rl = r < C;
-    const int mid = (nsel + 1) >> 1;
-    const int sb = h ? mid : 0, se = h ? nsel : mid;
-    int nm = 0, cs = 0;
-    for (int s0 = sb; s0 < se; s0 += kBatch) {
+  const int rr = t & (kRows - 1), h = t / kRows;
+  const int r = c * kRows + rr;
+  const bool rl = r < C;
+  const int mid = (nsel + 1) >> 1;
+  const int sb = h ? mid : 0, se = h ? nsel : mid;
+  int nm = 0, cs = 0;
+  for (int t0 = 0; t0 < nsel; t0 += kThreads) {        // CTA-uniform
+    __syncthreads();                                   // the previous tile has been read
+    if (t0 + t < nsel) {
+      const int jr = __ldg(row + t0 + t);
+      sm.jsel[t] = (jr >= 0 && jr < nB) ? jr : -1;
+    }
+    __syncthreads();
+    const int lo = max(sb, t0), hi = min(se, t0 + kThreads);
+    for (int s0 = lo; s0 < hi; s0 += kBatch) {
       int e[kBatch], hv[kBatch];
       uint32_t bb[kBatch];
 #pragma unroll
       for (int u = 0; u < kBatch; ++u) {
         const int sidx = s0 + u;
-        const int jr = sidx < se ? __ldg(row + sidx) : -1;
-        const bool ok = rl && jr >= 0 && jr < nB;
-        const size_t bj = hb + (ok ? jr : 0);
-        bb[u] = (uint32_t)(bj * block);
-        e[u] = ok ? (int)__ldg(st.seg_idx + bj * C + r) : 0xFF;
-        hv[u] = ok ? __ldg(st.blk_hist + bj * C + r) : 0;
+        const int jr = sidx < hi ? sm.jsel[sidx - t0] : -1;
+        const bool ok = rl && jr >= 0;
+        const int o = ok ? jr * C + r : 0;
+        bb[u] = eb + (uint32_t)(jr * block);
+        e[u] = ok ? (int)__ldg(seg_idx_h + o) : 0xFF;
+        hv[u] = ok ? __ldg(blk_hist_h + o) : 0;
       }
 #pragma unroll
       for (int u = 0; u < kBatch; ++u) {
@@ -84,67 +103,66 @@ comp_build_kernel(StatsPtrs st, const int32_t* __restrict__ kv_idx, const int32_
         cs += hv[u];                                     // zero where the cluster is absent
       }
     }
-    sm.nm[h][rr] = nm;
-    sm.csel[h][rr] = cs;
   }
+  sm.nm[h][rr] = nm;
+  sm.csel[h][rr] = cs;
   __syncthreads();
   if (t < kRows) {
-    const int r = c * kRows + t;
-    const int nU = r < C ? st.n_tot[hc + r] - sm.csel[0][t] - sm.csel[1][t] : 0;
+    const int rc = c * kRows + t;
+    const int nU = rc < C ? st.n_tot[hc + rc] - sm.csel[0][t] - sm.csel[1][t] : 0;
     sm.inv[t] = nU > 0 ? 1.f / (float)nU : 0.f;
     reinterpret_cast<float*>(chunk + kRows * kD * 2)[t] = nU > 0 ? log2f((float)nU) : -INFINITY;
+    const int a0 = min(sm.nm[0][t], kSlots), a1 = min(sm.nm[1][t], kSlots);
+    int n = 0;
+#pragma unroll
+    for (int k = 0; k < kSlots; ++k) {
+      if (k < a0) sm.lst[t][n++] = sm.ptr[0][t][k];
+      if (k < a1) sm.lst[t][n++] = sm.ptr[1][t][k];
+    }
+    sm.ne[t] = n;
   }
   __syncthreads();
 
   const int w = t >> 5, lane = t & 31;
+  const float* vs = st.seg_vsum + 4 * lane;
   for (int i0 = 0; i0 < 16; i0 += kGroup) {
-    float4 a[kGroup];
-    int nmq[2][kGroup];
+    float4 a[kGroup], acc[kGroup];
+    int ne[kGroup];
+    int emax = 0;
 #pragma unroll
     for (int q = 0; q < kGroup; ++q) {
       const int i = 16 * w + i0 + q;
-      const int r = c * kRows + i;
-      nmq[0][q] = sm.nm[0][i];
-      nmq[1][q] = sm.nm[1][i];
-      a[q] = r < C ? ldg4(st.S_tot + (hc + r) * kD + 4 * lane) : make_float4(0.f, 0.f, 0.f, 0.f);
+      const int rc = c * kRows + i;
+      ne[q] = sm.ne[i];
+      emax = max(emax, ne[q]);
+      a[q] = rc < C ? ldg4(st.S_tot + (hc + rc) * kD + 4 * lane) : make_float4(0.f, 0.f, 0.f, 0.f);
+      acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    float4 acc[kGroup];
+    for (int e = 0; e < emax; ++e) {                     // warp-uniform
+      float4 y[kGroup];
 #pragma unroll
-    for (int q = 0; q < kGroup; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int q = 0; q < kGroup; ++q)
+        if (e < ne[q]) y[q] = ldg4(vs + (size_t)sm.lst[16 * w + i0 + q][e] * kD);
 #pragma unroll
-    for (int k = 0; k < kSlots; ++k) {
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-#pragma unroll
-        for (int q = 0; q < kGroup; ++q) {
-          if (nmq[h][q] > k) {                           // warp-uniform
-            const float4 y = ldg4(st.seg_vsum + (size_t)sm.ptr[h][16 * w + i0 + q][k] * kD + 4 * lane);
-            acc[q].x += y.x; acc[q].y += y.y; acc[q].z += y.z; acc[q].w += y.w;
-          }
-        }
-      }
+      for (int q = 0; q < kGroup; ++q)
+        if (e < ne[q]) add4(acc[q], y[q]);
     }
 #pragma unroll
     for (int q = 0; q < kGroup; ++q) {
       const int i = 16 * w + i0 + q;
-      const int r = c * kRows + i;
+      const int rc = c * kRows + i;
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        if (nmq[h][q] <= kSlots) continue;               // warp-uniform
+      for (int hh = 0; hh < 2; ++hh) {
+        if (sm.nm[hh][i] <= kSlots) continue;            // warp-uniform
         // rare: the cluster sits in more than kSlots blocks of this half; the rest, in block order
-        const int mid = (nsel + 1) >> 1;
-        const int sb = h ? mid : 0, se = h ? nsel : mid;
+        const int hb0 = hh ? mid : 0, he = hh ? nsel : mid;
         int seen = 0;
-        for (int sidx = sb; sidx < se; ++sidx) {
+        for (int sidx = hb0; sidx < he; ++sidx) {
           const int jr = row[sidx];
           if (jr < 0 || jr >= nB) continue;
-          const size_t bj = hb + jr;
-          const int e = st.seg_idx[bj * C + r];
-          if (e == 0xFF) continue;
-          if (seen++ >= kSlots) {
-            const float4 y = ldg4(st.seg_vsum + (bj * block + e) * kD + 4 * lane);
-            acc[q].x += y.x; acc[q].y += y.y; acc[q].z += y.z; acc[q].w += y.w;
-          }
+          const int ei = seg_idx_h[jr * C + rc];
+          if (ei == 0xFF) continue;
+          if (seen++ >= kSlots) add4(acc[q], ldg4(vs + (size_t)(eb + (uint32_t)(jr * block + ei)) * kD));
         }
       }
       const float iv = sm.inv[i];
@@ -166,7 +184,7 @@ cudaError_t launch_comp_build(const Dims& g, const int32_t* kv_idx, const int32_
                               const StatsPtrs& st, void* out, cudaStream_t s) {
   const int nchunk = (g.C + kRows - 1) / kRows;
   const long long ctas = (long long)g.B * g.H * g.nB * nchunk;
-  if (ctas >= (1LL << 31)) return cudaErrorInvalidValue;
+  if (ctas >= (1LL << 31) || (long long)g.nB * g.C >= (1LL << 31)) return cudaErrorInvalidValue;
   comp_build_kernel<<<(unsigned)ctas, kThreads, 0, s>>>(st, kv_idx, kv_cnt, max_sel, g.N, g.C, g.nB, g.block, nchunk,
                                                         static_cast<uint8_t*>(out));
   return cudaGetLastError();
