@@ -32,10 +32,11 @@ import workloads as W
 ROOT = os.path.dirname(os.path.abspath(__file__))
 METRIC = "effective TFLOP/s & ms/call of reassign+fused sparse attn; % of bf16 TC peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# DRAM bytes (read + write) per launch of attention_tc_kernel at the 40-head workload: an ncu
-# capture of this kernel version on a 4-head cut of the same workload (695.9 MB), times 10 (work
-# and bytes are per head).  Set back to None whenever the kernel changes until it is re-captured.
-ATTENTION_TRAFFIC_BYTES = 6.959e9
+# DRAM bytes (read + write) per launch of attention_tc_kernel, by (workload, heads): an ncu
+# capture of this kernel version on a 4-head cut of the Wan2.1-14B workload (686.6 MB), times 10
+# (work and bytes are per head).  Other workloads report null.  Remove an entry whenever the
+# kernel changes, until it is re-captured.
+ATTENTION_TRAFFIC_BYTES = {("wan14b", 40): 6.866e9}
 
 
 def _peaks():
@@ -211,7 +212,14 @@ def _config(w: W.Workload, args):
                         f"C={w.C} density={w.density}",
             "B": w.B, "H": w.H, "N": w.N, "d": w.d, "block": w.block, "C": w.C, "density": w.density,
             "seed": args.seed, "parallelism": "independent heads per rank (weak)",
-            "l2": "inputs (Q,K,V 2.3 GB at wan14b) exceed the 126 MB L2; no flush between steps"}
+            "l2": _l2_note(w)}
+
+
+def _l2_note(w: W.Workload) -> str:
+    qkv = 3 * w.B * w.H * w.N * w.d * (2 if w.dtype == "bf16" else 4)
+    if qkv > 126e6:
+        return f"inputs (Q, K, V: {qkv / 1e9:.2f} GB) exceed the 126 MB L2; no flush between steps"
+    return f"inputs (Q, K, V: {qkv / 1e6:.1f} MB) fit in the 126 MB L2; steady state, no flush between steps"
 
 
 # ---------------------------------------------------------------------------
@@ -553,7 +561,7 @@ def main():
                          "peak": peak, "unit": "TFLOP/s", "frac": att_tflops / peak,
                          "peak_source": f"{kind} bf16 dense (burst)",
                          "frac_of_sustained": att_tflops / float(peaks.get("bf16_tflops_sustained", peak)),
-                         "traffic": ATTENTION_TRAFFIC_BYTES},
+                         "traffic": ATTENTION_TRAFFIC_BYTES.get((w.name, w.H))},
             "e2e": e2e,
             "gpu_launches": K_steps * LAUNCHES_PER_STEP,
             "clocks": clk.summary(),
