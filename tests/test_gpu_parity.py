@@ -196,6 +196,32 @@ def test_malformed_plan_is_reported_without_fault():
     assert eng.status() == da.STATUS_NAMES.index("DA_ERR_DEVICE_INDEX")
 
 
+def test_plans_longer_than_one_staging_tile():
+    """Rows with more selected blocks than the compensation pre-pass stages at a time (256): every
+    block but every fifth (270), every block (338, dense), and all but the first 10 and last 20
+    (308).  A 12-frame cut of the Wan2.1-14B shape: N = 43200, 338 blocks, the last one 64 keys."""
+    w = W.scaled(W.WORKLOADS["wan14b"], H=1, T=12)
+    assert w.nB == 338
+    inp = W.make_inputs(w, seed=15)
+    nB = w.nB
+    kinds = [np.array([j for j in range(nB) if j % 5 != 0], np.int32),
+             np.arange(nB, dtype=np.int32),
+             np.arange(10, nB - 20, dtype=np.int32)]
+    rows = [kinds[i % 3] for i in range(nB)]
+    inp.plans = [[rows] * w.H] * w.B
+    inp.kv_idx, inp.kv_cnt = _edge_plan(w, rows)
+    eng, O, lse = P.run_gpu(inp)
+    assert eng.status() == 0
+    a = eng.stats.assign.cpu().numpy()[0, 0].astype(np.int64)
+    P.check_attention(inp, 0, 0, O, lse, a, q_blocks=[0, 1, 2, 3, 4, 5, 166, 167, 168, nB - 3, nB - 2, nB - 1])
+    dense_rows = [i for i in range(nB) if i % 3 == 1]
+    q, k, v = (x[0, 0].cuda().float() for x in (inp.Q, inp.K, inp.V))
+    dense = torch.nn.functional.scaled_dot_product_attention(q[None], k[None], v[None])[0]
+    for i in dense_rows:
+        s0, s1 = i * w.block, min(w.N, (i + 1) * w.block)
+        assert (O[0, 0, s0:s1].float() - dense[s0:s1]).abs().max().item() <= P.ATT_TOL["bf16"]
+
+
 # ---------------------------------------------------------------------------
 # full-size workloads, in the launch configuration the benchmark times: sampled outputs
 
