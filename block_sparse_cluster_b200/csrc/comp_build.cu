@@ -184,7 +184,7 @@ cudaError_t launch_comp_build(const Dims& g, const int32_t* kv_idx, const int32_
                               const StatsPtrs& st, void* out, cudaStream_t s) {
   const int nchunk = (g.C + kRows - 1) / kRows;
   const long long ctas = (long long)g.B * g.H * g.nB * nchunk;
-  if (ctas >= (1LL << 31) || (long long)g.nB * g.C >= (1LL << 31)) return cudaErrorInvalidValue;
+  if (ctas >= (1LL << 31) || (long long)g.nB * g.C >= (1LL << 31)) return cudaErrorInvalidValue;   // also refused by the ABI
   comp_build_kernel<<<(unsigned)ctas, kThreads, 0, s>>>(st, kv_idx, kv_cnt, max_sel, g.N, g.C, g.nB, g.block, nchunk,
                                                         static_cast<uint8_t*>(out));
   return cudaGetLastError();

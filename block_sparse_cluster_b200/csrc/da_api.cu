@@ -31,6 +31,8 @@ da_status check_dims(const da_dims* dims, Dims* g) {
   const long long BH = (long long)dims->B * dims->H;
   // work items and block-row indices are int32 on the device
   if (BH * g->nB >= (1LL << 31) || BH * dims->N >= (1LL << 31)) return DA_ERR_SHAPE;
+  // a head's lookup rows (seg_idx, blk_hist: nB x C) are indexed in 32 bits
+  if ((long long)g->nB * dims->C >= (1LL << 31)) return DA_ERR_SHAPE;
   // the tensor-core path addresses block entries (block row x block + entry) in 32 bits
   if (g->bf16 && BH * g->nB * g->block >= (1LL << 32)) return DA_ERR_SHAPE;
   return DA_OK;

@@ -72,6 +72,8 @@ typedef struct {
   int block;       /* block size Bs of the q/kv partition */
   da_dtype dtype;  /* element type of Q, K, V, centroids and O */
 } da_dims;
+/* Size limits, with nB = ceil(N / block); a call outside them returns DA_ERR_SHAPE:
+ * B*H*nB < 2^31, B*H*N < 2^31, nB*C < 2^31, and on the bf16 path B*H*nB*block < 2^32. */
 
 /*
  * Reassign Cache output (DecoupAttn abstract: "reassigns the drifting keys to

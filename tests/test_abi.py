@@ -103,6 +103,11 @@ def test_mask_prepare_rejects_small_schedule():
 
 def test_shape_overflow_rejected():
     assert _call_reassign(_dims(B=64, H=1024, N=1 << 20)) == 2
+    # one head whose lookup rows (nB x C) reach 2^31 entries
+    big = _dims(B=1, H=1, N=1 << 28, C=1024)
+    assert _call_reassign(big) == 2
+    assert da.da_workspace_bytes(big) == 0
+    assert da.da_workspace_bytes(_dims(B=1, H=1, N=(1 << 28) - 128, C=1024)) > 0
 
 
 def test_split_attention_calls_reject_arguments():
