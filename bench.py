@@ -32,11 +32,26 @@ import workloads as W
 ROOT = os.path.dirname(os.path.abspath(__file__))
 METRIC = "effective TFLOP/s & ms/call of reassign+fused sparse attn; % of bf16 TC peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# DRAM bytes (read + write) per launch of attention_tc_kernel, by (workload, heads): an ncu
-# capture of this kernel version on a 4-head cut of the Wan2.1-14B workload (686.6 MB), times 10
-# (work and bytes are per head).  Other workloads report null.  Remove an entry whenever the
-# kernel changes, until it is re-captured.
-ATTENTION_TRAFFIC_BYTES = {("wan14b", 40): 6.866e9}
+ATT_SRC = os.path.join(ROOT, "block_sparse_cluster_b200", "csrc", "attention_tc.cu")
+ATT_PROFILE = os.path.join(ROOT, "profiles", "attention_tc_kernel_wan14b.md")
+
+
+def attention_traffic(w) -> "float | None":
+    """DRAM bytes (read + write) per launch of attention_tc_kernel from the committed ncu summary,
+    whose record line names the workload and the sha1 of the kernel source it was captured from:
+    null for another workload or once the source has changed since the capture."""
+    import hashlib
+    import re
+    try:
+        text = open(ATT_PROFILE).read()
+        sha = hashlib.sha1(open(ATT_SRC, "rb").read()).hexdigest()
+    except OSError:
+        return None
+    m = re.search(r"traffic record: workload=(\w+) heads=(\d+) bytes_per_launch=([0-9.e+]+) "
+                  r"attention_tc\.cu sha1=([0-9a-f]{40})", text)
+    if not m or m.group(1) != w.name or int(m.group(2)) != w.H or m.group(4) != sha:
+        return None
+    return float(m.group(3))
 
 
 def _peaks():
@@ -429,18 +444,15 @@ def main():
     torch.cuda.synchronize(dev)
 
     def step(evs=None):
-        # the three calls of da_attention's public halves; events between them time each kernel
+        # the two calls of a step; an event between them times each
         if evs is not None:
             evs[0].record(stream)
         da.da_reassign(dims, K, V, cent, eng.stats, eng.ws)
         if evs is not None:
             evs[1].record(stream)
-        da.da_compensation(dims, eng.mask, eng.stats, eng.ws)
+        da.da_attention(dims, Q, K, V, eng.mask, cent, eng.stats, 0.0, O, None, eng.ws)
         if evs is not None:
             evs[2].record(stream)
-        da.da_attention_prebuilt(dims, Q, K, V, eng.mask, cent, eng.stats, 0.0, O, None, eng.ws)
-        if evs is not None:
-            evs[3].record(stream)
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -449,7 +461,7 @@ def main():
         raise RuntimeError("device status after warm-up: " + da.da_status_string(eng.status()))
 
     K_steps = args.steps
-    att_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K_steps)]
+    att_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K_steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     _barrier(ws)
     torch.cuda.synchronize(dev)
@@ -464,11 +476,10 @@ def main():
     if st != 0:
         raise RuntimeError("device status after timing: " + da.da_status_string(st))
     ms_local = start.elapsed_time(end) / K_steps
-    step_ms = sorted(e[0].elapsed_time(e[3]) for e in att_ev)
+    step_ms = sorted(e[0].elapsed_time(e[2]) for e in att_ev)
     median_ms_local = step_ms[len(step_ms) // 2]
     reas_ms_local = sum(e[0].elapsed_time(e[1]) for e in att_ev) / K_steps
-    comp_ms_local = sum(e[1].elapsed_time(e[2]) for e in att_ev) / K_steps
-    att_ms_local = sum(e[2].elapsed_time(e[3]) for e in att_ev) / K_steps
+    att_ms_local = sum(e[1].elapsed_time(e[2]) for e in att_ev) / K_steps
     ms = _max_over_ranks(ms_local, ws, dev)
     att_ms = _max_over_ranks(att_ms_local, ws, dev)
     value = ws * eff / (ms * 1e-3) / 1e12
@@ -476,10 +487,10 @@ def main():
     # one cold step: L2 flushed by writing a 256 MB buffer first (the timed steps above run warm)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     flush.fill_(1)
-    cold = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    cold = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
     step(cold)
     torch.cuda.synchronize(dev)
-    cold_ms = _max_over_ranks(cold[0].elapsed_time(cold[3]), ws, dev)
+    cold_ms = _max_over_ranks(cold[0].elapsed_time(cold[2]), ws, dev)
     del flush
     median_ms = _max_over_ranks(median_ms_local, ws, dev)
 
@@ -548,20 +559,25 @@ def main():
         peaks, kind = _peaks()
         peak = float(peaks["bf16_tflops"])
         att_tflops = eff / (att_ms * 1e-3) / 1e12
+        sustained = float(peaks.get("bf16_tflops_sustained", peak))
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws, "steps": K_steps,
             "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
             "config": _config(w, args),
             "pct_of_bf16_peak": 100.0 * (value / ws) / peak,
-            "breakdown_ms": {"reassign": reas_ms_local, "compensation": comp_ms_local, "attention": att_ms_local},
+            "breakdown_ms": {"reassign": reas_ms_local, "attention": att_ms_local},
             "ms_per_step_median": median_ms, "cold_ms_per_step": cold_ms,
             "effective_flop_per_step_per_gpu": eff,
-            "roofline": {"bound": "tensor", "kernel": "attention_tc_kernel (fused exact + compensation attention)", "achieved": att_tflops,
-                         "peak": peak, "unit": "TFLOP/s", "frac": att_tflops / peak,
+            # the dominant kernel: the fused attention (exact blocks, cluster chunks and entry tiles in
+            # one kernel; its call also runs the few-microsecond entry-row count); frac_step is the
+            # whole step (reassign included) against the same peak
+            "roofline": {"bound": "tensor", "kernel": "attention_tc_kernel (fused exact + cluster compensation)",
+                         "achieved": att_tflops, "peak": peak, "unit": "TFLOP/s", "frac": att_tflops / peak,
                          "peak_source": f"{kind} bf16 dense (burst)",
-                         "frac_of_sustained": att_tflops / float(peaks.get("bf16_tflops_sustained", peak)),
-                         "traffic": ATTENTION_TRAFFIC_BYTES.get((w.name, w.H))},
+                         "frac_of_sustained": att_tflops / sustained,
+                         "frac_step": (value / ws) / peak,
+                         "traffic": attention_traffic(w)},
             "e2e": e2e,
             "gpu_launches": K_steps * LAUNCHES_PER_STEP,
             "clocks": clk.summary(),
@@ -575,7 +591,7 @@ def main():
 
 
 # kernels of ours per timed step: reassign (centroid norms, assignment with block statistics,
-# totals) + attention (compensation chunks, fused attention)
+# totals) + attention (entry-row count, fused attention)
 LAUNCHES_PER_STEP = 5
 
 if __name__ == "__main__":

@@ -8,13 +8,20 @@
 // where n^U_c = n_c - sum_{j in sel} n_{c,j} and vbar^U_c = (S_c - sum_{j in sel} S_{c,j}) / n^U_c
 // are the count and mean value of the cluster's keys outside the selected blocks.
 //
-// Work: items (head, q-block) from the plan's work order; a persistent CTA per SM walks
-// items blockIdx.x, blockIdx.x + gridDim.x, ...  An item is a sequence of steps: one per selected
-// block, then one per 128-cluster chunk.  Every step is a 128 x 128 score tile S = Q K^T (K a
-// key block or a centroid chunk) and a P V product (V a value block or the chunk's vbar^U rows).
+// The cluster columns are taken in the per-key correction form, which needs no per-q-block table:
+//   e^{s q.cbar_c} n^U_c vbar^U_c = e^{s q.cbar_c + ln n_c} (S_c / n_c)
+//                                   - sum_{j in sel} e^{s q.cbar_c + ln n_{c,j}} (S_{c,j} / n_{c,j}),
+// and the same with the counts alone for the denominator.  So an item's steps are
+//   - one per selected block (exact keys);
+//   - one per 128-cluster chunk of the head (centroid rows, bias log2 n_c, head-wide means);
+//   - its entry tiles: the entries of its selected blocks, 128 rows at a time (centroid rows,
+//     bias log2 n_e, negated entry means), whose weights leave the running sum.
+// The Reassign Cache writes the chunk and entry operands (compensation tiles, include/da.h);
+// the entry tiles are copied row-run by row-run with bulk copies, as they are stored swizzled.
 //
-// The compensation chunks (vbar^U rows in bf16 and log2 n^U per cluster) of every item are
-// written beforehand by comp_build.cu; here they are loaded like value blocks.
+// Work: items (head, q-block) from the plan's work order; a persistent CTA per SM walks
+// items blockIdx.x, blockIdx.x + gridDim.x, ...  Every step is a 128 x 128 score tile S = Q K^T
+// (K a key block, a centroid chunk or an entry tile) and a P V product.
 //
 // Inclusion-probability mode (AB-Attention abstract: sampled blocks "reweighted by inverse
 // inclusion probability"): with p.incl, an item's steps are its selected blocks only (one fully
@@ -29,11 +36,11 @@
 //              P written back to TMEM as bf16.  At the end of the item the two exchange their
 //              (max, sum) per row and each normalises and stores half of the columns of
 //              O = O_0 2^(m_0 - m) + O_1 2^(m_1 - m);
-//   warp 8     producer: loads Q, key tiles / centroid chunks (3-stage ring) and the softmax bias
-//              rows (4-stage ring, so a slot always serves the same warpgroup);
+//   warp 8     producer: loads Q, key tiles / centroid chunks / entry centroid rows (2-stage ring)
+//              and the softmax bias rows (4-stage ring, so a slot always serves the same warpgroup);
 //   warp 9     MMA: allocates TMEM, issues tcgen05.mma S(g+1) = Q K^T ahead of O_X += P(g) V(g);
-//   warp 10    producer of value tiles / compensation chunks (2-stage ring); a warp of its own,
-//              since divergent lanes of one warp waiting on different barriers hold each other up;
+//   warp 10    producer of value tiles / cluster means / entry means (3-stage ring); a warp of its
+//              own, since divergent lanes of one warp waiting on different barriers hold each other up;
 //   warp 11    idle (it completes the third warpgroup, whose registers go to the softmax).
 // TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,384), O_1 [384,512).
 //
@@ -52,7 +59,7 @@ constexpr int kD = 128;
 constexpr int kBM = 128;                 // query rows per item
 constexpr int kBN = 128;                 // keys per block / clusters per chunk
 constexpr int kKStages = 2;             // key / centroid tiles (freed as soon as S is computed)
-constexpr int kVStages = 3;             // value / vbar^U tiles (freed after P V)
+constexpr int kVStages = 3;             // value / mean tiles (freed after P V)
 constexpr int kBStages = 4;             // bias rows of the softmax (even: a slot serves one warpgroup)
 constexpr int kTile = kBN * kD * 2;      // 32 KB bf16 tile
 constexpr int kPanel = kBN * 128;        // one 64-column panel (128 rows x 128 B)
@@ -66,7 +73,7 @@ constexpr int kWarpProducerV = 10;
 constexpr int kRegSoftmax = 232, kRegIssue = 40;
 static_assert(128 * (2 * kRegSoftmax + kRegIssue) <= kThreads * 168, "register split above the launch");
 static_assert(kBStages % 2 == 0, "a bias slot must always serve the same softmax warpgroup");
-constexpr int kChunkBytes = kTile + kBN * 4;   // compensation chunk: vbar^U rows, then log2 n^U
+static_assert(kEntRows == kBN && kEntPanel == (size_t)kPanel, "entry tiles are read as key / value tiles");
 
 struct __align__(8) Bars {
   uint64_t q_full, q_empty;
@@ -80,7 +87,8 @@ struct __align__(8) Bars {
   uint64_t xch_full[2][2];
   uint32_t tmem_base;
   int abort;
-  int bflag[kBStages];                   // 1: the slot's bias row is all zero (a full key block)
+  int bflag[kBStages];                   // bit 0: the bias row is all zero (a full key block);
+                                         // bit 1: an entry tile (its weights leave the sum)
   float2 xch[2][2][kBM];                 // [item parity][warpgroup][row] = (max, sum)
 };
 
@@ -93,13 +101,15 @@ struct Params {
   const int32_t* kv_cnt;
   const int32_t* schedule;
   int max_sel;
-  StatsPtrs st;
+  const int32_t* seg_n;                  // entries per key block (from the Reassign Cache)
+  const int32_t* ent_rows;               // [items] entry rows an item streams (entry_rows_kernel)
+  const uint8_t* ent;                    // entry tiles, kEntTileBytes per (head, key block)
+  const float* cbias;                    // [BH][cpad] log2 n_c
   __nv_bfloat16* O;
   float* lse;
   int* status;
-  const uint8_t* comp;                   // [items][nchunk] compensation chunks of kChunkBytes
   const float* incl;                     // [items][max_sel] inclusion probabilities, or NULL
-  int N, C, nB, n_items, nchunk;
+  int N, C, nB, n_items, nchunk, cpad;
   float scale_log2;
 };
 
@@ -109,9 +119,15 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// Rows of key block j's entry tile that an item streams: its entries, padded to a multiple of 8.
+__device__ __forceinline__ int ent_rows_of(const int32_t* seg_n, int nB, int bh, int j) {
+  const int e = __ldg(seg_n + (size_t)bh * nB + j);
+  return (min(max(e, 0), kBN) + 7) & ~7;
+}
+
 // Item geometry shared by every role.
 struct Item {
-  int bh, i, q0, qlen, nsel, T;
+  int bh, i, q0, qlen, nsel, erows, T;
   const int32_t* row;
 };
 
@@ -126,7 +142,8 @@ __device__ __forceinline__ Item item_at(const Params& p, int k) {
   int cnt = p.kv_cnt[item];
   if (cnt < 0 || cnt > p.max_sel) cnt = 0;
   it.nsel = cnt;
-  it.T = p.incl ? max(cnt, 1) : cnt + p.nchunk;
+  it.erows = p.incl ? 0 : max(0, p.ent_rows[item]);
+  it.T = p.incl ? max(cnt, 1) : cnt + p.nchunk + (it.erows + kBN - 1) / kBN;
   it.row = p.kv_idx + (size_t)item * p.max_sel;
   return it;
 }
@@ -138,8 +155,28 @@ __device__ __forceinline__ int block_of(const Params& p, const Item& it, int s, 
   return *valid ? j : 0;
 }
 
-__device__ __forceinline__ const uint8_t* comp_chunk(const Params& p, const Item& it, int c) {
-  return p.comp + ((size_t)(it.bh * p.nB + it.i) * p.nchunk + c) * kChunkBytes;
+// One entry tile of `rows` rows: walks the item's selected blocks from the cursor (slot cs,
+// source row cr of that block's entry tile) and calls emit(dst_row, block, src_row, nrows) for
+// each run of rows, until the tile holds `rows` rows or the list ends.  Runs are multiples of 8
+// rows, so each lands on the 1024-byte swizzle period it was stored for.
+template <class F>
+__device__ __forceinline__ void ent_tile_walk(const Params& p, const Item& it, int rows, int& cs, int& cr, F&& emit) {
+  int r0 = 0;
+  while (r0 < rows && cs < it.nsel) {
+    bool valid;
+    const int j = block_of(p, it, cs, &valid);
+    const int e8 = valid ? ent_rows_of(p.seg_n, p.nB, it.bh, j) : 0;
+    const int take = min(e8 - cr, rows - r0);
+    if (take > 0) {
+      emit(r0, j, cr, take);
+      r0 += take;
+      cr += take;
+    }
+    if (cr >= e8) {
+      ++cs;
+      cr = 0;
+    }
+  }
 }
 
 // Orders later uses of r after a tcgen05.wait::ld already issued (emits no instruction).
@@ -210,7 +247,7 @@ __device__ __forceinline__ void chunk_exp(const uint32_t (&x)[32], uint64_t coef
 __global__ void __launch_bounds__(kThreads, 1)
 attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_c,
-                    const __grid_constant__ CUtensorMap tm_p, const Params p) {
+                    const __grid_constant__ CUtensorMap tm_m, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -250,6 +287,11 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     bars->abort = 0;
     fence_mbar_init();
   }
+  // Zero the key and value rings once: the rows past the end of an item's last entry tile keep
+  // whatever an earlier step left there (their bias is -inf, so P is 0 there), which must be finite.
+  for (int i = tid; i < (kKStages + kVStages) * kTile / 16; i += kThreads)
+    reinterpret_cast<uint4*>(sK)[i] = make_uint4(0u, 0u, 0u, 0u);
+  fence_async_smem();
   if (warp == kWarpMMA) {
     tmem_alloc(&bars->tmem_base, 512);
     tmem_relinquish();
@@ -275,6 +317,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       int n = 0, nq = 0;                 // items walked, query tiles loaded
       for (int k = blockIdx.x; k < p.n_items && !*abort; k += gridDim.x, ++n) {
         const Item it = item_at(p, k);
+        int cs = 0, cr = 0;                // entry cursor: selected slot, source row
         if (!mbar_wait(&bars->q_empty, (n & 1) ^ 1, abort, status)) break;
         ++nq;
         mbar_expect_tx(&bars->q_full, kTile);
@@ -310,7 +353,8 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                                    c + 2 < ncol ? w : -INFINITY, c + 3 < ncol ? w : -INFINITY);
             }
             mbar_arrive(&bars->b_full[bs]);
-          } else {
+          } else if (s < it.nsel + p.nchunk) {
+            // cluster chunk: centroid rows, bias log2 n_c
             const int c = s - it.nsel;
             mbar_expect_tx(&bars->k_full[ks], kTile);
             tma_load_3d(dk, &tm_c, &bars->k_full[ks], 0, c * kBN, it.bh);
@@ -318,7 +362,24 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             if (!mbar_wait(&bars->b_empty[bs], ((g / kBStages) & 1) ^ 1, abort, status)) { ok = false; break; }
             bars->bflag[bs] = 0;
             mbar_expect_tx(&bars->b_full[bs], kBN * 4);
-            bulk_load(sBias + bs * kBN, comp_chunk(p, it, c) + kTile, kBN * 4, &bars->b_full[bs]);
+            bulk_load(sBias + bs * kBN, p.cbias + (size_t)it.bh * p.cpad + c * kBN, kBN * 4, &bars->b_full[bs]);
+          } else {
+            // entry tile: centroid rows and bias log2 n_e of the selected blocks' entries; the rows
+            // past the item's last entry are masked (-inf, generic stores published by the arrive)
+            const int t = s - it.nsel - p.nchunk;
+            const int rows = min(kBN, it.erows - t * kBN);
+            if (!mbar_wait(&bars->b_empty[bs], ((g / kBStages) & 1) ^ 1, abort, status)) { ok = false; break; }
+            bars->bflag[bs] = 2;
+            float* bb = sBias + bs * kBN;
+            for (int c = rows; c < kBN; ++c) bb[c] = -INFINITY;
+            mbar_expect_tx(&bars->k_full[ks], rows * 256);
+            mbar_expect_tx(&bars->b_full[bs], rows * 4);
+            ent_tile_walk(p, it, rows, cs, cr, [&](int r0, int j, int sr, int nr) {
+              const uint8_t* src = p.ent + ((size_t)it.bh * p.nB + j) * kEntTileBytes;
+              bulk_load(dk + r0 * 128, src + sr * 128, nr * 128, &bars->k_full[ks]);
+              bulk_load(dk + kPanel + r0 * 128, src + kEntPanel + sr * 128, nr * 128, &bars->k_full[ks]);
+              bulk_load(bb + r0, src + kEntBiasOff + sr * 4, nr * 4, &bars->b_full[bs]);
+            });
           }
         }
         if (!ok) break;
@@ -335,11 +396,12 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     // ------------------------------------------------------------------ producer (values)
     if (lane == 0) {
       tma_prefetch(&tm_v);
-      tma_prefetch(&tm_p);
+      tma_prefetch(&tm_m);
       uint32_t g = 0;
       int n = 0;
       for (int k = blockIdx.x; k < p.n_items && !*abort; k += gridDim.x, ++n) {
         const Item it = item_at(p, k);
+        int cs = 0, cr = 0;                // entry cursor: selected slot, source row
         bool ok = true;
         for (int s = 0; s < it.T; ++s, ++g) {
           const int vs = g % kVStages;
@@ -351,11 +413,22 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             mbar_expect_tx(&bars->v_full[vs], kTile);
             tma_load_3d(dv, &tm_v, &bars->v_full[vs], 0, j * kBN, it.bh);
             tma_load_3d(dv + kPanel, &tm_v, &bars->v_full[vs], 64, j * kBN, it.bh);
-          } else {
-            const int z = (it.bh * p.nB + it.i) * p.nchunk + (s - it.nsel);
+          } else if (s < it.nsel + p.nchunk) {
+            // cluster chunk: the head-wide means S_c / n_c (rows past C read as zero)
+            const int c = s - it.nsel;
             mbar_expect_tx(&bars->v_full[vs], kTile);
-            tma_load_3d(dv, &tm_p, &bars->v_full[vs], 0, 0, z);
-            tma_load_3d(dv + kPanel, &tm_p, &bars->v_full[vs], 64, 0, z);
+            tma_load_3d(dv, &tm_m, &bars->v_full[vs], 0, c * kBN, it.bh);
+            tma_load_3d(dv + kPanel, &tm_m, &bars->v_full[vs], 64, c * kBN, it.bh);
+          } else {
+            // entry tile: the negated entry means, the same runs as the producer of keys
+            const int t = s - it.nsel - p.nchunk;
+            const int rows = min(kBN, it.erows - t * kBN);
+            mbar_expect_tx(&bars->v_full[vs], rows * 256);
+            ent_tile_walk(p, it, rows, cs, cr, [&](int r0, int j, int sr, int nr) {
+              const uint8_t* src = p.ent + ((size_t)it.bh * p.nB + j) * kEntTileBytes + kEntVOff;
+              bulk_load(dv + r0 * 128, src + sr * 128, nr * 128, &bars->v_full[vs]);
+              bulk_load(dv + kPanel + r0 * 128, src + kEntPanel + sr * 128, nr * 128, &bars->v_full[vs]);
+            });
           }
         }
         if (!ok) break;
@@ -448,11 +521,12 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         tc_fence_after();
         // The S row is loaded from TMEM once (128 registers): the row max, then p = 2^(y - m), the
         // row sum and the bf16 P written back over S.  Column c's logit is y_c = x_c * s*log2(e) +
-        // bias_c, the bias row in shared memory: log2 n^U_c on a compensation step, 0 on a key
-        // block (-inf past the end of a short last block).
+        // bias_c, the bias row in shared memory: log2 n_c on a cluster chunk, log2 n_e on an entry
+        // tile, 0 on a key block (-inf past the end of a short last block or of the entries).
         const uint32_t sbase = lane_addr + X * kBN;
         const float* bt = sBias + bs * kBN;
-        const bool plain = bars->bflag[bs] != 0 && p.scale_log2 > 0.f;
+        const int flag = bars->bflag[bs];
+        const bool plain = (flag & 1) && p.scale_log2 > 0.f;
         uint32_t x[4][32];
         tmem_ld32(sbase, x[0]);
         tmem_ld32(sbase + 32, x[1]);
@@ -505,7 +579,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           }
         }
         m = m_new;
-        l += rs;
+        l += (flag & 2) ? -rs : rs;               // entry tiles take their weight out again
         first = false;
         ++u;
         tmem_wait_st();
@@ -572,42 +646,68 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   }
 }
 
+// Entry rows each item streams (the sum over its valid selected blocks of ent_rows_of), so that
+// every role knows an item's step count without walking its list.  A warp per item.
+__global__ void __launch_bounds__(256) entry_rows_kernel(const int32_t* __restrict__ kv_idx,
+                                                         const int32_t* __restrict__ kv_cnt, int max_sel,
+                                                         const int32_t* __restrict__ seg_n, int nB, int n_items,
+                                                         int32_t* __restrict__ out) {
+  const int item = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (item >= n_items) return;
+  int cnt = kv_cnt[item];
+  if (cnt < 0 || cnt > max_sel) cnt = 0;
+  const int bh = item / nB;
+  const int32_t* row = kv_idx + (size_t)item * max_sel;
+  int sum = 0;
+  for (int s = lane; s < cnt; s += 32) {
+    const int j = row[s];
+    if (j >= 0 && j < nB) sum += ent_rows_of(seg_n, nB, bh, j);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if (lane == 0) out[item] = sum;
+}
+
 }  // namespace
 
 bool attention_tc_supported(const Dims& g) { return g.bf16 && g.d == kD && g.block == kBN; }
 
-size_t attention_tc_scratch_bytes(const Dims& g) {
-  if (!attention_tc_supported(g)) return 0;
-  return (size_t)g.B * g.H * g.nB * ((g.C + kBN - 1) / kBN) * kChunkBytes;
-}
-
 cudaError_t launch_attention_tc(const Dims& g, const void* Q, const void* K, const void* V,
                                 const int32_t* kv_idx, const int32_t* kv_cnt, int max_sel,
                                 const int32_t* schedule, const void* cent, const StatsPtrs& st, float scale,
-                                void* O, float* lse, int* status, void* comp, const float* incl, cudaStream_t s) {
-  CUtensorMap tq, tk, tv, tc, tp;
+                                void* O, float* lse, int* status, int32_t* ent_rows, const float* incl,
+                                cudaStream_t s) {
+  CUtensorMap tq, tk, tv, tc, tm;
   const unsigned long long BH = (unsigned long long)g.B * g.H;
-  const int nchunk = (g.C + kBN - 1) / kBN;
+  const CompLayout L = comp_layout(g);
+  // without compensation tiles (the inclusion-probability mode) K stands in for the cluster means
+  const void* cmean = (!incl && st.comp) ? static_cast<const void*>(st.comp + L.cmean) : K;
+  const unsigned long long mean_rows = (!incl && st.comp) ? (unsigned long long)g.C : (unsigned long long)g.N;
+  if (!incl && !st.comp) return cudaErrorInvalidValue;
   if (!make_tmap_bf16_3d(&tq, Q, kD, g.N, BH, 64, kBM) || !make_tmap_bf16_3d(&tk, K, kD, g.N, BH, 64, kBN) ||
       !make_tmap_bf16_3d(&tv, V, kD, g.N, BH, 64, kBN) || !make_tmap_bf16_3d(&tc, cent, kD, g.C, BH, 64, kBN) ||
-      !make_tmap_bf16_tiles(&tp, comp, kD, kBN, BH * g.nB * nchunk, kChunkBytes, kBN))
+      !make_tmap_bf16_3d(&tm, cmean, kD, mean_rows, BH, 64, kBN))
     return cudaErrorInvalidValue;
   Params p;
   p.kv_idx = kv_idx;
   p.kv_cnt = kv_cnt;
   p.schedule = schedule;
   p.max_sel = max_sel;
-  p.st = st;
+  p.seg_n = st.seg_n;
+  p.ent_rows = ent_rows;
+  p.ent = st.comp ? st.comp + L.ent : nullptr;
+  p.cbias = st.comp ? reinterpret_cast<const float*>(st.comp + L.cbias) : nullptr;
   p.O = (__nv_bfloat16*)O;
   p.lse = lse;
   p.status = status;
-  p.comp = static_cast<const uint8_t*>(comp);
   p.incl = incl;
   p.N = g.N;
   p.C = g.C;
   p.nB = g.nB;
   p.n_items = (int)(BH * g.nB);
-  p.nchunk = nchunk;
+  p.nchunk = (g.C + kBN - 1) / kBN;
+  p.cpad = L.cpad;
   p.scale_log2 = scale * 1.4426950408889634f;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
@@ -615,8 +715,14 @@ cudaError_t launch_attention_tc(const Dims& g, const void* Q, const void* K, con
   cudaError_t e = cudaFuncSetAttribute(attention_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kSmemBytes);
   if (e != cudaSuccess) return e;
+  if (!incl) {
+    entry_rows_kernel<<<(p.n_items + 7) / 8, 256, 0, s>>>(kv_idx, kv_cnt, max_sel, st.seg_n, g.nB, p.n_items,
+                                                          ent_rows);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
   const int grid = min(sms, p.n_items);
-  attention_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, tc, tp, p);
+  attention_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, tc, tm, p);
   return cudaGetLastError();
 }
 

@@ -56,32 +56,21 @@ extern "C" DA_API da_status da_reassign_noalloc(const da_dims* dims, const void*
                                                 const void* centroids, const da_cluster_stats* out,
                                                 da_stream stream) {
   using namespace da;
-  if (!dims || !K || !V || !centroids || !out) return DA_ERR_INVALID_ARG;
-  if (dims->B <= 0 || dims->H <= 0 || dims->N <= 0 || dims->d <= 0 || dims->C <= 0 || dims->block <= 0)
-    return DA_ERR_INVALID_ARG;
-  if (dims->dtype != DA_BF16 && dims->dtype != DA_F32) return DA_ERR_DTYPE;
-  if (dims->d != 64 && dims->d != 128) return DA_ERR_UNSUPPORTED;
-  if (dims->block != 64 && dims->block != 128) return DA_ERR_UNSUPPORTED;
-  if (dims->C % 32 != 0 || dims->C > 1024) return DA_ERR_UNSUPPORTED;
-  Dims g{dims->B, dims->H, dims->N, dims->d, dims->C, dims->block, (dims->N + dims->block - 1) / dims->block,
-         dims->dtype == DA_BF16};
-  const long long BH = (long long)g.B * g.H;
-  if (BH * g.nB >= (1LL << 31) || BH * g.N >= (1LL << 31)) return DA_ERR_SHAPE;
-  if ((size_t)BH * g.C > kNoAllocMaxNorms) return DA_ERR_WORKSPACE;   // beyond the built-in scratch
-  const void* ptrs[] = {K, V, centroids, out->assign, out->blk_hist, out->seg_idx, out->seg_n, out->seg_c,
-                        out->seg_cnt, out->seg_vsum, out->n_tot, out->S_tot};
-  for (const void* q : ptrs) {
-    if (!q) return DA_ERR_INVALID_ARG;
-    if (!aligned16(q)) return DA_ERR_ALIGNMENT;
-  }
+  // the same argument checks as da_reassign, then the size of the built-in scratch
+  Dims g;
+  da_status st = check_dims(dims, &g);
+  if (st != DA_OK) return st;
+  if (!K || !V || !centroids) return DA_ERR_INVALID_ARG;
+  if (!aligned16(K) || !aligned16(V) || !aligned16(centroids)) return DA_ERR_ALIGNMENT;
+  StatsPtrs sp;
+  if ((st = check_stats(g, out, &sp)) != DA_OK) return st;
+  if ((size_t)g.B * g.H * g.C > kNoAllocMaxNorms) return DA_ERR_WORKSPACE;   // beyond the built-in scratch
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return DA_ERR_CUDA;
   float* scratch = nullptr;
   if (scratch_address(dev, &scratch) != cudaSuccess) return DA_ERR_CUDA;
   int* status = reinterpret_cast<int*>(scratch);
   float* norms = scratch + kStatusFloats;
-  const StatsPtrs sp{out->assign, out->blk_hist, out->seg_idx, out->seg_n, out->seg_c,
-                     out->seg_cnt, out->seg_vsum, out->n_tot, out->S_tot};
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), s);
   if (e == cudaSuccess) {

@@ -25,6 +25,14 @@ SMALL = {
     "hunyuan_3f": W.scaled(W.WORKLOADS["hunyuan"], H=1, T=3),
     # two batch entries: (batch, head) slices are flattened in every kernel
     "wan13b_b2": W.scaled(W.WORKLOADS["wan13b"], B=2, H=2, T=2),
+    # C not a multiple of 128 on the tensor-core path: one partial chunk (C < 128), a partial last
+    # chunk of 32 centroids, and of 32 again after three full ones (reassign, statistics, attention)
+    "c96": W.scaled(W.WORKLOADS["wan14b"], H=2, T=2, C=96, cells=(2, 6, 8)),
+    "c160": W.scaled(W.WORKLOADS["wan14b"], H=1, T=2, C=160, cells=(2, 8, 10)),
+    "c416": W.scaled(W.WORKLOADS["wan14b"], H=1, T=2, C=416, cells=(2, 13, 16)),
+    # bf16 shapes of the CUDA-core path: d = 64 with block 64, and d = 128 with block 64
+    "bf16_d64": W.scaled(W.WORKLOADS["tiny"], dtype="bf16"),
+    "bf16_block64": W.scaled(W.WORKLOADS["tiny"], d=128, block=64, T=5, Hs=15, C=64, dtype="bf16"),
 }
 
 
@@ -42,6 +50,7 @@ def test_small_case_full_parity(name):
             P.check_assignment(inp, b, h, a)
             P.check_block_stats(inp, b, h, st, a)
             P.check_totals(inp, b, h, st, a)
+            P.check_comp_tiles(inp, b, h, st, a)
             P.check_attention(inp, b, h, O, lse, a)
 
 
@@ -160,20 +169,32 @@ def test_repeat_calls_are_bitwise_identical():
         assert torch.equal(v, getattr(eng.stats, k)), k
 
 
-def test_split_calls_equal_da_attention():
-    """da_compensation followed by da_attention_prebuilt is da_attention, bit for bit."""
-    import block_sparse_cluster_b200 as da
-    w = SMALL["wan14b_2f"]
-    inp = W.make_inputs(w, seed=17)
-    eng, O1, l1 = P.run_gpu(inp)
-    Q, K, V, cent = (x.cuda() for x in (inp.Q, inp.K, inp.V, inp.centroids))
-    O2 = torch.empty_like(O1)
-    l2 = torch.empty_like(l1)
-    da.da_compensation(eng.dims, eng.mask, eng.stats, eng.ws)
-    da.da_attention_prebuilt(eng.dims, Q, K, V, eng.mask, cent, eng.stats, 0.0, O2, l2, eng.ws)
-    torch.cuda.synchronize()
+def test_clusters_mostly_inside_the_selected_blocks():
+    """Every q-block selects all blocks but three, so each cluster keeps only a few of its keys
+    outside the selection (n_c / n^U_c of about 19 on average, and n^U_c = 0 for some clusters):
+    the fused kernel adds each cluster with its head-wide count and takes the selected blocks'
+    entries out again, and the difference must still match the complement form."""
+    w = W.scaled(W.WORKLOADS["wan14b"], H=2, T=2)
+    inp = W.make_inputs(w, seed=19)
+    nB = w.nB
+    rows = [np.array([j for j in range(nB) if j not in {(i + 7) % nB, (i + 19) % nB, (i + 31) % nB}], np.int32)
+            for i in range(nB)]
+    inp.plans = [[rows] * w.H] * w.B
+    inp.kv_idx, inp.kv_cnt = _edge_plan(w, rows)
+    eng, O, lse = P.run_gpu(inp)
     assert eng.status() == 0
-    assert torch.equal(O1, O2) and torch.equal(l1, l2)
+    a = eng.stats.assign.cpu().numpy()
+    n_tot = eng.stats.n_tot.cpu().numpy()
+    ratios = []
+    for h in range(w.H):
+        ah = a[0, h].astype(np.int64)
+        for i in range(0, nB, 7):
+            out = [j for j in range(nB) if j not in set(rows[i].tolist())]
+            n_u = np.bincount(np.concatenate([ah[j * w.block:(j + 1) * w.block] for j in out]), minlength=w.C)
+            live = n_u > 0
+            ratios.append(float((n_tot[0, h][live] / n_u[live]).mean()))
+        P.check_attention(inp, 0, h, O, lse, ah)
+    assert np.mean(ratios) > 10
 
 
 def test_malformed_plan_is_reported_without_fault():
@@ -196,10 +217,11 @@ def test_malformed_plan_is_reported_without_fault():
     assert eng.status() == da.STATUS_NAMES.index("DA_ERR_DEVICE_INDEX")
 
 
-def test_plans_longer_than_one_staging_tile():
-    """Rows with more selected blocks than the compensation pre-pass stages at a time (256): every
-    block but every fifth (270), every block (338, dense), and all but the first 10 and last 20
-    (308).  A 12-frame cut of the Wan2.1-14B shape: N = 43200, 338 blocks, the last one 64 keys."""
+def test_long_plans_with_many_entry_tiles():
+    """Rows with hundreds of selected blocks, so an item streams dozens of entry tiles and its
+    block runs straddle tile boundaries: every block but every fifth (270), every block (338,
+    dense), and all but the first 10 and last 20 (308).  A 12-frame cut of the Wan2.1-14B shape:
+    N = 43200, 338 blocks, the last one 64 keys."""
     w = W.scaled(W.WORKLOADS["wan14b"], H=1, T=12)
     assert w.nB == 338
     inp = W.make_inputs(w, seed=15)
