@@ -64,6 +64,7 @@ constexpr int kBStages = 4;             // bias rows of the softmax (even: a slo
 constexpr int kTile = kBN * kD * 2;      // 32 KB bf16 tile
 constexpr int kPanel = kBN * 128;        // one 64-column panel (128 rows x 128 B)
 constexpr float kRescaleLog2 = 8.0f;     // lazy rescale threshold (factor 256)
+constexpr int kEntSlots = 512;           // selected slots whose entry counts are prefetched
 constexpr int kThreads = 384;           // three warpgroups; warp 11 idle
 constexpr int kWarpProducer = 8;
 constexpr int kWarpMMA = 9;
@@ -90,6 +91,9 @@ struct __align__(8) Bars {
   int bflag[kBStages];                   // bit 0: the bias row is all zero (a full key block);
                                          // bit 1: an entry tile (its weights leave the sum)
   float2 xch[2][2][kBM];                 // [item parity][warpgroup][row] = (max, sum)
+  // entries of the current item's selected blocks, by slot, copied with cp.async by each producer
+  // during its exact steps (one array per producer: the two run independently)
+  int e8[2][kEntSlots];
 };
 
 constexpr size_t kSmemBytes = 1024 + kTile /*Q*/ + (kKStages + kVStages) * kTile /*K,V*/ +
@@ -155,20 +159,38 @@ __device__ __forceinline__ int block_of(const Params& p, const Item& it, int s, 
   return *valid ? j : 0;
 }
 
+// Entry rows of selected slot s: its block's entry count was copied into e8s[s] by cp.async during
+// the slot's exact step (slots beyond kEntSlots, or invalid blocks, are looked up here).
+__device__ __forceinline__ int ent_rows_at(const Params& p, const Item& it, const int* e8s, int s) {
+  bool valid;
+  const int j = block_of(p, it, s, &valid);
+  if (!valid) return 0;
+  if (s < kEntSlots) return (min(max(e8s[s], 0), kBN) + 7) & ~7;
+  return ent_rows_of(p.seg_n, p.nB, it.bh, j);
+}
+
+// Start the asynchronous copy of selected slot s's entry count into e8s[s] (exact step s).
+__device__ __forceinline__ void ent_prefetch(const Params& p, const Item& it, int* e8s, int s, int j, bool valid) {
+  if (s >= kEntSlots || !valid || p.incl) return;
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(e8s + s)),
+               "l"(reinterpret_cast<uint64_t>(p.seg_n + (size_t)it.bh * p.nB + j))
+               : "memory");
+}
+
 // One entry tile of `rows` rows: walks the item's selected blocks from the cursor (slot cs,
 // source row cr of that block's entry tile) and calls emit(dst_row, block, src_row, nrows) for
 // each run of rows, until the tile holds `rows` rows or the list ends.  Runs are multiples of 8
 // rows, so each lands on the 1024-byte swizzle period it was stored for.
 template <class F>
-__device__ __forceinline__ void ent_tile_walk(const Params& p, const Item& it, int rows, int& cs, int& cr, F&& emit) {
+__device__ __forceinline__ void ent_tile_walk(const Params& p, const Item& it, const int* e8s, int rows, int& cs,
+                                              int& cr, F&& emit) {
   int r0 = 0;
   while (r0 < rows && cs < it.nsel) {
-    bool valid;
-    const int j = block_of(p, it, cs, &valid);
-    const int e8 = valid ? ent_rows_of(p.seg_n, p.nB, it.bh, j) : 0;
+    const int e8 = ent_rows_at(p, it, e8s, cs);
     const int take = min(e8 - cr, rows - r0);
     if (take > 0) {
-      emit(r0, j, cr, take);
+      bool valid;
+      emit(r0, block_of(p, it, cs, &valid), cr, take);
       r0 += take;
       cr += take;
     }
@@ -334,6 +356,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             mbar_expect_tx(&bars->k_full[ks], kTile);
             tma_load_3d(dk, &tm_k, &bars->k_full[ks], 0, j * kBN, it.bh);
             tma_load_3d(dk + kPanel, &tm_k, &bars->k_full[ks], 64, j * kBN, it.bh);
+            ent_prefetch(p, it, bars->e8[0], s, j, valid);
             // bias row of a key block: 0 for its keys, -inf past the end of a short last block
             // (generic stores, published to the softmax by the arrive on b_full)
             if (!mbar_wait(&bars->b_empty[bs], ((g / kBStages) & 1) ^ 1, abort, status)) { ok = false; break; }
@@ -374,7 +397,8 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             for (int c = rows; c < kBN; ++c) bb[c] = -INFINITY;
             mbar_expect_tx(&bars->k_full[ks], rows * 256);
             mbar_expect_tx(&bars->b_full[bs], rows * 4);
-            ent_tile_walk(p, it, rows, cs, cr, [&](int r0, int j, int sr, int nr) {
+            if (t == 0) asm volatile("cp.async.wait_all;" ::: "memory");   // counts prefetched at the exact steps
+            ent_tile_walk(p, it, bars->e8[0], rows, cs, cr, [&](int r0, int j, int sr, int nr) {
               const uint8_t* src = p.ent + ((size_t)it.bh * p.nB + j) * kEntTileBytes;
               bulk_load(dk + r0 * 128, src + sr * 128, nr * 128, &bars->k_full[ks]);
               bulk_load(dk + kPanel + r0 * 128, src + kEntPanel + sr * 128, nr * 128, &bars->k_full[ks]);
@@ -413,6 +437,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             mbar_expect_tx(&bars->v_full[vs], kTile);
             tma_load_3d(dv, &tm_v, &bars->v_full[vs], 0, j * kBN, it.bh);
             tma_load_3d(dv + kPanel, &tm_v, &bars->v_full[vs], 64, j * kBN, it.bh);
+            ent_prefetch(p, it, bars->e8[1], s, j, valid);
           } else if (s < it.nsel + p.nchunk) {
             // cluster chunk: the head-wide means S_c / n_c (rows past C read as zero)
             const int c = s - it.nsel;
@@ -424,7 +449,8 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             const int t = s - it.nsel - p.nchunk;
             const int rows = min(kBN, it.erows - t * kBN);
             mbar_expect_tx(&bars->v_full[vs], rows * 256);
-            ent_tile_walk(p, it, rows, cs, cr, [&](int r0, int j, int sr, int nr) {
+            if (t == 0) asm volatile("cp.async.wait_all;" ::: "memory");   // counts prefetched at the exact steps
+            ent_tile_walk(p, it, bars->e8[1], rows, cs, cr, [&](int r0, int j, int sr, int nr) {
               const uint8_t* src = p.ent + ((size_t)it.bh * p.nB + j) * kEntTileBytes + kEntVOff;
               bulk_load(dv + r0 * 128, src + sr * 128, nr * 128, &bars->v_full[vs]);
               bulk_load(dv + kPanel + r0 * 128, src + kEntPanel + sr * 128, nr * 128, &bars->v_full[vs]);

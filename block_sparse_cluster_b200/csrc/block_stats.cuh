@@ -142,6 +142,11 @@ __device__ void block_stats_group(int t, int bar_id, const int* s_assign, int nk
   constexpr int NE = D / 32;
   for (int ee = warp; ee < E; ee += NT / 32) {
     const int p0 = sm.start_pos[ee], p1 = sm.start_pos[ee + 1];
+    // the entry's centroid row for its tile, loaded first so that its latency overlaps the sums
+    uint2 crow = make_uint2(0u, 0u);
+    if constexpr (NE == 4 && sizeof(T) == 2) {
+      if (ent_out) crow = *reinterpret_cast<const uint2*>(cent + (size_t)s_assign[sm.sorted_key[p0]] * 128 + lane * 4);
+    }
     float acc[NE];
 #pragma unroll
     for (int i = 0; i < NE; ++i) acc[i] = 0.f;
@@ -173,10 +178,9 @@ __device__ void block_stats_group(int t, int bar_id, const int* s_assign, int nk
       if (ent_out) {
         // lane l holds columns [4l, 4l + 4): panel l / 16, 16-byte chunk (l mod 16) / 2, half l mod 2
         const int n = p1 - p0;
-        const int c = s_assign[sm.sorted_key[p0]];
         const int k = (lane & 15) >> 1;
         const size_t off = (size_t)(lane >> 4) * kEntPanel + (size_t)ee * 128 + ((k ^ (ee & 7)) << 4) + ((lane & 1) << 3);
-        *reinterpret_cast<uint2*>(ent_out + off) = *reinterpret_cast<const uint2*>(cent + (size_t)c * 128 + lane * 4);
+        *reinterpret_cast<uint2*>(ent_out + off) = crow;
         const float fn = (float)n;
         uint2 vv;
         vv.x = pack_bf16x2(-(acc[0] / fn), -(acc[1] / fn));

@@ -170,11 +170,12 @@ def test_repeat_calls_are_bitwise_identical():
 
 
 def test_clusters_mostly_inside_the_selected_blocks():
-    """Every q-block selects all blocks but three, so each cluster keeps only a few of its keys
-    outside the selection (n_c / n^U_c of about 19 on average, and n^U_c = 0 for some clusters):
-    the fused kernel adds each cluster with its head-wide count and takes the selected blocks'
-    entries out again, and the difference must still match the complement form."""
-    w = W.scaled(W.WORKLOADS["wan14b"], H=2, T=2)
+    """Every q-block selects all blocks but three, and 64 clusters hold about 112 keys each, so a
+    cluster keeps only a few of its keys outside the selection (n_c / n^U_c about 40 on average,
+    up to 128, and n^U_c = 0 for many clusters): the fused kernel adds each cluster with its
+    head-wide count and takes the selected blocks' entries out again, and that difference of large
+    terms must still match the complement form within the bf16 tolerance."""
+    w = W.scaled(W.WORKLOADS["wan14b"], H=2, T=2, C=64, cells=(2, 4, 8))
     inp = W.make_inputs(w, seed=19)
     nB = w.nB
     rows = [np.array([j for j in range(nB) if j not in {(i + 7) % nB, (i + 19) % nB, (i + 31) % nB}], np.int32)
@@ -194,7 +195,7 @@ def test_clusters_mostly_inside_the_selected_blocks():
             live = n_u > 0
             ratios.append(float((n_tot[0, h][live] / n_u[live]).mean()))
         P.check_attention(inp, 0, h, O, lse, ah)
-    assert np.mean(ratios) > 10
+    assert np.mean(ratios) > 20
 
 
 def test_malformed_plan_is_reported_without_fault():
