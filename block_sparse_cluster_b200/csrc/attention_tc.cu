@@ -59,7 +59,7 @@ constexpr int kD = 128;
 constexpr int kBM = 128;                 // query rows per item
 constexpr int kBN = 128;                 // keys per block / clusters per chunk
 constexpr int kKStages = 2;             // key / centroid tiles (freed as soon as S is computed)
-constexpr int kVStages = 3;             // value / mean tiles (freed after P V)
+constexpr int kVStages = 2;             // value / mean tiles (freed after P V)
 constexpr int kBStages = 4;             // bias rows of the softmax (even: a slot serves one warpgroup)
 constexpr int kTile = kBN * kD * 2;      // 32 KB bf16 tile
 constexpr int kPanel = kBN * 128;        // one 64-column panel (128 rows x 128 B)
@@ -75,28 +75,35 @@ constexpr int kRegSoftmax = 232, kRegIssue = 40;
 static_assert(128 * (2 * kRegSoftmax + kRegIssue) <= kThreads * 168, "register split above the launch");
 static_assert(kBStages % 2 == 0, "a bias slot must always serve the same softmax warpgroup");
 static_assert(kEntRows == kBN && kEntPanel == (size_t)kPanel, "entry tiles are read as key / value tiles");
+// TMEM columns: the two score buffers, the one output accumulator, the two bf16 probability tiles
+constexpr uint32_t kColS = 0, kColO = 256, kColP = 384;
 
 struct __align__(8) Bars {
-  uint64_t q_full, q_empty;
+  uint64_t q_full[2], q_empty[2];        // query tile of item n in buffer n & 1
   uint64_t k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
   uint64_t b_full[kBStages], b_empty[kBStages];
-  uint64_t s_full[2], p_ready[2];
-  uint64_t o_done[2], o_free, drain;
-  // (max, sum) published: [item parity][warpgroup].  One barrier per item parity: a warpgroup
-  // without steps in an item could otherwise complete a barrier twice before the other
-  // warpgroup's parity wait on it runs.
+  uint64_t s_full[2];                    // S(g) computed into S_{g & 1}
+  uint64_t s_free[2];                    // softmax has read S_{g & 1} into registers
+  uint64_t p_ready[2];                   // P(g) written into P_{g & 1}
+  uint64_t p_free[2];                    // P(g) V(g) done: P_{g & 1} reusable, O holds step g
+  uint64_t m_pub[2];                     // warpgroup X published its running max of step g
+  uint64_t o_free, drain;
+  // (max, sum) published at the end of an item: [item parity][warpgroup].  One barrier per item
+  // parity: a warpgroup without steps in an item could otherwise complete a barrier twice before
+  // the other warpgroup's parity wait on it runs.
   uint64_t xch_full[2][2];
   uint32_t tmem_base;
   int abort;
   int bflag[kBStages];                   // bit 0: the bias row is all zero (a full key block);
                                          // bit 1: an entry tile (its weights leave the sum)
+  float mrow[2][kBM];                    // [warpgroup][row]: running max of its latest step
   float2 xch[2][2][kBM];                 // [item parity][warpgroup][row] = (max, sum)
   // entries of the current item's selected blocks, by slot, copied with cp.async by each producer
   // during its exact steps (one array per producer: the two run independently)
   int e8[2][kEntSlots];
 };
 
-constexpr size_t kSmemBytes = 1024 + kTile /*Q*/ + (kKStages + kVStages) * kTile /*K,V*/ +
+constexpr size_t kSmemBytes = 1024 + 2 * kTile /*Q*/ + (kKStages + kVStages) * kTile /*K,V*/ +
                               kBStages * kBN * sizeof(float) /*bias*/ + sizeof(Bars);
 static_assert(kSmemBytes <= 232448, "shared memory above the 227 KB per-block limit");
 
@@ -273,8 +280,8 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-  uint8_t* sQ = base;
-  uint8_t* sK = sQ + kTile;                       // kKStages tiles
+  uint8_t* sQ = base;                             // two query tiles
+  uint8_t* sK = sQ + 2 * kTile;                   // kKStages tiles
   uint8_t* sV = sK + kKStages * kTile;            // kVStages tiles
   float* sBias = reinterpret_cast<float*>(sV + kVStages * kTile);   // [kBStages][kBN]
   Bars* bars = reinterpret_cast<Bars*>(sBias + kBStages * kBN);
@@ -283,8 +290,17 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   const int warp = tid >> 5, lane = tid & 31;
 
   if (tid == 0) {
-    mbar_init(&bars->q_full, 1);
-    mbar_init(&bars->q_empty, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars->q_full[b], 1);
+      mbar_init(&bars->q_empty[b], 1);
+      mbar_init(&bars->s_full[b], 1);
+      mbar_init(&bars->s_free[b], 128);
+      mbar_init(&bars->p_ready[b], 128);
+      mbar_init(&bars->p_free[b], 1);
+      mbar_init(&bars->m_pub[b], 128);
+      mbar_init(&bars->xch_full[b][0], 128);
+      mbar_init(&bars->xch_full[b][1], 128);
+    }
     for (int s = 0; s < kKStages; ++s) {
       mbar_init(&bars->k_full[s], 1);
       mbar_init(&bars->k_empty[s], 1);
@@ -296,13 +312,6 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     for (int s = 0; s < kBStages; ++s) {
       mbar_init(&bars->b_full[s], 1);
       mbar_init(&bars->b_empty[s], 128);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&bars->s_full[b], 1);
-      mbar_init(&bars->p_ready[b], 128);
-      mbar_init(&bars->o_done[b], 1);
-      mbar_init(&bars->xch_full[b][0], 128);
-      mbar_init(&bars->xch_full[b][1], 128);
     }
     mbar_init(&bars->o_free, 256);
     mbar_init(&bars->drain, 1);
@@ -330,21 +339,21 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 
   if (warp == kWarpProducer) {
     // ------------------------------------------------------------------ producer (keys)
-    // query tiles, key / centroid tiles and the softmax bias rows
+    // query tiles (double buffered), key / centroid / entry tiles and the softmax bias rows
     if (lane == 0) {
       tma_prefetch(&tm_q);
       tma_prefetch(&tm_k);
       tma_prefetch(&tm_c);
       uint32_t g = 0;
-      int n = 0, nq = 0;                 // items walked, query tiles loaded
-      for (int k = blockIdx.x; k < p.n_items && !*abort; k += gridDim.x, ++n) {
+      int n = 0;                         // items walked = query tiles loaded
+      for (int k = blockIdx.x; k < p.n_items && !*abort; k += gridDim.x) {
         const Item it = item_at(p, k);
         int cs = 0, cr = 0;                // entry cursor: selected slot, source row
-        if (!mbar_wait(&bars->q_empty, (n & 1) ^ 1, abort, status)) break;
-        ++nq;
-        mbar_expect_tx(&bars->q_full, kTile);
-        tma_load_3d(sQ, &tm_q, &bars->q_full, 0, it.q0, it.bh);
-        tma_load_3d(sQ + kPanel, &tm_q, &bars->q_full, 64, it.q0, it.bh);
+        if (!mbar_wait(&bars->q_empty[n & 1], ((n >> 1) & 1) ^ 1, abort, status)) break;
+        mbar_expect_tx(&bars->q_full[n & 1], kTile);
+        tma_load_3d(sQ + (n & 1) * kTile, &tm_q, &bars->q_full[n & 1], 0, it.q0, it.bh);
+        tma_load_3d(sQ + (n & 1) * kTile + kPanel, &tm_q, &bars->q_full[n & 1], 64, it.q0, it.bh);
+        ++n;
         bool ok = true;
         for (int s = 0; s < it.T; ++s, ++g) {
           const int ks = g % kKStages, bs = g % kBStages;
@@ -410,7 +419,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       }
       // no copy may still be in flight when the CTA leaves (this matters only after an abort:
       // otherwise the consumers have waited for every load)
-      if (nq > 0) mbar_wait_drain(&bars->q_full, (nq - 1) & 1);
+      for (int nd = n >= 2 ? n - 2 : 0; nd < n; ++nd) mbar_wait_drain(&bars->q_full[nd & 1], (nd >> 1) & 1);
       for (uint32_t gd = g >= kKStages ? g - kKStages : 0; gd < g; ++gd)
         mbar_wait_drain(&bars->k_full[gd % kKStages], (gd / kKStages) & 1);
       for (uint32_t gd = g >= kBStages ? g - kBStages : 0; gd < g; ++gd)
@@ -422,8 +431,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       tma_prefetch(&tm_v);
       tma_prefetch(&tm_m);
       uint32_t g = 0;
-      int n = 0;
-      for (int k = blockIdx.x; k < p.n_items && !*abort; k += gridDim.x, ++n) {
+      for (int k = blockIdx.x; k < p.n_items && !*abort; k += gridDim.x) {
         const Item it = item_at(p, k);
         int cs = 0, cr = 0;                // entry cursor: selected slot, source row
         bool ok = true;
@@ -464,59 +472,76 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     }
   } else if (warp == kWarpMMA) {
     // ------------------------------------------------------------------ MMA issuer
+    // Two cursors over the CTA's steps: S runs two steps ahead of P V.  S(g + 2) goes into the S
+    // buffer that softmax(g) has just read into registers, so it overlaps softmax(g); P V(g)
+    // follows once P(g) is written.  The tensor core executes in issue order.
     if (lane == 0) {
       const uint32_t idesc_qk = idesc_bf16(kBM, kBN, 0, 0);   // Q, K both K-major
       const uint32_t idesc_pv = idesc_bf16(kBM, kD, 0, 1);    // P from TMEM, V MN-major
-      const uint32_t q0 = smem_u32(sQ);
-      uint32_t g = 0;
-      int n = 0;
-      auto issue_s = [&](uint32_t gs) {
-        const int ks = gs % kKStages;
-        const uint32_t kb = smem_u32(sK + ks * kTile);
-        const uint32_t d = tmem + (gs & 1) * kBN;
-#pragma unroll
-        for (int ks = 0; ks < kD / 16; ++ks) {
-          const uint32_t off = (ks >> 2) * kPanel + (ks & 3) * 32;
-          umma_ss(d, sdesc_sw128(q0 + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), idesc_qk, ks > 0);
+      // S cursor: schedule index, item count, step in the item, global step
+      int sk = blockIdx.x, sn = 0, ss = 0;
+      uint32_t sg = 0;
+      int sT = sk < p.n_items ? item_at(p, sk).T : 0;
+      // P V cursor
+      int pk = blockIdx.x, pn = 0, ps = 0;
+      uint32_t pg = 0;
+      int pT = pk < p.n_items ? item_at(p, pk).T : 0;
+      auto issue_s = [&]() -> bool {
+        if (ss == 0) {
+          if (!mbar_wait(&bars->q_full[sn & 1], (sn >> 1) & 1, abort, status)) return false;
         }
-        umma_commit(&bars->s_full[gs & 1]);
+        const int ks = sg % kKStages;
+        if (!mbar_wait(&bars->k_full[ks], (sg / kKStages) & 1, abort, status)) return false;
+        tc_fence_after();
+        const uint32_t qb = smem_u32(sQ + (sn & 1) * kTile), kb = smem_u32(sK + ks * kTile);
+        const uint32_t d = tmem + kColS + (sg & 1) * kBN;
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kPanel + (kk & 3) * 32;
+          umma_ss(d, sdesc_sw128(qb + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), idesc_qk, kk > 0);
+        }
+        umma_commit(&bars->s_full[sg & 1]);
         umma_commit(&bars->k_empty[ks]);
+        if (ss == sT - 1) umma_commit(&bars->q_empty[sn & 1]);
+        ++sg;
+        if (++ss == sT) {
+          ss = 0;
+          ++sn;
+          sk += gridDim.x;
+          sT = sk < p.n_items ? item_at(p, sk).T : 0;
+        }
+        return true;
       };
       bool ok = true;
-      for (int k = blockIdx.x; k < p.n_items && ok; k += gridDim.x, ++n) {
-        const Item it = item_at(p, k);
-        if (!mbar_wait(&bars->q_full, n & 1, abort, status)) break;
+      for (int i = 0; i < 2 && sT > 0 && ok; ++i) ok = issue_s();
+      while (ok && pT > 0) {
+        // S two steps ahead, once softmax(pg) has read S_{pg & 1}
+        if (sT > 0) {
+          if (!mbar_wait(&bars->s_free[pg & 1], (pg >> 1) & 1, abort, status)) break;
+          if (!issue_s()) break;
+        }
+        const int vs = pg % kVStages;
+        if (!mbar_wait(&bars->p_ready[pg & 1], (pg >> 1) & 1, abort, status)) break;
+        if (!mbar_wait(&bars->v_full[vs], (pg / kVStages) & 1, abort, status)) break;
+        if (ps == 0 && !mbar_wait(&bars->o_free, (pn & 1) ^ 1, abort, status)) break;
         tc_fence_after();
-        const uint32_t g0 = g;
-        if (!mbar_wait(&bars->k_full[g0 % kKStages], (g0 / kKStages) & 1, abort, status)) break;
-        tc_fence_after();
-        issue_s(g0);
-        for (int s = 0; s < it.T; ++s, ++g) {
-          if (s + 1 < it.T) {
-            const uint32_t gn = g + 1;
-            if (!mbar_wait(&bars->k_full[gn % kKStages], (gn / kKStages) & 1, abort, status)) { ok = false; break; }
-            tc_fence_after();
-            issue_s(gn);
-          } else {
-            umma_commit(&bars->q_empty);
-          }
-          const int vs = g % kVStages;
-          if (!mbar_wait(&bars->p_ready[g & 1], (g >> 1) & 1, abort, status)) { ok = false; break; }
-          if (!mbar_wait(&bars->v_full[vs], (g / kVStages) & 1, abort, status)) { ok = false; break; }
-          if (s == 0 && !mbar_wait(&bars->o_free, (n & 1) ^ 1, abort, status)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t vb = smem_u32(sV + vs * kTile);
-          const uint32_t pt = tmem + (g & 1) * kBN;       // P: bf16 pairs in the S buffer's first 64 columns
-          const uint32_t ot = tmem + (2 + (g & 1)) * kBN;  // O_X of the step's warpgroup
+        const uint32_t vb = smem_u32(sV + vs * kTile);
+        const uint32_t pt = tmem + kColP + (pg & 1) * (kBN / 2);   // P(pg): bf16 pairs, 64 columns
 #pragma unroll
-          for (int ks = 0; ks < kBN / 16; ++ks) {
-            // V rows (keys) 16*ks .. 16*ks+15: two 8-row groups of 1024 B; the first product of each
-            // accumulator in the item (steps 0 and 1) overwrites it
-            umma_ts(ot, pt + ks * 8, sdesc_sw128(vb + ks * 2048, kPanel, 1024), idesc_pv,
-                    (s > 1 || ks > 0) ? 1u : 0u);
-          }
-          umma_commit(&bars->v_empty[vs]);
-          umma_commit(&bars->o_done[g & 1]);
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          // V rows (keys) 16 kk .. 16 kk + 15: two 8-row groups of 1024 B; the first product of an
+          // item overwrites O
+          umma_ts(tmem + kColO, pt + kk * 8, sdesc_sw128(vb + kk * 2048, kPanel, 1024), idesc_pv,
+                  (ps > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&bars->v_empty[vs]);
+        umma_commit(&bars->p_free[pg & 1]);
+        ++pg;
+        if (++ps == pT) {
+          ps = 0;
+          ++pn;
+          pk += gridDim.x;
+          pT = pk < p.n_items ? item_at(p, pk).T : 0;
         }
       }
       umma_commit(&bars->drain);
@@ -528,28 +553,28 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const int X = warp >> 2;                                  // warpgroup: steps g with g & 1 == X
     const int r = tid & 127;                                  // query row = TMEM lane
     const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-    const uint32_t o_own = lane_addr + (2 + X) * kBN;
+    const uint32_t o_row = lane_addr + kColO;
+    const uint32_t p_own = lane_addr + kColP + X * (kBN / 2);
     uint32_t g0 = 0;                                          // first step of the item
-    uint32_t u = 0;                                           // products into O_X issued so far
     int n = 0;
     // (no abort test in the loop condition: a warp leaves as a whole, on its __all_sync'd waits)
     for (int k = blockIdx.x; k < p.n_items; k += gridDim.x, ++n) {
       const Item it = item_at(p, k);
-      float m = -INFINITY, l = 0.f;
-      bool ok = true, first = true;
+      // m_at, l: this warpgroup's share of the row sum, expressed at the running max m_at
+      float m_at = -INFINITY, l = 0.f;
+      bool ok = true;
       for (int s = (int)((X - g0) & 1u); s < it.T; s += 2) {
         const uint32_t g = g0 + s;
-        // every phase of this warpgroup's b_full slots and of s_full[X] is waited, in order
         const int bs = g % kBStages;
         bool w_ok = mbar_wait(&bars->b_full[bs], (g / kBStages) & 1, abort, status);
         w_ok = w_ok && mbar_wait(&bars->s_full[X], (g >> 1) & 1, abort, status);
         if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
         tc_fence_after();
-        // The S row is loaded from TMEM once (128 registers): the row max, then p = 2^(y - m), the
-        // row sum and the bf16 P written back over S.  Column c's logit is y_c = x_c * s*log2(e) +
-        // bias_c, the bias row in shared memory: log2 n_c on a cluster chunk, log2 n_e on an entry
-        // tile, 0 on a key block (-inf past the end of a short last block or of the entries).
-        const uint32_t sbase = lane_addr + X * kBN;
+        // The S row is loaded from TMEM once (128 registers); S_X is then free for S(g + 2).
+        // Column c's logit is y_c = x_c * s*log2(e) + bias_c, the bias row in shared memory:
+        // log2 n_c on a cluster chunk, log2 n_e on an entry tile, 0 on a key block (-inf past the
+        // end of a short last block or of the entries).
+        const uint32_t sbase = lane_addr + kColS + X * kBN;
         const float* bt = sBias + bs * kBN;
         const int flag = bars->bflag[bs];
         const bool plain = (flag & 1) && p.scale_log2 > 0.f;
@@ -562,12 +587,30 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         reg_fence32(x[1]);
         reg_fence32(x[2]);
         reg_fence32(x[3]);
+        tc_fence_before();
+        mbar_arrive(&bars->s_free[X]);
         const float mx = row_logits_max(x, bt, plain, p.scale_log2);
-        // lazy rescaling: the running max moves only when it grows by more than 2^8
-        const bool grow = mx > m + kRescaleLog2 || (m == -INFINITY && mx > -INFINITY);
-        const bool need_o = grow && !first && m > -INFINITY;
-        const float m_new = grow ? mx : m;
+        // The running max is shared by the two warpgroups (one accumulator O): take the other's
+        // latest one (every phase of m_pub is waited, in order), and let it move only when it grows
+        // by more than 2^8 (lazy rescaling).  An item starts from -inf.
+        float mprev = -INFINITY;
+        if (g >= 1) {
+          const bool m_ok = mbar_wait(&bars->m_pub[X ^ 1], ((g - 1) >> 1) & 1, abort, status);
+          if (!__all_sync(0xffffffffu, m_ok)) { ok = false; break; }
+          const float mo = bars->mrow[X ^ 1][r];
+          if (s > 0) mprev = mo;
+        }
+        const bool grow = mx > mprev + kRescaleLog2 || (mprev == -INFINITY && mx > -INFINITY);
+        const float m_new = grow ? mx : mprev;
+        bars->mrow[X][r] = m_new;
+        mbar_arrive(&bars->m_pub[X]);
         const float mu = (m_new == -INFINITY) ? 0.f : m_new;
+        // P_X is free once P V(g - 2) is done (every phase of p_free[X] is waited, in order)
+        if (g >= 2) {
+          const bool f_ok = mbar_wait(&bars->p_free[X], ((g - 2) >> 1) & 1, abort, status);
+          if (!__all_sync(0xffffffffu, f_ok)) { ok = false; break; }
+          tc_fence_after();
+        }
         uint64_t rsum = 0;
         {
           const uint64_t negmu = f2_pack(-mu, -mu);
@@ -576,83 +619,74 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           for (int q = 0; q < 4; ++q) {
             uint32_t pk[16];
             chunk_exp(x[q], coef, negmu, pk, rsum);
-            tmem_st16(sbase + q * 16, pk);
+            tmem_st16(p_own + q * 16, pk);
           }
         }
         mbar_arrive(&bars->b_empty[bs]);          // this thread has read the bias row
         float rs_lo, rs_hi;
         f2_unpack(rsum, rs_lo, rs_hi);
         const float rs = rs_lo + rs_hi;
-        if (!first) {
-          // this warpgroup's previous product has landed in O_X: every phase of o_done[X] is
-          // waited, in order; a row whose max moved rescales its O_X (warp-uniform, as
-          // tcgen05.ld/st are)
-          const bool d_ok = mbar_wait(&bars->o_done[X], (u - 1) & 1, abort, status);
+        // O holds every product up to step g - 1 once P V(g - 1) is done (every phase of the other
+        // warpgroup's p_free is waited, in order); a row whose max moved rescales it
+        if (g >= 1) {
+          const bool d_ok = mbar_wait(&bars->p_free[X ^ 1], ((g - 1) >> 1) & 1, abort, status);
           if (!__all_sync(0xffffffffu, d_ok)) { ok = false; break; }
           tc_fence_after();
-          if (__any_sync(0xffffffffu, need_o)) {
-            const float alpha = need_o ? ex2(m - m_new) : 1.f;
+        }
+        const bool need_o = grow && s > 0 && mprev > -INFINITY;
+        if (__any_sync(0xffffffffu, need_o)) {
+          const float alpha = need_o ? ex2(mprev - m_new) : 1.f;
 #pragma unroll 1
-            for (int q = 0; q < 4; ++q) {
-              uint32_t rr[32];
-              tmem_ld32(o_own + q * 32, rr);
-              tmem_wait_ld();
+          for (int q = 0; q < 4; ++q) {
+            uint32_t rr[32];
+            tmem_ld32(o_row + q * 32, rr);
+            tmem_wait_ld();
 #pragma unroll
-              for (int v = 0; v < 32; ++v) rr[v] = __float_as_uint(__uint_as_float(rr[v]) * alpha);
-              tmem_st32(o_own + q * 32, rr);
-            }
-            if (need_o) l *= alpha;
+            for (int v = 0; v < 32; ++v) rr[v] = __float_as_uint(__uint_as_float(rr[v]) * alpha);
+            tmem_st32(o_row + q * 32, rr);
           }
         }
-        m = m_new;
+        if (m_new != m_at) {                      // the running max only grows
+          if (m_at > -INFINITY) l *= ex2(m_at - m_new);
+          m_at = m_new;
+        }
         l += (flag & 2) ? -rs : rs;               // entry tiles take their weight out again
-        first = false;
-        ++u;
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&bars->p_ready[X]);
       }
       if (!ok) break;
-      // epilogue: once this warpgroup's last product has landed, exchange (max, sum) per row with
-      // the other warpgroup; warpgroup X normalises and stores columns [64X, 64X + 64) of
-      // O = (O_0 2^(m_0 - M) + O_1 2^(m_1 - M)) / (l_0 2^(m_0 - M) + l_1 2^(m_1 - M)).
-      // A warpgroup without a step in the item (a one-step item) has an unwritten O_X: skipped.
-      const bool had0 = it.T >= 2 || (g0 & 1u) == 0u;
-      const bool had1 = it.T >= 2 || (g0 & 1u) == 1u;
-      bool e_ok = first || mbar_wait(&bars->o_done[X], (u - 1) & 1, abort, status);
-      bars->xch[n & 1][X][r] = make_float2(m, l);
+      // epilogue: once the item's last product has landed, exchange (max, sum) per row with the
+      // other warpgroup; warpgroup X normalises and stores columns [64X, 64X + 64) of
+      // O / (l_0 2^(m_0 - M) + l_1 2^(m_1 - M)), O being expressed at M, the larger of the two.
+      const uint32_t gl = g0 + it.T - 1;
+      bool e_ok = mbar_wait(&bars->p_free[gl & 1], (gl >> 1) & 1, abort, status);
+      bars->xch[n & 1][X][r] = make_float2(m_at, l);
       mbar_arrive(&bars->xch_full[n & 1][X]);
       e_ok = e_ok && mbar_wait(&bars->xch_full[n & 1][X ^ 1], (n >> 1) & 1, abort, status);
       if (!__all_sync(0xffffffffu, e_ok)) break;
       tc_fence_after();
       const float2 e0 = bars->xch[n & 1][0][r], e1 = bars->xch[n & 1][1][r];
       const float M = fmaxf(e0.x, e1.x);
-      const float f0 = (had0 && e0.x > -INFINITY) ? ex2(e0.x - M) : 0.f;
-      const float f1 = (had1 && e1.x > -INFINITY) ? ex2(e1.x - M) : 0.f;
+      const float f0 = e0.x > -INFINITY ? ex2(e0.x - M) : 0.f;
+      const float f1 = e1.x > -INFINITY ? ex2(e1.x - M) : 0.f;
       const float L = e0.y * f0 + e1.y * f1;
       const float inv = L > 0.f ? 1.f / L : 0.f;
-      const float c0 = f0 * inv, c1 = f1 * inv;
       const bool live = r < it.qlen;
       __nv_bfloat16* op = p.O + ((size_t)it.bh * p.N + it.q0 + r) * kD + 64 * X;
 #pragma unroll 1
       for (int q = 0; q < 2; ++q) {
-        const uint32_t col = 64 * X + 32 * q;
-        uint32_t ra[32], rb[32];
-        if (had0) tmem_ld32(lane_addr + 2 * kBN + col, ra);
-        if (had1) tmem_ld32(lane_addr + 3 * kBN + col, rb);
+        uint32_t ra[32];
+        tmem_ld32(o_row + 64 * X + 32 * q, ra);
         tmem_wait_ld();
         if (live) {
-          auto o = [&](int v) {
-            const float a = had0 ? __uint_as_float(ra[v]) * c0 : 0.f;
-            return had1 ? fmaf(__uint_as_float(rb[v]), c1, a) : a;
-          };
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
             uint4 w;
-            w.x = pack_bf16x2(o(8 * v + 0), o(8 * v + 1));
-            w.y = pack_bf16x2(o(8 * v + 2), o(8 * v + 3));
-            w.z = pack_bf16x2(o(8 * v + 4), o(8 * v + 5));
-            w.w = pack_bf16x2(o(8 * v + 6), o(8 * v + 7));
+            w.x = pack_bf16x2(__uint_as_float(ra[8 * v + 0]) * inv, __uint_as_float(ra[8 * v + 1]) * inv);
+            w.y = pack_bf16x2(__uint_as_float(ra[8 * v + 2]) * inv, __uint_as_float(ra[8 * v + 3]) * inv);
+            w.z = pack_bf16x2(__uint_as_float(ra[8 * v + 4]) * inv, __uint_as_float(ra[8 * v + 5]) * inv);
+            w.w = pack_bf16x2(__uint_as_float(ra[8 * v + 6]) * inv, __uint_as_float(ra[8 * v + 7]) * inv);
             *reinterpret_cast<uint4*>(op + q * 32 + v * 8) = w;
           }
         }

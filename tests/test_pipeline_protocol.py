@@ -1,32 +1,34 @@
 """Host-side model of the fused attention kernel's synchronisation protocol.
 
-The kernel's roles (TMA producer lanes, MMA issuer, two softmax warpgroups)
-talk only through mbarriers.  An mbarrier wait names a phase by its
-parity alone, so a wait is only meaningful while the barrier is within one
-phase of the awaited one; a role that falls two phases behind (or waits one
-phase early) reads the wrong phase.  This model replays the roles' exact
-sequence of arrivals and waits, with the tensor core executing its queue in
-order and the TMA unit completing loads in any order, under many random
-interleavings, and checks that
+The kernel's roles (TMA producers, MMA issuer, two softmax warpgroups) talk only
+through mbarriers.  An mbarrier wait names a phase by its parity alone, so a
+wait is only meaningful while the barrier is within one phase of the awaited
+one; a role that falls two phases behind (or waits one phase early) reads the
+wrong phase.  This model replays the roles' exact sequence of arrivals and
+waits, with the tensor core executing its queue in order and the TMA unit
+completing loads in any order, under many random interleavings, and checks that
 
 * every parity wait is evaluated only while the barrier is at the awaited
   phase or one past it;
 * no phase receives more arrivals than its count, and the transaction count
   never goes negative;
-* no shared-memory slot, TMEM buffer or the query tile is overwritten while an
+* no shared-memory slot, TMEM buffer or query tile is overwritten while an
   operation that reads it is still in flight, and every consumer reads the
-  tile of its own step;
+  tile (and the published running max) of its own step;
 * every role finishes (no deadlock).
 
 It mirrors the step structure of attention_tc.cu: per work item, one step per
 selected block, one per 128-cluster chunk, then one per entry tile of the
-selected blocks' cluster entries; key, value and bias-row rings; softmax
-warpgroup X taking the steps g with g & 1 == X, with its own S buffer (P
-written over it) and accumulator O_X; at the end of an item the two
-warpgroups exchange (max, sum) through a double-buffered shared array and each
-reads both accumulators.  Chunk and entry tiles are written by the Reassign
-Cache before the kernel starts, so they are plain inputs here; an entry tile
-arrives as several copies on one barrier, which the model counts as one
+selected blocks' cluster entries; double-buffered query tiles; key, value and
+bias-row rings; the MMA issuer running S two steps ahead of P V, S(g + 2) into
+the score buffer softmax(g) has just read; softmax warpgroup X taking the steps
+g with g & 1 == X, with its own score buffer S_X and probability tile P_X; one
+output accumulator O shared by both, with the running max passed between the
+warpgroups at every step and O rescaled by whichever raises it; at the end of
+an item the two warpgroups exchange (max, sum) through a double-buffered shared
+array and each reads half of O.  Chunk and entry tiles are written by the
+Reassign Cache before the kernel starts, so they are plain inputs here; an entry
+tile arrives as several copies on one barrier, which the model counts as one
 transaction.
 """
 import random
@@ -34,7 +36,7 @@ import random
 import pytest
 
 KSTAGES = 2   # key / centroid tiles, freed when S is computed
-VSTAGES = 3   # value / vbar^U tiles, freed after P V
+VSTAGES = 2   # value / mean tiles, freed after P V
 BSTAGES = 4   # softmax bias rows, freed after the softmax has read them (even: one warpgroup per slot)
 
 
@@ -73,18 +75,24 @@ class Barrier:
 
 class Machine:
     def __init__(self, items, nchunk, rng, lazy_v_wait=False, skip_b_empty=False, single_xch=False,
-                 no_final_wait=False, single_xch_barrier=False):
+                 no_final_wait=False, single_xch_barrier=False, s_before_read=False, no_pfree_wait=False,
+                 no_rescale_wait=False, single_q=False, skip_m_wait=False):
         # per item of one CTA: nsel, or (nsel, entry tiles)
         self.items = [(x, 0) if isinstance(x, int) else tuple(x) for x in items]
         self.nchunk = nchunk
         self.rng = rng
-        self.lazy_v_wait = lazy_v_wait         # planted: value lane waits for a free slot only at chunk steps
+        self.lazy_v_wait = lazy_v_wait         # planted: value producer waits for a free slot only at chunk steps
         self.skip_b_empty = skip_b_empty       # planted: bias rows loaded without waiting for a free slot
         self.single_xch = single_xch           # planted: one (max, sum) exchange buffer for all items
         self.no_final_wait = no_final_wait     # planted: epilogue without waiting for the last product
         self.single_xch_barrier = single_xch_barrier   # planted: one exchange barrier per warpgroup
+        self.s_before_read = s_before_read     # planted: softmax releases S before reading it
+        self.no_pfree_wait = no_pfree_wait     # planted: P written without waiting for P V(g - 2)
+        self.no_rescale_wait = no_rescale_wait  # planted: O rescaled without waiting for P V(g - 1)
+        self.single_q = single_q               # planted: one query buffer, with the waits of two
+        self.skip_m_wait = skip_m_wait         # planted: the running max read without its barrier
         B = Barrier
-        self.q_full, self.q_empty = B("q_full", 1), B("q_empty", 1)
+        self.q_full, self.q_empty = [B(f"q_full{i}", 1) for i in range(2)], [B(f"q_empty{i}", 1) for i in range(2)]
         self.k_full = [B(f"k_full{i}", 1) for i in range(KSTAGES)]
         self.k_empty = [B(f"k_empty{i}", 1) for i in range(KSTAGES)]
         self.v_full = [B(f"v_full{i}", 1) for i in range(VSTAGES)]
@@ -93,17 +101,25 @@ class Machine:
         self.b_empty = [B(f"b_empty{i}", 1) for i in range(BSTAGES)]
         self.version = {}                      # buffer -> step whose tile it holds
         self.s_full = [B(f"s_full{i}", 1) for i in range(2)]
+        self.s_free = [B(f"s_free{i}", 1) for i in range(2)]     # 128 threads, one arrival here
         self.p_ready = [B(f"p_ready{i}", 1) for i in range(2)]
-        self.o_done = [B(f"o_done{i}", 1) for i in range(2)]
+        self.p_free = [B(f"p_free{i}", 1) for i in range(2)]
+        self.m_pub = [B(f"m_pub{i}", 1) for i in range(2)]
+        self.mrow = [None, None]               # warpgroup -> step whose running max it holds
         self.o_free = B("o_free", 2)           # one arrival per warpgroup (128 threads each)
         # exchange published: [item parity][warpgroup]; one barrier per item parity, so a warpgroup
         # without steps cannot complete a barrier twice before the other has waited on it once
         self.xch_full = [[B(f"xch_full{j}{i}", 1) for i in range(2)] for j in range(2)]
         self.xch = [[None, None], [None, None]]   # [item parity][warpgroup] -> item whose (max, sum) it holds
-        self.o_content = [None, None]          # accumulator -> (item, products accumulated), at issue
+        self.o_content = None                  # (item, last step accumulated), at issue
+        self.o_scaled = None                   # (item, step) of the last rescale of O
         self.tc_queue = []                     # in-order tensor core: ("mma", reads, writes) / ("commit", bar)
         self.tma = []                          # in flight: (bar, buffer written, buffers read)
         self.readers = {}                      # resource -> units with an operation in flight on it
+
+    def T(self, n):
+        nsel, nent = self.items[n]
+        return nsel + self.nchunk + nent
 
     # ---- resources: in-flight users of each buffer, tagged by unit
     def _start_read(self, res, unit):
@@ -159,16 +175,19 @@ class Machine:
     def holds(self, res, step):
         assert self.version.get(res) == step, f"{res} holds step {self.version.get(res)}, read at step {step}"
 
+    def qbuf(self, n):
+        return 0 if self.single_q else n & 1
+
     # ---- roles (generators yield a predicate to wait on)
     def producer(self):
-        """Lane 0 of the producer warp: query tiles, key / centroid tiles, bias rows."""
+        """The producer of keys: query tiles, key / centroid / entry tiles, bias rows."""
         g = 0
-        for n, (nsel, nent) in enumerate(self.items):
-            T = nsel + self.nchunk + nent
-            yield lambda: self.q_empty.test(n - 1)
-            self.q_full.expect_tx(1)
-            self.tma_load(self.q_full, "Q", n)
-            for s in range(T):
+        for n in range(len(self.items)):
+            qb = self.qbuf(n)
+            yield lambda: self.q_empty[n & 1].test((n >> 1) - 1)
+            self.q_full[n & 1].expect_tx(1)
+            self.tma_load(self.q_full[n & 1], f"Q{qb}", ("q", n))
+            for s in range(self.T(n)):
                 ks, bs = g % KSTAGES, g % BSTAGES
                 yield lambda: self.k_empty[ks].test(g // KSTAGES - 1)
                 self.k_full[ks].expect_tx(1)
@@ -182,11 +201,11 @@ class Machine:
                 g += 1
 
     def producer_v(self):
-        """Lane 1 of the producer warp: value / vbar^U tiles."""
+        """The producer of values / means / entry means."""
         g = 0
-        for n, (nsel, nent) in enumerate(self.items):
-            T = nsel + self.nchunk + nent
-            for s in range(T):
+        for n in range(len(self.items)):
+            nsel = self.items[n][0]
+            for s in range(self.T(n)):
                 vs = g % VSTAGES
                 if not self.lazy_v_wait or s >= nsel:
                     yield lambda: self.v_empty[vs].test(g // VSTAGES - 1)
@@ -194,64 +213,96 @@ class Machine:
                 self.tma_load(self.v_full[vs], f"V{vs}", g)
                 g += 1
 
-    def mma(self):
+    def _steps(self):
+        """(item, step in item, global step) of every step of the CTA, in order."""
         g = 0
-        for n, (nsel, nent) in enumerate(self.items):
-            T = nsel + self.nchunk + nent
-            yield lambda: self.q_full.test(n)
+        for n in range(len(self.items)):
+            for s in range(self.T(n)):
+                yield n, s, g
+                g += 1
+
+    def mma(self):
+        steps = list(self._steps())
+        si = 0                                  # S cursor (index into steps)
+
+        def issue_s():
+            nonlocal si
+            n, s, g = steps[si]
+            qb = self.qbuf(n)
+            if s == 0:
+                yield lambda: self.q_full[n & 1].test(n >> 1)
             yield lambda: self.k_full[g % KSTAGES].test(g // KSTAGES)
-            self.holds("Q", n)
+            self.holds(f"Q{qb}", ("q", n))
             self.holds(f"K{g % KSTAGES}", g)
-            self.tc_issue_mma(["Q", f"K{g % KSTAGES}"], [f"S{g & 1}"])
+            self.tc_issue_mma([f"Q{qb}", f"K{g % KSTAGES}"], [f"S{g & 1}"])
+            self.version[f"S{g & 1}"] = g
             self.tc_commit(self.s_full[g & 1])
             self.tc_commit(self.k_empty[g % KSTAGES])
-            for s in range(T):
-                if s + 1 < T:
-                    gn = g + 1
-                    yield lambda: self.k_full[gn % KSTAGES].test(gn // KSTAGES)
-                    self.holds(f"K{gn % KSTAGES}", gn)
-                    self.tc_issue_mma(["Q", f"K{gn % KSTAGES}"], [f"S{gn & 1}"])
-                    self.tc_commit(self.s_full[gn & 1])
-                    self.tc_commit(self.k_empty[gn % KSTAGES])
-                else:
-                    self.tc_commit(self.q_empty)
-                yield lambda: self.p_ready[g & 1].test(g >> 1)
-                yield lambda: self.v_full[g % VSTAGES].test(g // VSTAGES)
-                if s == 0:
-                    yield lambda: self.o_free.test(n - 1)
-                self.holds(f"V{g % VSTAGES}", g)
-                x = g & 1
-                self.tc_issue_mma([f"S{x}", f"V{g % VSTAGES}"], [f"O{x}"])
-                self.o_content[x] = (n, 1) if s <= 1 else (n, self.o_content[x][1] + 1)
-                self.tc_commit(self.v_empty[g % VSTAGES])
-                self.tc_commit(self.o_done[x])
-                g += 1
+            if s == self.T(n) - 1:
+                self.tc_commit(self.q_empty[n & 1])
+            si += 1
+
+        for _ in range(2):
+            if si < len(steps):
+                yield from issue_s()
+        for n, s, g in steps:
+            if si < len(steps):
+                yield lambda: self.s_free[g & 1].test(g >> 1)
+                yield from issue_s()
+            yield lambda: self.p_ready[g & 1].test(g >> 1)
+            yield lambda: self.v_full[g % VSTAGES].test(g // VSTAGES)
+            if s == 0:
+                yield lambda: self.o_free.test(n - 1)
+            self.holds(f"V{g % VSTAGES}", g)
+            self.holds(f"P{g & 1}", g)
+            if s > 0:
+                assert self.o_content == (n, g - 1), f"O holds {self.o_content} before P V of step {g}"
+            self.tc_issue_mma([f"P{g & 1}", f"V{g % VSTAGES}"], ["O"])
+            self.o_content = (n, g)
+            self.tc_commit(self.v_empty[g % VSTAGES])
+            self.tc_commit(self.p_free[g & 1])
 
     def softmax(self, X):
         g0 = 0
-        u = 0                                   # products into O_X issued so far
-        for n, (nsel, nent) in enumerate(self.items):
-            T = nsel + self.nchunk + nent
-            first = True
+        for n in range(len(self.items)):
+            T = self.T(n)
             for s in range((X - g0) & 1, T, 2):
                 g = g0 + s
                 bs = g % BSTAGES
                 yield lambda: self.b_full[bs].test(g // BSTAGES)
                 yield lambda: self.s_full[X].test(g >> 1)
-                assert not self.readers.get(f"S{X}"), "S read before its MMA completed"
                 assert not self.readers.get(f"BIAS{bs}"), "bias row read before it landed"
                 self.holds(f"BIAS{bs}", g)
-                self._write(f"S{X}", "softmax (P)")
+                if self.s_before_read:
+                    self.s_free[X].arrive()
+                    yield lambda: True                 # the row is read from TMEM after the release
+                assert not self.readers.get(f"S{X}"), "S read before its MMA completed or while it is rewritten"
+                self.holds(f"S{X}", g)
+                if not self.s_before_read:
+                    self.s_free[X].arrive()
+                if g >= 1:
+                    if not self.skip_m_wait:
+                        yield lambda: self.m_pub[X ^ 1].test((g - 1) >> 1)
+                    assert self.mrow[X ^ 1] == g - 1, f"running max of step {self.mrow[X ^ 1]} read at step {g}"
+                if g >= 2:
+                    assert self.mrow[X] is None or self.mrow[X] == g - 2
+                self.mrow[X] = g
+                self.m_pub[X].arrive()
+                if g >= 2 and not self.no_pfree_wait:
+                    yield lambda: self.p_free[X].test((g - 2) >> 1)
+                self._write(f"P{X}", "softmax (P)")
+                self.version[f"P{X}"] = g
                 self.b_empty[bs].arrive()
-                if not first:
-                    yield lambda: self.o_done[X].test(u - 1)
-                    self._write(f"O{X}", "softmax (rescale)")
+                if g >= 1 and not self.no_rescale_wait:
+                    yield lambda: self.p_free[X ^ 1].test((g - 1) >> 1)
+                if s > 0:                          # a rescale of O may happen here
+                    self._write("O", "softmax (rescale)")
+                    assert self.o_content == (n, g - 1), f"O holds {self.o_content} at the rescale of step {g}"
                 self.p_ready[X].arrive()
-                first = False
-                u += 1
             # epilogue
-            if not first and not self.no_final_wait:
-                yield lambda: self.o_done[X].test(u - 1)
+            gl = g0 + T - 1
+            if not self.no_final_wait:
+                yield lambda: self.p_free[gl & 1].test(gl >> 1)
             slot = 0 if self.single_xch else n & 1
             self.xch[slot][X] = n
             if self.single_xch_barrier:
@@ -261,15 +312,12 @@ class Machine:
                 self.xch_full[n & 1][X].arrive()
                 yield lambda: self.xch_full[n & 1][X ^ 1].test(n >> 1)
             assert self.xch[slot][X ^ 1] == n, f"exchange slot holds item {self.xch[slot][X ^ 1]}, read for item {n}"
-            for Y in (0, 1):
-                steps = len(range((Y - g0) & 1, T, 2))
-                if steps:
-                    assert not self.readers.get(f"O{Y}"), f"O{Y} read while a product into it is in flight"
-                    assert self.o_content[Y] == (n, steps), f"O{Y} holds {self.o_content[Y]} at the end of item {n}"
+            assert not self.readers.get("O"), "O read while a product into it is in flight"
+            assert self.o_content == (n, gl), f"O holds {self.o_content} at the end of item {n}"
             self.o_free.arrive()
             g0 += T
 
-    def run(self, max_iters=200000):
+    def run(self, max_iters=400000):
         roles = [self.producer(), self.producer_v(), self.mma(), self.softmax(0), self.softmax(1)]
         waits = [None] * len(roles)
         done = [False] * len(roles)
@@ -333,17 +381,34 @@ def test_model_catches_bias_rows_loaded_without_a_free_slot():
     assert _caught([3, 3, 3, 3, 3], 2, skip_b_empty=True) > 0
 
 
-def test_model_catches_a_single_exchange_buffer():
-    """With one-step items a warpgroup without steps reaches the next exchange while the other
-    still reads the previous one."""
-    assert _caught([0, 0, 0, 0, 0, 0], 1, single_xch=True) > 0
-
-
 def test_model_catches_an_epilogue_that_does_not_wait_for_the_last_product():
     assert _caught([3, 4, 1], 2, no_final_wait=True) > 0
 
 
-def test_model_catches_one_exchange_barrier_per_warpgroup():
-    """A warpgroup without steps in an item can complete a single exchange barrier twice before
-    the other warpgroup's parity wait on it runs."""
-    assert _caught([1, 0, 0, 1], 1, single_xch_barrier=True) > 0
+def test_one_exchange_barrier_per_warpgroup_is_now_safe():
+    """With one accumulator, the first product of item n + 1 waits for item n's epilogue (o_free),
+    and item n + 1's epilogue waits for that product, so a warpgroup cannot complete a single
+    exchange barrier twice before the other has waited on it; the double buffer stays as a margin."""
+    assert _caught([1, 0, 0, 1], 1, single_xch_barrier=True) == 0
+
+
+def test_model_catches_s_released_before_it_is_read():
+    assert _caught([5, 5], 2, s_before_read=True) > 0
+
+
+def test_model_catches_p_written_during_its_product():
+    assert _caught([6, 4], 2, no_pfree_wait=True) > 0
+
+
+def test_model_catches_a_rescale_during_the_previous_product():
+    assert _caught([6, 4], 2, no_rescale_wait=True) > 0
+
+
+def test_model_catches_a_single_query_buffer():
+    """With S two steps ahead of P V, the next item's first S is issued while the current item's
+    query tile is still read; one buffer would be overwritten."""
+    assert _caught([1, 1, 1, 1, 2, 1], 1, single_q=True) > 0
+
+
+def test_model_catches_the_running_max_read_without_its_barrier():
+    assert _caught([6, 6], 2, skip_m_wait=True) > 0
