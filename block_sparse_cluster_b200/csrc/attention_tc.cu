@@ -605,36 +605,37 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         bars->mrow[X][r] = m_new;
         mbar_arrive(&bars->m_pub[X]);
         const float mu = (m_new == -INFINITY) ? 0.f : m_new;
+        // the row's probabilities, packed to bf16 pairs in registers (each chunk of scores dies as
+        // its probabilities are formed)
+        uint64_t rsum = 0;
+        uint32_t pk[4][16];
+        {
+          const uint64_t negmu = f2_pack(-mu, -mu);
+          const uint64_t coef = plain ? f2_pack(p.scale_log2, p.scale_log2) : f2_pack(1.f, 1.f);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) chunk_exp(x[q], coef, negmu, pk[q], rsum);
+        }
         // P_X is free once P V(g - 2) is done (every phase of p_free[X] is waited, in order)
         if (g >= 2) {
           const bool f_ok = mbar_wait(&bars->p_free[X], ((g - 2) >> 1) & 1, abort, status);
           if (!__all_sync(0xffffffffu, f_ok)) { ok = false; break; }
           tc_fence_after();
         }
-        uint64_t rsum = 0;
-        {
-          const uint64_t negmu = f2_pack(-mu, -mu);
-          const uint64_t coef = plain ? f2_pack(p.scale_log2, p.scale_log2) : f2_pack(1.f, 1.f);
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint32_t pk[16];
-            chunk_exp(x[q], coef, negmu, pk, rsum);
-            tmem_st16(p_own + q * 16, pk);
-          }
-        }
+        for (int q = 0; q < 4; ++q) tmem_st16(p_own + q * 16, pk[q]);
         mbar_arrive(&bars->b_empty[bs]);          // this thread has read the bias row
         float rs_lo, rs_hi;
         f2_unpack(rsum, rs_lo, rs_hi);
         const float rs = rs_lo + rs_hi;
-        // O holds every product up to step g - 1 once P V(g - 1) is done (every phase of the other
-        // warpgroup's p_free is waited, in order); a row whose max moved rescales it
-        if (g >= 1) {
+        // A row whose max moved rescales O, which must first hold every product up to step g - 1.
+        // Only a warp that rescales waits for P V(g - 1): P V(g - 2) is known done here (p_free[X]
+        // above) and P V(g + 1) cannot start before this step's P is ready, so the other
+        // warpgroup's p_free is within one phase of the awaited one whenever it is waited.
+        const bool need_o = grow && s > 0 && mprev > -INFINITY;
+        if (__any_sync(0xffffffffu, need_o)) {
           const bool d_ok = mbar_wait(&bars->p_free[X ^ 1], ((g - 1) >> 1) & 1, abort, status);
           if (!__all_sync(0xffffffffu, d_ok)) { ok = false; break; }
           tc_fence_after();
-        }
-        const bool need_o = grow && s > 0 && mprev > -INFINITY;
-        if (__any_sync(0xffffffffu, need_o)) {
           const float alpha = need_o ? ex2(mprev - m_new) : 1.f;
 #pragma unroll 1
           for (int q = 0; q < 4; ++q) {
@@ -659,8 +660,10 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       // epilogue: once the item's last product has landed, exchange (max, sum) per row with the
       // other warpgroup; warpgroup X normalises and stores columns [64X, 64X + 64) of
       // O / (l_0 2^(m_0 - M) + l_1 2^(m_1 - M)), O being expressed at M, the larger of the two.
+      // (P V(gl - 1) first: after it, P V(gl)'s barrier is within one phase of the awaited one)
       const uint32_t gl = g0 + it.T - 1;
-      bool e_ok = mbar_wait(&bars->p_free[gl & 1], (gl >> 1) & 1, abort, status);
+      bool e_ok = gl < 1 || mbar_wait(&bars->p_free[(gl - 1) & 1], ((gl - 1) >> 1) & 1, abort, status);
+      e_ok = e_ok && mbar_wait(&bars->p_free[gl & 1], (gl >> 1) & 1, abort, status);
       bars->xch[n & 1][X][r] = make_float2(m_at, l);
       mbar_arrive(&bars->xch_full[n & 1][X]);
       e_ok = e_ok && mbar_wait(&bars->xch_full[n & 1][X ^ 1], (n >> 1) & 1, abort, status);

@@ -293,15 +293,19 @@ class Machine:
                 self._write(f"P{X}", "softmax (P)")
                 self.version[f"P{X}"] = g
                 self.b_empty[bs].arrive()
-                if g >= 1 and not self.no_rescale_wait:
-                    yield lambda: self.p_free[X ^ 1].test((g - 1) >> 1)
-                if s > 0:                          # a rescale of O may happen here
+                # a rescale of O (only when the running max moved: here at random, and always at an
+                # item's second step) waits for P V(g - 1) first
+                if s > 0 and (s == 1 or self.rng.random() < 0.3):
+                    if not self.no_rescale_wait:
+                        yield lambda: self.p_free[X ^ 1].test((g - 1) >> 1)
                     self._write("O", "softmax (rescale)")
                     assert self.o_content == (n, g - 1), f"O holds {self.o_content} at the rescale of step {g}"
                 self.p_ready[X].arrive()
             # epilogue
             gl = g0 + T - 1
             if not self.no_final_wait:
+                if gl >= 1:
+                    yield lambda: self.p_free[(gl - 1) & 1].test((gl - 1) >> 1)
                 yield lambda: self.p_free[gl & 1].test(gl >> 1)
             slot = 0 if self.single_xch else n & 1
             self.xch[slot][X] = n
