@@ -29,20 +29,25 @@
 // 1 / pi_j in both sums of the softmax; no cluster columns.
 //
 // Roles (384 threads):
-//   warps 0-3, 4-7  two softmax warpgroups X = 0, 1; warpgroup X takes the steps g with g & 1 = X
-//              of every item, so the two overlap each other and the tensor core.  Thread t of a
-//              warpgroup owns query row t = TMEM lane t: online softmax with lazy rescaling (the
-//              running max only moves when it grows by more than 2^8) of its own accumulator O_X,
-//              P written back to TMEM as bf16.  At the end of the item the two exchange their
-//              (max, sum) per row and each normalises and stores half of the columns of
-//              O = O_0 2^(m_0 - m) + O_1 2^(m_1 - m);
-//   warp 8     producer: loads Q, key tiles / centroid chunks / entry centroid rows (2-stage ring)
-//              and the softmax bias rows (4-stage ring, so a slot always serves the same warpgroup);
-//   warp 9     MMA: allocates TMEM, issues tcgen05.mma S(g+1) = Q K^T ahead of O_X += P(g) V(g);
-//   warp 10    producer of value tiles / cluster means / entry means (3-stage ring); a warp of its
+//   warps 0-3, 4-7  two softmax warpgroups X = 0, 1 (barriers they arrive on count warps: lane 0
+//              arrives after a warp barrier); warpgroup X takes the steps g with g & 1 = X of
+//              every item, so the two overlap each other and the tensor core.  Thread t of a
+//              warpgroup owns query row t = TMEM lane t.  It reads S_X into registers (S_X is then
+//              free for S(g + 2)), takes the running max of the other warpgroup's latest step and
+//              lets it grow lazily (only by more than 2^8), writes P as bf16 into its own P_X and
+//              keeps its share of the row sum.  The two share one accumulator O: whichever raises
+//              the max rescales O, once the previous product has landed.  At the end of an item
+//              they exchange (max, sum) per row and each normalises and stores half of O's columns;
+//   warp 8     producer: loads Q, key tiles / centroid chunks / entry centroid rows (3-stage ring,
+//              so that a key tile loads while the two before it are read) and the softmax bias rows (4-stage ring, so a slot always serves the
+//              same warpgroup);
+//   warp 9     MMA issuer of S(g) = Q K^T into S_{g & 1} once softmax(g - 2) has read it (and TMEM
+//              allocation); S thus overlaps the softmax of two steps before;
+//   warp 10    producer of value tiles / cluster means / entry means (2-stage ring); a warp of its
 //              own, since divergent lanes of one warp waiting on different barriers hold each other up;
-//   warp 11    idle (it completes the third warpgroup, whose registers go to the softmax).
-// TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,384), O_1 [384,512).
+//   warp 11    MMA issuer of O += P(g) V(g), a thread of its own: each issuer waits on its own
+//              barriers while the other's products run, so the tensor core is fed from two queues.
+// TMEM columns: S_0 [0,128), S_1 [128,256), O [256,384), P_0 [384,448), P_1 [448,512).
 //
 // Every mbarrier is waited at every phase, in order, by each role that waits on it (a parity
 // wait is only meaningful within one phase); the host-side protocol model in the tests replays
@@ -58,7 +63,8 @@ namespace {
 constexpr int kD = 128;
 constexpr int kBM = 128;                 // query rows per item
 constexpr int kBN = 128;                 // keys per block / clusters per chunk
-constexpr int kKStages = 2;             // key / centroid tiles (freed as soon as S is computed)
+constexpr int kQStages = 1;             // query tiles (freed once the item's last S is computed)
+constexpr int kKStages = 3;             // key / centroid tiles (freed as soon as S is computed)
 constexpr int kVStages = 2;             // value / mean tiles (freed after P V)
 constexpr int kBStages = 4;             // bias rows of the softmax (even: a slot serves one warpgroup)
 constexpr int kTile = kBN * kD * 2;      // 32 KB bf16 tile
@@ -69,6 +75,7 @@ constexpr int kThreads = 384;           // three warpgroups; warp 11 idle
 constexpr int kWarpProducer = 8;
 constexpr int kWarpMMA = 9;
 constexpr int kWarpProducerV = 10;
+constexpr int kWarpPV = 11;
 // Register split (setmaxnreg): the launch holds 384 x 168 registers; the softmax warpgroups grow,
 // the producer / MMA warpgroup shrinks.
 constexpr int kRegSoftmax = 232, kRegIssue = 40;
@@ -79,7 +86,7 @@ static_assert(kEntRows == kBN && kEntPanel == (size_t)kPanel, "entry tiles are r
 constexpr uint32_t kColS = 0, kColO = 256, kColP = 384;
 
 struct __align__(8) Bars {
-  uint64_t q_full[2], q_empty[2];        // query tile of item n in buffer n & 1
+  uint64_t q_full[kQStages], q_empty[kQStages];   // query tile of item n in buffer n % kQStages
   uint64_t k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
   uint64_t b_full[kBStages], b_empty[kBStages];
   uint64_t s_full[2];                    // S(g) computed into S_{g & 1}
@@ -87,7 +94,7 @@ struct __align__(8) Bars {
   uint64_t p_ready[2];                   // P(g) written into P_{g & 1}
   uint64_t p_free[2];                    // P(g) V(g) done: P_{g & 1} reusable, O holds step g
   uint64_t m_pub[2];                     // warpgroup X published its running max of step g
-  uint64_t o_free, drain;
+  uint64_t o_free, drain[2];
   // (max, sum) published at the end of an item: [item parity][warpgroup].  One barrier per item
   // parity: a warpgroup without steps in an item could otherwise complete a barrier twice before
   // the other warpgroup's parity wait on it runs.
@@ -103,7 +110,7 @@ struct __align__(8) Bars {
   int e8[2][kEntSlots];
 };
 
-constexpr size_t kSmemBytes = 1024 + 2 * kTile /*Q*/ + (kKStages + kVStages) * kTile /*K,V*/ +
+constexpr size_t kSmemBytes = 1024 + (kQStages + kKStages + kVStages) * kTile /*Q,K,V*/ +
                               kBStages * kBN * sizeof(float) /*bias*/ + sizeof(Bars);
 static_assert(kSmemBytes <= 232448, "shared memory above the 227 KB per-block limit");
 
@@ -123,6 +130,14 @@ struct Params {
   int N, C, nB, n_items, nchunk, cpad;
   float scale_log2;
 };
+
+// One arrival per warp: the lanes' earlier shared-memory and tensor-memory accesses are ordered
+// before lane 0's arrive by the warp barrier (barrier counts are in warps, not threads, so that an
+// arrival is one shared-memory atomic instead of 32).
+__device__ __forceinline__ void warp_arrive(uint64_t* bar, int lane) {
+  __syncwarp();
+  if (lane == 0) mbar_arrive(bar);
+}
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -218,6 +233,41 @@ __device__ __forceinline__ void reg_fence32(uint32_t (&r)[32]) {
                  "+r"(r[29]), "+r"(r[30]), "+r"(r[31]));
 }
 
+// Columns [0, 64) of the O row at o_col, times inv, stored as bf16 to out (warp-collective; once
+// per item, so kept out of line).
+__device__ __forceinline__ void store_row_half(uint32_t o_col, __nv_bfloat16* out, float inv, bool live) {
+#pragma unroll 1
+  for (int q = 0; q < 2; ++q) {
+    uint32_t ra[32];
+    tmem_ld32(o_col + 32 * q, ra);
+    tmem_wait_ld();
+    if (live) {
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        uint4 w;
+        w.x = pack_bf16x2(__uint_as_float(ra[8 * v + 0]) * inv, __uint_as_float(ra[8 * v + 1]) * inv);
+        w.y = pack_bf16x2(__uint_as_float(ra[8 * v + 2]) * inv, __uint_as_float(ra[8 * v + 3]) * inv);
+        w.z = pack_bf16x2(__uint_as_float(ra[8 * v + 4]) * inv, __uint_as_float(ra[8 * v + 5]) * inv);
+        w.w = pack_bf16x2(__uint_as_float(ra[8 * v + 6]) * inv, __uint_as_float(ra[8 * v + 7]) * inv);
+        *reinterpret_cast<uint4*>(out + q * 32 + v * 8) = w;
+      }
+    }
+  }
+}
+
+// O row *= alpha in tensor memory (warp-collective; rare).
+__device__ __forceinline__ void rescale_row(uint32_t o_row, float alpha) {
+#pragma unroll 1
+  for (int q = 0; q < 4; ++q) {
+    uint32_t rr[32];
+    tmem_ld32(o_row + q * 32, rr);
+    tmem_wait_ld();
+#pragma unroll
+    for (int v = 0; v < 32; ++v) rr[v] = __float_as_uint(__uint_as_float(rr[v]) * alpha);
+    tmem_st32(o_row + q * 32, rr);
+  }
+}
+
 // Softmax of one S row held in registers (128 columns as raw fp32 bits).  A column's logit in
 // log2 units is y_c = x_c * s*log2(e) + bias_c.  On a full key block the bias row is zero and
 // the row max is taken on the raw scores (the scale is positive); otherwise y is formed in
@@ -280,8 +330,8 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-  uint8_t* sQ = base;                             // two query tiles
-  uint8_t* sK = sQ + 2 * kTile;                   // kKStages tiles
+  uint8_t* sQ = base;                             // kQStages query tiles
+  uint8_t* sK = sQ + kQStages * kTile;            // kKStages tiles
   uint8_t* sV = sK + kKStages * kTile;            // kVStages tiles
   float* sBias = reinterpret_cast<float*>(sV + kVStages * kTile);   // [kBStages][kBN]
   Bars* bars = reinterpret_cast<Bars*>(sBias + kBStages * kBN);
@@ -291,15 +341,17 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 
   if (tid == 0) {
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&bars->q_full[b], 1);
-      mbar_init(&bars->q_empty[b], 1);
       mbar_init(&bars->s_full[b], 1);
-      mbar_init(&bars->s_free[b], 128);
-      mbar_init(&bars->p_ready[b], 128);
+      mbar_init(&bars->s_free[b], 4);
+      mbar_init(&bars->p_ready[b], 4);
       mbar_init(&bars->p_free[b], 1);
-      mbar_init(&bars->m_pub[b], 128);
-      mbar_init(&bars->xch_full[b][0], 128);
-      mbar_init(&bars->xch_full[b][1], 128);
+      mbar_init(&bars->m_pub[b], 4);
+      mbar_init(&bars->xch_full[b][0], 4);
+      mbar_init(&bars->xch_full[b][1], 4);
+    }
+    for (int s = 0; s < kQStages; ++s) {
+      mbar_init(&bars->q_full[s], 1);
+      mbar_init(&bars->q_empty[s], 1);
     }
     for (int s = 0; s < kKStages; ++s) {
       mbar_init(&bars->k_full[s], 1);
@@ -311,10 +363,11 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     }
     for (int s = 0; s < kBStages; ++s) {
       mbar_init(&bars->b_full[s], 1);
-      mbar_init(&bars->b_empty[s], 128);
+      mbar_init(&bars->b_empty[s], 4);
     }
-    mbar_init(&bars->o_free, 256);
-    mbar_init(&bars->drain, 1);
+    mbar_init(&bars->o_free, 8);
+    mbar_init(&bars->drain[0], 1);
+    mbar_init(&bars->drain[1], 1);
     bars->abort = 0;
     fence_mbar_init();
   }
@@ -349,10 +402,11 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       for (int k = blockIdx.x; k < p.n_items && !*abort; k += gridDim.x) {
         const Item it = item_at(p, k);
         int cs = 0, cr = 0;                // entry cursor: selected slot, source row
-        if (!mbar_wait(&bars->q_empty[n & 1], ((n >> 1) & 1) ^ 1, abort, status)) break;
-        mbar_expect_tx(&bars->q_full[n & 1], kTile);
-        tma_load_3d(sQ + (n & 1) * kTile, &tm_q, &bars->q_full[n & 1], 0, it.q0, it.bh);
-        tma_load_3d(sQ + (n & 1) * kTile + kPanel, &tm_q, &bars->q_full[n & 1], 64, it.q0, it.bh);
+        const int qs = n % kQStages;
+        if (!mbar_wait(&bars->q_empty[qs], ((n / kQStages) & 1) ^ 1, abort, status)) break;
+        mbar_expect_tx(&bars->q_full[qs], kTile);
+        tma_load_3d(sQ + qs * kTile, &tm_q, &bars->q_full[qs], 0, it.q0, it.bh);
+        tma_load_3d(sQ + qs * kTile + kPanel, &tm_q, &bars->q_full[qs], 64, it.q0, it.bh);
         ++n;
         bool ok = true;
         for (int s = 0; s < it.T; ++s, ++g) {
@@ -419,7 +473,8 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       }
       // no copy may still be in flight when the CTA leaves (this matters only after an abort:
       // otherwise the consumers have waited for every load)
-      for (int nd = n >= 2 ? n - 2 : 0; nd < n; ++nd) mbar_wait_drain(&bars->q_full[nd & 1], (nd >> 1) & 1);
+      for (int nd = n >= kQStages ? n - kQStages : 0; nd < n; ++nd)
+        mbar_wait_drain(&bars->q_full[nd % kQStages], (nd / kQStages) & 1);
       for (uint32_t gd = g >= kKStages ? g - kKStages : 0; gd < g; ++gd)
         mbar_wait_drain(&bars->k_full[gd % kKStages], (gd / kKStages) & 1);
       for (uint32_t gd = g >= kBStages ? g - kBStages : 0; gd < g; ++gd)
@@ -471,81 +526,70 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         mbar_wait_drain(&bars->v_full[gd % kVStages], (gd / kVStages) & 1);
     }
   } else if (warp == kWarpMMA) {
-    // ------------------------------------------------------------------ MMA issuer
-    // Two cursors over the CTA's steps: S runs two steps ahead of P V.  S(g + 2) goes into the S
-    // buffer that softmax(g) has just read into registers, so it overlaps softmax(g); P V(g)
-    // follows once P(g) is written.  The tensor core executes in issue order.
+    // ------------------------------------------------------------------ MMA issuer of S = Q K^T
+    // S(g) goes into the score buffer S_{g & 1} as soon as softmax(g - 2) has read it into
+    // registers, so it overlaps that softmax.  Products of this thread and of the P V issuer
+    // (warp 11) share the tensor core; each thread's commits track its own products.
     if (lane == 0) {
       const uint32_t idesc_qk = idesc_bf16(kBM, kBN, 0, 0);   // Q, K both K-major
-      const uint32_t idesc_pv = idesc_bf16(kBM, kD, 0, 1);    // P from TMEM, V MN-major
-      // S cursor: schedule index, item count, step in the item, global step
-      int sk = blockIdx.x, sn = 0, ss = 0;
-      uint32_t sg = 0;
-      int sT = sk < p.n_items ? item_at(p, sk).T : 0;
-      // P V cursor
-      int pk = blockIdx.x, pn = 0, ps = 0;
-      uint32_t pg = 0;
-      int pT = pk < p.n_items ? item_at(p, pk).T : 0;
-      auto issue_s = [&]() -> bool {
-        if (ss == 0) {
-          if (!mbar_wait(&bars->q_full[sn & 1], (sn >> 1) & 1, abort, status)) return false;
-        }
-        const int ks = sg % kKStages;
-        if (!mbar_wait(&bars->k_full[ks], (sg / kKStages) & 1, abort, status)) return false;
-        tc_fence_after();
-        const uint32_t qb = smem_u32(sQ + (sn & 1) * kTile), kb = smem_u32(sK + ks * kTile);
-        const uint32_t d = tmem + kColS + (sg & 1) * kBN;
-#pragma unroll
-        for (int kk = 0; kk < kD / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kPanel + (kk & 3) * 32;
-          umma_ss(d, sdesc_sw128(qb + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), idesc_qk, kk > 0);
-        }
-        umma_commit(&bars->s_full[sg & 1]);
-        umma_commit(&bars->k_empty[ks]);
-        if (ss == sT - 1) umma_commit(&bars->q_empty[sn & 1]);
-        ++sg;
-        if (++ss == sT) {
-          ss = 0;
-          ++sn;
-          sk += gridDim.x;
-          sT = sk < p.n_items ? item_at(p, sk).T : 0;
-        }
-        return true;
-      };
+      uint32_t g = 0;
+      int n = 0;
       bool ok = true;
-      for (int i = 0; i < 2 && sT > 0 && ok; ++i) ok = issue_s();
-      while (ok && pT > 0) {
-        // S two steps ahead, once softmax(pg) has read S_{pg & 1}
-        if (sT > 0) {
-          if (!mbar_wait(&bars->s_free[pg & 1], (pg >> 1) & 1, abort, status)) break;
-          if (!issue_s()) break;
-        }
-        const int vs = pg % kVStages;
-        if (!mbar_wait(&bars->p_ready[pg & 1], (pg >> 1) & 1, abort, status)) break;
-        if (!mbar_wait(&bars->v_full[vs], (pg / kVStages) & 1, abort, status)) break;
-        if (ps == 0 && !mbar_wait(&bars->o_free, (pn & 1) ^ 1, abort, status)) break;
-        tc_fence_after();
-        const uint32_t vb = smem_u32(sV + vs * kTile);
-        const uint32_t pt = tmem + kColP + (pg & 1) * (kBN / 2);   // P(pg): bf16 pairs, 64 columns
+      for (int k = blockIdx.x; k < p.n_items && ok; k += gridDim.x, ++n) {
+        const int T = item_at(p, k).T;
+        const int qs = n % kQStages;
+        const uint32_t qb = smem_u32(sQ + qs * kTile);
+        for (int s = 0; s < T; ++s, ++g) {
+          if (g >= 2 && !mbar_wait(&bars->s_free[g & 1], ((g - 2) >> 1) & 1, abort, status)) { ok = false; break; }
+          if (s == 0 && !mbar_wait(&bars->q_full[qs], (n / kQStages) & 1, abort, status)) { ok = false; break; }
+          const int ks = g % kKStages;
+          if (!mbar_wait(&bars->k_full[ks], (g / kKStages) & 1, abort, status)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t kb = smem_u32(sK + ks * kTile);
+          const uint32_t d = tmem + kColS + (g & 1) * kBN;
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          // V rows (keys) 16 kk .. 16 kk + 15: two 8-row groups of 1024 B; the first product of an
-          // item overwrites O
-          umma_ts(tmem + kColO, pt + kk * 8, sdesc_sw128(vb + kk * 2048, kPanel, 1024), idesc_pv,
-                  (ps > 0 || kk > 0) ? 1u : 0u);
-        }
-        umma_commit(&bars->v_empty[vs]);
-        umma_commit(&bars->p_free[pg & 1]);
-        ++pg;
-        if (++ps == pT) {
-          ps = 0;
-          ++pn;
-          pk += gridDim.x;
-          pT = pk < p.n_items ? item_at(p, pk).T : 0;
+          for (int kk = 0; kk < kD / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * kPanel + (kk & 3) * 32;
+            umma_ss(d, sdesc_sw128(qb + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), idesc_qk, kk > 0);
+          }
+          umma_commit(&bars->s_full[g & 1]);
+          umma_commit(&bars->k_empty[ks]);
+          if (s == T - 1) umma_commit(&bars->q_empty[qs]);
         }
       }
-      umma_commit(&bars->drain);
-      mbar_wait_drain(&bars->drain, 0);
+      umma_commit(&bars->drain[0]);
+      mbar_wait_drain(&bars->drain[0], 0);
+    }
+  } else if (warp == kWarpPV) {
+    // ------------------------------------------------------------------ MMA issuer of O += P V
+    if (lane == 0) {
+      const uint32_t idesc_pv = idesc_bf16(kBM, kD, 0, 1);    // P from TMEM, V MN-major
+      uint32_t g = 0;
+      int n = 0;
+      bool ok = true;
+      for (int k = blockIdx.x; k < p.n_items && ok; k += gridDim.x, ++n) {
+        const int T = item_at(p, k).T;
+        for (int s = 0; s < T; ++s, ++g) {
+          const int vs = g % kVStages;
+          if (!mbar_wait(&bars->p_ready[g & 1], (g >> 1) & 1, abort, status)) { ok = false; break; }
+          if (!mbar_wait(&bars->v_full[vs], (g / kVStages) & 1, abort, status)) { ok = false; break; }
+          if (s == 0 && !mbar_wait(&bars->o_free, (n & 1) ^ 1, abort, status)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t vb = smem_u32(sV + vs * kTile);
+          const uint32_t pt = tmem + kColP + (g & 1) * (kBN / 2);   // P(g): bf16 pairs, 64 columns
+#pragma unroll
+          for (int kk = 0; kk < kBN / 16; ++kk) {
+            // V rows (keys) 16 kk .. 16 kk + 15: two 8-row groups of 1024 B; the first product of
+            // an item overwrites O
+            umma_ts(tmem + kColO, pt + kk * 8, sdesc_sw128(vb + kk * 2048, kPanel, 1024), idesc_pv,
+                    (s > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&bars->v_empty[vs]);
+          umma_commit(&bars->p_free[g & 1]);
+        }
+      }
+      umma_commit(&bars->drain[1]);
+      mbar_wait_drain(&bars->drain[1], 0);
     }
   } else if (warp < 8) {
     // ------------------------------------------------------------------ softmax (warps 0-7)
@@ -588,7 +632,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         reg_fence32(x[2]);
         reg_fence32(x[3]);
         tc_fence_before();
-        mbar_arrive(&bars->s_free[X]);
+        warp_arrive(&bars->s_free[X], lane);
         const float mx = row_logits_max(x, bt, plain, p.scale_log2);
         // The running max is shared by the two warpgroups (one accumulator O): take the other's
         // latest one (every phase of m_pub is waited, in order), and let it move only when it grows
@@ -603,7 +647,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const bool grow = mx > mprev + kRescaleLog2 || (mprev == -INFINITY && mx > -INFINITY);
         const float m_new = grow ? mx : mprev;
         bars->mrow[X][r] = m_new;
-        mbar_arrive(&bars->m_pub[X]);
+        warp_arrive(&bars->m_pub[X], lane);
         const float mu = (m_new == -INFINITY) ? 0.f : m_new;
         // the row's probabilities, packed to bf16 pairs in registers (each chunk of scores dies as
         // its probabilities are formed)
@@ -623,7 +667,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
 #pragma unroll
         for (int q = 0; q < 4; ++q) tmem_st16(p_own + q * 16, pk[q]);
-        mbar_arrive(&bars->b_empty[bs]);          // this thread has read the bias row
+        warp_arrive(&bars->b_empty[bs], lane);    // the warp has read the bias row
         float rs_lo, rs_hi;
         f2_unpack(rsum, rs_lo, rs_hi);
         const float rs = rs_lo + rs_hi;
@@ -636,16 +680,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           const bool d_ok = mbar_wait(&bars->p_free[X ^ 1], ((g - 1) >> 1) & 1, abort, status);
           if (!__all_sync(0xffffffffu, d_ok)) { ok = false; break; }
           tc_fence_after();
-          const float alpha = need_o ? ex2(mprev - m_new) : 1.f;
-#pragma unroll 1
-          for (int q = 0; q < 4; ++q) {
-            uint32_t rr[32];
-            tmem_ld32(o_row + q * 32, rr);
-            tmem_wait_ld();
-#pragma unroll
-            for (int v = 0; v < 32; ++v) rr[v] = __float_as_uint(__uint_as_float(rr[v]) * alpha);
-            tmem_st32(o_row + q * 32, rr);
-          }
+          rescale_row(o_row, need_o ? ex2(mprev - m_new) : 1.f);
         }
         if (m_new != m_at) {                      // the running max only grows
           if (m_at > -INFINITY) l *= ex2(m_at - m_new);
@@ -654,7 +689,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         l += (flag & 2) ? -rs : rs;               // entry tiles take their weight out again
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&bars->p_ready[X]);
+        warp_arrive(&bars->p_ready[X], lane);
       }
       if (!ok) break;
       // epilogue: once the item's last product has landed, exchange (max, sum) per row with the
@@ -665,7 +700,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       bool e_ok = gl < 1 || mbar_wait(&bars->p_free[(gl - 1) & 1], ((gl - 1) >> 1) & 1, abort, status);
       e_ok = e_ok && mbar_wait(&bars->p_free[gl & 1], (gl >> 1) & 1, abort, status);
       bars->xch[n & 1][X][r] = make_float2(m_at, l);
-      mbar_arrive(&bars->xch_full[n & 1][X]);
+      warp_arrive(&bars->xch_full[n & 1][X], lane);
       e_ok = e_ok && mbar_wait(&bars->xch_full[n & 1][X ^ 1], (n >> 1) & 1, abort, status);
       if (!__all_sync(0xffffffffu, e_ok)) break;
       tc_fence_after();
@@ -676,27 +711,10 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       const float L = e0.y * f0 + e1.y * f1;
       const float inv = L > 0.f ? 1.f / L : 0.f;
       const bool live = r < it.qlen;
-      __nv_bfloat16* op = p.O + ((size_t)it.bh * p.N + it.q0 + r) * kD + 64 * X;
-#pragma unroll 1
-      for (int q = 0; q < 2; ++q) {
-        uint32_t ra[32];
-        tmem_ld32(o_row + 64 * X + 32 * q, ra);
-        tmem_wait_ld();
-        if (live) {
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(ra[8 * v + 0]) * inv, __uint_as_float(ra[8 * v + 1]) * inv);
-            w.y = pack_bf16x2(__uint_as_float(ra[8 * v + 2]) * inv, __uint_as_float(ra[8 * v + 3]) * inv);
-            w.z = pack_bf16x2(__uint_as_float(ra[8 * v + 4]) * inv, __uint_as_float(ra[8 * v + 5]) * inv);
-            w.w = pack_bf16x2(__uint_as_float(ra[8 * v + 6]) * inv, __uint_as_float(ra[8 * v + 7]) * inv);
-            *reinterpret_cast<uint4*>(op + q * 32 + v * 8) = w;
-          }
-        }
-      }
+      store_row_half(o_row + 64 * X, p.O + ((size_t)it.bh * p.N + it.q0 + r) * kD + 64 * X, inv, live);
       if (X == 0 && live && p.lse) p.lse[(size_t)it.bh * p.N + it.q0 + r] = (M + __log2f(L)) * 0.69314718055994531f;
       tc_fence_before();
-      mbar_arrive(&bars->o_free);
+      warp_arrive(&bars->o_free, lane);
       g0 += it.T;
     }
   }

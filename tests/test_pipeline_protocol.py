@@ -20,8 +20,9 @@ completing loads in any order, under many random interleavings, and checks that
 It mirrors the step structure of attention_tc.cu: per work item, one step per
 selected block, one per 128-cluster chunk, then one per entry tile of the
 selected blocks' cluster entries; double-buffered query tiles; key, value and
-bias-row rings; the MMA issuer running S two steps ahead of P V, S(g + 2) into
-the score buffer softmax(g) has just read; softmax warpgroup X taking the steps
+bias-row rings; two MMA issuing threads, one for S = Q K^T (S(g) into the
+score buffer softmax(g - 2) has just read) and one for O += P V, each with its
+own commits; softmax warpgroup X taking the steps
 g with g & 1 == X, with its own score buffer S_X and probability tile P_X; one
 output accumulator O shared by both, with the running max passed between the
 warpgroups at every step and O rescaled by whichever raises it; at the end of
@@ -35,7 +36,8 @@ import random
 
 import pytest
 
-KSTAGES = 2   # key / centroid tiles, freed when S is computed
+QSTAGES = 1   # query tiles, freed when the item's last S is computed
+KSTAGES = 3   # key / centroid tiles, freed when S is computed
 VSTAGES = 2   # value / mean tiles, freed after P V
 BSTAGES = 4   # softmax bias rows, freed after the softmax has read them (even: one warpgroup per slot)
 
@@ -92,7 +94,8 @@ class Machine:
         self.single_q = single_q               # planted: one query buffer, with the waits of two
         self.skip_m_wait = skip_m_wait         # planted: the running max read without its barrier
         B = Barrier
-        self.q_full, self.q_empty = [B(f"q_full{i}", 1) for i in range(2)], [B(f"q_empty{i}", 1) for i in range(2)]
+        self.q_full = [B(f"q_full{i}", 1) for i in range(QSTAGES)]
+        self.q_empty = [B(f"q_empty{i}", 1) for i in range(QSTAGES)]
         self.k_full = [B(f"k_full{i}", 1) for i in range(KSTAGES)]
         self.k_empty = [B(f"k_empty{i}", 1) for i in range(KSTAGES)]
         self.v_full = [B(f"v_full{i}", 1) for i in range(VSTAGES)]
@@ -113,7 +116,9 @@ class Machine:
         self.xch = [[None, None], [None, None]]   # [item parity][warpgroup] -> item whose (max, sum) it holds
         self.o_content = None                  # (item, last step accumulated), at issue
         self.o_scaled = None                   # (item, step) of the last rescale of O
-        self.tc_queue = []                     # in-order tensor core: ("mma", reads, writes) / ("commit", bar)
+        # per issuing thread, in order: ("mma", buffers) / ("commit", bar); a commit arrives once that
+        # thread's earlier products are done (the two threads' products interleave in any order)
+        self.tc_queues = {"s": [], "pv": []}
         self.tma = []                          # in flight: (bar, buffer written, buffers read)
         self.readers = {}                      # resource -> units with an operation in flight on it
 
@@ -135,20 +140,26 @@ class Machine:
         assert not busy, f"{who} overwrites {res} while {busy} use it"
 
     # ---- asynchronous units
-    def tc_issue_mma(self, reads, writes):
+    def tc_issue_mma(self, q, reads, writes):
         for w in writes:
             self._write(w, "tensor core", unit="tc")
         for r in reads + writes:     # the destination is busy until the MMA completes
             self._start_read(r, "tc")
-        self.tc_queue.append(("mma", reads + writes))
+        self.tc_queues[q].append(("mma", reads + writes))
 
-    def tc_commit(self, bar):
-        self.tc_queue.append(("commit", bar))
+    def tc_commit(self, q, bar):
+        self.tc_queues[q].append(("commit", bar))
+
+    @property
+    def tc_busy(self):
+        return any(self.tc_queues.values())
 
     def step_units(self):
         progressed = False
-        if self.tc_queue and self.rng.random() < 0.5:
-            kind, x = self.tc_queue.pop(0)
+        live = [q for q in self.tc_queues.values() if q]
+        if live and self.rng.random() < 0.6:
+            q = self.rng.choice(live)
+            kind, x = q.pop(0)
             if kind == "mma":
                 for r in x:
                     self._end_read(r, "tc")
@@ -176,7 +187,7 @@ class Machine:
         assert self.version.get(res) == step, f"{res} holds step {self.version.get(res)}, read at step {step}"
 
     def qbuf(self, n):
-        return 0 if self.single_q else n & 1
+        return 0 if self.single_q else n % QSTAGES
 
     # ---- roles (generators yield a predicate to wait on)
     def producer(self):
@@ -184,9 +195,10 @@ class Machine:
         g = 0
         for n in range(len(self.items)):
             qb = self.qbuf(n)
-            yield lambda: self.q_empty[n & 1].test((n >> 1) - 1)
-            self.q_full[n & 1].expect_tx(1)
-            self.tma_load(self.q_full[n & 1], f"Q{qb}", ("q", n))
+            qs = n % QSTAGES
+            yield lambda: self.q_empty[qs].test(n // QSTAGES - 1)
+            self.q_full[qs].expect_tx(1)
+            self.tma_load(self.q_full[qs], f"Q{qb}", ("q", n))
             for s in range(self.T(n)):
                 ks, bs = g % KSTAGES, g % BSTAGES
                 yield lambda: self.k_empty[ks].test(g // KSTAGES - 1)
@@ -221,34 +233,27 @@ class Machine:
                 yield n, s, g
                 g += 1
 
-    def mma(self):
-        steps = list(self._steps())
-        si = 0                                  # S cursor (index into steps)
-
-        def issue_s():
-            nonlocal si
-            n, s, g = steps[si]
+    def mma_s(self):
+        """The issuer of S = Q K^T: S(g) once softmax(g - 2) has read S_{g & 1}."""
+        for n, s, g in self._steps():
             qb = self.qbuf(n)
+            if g >= 2:
+                yield lambda: self.s_free[g & 1].test((g - 2) >> 1)
             if s == 0:
-                yield lambda: self.q_full[n & 1].test(n >> 1)
+                yield lambda: self.q_full[n % QSTAGES].test(n // QSTAGES)
             yield lambda: self.k_full[g % KSTAGES].test(g // KSTAGES)
             self.holds(f"Q{qb}", ("q", n))
             self.holds(f"K{g % KSTAGES}", g)
-            self.tc_issue_mma([f"Q{qb}", f"K{g % KSTAGES}"], [f"S{g & 1}"])
+            self.tc_issue_mma("s", [f"Q{qb}", f"K{g % KSTAGES}"], [f"S{g & 1}"])
             self.version[f"S{g & 1}"] = g
-            self.tc_commit(self.s_full[g & 1])
-            self.tc_commit(self.k_empty[g % KSTAGES])
+            self.tc_commit("s", self.s_full[g & 1])
+            self.tc_commit("s", self.k_empty[g % KSTAGES])
             if s == self.T(n) - 1:
-                self.tc_commit(self.q_empty[n & 1])
-            si += 1
+                self.tc_commit("s", self.q_empty[n % QSTAGES])
 
-        for _ in range(2):
-            if si < len(steps):
-                yield from issue_s()
-        for n, s, g in steps:
-            if si < len(steps):
-                yield lambda: self.s_free[g & 1].test(g >> 1)
-                yield from issue_s()
+    def mma_pv(self):
+        """The issuer of O += P V: P V(g) once P(g) is written."""
+        for n, s, g in self._steps():
             yield lambda: self.p_ready[g & 1].test(g >> 1)
             yield lambda: self.v_full[g % VSTAGES].test(g // VSTAGES)
             if s == 0:
@@ -257,10 +262,10 @@ class Machine:
             self.holds(f"P{g & 1}", g)
             if s > 0:
                 assert self.o_content == (n, g - 1), f"O holds {self.o_content} before P V of step {g}"
-            self.tc_issue_mma([f"P{g & 1}", f"V{g % VSTAGES}"], ["O"])
+            self.tc_issue_mma("pv", [f"P{g & 1}", f"V{g % VSTAGES}"], ["O"])
             self.o_content = (n, g)
-            self.tc_commit(self.v_empty[g % VSTAGES])
-            self.tc_commit(self.p_free[g & 1])
+            self.tc_commit("pv", self.v_empty[g % VSTAGES])
+            self.tc_commit("pv", self.p_free[g & 1])
 
     def softmax(self, X):
         g0 = 0
@@ -322,11 +327,11 @@ class Machine:
             g0 += T
 
     def run(self, max_iters=400000):
-        roles = [self.producer(), self.producer_v(), self.mma(), self.softmax(0), self.softmax(1)]
+        roles = [self.producer(), self.producer_v(), self.mma_s(), self.mma_pv(), self.softmax(0), self.softmax(1)]
         waits = [None] * len(roles)
         done = [False] * len(roles)
         for _ in range(max_iters):
-            if all(done) and not self.tc_queue and not self.tma:
+            if all(done) and not self.tc_busy and not self.tma:
                 return True
             order = list(range(len(roles)))
             self.rng.shuffle(order)
@@ -345,7 +350,7 @@ class Machine:
                 if self.rng.random() < 0.5:
                     break
             progressed = self.step_units() or progressed
-            if not progressed and not self.tc_queue and not self.tma:
+            if not progressed and not self.tc_busy and not self.tma:
                 raise AssertionError("deadlock: no role can progress")
         raise AssertionError("did not finish")
 
@@ -408,9 +413,10 @@ def test_model_catches_a_rescale_during_the_previous_product():
     assert _caught([6, 4], 2, no_rescale_wait=True) > 0
 
 
+@pytest.mark.skipif(QSTAGES < 2, reason="one query buffer is the design: its waits are those of one buffer")
 def test_model_catches_a_single_query_buffer():
-    """With S two steps ahead of P V, the next item's first S is issued while the current item's
-    query tile is still read; one buffer would be overwritten."""
+    """Two query buffers waited as two while one is used: the next item's query tile would
+    overwrite the one the current item's S still reads."""
     assert _caught([1, 1, 1, 1, 2, 1], 1, single_q=True) > 0
 
 
