@@ -32,8 +32,8 @@
 //   warps 0-3, 4-7  two softmax warpgroups X = 0, 1 (barriers they arrive on count warps: lane 0
 //              arrives after a warp barrier); warpgroup X takes the steps g with g & 1 = X of
 //              every item, so the two overlap each other and the tensor core.  Thread t of a
-//              warpgroup owns query row t = TMEM lane t.  It reads S_X into registers (S_X is then
-//              free for S(g + 2)), takes the running max of the other warpgroup's latest step and
+//              warpgroup owns query row t = TMEM lane t.  It reads S into registers (S is then
+//              free for S(g + 1)), takes the running max of the other warpgroup's latest step and
 //              lets it grow lazily (only by more than 2^8), writes P as bf16 into its own P_X and
 //              keeps its share of the row sum.  The two share one accumulator O: whichever raises
 //              the max rescales O, once the previous product has landed.  At the end of an item
@@ -41,13 +41,14 @@
 //   warp 8     producer: loads Q, key tiles / centroid chunks / entry centroid rows (3-stage ring,
 //              so that a key tile loads while the two before it are read) and the softmax bias rows (4-stage ring, so a slot always serves the
 //              same warpgroup);
-//   warp 9     MMA issuer of S(g) = Q K^T into S_{g & 1} once softmax(g - 2) has read it (and TMEM
-//              allocation); S thus overlaps the softmax of two steps before;
+//   warp 9     MMA issuer of S(g) = Q K^T (and TMEM allocation): at an item's start it copies the
+//              query tile into tensor memory (tcgen05.cp), so S reads only the key tile from shared
+//              memory; S(g) goes into the one score buffer once softmax(g - 1) has read it;
 //   warp 10    producer of value tiles / cluster means / entry means (2-stage ring); a warp of its
 //              own, since divergent lanes of one warp waiting on different barriers hold each other up;
 //   warp 11    MMA issuer of O += P(g) V(g), a thread of its own: each issuer waits on its own
 //              barriers while the other's products run, so the tensor core is fed from two queues.
-// TMEM columns: S_0 [0,128), S_1 [128,256), O [256,384), P_0 [384,448), P_1 [448,512).
+// TMEM columns: S [0,128), O [128,256), P_0 [256,320), P_1 [320,384), Q_0 [384,448), Q_1 [448,512).
 //
 // Every mbarrier is waited at every phase, in order, by each role that waits on it (a parity
 // wait is only meaningful within one phase); the host-side protocol model in the tests replays
@@ -82,8 +83,9 @@ constexpr int kRegSoftmax = 232, kRegIssue = 40;
 static_assert(128 * (2 * kRegSoftmax + kRegIssue) <= kThreads * 168, "register split above the launch");
 static_assert(kBStages % 2 == 0, "a bias slot must always serve the same softmax warpgroup");
 static_assert(kEntRows == kBN && kEntPanel == (size_t)kPanel, "entry tiles are read as key / value tiles");
-// TMEM columns: the two score buffers, the one output accumulator, the two bf16 probability tiles
-constexpr uint32_t kColS = 0, kColO = 256, kColP = 384;
+// TMEM columns: the score buffer, the output accumulator, the two bf16 probability tiles and the
+// two bf16 query tiles (the A operand of S = Q K^T, by item parity)
+constexpr uint32_t kColS = 0, kColO = 128, kColP = 256, kColQ = 384;
 
 struct __align__(8) Bars {
   uint64_t q_full[kQStages], q_empty[kQStages];   // query tile of item n in buffer n % kQStages
@@ -323,6 +325,15 @@ __device__ __forceinline__ void chunk_exp(const uint32_t (&x)[32], uint64_t coef
   rsum = f2_add(rsum, f2_add(s0, s1));
 }
 
+// pk (bf16 pairs) *= f, in place.
+__device__ __forceinline__ void scale_bf16x2(uint32_t (&pk)[16], float f) {
+#pragma unroll
+  for (int v = 0; v < 16; ++v) {
+    const float lo = __uint_as_float(pk[v] << 16), hi = __uint_as_float(pk[v] & 0xFFFF0000u);
+    pk[v] = pack_bf16x2(lo * f, hi * f);
+  }
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_c,
@@ -527,9 +538,10 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     }
   } else if (warp == kWarpMMA) {
     // ------------------------------------------------------------------ MMA issuer of S = Q K^T
-    // S(g) goes into the score buffer S_{g & 1} as soon as softmax(g - 2) has read it into
-    // registers, so it overlaps that softmax.  Products of this thread and of the P V issuer
-    // (warp 11) share the tensor core; each thread's commits track its own products.
+    // The item's query tile is copied into tensor memory first, so that S reads only the key tile
+    // from shared memory; S(g) goes into the score buffer as soon as softmax(g - 1) has read it into
+    // registers.  Products of this thread and of the P V issuer (warp 11) share the tensor core; each
+    // thread's commits track its own products (and its copies, which run in order with them).
     if (lane == 0) {
       const uint32_t idesc_qk = idesc_bf16(kBM, kBN, 0, 0);   // Q, K both K-major
       uint32_t g = 0;
@@ -539,22 +551,31 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const int T = item_at(p, k).T;
         const int qs = n % kQStages;
         const uint32_t qb = smem_u32(sQ + qs * kTile);
+        const uint32_t qt = tmem + kColQ + (n & 1) * (kD / 2);    // this item's query tile
         for (int s = 0; s < T; ++s, ++g) {
-          if (g >= 2 && !mbar_wait(&bars->s_free[g & 1], ((g - 2) >> 1) & 1, abort, status)) { ok = false; break; }
-          if (s == 0 && !mbar_wait(&bars->q_full[qs], (n / kQStages) & 1, abort, status)) { ok = false; break; }
+          if (s == 0) {
+            // the query tile into tensor memory (in order with this thread's products; the copy of
+            // item n + 2 into the same columns follows item n's last S)
+            if (!mbar_wait(&bars->q_full[qs], (n / kQStages) & 1, abort, status)) { ok = false; break; }
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < kD / 16; ++kk)
+              tmem_cp_128x256b(qt + kk * 8, sdesc_sw128(qb + (kk >> 2) * kPanel + (kk & 3) * 32, 16, 1024));
+            umma_commit(&bars->q_empty[qs]);
+          }
+          // the one score buffer is free once softmax(g - 1) has read it
+          if (g >= 1 && !mbar_wait(&bars->s_free[(g - 1) & 1], ((g - 1) >> 1) & 1, abort, status)) { ok = false; break; }
           const int ks = g % kKStages;
           if (!mbar_wait(&bars->k_full[ks], (g / kKStages) & 1, abort, status)) { ok = false; break; }
           tc_fence_after();
           const uint32_t kb = smem_u32(sK + ks * kTile);
-          const uint32_t d = tmem + kColS + (g & 1) * kBN;
 #pragma unroll
           for (int kk = 0; kk < kD / 16; ++kk) {
             const uint32_t off = (kk >> 2) * kPanel + (kk & 3) * 32;
-            umma_ss(d, sdesc_sw128(qb + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), idesc_qk, kk > 0);
+            umma_ts(tmem + kColS, qt + kk * 8, sdesc_sw128(kb + off, 16, 1024), idesc_qk, kk > 0);
           }
           umma_commit(&bars->s_full[g & 1]);
           umma_commit(&bars->k_empty[ks]);
-          if (s == T - 1) umma_commit(&bars->q_empty[qs]);
         }
       }
       umma_commit(&bars->drain[0]);
@@ -598,7 +619,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const int r = tid & 127;                                  // query row = TMEM lane
     const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const uint32_t o_row = lane_addr + kColO;
-    const uint32_t p_own = lane_addr + kColP + X * (kBN / 2);
+    const uint32_t p_own = lane_addr + kColP + X * (kBN / 2);   // P_X
     uint32_t g0 = 0;                                          // first step of the item
     int n = 0;
     // (no abort test in the loop condition: a warp leaves as a whole, on its __all_sync'd waits)
@@ -606,6 +627,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       const Item it = item_at(p, k);
       // m_at, l: this warpgroup's share of the row sum, expressed at the running max m_at
       float m_at = -INFINITY, l = 0.f;
+      float m_seen = -INFINITY;                               // the running max of this warpgroup's last step
       bool ok = true;
       for (int s = (int)((X - g0) & 1u); s < it.T; s += 2) {
         const uint32_t g = g0 + s;
@@ -618,7 +640,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         // Column c's logit is y_c = x_c * s*log2(e) + bias_c, the bias row in shared memory:
         // log2 n_c on a cluster chunk, log2 n_e on an entry tile, 0 on a key block (-inf past the
         // end of a short last block or of the entries).
-        const uint32_t sbase = lane_addr + kColS + X * kBN;
+        const uint32_t sbase = lane_addr + kColS;
         const float* bt = sBias + bs * kBN;
         const int flag = bars->bflag[bs];
         const bool plain = (flag & 1) && p.scale_log2 > 0.f;
@@ -634,9 +656,23 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         tc_fence_before();
         warp_arrive(&bars->s_free[X], lane);
         const float mx = row_logits_max(x, bt, plain, p.scale_log2);
-        // The running max is shared by the two warpgroups (one accumulator O): take the other's
-        // latest one (every phase of m_pub is waited, in order), and let it move only when it grows
-        // by more than 2^8 (lazy rescaling).  An item starts from -inf.
+        // The running max is shared by the two warpgroups (one accumulator O) and moves only when a
+        // row's max grows by more than 2^8 (lazy rescaling); an item starts from -inf.  The
+        // exponentials are taken with the max this warpgroup saw at its previous step, before
+        // waiting for the other warpgroup's latest one, so that the two warpgroups' exponentials do
+        // not run in lockstep; a row whose max turns out different rescales its P and sum.
+        const bool grow_g = mx > m_seen + kRescaleLog2 || (m_seen == -INFINITY && mx > -INFINITY);
+        const float m_guess = grow_g ? mx : m_seen;
+        uint64_t rsum = 0;
+        uint32_t pk[4][16];
+        {
+          const float mu = (m_guess == -INFINITY) ? 0.f : m_guess;
+          const uint64_t negmu = f2_pack(-mu, -mu);
+          const uint64_t coef = plain ? f2_pack(p.scale_log2, p.scale_log2) : f2_pack(1.f, 1.f);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) chunk_exp(x[q], coef, negmu, pk[q], rsum);
+        }
+        // the other warpgroup's running max of step g - 1 (every phase of m_pub is waited, in order)
         float mprev = -INFINITY;
         if (g >= 1) {
           const bool m_ok = mbar_wait(&bars->m_pub[X ^ 1], ((g - 1) >> 1) & 1, abort, status);
@@ -648,16 +684,16 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const float m_new = grow ? mx : mprev;
         bars->mrow[X][r] = m_new;
         warp_arrive(&bars->m_pub[X], lane);
-        const float mu = (m_new == -INFINITY) ? 0.f : m_new;
-        // the row's probabilities, packed to bf16 pairs in registers (each chunk of scores dies as
-        // its probabilities are formed)
-        uint64_t rsum = 0;
-        uint32_t pk[4][16];
-        {
-          const uint64_t negmu = f2_pack(-mu, -mu);
-          const uint64_t coef = plain ? f2_pack(p.scale_log2, p.scale_log2) : f2_pack(1.f, 1.f);
+        m_seen = m_new;
+        float rs_lo, rs_hi;
+        f2_unpack(rsum, rs_lo, rs_hi);
+        float rs = rs_lo + rs_hi;
+        if (m_new != m_guess && m_guess > -INFINITY) {
+          // P <= 2^8 either way: m_new and m_guess both lie within 2^8 above the row's max
+          const float f = ex2(m_guess - m_new);
 #pragma unroll
-          for (int q = 0; q < 4; ++q) chunk_exp(x[q], coef, negmu, pk[q], rsum);
+          for (int q = 0; q < 4; ++q) scale_bf16x2(pk[q], f);
+          rs *= f;
         }
         // P_X is free once P V(g - 2) is done (every phase of p_free[X] is waited, in order)
         if (g >= 2) {
@@ -668,9 +704,6 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 #pragma unroll
         for (int q = 0; q < 4; ++q) tmem_st16(p_own + q * 16, pk[q]);
         warp_arrive(&bars->b_empty[bs], lane);    // the warp has read the bias row
-        float rs_lo, rs_hi;
-        f2_unpack(rsum, rs_lo, rs_hi);
-        const float rs = rs_lo + rs_hi;
         // A row whose max moved rescales O, which must first hold every product up to step g - 1.
         // Only a warp that rescales waits for P V(g - 1): P V(g - 2) is known done here (p_free[X]
         // above) and P V(g + 1) cannot start before this step's P is ready, so the other

@@ -20,9 +20,10 @@ completing loads in any order, under many random interleavings, and checks that
 It mirrors the step structure of attention_tc.cu: per work item, one step per
 selected block, one per 128-cluster chunk, then one per entry tile of the
 selected blocks' cluster entries; double-buffered query tiles; key, value and
-bias-row rings; two MMA issuing threads, one for S = Q K^T (S(g) into the
-score buffer softmax(g - 2) has just read) and one for O += P V, each with its
-own commits; softmax warpgroup X taking the steps
+bias-row rings; two MMA issuing threads, one for S = Q K^T (the query tile
+copied into tensor memory at an item's start, S(g) into the one score buffer
+once softmax(g - 1) has read it) and one for O += P V, each with its own
+commits; softmax warpgroup X taking the steps
 g with g & 1 == X, with its own score buffer S_X and probability tile P_X; one
 output accumulator O shared by both, with the running max passed between the
 warpgroups at every step and O rescaled by whichever raises it; at the end of
@@ -78,7 +79,7 @@ class Barrier:
 class Machine:
     def __init__(self, items, nchunk, rng, lazy_v_wait=False, skip_b_empty=False, single_xch=False,
                  no_final_wait=False, single_xch_barrier=False, s_before_read=False, no_pfree_wait=False,
-                 no_rescale_wait=False, single_q=False, skip_m_wait=False):
+                 no_rescale_wait=False, single_q=False, skip_m_wait=False, s_early=False):
         # per item of one CTA: nsel, or (nsel, entry tiles)
         self.items = [(x, 0) if isinstance(x, int) else tuple(x) for x in items]
         self.nchunk = nchunk
@@ -93,6 +94,7 @@ class Machine:
         self.no_rescale_wait = no_rescale_wait  # planted: O rescaled without waiting for P V(g - 1)
         self.single_q = single_q               # planted: one query buffer, with the waits of two
         self.skip_m_wait = skip_m_wait         # planted: the running max read without its barrier
+        self.s_early = s_early                 # planted: S(g) issued without waiting for softmax(g - 1)
         B = Barrier
         self.q_full = [B(f"q_full{i}", 1) for i in range(QSTAGES)]
         self.q_empty = [B(f"q_empty{i}", 1) for i in range(QSTAGES)]
@@ -234,22 +236,26 @@ class Machine:
                 g += 1
 
     def mma_s(self):
-        """The issuer of S = Q K^T: S(g) once softmax(g - 2) has read S_{g & 1}."""
+        """The issuer of S = Q K^T: at an item's start it copies the query tile into tensor memory
+        (buffer n & 1; in order with its products), then S(g) into the one score buffer once
+        softmax(g - 1) has read it."""
         for n, s, g in self._steps():
             qb = self.qbuf(n)
-            if g >= 2:
-                yield lambda: self.s_free[g & 1].test((g - 2) >> 1)
             if s == 0:
                 yield lambda: self.q_full[n % QSTAGES].test(n // QSTAGES)
+                self.holds(f"Q{qb}", ("q", n))
+                self.tc_issue_mma("s", [f"Q{qb}"], [f"QT{n & 1}"])    # tcgen05.cp into tensor memory
+                self.version[f"QT{n & 1}"] = n
+                self.tc_commit("s", self.q_empty[n % QSTAGES])
+            if g >= 1 and not self.s_early:
+                yield lambda: self.s_free[(g - 1) & 1].test((g - 1) >> 1)
             yield lambda: self.k_full[g % KSTAGES].test(g // KSTAGES)
-            self.holds(f"Q{qb}", ("q", n))
+            self.holds(f"QT{n & 1}", n)
             self.holds(f"K{g % KSTAGES}", g)
-            self.tc_issue_mma("s", [f"Q{qb}", f"K{g % KSTAGES}"], [f"S{g & 1}"])
-            self.version[f"S{g & 1}"] = g
+            self.tc_issue_mma("s", [f"QT{n & 1}", f"K{g % KSTAGES}"], ["S"])
+            self.version["S"] = g
             self.tc_commit("s", self.s_full[g & 1])
             self.tc_commit("s", self.k_empty[g % KSTAGES])
-            if s == self.T(n) - 1:
-                self.tc_commit("s", self.q_empty[n % QSTAGES])
 
     def mma_pv(self):
         """The issuer of O += P V: P V(g) once P(g) is written."""
@@ -281,10 +287,11 @@ class Machine:
                 if self.s_before_read:
                     self.s_free[X].arrive()
                     yield lambda: True                 # the row is read from TMEM after the release
-                assert not self.readers.get(f"S{X}"), "S read before its MMA completed or while it is rewritten"
-                self.holds(f"S{X}", g)
+                assert not self.readers.get("S"), "S read before its MMA completed or while it is rewritten"
+                self.holds("S", g)
                 if not self.s_before_read:
                     self.s_free[X].arrive()
+                yield lambda: True                     # the row max and the exponentials
                 if g >= 1:
                     if not self.skip_m_wait:
                         yield lambda: self.m_pub[X ^ 1].test((g - 1) >> 1)
@@ -421,4 +428,14 @@ def test_model_catches_a_single_query_buffer():
 
 
 def test_model_catches_the_running_max_read_without_its_barrier():
-    assert _caught([6, 6], 2, skip_m_wait=True) > 0
+    caught = 0
+    for seed in range(400):
+        try:
+            Machine([6, 6, 3], 2, random.Random(seed), skip_m_wait=True).run()
+        except AssertionError:
+            caught += 1
+    assert caught > 0
+
+
+def test_model_catches_s_issued_before_the_previous_softmax_read_it():
+    assert _caught([5, 5], 2, s_early=True) > 0
