@@ -179,7 +179,7 @@ __device__ void block_stats_group(int t, int bar_id, const int* s_assign, int nk
         // lane l holds columns [4l, 4l + 4): panel l / 16, 16-byte chunk (l mod 16) / 2, half l mod 2
         const int n = p1 - p0;
         const int k = (lane & 15) >> 1;
-        const size_t off = (size_t)(lane >> 4) * kEntPanel + (size_t)ee * 128 + ((k ^ (ee & 7)) << 4) + ((lane & 1) << 3);
+        const size_t off = ent_byte(ee, lane >> 4, k) + ((lane & 1) << 3);
         *reinterpret_cast<uint2*>(ent_out + off) = crow;
         const float fn = (float)n;
         uint2 vv;
@@ -195,8 +195,8 @@ __device__ void block_stats_group(int t, int bar_id, const int* s_assign, int nk
       // rows [E, E8) of the four 128-row panels are zero, their bias -inf
       const int E8 = (E + 7) & ~7;
       for (int i = t; i < (E8 - E) * 32; i += NT) {
-        const int r = E + (i >> 5), panel = (i >> 3) & 3, chunk = i & 7;
-        *reinterpret_cast<uint4*>(ent_out + panel * kEntPanel + (size_t)r * 128 + chunk * 16) = make_uint4(0, 0, 0, 0);
+        const int r = E + (i >> 5), half = (i >> 4) & 1, panel = (i >> 3) & 1, chunk = i & 7;
+        *reinterpret_cast<uint4*>(ent_out + half * kEntVOff + ent_byte(r, panel, chunk)) = make_uint4(0, 0, 0, 0);
       }
       for (int r = E + t; r < E8; r += NT) reinterpret_cast<float*>(ent_out + kEntBiasOff)[r] = -INFINITY;
     }

@@ -38,10 +38,16 @@ struct WsLayout {
 WsLayout ws_layout(const Dims& g);
 
 // Compensation tiles (byte offsets inside da_cluster_stats.comp_tiles; layout in include/da.h).
+// An entry tile's operand rows come in groups of 8: group a holds the 64-column panel 0 of its
+// 8 rows (1024 B) and then panel 1 (1024 B), each 128-byte row with 16-byte chunk k stored at
+// k XOR (row mod 8).  A run of whole groups is thus one contiguous range for both panels.
 constexpr int kEntRows = 128;                           // rows of one block's entry tile (= block)
-constexpr size_t kEntPanel = 128 * 128;                  // one 64-column panel: 128 rows x 128 B
-constexpr size_t kEntVOff = 2 * kEntPanel;               // -S_e / n_e rows
-constexpr size_t kEntBiasOff = 4 * kEntPanel;            // log2 n_e per row (fp32)
+constexpr size_t kEntGroup = 2048;                       // 8 rows x 2 panels x 128 B
+constexpr size_t kEntVOff = 16 * kEntGroup;              // -S_e / n_e rows (after the 32 KB of centroid rows)
+constexpr size_t kEntBiasOff = 2 * kEntVOff;             // log2 n_e per row (fp32)
+__host__ __device__ constexpr size_t ent_byte(int row, int panel, int chunk) {
+  return (size_t)(row >> 3) * kEntGroup + (size_t)panel * 1024 + (size_t)(row & 7) * 128 + (size_t)((chunk ^ (row & 7)) << 4);
+}
 constexpr size_t kEntTileBytes = kEntBiasOff + kEntRows * sizeof(float);   // 66048
 struct CompLayout {
   size_t ent, cmean, cbias, total;

@@ -109,8 +109,10 @@ typedef struct {
  *   entry tiles   [B,H,nB] x 66048 bytes, one per key block, rows = the block's
  *                 entries e in list order, padded with zero rows (and bias
  *                 -inf) to a multiple of 8 rows:
- *                   bytes [0, 32768)      cbar_{c_e} as bf16, two 64-column
- *                                         panels of 128 rows x 128 bytes;
+ *                   bytes [0, 32768)      cbar_{c_e} as bf16, in groups of 8
+ *                                         rows: group a at 2048 a holds the
+ *                                         columns 0-63 of its 8 rows (128 bytes
+ *                                         each), then the columns 64-127;
  *                   bytes [32768, 65536)  -S_e / n_e as bf16, same layout;
  *                   bytes [65536, 66048)  log2 n_e as fp32 per row;
  *                 every 128-byte row stored with the 16-byte chunks of row r

@@ -124,12 +124,14 @@ def check_attention(inp, b, h, O, lse, a_gpu, q_blocks=None, scale=None):
 
 
 def _unswizzle_rows(tile: np.ndarray, rows: int) -> np.ndarray:
-    """[2 panels][128 rows][128 B] with chunk k of row r stored at k ^ (r % 8) -> [rows][128] bf16 bits."""
-    t = tile.reshape(2, 128, 8, 16)[:, :rows]
-    r = np.arange(rows)[:, None]
+    """An entry tile's operand (32 KB): 8-row groups of 2048 B holding panel 0 (columns 0-63) then
+    panel 1 of their rows, 128 B per row, chunk k of row r stored at k ^ (r % 8) -> [rows][128]
+    bf16 bits."""
+    t = tile.reshape(16, 2, 8, 8, 16)[: rows // 8]          # [group][panel][row in group][chunk][byte]
+    r = np.arange(8)[:, None]
     k = np.arange(8)[None, :]
-    out = np.stack([t[p][r, k ^ (r % 8)] for p in range(2)])        # [2, rows, 8, 16] logical order
-    return np.ascontiguousarray(out.transpose(1, 0, 2, 3)).reshape(rows, 256).view(np.uint16)
+    out = t[:, :, r, k ^ r]                                   # [group][panel][row][chunk][byte], logical chunks
+    return np.ascontiguousarray(out.transpose(0, 2, 1, 3, 4)).reshape(rows, 256).view(np.uint16)
 
 
 def _bf16_bits_to_f64(b: np.ndarray) -> np.ndarray:
