@@ -26,9 +26,10 @@ DA_BF16, DA_F32 = 0, 1
 STATUS_NAMES = ["DA_OK", "DA_ERR_INVALID_ARG", "DA_ERR_SHAPE", "DA_ERR_DTYPE", "DA_ERR_ALIGNMENT",
                 "DA_ERR_UNSUPPORTED", "DA_ERR_CUDA", "DA_ERR_TIMEOUT", "DA_ERR_DEVICE_INDEX",
                 "DA_ERR_WORKSPACE"]
-EXPORTS = ["da_version", "da_workspace_bytes", "da_schedule_bytes", "da_comp_tiles_bytes", "da_reassign",
-           "da_mask_prepare", "da_attention", "da_device_status", "da_status_string", "da_reassign_noalloc",
-           "da_centroid_update", "da_cluster_spread", "da_attention_spread", "da_attention_sip"]
+EXPORTS = ["da_version", "da_workspace_bytes", "da_schedule_bytes", "da_reassign", "da_mask_prepare",
+           "da_attention", "da_device_status", "da_status_string", "da_reassign_noalloc", "da_compensation",
+           "da_attention_prebuilt", "da_centroid_update", "da_cluster_spread", "da_attention_spread",
+           "da_attention_sip"]
 
 
 class DAError(RuntimeError):
@@ -45,8 +46,7 @@ class _Dims(ctypes.Structure):
 
 class _Stats(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
-                ("assign", "blk_hist", "seg_idx", "seg_n", "seg_c", "seg_cnt", "seg_vsum", "n_tot", "S_tot",
-                 "comp_tiles")]
+                ("assign", "blk_hist", "seg_idx", "seg_n", "seg_c", "seg_cnt", "seg_vsum", "n_tot", "S_tot")]
 
 
 class _Mask(ctypes.Structure):
@@ -60,8 +60,6 @@ _lib.da_workspace_bytes.restype = ctypes.c_size_t
 _lib.da_workspace_bytes.argtypes = [ctypes.POINTER(_Dims)]
 _lib.da_schedule_bytes.restype = ctypes.c_size_t
 _lib.da_schedule_bytes.argtypes = [ctypes.POINTER(_Dims)]
-_lib.da_comp_tiles_bytes.restype = ctypes.c_size_t
-_lib.da_comp_tiles_bytes.argtypes = [ctypes.POINTER(_Dims)]
 _lib.da_reassign.restype = ctypes.c_int
 _lib.da_reassign.argtypes = [ctypes.POINTER(_Dims), _P, _P, _P, ctypes.POINTER(_Stats), _P, ctypes.c_size_t, _P]
 _lib.da_mask_prepare.restype = ctypes.c_int
@@ -70,6 +68,11 @@ _lib.da_mask_prepare.argtypes = [ctypes.POINTER(_Dims), ctypes.POINTER(_Mask), _
 _lib.da_attention.restype = ctypes.c_int
 _lib.da_attention.argtypes = [ctypes.POINTER(_Dims), _P, _P, _P, ctypes.POINTER(_Mask), _P,
                               ctypes.POINTER(_Stats), ctypes.c_float, _P, _P, _P, ctypes.c_size_t, _P]
+_lib.da_attention_prebuilt.restype = ctypes.c_int
+_lib.da_attention_prebuilt.argtypes = _lib.da_attention.argtypes
+_lib.da_compensation.restype = ctypes.c_int
+_lib.da_compensation.argtypes = [ctypes.POINTER(_Dims), ctypes.POINTER(_Mask), ctypes.POINTER(_Stats), _P,
+                                 ctypes.c_size_t, _P]
 _lib.da_centroid_update.restype = ctypes.c_int
 _lib.da_centroid_update.argtypes = [ctypes.POINTER(_Dims), ctypes.POINTER(_Stats), _P, _P]
 _lib.da_cluster_spread.restype = ctypes.c_int
@@ -109,9 +112,7 @@ class Dims:
 
 @dataclass
 class ClusterStats:
-    """Caller-owned Reassign Cache output (layouts in include/da.h).  comp_tiles holds the same
-    statistics as the fused attention kernel's operand tiles (an empty tensor when the dims do not
-    take the tensor-core path)."""
+    """Caller-owned Reassign Cache output (layouts in include/da.h)."""
     assign: torch.Tensor
     blk_hist: torch.Tensor
     seg_idx: torch.Tensor
@@ -121,7 +122,6 @@ class ClusterStats:
     seg_vsum: torch.Tensor
     n_tot: torch.Tensor
     S_tot: torch.Tensor
-    comp_tiles: torch.Tensor
 
     @staticmethod
     def empty(dims: Dims, device="cuda") -> "ClusterStats":
@@ -137,12 +137,10 @@ class ClusterStats:
             seg_vsum=torch.empty(B, H, nB, bs, d, dtype=torch.float32, device=device),
             n_tot=torch.empty(B, H, C, **i32),
             S_tot=torch.empty(B, H, C, d, dtype=torch.float32, device=device),
-            comp_tiles=torch.empty(da_comp_tiles_bytes(dims), dtype=torch.uint8, device=device),
         )
 
     def c(self) -> _Stats:
-        ptr = lambda t: t.data_ptr() if t.numel() > 0 else None
-        return _Stats(*[ptr(getattr(self, n)) for n, _ in _Stats._fields_])
+        return _Stats(*[getattr(self, n).data_ptr() for n, _ in _Stats._fields_])
 
 
 @dataclass
@@ -183,10 +181,6 @@ def da_schedule_bytes(dims: Dims) -> int:
     return _lib.da_schedule_bytes(ctypes.byref(dims.c()))
 
 
-def da_comp_tiles_bytes(dims: Dims) -> int:
-    return _lib.da_comp_tiles_bytes(ctypes.byref(dims.c()))
-
-
 def workspace(dims: Dims, device="cuda") -> torch.Tensor:
     """A zero-filled workspace of da_workspace_bytes(dims) bytes."""
     n = da_workspace_bytes(dims)
@@ -225,6 +219,23 @@ def da_attention(dims: Dims, Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, 
                              ctypes.byref(mask.c()), centroids.data_ptr(), ctypes.byref(stats.c()),
                              float(scale), O.data_ptr(), lse.data_ptr() if lse is not None else None,
                              ws.data_ptr(), ws.numel(), _stream(stream)), "da_attention")
+    return O
+
+
+def da_compensation(dims: Dims, mask: BlockMask, stats: ClusterStats, ws: torch.Tensor, stream=None) -> None:
+    """First half of da_attention: the compensation values of every q-block, into ws."""
+    _check(_lib.da_compensation(ctypes.byref(dims.c()), ctypes.byref(mask.c()), ctypes.byref(stats.c()),
+                                ws.data_ptr(), ws.numel(), _stream(stream)), "da_compensation")
+
+
+def da_attention_prebuilt(dims: Dims, Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, mask: BlockMask,
+                          centroids: torch.Tensor, stats: ClusterStats, scale: float, O: torch.Tensor,
+                          lse: Optional[torch.Tensor], ws: torch.Tensor, stream=None) -> torch.Tensor:
+    """Second half of da_attention: the fused kernel on the values da_compensation left in ws."""
+    _check(_lib.da_attention_prebuilt(ctypes.byref(dims.c()), Q.data_ptr(), K.data_ptr(), V.data_ptr(),
+                                      ctypes.byref(mask.c()), centroids.data_ptr(), ctypes.byref(stats.c()),
+                                      float(scale), O.data_ptr(), lse.data_ptr() if lse is not None else None,
+                                      ws.data_ptr(), ws.numel(), _stream(stream)), "da_attention_prebuilt")
     return O
 
 

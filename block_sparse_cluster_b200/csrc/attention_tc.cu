@@ -8,22 +8,13 @@
 // where n^U_c = n_c - sum_{j in sel} n_{c,j} and vbar^U_c = (S_c - sum_{j in sel} S_{c,j}) / n^U_c
 // are the count and mean value of the cluster's keys outside the selected blocks.
 //
-// The cluster columns are taken in the per-key correction form, which needs no per-q-block table:
-//   e^{s q.cbar_c} n^U_c vbar^U_c = e^{s q.cbar_c + ln n_c} (S_c / n_c)
-//                                   - sum_{j in sel} e^{s q.cbar_c + ln n_{c,j}} (S_{c,j} / n_{c,j}),
-// and the same with the counts alone for the denominator.  So an item's steps are
-//   - one per selected block (exact keys);
-//   - one per 128-cluster chunk of the head (centroid rows, bias log2 n_c, head-wide means);
-//   - its entry tiles: the entries of its selected blocks, 128 rows at a time (centroid rows,
-//     bias log2 n_e, negated entry means), whose weights leave the running sum.
-// The Reassign Cache writes the chunk and entry operands (compensation tiles, include/da.h);
-// an entry tile is copied run by run (a selected block's entries) with bulk copies, as it is
-// stored swizzled, in 8-row groups of both 64-column panels, so that a run is one contiguous copy;
-// its MMA descriptors stride by those groups.
-//
 // Work: items (head, q-block) from the plan's work order; a persistent CTA per SM walks
-// items blockIdx.x, blockIdx.x + gridDim.x, ...  Every step is a 128 x 128 score tile S = Q K^T
-// (K a key block, a centroid chunk or an entry tile) and a P V product.
+// items blockIdx.x, blockIdx.x + gridDim.x, ...  An item is a sequence of steps: one per selected
+// block, then one per 128-cluster chunk.  Every step is a 128 x 128 score tile S = Q K^T (K a
+// key block or a centroid chunk) and a P V product (V a value block or the chunk's vbar^U rows).
+//
+// The compensation chunks (vbar^U rows in bf16 and log2 n^U per cluster) of every item are
+// written beforehand by comp_build.cu; here they are loaded like value blocks.
 //
 // Inclusion-probability mode (AB-Attention abstract: sampled blocks "reweighted by inverse
 // inclusion probability"): with p.incl, an item's steps are its selected blocks only (one fully
@@ -38,11 +29,11 @@
 //              P written back to TMEM as bf16.  At the end of the item the two exchange their
 //              (max, sum) per row and each normalises and stores half of the columns of
 //              O = O_0 2^(m_0 - m) + O_1 2^(m_1 - m);
-//   warp 8     producer: loads Q, key tiles / centroid chunks / entry centroid rows (2-stage ring)
-//              and the softmax bias rows (4-stage ring, so a slot always serves the same warpgroup);
+//   warp 8     producer: loads Q, key tiles / centroid chunks (3-stage ring) and the softmax bias
+//              rows (4-stage ring, so a slot always serves the same warpgroup);
 //   warp 9     MMA: allocates TMEM, issues tcgen05.mma S(g+1) = Q K^T ahead of O_X += P(g) V(g);
-//   warp 10    producer of value tiles / cluster means / entry means (3-stage ring); a warp of its
-//              own, since divergent lanes of one warp waiting on different barriers hold each other up;
+//   warp 10    producer of value tiles / compensation chunks (2-stage ring); a warp of its own,
+//              since divergent lanes of one warp waiting on different barriers hold each other up;
 //   warp 11    idle (it completes the third warpgroup, whose registers go to the softmax).
 // TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,384), O_1 [384,512).
 //
@@ -61,12 +52,11 @@ constexpr int kD = 128;
 constexpr int kBM = 128;                 // query rows per item
 constexpr int kBN = 128;                 // keys per block / clusters per chunk
 constexpr int kKStages = 2;             // key / centroid tiles (freed as soon as S is computed)
-constexpr int kVStages = 3;             // value / mean tiles (freed after P V)
+constexpr int kVStages = 3;             // value / vbar^U tiles (freed after P V)
 constexpr int kBStages = 4;             // bias rows of the softmax (even: a slot serves one warpgroup)
 constexpr int kTile = kBN * kD * 2;      // 32 KB bf16 tile
 constexpr int kPanel = kBN * 128;        // one 64-column panel (128 rows x 128 B)
 constexpr float kRescaleLog2 = 8.0f;     // lazy rescale threshold (factor 256)
-constexpr int kEntSlots = 512;           // selected slots whose entry counts are prefetched
 constexpr int kThreads = 384;           // three warpgroups; warp 11 idle
 constexpr int kWarpProducer = 8;
 constexpr int kWarpMMA = 9;
@@ -76,7 +66,7 @@ constexpr int kWarpProducerV = 10;
 constexpr int kRegSoftmax = 232, kRegIssue = 40;
 static_assert(128 * (2 * kRegSoftmax + kRegIssue) <= kThreads * 168, "register split above the launch");
 static_assert(kBStages % 2 == 0, "a bias slot must always serve the same softmax warpgroup");
-static_assert(kEntRows == kBN && kEntVOff == (size_t)kTile, "an entry tile's operands have the size of a key tile");
+constexpr int kChunkBytes = kTile + kBN * 4;   // compensation chunk: vbar^U rows, then log2 n^U
 
 struct __align__(8) Bars {
   uint64_t q_full, q_empty;
@@ -90,13 +80,8 @@ struct __align__(8) Bars {
   uint64_t xch_full[2][2];
   uint32_t tmem_base;
   int abort;
-  int bflag[kBStages];                   // bit 0: the bias row is all zero (a full key block);
-                                         // bit 1: an entry tile (its weights leave the sum)
+  int bflag[kBStages];                   // 1: the slot's bias row is all zero (a full key block)
   float2 xch[2][2][kBM];                 // [item parity][warpgroup][row] = (max, sum)
-  // entries of the current item's selected blocks, by slot, copied with cp.async by each producer
-  // during its exact steps (one array per producer: the two run independently)
-  int e8[2][kEntSlots];
-  int jsel[2][kEntSlots];                // and the slot's block (-1: not a valid block)
 };
 
 constexpr size_t kSmemBytes = 1024 + kTile /*Q*/ + (kKStages + kVStages) * kTile /*K,V*/ +
@@ -108,25 +93,15 @@ struct Params {
   const int32_t* kv_cnt;
   const int32_t* schedule;
   int max_sel;
-  const int32_t* seg_n;                  // entries per key block (from the Reassign Cache)
-  const int32_t* ent_rows;               // [items] entry rows an item streams (entry_rows_kernel)
-  const uint8_t* ent;                    // entry tiles, kEntTileBytes per (head, key block)
-  const float* cbias;                    // [BH][cpad] log2 n_c
+  StatsPtrs st;
   __nv_bfloat16* O;
   float* lse;
   int* status;
+  const uint8_t* comp;                   // [items][nchunk] compensation chunks of kChunkBytes
   const float* incl;                     // [items][max_sel] inclusion probabilities, or NULL
-  int N, C, nB, n_items, nchunk, cpad;
+  int N, C, nB, n_items, nchunk;
   float scale_log2;
 };
-
-// A wait taken by lane 0 for the whole warp (one poller instead of 32); the shuffle's warp
-// barrier orders the other lanes' later accesses after lane 0's acquire.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int* status, int lane) {
-  bool ok = true;
-  if (lane == 0) ok = mbar_wait(bar, parity, abort, status);
-  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-}
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -134,15 +109,9 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// Rows of key block j's entry tile that an item streams: its entries, padded to a multiple of 8.
-__device__ __forceinline__ int ent_rows_of(const int32_t* seg_n, int nB, int bh, int j) {
-  const int e = __ldg(seg_n + (size_t)bh * nB + j);
-  return (min(max(e, 0), kBN) + 7) & ~7;
-}
-
 // Item geometry shared by every role.
 struct Item {
-  int bh, i, q0, qlen, nsel, erows, T;
+  int bh, i, q0, qlen, nsel, T;
   const int32_t* row;
 };
 
@@ -157,8 +126,7 @@ __device__ __forceinline__ Item item_at(const Params& p, int k) {
   int cnt = p.kv_cnt[item];
   if (cnt < 0 || cnt > p.max_sel) cnt = 0;
   it.nsel = cnt;
-  it.erows = p.incl ? 0 : max(0, p.ent_rows[item]);
-  it.T = p.incl ? max(cnt, 1) : cnt + p.nchunk + (it.erows + kBN - 1) / kBN;
+  it.T = p.incl ? max(cnt, 1) : cnt + p.nchunk;
   it.row = p.kv_idx + (size_t)item * p.max_sel;
   return it;
 }
@@ -170,61 +138,8 @@ __device__ __forceinline__ int block_of(const Params& p, const Item& it, int s, 
   return *valid ? j : 0;
 }
 
-// Entry rows of selected slot s: its block's entry count was copied into e8s[s] by cp.async during
-// the slot's exact step (slots beyond kEntSlots, or invalid blocks, are looked up here).
-__device__ __forceinline__ int ent_rows_at(const Params& p, const Item& it, const int* e8s, const int* js, int s,
-                                           int* j_out) {
-  if (s < kEntSlots) {
-    const int j = js[s];
-    *j_out = j;
-    return j < 0 ? 0 : (min(max(e8s[s], 0), kBN) + 7) & ~7;
-  }
-  bool valid;
-  const int j = block_of(p, it, s, &valid);
-  *j_out = j;
-  return valid ? ent_rows_of(p.seg_n, p.nB, it.bh, j) : 0;
-}
-
-// At exact step s: note the slot's block in js[s] and start the asynchronous copy of its entry
-// count into e8s[s], so that the entry tiles' walk reads both from shared memory.
-__device__ __forceinline__ void ent_prefetch(const Params& p, const Item& it, int* e8s, int* js, int s, int j,
-                                             bool valid) {
-  if (s >= kEntSlots || p.incl) return;
-  js[s] = valid ? j : -1;
-  if (!valid) return;
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(e8s + s)),
-               "l"(reinterpret_cast<uint64_t>(p.seg_n + (size_t)it.bh * p.nB + j))
-               : "memory");
-}
-
-// One entry tile of `rows` rows: the item's selected blocks from the cursor (slot cs, source row
-// cr of that block's entry tile) give runs of rows (dst_row, block, src_row, nrows) until the tile
-// holds `rows` rows or the list ends.  Every lane walks the same runs (from shared memory) and
-// returns run number `lane` (nr = 0: none), and the cursor after the tile.  Runs are multiples of
-// 8 rows, so each lands on the swizzle period it was stored for; a tile has at most 16 of them.
-struct EntRun {
-  int r0, j, sr, nr;
-};
-__device__ __forceinline__ EntRun ent_tile_runs(const Params& p, const Item& it, const int* e8s, const int* js,
-                                                int rows, int& cs, int& cr, int lane) {
-  EntRun mine{0, 0, 0, 0};
-  int r0 = 0, idx = 0;
-  while (r0 < rows && cs < it.nsel) {
-    int j;
-    const int e8 = ent_rows_at(p, it, e8s, js, cs, &j);
-    const int take = min(e8 - cr, rows - r0);
-    if (take > 0) {
-      if (idx == lane) mine = EntRun{r0, j, cr, take};
-      ++idx;
-      r0 += take;
-      cr += take;
-    }
-    if (cr >= e8) {
-      ++cs;
-      cr = 0;
-    }
-  }
-  return mine;
+__device__ __forceinline__ const uint8_t* comp_chunk(const Params& p, const Item& it, int c) {
+  return p.comp + ((size_t)(it.bh * p.nB + it.i) * p.nchunk + c) * kChunkBytes;
 }
 
 // Orders later uses of r after a tcgen05.wait::ld already issued (emits no instruction).
@@ -295,7 +210,7 @@ __device__ __forceinline__ void chunk_exp(const uint32_t (&x)[32], uint64_t coef
 __global__ void __launch_bounds__(kThreads, 1)
 attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_c,
-                    const __grid_constant__ CUtensorMap tm_m, const Params p) {
+                    const __grid_constant__ CUtensorMap tm_p, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -335,11 +250,6 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     bars->abort = 0;
     fence_mbar_init();
   }
-  // Zero the key and value rings once: the rows past the end of an item's last entry tile keep
-  // whatever an earlier step left there (their bias is -inf, so P is 0 there), which must be finite.
-  for (int i = tid; i < (kKStages + kVStages) * kTile / 16; i += kThreads)
-    reinterpret_cast<uint4*>(sK)[i] = make_uint4(0u, 0u, 0u, 0u);
-  fence_async_smem();
   if (warp == kWarpMMA) {
     tmem_alloc(&bars->tmem_base, 512);
     tmem_relinquish();
@@ -356,113 +266,65 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 
   if (warp == kWarpProducer) {
     // ------------------------------------------------------------------ producer (keys)
-    // query tiles, key / centroid / entry tiles and the softmax bias rows.  The whole warp runs the
-    // loop (its waits made warp-uniform): lane 0 issues the tensor copies and the barrier
-    // operations, the lanes share the bias rows, and lane i issues run i of an entry tile, so that a
-    // tile's runs go out in one instruction.
+    // query tiles, key / centroid tiles and the softmax bias rows
     if (lane == 0) {
       tma_prefetch(&tm_q);
       tma_prefetch(&tm_k);
       tma_prefetch(&tm_c);
-    }
-    uint32_t g = 0;
-    int n = 0, nq = 0;                   // items walked, query tiles loaded
-    for (int k = blockIdx.x; k < p.n_items && !__any_sync(0xffffffffu, *abort); k += gridDim.x, ++n) {
-      const Item it = item_at(p, k);
-      int cs = 0, cr = 0;                // entry cursor: selected slot, source row
-      if (!warp_wait(&bars->q_empty, (n & 1) ^ 1, abort, status, lane)) break;
-      ++nq;
-      if (lane == 0) {
+      uint32_t g = 0;
+      int n = 0, nq = 0;                 // items walked, query tiles loaded
+      for (int k = blockIdx.x; k < p.n_items && !*abort; k += gridDim.x, ++n) {
+        const Item it = item_at(p, k);
+        if (!mbar_wait(&bars->q_empty, (n & 1) ^ 1, abort, status)) break;
+        ++nq;
         mbar_expect_tx(&bars->q_full, kTile);
         tma_load_3d(sQ, &tm_q, &bars->q_full, 0, it.q0, it.bh);
         tma_load_3d(sQ + kPanel, &tm_q, &bars->q_full, 64, it.q0, it.bh);
-      }
-      bool ok = true;
-      for (int s = 0; s < it.T; ++s, ++g) {
-        const int ks = g % kKStages, bs = g % kBStages;
-        if (!warp_wait(&bars->k_empty[ks], ((g / kKStages) & 1) ^ 1, abort, status, lane)) {
-          ok = false;
-          break;
-        }
-        uint8_t* dk = sK + ks * kTile;
-        float* bb = sBias + bs * kBN;
-        if (s < it.nsel || p.incl) {
-          bool valid;
-          const int j = block_of(p, it, s, &valid);
-          if (lane == 0) {
+        bool ok = true;
+        for (int s = 0; s < it.T; ++s, ++g) {
+          const int ks = g % kKStages, bs = g % kBStages;
+          if (!mbar_wait(&bars->k_empty[ks], ((g / kKStages) & 1) ^ 1, abort, status)) { ok = false; break; }
+          uint8_t* dk = sK + ks * kTile;
+          if (s < it.nsel || p.incl) {
+            bool valid;
+            const int j = block_of(p, it, s, &valid);
             mbar_expect_tx(&bars->k_full[ks], kTile);
             tma_load_3d(dk, &tm_k, &bars->k_full[ks], 0, j * kBN, it.bh);
             tma_load_3d(dk + kPanel, &tm_k, &bars->k_full[ks], 64, j * kBN, it.bh);
-            ent_prefetch(p, it, bars->e8[0], bars->jsel[0], s, j, valid);
-          }
-          // bias row of a key block: 0 for its keys, -inf past the end of a short last block
-          // (generic stores, published to the softmax by lane 0's arrive on b_full)
-          if (!warp_wait(&bars->b_empty[bs], ((g / kBStages) & 1) ^ 1, abort, status, lane)) {
-            ok = false;
-            break;
-          }
-          int ncol = valid ? min(kBN, p.N - j * kBN) : 0;
-          float w = 0.f;                 // log2 weight of the block's columns
-          if (p.incl && ncol > 0) {
-            const float pi = p.incl[(size_t)(it.bh * p.nB + it.i) * p.max_sel + s];
-            if (pi > 0.f) w = -__log2f(pi);
-            else ncol = 0;               // a block that is never included: left out
-          }
-          if (lane == 0) bars->bflag[bs] = (ncol == kBN && !p.incl) ? 1 : 0;
-          const int c = 4 * lane;
-          reinterpret_cast<float4*>(bb)[lane] =
-              make_float4(c < ncol ? w : -INFINITY, c + 1 < ncol ? w : -INFINITY, c + 2 < ncol ? w : -INFINITY,
-                          c + 3 < ncol ? w : -INFINITY);
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&bars->b_full[bs]);
-        } else if (s < it.nsel + p.nchunk) {
-          // cluster chunk: centroid rows, bias log2 n_c
-          const int c = s - it.nsel;
-          if (lane == 0) {
+            // bias row of a key block: 0 for its keys, -inf past the end of a short last block
+            // (generic stores, published to the softmax by the arrive on b_full)
+            if (!mbar_wait(&bars->b_empty[bs], ((g / kBStages) & 1) ^ 1, abort, status)) { ok = false; break; }
+            int ncol = valid ? min(kBN, p.N - j * kBN) : 0;
+            float w = 0.f;                 // log2 weight of the block's columns
+            if (p.incl && ncol > 0) {
+              const float pi = p.incl[(size_t)(it.bh * p.nB + it.i) * p.max_sel + s];
+              if (pi > 0.f) w = -__log2f(pi);
+              else ncol = 0;               // a block that is never included: left out
+            }
+            bars->bflag[bs] = (ncol == kBN && !p.incl) ? 1 : 0;
+            float4* bb = reinterpret_cast<float4*>(sBias + bs * kBN);
+#pragma unroll 4
+            for (int c4 = 0; c4 < kBN / 4; ++c4) {
+              const int c = 4 * c4;
+              bb[c4] = make_float4(c < ncol ? w : -INFINITY, c + 1 < ncol ? w : -INFINITY,
+                                   c + 2 < ncol ? w : -INFINITY, c + 3 < ncol ? w : -INFINITY);
+            }
+            mbar_arrive(&bars->b_full[bs]);
+          } else {
+            const int c = s - it.nsel;
             mbar_expect_tx(&bars->k_full[ks], kTile);
             tma_load_3d(dk, &tm_c, &bars->k_full[ks], 0, c * kBN, it.bh);
             tma_load_3d(dk + kPanel, &tm_c, &bars->k_full[ks], 64, c * kBN, it.bh);
-          }
-          if (!warp_wait(&bars->b_empty[bs], ((g / kBStages) & 1) ^ 1, abort, status, lane)) {
-            ok = false;
-            break;
-          }
-          if (lane == 0) {
+            if (!mbar_wait(&bars->b_empty[bs], ((g / kBStages) & 1) ^ 1, abort, status)) { ok = false; break; }
             bars->bflag[bs] = 0;
             mbar_expect_tx(&bars->b_full[bs], kBN * 4);
-            bulk_load(bb, p.cbias + (size_t)it.bh * p.cpad + c * kBN, kBN * 4, &bars->b_full[bs]);
-          }
-        } else {
-          // entry tile: centroid rows and bias log2 n_e of the selected blocks' entries; the rows
-          // past the item's last entry are masked (-inf, generic stores published by the arrive)
-          const int t = s - it.nsel - p.nchunk;
-          const int rows = min(kBN, it.erows - t * kBN);
-          if (!warp_wait(&bars->b_empty[bs], ((g / kBStages) & 1) ^ 1, abort, status, lane)) {
-            ok = false;
-            break;
-          }
-          for (int c = rows + lane; c < kBN; c += 32) bb[c] = -INFINITY;
-          if (lane == 0 && t == 0) asm volatile("cp.async.wait_all;" ::: "memory");   // counts prefetched at the exact steps
-          __syncwarp();
-          if (lane == 0) {
-            bars->bflag[bs] = 2;
-            mbar_expect_tx(&bars->k_full[ks], rows * 256);
-            mbar_expect_tx(&bars->b_full[bs], rows * 4);
-          }
-          __syncwarp();
-          EntRun run = ent_tile_runs(p, it, bars->e8[0], bars->jsel[0], rows, cs, cr, lane);
-          if (run.nr > 0) {
-            const uint8_t* src = p.ent + ((size_t)it.bh * p.nB + run.j) * kEntTileBytes;
-            bulk_load(dk + run.r0 * 256, src + run.sr * 256, run.nr * 256, &bars->k_full[ks]);   // whole 8-row groups
-            bulk_load(bb + run.r0, src + kEntBiasOff + run.sr * 4, run.nr * 4, &bars->b_full[bs]);
+            bulk_load(sBias + bs * kBN, comp_chunk(p, it, c) + kTile, kBN * 4, &bars->b_full[bs]);
           }
         }
+        if (!ok) break;
       }
-      if (!ok) break;
-    }
-    // no copy may still be in flight when the CTA leaves (this matters only after an abort:
-    // otherwise the consumers have waited for every load)
-    if (lane == 0) {
+      // no copy may still be in flight when the CTA leaves (this matters only after an abort:
+      // otherwise the consumers have waited for every load)
       if (nq > 0) mbar_wait_drain(&bars->q_full, (nq - 1) & 1);
       for (uint32_t gd = g >= kKStages ? g - kKStages : 0; gd < g; ++gd)
         mbar_wait_drain(&bars->k_full[gd % kKStages], (gd / kKStages) & 1);
@@ -471,61 +333,36 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     }
   } else if (warp == kWarpProducerV) {
     // ------------------------------------------------------------------ producer (values)
-    // (the whole warp runs the loop, as the producer of keys)
     if (lane == 0) {
       tma_prefetch(&tm_v);
-      tma_prefetch(&tm_m);
-    }
-    uint32_t g = 0;
-    for (int k = blockIdx.x; k < p.n_items && !__any_sync(0xffffffffu, *abort); k += gridDim.x) {
-      const Item it = item_at(p, k);
-      int cs = 0, cr = 0;                // entry cursor: selected slot, source row
-      bool ok = true;
-      for (int s = 0; s < it.T; ++s, ++g) {
-        const int vs = g % kVStages;
-        if (!warp_wait(&bars->v_empty[vs], ((g / kVStages) & 1) ^ 1, abort, status, lane)) {
-          ok = false;
-          break;
-        }
-        uint8_t* dv = sV + vs * kTile;
-        if (s < it.nsel || p.incl) {
-          if (lane == 0) {
+      tma_prefetch(&tm_p);
+      uint32_t g = 0;
+      int n = 0;
+      for (int k = blockIdx.x; k < p.n_items && !*abort; k += gridDim.x, ++n) {
+        const Item it = item_at(p, k);
+        bool ok = true;
+        for (int s = 0; s < it.T; ++s, ++g) {
+          const int vs = g % kVStages;
+          if (!mbar_wait(&bars->v_empty[vs], ((g / kVStages) & 1) ^ 1, abort, status)) { ok = false; break; }
+          uint8_t* dv = sV + vs * kTile;
+          if (s < it.nsel || p.incl) {
             bool valid;
             const int j = block_of(p, it, s, &valid);
             mbar_expect_tx(&bars->v_full[vs], kTile);
             tma_load_3d(dv, &tm_v, &bars->v_full[vs], 0, j * kBN, it.bh);
             tma_load_3d(dv + kPanel, &tm_v, &bars->v_full[vs], 64, j * kBN, it.bh);
-            ent_prefetch(p, it, bars->e8[1], bars->jsel[1], s, j, valid);
-          }
-        } else if (s < it.nsel + p.nchunk) {
-          // cluster chunk: the head-wide means S_c / n_c (rows past C read as zero)
-          const int c = s - it.nsel;
-          if (lane == 0) {
+          } else {
+            const int z = (it.bh * p.nB + it.i) * p.nchunk + (s - it.nsel);
             mbar_expect_tx(&bars->v_full[vs], kTile);
-            tma_load_3d(dv, &tm_m, &bars->v_full[vs], 0, c * kBN, it.bh);
-            tma_load_3d(dv + kPanel, &tm_m, &bars->v_full[vs], 64, c * kBN, it.bh);
-          }
-        } else {
-          // entry tile: the negated entry means, the same runs as the producer of keys
-          const int t = s - it.nsel - p.nchunk;
-          const int rows = min(kBN, it.erows - t * kBN);
-          if (lane == 0) {
-            if (t == 0) asm volatile("cp.async.wait_all;" ::: "memory");   // counts prefetched at the exact steps
-            mbar_expect_tx(&bars->v_full[vs], rows * 256);
-          }
-          __syncwarp();
-          EntRun run = ent_tile_runs(p, it, bars->e8[1], bars->jsel[1], rows, cs, cr, lane);
-          if (run.nr > 0) {
-            const uint8_t* src = p.ent + ((size_t)it.bh * p.nB + run.j) * kEntTileBytes + kEntVOff;
-            bulk_load(dv + run.r0 * 256, src + run.sr * 256, run.nr * 256, &bars->v_full[vs]);   // whole 8-row groups
+            tma_load_3d(dv, &tm_p, &bars->v_full[vs], 0, 0, z);
+            tma_load_3d(dv + kPanel, &tm_p, &bars->v_full[vs], 64, 0, z);
           }
         }
+        if (!ok) break;
       }
-      if (!ok) break;
-    }
-    if (lane == 0)
       for (uint32_t gd = g >= kVStages ? g - kVStages : 0; gd < g; ++gd)
         mbar_wait_drain(&bars->v_full[gd % kVStages], (gd / kVStages) & 1);
+    }
   } else if (warp == kWarpMMA) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -534,19 +371,15 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       const uint32_t q0 = smem_u32(sQ);
       uint32_t g = 0;
       int n = 0;
-      // Descriptors are built once per tile and advanced in their 16-byte address field per
-      // K-slice.  ent: an entry tile, whose rows come in 8-row groups of both panels (2048 B apart,
-      // the second panel 1024 B after the first) instead of two 16 KB panels of 128 rows.
-      const uint64_t qd = sdesc_sw128(q0, 16, 1024);
-      auto issue_s = [&](uint32_t gs, bool ent) {
+      auto issue_s = [&](uint32_t gs) {
         const int ks = gs % kKStages;
-        const uint64_t kd = sdesc_sw128(smem_u32(sK + ks * kTile), 16, ent ? 2048u : 1024u);
-        const uint32_t kpanel = ent ? 1024u / 16 : (uint32_t)kPanel / 16;
+        const uint32_t kb = smem_u32(sK + ks * kTile);
         const uint32_t d = tmem + (gs & 1) * kBN;
 #pragma unroll
-        for (int kk = 0; kk < kD / 16; ++kk)
-          umma_ss(d, qd + ((kk >> 2) * (kPanel / 16) + (kk & 3) * 2), kd + ((kk >> 2) * kpanel + (kk & 3) * 2),
-                  idesc_qk, kk > 0);
+        for (int ks = 0; ks < kD / 16; ++ks) {
+          const uint32_t off = (ks >> 2) * kPanel + (ks & 3) * 32;
+          umma_ss(d, sdesc_sw128(q0 + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), idesc_qk, ks > 0);
+        }
         umma_commit(&bars->s_full[gs & 1]);
         umma_commit(&bars->k_empty[ks]);
       };
@@ -558,14 +391,13 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const uint32_t g0 = g;
         if (!mbar_wait(&bars->k_full[g0 % kKStages], (g0 / kKStages) & 1, abort, status)) break;
         tc_fence_after();
-        const int ent0 = p.incl ? it.T : it.nsel + p.nchunk;   // first entry step of the item
-        issue_s(g0, 0 >= ent0);
+        issue_s(g0);
         for (int s = 0; s < it.T; ++s, ++g) {
           if (s + 1 < it.T) {
             const uint32_t gn = g + 1;
             if (!mbar_wait(&bars->k_full[gn % kKStages], (gn / kKStages) & 1, abort, status)) { ok = false; break; }
             tc_fence_after();
-            issue_s(gn, s + 1 >= ent0);
+            issue_s(gn);
           } else {
             umma_commit(&bars->q_empty);
           }
@@ -577,15 +409,12 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           const uint32_t vb = smem_u32(sV + vs * kTile);
           const uint32_t pt = tmem + (g & 1) * kBN;       // P: bf16 pairs in the S buffer's first 64 columns
           const uint32_t ot = tmem + (2 + (g & 1)) * kBN;  // O_X of the step's warpgroup
-          // V rows (keys) 16 kk .. 16 kk + 15: two 8-row groups, 1024 B apart in a value tile and
-          // 2048 B apart in an entry tile, whose second panel follows the first by 1024 B
-          const bool ent = s >= ent0;
-          const uint64_t vd = ent ? sdesc_sw128(vb, 1024, 2048) : sdesc_sw128(vb, kPanel, 1024);
-          const uint32_t vstep = ent ? 4096u / 16 : 2048u / 16;
 #pragma unroll
-          for (int kk = 0; kk < kBN / 16; ++kk) {
-            // the first product of each accumulator in the item (steps 0 and 1) overwrites it
-            umma_ts(ot, pt + kk * 8, vd + kk * vstep, idesc_pv, (s > 1 || kk > 0) ? 1u : 0u);
+          for (int ks = 0; ks < kBN / 16; ++ks) {
+            // V rows (keys) 16*ks .. 16*ks+15: two 8-row groups of 1024 B; the first product of each
+            // accumulator in the item (steps 0 and 1) overwrites it
+            umma_ts(ot, pt + ks * 8, sdesc_sw128(vb + ks * 2048, kPanel, 1024), idesc_pv,
+                    (s > 1 || ks > 0) ? 1u : 0u);
           }
           umma_commit(&bars->v_empty[vs]);
           umma_commit(&bars->o_done[g & 1]);
@@ -619,12 +448,11 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         tc_fence_after();
         // The S row is loaded from TMEM once (128 registers): the row max, then p = 2^(y - m), the
         // row sum and the bf16 P written back over S.  Column c's logit is y_c = x_c * s*log2(e) +
-        // bias_c, the bias row in shared memory: log2 n_c on a cluster chunk, log2 n_e on an entry
-        // tile, 0 on a key block (-inf past the end of a short last block or of the entries).
+        // bias_c, the bias row in shared memory: log2 n^U_c on a compensation step, 0 on a key
+        // block (-inf past the end of a short last block).
         const uint32_t sbase = lane_addr + X * kBN;
         const float* bt = sBias + bs * kBN;
-        const int flag = bars->bflag[bs];
-        const bool plain = (flag & 1) && p.scale_log2 > 0.f;
+        const bool plain = bars->bflag[bs] != 0 && p.scale_log2 > 0.f;
         uint32_t x[4][32];
         tmem_ld32(sbase, x[0]);
         tmem_ld32(sbase + 32, x[1]);
@@ -677,7 +505,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           }
         }
         m = m_new;
-        l += (flag & 2) ? -rs : rs;               // entry tiles take their weight out again
+        l += rs;
         first = false;
         ++u;
         tmem_wait_st();
@@ -744,68 +572,42 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   }
 }
 
-// Entry rows each item streams (the sum over its valid selected blocks of ent_rows_of), so that
-// every role knows an item's step count without walking its list.  A warp per item.
-__global__ void __launch_bounds__(256) entry_rows_kernel(const int32_t* __restrict__ kv_idx,
-                                                         const int32_t* __restrict__ kv_cnt, int max_sel,
-                                                         const int32_t* __restrict__ seg_n, int nB, int n_items,
-                                                         int32_t* __restrict__ out) {
-  const int item = blockIdx.x * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (item >= n_items) return;
-  int cnt = kv_cnt[item];
-  if (cnt < 0 || cnt > max_sel) cnt = 0;
-  const int bh = item / nB;
-  const int32_t* row = kv_idx + (size_t)item * max_sel;
-  int sum = 0;
-  for (int s = lane; s < cnt; s += 32) {
-    const int j = row[s];
-    if (j >= 0 && j < nB) sum += ent_rows_of(seg_n, nB, bh, j);
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-  if (lane == 0) out[item] = sum;
-}
-
 }  // namespace
 
 bool attention_tc_supported(const Dims& g) { return g.bf16 && g.d == kD && g.block == kBN; }
 
+size_t attention_tc_scratch_bytes(const Dims& g) {
+  if (!attention_tc_supported(g)) return 0;
+  return (size_t)g.B * g.H * g.nB * ((g.C + kBN - 1) / kBN) * kChunkBytes;
+}
+
 cudaError_t launch_attention_tc(const Dims& g, const void* Q, const void* K, const void* V,
                                 const int32_t* kv_idx, const int32_t* kv_cnt, int max_sel,
                                 const int32_t* schedule, const void* cent, const StatsPtrs& st, float scale,
-                                void* O, float* lse, int* status, int32_t* ent_rows, const float* incl,
-                                cudaStream_t s) {
-  CUtensorMap tq, tk, tv, tc, tm;
+                                void* O, float* lse, int* status, void* comp, const float* incl, cudaStream_t s) {
+  CUtensorMap tq, tk, tv, tc, tp;
   const unsigned long long BH = (unsigned long long)g.B * g.H;
-  const CompLayout L = comp_layout(g);
-  // without compensation tiles (the inclusion-probability mode) K stands in for the cluster means
-  const void* cmean = (!incl && st.comp) ? static_cast<const void*>(st.comp + L.cmean) : K;
-  const unsigned long long mean_rows = (!incl && st.comp) ? (unsigned long long)g.C : (unsigned long long)g.N;
-  if (!incl && !st.comp) return cudaErrorInvalidValue;
+  const int nchunk = (g.C + kBN - 1) / kBN;
   if (!make_tmap_bf16_3d(&tq, Q, kD, g.N, BH, 64, kBM) || !make_tmap_bf16_3d(&tk, K, kD, g.N, BH, 64, kBN) ||
       !make_tmap_bf16_3d(&tv, V, kD, g.N, BH, 64, kBN) || !make_tmap_bf16_3d(&tc, cent, kD, g.C, BH, 64, kBN) ||
-      !make_tmap_bf16_3d(&tm, cmean, kD, mean_rows, BH, 64, kBN))
+      !make_tmap_bf16_tiles(&tp, comp, kD, kBN, BH * g.nB * nchunk, kChunkBytes, kBN))
     return cudaErrorInvalidValue;
   Params p;
   p.kv_idx = kv_idx;
   p.kv_cnt = kv_cnt;
   p.schedule = schedule;
   p.max_sel = max_sel;
-  p.seg_n = st.seg_n;
-  p.ent_rows = ent_rows;
-  p.ent = st.comp ? st.comp + L.ent : nullptr;
-  p.cbias = st.comp ? reinterpret_cast<const float*>(st.comp + L.cbias) : nullptr;
+  p.st = st;
   p.O = (__nv_bfloat16*)O;
   p.lse = lse;
   p.status = status;
+  p.comp = static_cast<const uint8_t*>(comp);
   p.incl = incl;
   p.N = g.N;
   p.C = g.C;
   p.nB = g.nB;
   p.n_items = (int)(BH * g.nB);
-  p.nchunk = (g.C + kBN - 1) / kBN;
-  p.cpad = L.cpad;
+  p.nchunk = nchunk;
   p.scale_log2 = scale * 1.4426950408889634f;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
@@ -813,14 +615,8 @@ cudaError_t launch_attention_tc(const Dims& g, const void* Q, const void* K, con
   cudaError_t e = cudaFuncSetAttribute(attention_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kSmemBytes);
   if (e != cudaSuccess) return e;
-  if (!incl) {
-    entry_rows_kernel<<<(p.n_items + 7) / 8, 256, 0, s>>>(kv_idx, kv_cnt, max_sel, st.seg_n, g.nB, p.n_items,
-                                                          ent_rows);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-  }
   const int grid = min(sms, p.n_items);
-  attention_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, tc, tm, p);
+  attention_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, tc, tp, p);
   return cudaGetLastError();
 }
 

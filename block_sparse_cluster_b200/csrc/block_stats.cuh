@@ -7,15 +7,11 @@
 //   - entry index row      e(c) or 0xFF        (seg_idx[j][0..C))
 //   - sorted entry list    (c, n_{c,j})        (seg_c, seg_cnt, seg_n)
 //   - value sum per entry  S_{c,j} = sum v_k   (seg_vsum, fp32, keys summed in index order)
-//   - optionally the block's entry tile for the fused attention kernel: per entry e the cached
-//     centroid cbar_{c_e}, the negated mean -S_e / n_e (bf16) and log2 n_e, rows padded with zeros
-//     (bias -inf) to a multiple of 8, in the 128-byte swizzled layout of include/da.h
 // The block's keys are ranked by (cluster, key index), so every entry is a contiguous run and
 // the sums are reduced in a fixed order: no atomics, deterministic bits.
 #pragma once
 
 #include "da_common.cuh"
-#include "da_internal.h"
 
 namespace da {
 
@@ -37,8 +33,7 @@ __device__ __forceinline__ void group_sync(int bar_id) {
 // call this.
 // s_assign: the block's clusters in shared memory (nk <= 128 entries, each in [0, C)).
 // Vblk: value rows of the block (row k at Vblk + k*D).  Output pointers are already offset to
-// this block.  cent (the head's centroids, bf16 [C][128]) and ent_out (this block's entry tile)
-// are used only for bf16 with D = 128; ent_out NULL skips the tile.
+// this block.
 //   1. Keys with equal clusters are grouped per warp (match_any); the warps, in order, add their
 //      groups to the histogram row, so a key's rank among its cluster's keys is its key-index
 //      rank, without atomics.
@@ -49,8 +44,7 @@ __device__ void block_stats_group(int t, int bar_id, const int* s_assign, int nk
                                   int C, int32_t* __restrict__ hist_out, uint8_t* __restrict__ idx_out,
                                   int32_t* __restrict__ segn_out, int32_t* __restrict__ segc_out,
                                   int32_t* __restrict__ segcnt_out, float* __restrict__ vsum_out,
-                                  StatsSmem& sm, const __nv_bfloat16* __restrict__ cent = nullptr,
-                                  uint8_t* __restrict__ ent_out = nullptr) {
+                                  StatsSmem& sm) {
   const int warp = t >> 5, lane = t & 31;
   const unsigned below = (1u << lane) - 1u;
   static_assert(NT == 128 || NT == 256, "a group of 4 or 8 warps");
@@ -142,11 +136,6 @@ __device__ void block_stats_group(int t, int bar_id, const int* s_assign, int nk
   constexpr int NE = D / 32;
   for (int ee = warp; ee < E; ee += NT / 32) {
     const int p0 = sm.start_pos[ee], p1 = sm.start_pos[ee + 1];
-    // the entry's centroid row for its tile, loaded first so that its latency overlaps the sums
-    uint2 crow = make_uint2(0u, 0u);
-    if constexpr (NE == 4 && sizeof(T) == 2) {
-      if (ent_out) crow = *reinterpret_cast<const uint2*>(cent + (size_t)s_assign[sm.sorted_key[p0]] * 128 + lane * 4);
-    }
     float acc[NE];
 #pragma unroll
     for (int i = 0; i < NE; ++i) acc[i] = 0.f;
@@ -173,32 +162,6 @@ __device__ void block_stats_group(int t, int bar_id, const int* s_assign, int nk
     } else {
 #pragma unroll
       for (int i = 0; i < NE; ++i) dst[i] = acc[i];
-    }
-    if constexpr (NE == 4 && sizeof(T) == 2) {
-      if (ent_out) {
-        // lane l holds columns [4l, 4l + 4): panel l / 16, 16-byte chunk (l mod 16) / 2, half l mod 2
-        const int n = p1 - p0;
-        const int k = (lane & 15) >> 1;
-        const size_t off = ent_byte(ee, lane >> 4, k) + ((lane & 1) << 3);
-        *reinterpret_cast<uint2*>(ent_out + off) = crow;
-        const float fn = (float)n;
-        uint2 vv;
-        vv.x = pack_bf16x2(-(acc[0] / fn), -(acc[1] / fn));
-        vv.y = pack_bf16x2(-(acc[2] / fn), -(acc[3] / fn));
-        *reinterpret_cast<uint2*>(ent_out + kEntVOff + off) = vv;
-        if (lane == 0) reinterpret_cast<float*>(ent_out + kEntBiasOff)[ee] = log2f(fn);
-      }
-    }
-  }
-  if constexpr (NE == 4 && sizeof(T) == 2) {
-    if (ent_out) {
-      // rows [E, E8) of the four 128-row panels are zero, their bias -inf
-      const int E8 = (E + 7) & ~7;
-      for (int i = t; i < (E8 - E) * 32; i += NT) {
-        const int r = E + (i >> 5), half = (i >> 4) & 1, panel = (i >> 3) & 1, chunk = i & 7;
-        *reinterpret_cast<uint4*>(ent_out + half * kEntVOff + ent_byte(r, panel, chunk)) = make_uint4(0, 0, 0, 0);
-      }
-      for (int r = E + t; r < E8; r += NT) reinterpret_cast<float*>(ent_out + kEntBiasOff)[r] = -INFINITY;
     }
   }
   group_sync<NT>(bar_id);

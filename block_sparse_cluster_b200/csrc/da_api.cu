@@ -42,7 +42,7 @@ da_status check_dims(const da_dims* dims, Dims* g) {
   return DA_OK;
 }
 
-da_status check_stats(const Dims& g, const da_cluster_stats* st, StatsPtrs* p) {
+da_status check_stats(const da_cluster_stats* st, StatsPtrs* p) {
   if (!st) return DA_ERR_INVALID_ARG;
   if (!st->assign || !st->blk_hist || !st->seg_idx || !st->seg_n || !st->seg_c || !st->seg_cnt ||
       !st->seg_vsum || !st->n_tot || !st->S_tot)
@@ -51,14 +51,8 @@ da_status check_stats(const Dims& g, const da_cluster_stats* st, StatsPtrs* p) {
       !aligned16(st->seg_c) || !aligned16(st->seg_cnt) || !aligned16(st->seg_vsum) || !aligned16(st->n_tot) ||
       !aligned16(st->S_tot))
     return DA_ERR_ALIGNMENT;
-  uint8_t* comp = nullptr;
-  if (comp_tiles_used(g)) {
-    if (!st->comp_tiles) return DA_ERR_INVALID_ARG;
-    if ((reinterpret_cast<uintptr_t>(st->comp_tiles) & 255u) != 0) return DA_ERR_ALIGNMENT;
-    comp = static_cast<uint8_t*>(st->comp_tiles);
-  }
   *p = StatsPtrs{st->assign, st->blk_hist, st->seg_idx, st->seg_n, st->seg_c,
-                 st->seg_cnt, st->seg_vsum, st->n_tot, st->S_tot, comp};
+                 st->seg_cnt, st->seg_vsum, st->n_tot, st->S_tot};
   return DA_OK;
 }
 
@@ -88,13 +82,7 @@ da_status cuda_status(cudaError_t e) { return e == cudaSuccess ? DA_OK : DA_ERR_
 
 extern "C" {
 
-int da_version(void) { return 200; }
-
-size_t da_comp_tiles_bytes(const da_dims* dims) {
-  Dims g;
-  if (check_dims(dims, &g) != DA_OK) return 0;
-  return comp_layout(g).total;
-}
+int da_version(void) { return 103; }
 
 size_t da_workspace_bytes(const da_dims* dims) {
   Dims g;
@@ -116,7 +104,7 @@ da_status da_reassign(const da_dims* dims, const void* K, const void* V, const v
   if (!K || !V || !centroids) return DA_ERR_INVALID_ARG;
   if (!aligned16(K) || !aligned16(V) || !aligned16(centroids)) return DA_ERR_ALIGNMENT;
   StatsPtrs sp;
-  if ((st = check_stats(g, out, &sp)) != DA_OK) return st;
+  if ((st = check_stats(out, &sp)) != DA_OK) return st;
   if ((st = check_ws(g, ws, ws_bytes)) != DA_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const WsLayout L = ws_layout(g);
@@ -151,13 +139,13 @@ da_status da_mask_prepare(const da_dims* dims, const da_block_mask* mask, int32_
                                      reinterpret_cast<cudaStream_t>(stream)));
 }
 
-// Validation shared by da_attention and da_attention_spread.
+// Validation shared by da_compensation, da_attention_prebuilt and da_attention.
 static da_status attention_common(const da_dims* dims, const da_block_mask* mask, const da_cluster_stats* stats,
                                   void* ws, size_t ws_bytes, Dims* g, StatsPtrs* sp) {
   da_status st = check_dims(dims, g);
   if (st != DA_OK) return st;
   if ((st = check_mask(*g, mask)) != DA_OK) return st;
-  if ((st = check_stats(*g, stats, sp)) != DA_OK) return st;
+  if ((st = check_stats(stats, sp)) != DA_OK) return st;
   return check_ws(*g, ws, ws_bytes);
 }
 
@@ -168,6 +156,13 @@ static da_status check_attention_ptrs(const void* Q, const void* K, const void* 
       (lse && !aligned16(lse)))
     return DA_ERR_ALIGNMENT;
   return DA_OK;
+}
+
+static cudaError_t compensation_launch(const Dims& g, const da_block_mask* mask, const StatsPtrs& sp, void* ws,
+                                       cudaStream_t s) {
+  if (!attention_tc_supported(g)) return cudaSuccess;   // the CUDA-core path compensates in-kernel
+  const WsLayout L = ws_layout(g);
+  return launch_comp_build(g, mask->kv_idx, mask->kv_cnt, mask->max_sel, sp, static_cast<char*>(ws) + L.comp, s);
 }
 
 static da_status attention_launch(const Dims& g, const void* Q, const void* K, const void* V,
@@ -188,14 +183,32 @@ static da_status attention_launch(const Dims& g, const void* Q, const void* K, c
   if (e == cudaSuccess) {
     if (attention_tc_supported(g))
       e = launch_attention_tc(g, Q, K, V, mask->kv_idx, mask->kv_cnt, mask->max_sel, sched, centroids, sp, scale, O,
-                              lse, status, reinterpret_cast<int32_t*>(static_cast<char*>(ws) + L.ent_rows), nullptr,
-                              s);
+                              lse, status, static_cast<char*>(ws) + L.comp, nullptr, s);
     else
       e = (g.bf16 ? launch_attention_simt_bf16 : launch_attention_simt_f32)(
           g, Q, K, V, mask->kv_idx, mask->kv_cnt, mask->max_sel, sched, centroids, sp, nullptr, scale, O, lse, status,
           s);
   }
   return cuda_status(e);
+}
+
+da_status da_compensation(const da_dims* dims, const da_block_mask* mask, const da_cluster_stats* stats, void* ws,
+                          size_t ws_bytes, da_stream stream) {
+  Dims g;
+  StatsPtrs sp;
+  da_status st = attention_common(dims, mask, stats, ws, ws_bytes, &g, &sp);
+  if (st != DA_OK) return st;
+  return cuda_status(compensation_launch(g, mask, sp, ws, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+da_status da_attention_prebuilt(const da_dims* dims, const void* Q, const void* K, const void* V,
+                                const da_block_mask* mask, const void* centroids, const da_cluster_stats* stats,
+                                float scale, void* O, float* lse, void* ws, size_t ws_bytes, da_stream stream) {
+  Dims g;
+  StatsPtrs sp;
+  da_status st = attention_common(dims, mask, stats, ws, ws_bytes, &g, &sp);
+  if (st != DA_OK) return st;
+  return attention_launch(g, Q, K, V, mask, centroids, sp, scale, O, lse, ws, reinterpret_cast<cudaStream_t>(stream));
 }
 
 da_status da_attention(const da_dims* dims, const void* Q, const void* K, const void* V,
@@ -205,7 +218,11 @@ da_status da_attention(const da_dims* dims, const void* Q, const void* K, const 
   StatsPtrs sp;
   da_status st = attention_common(dims, mask, stats, ws, ws_bytes, &g, &sp);
   if (st != DA_OK) return st;
-  return attention_launch(g, Q, K, V, mask, centroids, sp, scale, O, lse, ws, reinterpret_cast<cudaStream_t>(stream));
+  if ((st = check_attention_ptrs(Q, K, V, centroids, O, lse)) != DA_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const cudaError_t e = compensation_launch(g, mask, sp, ws, s);
+  if (e != cudaSuccess) return cuda_status(e);
+  return attention_launch(g, Q, K, V, mask, centroids, sp, scale, O, lse, ws, s);
 }
 
 da_status da_centroid_update(const da_dims* dims, const da_cluster_stats* stats, void* centroids,
@@ -216,7 +233,7 @@ da_status da_centroid_update(const da_dims* dims, const da_cluster_stats* stats,
   if (!centroids) return DA_ERR_INVALID_ARG;
   if (!aligned16(centroids)) return DA_ERR_ALIGNMENT;
   StatsPtrs sp;
-  if ((st = check_stats(g, stats, &sp)) != DA_OK) return st;
+  if ((st = check_stats(stats, &sp)) != DA_OK) return st;
   return cuda_status(launch_centroid_update(g, sp, centroids, reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -228,7 +245,7 @@ da_status da_cluster_spread(const da_dims* dims, const void* K, const void* cent
   if (!K || !centroids || !spread) return DA_ERR_INVALID_ARG;
   if (!aligned16(K) || !aligned16(centroids) || !aligned16(spread)) return DA_ERR_ALIGNMENT;
   StatsPtrs sp;
-  if ((st = check_stats(g, stats, &sp)) != DA_OK) return st;
+  if ((st = check_stats(stats, &sp)) != DA_OK) return st;
   return cuda_status(launch_cluster_spread(g, K, centroids, sp, spread, reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -287,7 +304,7 @@ da_status da_attention_sip(const da_dims* dims, const void* Q, const void* K, co
   // no cluster steps: the centroid map is never read (K stands in for it), nor are the statistics
   if (e == cudaSuccess)
     e = launch_attention_tc(g, Q, K, V, mask->kv_idx, mask->kv_cnt, mask->max_sel, sched, K, StatsPtrs{}, scale, O,
-                            lse, status, reinterpret_cast<int32_t*>(static_cast<char*>(ws) + L.ent_rows), incl, s);
+                            lse, status, static_cast<char*>(ws) + L.comp, incl, s);
   return cuda_status(e);
 }
 

@@ -1,4 +1,4 @@
-// Internal launch interface between the C ABI (da_api.cu, noalloc.cu) and the kernel files.
+// Internal launch interface between the C ABI (da_api.cu) and the kernel files.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -18,7 +18,6 @@ struct StatsPtrs {
   float* seg_vsum;
   int32_t* n_tot;
   float* S_tot;
-  uint8_t* comp;       // compensation tiles of the tensor-core path, or NULL
 };
 
 struct Dims {
@@ -27,34 +26,15 @@ struct Dims {
 };
 
 // Argument checks shared by every entry point (da_api.cu).  check_dims fills g from dims and
-// enforces every size limit of include/da.h; check_stats validates the output pointers for g.
+// enforces every size limit of include/da.h; check_stats validates the output pointers.
 da_status check_dims(const da_dims* dims, Dims* g);
-da_status check_stats(const Dims& g, const da_cluster_stats* st, StatsPtrs* p);
+da_status check_stats(const da_cluster_stats* st, StatsPtrs* p);
 
 // Workspace layout (byte offsets), shared by every call.
 struct WsLayout {
-  size_t status, norms, sched, ent_rows, total;
+  size_t status, norms, sched, comp, total;
 };
 WsLayout ws_layout(const Dims& g);
-
-// Compensation tiles (byte offsets inside da_cluster_stats.comp_tiles; layout in include/da.h).
-// An entry tile's operand rows come in groups of 8: group a holds the 64-column panel 0 of its
-// 8 rows (1024 B) and then panel 1 (1024 B), each 128-byte row with 16-byte chunk k stored at
-// k XOR (row mod 8).  A run of whole groups is thus one contiguous range for both panels.
-constexpr int kEntRows = 128;                           // rows of one block's entry tile (= block)
-constexpr size_t kEntGroup = 2048;                       // 8 rows x 2 panels x 128 B
-constexpr size_t kEntVOff = 16 * kEntGroup;              // -S_e / n_e rows (after the 32 KB of centroid rows)
-constexpr size_t kEntBiasOff = 2 * kEntVOff;             // log2 n_e per row (fp32)
-__host__ __device__ constexpr size_t ent_byte(int row, int panel, int chunk) {
-  return (size_t)(row >> 3) * kEntGroup + (size_t)panel * 1024 + (size_t)(row & 7) * 128 + (size_t)((chunk ^ (row & 7)) << 4);
-}
-constexpr size_t kEntTileBytes = kEntBiasOff + kEntRows * sizeof(float);   // 66048
-struct CompLayout {
-  size_t ent, cmean, cbias, total;
-  int cpad;                                              // C rounded up to 128 (bias row length)
-};
-bool comp_tiles_used(const Dims& g);                     // the tensor-core path
-CompLayout comp_layout(const Dims& g);                   // total 0 when not used
 
 // stats.cu
 cudaError_t launch_centroid_norms(const Dims& g, const void* cent, float* norms, cudaStream_t s);
@@ -73,13 +53,16 @@ cudaError_t launch_reassign_tc(const Dims& g, const void* K, const void* V, cons
 
 // attention_tc.cu
 bool attention_tc_supported(const Dims& g);
-// ent_rows: [B*H*nB] int32 workspace for the per-item entry row counts (written, then read, by
-// this call); stats unused (a zero StatsPtrs) in the inclusion-probability mode.
+size_t attention_tc_scratch_bytes(const Dims& g);   // compensation chunks of every item
 cudaError_t launch_attention_tc(const Dims& g, const void* Q, const void* K, const void* V,
                                 const int32_t* kv_idx, const int32_t* kv_cnt, int max_sel,
                                 const int32_t* schedule, const void* cent, const StatsPtrs& st, float scale,
-                                void* O, float* lse, int* status, int32_t* ent_rows, const float* incl,
+                                void* O, float* lse, int* status, void* comp, const float* incl,
                                 cudaStream_t s);
+
+// comp_build.cu
+cudaError_t launch_comp_build(const Dims& g, const int32_t* kv_idx, const int32_t* kv_cnt, int max_sel,
+                              const StatsPtrs& st, void* out, cudaStream_t s);
 
 // simt_f32.cu / simt_bf16.cu
 #define DA_SIMT_DECL(SUFFIX)                                                                                 \

@@ -63,7 +63,7 @@ extern "C" DA_API da_status da_reassign_noalloc(const da_dims* dims, const void*
   if (!K || !V || !centroids) return DA_ERR_INVALID_ARG;
   if (!aligned16(K) || !aligned16(V) || !aligned16(centroids)) return DA_ERR_ALIGNMENT;
   StatsPtrs sp;
-  if ((st = check_stats(g, out, &sp)) != DA_OK) return st;
+  if ((st = check_stats(out, &sp)) != DA_OK) return st;
   if ((size_t)g.B * g.H * g.C > kNoAllocMaxNorms) return DA_ERR_WORKSPACE;   // beyond the built-in scratch
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return DA_ERR_CUDA;

@@ -9,9 +9,8 @@
 //   3. Every thread owns one key (= one TMEM lane) and keeps the running argmin of
 //      ||cbar_c||^2 - 2 k.cbar_c (ties to the lowest c; the key's own norm is the same for
 //      every c and is dropped).
-//   4. The same threads refresh the block's statistics (block_stats.cuh): sorted entry list,
-//      histogram row, entry index row, fp32 value sums and the block's entry tile for the fused
-//      attention (centroid rows, negated means, log2 counts), reading the block's value rows from
+//   4. The same 128 threads refresh the block's statistics (block_stats.cuh): sorted entry list,
+//      histogram row, entry index row and fp32 value sums, reading the block's value rows from
 //      shared memory (copied with cp.async into centroid buffer 0 once the last MMA reading it is
 //      done, overlapping the remaining epilogues).
 // The CTA takes about 109 KB of shared memory and 256 TMEM columns, so two CTAs share an SM and
@@ -51,7 +50,7 @@ static_assert(2 * (kSmemBytes + 1024) <= 233472, "two CTAs per SM");
 __global__ void __launch_bounds__(kThreads, 2)
 reassign_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_c,
                    const __nv_bfloat16* __restrict__ V, const float* __restrict__ norms, StatsPtrs st, int N,
-                   int C, int nB, int* status, const __nv_bfloat16* __restrict__ cent) {
+                   int C, int nB, int* status) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -221,8 +220,7 @@ reassign_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     block_stats_group<__nv_bfloat16, kD, kThreads>(t, 1, s_assign, nk, reinterpret_cast<const __nv_bfloat16*>(sC0), C,
                                                    st.blk_hist + bj * C, st.seg_idx + bj * C, st.seg_n + bj,
                                                    st.seg_c + bj * kKeys, st.seg_cnt + bj * kKeys,
-                                                   st.seg_vsum + bj * kKeys * kD, *ssm, cent + (size_t)bh * C * kD,
-                                                   st.comp ? st.comp + bj * kEntTileBytes : nullptr);
+                                                   st.seg_vsum + bj * kKeys * kD, *ssm);
   }
   tc_fence_before();
   __syncthreads();
@@ -247,7 +245,7 @@ cudaError_t launch_reassign_tc(const Dims& g, const void* K, const void* V, cons
   if (e != cudaSuccess) return e;
   dim3 grid(g.nB, (unsigned)BH);
   reassign_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(tk, tc, static_cast<const __nv_bfloat16*>(V), norms, st, g.N,
-                                                   g.C, g.nB, status, static_cast<const __nv_bfloat16*>(cent));
+                                                   g.C, g.nB, status);
   return cudaGetLastError();
 }
 

@@ -17,22 +17,8 @@ WsLayout ws_layout(const Dims& g) {
   L.status = 0;
   L.norms = 256;
   L.sched = L.norms + up(BH * g.C * sizeof(float));
-  L.ent_rows = L.sched + up(BH * g.nB * sizeof(int32_t));
-  L.total = L.ent_rows + up(BH * g.nB * sizeof(int32_t));
-  return L;
-}
-
-bool comp_tiles_used(const Dims& g) { return attention_tc_supported(g); }
-
-CompLayout comp_layout(const Dims& g) {
-  auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
-  CompLayout L{0, 0, 0, 0, (g.C + 127) / 128 * 128};
-  if (!comp_tiles_used(g)) return L;
-  const size_t BH = (size_t)g.B * g.H;
-  L.ent = 0;
-  L.cmean = up(BH * g.nB * kEntTileBytes);
-  L.cbias = L.cmean + up(BH * g.C * g.d * 2);
-  L.total = L.cbias + up(BH * L.cpad * sizeof(float));
+  L.comp = L.sched + up(BH * g.nB * sizeof(int32_t));
+  L.total = L.comp + up(attention_tc_scratch_bytes(g));
   return L;
 }
 
@@ -75,20 +61,13 @@ __global__ void __launch_bounds__(128) block_stats_kernel(const T* __restrict__ 
 // A warp per (head, cluster): it walks the blocks in order, finds the cluster's entry through
 // seg_idx (eight blocks looked up at a time) and adds the entry row, lanes over the value columns
 // (coalesced rows; registers; blocks in order: deterministic bits).
-// With compensation tiles (cmean != NULL) it also writes the cluster's mean S_c / n_c in bf16 and
-// log2 n_c (-inf when empty); the bias row of a head is padded to cpad with -inf.
 template <int D>
-__global__ void __launch_bounds__(128) totals_kernel(StatsPtrs st, int C, int block, int nB,
-                                                     __nv_bfloat16* __restrict__ cmean, float* __restrict__ cbias,
-                                                     int cpad) {
+__global__ void __launch_bounds__(128) totals_kernel(StatsPtrs st, int C, int block, int nB) {
   constexpr int NS = D / 32;              // columns per lane
   const int bh = blockIdx.x;
   const int c = blockIdx.y * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (c >= C) {
-    if (cbias && c < cpad && lane == 0) cbias[(size_t)bh * cpad + c] = -INFINITY;
-    return;
-  }
+  if (c >= C) return;                     // (C is a multiple of 32)
   float acc[NS];
 #pragma unroll
   for (int i = 0; i < NS; ++i) acc[i] = 0.f;
@@ -118,16 +97,6 @@ __global__ void __launch_bounds__(128) totals_kernel(StatsPtrs st, int C, int bl
     for (int i = 0; i < NS; ++i) dst[i] = acc[i];
   }
   if (lane == 0) st.n_tot[(size_t)bh * C + c] = n;
-  if (cmean) {
-    const int nt = __shfl_sync(0xffffffffu, n, 0);
-    __nv_bfloat16* mrow = cmean + ((size_t)bh * C + c) * D + lane * NS;
-#pragma unroll
-    for (int i = 0; i < NS; i += 2) {
-      const float a = nt > 0 ? acc[i] / (float)nt : 0.f, b = nt > 0 ? acc[i + 1] / (float)nt : 0.f;
-      *reinterpret_cast<__nv_bfloat162*>(mrow + i) = __floats2bfloat162_rn(a, b);
-    }
-    if (lane == 0) cbias[(size_t)bh * cpad + c] = nt > 0 ? log2f((float)nt) : -INFINITY;
-  }
 }
 
 // Second moment of each cluster's keys about its representative (the variance correction of
@@ -265,13 +234,9 @@ cudaError_t launch_centroid_update(const Dims& g, const StatsPtrs& st, void* cen
 }
 
 cudaError_t launch_totals(const Dims& g, const StatsPtrs& st, cudaStream_t s) {
-  const CompLayout L = comp_layout(g);
-  __nv_bfloat16* cmean = st.comp ? reinterpret_cast<__nv_bfloat16*>(st.comp + L.cmean) : nullptr;
-  float* cbias = st.comp ? reinterpret_cast<float*>(st.comp + L.cbias) : nullptr;
-  const int rows = st.comp ? L.cpad : g.C;
-  dim3 grid(g.B * g.H, (rows + 3) / 4);                 // 4 clusters (warps) per CTA
-  if (g.d == 128) totals_kernel<128><<<grid, 128, 0, s>>>(st, g.C, g.block, g.nB, cmean, cbias, L.cpad);
-  else totals_kernel<64><<<grid, 128, 0, s>>>(st, g.C, g.block, g.nB, nullptr, nullptr, L.cpad);
+  dim3 grid(g.B * g.H, (g.C + 3) / 4);                  // 4 clusters (warps) per CTA
+  if (g.d == 128) totals_kernel<128><<<grid, 128, 0, s>>>(st, g.C, g.block, g.nB);
+  else totals_kernel<64><<<grid, 128, 0, s>>>(st, g.C, g.block, g.nB);
   return cudaGetLastError();
 }
 

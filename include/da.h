@@ -90,40 +90,7 @@ typedef struct {
   float*   seg_vsum;  /* [B,H,nB,block,d] fp32 sum of the entry's value rows */
   int32_t* n_tot;     /* [B,H,C]          n_c = sum_j n_{c,j} */
   float*   S_tot;     /* [B,H,C,d]        S_c = sum of the value rows of cluster c (fp32) */
-  void*    comp_tiles;/* da_comp_tiles_bytes(dims) bytes: the same statistics laid out as the
-                         operand tiles of the fused attention kernel (see below); required when
-                         that byte count is non-zero, ignored (may be NULL) when it is zero */
 } da_cluster_stats;
-
-/*
- * Compensation tiles (comp_tiles), written by da_reassign for the tensor-core
- * attention path (bf16, d = 128, block = 128; da_comp_tiles_bytes is 0 for
- * other dims).  The compensated term of q-block i is computed in the per-key
- * correction form: every cluster enters once with its head-wide count and
- * mean, and the entries of the selected blocks are taken out again:
- *   sum_c e^{s q.cbar_c} (S_c - sum_{j in sel(i)} S_{c,j})
- *     = sum_c e^{s q.cbar_c + ln n_c} (S_c / n_c)
- *       - sum_{j in sel(i)} sum_{e in block j} e^{s q.cbar_{c_e} + ln n_e} (S_e / n_e),
- * and likewise for the denominator with the counts.  Regions, in this order,
- * each starting on a 256-byte boundary:
- *   entry tiles   [B,H,nB] x 66048 bytes, one per key block, rows = the block's
- *                 entries e in list order, padded with zero rows (and bias
- *                 -inf) to a multiple of 8 rows:
- *                   bytes [0, 32768)      cbar_{c_e} as bf16, in groups of 8
- *                                         rows: group a at 2048 a holds the
- *                                         columns 0-63 of its 8 rows (128 bytes
- *                                         each), then the columns 64-127;
- *                   bytes [32768, 65536)  -S_e / n_e as bf16, same layout;
- *                   bytes [65536, 66048)  log2 n_e as fp32 per row;
- *                 every 128-byte row stored with the 16-byte chunks of row r
- *                 permuted as chunk k -> k XOR (r mod 8) (the 128-byte swizzle
- *                 the tensor-core operand descriptors read);
- *   cluster means [B,H,C,d] bf16, S_c / n_c (0 for an empty cluster);
- *   cluster bias  [B,H,ceil(C/128)*128] fp32, log2 n_c (-inf for an empty
- *                 cluster and past C).
- */
-/* Bytes of da_cluster_stats.comp_tiles for these dims (0: not used). */
-DA_API size_t da_comp_tiles_bytes(const da_dims* dims);
 
 /*
  * Fixed block plan ("a few blocks fixed once offline by position",
@@ -145,8 +112,7 @@ typedef struct {
 DA_API int da_version(void);
 
 /* Bytes of device workspace da_reassign and da_attention need for these dims
- * (status word, centroid norms, work order, per-item entry row counts).
- * Returns 0 for invalid dims.
+ * (status word, centroid norms, work order).  Returns 0 for invalid dims.
  * The workspace must be zero-filled once before its first use; afterwards
  * the library keeps it consistent itself. */
 DA_API size_t da_workspace_bytes(const da_dims* dims);
@@ -189,15 +155,39 @@ DA_API da_status da_mask_prepare(const da_dims* dims, const da_block_mask* mask,
  * runs over both kinds of logits with fp32 accumulation; O = [B,H,N,d] in
  * dims.dtype; lse (nullable) = [B,H,N] fp32 natural-log sum of exponentials.
  * scale <= 0 selects 1/sqrt(d).  stats must come from da_reassign on the
- * same K, V, centroids.  On the tensor-core path the cluster terms are taken
- * in the per-key correction form of stats.comp_tiles (one fused kernel, no
- * per-q-block table); the CUDA-core path counts n^U_c and sums vbar^U_c per
- * q-block itself.  Both give the complement form above up to rounding.
+ * same K, V, centroids.
  */
 DA_API da_status da_attention(const da_dims* dims, const void* Q, const void* K, const void* V,
                        const da_block_mask* mask, const void* centroids,
                        const da_cluster_stats* stats, float scale, void* O, float* lse,
                        void* ws, size_t ws_bytes, da_stream stream);
+
+/*
+ * The two halves of da_attention, for callers that time or schedule them
+ * apart; da_attention(...) is da_compensation(...) followed by
+ * da_attention_prebuilt(...) with the same arguments.
+ *
+ * da_compensation: the per-q-block compensation statistics (DecoupAttn
+ * abstract: every key outside the fixed blocks is compensated through its
+ * cluster).  For every q-block i and cluster c it writes, into the workspace,
+ *   n^U_c = n_c - sum_{j in sel(i)} n_{c,j}   (as log2 n^U_c, -inf when 0)
+ *   vbar^U_c = (S_c - sum_{j in sel(i)} S_{c,j}) / n^U_c   (bf16),
+ * the fp32 subtraction summed in a fixed order.  bf16 inputs with d = 128 and
+ * block = 128 only; for other dims it launches nothing and returns DA_OK (the
+ * CUDA-core attention path forms these values itself).
+ *
+ * da_attention_prebuilt: the fused attention of da_attention, reading the
+ * compensation values da_compensation left in the same workspace.  Those
+ * values belong to the stats and mask they were built from: after
+ * da_reassign refreshes stats, or with another mask, call da_compensation
+ * again first.  Arguments, layouts and errors as in da_attention.
+ */
+DA_API da_status da_compensation(const da_dims* dims, const da_block_mask* mask, const da_cluster_stats* stats,
+                          void* ws, size_t ws_bytes, da_stream stream);
+DA_API da_status da_attention_prebuilt(const da_dims* dims, const void* Q, const void* K, const void* V,
+                                const da_block_mask* mask, const void* centroids,
+                                const da_cluster_stats* stats, float scale, void* O, float* lse,
+                                void* ws, size_t ws_bytes, da_stream stream);
 
 /*
  * Lloyd update step (the clustering the pages build on: "Least squares
@@ -232,7 +222,7 @@ DA_API da_status da_centroid_update(const da_dims* dims, const da_cluster_stats*
  *   s q.cbar_c + ln n^U_c + s^2/2 sum_t q_t^2 D_{c,t},
  * D = spread.  It runs on the CUDA cores for both dtypes (fp32 arithmetic,
  * the bf16 inputs upcast): a reference-grade path, not the tensor-core one.
- * Arguments, layouts and errors as
+ * It does not use da_compensation's values.  Arguments, layouts and errors as
  * in da_attention, plus spread ([B,H,C,d] fp32, read; DA_ERR_INVALID_ARG if
  * NULL).
  */

@@ -122,62 +122,3 @@ def check_attention(inp, b, h, O, lse, a_gpu, q_blocks=None, scale=None):
         worst = max(worst, float(err))
     return worst
 
-
-def _unswizzle_rows(tile: np.ndarray, rows: int) -> np.ndarray:
-    """An entry tile's operand (32 KB): 8-row groups of 2048 B holding panel 0 (columns 0-63) then
-    panel 1 of their rows, 128 B per row, chunk k of row r stored at k ^ (r % 8) -> [rows][128]
-    bf16 bits."""
-    t = tile.reshape(16, 2, 8, 8, 16)[: rows // 8]          # [group][panel][row in group][chunk][byte]
-    r = np.arange(8)[:, None]
-    k = np.arange(8)[None, :]
-    out = t[:, :, r, k ^ r]                                   # [group][panel][row][chunk][byte], logical chunks
-    return np.ascontiguousarray(out.transpose(0, 2, 1, 3, 4)).reshape(rows, 256).view(np.uint16)
-
-
-def _bf16_bits_to_f64(b: np.ndarray) -> np.ndarray:
-    return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
-
-
-def check_comp_tiles(inp, b, h, st, a_gpu, blocks=None):
-    """The compensation tiles of the tensor-core path against the oracle's block entries and totals:
-    centroid rows bit-exact, negated entry means and cluster means within one bf16 rounding of the
-    fp64 values, log2 counts, zero rows and -inf bias past the entries."""
-    import block_sparse_cluster_b200 as da
-    w = inp.w
-    dims = dims_of(w)
-    if da.da_comp_tiles_bytes(dims) == 0:
-        return
-    N, C, bs, nB, d = w.N, w.C, w.block, w.nB, w.d
-    up = lambda x: (x + 255) // 256 * 256
-    BH = w.B * w.H
-    bh = b * w.H + h
-    comp = st.comp_tiles.cpu().numpy()
-    tile_bytes = 66048
-    cent_bits = inp.centroids[b, h].contiguous().view(torch.int16).numpy().view(np.uint16)
-    js = range(nB) if blocks is None else blocks
-    for j in js:
-        c, n, S = oracle.block_entries(a_gpu, inp.V[b, h], C, N, bs, j)
-        E = len(c)
-        E8 = (E + 7) // 8 * 8
-        t = comp[(bh * nB + j) * tile_bytes:(bh * nB + j + 1) * tile_bytes]
-        kb = _unswizzle_rows(t[:32768], E8)
-        vb = _unswizzle_rows(t[32768:65536], E8)
-        bias = t[65536:].view(np.float32)[:E8]
-        assert np.array_equal(kb[:E], cent_bits[c]), f"block {j}: entry centroid rows"
-        want = -S / n[:, None]
-        got = _bf16_bits_to_f64(vb[:E])
-        assert (np.abs(got - want) <= 2.0 ** -8 * np.abs(want) + 1e-6).all(), f"block {j}: entry means"
-        assert np.allclose(bias[:E], np.log2(n), rtol=0, atol=1e-6), f"block {j}: entry bias"
-        assert not kb[E:].any() and not vb[E:].any() and np.isneginf(bias[E:]).all(), f"block {j}: padding rows"
-    cmean_off = up(BH * nB * tile_bytes)
-    cbias_off = cmean_off + up(BH * C * d * 2)
-    cpad = (C + 127) // 128 * 128
-    nt, St = oracle.cluster_totals(a_gpu, inp.V[b, h], C)
-    means = _bf16_bits_to_f64(comp[cmean_off + bh * C * d * 2:cmean_off + (bh + 1) * C * d * 2].view(np.uint16))
-    means = means.reshape(C, d)
-    want = np.where(nt[:, None] > 0, St / np.maximum(nt, 1)[:, None], 0.0)
-    assert (np.abs(means - want) <= 2.0 ** -8 * np.abs(want) + 1e-6).all(), "cluster means"
-    cb = comp[cbias_off + bh * cpad * 4:cbias_off + (bh + 1) * cpad * 4].view(np.float32)
-    live = nt > 0
-    assert np.allclose(cb[:C][live], np.log2(nt[live]), rtol=0, atol=1e-6), "cluster bias"
-    assert np.isneginf(cb[:C][~live]).all() and np.isneginf(cb[C:]).all(), "cluster bias padding"

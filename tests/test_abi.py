@@ -32,7 +32,7 @@ def test_every_declared_symbol_is_exported():
 
 
 def test_version_and_strings():
-    assert da.da_version() == 200
+    assert da.da_version() == 103
     for code in range(10):
         assert da.da_status_string(code) and da.da_status_string(code) != "unknown status"
 
@@ -52,13 +52,13 @@ def test_workspace_bytes():
 
 
 def _call_reassign(dims, K=0x1000, V=0x1000, C=0x1000, stats=None, ws=0x1000, ws_bytes=1 << 30):
-    s = stats if stats is not None else da._Stats(*([0x1000] * 10))
+    s = stats if stats is not None else da._Stats(*([0x1000] * 9))
     return da._lib.da_reassign(ctypes.byref(dims.c()), K, V, C, ctypes.byref(s), ws, ws_bytes, None)
 
 
 def _call_attention(dims, mask=None, O=0x1000, lse=None, ws_bytes=1 << 30):
     m = mask if mask is not None else da._Mask(0x1000, 0x1000, 4, None)
-    s = da._Stats(*([0x1000] * 10))
+    s = da._Stats(*([0x1000] * 9))
     return da._lib.da_attention(ctypes.byref(dims.c()), 0x1000, 0x1000, 0x1000, ctypes.byref(m), 0x1000,
                                 ctypes.byref(s), 0.0, O, lse, 0x1000, ws_bytes, None)
 
@@ -75,9 +75,9 @@ def test_reassign_rejects_pointers_and_workspace():
     d = _dims()
     assert _call_reassign(d, K=None) == 1
     assert _call_reassign(d, V=0x1008) == 4
-    bad = da._Stats(*([0x1000] * 8 + [None, 0x1000]))
+    bad = da._Stats(*([0x1000] * 8 + [None]))
     assert _call_reassign(d, stats=bad) == 1
-    bad = da._Stats(*([0x1000] * 7 + [0x1004, 0x1000, 0x1000]))
+    bad = da._Stats(*([0x1000] * 7 + [0x1004, 0x1000]))
     assert _call_reassign(d, stats=bad) == 4
     assert _call_reassign(d, ws=None) == 1
     assert _call_reassign(d, ws_bytes=16) == 9
@@ -110,69 +110,37 @@ def test_shape_overflow_rejected():
     assert da.da_workspace_bytes(_dims(B=1, H=1, N=(1 << 28) - 128, C=1024)) > 0
 
 
-def test_comp_tiles_bytes_and_pointer():
-    # the tensor-core path (bf16, d = 128, block = 128) needs the compensation tiles; others do not
+def test_split_attention_calls_reject_arguments():
     d = _dims()
-    nB, BH, C = d.nB, 12, 256
-    up = lambda x: (x + 255) // 256 * 256
-    want = up(BH * nB * 66048) + up(BH * C * 128 * 2) + up(BH * 256 * 4)
-    assert da.da_comp_tiles_bytes(d) == want
-    assert da.da_comp_tiles_bytes(_dims(dtype=torch.float32)) == 0
-    assert da.da_comp_tiles_bytes(_dims(d=64)) == 0
-    assert da.da_comp_tiles_bytes(_dims(block=64)) == 0
-    assert da.da_comp_tiles_bytes(_dims(C=416)) == up(BH * nB * 66048) + up(BH * 416 * 256) + up(BH * 512 * 4)
-    no_tiles = da._Stats(*([0x1000] * 9 + [None]))
-    assert _call_reassign(d, stats=no_tiles) == 1
-    assert _call_attention_stats(d, no_tiles) == 1
-    assert _call_reassign(d, stats=da._Stats(*([0x1000] * 9 + [0x1080]))) == 4    # 256-byte alignment
-    assert _call_reassign(_dims(dtype=torch.float32), stats=no_tiles) != 1       # not needed there
-
-
-def _call_attention_stats(dims, st):
+    st = da._Stats(*([0x1000] * 9))
     m = da._Mask(0x1000, 0x1000, 4, None)
-    return da._lib.da_attention(ctypes.byref(dims.c()), 0x1000, 0x1000, 0x1000, ctypes.byref(m), 0x1000,
-                                ctypes.byref(st), 0.0, 0x1000, None, 0x1000, 1 << 30, None)
-
-
-def test_noalloc_checks_match_da_reassign():
-    """da_reassign_noalloc shares da_reassign's argument checks, so both accept the same dims and
-    refuse the same ones with the same codes, the size limits of the header included."""
-    cases = [dict(dtype=torch.float16), dict(d=96), dict(C=48), dict(N=0),
-             dict(B=64, H=1024, N=1 << 20),                       # B*H*nB >= 2^31
-             dict(B=1, H=1, N=1 << 28, C=1024)]                   # nB*C >= 2^31 (one head's lookup rows)
-    for kw in cases:
-        d = _dims(**kw)
-        s = da._Stats(*([0x1000] * 10))
-        want = _call_reassign(d, stats=s)
-        got = da._lib.da_reassign_noalloc(ctypes.byref(d.c()), 0x1000, 0x1000, 0x1000, ctypes.byref(s), None)
-        assert want != 0 and got == want, (kw, want, got)
-    d = _dims()
-    for st in (da._Stats(*([0x1000] * 9 + [None])), da._Stats(*([0x1000] * 7 + [0x1004, 0x1000, 0x1000]))):
-        want = _call_reassign(d, stats=st)
-        got = da._lib.da_reassign_noalloc(ctypes.byref(d.c()), 0x1000, 0x1000, 0x1000, ctypes.byref(st), None)
-        assert got == want, (want, got)
-    assert da._lib.da_reassign_noalloc(ctypes.byref(d.c()), None, 0x1000, 0x1000,
-                                       ctypes.byref(da._Stats(*([0x1000] * 10))), None) == 1
+    assert da._lib.da_compensation(ctypes.byref(d.c()), ctypes.byref(m), ctypes.byref(st), 0x1000, 0, None) == 9
+    assert da._lib.da_compensation(ctypes.byref(d.c()), ctypes.byref(da._Mask(None, 0x1000, 4, None)),
+                                   ctypes.byref(st), 0x1000, 1 << 30, None) == 1
+    assert da._lib.da_attention_prebuilt(ctypes.byref(d.c()), 0x1000, 0x1000, 0x1000, ctypes.byref(m), 0x1000,
+                                         ctypes.byref(st), 0.0, None, None, 0x1000, 1 << 30, None) == 1
+    assert da._lib.da_attention_prebuilt(ctypes.byref(d.c()), 0x1000, 0x1000, 0x1000, ctypes.byref(m), 0x1000,
+                                         ctypes.byref(st), 0.0, 0x1002, None, 0x1000, 1 << 30, None) == 4
 
 
 def test_centroid_update_rejects_arguments():
     d = _dims()
-    st = da._Stats(*([0x1000] * 10))
+    st = da._Stats(*([0x1000] * 9))
     assert da._lib.da_centroid_update(ctypes.byref(d.c()), ctypes.byref(st), None, None) == 1
     assert da._lib.da_centroid_update(ctypes.byref(d.c()), ctypes.byref(st), 0x1004, None) == 4
-    bad = da._Stats(*([0x1000] * 7 + [0x1004, 0x1000, 0x1000]))
+    bad = da._Stats(*([0x1000] * 7 + [0x1004, 0x1000]))
     assert da._lib.da_centroid_update(ctypes.byref(d.c()), ctypes.byref(bad), 0x1000, None) == 4
 
 
 def test_spread_calls_reject_arguments():
     d = _dims()
-    st = da._Stats(*([0x1000] * 10))
+    st = da._Stats(*([0x1000] * 9))
     m = da._Mask(0x1000, 0x1000, 4, None)
     sp = da._lib.da_cluster_spread
     assert sp(ctypes.byref(d.c()), 0x1000, 0x1000, ctypes.byref(st), None, None) == 1
     assert sp(ctypes.byref(d.c()), None, 0x1000, ctypes.byref(st), 0x1000, None) == 1
     assert sp(ctypes.byref(d.c()), 0x1000, 0x1000, ctypes.byref(st), 0x1008, None) == 4
-    bad = da._Stats(*([0x1000] * 7 + [0x1004, 0x1000, 0x1000]))
+    bad = da._Stats(*([0x1000] * 7 + [0x1004, 0x1000]))
     assert sp(ctypes.byref(d.c()), 0x1000, 0x1000, ctypes.byref(bad), 0x1000, None) == 4
     at = da._lib.da_attention_spread
     ok = (0x1000, 0x1000, 0x1000, ctypes.byref(m), 0x1000, ctypes.byref(st))
@@ -192,3 +160,24 @@ def test_sip_call_rejects_arguments():
     assert f(ctypes.byref(d.c()), *ok, 0x1000, 0.0, 0x1000, None, 0x1000, 0, None) == 9
     f32 = _dims(dtype=torch.float32)
     assert f(ctypes.byref(f32.c()), *ok, 0x1000, 0.0, 0x1000, None, 0x1000, 1 << 30, None) == 5
+
+
+def test_noalloc_checks_match_da_reassign():
+    """da_reassign_noalloc shares da_reassign's argument checks, so both accept the same dims and
+    refuse the same ones with the same codes, the size limits of include/da.h included."""
+    cases = [dict(dtype=torch.float16), dict(d=96), dict(C=48), dict(N=0),
+             dict(B=64, H=1024, N=1 << 20),                       # B*H*nB >= 2^31
+             dict(B=1, H=1, N=1 << 28, C=1024)]                   # nB*C >= 2^31 (one head's lookup rows)
+    for kw in cases:
+        d = _dims(**kw)
+        s = da._Stats(*([0x1000] * 9))
+        want = _call_reassign(d, stats=s)
+        got = da._lib.da_reassign_noalloc(ctypes.byref(d.c()), 0x1000, 0x1000, 0x1000, ctypes.byref(s), None)
+        assert want != 0 and got == want, (kw, want, got)
+    d = _dims()
+    for st in (da._Stats(*([0x1000] * 8 + [None])), da._Stats(*([0x1000] * 7 + [0x1004, 0x1000]))):
+        want = _call_reassign(d, stats=st)
+        got = da._lib.da_reassign_noalloc(ctypes.byref(d.c()), 0x1000, 0x1000, 0x1000, ctypes.byref(st), None)
+        assert got == want, (want, got)
+    assert da._lib.da_reassign_noalloc(ctypes.byref(d.c()), None, 0x1000, 0x1000,
+                                       ctypes.byref(da._Stats(*([0x1000] * 9))), None) == 1

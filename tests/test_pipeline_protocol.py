@@ -19,15 +19,12 @@ interleavings, and checks that
 * every role finishes (no deadlock).
 
 It mirrors the step structure of attention_tc.cu: per work item, one step per
-selected block, one per 128-cluster chunk, then one per entry tile of the
-selected blocks' cluster entries; key, value and bias-row rings; softmax
-warpgroup X taking the steps g with g & 1 == X, with its own S buffer (P
-written over it) and accumulator O_X; at the end of an item the two
-warpgroups exchange (max, sum) through a double-buffered shared array and each
-reads both accumulators.  Chunk and entry tiles are written by the Reassign
-Cache before the kernel starts, so they are plain inputs here; an entry tile
-arrives as several copies on one barrier, which the model counts as one
-transaction.
+selected block followed by one step per 128-cluster chunk; key, value and
+bias-row rings; softmax warpgroup X taking the steps g with g & 1 == X, with its
+own S buffer (P written over it) and accumulator O_X; at the end of an item the
+two warpgroups exchange (max, sum) through a double-buffered shared array and
+each reads both accumulators.  The compensation chunks are written by an
+earlier kernel, so they are plain inputs here.
 """
 import random
 
@@ -74,8 +71,7 @@ class Barrier:
 class Machine:
     def __init__(self, items, nchunk, rng, lazy_v_wait=False, skip_b_empty=False, single_xch=False,
                  no_final_wait=False, single_xch_barrier=False):
-        # per item of one CTA: nsel, or (nsel, entry tiles)
-        self.items = [(x, 0) if isinstance(x, int) else tuple(x) for x in items]
+        self.items = items                     # list of nsel per item of one CTA
         self.nchunk = nchunk
         self.rng = rng
         self.lazy_v_wait = lazy_v_wait         # planted: value lane waits for a free slot only at chunk steps
@@ -163,8 +159,8 @@ class Machine:
     def producer(self):
         """Lane 0 of the producer warp: query tiles, key / centroid tiles, bias rows."""
         g = 0
-        for n, (nsel, nent) in enumerate(self.items):
-            T = nsel + self.nchunk + nent
+        for n, nsel in enumerate(self.items):
+            T = nsel + self.nchunk
             yield lambda: self.q_empty.test(n - 1)
             self.q_full.expect_tx(1)
             self.tma_load(self.q_full, "Q", n)
@@ -184,8 +180,8 @@ class Machine:
     def producer_v(self):
         """Lane 1 of the producer warp: value / vbar^U tiles."""
         g = 0
-        for n, (nsel, nent) in enumerate(self.items):
-            T = nsel + self.nchunk + nent
+        for n, nsel in enumerate(self.items):
+            T = nsel + self.nchunk
             for s in range(T):
                 vs = g % VSTAGES
                 if not self.lazy_v_wait or s >= nsel:
@@ -196,8 +192,8 @@ class Machine:
 
     def mma(self):
         g = 0
-        for n, (nsel, nent) in enumerate(self.items):
-            T = nsel + self.nchunk + nent
+        for n, nsel in enumerate(self.items):
+            T = nsel + self.nchunk
             yield lambda: self.q_full.test(n)
             yield lambda: self.k_full[g % KSTAGES].test(g // KSTAGES)
             self.holds("Q", n)
@@ -230,8 +226,8 @@ class Machine:
     def softmax(self, X):
         g0 = 0
         u = 0                                   # products into O_X issued so far
-        for n, (nsel, nent) in enumerate(self.items):
-            T = nsel + self.nchunk + nent
+        for n, nsel in enumerate(self.items):
+            T = nsel + self.nchunk
             first = True
             for s in range((X - g0) & 1, T, 2):
                 g = g0 + s
@@ -301,9 +297,6 @@ class Machine:
 CASES = [
     ([4], 2), ([37], 2), ([0], 2), ([0, 37, 2, 0, 5], 2), ([30, 30, 30], 4), ([1, 0, 0, 1], 1),
     ([9, 3, 0, 12], 8), ([2], 1), ([0, 0, 0], 3), ([40, 1], 4),
-    # with entry tiles: a block's entries always fill at least one tile row, so nsel > 0 => tiles > 0
-    ([(30, 8), (26, 7), (30, 8)], 4), ([(1, 1), (0, 0), (2, 1), (0, 0)], 1), ([(9, 3), (1, 1)], 8),
-    ([(3, 1), (3, 1), (3, 1), (3, 1)], 2),
 ]
 
 

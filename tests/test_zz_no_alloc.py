@@ -19,7 +19,7 @@ from tests import parity as P
 def test_noalloc_rejects_dims_beyond_its_scratch():
     import block_sparse_cluster_b200 as da
     dims = da.Dims(B=1, H=512, N=4096, d=128, C=1024, block=128)       # B*H*C = 524288 > 262144
-    s = da._Stats(*([0x1000] * 10))
+    s = da._Stats(*([0x1000] * 9))
     code = da._lib.da_reassign_noalloc(ctypes.byref(dims.c()), 0x1000, 0x1000, 0x1000, ctypes.byref(s), None)
     assert code == da.STATUS_NAMES.index("DA_ERR_WORKSPACE")
 
