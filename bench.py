@@ -132,6 +132,22 @@ def _dist():
     return ws, rank, local
 
 
+def head_slice(H: int, rank: int, world: int) -> range:
+    """The heads rank `rank` of `world` takes when the ranks split one workload's heads: contiguous
+    slices, the first H % world ranks one head more."""
+    base, extra = divmod(H, world)
+    lo = rank * base + min(rank, extra)
+    return range(lo, lo + base + (1 if rank < extra else 0))
+
+
+def _sum_over_ranks(x: float, ws: int, device) -> float:
+    if ws == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
+    return float(t.item())
+
+
 def _max_over_ranks(x: float, ws: int, device) -> float:
     if ws == 1:
         return x
@@ -227,7 +243,9 @@ def _config(w: W.Workload, args):
     return {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} ({w.T}x{w.Hs}x{w.Ws} latent) d={w.d} block={w.block} "
                         f"C={w.C} density={w.density}",
             "B": w.B, "H": w.H, "N": w.N, "d": w.d, "block": w.block, "C": w.C, "density": w.density,
-            "seed": args.seed, "parallelism": "independent heads per rank (weak)",
+            "seed": args.seed,
+            "parallelism": ("heads split over the ranks (strong)" if getattr(args, "split_heads", False)
+                            else "independent heads per rank (weak)"),
             "l2": _l2_note(w)}
 
 
@@ -403,6 +421,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--heads", type=int, default=0, help="override the head count (profiling runs)")
+    ap.add_argument("--split-heads", action="store_true",
+                    help="under torchrun, the ranks share one workload's heads (strong scaling) instead of each "
+                         "running its own copy")
     ap.add_argument("--loop", action="store_true", help="run the reassign-cache loop workload instead")
     ap.add_argument("--spread", action="store_true",
                     help="time the variance-corrected path (reassign + cluster spread + corrected attention)")
@@ -432,10 +453,19 @@ def main():
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    seed = args.seed + 1000 * rank
-    inp = W.make_inputs(w, seed=seed)
+    if args.split_heads:
+        # the ranks share one workload's heads (strong scaling): same seed, a slice of heads each
+        seed = args.seed
+        inp = W.make_inputs(w, seed=seed, heads=head_slice(w.H, rank, ws))
+    else:
+        # every rank its own copy of the workload (weak scaling)
+        seed = args.seed + 1000 * rank
+        inp = W.make_inputs(w, seed=seed)
+    full_w = w
+    w = inp.w
     dims = da.Dims(w.B, w.H, w.N, w.d, w.C, w.block, w.torch_dtype)
     eff = W.effective_flops(w, inp.kv_cnt, inp.kv_idx)
+    eff_job = _sum_over_ranks(eff, ws, dev)
 
     stream = torch.cuda.current_stream(dev)
     eng = da.DecoupledAttention(dims, dev)
@@ -489,7 +519,7 @@ def main():
     ms = _max_over_ranks(ms_local, ws, dev)
     att_ms = _max_over_ranks(att_ms_local, ws, dev)
     comp_ms = _max_over_ranks(comp_ms_local, ws, dev)
-    value = ws * eff / (ms * 1e-3) / 1e12
+    value = eff_job / (ms * 1e-3) / 1e12
 
     # one cold step: L2 flushed by writing a 256 MB buffer first (the timed steps above run warm)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -559,7 +589,7 @@ def main():
             if e.status() != 0:
                 raise RuntimeError("device status after the end-to-end steps")
         e2e_ms = _max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, ws, dev)
-        e2e = {"value": ws * eff / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+        e2e = {"value": eff_job / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "head_groups": groups}
 
     if rank == 0:
@@ -569,13 +599,14 @@ def main():
         sustained = float(peaks.get("bf16_tflops_sustained", peak))
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws, "steps": K_steps,
-            "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "strong" if args.split_heads else "weak",
             "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
-            "config": _config(w, args),
+            "config": _config(full_w, args),
             "pct_of_bf16_peak": 100.0 * (value / ws) / peak,
             "breakdown_ms": {"reassign": reas_ms_local, "compensation": comp_ms_local, "attention": att_ms_local},
             "ms_per_step_median": median_ms, "cold_ms_per_step": cold_ms,
-            "effective_flop_per_step_per_gpu": eff,
+            "effective_flop_per_step_per_gpu": eff_job / ws,
             # the dominant kernel: attention_tc_kernel alone (exact blocks and cluster columns in one
             # online softmax, on compensation values built by the pre-pass); frac_incl_compensation
             # counts the pre-pass kernel's time too, frac_step the whole step (reassign included)

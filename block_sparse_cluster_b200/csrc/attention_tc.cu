@@ -510,7 +510,16 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         ++u;
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&bars->p_ready[X]);
+#ifdef DA_FAULT_INJECT
+        // Test build only (libda_fault.so): the second softmax warpgroup of CTA 0 withholds its
+        // P-ready arrival at step 5, a plain software arrival (no copy or product is left in
+        // flight).  The MMA issuer's bounded wait for it gives up, records DA_ERR_TIMEOUT and makes
+        // every role of the CTA leave; the producers drain their copies first.
+        const bool withhold = blockIdx.x == 0 && g == 5;
+#else
+        constexpr bool withhold = false;
+#endif
+        if (!withhold) mbar_arrive(&bars->p_ready[X]);
       }
       if (!ok) break;
       // epilogue: once this warpgroup's last product has landed, exchange (max, sum) per row with

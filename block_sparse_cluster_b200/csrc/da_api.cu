@@ -1,6 +1,7 @@
 // C ABI of libda.so: argument checks, workspace layout and kernel launches.
 // Every check happens before the first launch, so a call that returns an error launched nothing.
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 #include <stdint.h>
 
 #include "da.h"
@@ -60,6 +61,14 @@ da_status check_stats(const da_cluster_stats* st, StatsPtrs* p) {
 
 namespace {
 
+// An NVTX range around the host side of a call (argument checks and launches), named after the
+// call, so that a profiler's timeline groups each call's kernels; header-only NVTX costs next to
+// nothing without a profiler attached.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+};
+
 da_status check_ws(const Dims& g, void* ws, size_t ws_bytes) {
   if (!ws) return DA_ERR_INVALID_ARG;
   if (!aligned16(ws)) return DA_ERR_ALIGNMENT;
@@ -98,6 +107,7 @@ size_t da_schedule_bytes(const da_dims* dims) {
 
 da_status da_reassign(const da_dims* dims, const void* K, const void* V, const void* centroids,
                       const da_cluster_stats* out, void* ws, size_t ws_bytes, da_stream stream) {
+  NvtxRange nvtx("da_reassign");
   Dims g;
   da_status st = check_dims(dims, &g);
   if (st != DA_OK) return st;
@@ -125,6 +135,7 @@ da_status da_reassign(const da_dims* dims, const void* K, const void* V, const v
 
 da_status da_mask_prepare(const da_dims* dims, const da_block_mask* mask, int32_t* schedule,
                           size_t schedule_bytes, void* ws, size_t ws_bytes, da_stream stream) {
+  NvtxRange nvtx("da_mask_prepare");
   Dims g;
   da_status st = check_dims(dims, &g);
   if (st != DA_OK) return st;
@@ -194,6 +205,7 @@ static da_status attention_launch(const Dims& g, const void* Q, const void* K, c
 
 da_status da_compensation(const da_dims* dims, const da_block_mask* mask, const da_cluster_stats* stats, void* ws,
                           size_t ws_bytes, da_stream stream) {
+  NvtxRange nvtx("da_compensation");
   Dims g;
   StatsPtrs sp;
   da_status st = attention_common(dims, mask, stats, ws, ws_bytes, &g, &sp);
@@ -204,6 +216,7 @@ da_status da_compensation(const da_dims* dims, const da_block_mask* mask, const 
 da_status da_attention_prebuilt(const da_dims* dims, const void* Q, const void* K, const void* V,
                                 const da_block_mask* mask, const void* centroids, const da_cluster_stats* stats,
                                 float scale, void* O, float* lse, void* ws, size_t ws_bytes, da_stream stream) {
+  NvtxRange nvtx("da_attention_prebuilt");
   Dims g;
   StatsPtrs sp;
   da_status st = attention_common(dims, mask, stats, ws, ws_bytes, &g, &sp);
@@ -214,6 +227,7 @@ da_status da_attention_prebuilt(const da_dims* dims, const void* Q, const void* 
 da_status da_attention(const da_dims* dims, const void* Q, const void* K, const void* V,
                        const da_block_mask* mask, const void* centroids, const da_cluster_stats* stats,
                        float scale, void* O, float* lse, void* ws, size_t ws_bytes, da_stream stream) {
+  NvtxRange nvtx("da_attention");
   Dims g;
   StatsPtrs sp;
   da_status st = attention_common(dims, mask, stats, ws, ws_bytes, &g, &sp);
@@ -227,6 +241,7 @@ da_status da_attention(const da_dims* dims, const void* Q, const void* K, const 
 
 da_status da_centroid_update(const da_dims* dims, const da_cluster_stats* stats, void* centroids,
                              da_stream stream) {
+  NvtxRange nvtx("da_centroid_update");
   Dims g;
   da_status st = check_dims(dims, &g);
   if (st != DA_OK) return st;
@@ -239,6 +254,7 @@ da_status da_centroid_update(const da_dims* dims, const da_cluster_stats* stats,
 
 da_status da_cluster_spread(const da_dims* dims, const void* K, const void* centroids, const da_cluster_stats* stats,
                             float* spread, da_stream stream) {
+  NvtxRange nvtx("da_cluster_spread");
   Dims g;
   da_status st = check_dims(dims, &g);
   if (st != DA_OK) return st;
@@ -253,6 +269,7 @@ da_status da_attention_spread(const da_dims* dims, const void* Q, const void* K,
                               const da_block_mask* mask, const void* centroids, const da_cluster_stats* stats,
                               const float* spread, float scale, void* O, float* lse, void* ws, size_t ws_bytes,
                               da_stream stream) {
+  NvtxRange nvtx("da_attention_spread");
   Dims g;
   StatsPtrs sp;
   da_status st = attention_common(dims, mask, stats, ws, ws_bytes, &g, &sp);
@@ -281,6 +298,7 @@ da_status da_attention_spread(const da_dims* dims, const void* Q, const void* K,
 da_status da_attention_sip(const da_dims* dims, const void* Q, const void* K, const void* V,
                            const da_block_mask* mask, const float* incl, float scale, void* O, float* lse, void* ws,
                            size_t ws_bytes, da_stream stream) {
+  NvtxRange nvtx("da_attention_sip");
   Dims g;
   da_status st = check_dims(dims, &g);
   if (st != DA_OK) return st;

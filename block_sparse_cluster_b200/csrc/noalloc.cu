@@ -13,6 +13,7 @@
 // contents; the status word is cleared at the start of each call, the norms are rewritten in
 // full.  Calls whose kernels overlap on the GPU (for instance on two streams) race on it.
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <mutex>
 
@@ -52,9 +53,21 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 }  // namespace
 
+static da_status reassign_noalloc(const da_dims* dims, const void* K, const void* V, const void* centroids,
+                                  const da_cluster_stats* out, da_stream stream);
+
 extern "C" DA_API da_status da_reassign_noalloc(const da_dims* dims, const void* K, const void* V,
                                                 const void* centroids, const da_cluster_stats* out,
                                                 da_stream stream) {
+  using namespace da;
+  nvtxRangePushA("da_reassign_noalloc");
+  const da_status st = reassign_noalloc(dims, K, V, centroids, out, stream);
+  nvtxRangePop();
+  return st;
+}
+
+static da_status reassign_noalloc(const da_dims* dims, const void* K, const void* V, const void* centroids,
+                                  const da_cluster_stats* out, da_stream stream) {
   using namespace da;
   // the same argument checks as da_reassign, then the size of the built-in scratch
   Dims g;

@@ -57,3 +57,45 @@ def test_reference_arm_under_torchrun_prints_once():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
+
+
+def _split_worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    sys.path.insert(0, ROOT)
+    import bench
+    import workloads as W
+    ws, r, _ = bench._dist()
+    w = W.scaled(W.WORKLOADS["tiny"], H=5)                 # five heads over two ranks: 3 + 2
+    heads = bench.head_slice(w.H, r, ws)
+    inp = W.make_inputs(w, seed=3, heads=heads)
+    eff = W.effective_flops(inp.w, inp.kv_cnt, inp.kv_idx)
+    total = bench._sum_over_ranks(eff, ws, "cpu")
+    q.put((r, list(heads), eff, total, inp.K.sum().item(), inp.kv_cnt.sum().item()))
+    torch.distributed.destroy_process_group()
+
+
+def test_split_heads_partition_the_workload_with_gloo():
+    """--split-heads: the ranks' head slices partition the heads, each slice holds exactly those
+    heads of the full workload, and the job's effective FLOPs (summed over ranks) are the full
+    workload's."""
+    sys.path.insert(0, ROOT)
+    import workloads as W
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_split_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=180)
+        assert p.exitcode == 0
+    got = sorted(q.get(timeout=5) for _ in range(2))
+    assert got[0][1] == [0, 1, 2] and got[1][1] == [3, 4]
+    w = W.scaled(W.WORKLOADS["tiny"], H=5)
+    full = W.make_inputs(w, seed=3)
+    assert abs(got[0][3] - W.effective_flops(w, full.kv_cnt, full.kv_idx)) < 1e-6 * got[0][3]
+    assert got[0][3] == got[1][3] == got[0][2] + got[1][2]
+    for r, heads, _, _, ksum, cnt in got:
+        assert abs(ksum - full.K[:, heads].sum().item()) < 1e-3 * max(1.0, abs(ksum))
+        assert cnt == full.kv_cnt[:, heads].sum().item()

@@ -221,9 +221,12 @@ class Inputs:
     plans: list = field(default_factory=list)   # [B][H] lists of row arrays
 
 
-def make_inputs(w: Workload, seed: int = 0, step: int = 0) -> Inputs:
-    """Full inputs of a workload on the CPU."""
-    B, H, N, d, C = w.B, w.H, w.N, w.d, w.C
+def make_inputs(w: Workload, seed: int = 0, step: int = 0, heads: Optional[Sequence[int]] = None) -> Inputs:
+    """Inputs of a workload on the CPU: every head, or the given heads (global indices, so that a
+    slice holds exactly the same tensors as those heads of the full workload).  The returned
+    Inputs' workload has H = the number of heads returned."""
+    heads = list(range(w.H)) if heads is None else [int(h) for h in heads]
+    B, H, N, d, C = w.B, len(heads), w.N, w.d, w.C
     dt = w.torch_dtype
     Q = torch.empty(B, H, N, d, dtype=dt)
     K = torch.empty_like(Q)
@@ -232,13 +235,13 @@ def make_inputs(w: Workload, seed: int = 0, step: int = 0) -> Inputs:
     plans = []
     for b in range(B):
         hp = []
-        for h in range(H):
+        for i, h in enumerate(heads):
             q, k, v, mu = head_qkv(w, seed, b, h, step)
-            Q[b, h], K[b, h], V[b, h], cent[b, h] = q, k, v, mu
+            Q[b, i], K[b, i], V[b, i], cent[b, i] = q, k, v, mu
             hp.append(head_plan(w, seed, b, h))
         plans.append(hp)
     kv_idx, kv_cnt = pack_plan(plans, w.nB)
-    return Inputs(w, seed, Q, K, V, cent, kv_idx, kv_cnt, plans)
+    return Inputs(replace(w, H=H), seed, Q, K, V, cent, kv_idx, kv_cnt, plans)
 
 
 def effective_flops(w: Workload, kv_cnt: torch.Tensor, kv_idx: torch.Tensor) -> float:
