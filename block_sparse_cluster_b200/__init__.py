@@ -29,7 +29,7 @@ STATUS_NAMES = ["DA_OK", "DA_ERR_INVALID_ARG", "DA_ERR_SHAPE", "DA_ERR_DTYPE", "
 EXPORTS = ["da_version", "da_workspace_bytes", "da_schedule_bytes", "da_reassign", "da_mask_prepare",
            "da_attention", "da_device_status", "da_status_string", "da_reassign_noalloc", "da_compensation",
            "da_attention_prebuilt", "da_centroid_update", "da_cluster_spread", "da_attention_spread",
-           "da_attention_sip"]
+           "da_attention_sip", "da_noalloc_device_status"]
 
 
 class DAError(RuntimeError):
@@ -85,6 +85,8 @@ _lib.da_attention_sip.argtypes = [ctypes.POINTER(_Dims), _P, _P, _P, ctypes.POIN
                                   _P, _P, ctypes.c_size_t, _P]
 _lib.da_reassign_noalloc.restype = ctypes.c_int
 _lib.da_reassign_noalloc.argtypes = [ctypes.POINTER(_Dims), _P, _P, _P, ctypes.POINTER(_Stats), _P]
+_lib.da_noalloc_device_status.restype = ctypes.c_int
+_lib.da_noalloc_device_status.argtypes = [_P]
 _lib.da_device_status.restype = ctypes.c_int
 _lib.da_device_status.argtypes = [_P, _P]
 _lib.da_status_string.restype = ctypes.c_char_p
@@ -293,6 +295,11 @@ def kmeans(dims: Dims, K: torch.Tensor, centroids: torch.Tensor, iters: int, sta
 def da_device_status(ws: torch.Tensor, stream=None) -> int:
     """Synchronise and return (and clear) the device status word as a status code."""
     return _lib.da_device_status(ws.data_ptr(), _stream(stream))
+
+
+def da_noalloc_device_status(stream=None) -> int:
+    """Synchronise and return (and clear) the status word of da_reassign_noalloc's scratch."""
+    return _lib.da_noalloc_device_status(_stream(stream))
 
 
 class DecoupledAttention:

@@ -21,6 +21,14 @@
 // masked step if it has none), and block j's logits carry the bias -log2 pi_j, i.e. the weight
 // 1 / pi_j in both sums of the softmax; no cluster columns.
 //
+// Variance-corrected mode (kSpread; ESTRA abstract, second-order correction of the cluster
+// logits): a cluster column's logit gains s^2/2 sum_t q_t^2 D_{c,t}, D_c the second moment of the
+// cluster's keys about its representative.  The correction is a second contraction into the same
+// score tile: S = Q cbar^T + Q2 Dh^T, with Q2 = q o q (bf16, written into shared memory from the
+// query tile by warp 11) and Dh = (s/2) D (bf16, from the host side).  A chunk step therefore takes
+// two key-ring tiles (the centroid chunk, then the Dh chunk), so the key ring counts tiles, not
+// steps; the query tile Q2 takes the place of one value-ring slot (two slots in this mode).
+//
 // Roles (384 threads):
 //   warps 0-3, 4-7  two softmax warpgroups X = 0, 1; warpgroup X takes the steps g with g & 1 = X
 //              of every item, so the two overlap each other and the tensor core.  Thread t of a
@@ -34,7 +42,8 @@
 //   warp 9     MMA: allocates TMEM, issues tcgen05.mma S(g+1) = Q K^T ahead of O_X += P(g) V(g);
 //   warp 10    producer of value tiles / compensation chunks (2-stage ring); a warp of its own,
 //              since divergent lanes of one warp waiting on different barriers hold each other up;
-//   warp 11    idle (it completes the third warpgroup, whose registers go to the softmax).
+//   warp 11    idle (it completes the third warpgroup, whose registers go to the softmax); in the
+//              variance-corrected mode it writes Q2 for each item once the query tile has landed.
 // TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,384), O_1 [384,512).
 //
 // Every mbarrier is waited at every phase, in order, by each role that waits on it (a parity
@@ -61,6 +70,7 @@ constexpr int kThreads = 384;           // three warpgroups; warp 11 idle
 constexpr int kWarpProducer = 8;
 constexpr int kWarpMMA = 9;
 constexpr int kWarpProducerV = 10;
+constexpr int kWarpQ2 = 11;
 // Register split (setmaxnreg): the launch holds 384 x 168 registers; the softmax warpgroups grow,
 // the producer / MMA warpgroup shrinks.
 constexpr int kRegSoftmax = 232, kRegIssue = 40;
@@ -69,7 +79,7 @@ static_assert(kBStages % 2 == 0, "a bias slot must always serve the same softmax
 constexpr int kChunkBytes = kTile + kBN * 4;   // compensation chunk: vbar^U rows, then log2 n^U
 
 struct __align__(8) Bars {
-  uint64_t q_full, q_empty;
+  uint64_t q_full, q_empty, q2_full;
   uint64_t k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
   uint64_t b_full[kBStages], b_empty[kBStages];
   uint64_t s_full[2], p_ready[2];
@@ -84,6 +94,7 @@ struct __align__(8) Bars {
   float2 xch[2][2][kBM];                 // [item parity][warpgroup][row] = (max, sum)
 };
 
+// (the variance-corrected mode holds Q2 in place of one value-ring slot: the same size)
 constexpr size_t kSmemBytes = 1024 + kTile /*Q*/ + (kKStages + kVStages) * kTile /*K,V*/ +
                               kBStages * kBN * sizeof(float) /*bias*/ + sizeof(Bars);
 static_assert(kSmemBytes <= 232448, "shared memory above the 227 KB per-block limit");
@@ -107,6 +118,13 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// q o q for a pair of bf16 values: each square rounded once to bf16.
+__device__ __forceinline__ uint32_t square_bf16x2(uint32_t w) {
+  __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162*>(&w);
+  h = __hmul2(h, h);
+  return *reinterpret_cast<const uint32_t*>(&h);
 }
 
 // Item geometry shared by every role.
@@ -207,17 +225,23 @@ __device__ __forceinline__ void chunk_exp(const uint32_t (&x)[32], uint64_t coef
   rsum = f2_add(rsum, f2_add(s0, s1));
 }
 
+// kSpread: the variance-corrected mode (tm_d maps Dh = (s/2) D, [B*H][C][d] bf16); otherwise tm_d
+// is unused.
+template <bool kSpread>
 __global__ void __launch_bounds__(kThreads, 1)
 attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_c,
-                    const __grid_constant__ CUtensorMap tm_p, const Params p) {
+                    const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_d,
+                    const Params p) {
+  constexpr int kVSt = kSpread ? kVStages - 1 : kVStages;   // value-ring slots
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   uint8_t* sQ = base;
-  uint8_t* sK = sQ + kTile;                       // kKStages tiles
-  uint8_t* sV = sK + kKStages * kTile;            // kVStages tiles
-  float* sBias = reinterpret_cast<float*>(sV + kVStages * kTile);   // [kBStages][kBN]
+  uint8_t* sQ2 = sQ + kTile;                      // variance-corrected mode only
+  uint8_t* sK = sQ + (kSpread ? 2 : 1) * kTile;   // kKStages tiles
+  uint8_t* sV = sK + kKStages * kTile;            // kVSt tiles
+  float* sBias = reinterpret_cast<float*>(sV + kVSt * kTile);   // [kBStages][kBN]
   Bars* bars = reinterpret_cast<Bars*>(sBias + kBStages * kBN);
 
   const int tid = threadIdx.x;
@@ -226,11 +250,12 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   if (tid == 0) {
     mbar_init(&bars->q_full, 1);
     mbar_init(&bars->q_empty, 1);
+    mbar_init(&bars->q2_full, 1);
     for (int s = 0; s < kKStages; ++s) {
       mbar_init(&bars->k_full[s], 1);
       mbar_init(&bars->k_empty[s], 1);
     }
-    for (int s = 0; s < kVStages; ++s) {
+    for (int s = 0; s < kVSt; ++s) {
       mbar_init(&bars->v_full[s], 1);
       mbar_init(&bars->v_empty[s], 1);
     }
@@ -271,7 +296,10 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       tma_prefetch(&tm_q);
       tma_prefetch(&tm_k);
       tma_prefetch(&tm_c);
+      if (kSpread) tma_prefetch(&tm_d);
       uint32_t g = 0;
+      uint32_t kt = 0;                   // key-ring tiles loaded (one per step; two per chunk step
+                                         // in the variance-corrected mode)
       int n = 0, nq = 0;                 // items walked, query tiles loaded
       for (int k = blockIdx.x; k < p.n_items && !*abort; k += gridDim.x, ++n) {
         const Item it = item_at(p, k);
@@ -282,9 +310,11 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         tma_load_3d(sQ + kPanel, &tm_q, &bars->q_full, 64, it.q0, it.bh);
         bool ok = true;
         for (int s = 0; s < it.T; ++s, ++g) {
-          const int ks = g % kKStages, bs = g % kBStages;
-          if (!mbar_wait(&bars->k_empty[ks], ((g / kKStages) & 1) ^ 1, abort, status)) { ok = false; break; }
+          if (!kSpread) kt = g;          // one tile per step
+          const int ks = kt % kKStages, bs = g % kBStages;
+          if (!mbar_wait(&bars->k_empty[ks], ((kt / kKStages) & 1) ^ 1, abort, status)) { ok = false; break; }
           uint8_t* dk = sK + ks * kTile;
+          ++kt;
           if (s < it.nsel || p.incl) {
             bool valid;
             const int j = block_of(p, it, s, &valid);
@@ -315,6 +345,16 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             mbar_expect_tx(&bars->k_full[ks], kTile);
             tma_load_3d(dk, &tm_c, &bars->k_full[ks], 0, c * kBN, it.bh);
             tma_load_3d(dk + kPanel, &tm_c, &bars->k_full[ks], 64, c * kBN, it.bh);
+            if (kSpread) {
+              // the chunk's rows of Dh, into the next key-ring slot
+              const int kd = kt % kKStages;
+              if (!mbar_wait(&bars->k_empty[kd], ((kt / kKStages) & 1) ^ 1, abort, status)) { ok = false; break; }
+              uint8_t* dd = sK + kd * kTile;
+              ++kt;
+              mbar_expect_tx(&bars->k_full[kd], kTile);
+              tma_load_3d(dd, &tm_d, &bars->k_full[kd], 0, c * kBN, it.bh);
+              tma_load_3d(dd + kPanel, &tm_d, &bars->k_full[kd], 64, c * kBN, it.bh);
+            }
             if (!mbar_wait(&bars->b_empty[bs], ((g / kBStages) & 1) ^ 1, abort, status)) { ok = false; break; }
             bars->bflag[bs] = 0;
             mbar_expect_tx(&bars->b_full[bs], kBN * 4);
@@ -326,7 +366,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       // no copy may still be in flight when the CTA leaves (this matters only after an abort:
       // otherwise the consumers have waited for every load)
       if (nq > 0) mbar_wait_drain(&bars->q_full, (nq - 1) & 1);
-      for (uint32_t gd = g >= kKStages ? g - kKStages : 0; gd < g; ++gd)
+      for (uint32_t gd = kt >= kKStages ? kt - kKStages : 0; gd < kt; ++gd)
         mbar_wait_drain(&bars->k_full[gd % kKStages], (gd / kKStages) & 1);
       for (uint32_t gd = g >= kBStages ? g - kBStages : 0; gd < g; ++gd)
         mbar_wait_drain(&bars->b_full[gd % kBStages], (gd / kBStages) & 1);
@@ -342,8 +382,8 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const Item it = item_at(p, k);
         bool ok = true;
         for (int s = 0; s < it.T; ++s, ++g) {
-          const int vs = g % kVStages;
-          if (!mbar_wait(&bars->v_empty[vs], ((g / kVStages) & 1) ^ 1, abort, status)) { ok = false; break; }
+          const int vs = g % kVSt;
+          if (!mbar_wait(&bars->v_empty[vs], ((g / kVSt) & 1) ^ 1, abort, status)) { ok = false; break; }
           uint8_t* dv = sV + vs * kTile;
           if (s < it.nsel || p.incl) {
             bool valid;
@@ -360,8 +400,8 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
         if (!ok) break;
       }
-      for (uint32_t gd = g >= kVStages ? g - kVStages : 0; gd < g; ++gd)
-        mbar_wait_drain(&bars->v_full[gd % kVStages], (gd / kVStages) & 1);
+      for (uint32_t gd = g >= kVSt ? g - kVSt : 0; gd < g; ++gd)
+        mbar_wait_drain(&bars->v_full[gd % kVSt], (gd / kVSt) & 1);
     }
   } else if (warp == kWarpMMA) {
     // ------------------------------------------------------------------ MMA issuer
@@ -370,40 +410,59 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       const uint32_t idesc_pv = idesc_bf16(kBM, kD, 0, 1);    // P from TMEM, V MN-major
       const uint32_t q0 = smem_u32(sQ);
       uint32_t g = 0;
+      uint32_t kt = 0;                   // key-ring tiles consumed
       int n = 0;
-      auto issue_s = [&](uint32_t gs) {
-        const int ks = gs % kKStages;
-        const uint32_t kb = smem_u32(sK + ks * kTile);
+      // S(gs) of step s of item `it` (the n-th of this CTA): waits for its key-ring tile(s) (and,
+      // at the item's first chunk step in the variance-corrected mode, for Q2), issues the product
+      // and frees the tile(s) when it completes.
+      auto issue_s = [&](uint32_t gs, const Item& it, int s) -> bool {
+        const bool two = kSpread && !p.incl && s >= it.nsel;
+        const uint32_t t0 = kSpread ? kt : gs;   // one tile per step outside the corrected mode
+        if (!mbar_wait(&bars->k_full[t0 % kKStages], (t0 / kKStages) & 1, abort, status)) return false;
+        if (two) {
+          const uint32_t t1 = t0 + 1;
+          if (!mbar_wait(&bars->k_full[t1 % kKStages], (t1 / kKStages) & 1, abort, status)) return false;
+          if (s == it.nsel && !mbar_wait(&bars->q2_full, n & 1, abort, status)) return false;
+        }
+        tc_fence_after();
+        const uint32_t kb = smem_u32(sK + (t0 % kKStages) * kTile);
         const uint32_t d = tmem + (gs & 1) * kBN;
 #pragma unroll
         for (int ks = 0; ks < kD / 16; ++ks) {
           const uint32_t off = (ks >> 2) * kPanel + (ks & 3) * 32;
           umma_ss(d, sdesc_sw128(q0 + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), idesc_qk, ks > 0);
         }
+        if (two) {
+          // + Q2 Dh^T: the correction of the cluster logits, into the same accumulator
+          const uint32_t q2 = smem_u32(sQ2);
+          const uint32_t db = smem_u32(sK + ((t0 + 1) % kKStages) * kTile);
+#pragma unroll 1
+          for (int ks = 0; ks < kD / 16; ++ks) {
+            const uint32_t off = (ks >> 2) * kPanel + (ks & 3) * 32;
+            umma_ss(d, sdesc_sw128(q2 + off, 16, 1024), sdesc_sw128(db + off, 16, 1024), idesc_qk, 1u);
+          }
+        }
         umma_commit(&bars->s_full[gs & 1]);
-        umma_commit(&bars->k_empty[ks]);
+        umma_commit(&bars->k_empty[t0 % kKStages]);
+        if (two) umma_commit(&bars->k_empty[(t0 + 1) % kKStages]);
+        if (kSpread) kt = t0 + (two ? 2u : 1u);
+        return true;
       };
       bool ok = true;
       for (int k = blockIdx.x; k < p.n_items && ok; k += gridDim.x, ++n) {
         const Item it = item_at(p, k);
         if (!mbar_wait(&bars->q_full, n & 1, abort, status)) break;
         tc_fence_after();
-        const uint32_t g0 = g;
-        if (!mbar_wait(&bars->k_full[g0 % kKStages], (g0 / kKStages) & 1, abort, status)) break;
-        tc_fence_after();
-        issue_s(g0);
+        if (!issue_s(g, it, 0)) break;
         for (int s = 0; s < it.T; ++s, ++g) {
           if (s + 1 < it.T) {
-            const uint32_t gn = g + 1;
-            if (!mbar_wait(&bars->k_full[gn % kKStages], (gn / kKStages) & 1, abort, status)) { ok = false; break; }
-            tc_fence_after();
-            issue_s(gn);
+            if (!issue_s(g + 1, it, s + 1)) { ok = false; break; }
           } else {
             umma_commit(&bars->q_empty);
           }
-          const int vs = g % kVStages;
+          const int vs = g % kVSt;
           if (!mbar_wait(&bars->p_ready[g & 1], (g >> 1) & 1, abort, status)) { ok = false; break; }
-          if (!mbar_wait(&bars->v_full[vs], (g / kVStages) & 1, abort, status)) { ok = false; break; }
+          if (!mbar_wait(&bars->v_full[vs], (g / kVSt) & 1, abort, status)) { ok = false; break; }
           if (s == 0 && !mbar_wait(&bars->o_free, (n & 1) ^ 1, abort, status)) { ok = false; break; }
           tc_fence_after();
           const uint32_t vb = smem_u32(sV + vs * kTile);
@@ -422,6 +481,32 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       }
       umma_commit(&bars->drain);
       mbar_wait_drain(&bars->drain, 0);
+    }
+  } else if (kSpread && warp == kWarpQ2) {
+    // ------------------------------------------------------------------ Q2 writer (warp 11)
+    // Once query tile n has landed, Q2 = q o q in the same swizzled layout (the square is taken
+    // elementwise, so the 128-byte swizzle carries over), published to the tensor core by a proxy
+    // fence and an arrival on q2_full.  The MMA waits for it at the item's first chunk step; the
+    // query tile of item n + 1 is loaded only after every product of item n (so every read of Q2)
+    // has completed, so Q2 is free when q_full announces the next tile.
+    int n = 0;
+    for (int k = blockIdx.x; k < p.n_items; k += gridDim.x, ++n) {
+      const bool w_ok = mbar_wait(&bars->q_full, n & 1, abort, status);
+      if (!__all_sync(0xffffffffu, w_ok)) break;
+      const uint4* src = reinterpret_cast<const uint4*>(sQ);
+      uint4* dst = reinterpret_cast<uint4*>(sQ2);
+#pragma unroll 1
+      for (int i = lane; i < kTile / 16; i += 32) {
+        uint4 v = src[i];
+        v.x = square_bf16x2(v.x);
+        v.y = square_bf16x2(v.y);
+        v.z = square_bf16x2(v.z);
+        v.w = square_bf16x2(v.w);
+        dst[i] = v;
+      }
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->q2_full);
     }
   } else if (warp < 8) {
     // ------------------------------------------------------------------ softmax (warps 0-7)
@@ -593,14 +678,18 @@ size_t attention_tc_scratch_bytes(const Dims& g) {
 cudaError_t launch_attention_tc(const Dims& g, const void* Q, const void* K, const void* V,
                                 const int32_t* kv_idx, const int32_t* kv_cnt, int max_sel,
                                 const int32_t* schedule, const void* cent, const StatsPtrs& st, float scale,
-                                void* O, float* lse, int* status, void* comp, const float* incl, cudaStream_t s) {
-  CUtensorMap tq, tk, tv, tc, tp;
+                                void* O, float* lse, int* status, void* comp, const float* incl,
+                                const void* spread_half, cudaStream_t s) {
+  if (spread_half && incl) return cudaErrorInvalidValue;   // the two modes do not combine
+  CUtensorMap tq, tk, tv, tc, tp, td;
   const unsigned long long BH = (unsigned long long)g.B * g.H;
   const int nchunk = (g.C + kBN - 1) / kBN;
   if (!make_tmap_bf16_3d(&tq, Q, kD, g.N, BH, 64, kBM) || !make_tmap_bf16_3d(&tk, K, kD, g.N, BH, 64, kBN) ||
       !make_tmap_bf16_3d(&tv, V, kD, g.N, BH, 64, kBN) || !make_tmap_bf16_3d(&tc, cent, kD, g.C, BH, 64, kBN) ||
       !make_tmap_bf16_tiles(&tp, comp, kD, kBN, BH * g.nB * nchunk, kChunkBytes, kBN))
     return cudaErrorInvalidValue;
+  td = tc;                                                   // unused unless spread_half is given
+  if (spread_half && !make_tmap_bf16_3d(&td, spread_half, kD, g.C, BH, 64, kBN)) return cudaErrorInvalidValue;
   Params p;
   p.kv_idx = kv_idx;
   p.kv_cnt = kv_cnt;
@@ -621,11 +710,11 @@ cudaError_t launch_attention_tc(const Dims& g, const void* Q, const void* K, con
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  cudaError_t e = cudaFuncSetAttribute(attention_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)kSmemBytes);
+  auto kernel = spread_half ? attention_tc_kernel<true> : attention_tc_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   const int grid = min(sms, p.n_items);
-  attention_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, tc, tp, p);
+  kernel<<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, tc, tp, td, p);
   return cudaGetLastError();
 }
 

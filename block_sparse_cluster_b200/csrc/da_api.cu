@@ -194,7 +194,7 @@ static da_status attention_launch(const Dims& g, const void* Q, const void* K, c
   if (e == cudaSuccess) {
     if (attention_tc_supported(g))
       e = launch_attention_tc(g, Q, K, V, mask->kv_idx, mask->kv_cnt, mask->max_sel, sched, centroids, sp, scale, O,
-                              lse, status, static_cast<char*>(ws) + L.comp, nullptr, s);
+                              lse, status, static_cast<char*>(ws) + L.comp, nullptr, nullptr, s);
     else
       e = (g.bf16 ? launch_attention_simt_bf16 : launch_attention_simt_f32)(
           g, Q, K, V, mask->kv_idx, mask->kv_cnt, mask->max_sel, sched, centroids, sp, nullptr, scale, O, lse, status,
@@ -288,10 +288,20 @@ da_status da_attention_spread(const da_dims* dims, const void* Q, const void* K,
     e = launch_schedule(g, mask->kv_idx, mask->kv_cnt, mask->max_sel, own, status, s);
     sched = own;
   }
-  if (e == cudaSuccess)
+  if (e == cudaSuccess && attention_tc_supported(g)) {
+    // tensor cores: the compensation pre-pass, Dh = (s/2) D in bf16, then the fused kernel in its
+    // variance-corrected mode
+    void* dh = static_cast<char*>(ws) + L.spread;
+    e = launch_comp_build(g, mask->kv_idx, mask->kv_cnt, mask->max_sel, sp, static_cast<char*>(ws) + L.comp, s);
+    if (e == cudaSuccess) e = launch_spread_half(g, spread, scale, dh, s);
+    if (e == cudaSuccess)
+      e = launch_attention_tc(g, Q, K, V, mask->kv_idx, mask->kv_cnt, mask->max_sel, sched, centroids, sp, scale, O,
+                              lse, status, static_cast<char*>(ws) + L.comp, nullptr, dh, s);
+  } else if (e == cudaSuccess) {
     e = (g.bf16 ? launch_attention_simt_bf16 : launch_attention_simt_f32)(
         g, Q, K, V, mask->kv_idx, mask->kv_cnt, mask->max_sel, sched, centroids, sp, spread, scale, O, lse, status,
         s);
+  }
   return cuda_status(e);
 }
 
@@ -322,7 +332,7 @@ da_status da_attention_sip(const da_dims* dims, const void* Q, const void* K, co
   // no cluster steps: the centroid map is never read (K stands in for it), nor are the statistics
   if (e == cudaSuccess)
     e = launch_attention_tc(g, Q, K, V, mask->kv_idx, mask->kv_cnt, mask->max_sel, sched, K, StatsPtrs{}, scale, O,
-                            lse, status, static_cast<char*>(ws) + L.comp, incl, s);
+                            lse, status, static_cast<char*>(ws) + L.comp, incl, nullptr, s);
   return cuda_status(e);
 }
 

@@ -32,7 +32,7 @@ da_status check_stats(const da_cluster_stats* st, StatsPtrs* p);
 
 // Workspace layout (byte offsets), shared by every call.
 struct WsLayout {
-  size_t status, norms, sched, comp, total;
+  size_t status, norms, sched, comp, spread, total;
 };
 WsLayout ws_layout(const Dims& g);
 
@@ -45,6 +45,9 @@ cudaError_t launch_cluster_spread(const Dims& g, const void* K, const void* cent
                                   cudaStream_t s);
 cudaError_t launch_schedule(const Dims& g, const int32_t* kv_idx, const int32_t* kv_cnt, int max_sel,
                             int32_t* schedule, int* status, cudaStream_t s);
+// Dh = (scale / 2) D in bf16, the second operand of the variance-corrected cluster logits on the
+// tensor cores ([B*H][C][d], from the fp32 second moments D).
+cudaError_t launch_spread_half(const Dims& g, const float* spread, float scale, void* out, cudaStream_t s);
 
 // reassign_tc.cu
 bool reassign_tc_supported(const Dims& g);
@@ -58,7 +61,7 @@ cudaError_t launch_attention_tc(const Dims& g, const void* Q, const void* K, con
                                 const int32_t* kv_idx, const int32_t* kv_cnt, int max_sel,
                                 const int32_t* schedule, const void* cent, const StatsPtrs& st, float scale,
                                 void* O, float* lse, int* status, void* comp, const float* incl,
-                                cudaStream_t s);
+                                const void* spread_half, cudaStream_t s);
 
 // comp_build.cu
 cudaError_t launch_comp_build(const Dims& g, const int32_t* kv_idx, const int32_t* kv_cnt, int max_sel,

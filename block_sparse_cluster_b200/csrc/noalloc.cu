@@ -15,8 +15,6 @@
 #include <cuda_runtime.h>
 #include <nvtx3/nvToolsExt.h>
 
-#include <mutex>
-
 #include "da.h"
 #include "da_internal.h"
 
@@ -29,23 +27,16 @@ static __device__ __align__(256) float g_noalloc_scratch[kStatusFloats + kNoAllo
 
 namespace {
 
-// Device address of g_noalloc_scratch per device.  In host code the symbol's name is a host-side
-// stand-in, not a device address: the address comes from cudaGetSymbolAddress, taken once per
-// device with that device current (the first call on a device does it).
-constexpr int kMaxDevices = 64;
-std::mutex g_lock;
-float* g_addr[kMaxDevices] = {};
-
-cudaError_t scratch_address(int dev, float** out) {
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> guard(g_lock);
-  if (!g_addr[dev]) {
-    void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess) return e;
-    g_addr[dev] = static_cast<float*>(p);
-  }
-  *out = g_addr[dev];
+// Device address of g_noalloc_scratch on the current device.  In host code the symbol's name is a
+// host-side stand-in, not a device address: the address comes from cudaGetSymbolAddress with the
+// device current.  It is looked up on every call, not cached, so that a context that was torn down
+// and made again (cudaDeviceReset) never leaves a stale address behind; after the first call on a
+// device, which loads the library's module there, the lookup is a table read.
+cudaError_t scratch_address(float** out) {
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+  if (e != cudaSuccess) return e;
+  *out = static_cast<float*>(p);
   return cudaSuccess;
 }
 
@@ -78,10 +69,8 @@ static da_status reassign_noalloc(const da_dims* dims, const void* K, const void
   StatsPtrs sp;
   if ((st = check_stats(out, &sp)) != DA_OK) return st;
   if ((size_t)g.B * g.H * g.C > kNoAllocMaxNorms) return DA_ERR_WORKSPACE;   // beyond the built-in scratch
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return DA_ERR_CUDA;
   float* scratch = nullptr;
-  if (scratch_address(dev, &scratch) != cudaSuccess) return DA_ERR_CUDA;
+  if (scratch_address(&scratch) != cudaSuccess) return DA_ERR_CUDA;
   int* status = reinterpret_cast<int*>(scratch);
   float* norms = scratch + kStatusFloats;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -98,4 +87,23 @@ static da_status reassign_noalloc(const da_dims* dims, const void* K, const void
   }
   if (e == cudaSuccess) e = launch_totals(g, sp, s);
   return e == cudaSuccess ? DA_OK : DA_ERR_CUDA;
+}
+
+// The status word of the built-in scratch on the current device: synchronise `stream`, read the
+// word, clear it.  The same codes as da_device_status.
+extern "C" DA_API da_status da_noalloc_device_status(da_stream stream) {
+  float* scratch = nullptr;
+  if (scratch_address(&scratch) != cudaSuccess) return DA_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int word = 0;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return DA_ERR_CUDA;
+  if (cudaMemcpyAsync(&word, scratch, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess) return DA_ERR_CUDA;
+  if (cudaMemsetAsync(scratch, 0, sizeof(int), s) != cudaSuccess) return DA_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return DA_ERR_CUDA;
+  switch (word) {
+    case 0: return DA_OK;
+    case DA_ERR_TIMEOUT: return DA_ERR_TIMEOUT;
+    case DA_ERR_DEVICE_INDEX: return DA_ERR_DEVICE_INDEX;
+    default: return DA_ERR_CUDA;
+  }
 }

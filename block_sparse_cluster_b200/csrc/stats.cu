@@ -18,7 +18,9 @@ WsLayout ws_layout(const Dims& g) {
   L.norms = 256;
   L.sched = L.norms + up(BH * g.C * sizeof(float));
   L.comp = L.sched + up(BH * g.nB * sizeof(int32_t));
-  L.total = L.comp + up(attention_tc_scratch_bytes(g));
+  L.spread = L.comp + up(attention_tc_scratch_bytes(g));
+  // Dh of the variance-corrected mode on the tensor cores (bf16 [B*H][C][d])
+  L.total = L.spread + (attention_tc_supported(g) ? up(BH * g.C * g.d * 2) : 0);
   return L;
 }
 
@@ -182,6 +184,15 @@ __global__ void schedule_kernel(const int32_t* __restrict__ kv_idx, const int32_
   }
 }
 
+// Dh = (scale / 2) D rounded to bf16; one thread per 4 values (C * d is a multiple of 4).
+__global__ void spread_half_kernel(const float4* __restrict__ D, float half_scale, uint2* __restrict__ out,
+                                   long long n4) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n4) return;
+  const float4 v = D[i];
+  out[i] = make_uint2(pack_bf16x2(v.x * half_scale, v.y * half_scale), pack_bf16x2(v.z * half_scale, v.w * half_scale));
+}
+
 // ------------------------------------------------------------------------------------------
 // launches
 
@@ -251,6 +262,14 @@ cudaError_t launch_cluster_spread(const Dims& g, const void* K, const void* cent
     if (g.d == 128) DA_SPREAD(float, 128); else DA_SPREAD(float, 64);
   }
 #undef DA_SPREAD
+  return cudaGetLastError();
+}
+
+cudaError_t launch_spread_half(const Dims& g, const float* spread, float scale, void* out, cudaStream_t s) {
+  const long long n4 = (long long)g.B * g.H * g.C * g.d / 4;
+  const unsigned grid = (unsigned)((n4 + 255) / 256);
+  spread_half_kernel<<<grid, 256, 0, s>>>(reinterpret_cast<const float4*>(spread), 0.5f * scale,
+                                           static_cast<uint2*>(out), n4);
   return cudaGetLastError();
 }
 

@@ -220,11 +220,14 @@ DA_API da_status da_centroid_update(const da_dims* dims, const da_cluster_stats*
  *
  * da_attention_spread: da_attention with every cluster logit corrected,
  *   s q.cbar_c + ln n^U_c + s^2/2 sum_t q_t^2 D_{c,t},
- * D = spread.  It runs on the CUDA cores for both dtypes (fp32 arithmetic,
- * the bf16 inputs upcast): a reference-grade path, not the tensor-core one.
- * It does not use da_compensation's values.  Arguments, layouts and errors as
- * in da_attention, plus spread ([B,H,C,d] fp32, read; DA_ERR_INVALID_ARG if
- * NULL).
+ * D = spread.  For bf16 with d = 128 and block = 128 it runs on the tensor
+ * cores: the compensation pre-pass (as da_compensation, into the workspace),
+ * Dh = (s/2) D rounded to bf16 (into the workspace), then the fused kernel with
+ * a second contraction (q o q, rounded to bf16) . Dh added to every cluster
+ * column's score.  Other shapes and fp32 run on the CUDA cores in fp32
+ * arithmetic.  Arguments, layouts and errors as in da_attention, plus spread
+ * ([B,H,C,d] fp32, read; DA_ERR_INVALID_ARG if NULL).  It overwrites the
+ * compensation values a da_compensation call left in the workspace.
  */
 /*
  * Inclusion-probability reweighting ("AB-Attention", abstract: sampled blocks
@@ -263,15 +266,22 @@ DA_API da_status da_attention_spread(const da_dims* dims, const void* Q, const v
  * and a status word) in a fixed file-scope device array of the library, about 1 MiB, held by every
  * GPU that loads libda.so until the process exits.  It allocates nothing.
  *   - Limit: B*H*C <= 262144; larger dims return DA_ERR_WORKSPACE before any launch.
- *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
- *     that device current; make that first call before any stream capture.
+ *   - Each call looks up the array's device address (cudaGetSymbolAddress) on the current device;
+ *     the first call on a device also loads the library's module there, so make that first call
+ *     before any stream capture.
  *   - Every call on a device shares the array and leaves its contents behind; the status word is
  *     cleared at the start of each call.  Calls whose kernels overlap on the GPU (for instance on
  *     two streams) race on the array.
- *   - Device-side problems (a bounded wait that gave up) are not reported by this call.
+ *   - Device-side problems (a bounded wait that gave up) are recorded in the array's status word;
+ *     da_noalloc_device_status() reports them.
  */
 DA_API da_status da_reassign_noalloc(const da_dims* dims, const void* K, const void* V, const void* centroids,
                                      const da_cluster_stats* out, da_stream stream);
+
+/* Synchronise `stream`, then report and clear the status word of da_reassign_noalloc's built-in
+ * scratch on the current device: DA_OK, DA_ERR_TIMEOUT or DA_ERR_DEVICE_INDEX (DA_ERR_CUDA if the
+ * synchronisation or the read failed).  Allocates nothing. */
+DA_API da_status da_noalloc_device_status(da_stream stream);
 
 /* Synchronise `stream`, then report and clear the workspace status word:
  * DA_OK, DA_ERR_TIMEOUT or DA_ERR_DEVICE_INDEX (or DA_ERR_CUDA if the

@@ -25,6 +25,13 @@ own S buffer (P written over it) and accumulator O_X; at the end of an item the
 two warpgroups exchange (max, sum) through a double-buffered shared array and
 each reads both accumulators.  The compensation chunks are written by an
 earlier kernel, so they are plain inputs here.
+
+The variance-corrected mode (spread=True) changes three things: a chunk step's
+score tile reads two key-ring tiles (the centroid chunk and the chunk of the
+scaled spread), so the key ring counts tiles, not steps; the value ring has
+two slots; and an otherwise idle warp writes the squared query tile Q2 for each
+item (after the query tile has landed), which the first chunk step of the item
+waits for.
 """
 import random
 
@@ -70,10 +77,16 @@ class Barrier:
 
 class Machine:
     def __init__(self, items, nchunk, rng, lazy_v_wait=False, skip_b_empty=False, single_xch=False,
-                 no_final_wait=False, single_xch_barrier=False):
+                 no_final_wait=False, single_xch_barrier=False, spread=False, q2_no_wait=False,
+                 mma_no_q2_wait=False, chunk_frees_one_tile=False):
         self.items = items                     # list of nsel per item of one CTA
         self.nchunk = nchunk
         self.rng = rng
+        self.spread = spread                   # variance-corrected mode: two key tiles per chunk step
+        self.vstages = 2 if spread else VSTAGES
+        self.q2_no_wait = q2_no_wait           # planted: Q2 written without waiting for the query tile
+        self.mma_no_q2_wait = mma_no_q2_wait   # planted: chunk scores issued without waiting for Q2
+        self.chunk_frees_one_tile = chunk_frees_one_tile   # planted: a chunk step frees only its first key tile
         self.lazy_v_wait = lazy_v_wait         # planted: value lane waits for a free slot only at chunk steps
         self.skip_b_empty = skip_b_empty       # planted: bias rows loaded without waiting for a free slot
         self.single_xch = single_xch           # planted: one (max, sum) exchange buffer for all items
@@ -83,8 +96,9 @@ class Machine:
         self.q_full, self.q_empty = B("q_full", 1), B("q_empty", 1)
         self.k_full = [B(f"k_full{i}", 1) for i in range(KSTAGES)]
         self.k_empty = [B(f"k_empty{i}", 1) for i in range(KSTAGES)]
-        self.v_full = [B(f"v_full{i}", 1) for i in range(VSTAGES)]
-        self.v_empty = [B(f"v_empty{i}", 1) for i in range(VSTAGES)]
+        self.v_full = [B(f"v_full{i}", 1) for i in range(self.vstages)]
+        self.v_empty = [B(f"v_empty{i}", 1) for i in range(self.vstages)]
+        self.q2_full = B("q2_full", 1)
         self.b_full = [B(f"b_full{i}", 1) for i in range(BSTAGES)]
         self.b_empty = [B(f"b_empty{i}", 1) for i in range(BSTAGES)]
         self.version = {}                      # buffer -> step whose tile it holds
@@ -156,19 +170,27 @@ class Machine:
         assert self.version.get(res) == step, f"{res} holds step {self.version.get(res)}, read at step {step}"
 
     # ---- roles (generators yield a predicate to wait on)
+    def tiles_of(self, s, nsel):
+        """Key-ring tiles of step s: the chunk of the scaled spread follows a centroid chunk."""
+        return 2 if self.spread and s >= nsel else 1
+
     def producer(self):
         """Lane 0 of the producer warp: query tiles, key / centroid tiles, bias rows."""
         g = 0
+        kt = 0                                  # key-ring tiles loaded
         for n, nsel in enumerate(self.items):
             T = nsel + self.nchunk
             yield lambda: self.q_empty.test(n - 1)
             self.q_full.expect_tx(1)
             self.tma_load(self.q_full, "Q", n)
             for s in range(T):
-                ks, bs = g % KSTAGES, g % BSTAGES
-                yield lambda: self.k_empty[ks].test(g // KSTAGES - 1)
-                self.k_full[ks].expect_tx(1)
-                self.tma_load(self.k_full[ks], f"K{ks}", g)
+                bs = g % BSTAGES
+                for _ in range(self.tiles_of(s, nsel)):
+                    ks = kt % KSTAGES
+                    yield lambda: self.k_empty[ks].test(kt // KSTAGES - 1)
+                    self.k_full[ks].expect_tx(1)
+                    self.tma_load(self.k_full[ks], f"K{ks}", kt)
+                    kt += 1
                 if not self.skip_b_empty:
                     yield lambda: self.b_empty[bs].test(g // BSTAGES - 1)
                     self.b_full[bs].expect_tx(1)
@@ -183,43 +205,68 @@ class Machine:
         for n, nsel in enumerate(self.items):
             T = nsel + self.nchunk
             for s in range(T):
-                vs = g % VSTAGES
+                vs = g % self.vstages
                 if not self.lazy_v_wait or s >= nsel:
-                    yield lambda: self.v_empty[vs].test(g // VSTAGES - 1)
+                    yield lambda: self.v_empty[vs].test(g // self.vstages - 1)
                 self.v_full[vs].expect_tx(1)
                 self.tma_load(self.v_full[vs], f"V{vs}", g)
                 g += 1
 
+    def q2_writer(self):
+        """Warp 11 in the variance-corrected mode: Q2 = Q o Q (generic stores) once Q has landed."""
+        for n, nsel in enumerate(self.items):
+            if not self.q2_no_wait:
+                yield lambda: self.q_full.test(n)
+            assert "tma" not in self.readers.get("Q", []), "Q read by the Q2 writer before it landed"
+            self.holds("Q", n)
+            self._write("Q2", "Q2 writer")
+            self.version["Q2"] = n
+            self.q2_full.arrive()
+
     def mma(self):
         g = 0
+        kt = 0                                  # key-ring tiles consumed
         for n, nsel in enumerate(self.items):
             T = nsel + self.nchunk
+
+            def issue_s(s, gs):
+                nonlocal kt
+                reads = ["Q"]
+                for _ in range(self.tiles_of(s, nsel)):
+                    t = kt
+                    yield lambda: self.k_full[t % KSTAGES].test(t // KSTAGES)
+                    self.holds(f"K{t % KSTAGES}", t)
+                    reads.append(f"K{t % KSTAGES}")
+                    kt += 1
+                if self.tiles_of(s, nsel) == 2:
+                    if s == nsel and not self.mma_no_q2_wait:
+                        yield lambda: self.q2_full.test(n)
+                    self.holds("Q2", n)
+                    reads.append("Q2")
+                self.tc_issue_mma(reads, [f"S{gs & 1}"])
+                self.tc_commit(self.s_full[gs & 1])
+                freed = reads[1:2] if self.chunk_frees_one_tile else [r for r in reads if r.startswith("K")]
+                for r in freed:
+                    self.tc_commit(self.k_empty[int(r[1:])])
+
             yield lambda: self.q_full.test(n)
-            yield lambda: self.k_full[g % KSTAGES].test(g // KSTAGES)
             self.holds("Q", n)
-            self.holds(f"K{g % KSTAGES}", g)
-            self.tc_issue_mma(["Q", f"K{g % KSTAGES}"], [f"S{g & 1}"])
-            self.tc_commit(self.s_full[g & 1])
-            self.tc_commit(self.k_empty[g % KSTAGES])
+            yield from issue_s(0, g)
             for s in range(T):
                 if s + 1 < T:
-                    gn = g + 1
-                    yield lambda: self.k_full[gn % KSTAGES].test(gn // KSTAGES)
-                    self.holds(f"K{gn % KSTAGES}", gn)
-                    self.tc_issue_mma(["Q", f"K{gn % KSTAGES}"], [f"S{gn & 1}"])
-                    self.tc_commit(self.s_full[gn & 1])
-                    self.tc_commit(self.k_empty[gn % KSTAGES])
+                    yield from issue_s(s + 1, g + 1)
                 else:
                     self.tc_commit(self.q_empty)
+                vs = g % self.vstages
                 yield lambda: self.p_ready[g & 1].test(g >> 1)
-                yield lambda: self.v_full[g % VSTAGES].test(g // VSTAGES)
+                yield lambda: self.v_full[vs].test(g // self.vstages)
                 if s == 0:
                     yield lambda: self.o_free.test(n - 1)
-                self.holds(f"V{g % VSTAGES}", g)
+                self.holds(f"V{vs}", g)
                 x = g & 1
-                self.tc_issue_mma([f"S{x}", f"V{g % VSTAGES}"], [f"O{x}"])
+                self.tc_issue_mma([f"S{x}", f"V{vs}"], [f"O{x}"])
                 self.o_content[x] = (n, 1) if s <= 1 else (n, self.o_content[x][1] + 1)
-                self.tc_commit(self.v_empty[g % VSTAGES])
+                self.tc_commit(self.v_empty[vs])
                 self.tc_commit(self.o_done[x])
                 g += 1
 
@@ -267,6 +314,8 @@ class Machine:
 
     def run(self, max_iters=200000):
         roles = [self.producer(), self.producer_v(), self.mma(), self.softmax(0), self.softmax(1)]
+        if self.spread:
+            roles.append(self.q2_writer())
         waits = [None] * len(roles)
         done = [False] * len(roles)
         for _ in range(max_iters):
@@ -306,6 +355,12 @@ def test_protocol_random_interleavings(items, nchunk):
         Machine(items, nchunk, random.Random(seed)).run()
 
 
+@pytest.mark.parametrize("items,nchunk", [c for c in CASES if c[1] >= 1])
+def test_protocol_random_interleavings_variance_corrected(items, nchunk):
+    for seed in range(60):
+        Machine(items, nchunk, random.Random(seed), spread=True).run()
+
+
 def _caught(items, nchunk, **planted):
     caught = 0
     for seed in range(40):
@@ -340,3 +395,15 @@ def test_model_catches_one_exchange_barrier_per_warpgroup():
     """A warpgroup without steps in an item can complete a single exchange barrier twice before
     the other warpgroup's parity wait on it runs."""
     assert _caught([1, 0, 0, 1], 1, single_xch_barrier=True) > 0
+
+
+def test_model_catches_q2_written_before_the_query_tile_lands():
+    assert _caught([2, 0, 3, 1], 2, spread=True, q2_no_wait=True) > 0
+
+
+def test_model_catches_chunk_scores_issued_without_waiting_for_q2():
+    assert _caught([0, 1, 0, 2], 2, spread=True, mma_no_q2_wait=True) > 0
+
+
+def test_model_catches_a_chunk_step_that_frees_one_of_its_two_key_tiles():
+    assert _caught([3, 0, 2], 2, spread=True, chunk_frees_one_tile=True) > 0
