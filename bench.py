@@ -317,7 +317,8 @@ def run_loop(args):
 def run_spread(args):
     """The variance-corrected cluster logits (ESTRA abstract's correction, read as a diagonal
     Gaussian about each representative): da_reassign + da_cluster_spread + da_attention_spread,
-    which runs on the CUDA cores.  One JSON line with the step time and its split."""
+    which runs on the tensor cores for bf16 with d = block = 128 (the CUDA cores otherwise).  One
+    JSON line with the step time and its split."""
     import block_sparse_cluster_b200 as da
     w = W.WORKLOADS[args.workload]
     if args.heads > 0:
