@@ -38,6 +38,7 @@ struct __align__(8) Bars {
   uint64_t kfull;
   uint64_t cfull[2];
   uint64_t mdone[2];
+  uint64_t tfree[2];      // TMEM buffer read out by all 8 warps (one arrival per warp)
   uint32_t tmem_base;
   int abort;
 };
@@ -79,6 +80,8 @@ reassign_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     mbar_init(&bars->cfull[1], 1);
     mbar_init(&bars->mdone[0], 1);
     mbar_init(&bars->mdone[1], 1);
+    mbar_init(&bars->tfree[0], kThreads / 32);
+    mbar_init(&bars->tfree[1], kThreads / 32);
     bars->abort = 0;
     fence_mbar_init();
   }
@@ -100,6 +103,8 @@ reassign_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     tma_load_3d(dst + kPanelC, &tm_c, &bars->cfull[c & 1], 64, c * kChunk, bh);
   };
   auto issue_mma = [&](int c) -> bool {
+    // TMEM buffer c & 1 was last written for chunk c - 2: every warp must have read it out
+    if (c >= 2 && !mbar_wait(&bars->tfree[c & 1], ((c - 2) >> 1) & 1, abort, status)) return false;
     if (!mbar_wait(&bars->cfull[c & 1], (c >> 1) & 1, abort, status)) return false;
     tc_fence_after();
     const int n = min(kChunk, C - c * kChunk);
@@ -181,9 +186,10 @@ reassign_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         }
       }
     }
+    // this warp has read TMEM buffer c & 1: the MMA of chunk c + 2 may overwrite it
     tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
+    __syncwarp();
+    if ((t & 31) == 0) mbar_arrive(&bars->tfree[c & 1]);
   }
   // merge: the smallest distance, the lowest cluster among equal ones; warpgroup 1 hands its
   // minimum to warpgroup 0 through shared memory

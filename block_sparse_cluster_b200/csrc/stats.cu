@@ -60,45 +60,100 @@ __global__ void __launch_bounds__(128) block_stats_kernel(const T* __restrict__ 
 }
 
 // Per-head totals n_c, S_c = sum over blocks of the block entries, in a fixed order.
-// A warp per (head, cluster): it walks the blocks in order, finds the cluster's entry through
-// seg_idx (eight blocks looked up at a time) and adds the entry row, lanes over the value columns
-// (coalesced rows; registers; blocks in order: deterministic bits).
+// A warp per (head, 8 clusters), lanes over the value columns.  Per batch of 32 blocks, lane u
+// looks up the 8 clusters' entries in block j0 + u (one 8-byte load of seg_idx); the present
+// (block, cluster) pairs are compacted into a per-warp list ordered by block, then cluster; the
+// list's entry rows are loaded 8 at a time and added, in list order, into the clusters'
+// accumulators in shared memory.  Every cluster's sum therefore takes its blocks' entries in block
+// order, the same fp32 additions in the same order as a walk over one cluster's blocks:
+// deterministic bits, with 8 lookups per load and 8 row loads in flight.
 template <int D>
 __global__ void __launch_bounds__(128) totals_kernel(StatsPtrs st, int C, int block, int nB) {
   constexpr int NS = D / 32;              // columns per lane
+  constexpr int G = 8;                    // clusters per warp
+  constexpr int kWarps = 4;
+  constexpr int kInFlight = 8;            // entry rows loaded per group
+  __shared__ __align__(16) float s_acc[kWarps][G][D];
+  __shared__ int s_list[kWarps][32 * G];  // (u << 11) | (g << 8) | entry
+  __shared__ int s_n[kWarps][G];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.x;
-  const int c = blockIdx.y * 4 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (c >= C) return;                     // (C is a multiple of 32)
-  float acc[NS];
+  const int c0 = (blockIdx.y * kWarps + warp) * G;
+  if (c0 >= C) return;                    // (C is a multiple of 32: whole warps)
+  float(*acc)[D] = s_acc[warp];
+  int* list = s_list[warp];
 #pragma unroll
-  for (int i = 0; i < NS; ++i) acc[i] = 0.f;
-  int n = 0;
+  for (int g = 0; g < G; ++g)
+#pragma unroll
+    for (int i = 0; i < NS; ++i) acc[g][lane * NS + i] = 0.f;
+  if (lane < G) s_n[warp][lane] = 0;
+  __syncwarp();
   const size_t hb = (size_t)bh * nB;
-  constexpr int kB = 8;                   // blocks looked up per batch
-  for (int j0 = 0; j0 < nB; j0 += kB) {
-    int e[kB];
+  for (int j0 = 0; j0 < nB; j0 += 32) {
+    // lookups: the 8 entry indices of block j0 + lane
+    uint2 w = make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);
+    if (j0 + lane < nB) w = *reinterpret_cast<const uint2*>(st.seg_idx + (hb + j0 + lane) * C + c0);
+    unsigned present = 0;
 #pragma unroll
-    for (int u = 0; u < kB; ++u) e[u] = j0 + u < nB ? (int)st.seg_idx[(hb + j0 + u) * C + c] : 0xFF;
+    for (int g = 0; g < G; ++g) {
+      const unsigned e = ((g < 4 ? w.x : w.y) >> (8 * (g & 3))) & 0xFFu;
+      present |= (e != 0xFFu ? 1u : 0u) << g;
+    }
+    // exclusive prefix of the counts over the lanes (blocks in order)
+    const int cnt = __popc(present);
+    int incl = cnt;
 #pragma unroll
-    for (int u = 0; u < kB; ++u) {
-      if (e[u] == 0xFF) continue;         // warp-uniform
-      const size_t row = (hb + j0 + u) * block + e[u];
-      if (lane == 0) n += st.seg_cnt[row];
-      float y[NS];
-      load_vec(st.seg_vsum + row * D + lane * NS, y, NS);
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const int total = __shfl_sync(0xffffffffu, incl, 31);
+    int pos = incl - cnt;
 #pragma unroll
-      for (int i = 0; i < NS; ++i) acc[i] += y[i];
+    for (int g = 0; g < G; ++g) {
+      if (present & (1u << g)) {
+        const unsigned e = ((g < 4 ? w.x : w.y) >> (8 * (g & 3))) & 0xFFu;
+        list[pos++] = (lane << 11) | (g << 8) | (int)e;
+      }
+    }
+    __syncwarp();
+    for (int i0 = 0; i0 < total; i0 += kInFlight) {
+      float y[kInFlight][NS];
+      int cnt_k[kInFlight] = {};
+      int item[kInFlight];
+#pragma unroll
+      for (int k = 0; k < kInFlight; ++k) {
+        item[k] = i0 + k < total ? list[i0 + k] : -1;
+        if (item[k] >= 0) {
+          const size_t row = (hb + j0 + (item[k] >> 11)) * block + (item[k] & 0xFF);
+          load_vec(st.seg_vsum + row * D + lane * NS, y[k], NS);
+          cnt_k[k] = lane == 0 ? st.seg_cnt[row] : 0;
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < kInFlight; ++k) {
+        if (item[k] >= 0) {                 // warp-uniform
+          const int g = (item[k] >> 8) & 7;
+#pragma unroll
+          for (int i = 0; i < NS; ++i) acc[g][lane * NS + i] += y[k][i];
+          if (lane == 0) s_n[warp][g] += cnt_k[k];
+        }
+      }
+    }
+    __syncwarp();                           // the list is rewritten by the next batch
+  }
+  __syncwarp();
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    float* dst = st.S_tot + ((size_t)bh * C + c0 + g) * D + lane * NS;
+    if constexpr (NS == 4) {
+      *reinterpret_cast<float4*>(dst) = *reinterpret_cast<const float4*>(&acc[g][lane * NS]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < NS; ++i) dst[i] = acc[g][lane * NS + i];
     }
   }
-  float* dst = st.S_tot + ((size_t)bh * C + c) * D + lane * NS;
-  if constexpr (NS == 4) {
-    *reinterpret_cast<float4*>(dst) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-  } else {
-#pragma unroll
-    for (int i = 0; i < NS; ++i) dst[i] = acc[i];
-  }
-  if (lane == 0) st.n_tot[(size_t)bh * C + c] = n;
+  if (lane < G) st.n_tot[(size_t)bh * C + c0 + lane] = s_n[warp][lane];
 }
 
 // Second moment of each cluster's keys about its representative (the variance correction of
@@ -245,7 +300,7 @@ cudaError_t launch_centroid_update(const Dims& g, const StatsPtrs& st, void* cen
 }
 
 cudaError_t launch_totals(const Dims& g, const StatsPtrs& st, cudaStream_t s) {
-  dim3 grid(g.B * g.H, (g.C + 3) / 4);                  // 4 clusters (warps) per CTA
+  dim3 grid(g.B * g.H, (g.C + 31) / 32);                // 4 warps of 8 clusters per CTA
   if (g.d == 128) totals_kernel<128><<<grid, 128, 0, s>>>(st, g.C, g.block, g.nB);
   else totals_kernel<64><<<grid, 128, 0, s>>>(st, g.C, g.block, g.nB);
   return cudaGetLastError();
