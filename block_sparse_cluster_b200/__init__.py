@@ -25,7 +25,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 DA_BF16, DA_F32 = 0, 1
 STATUS_NAMES = ["DA_OK", "DA_ERR_INVALID_ARG", "DA_ERR_SHAPE", "DA_ERR_DTYPE", "DA_ERR_ALIGNMENT",
                 "DA_ERR_UNSUPPORTED", "DA_ERR_CUDA", "DA_ERR_TIMEOUT", "DA_ERR_DEVICE_INDEX",
-                "DA_ERR_WORKSPACE"]
+                "DA_ERR_WORKSPACE", "DA_ERR_RANGE"]
 EXPORTS = ["da_version", "da_workspace_bytes", "da_schedule_bytes", "da_reassign", "da_mask_prepare",
            "da_attention", "da_device_status", "da_status_string", "da_reassign_noalloc", "da_compensation",
            "da_attention_prebuilt", "da_centroid_update", "da_cluster_spread", "da_attention_spread",

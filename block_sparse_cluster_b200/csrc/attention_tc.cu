@@ -32,11 +32,12 @@
 // Roles (384 threads):
 //   warps 0-3, 4-7  two softmax warpgroups X = 0, 1; warpgroup X takes the steps g with g & 1 = X
 //              of every item, so the two overlap each other and the tensor core.  Thread t of a
-//              warpgroup owns query row t = TMEM lane t: online softmax with lazy rescaling (the
-//              running max only moves when it grows by more than 2^8) of its own accumulator O_X,
-//              P written back to TMEM as bf16.  At the end of the item the two exchange their
-//              (max, sum) per row and each normalises and stores half of the columns of
-//              O = O_0 2^(m_0 - m) + O_1 2^(m_1 - m);
+//              warpgroup owns query row t = TMEM lane t.  Both warpgroups exponentiate against one
+//              reference max per row and item, the row max of the item's first step (handed to
+//              the other warpgroup through shared memory), so their products add into one
+//              accumulator O and no rescaling is ever needed; P is written back to TMEM as bf16.
+//              At the end of the item the two exchange their row sums and each normalises and
+//              stores half of the columns of O;
 //   warp 8     producer: loads Q, key tiles / centroid chunks (3-stage ring) and the softmax bias
 //              rows (4-stage ring, so a slot always serves the same warpgroup);
 //   warp 9     MMA: allocates TMEM, issues tcgen05.mma S(g+1) = Q K^T ahead of O_X += P(g) V(g);
@@ -44,7 +45,13 @@
 //              since divergent lanes of one warp waiting on different barriers hold each other up;
 //   warp 11    idle (it completes the third warpgroup, whose registers go to the softmax); in the
 //              variance-corrected mode it writes Q2 for each item once the query tile has landed.
-// TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,384), O_1 [384,512).
+// TMEM columns: S_0 [0,128), S_1 [128,256), S_2 [256,384), O [384,512).  Step g's scores go to
+// S_(g mod 3): the tensor core computes S(g+2) while the softmax of step g runs, and S(g+3) is
+// issued right after P(g) V(g), which frees its buffer (the tensor core executes in order).
+//
+// Range: P = 2^(y - m_ref) with m_ref the row max of the item's first step.  Later steps may
+// exceed it; a row whose logits exceed m_ref by more than 2^96 (in log2 units) in some step is
+// reported as DA_ERR_RANGE, since its sums could overflow fp32.
 //
 // Every mbarrier is waited at every phase, in order, by each role that waits on it (a parity
 // wait is only meaningful within one phase); the host-side protocol model in the tests replays
@@ -65,7 +72,8 @@ constexpr int kVStages = 3;             // value / vbar^U tiles (freed after P V
 constexpr int kBStages = 4;             // bias rows of the softmax (even: a slot serves one warpgroup)
 constexpr int kTile = kBN * kD * 2;      // 32 KB bf16 tile
 constexpr int kPanel = kBN * 128;        // one 64-column panel (128 rows x 128 B)
-constexpr float kRescaleLog2 = 8.0f;     // lazy rescale threshold (factor 256)
+constexpr int kSBufs = 3;                // score buffers in TMEM (and one accumulator O)
+constexpr float kRangeLog2 = 96.0f;      // largest step max above the reference max (log2 units)
 constexpr int kThreads = 384;           // three warpgroups; warp 11 idle
 constexpr int kWarpProducer = 8;
 constexpr int kWarpMMA = 9;
@@ -82,16 +90,21 @@ struct __align__(8) Bars {
   uint64_t q_full, q_empty, q2_full;
   uint64_t k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
   uint64_t b_full[kBStages], b_empty[kBStages];
-  uint64_t s_full[2], p_ready[2];
-  uint64_t o_done[2], o_free, drain;
-  // (max, sum) published: [item parity][warpgroup].  One barrier per item parity: a warpgroup
-  // without steps in an item could otherwise complete a barrier twice before the other
+  // s_full[g mod 6]: S(g) computed (g mod 6 fixes the buffer and the warpgroup, so each barrier
+  // is waited by one warpgroup at every phase); p_ready[g mod 3]: P(g) written
+  uint64_t s_full[2 * kSBufs], p_ready[kSBufs];
+  uint64_t o_full, o_free, drain;
+  // reference max published by the item's first step: [item parity]
+  uint64_t mref_full[2];
+  // (reference max, sum) published: [item parity][warpgroup].  One barrier per item parity: a
+  // warpgroup without steps in an item could otherwise complete a barrier twice before the other
   // warpgroup's parity wait on it runs.
   uint64_t xch_full[2][2];
   uint32_t tmem_base;
   int abort;
   int bflag[kBStages];                   // 1: the slot's bias row is all zero (a full key block)
-  float2 xch[2][2][kBM];                 // [item parity][warpgroup][row] = (max, sum)
+  float2 xch[2][2][kBM];                 // [item parity][warpgroup][row] = (reference max, sum)
+  float mref[2][kBM];                    // [item parity][row]
 };
 
 // (the variance-corrected mode holds Q2 in place of one value-ring slot: the same size)
@@ -263,13 +276,14 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       mbar_init(&bars->b_full[s], 1);
       mbar_init(&bars->b_empty[s], 128);
     }
+    for (int b = 0; b < 2 * kSBufs; ++b) mbar_init(&bars->s_full[b], 1);
+    for (int b = 0; b < kSBufs; ++b) mbar_init(&bars->p_ready[b], 128);
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&bars->s_full[b], 1);
-      mbar_init(&bars->p_ready[b], 128);
-      mbar_init(&bars->o_done[b], 1);
+      mbar_init(&bars->mref_full[b], 128);
       mbar_init(&bars->xch_full[b][0], 128);
       mbar_init(&bars->xch_full[b][1], 128);
     }
+    mbar_init(&bars->o_full, 1);
     mbar_init(&bars->o_free, 256);
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
@@ -414,7 +428,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       int n = 0;
       // S(gs) of step s of item `it` (the n-th of this CTA): waits for its key-ring tile(s) (and,
       // at the item's first chunk step in the variance-corrected mode, for Q2), issues the product
-      // and frees the tile(s) when it completes.
+      // into S_(gs mod 3) and frees the tile(s) when it completes.
       auto issue_s = [&](uint32_t gs, const Item& it, int s) -> bool {
         const bool two = kSpread && !p.incl && s >= it.nsel;
         const uint32_t t0 = kSpread ? kt : gs;   // one tile per step outside the corrected mode
@@ -426,7 +440,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
         tc_fence_after();
         const uint32_t kb = smem_u32(sK + (t0 % kKStages) * kTile);
-        const uint32_t d = tmem + (gs & 1) * kBN;
+        const uint32_t d = tmem + (gs % kSBufs) * kBN;
 #pragma unroll
         for (int ks = 0; ks < kD / 16; ++ks) {
           const uint32_t off = (ks >> 2) * kPanel + (ks & 3) * 32;
@@ -442,41 +456,42 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             umma_ss(d, sdesc_sw128(q2 + off, 16, 1024), sdesc_sw128(db + off, 16, 1024), idesc_qk, 1u);
           }
         }
-        umma_commit(&bars->s_full[gs & 1]);
+        umma_commit(&bars->s_full[gs % (2 * kSBufs)]);
         umma_commit(&bars->k_empty[t0 % kKStages]);
         if (two) umma_commit(&bars->k_empty[(t0 + 1) % kKStages]);
+        if (s == it.T - 1) umma_commit(&bars->q_empty);   // the item's last read of Q (and Q2)
         if (kSpread) kt = t0 + (two ? 2u : 1u);
         return true;
       };
+      const uint32_t ot = tmem + kSBufs * kBN;          // O
       bool ok = true;
       for (int k = blockIdx.x; k < p.n_items && ok; k += gridDim.x, ++n) {
         const Item it = item_at(p, k);
         if (!mbar_wait(&bars->q_full, n & 1, abort, status)) break;
         tc_fence_after();
-        if (!issue_s(g, it, 0)) break;
-        for (int s = 0; s < it.T; ++s, ++g) {
-          if (s + 1 < it.T) {
-            if (!issue_s(g + 1, it, s + 1)) { ok = false; break; }
-          } else {
-            umma_commit(&bars->q_empty);
-          }
+        // the first kSBufs score tiles of the item: their buffers were freed by the previous
+        // item's products, issued before them
+        const int pre = min(kSBufs, it.T);
+        for (int j = 0; j < pre && ok; ++j) ok = issue_s(g + j, it, j);
+        for (int s = 0; s < it.T && ok; ++s, ++g) {
           const int vs = g % kVSt;
-          if (!mbar_wait(&bars->p_ready[g & 1], (g >> 1) & 1, abort, status)) { ok = false; break; }
+          if (!mbar_wait(&bars->p_ready[g % kSBufs], (g / kSBufs) & 1, abort, status)) { ok = false; break; }
           if (!mbar_wait(&bars->v_full[vs], (g / kVSt) & 1, abort, status)) { ok = false; break; }
           if (s == 0 && !mbar_wait(&bars->o_free, (n & 1) ^ 1, abort, status)) { ok = false; break; }
           tc_fence_after();
           const uint32_t vb = smem_u32(sV + vs * kTile);
-          const uint32_t pt = tmem + (g & 1) * kBN;       // P: bf16 pairs in the S buffer's first 64 columns
-          const uint32_t ot = tmem + (2 + (g & 1)) * kBN;  // O_X of the step's warpgroup
+          const uint32_t pt = tmem + (g % kSBufs) * kBN;  // P: bf16 pairs in the S buffer's first 64 columns
 #pragma unroll
           for (int ks = 0; ks < kBN / 16; ++ks) {
-            // V rows (keys) 16*ks .. 16*ks+15: two 8-row groups of 1024 B; the first product of each
-            // accumulator in the item (steps 0 and 1) overwrites it
+            // V rows (keys) 16*ks .. 16*ks+15: two 8-row groups of 1024 B; the item's first product
+            // overwrites O
             umma_ts(ot, pt + ks * 8, sdesc_sw128(vb + ks * 2048, kPanel, 1024), idesc_pv,
-                    (s > 1 || ks > 0) ? 1u : 0u);
+                    (s > 0 || ks > 0) ? 1u : 0u);
           }
           umma_commit(&bars->v_empty[vs]);
-          umma_commit(&bars->o_done[g & 1]);
+          if (s == it.T - 1) umma_commit(&bars->o_full);
+          // S(g + 3) reuses the buffer that P(g) V(g), queued before it, reads
+          if (s + kSBufs < it.T && !issue_s(g + kSBufs, it, s + kSBufs)) { ok = false; break; }
         }
       }
       umma_commit(&bars->drain);
@@ -514,28 +529,26 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const int X = warp >> 2;                                  // warpgroup: steps g with g & 1 == X
     const int r = tid & 127;                                  // query row = TMEM lane
     const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-    const uint32_t o_own = lane_addr + (2 + X) * kBN;
     uint32_t g0 = 0;                                          // first step of the item
-    uint32_t u = 0;                                           // products into O_X issued so far
     int n = 0;
     // (no abort test in the loop condition: a warp leaves as a whole, on its __all_sync'd waits)
     for (int k = blockIdx.x; k < p.n_items; k += gridDim.x, ++n) {
       const Item it = item_at(p, k);
-      float m = -INFINITY, l = 0.f;
-      bool ok = true, first = true;
+      float mref = -INFINITY, l = 0.f;                       // -inf: no step of this warpgroup yet
+      bool ok = true;
       for (int s = (int)((X - g0) & 1u); s < it.T; s += 2) {
         const uint32_t g = g0 + s;
-        // every phase of this warpgroup's b_full slots and of s_full[X] is waited, in order
+        // every phase of this warpgroup's b_full slots and s_full barriers is waited, in order
         const int bs = g % kBStages;
         bool w_ok = mbar_wait(&bars->b_full[bs], (g / kBStages) & 1, abort, status);
-        w_ok = w_ok && mbar_wait(&bars->s_full[X], (g >> 1) & 1, abort, status);
+        w_ok = w_ok && mbar_wait(&bars->s_full[g % (2 * kSBufs)], (g / (2 * kSBufs)) & 1, abort, status);
         if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
         tc_fence_after();
-        // The S row is loaded from TMEM once (128 registers): the row max, then p = 2^(y - m), the
-        // row sum and the bf16 P written back over S.  Column c's logit is y_c = x_c * s*log2(e) +
-        // bias_c, the bias row in shared memory: log2 n^U_c on a compensation step, 0 on a key
-        // block (-inf past the end of a short last block).
-        const uint32_t sbase = lane_addr + X * kBN;
+        // The S row is loaded from TMEM once (128 registers): the row max, then p = 2^(y - m_ref),
+        // the row sum and the bf16 P written back over S.  Column c's logit is y_c = x_c *
+        // s*log2(e) + bias_c, the bias row in shared memory: log2 n^U_c on a compensation step, 0
+        // on a key block (-inf past the end of a short last block).
+        const uint32_t sbase = lane_addr + (g % kSBufs) * kBN;
         const float* bt = sBias + bs * kBN;
         const bool plain = bars->bflag[bs] != 0 && p.scale_log2 > 0.f;
         uint32_t x[4][32];
@@ -548,14 +561,21 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         reg_fence32(x[2]);
         reg_fence32(x[3]);
         const float mx = row_logits_max(x, bt, plain, p.scale_log2);
-        // lazy rescaling: the running max moves only when it grows by more than 2^8
-        const bool grow = mx > m + kRescaleLog2 || (m == -INFINITY && mx > -INFINITY);
-        const bool need_o = grow && !first && m > -INFINITY;
-        const float m_new = grow ? mx : m;
-        const float mu = (m_new == -INFINITY) ? 0.f : m_new;
+        if (s == 0) {
+          // the item's first step sets the row's reference max for both warpgroups
+          mref = mx > -INFINITY ? mx : 0.f;
+          bars->mref[n & 1][r] = mref;
+          mbar_arrive(&bars->mref_full[n & 1]);
+        } else if (s == 1) {
+          // this warpgroup's first step of the item: the other one published the reference
+          const bool m_ok = mbar_wait(&bars->mref_full[n & 1], (n >> 1) & 1, abort, status);
+          if (!__all_sync(0xffffffffu, m_ok)) { ok = false; break; }
+          mref = bars->mref[n & 1][r];
+        }
+        if (mx > mref + kRangeLog2) set_status(status, DA_ERR_RANGE);
         uint64_t rsum = 0;
         {
-          const uint64_t negmu = f2_pack(-mu, -mu);
+          const uint64_t negmu = f2_pack(-mref, -mref);
           const uint64_t coef = plain ? f2_pack(p.scale_log2, p.scale_log2) : f2_pack(1.f, 1.f);
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
@@ -567,32 +587,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         mbar_arrive(&bars->b_empty[bs]);          // this thread has read the bias row
         float rs_lo, rs_hi;
         f2_unpack(rsum, rs_lo, rs_hi);
-        const float rs = rs_lo + rs_hi;
-        if (!first) {
-          // this warpgroup's previous product has landed in O_X: every phase of o_done[X] is
-          // waited, in order; a row whose max moved rescales its O_X (warp-uniform, as
-          // tcgen05.ld/st are)
-          const bool d_ok = mbar_wait(&bars->o_done[X], (u - 1) & 1, abort, status);
-          if (!__all_sync(0xffffffffu, d_ok)) { ok = false; break; }
-          tc_fence_after();
-          if (__any_sync(0xffffffffu, need_o)) {
-            const float alpha = need_o ? ex2(m - m_new) : 1.f;
-#pragma unroll 1
-            for (int q = 0; q < 4; ++q) {
-              uint32_t rr[32];
-              tmem_ld32(o_own + q * 32, rr);
-              tmem_wait_ld();
-#pragma unroll
-              for (int v = 0; v < 32; ++v) rr[v] = __float_as_uint(__uint_as_float(rr[v]) * alpha);
-              tmem_st32(o_own + q * 32, rr);
-            }
-            if (need_o) l *= alpha;
-          }
-        }
-        m = m_new;
-        l += rs;
-        first = false;
-        ++u;
+        l += rs_lo + rs_hi;
         tmem_wait_st();
         tc_fence_before();
 #ifdef DA_FAULT_INJECT
@@ -604,49 +599,38 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 #else
         constexpr bool withhold = false;
 #endif
-        if (!withhold) mbar_arrive(&bars->p_ready[X]);
+        if (!withhold) mbar_arrive(&bars->p_ready[g % kSBufs]);
       }
       if (!ok) break;
-      // epilogue: once this warpgroup's last product has landed, exchange (max, sum) per row with
-      // the other warpgroup; warpgroup X normalises and stores columns [64X, 64X + 64) of
-      // O = (O_0 2^(m_0 - M) + O_1 2^(m_1 - M)) / (l_0 2^(m_0 - M) + l_1 2^(m_1 - M)).
-      // A warpgroup without a step in the item (a one-step item) has an unwritten O_X: skipped.
-      const bool had0 = it.T >= 2 || (g0 & 1u) == 0u;
-      const bool had1 = it.T >= 2 || (g0 & 1u) == 1u;
-      bool e_ok = first || mbar_wait(&bars->o_done[X], (u - 1) & 1, abort, status);
-      bars->xch[n & 1][X][r] = make_float2(m, l);
+      // epilogue: once the item's last product has landed in O, exchange (reference max, sum) per
+      // row with the other warpgroup; warpgroup X normalises and stores columns [64X, 64X + 64) of
+      // O / (l_0 + l_1).  Both sums are taken against the same reference; a warpgroup without a
+      // step in the item (a one-step item) publishes (-inf, 0).
+      bool e_ok = mbar_wait(&bars->o_full, n & 1, abort, status);
+      bars->xch[n & 1][X][r] = make_float2(mref, l);
       mbar_arrive(&bars->xch_full[n & 1][X]);
       e_ok = e_ok && mbar_wait(&bars->xch_full[n & 1][X ^ 1], (n >> 1) & 1, abort, status);
       if (!__all_sync(0xffffffffu, e_ok)) break;
       tc_fence_after();
       const float2 e0 = bars->xch[n & 1][0][r], e1 = bars->xch[n & 1][1][r];
       const float M = fmaxf(e0.x, e1.x);
-      const float f0 = (had0 && e0.x > -INFINITY) ? ex2(e0.x - M) : 0.f;
-      const float f1 = (had1 && e1.x > -INFINITY) ? ex2(e1.x - M) : 0.f;
-      const float L = e0.y * f0 + e1.y * f1;
+      const float L = e0.y + e1.y;
       const float inv = L > 0.f ? 1.f / L : 0.f;
-      const float c0 = f0 * inv, c1 = f1 * inv;
       const bool live = r < it.qlen;
       __nv_bfloat16* op = p.O + ((size_t)it.bh * p.N + it.q0 + r) * kD + 64 * X;
 #pragma unroll 1
       for (int q = 0; q < 2; ++q) {
-        const uint32_t col = 64 * X + 32 * q;
-        uint32_t ra[32], rb[32];
-        if (had0) tmem_ld32(lane_addr + 2 * kBN + col, ra);
-        if (had1) tmem_ld32(lane_addr + 3 * kBN + col, rb);
+        uint32_t ra[32];
+        tmem_ld32(lane_addr + kSBufs * kBN + 64 * X + 32 * q, ra);
         tmem_wait_ld();
         if (live) {
-          auto o = [&](int v) {
-            const float a = had0 ? __uint_as_float(ra[v]) * c0 : 0.f;
-            return had1 ? fmaf(__uint_as_float(rb[v]), c1, a) : a;
-          };
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
             uint4 w;
-            w.x = pack_bf16x2(o(8 * v + 0), o(8 * v + 1));
-            w.y = pack_bf16x2(o(8 * v + 2), o(8 * v + 3));
-            w.z = pack_bf16x2(o(8 * v + 4), o(8 * v + 5));
-            w.w = pack_bf16x2(o(8 * v + 6), o(8 * v + 7));
+            w.x = pack_bf16x2(__uint_as_float(ra[8 * v + 0]) * inv, __uint_as_float(ra[8 * v + 1]) * inv);
+            w.y = pack_bf16x2(__uint_as_float(ra[8 * v + 2]) * inv, __uint_as_float(ra[8 * v + 3]) * inv);
+            w.z = pack_bf16x2(__uint_as_float(ra[8 * v + 4]) * inv, __uint_as_float(ra[8 * v + 5]) * inv);
+            w.w = pack_bf16x2(__uint_as_float(ra[8 * v + 6]) * inv, __uint_as_float(ra[8 * v + 7]) * inv);
             *reinterpret_cast<uint4*>(op + q * 32 + v * 8) = w;
           }
         }

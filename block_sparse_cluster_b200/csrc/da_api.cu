@@ -348,6 +348,7 @@ da_status da_device_status(void* ws, da_stream stream) {
     case 0: return DA_OK;
     case DA_ERR_TIMEOUT: return DA_ERR_TIMEOUT;
     case DA_ERR_DEVICE_INDEX: return DA_ERR_DEVICE_INDEX;
+    case DA_ERR_RANGE: return DA_ERR_RANGE;
     default: return DA_ERR_CUDA;
   }
 }
@@ -364,6 +365,7 @@ const char* da_status_string(da_status s) {
     case DA_ERR_TIMEOUT: return "a bounded device wait gave up";
     case DA_ERR_DEVICE_INDEX: return "malformed block plan seen on the device";
     case DA_ERR_WORKSPACE: return "workspace or schedule buffer too small";
+    case DA_ERR_RANGE: return "logits beyond the attention kernel's range (a later step's max far above the first's)";
   }
   return "unknown status";
 }

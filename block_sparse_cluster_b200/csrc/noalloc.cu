@@ -104,6 +104,7 @@ extern "C" DA_API da_status da_noalloc_device_status(da_stream stream) {
     case 0: return DA_OK;
     case DA_ERR_TIMEOUT: return DA_ERR_TIMEOUT;
     case DA_ERR_DEVICE_INDEX: return DA_ERR_DEVICE_INDEX;
+    case DA_ERR_RANGE: return DA_ERR_RANGE;
     default: return DA_ERR_CUDA;
   }
 }

@@ -59,7 +59,10 @@ typedef enum {
   DA_ERR_TIMEOUT = 7,       /* a bounded device-side wait gave up (from da_device_status) */
   DA_ERR_DEVICE_INDEX = 8,  /* the device found a block index out of range, unsorted or repeated,
                                or kv_cnt outside [0, max_sel] (from da_device_status) */
-  DA_ERR_WORKSPACE = 9      /* workspace or schedule buffer too small */
+  DA_ERR_WORKSPACE = 9,     /* workspace or schedule buffer too small */
+  DA_ERR_RANGE = 10         /* the tensor-core attention found a row whose logits in a later step
+                               exceed its first step's max by more than 2^96 (log2 units, about
+                               66.5 nats): its sums may have overflowed (from da_device_status) */
 } da_status;
 
 typedef enum { DA_BF16 = 0, DA_F32 = 1 } da_dtype;
@@ -284,7 +287,7 @@ DA_API da_status da_reassign_noalloc(const da_dims* dims, const void* K, const v
 DA_API da_status da_noalloc_device_status(da_stream stream);
 
 /* Synchronise `stream`, then report and clear the workspace status word:
- * DA_OK, DA_ERR_TIMEOUT or DA_ERR_DEVICE_INDEX (or DA_ERR_CUDA if the
+ * DA_OK, DA_ERR_TIMEOUT, DA_ERR_DEVICE_INDEX or DA_ERR_RANGE (or DA_ERR_CUDA if the
  * synchronisation itself failed). */
 DA_API da_status da_device_status(void* ws, da_stream stream);
 

@@ -33,7 +33,7 @@ def test_every_declared_symbol_is_exported():
 
 def test_version_and_strings():
     assert da.da_version() == 103
-    for code in range(10):
+    for code in range(11):
         assert da.da_status_string(code) and da.da_status_string(code) != "unknown status"
 
 

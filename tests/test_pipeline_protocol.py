@@ -20,11 +20,15 @@ interleavings, and checks that
 
 It mirrors the step structure of attention_tc.cu: per work item, one step per
 selected block followed by one step per 128-cluster chunk; key, value and
-bias-row rings; softmax warpgroup X taking the steps g with g & 1 == X, with its
-own S buffer (P written over it) and accumulator O_X; at the end of an item the
-two warpgroups exchange (max, sum) through a double-buffered shared array and
-each reads both accumulators.  The compensation chunks are written by an
-earlier kernel, so they are plain inputs here.
+bias-row rings; softmax warpgroup X taking the steps g with g & 1 == X; three
+score buffers in TMEM, step g's S (and then P, written over it) in buffer
+g mod 3, and one accumulator O shared by both warpgroups, which exponentiate
+against a reference max that the item's first step publishes to the other
+warpgroup.  The tensor core executes in issue order, so S(g + 3) is queued after
+P(g) V(g), which reads the buffer.  At the end of an item the two warpgroups
+exchange their row sums through a double-buffered shared array and each reads
+half of O.  The compensation chunks are written by an earlier kernel, so they
+are plain inputs here.
 
 The variance-corrected mode (spread=True) changes three things: a chunk step's
 score tile reads two key-ring tiles (the centroid chunk and the chunk of the
@@ -40,6 +44,7 @@ import pytest
 KSTAGES = 2   # key / centroid tiles, freed when S is computed
 VSTAGES = 3   # value / vbar^U tiles, freed after P V
 BSTAGES = 4   # softmax bias rows, freed after the softmax has read them (even: one warpgroup per slot)
+SBUFS = 3     # score buffers in TMEM
 
 
 class Barrier:
@@ -78,7 +83,8 @@ class Barrier:
 class Machine:
     def __init__(self, items, nchunk, rng, lazy_v_wait=False, skip_b_empty=False, single_xch=False,
                  no_final_wait=False, single_xch_barrier=False, spread=False, q2_no_wait=False,
-                 mma_no_q2_wait=False, chunk_frees_one_tile=False):
+                 mma_no_q2_wait=False, chunk_frees_one_tile=False, s_before_pv=False, no_mref_wait=False,
+                 no_o_free_wait=False):
         self.items = items                     # list of nsel per item of one CTA
         self.nchunk = nchunk
         self.rng = rng
@@ -87,6 +93,9 @@ class Machine:
         self.q2_no_wait = q2_no_wait           # planted: Q2 written without waiting for the query tile
         self.mma_no_q2_wait = mma_no_q2_wait   # planted: chunk scores issued without waiting for Q2
         self.chunk_frees_one_tile = chunk_frees_one_tile   # planted: a chunk step frees only its first key tile
+        self.s_before_pv = s_before_pv         # planted: S(g + 3) queued before P(g) V(g)
+        self.no_mref_wait = no_mref_wait       # planted: the second warpgroup reads the reference unpublished
+        self.no_o_free_wait = no_o_free_wait   # planted: an item's first product without waiting for O's readers
         self.lazy_v_wait = lazy_v_wait         # planted: value lane waits for a free slot only at chunk steps
         self.skip_b_empty = skip_b_empty       # planted: bias rows loaded without waiting for a free slot
         self.single_xch = single_xch           # planted: one (max, sum) exchange buffer for all items
@@ -102,15 +111,17 @@ class Machine:
         self.b_full = [B(f"b_full{i}", 1) for i in range(BSTAGES)]
         self.b_empty = [B(f"b_empty{i}", 1) for i in range(BSTAGES)]
         self.version = {}                      # buffer -> step whose tile it holds
-        self.s_full = [B(f"s_full{i}", 1) for i in range(2)]
-        self.p_ready = [B(f"p_ready{i}", 1) for i in range(2)]
-        self.o_done = [B(f"o_done{i}", 1) for i in range(2)]
+        self.s_full = [B(f"s_full{i}", 1) for i in range(2 * SBUFS)]   # [g mod 6]
+        self.p_ready = [B(f"p_ready{i}", 1) for i in range(SBUFS)]     # [g mod 3]
+        self.o_full = B("o_full", 1)
         self.o_free = B("o_free", 2)           # one arrival per warpgroup (128 threads each)
+        self.mref_full = [B(f"mref_full{i}", 1) for i in range(2)]
+        self.mref = [None, None]               # [item parity] -> item whose reference it holds
         # exchange published: [item parity][warpgroup]; one barrier per item parity, so a warpgroup
         # without steps cannot complete a barrier twice before the other has waited on it once
         self.xch_full = [[B(f"xch_full{j}{i}", 1) for i in range(2)] for j in range(2)]
         self.xch = [[None, None], [None, None]]   # [item parity][warpgroup] -> item whose (max, sum) it holds
-        self.o_content = [None, None]          # accumulator -> (item, products accumulated), at issue
+        self.o_content = None                  # (item, products accumulated), at execution
         self.tc_queue = []                     # in-order tensor core: ("mma", reads, writes) / ("commit", bar)
         self.tma = []                          # in flight: (bar, buffer written, buffers read)
         self.readers = {}                      # resource -> units with an operation in flight on it
@@ -129,12 +140,14 @@ class Machine:
         assert not busy, f"{who} overwrites {res} while {busy} use it"
 
     # ---- asynchronous units
-    def tc_issue_mma(self, reads, writes):
+    def tc_issue_mma(self, reads, writes, expect=None, produce=None, on_exec=None):
+        """Queue a product.  expect: {buffer: version it must hold when the product executes};
+        produce: {buffer: version it holds afterwards}; on_exec: a callback run at execution."""
         for w in writes:
             self._write(w, "tensor core", unit="tc")
         for r in reads + writes:     # the destination is busy until the MMA completes
             self._start_read(r, "tc")
-        self.tc_queue.append(("mma", reads + writes))
+        self.tc_queue.append(("mma", (reads + writes, expect or {}, produce or {}, on_exec)))
 
     def tc_commit(self, bar):
         self.tc_queue.append(("commit", bar))
@@ -144,7 +157,14 @@ class Machine:
         if self.tc_queue and self.rng.random() < 0.5:
             kind, x = self.tc_queue.pop(0)
             if kind == "mma":
-                for r in x:
+                bufs, expect, produce, on_exec = x
+                for b, v in expect.items():
+                    assert self.version.get(b) == v, f"a product reads {b} holding {self.version.get(b)}, wants {v}"
+                for b, v in produce.items():
+                    self.version[b] = v
+                if on_exec:
+                    on_exec()
+                for r in bufs:
                     self._end_read(r, "tc")
             else:
                 x.arrive()
@@ -243,58 +263,70 @@ class Machine:
                         yield lambda: self.q2_full.test(n)
                     self.holds("Q2", n)
                     reads.append("Q2")
-                self.tc_issue_mma(reads, [f"S{gs & 1}"])
-                self.tc_commit(self.s_full[gs & 1])
+                b = gs % SBUFS
+                self.tc_issue_mma(reads, [f"S{b}"], produce={f"S{b}": ("S", gs)})
+                self.tc_commit(self.s_full[gs % (2 * SBUFS)])
                 freed = reads[1:2] if self.chunk_frees_one_tile else [r for r in reads if r.startswith("K")]
                 for r in freed:
                     self.tc_commit(self.k_empty[int(r[1:])])
+                if s == T - 1:
+                    self.tc_commit(self.q_empty)
 
             yield lambda: self.q_full.test(n)
             self.holds("Q", n)
-            yield from issue_s(0, g)
+            pending = []                        # S issues postponed by the planted order
+            for j in range(min(SBUFS, T)):
+                yield from issue_s(j, g + j)
             for s in range(T):
-                if s + 1 < T:
-                    yield from issue_s(s + 1, g + 1)
-                else:
-                    self.tc_commit(self.q_empty)
+                if self.s_before_pv and s + SBUFS < T:
+                    yield from issue_s(s + SBUFS, g + SBUFS)
                 vs = g % self.vstages
-                yield lambda: self.p_ready[g & 1].test(g >> 1)
+                yield lambda: self.p_ready[g % SBUFS].test(g // SBUFS)
                 yield lambda: self.v_full[vs].test(g // self.vstages)
-                if s == 0:
+                if s == 0 and not self.no_o_free_wait:
                     yield lambda: self.o_free.test(n - 1)
                 self.holds(f"V{vs}", g)
-                x = g & 1
-                self.tc_issue_mma([f"S{x}", f"V{vs}"], [f"O{x}"])
-                self.o_content[x] = (n, 1) if s <= 1 else (n, self.o_content[x][1] + 1)
+
+                def count(n=n, s=s):
+                    self.o_content = (n, 1) if s == 0 else (n, self.o_content[1] + 1)
+                self.tc_issue_mma([f"S{g % SBUFS}", f"V{vs}"], ["O"], expect={f"S{g % SBUFS}": ("P", g)},
+                                  on_exec=count)
                 self.tc_commit(self.v_empty[vs])
-                self.tc_commit(self.o_done[x])
+                if s == T - 1:
+                    self.tc_commit(self.o_full)
+                if not self.s_before_pv and s + SBUFS < T:
+                    yield from issue_s(s + SBUFS, g + SBUFS)
                 g += 1
 
     def softmax(self, X):
         g0 = 0
-        u = 0                                   # products into O_X issued so far
         for n, nsel in enumerate(self.items):
             T = nsel + self.nchunk
-            first = True
-            for s in range((X - g0) & 1, T, 2):
+            steps = list(range((X - g0) & 1, T, 2))
+            for s in steps:
                 g = g0 + s
                 bs = g % BSTAGES
+                b = g % SBUFS
                 yield lambda: self.b_full[bs].test(g // BSTAGES)
-                yield lambda: self.s_full[X].test(g >> 1)
-                assert not self.readers.get(f"S{X}"), "S read before its MMA completed"
+                yield lambda: self.s_full[g % (2 * SBUFS)].test(g // (2 * SBUFS))
+                assert not self.readers.get(f"S{b}"), "S read before its MMA completed"
+                assert self.version.get(f"S{b}") == ("S", g), f"S{b} holds {self.version.get(f'S{b}')} at step {g}"
                 assert not self.readers.get(f"BIAS{bs}"), "bias row read before it landed"
                 self.holds(f"BIAS{bs}", g)
-                self._write(f"S{X}", "softmax (P)")
+                if s == 0:
+                    self.mref[n & 1] = n
+                    self.mref_full[n & 1].arrive()
+                elif s == 1:
+                    if not self.no_mref_wait:
+                        yield lambda: self.mref_full[n & 1].test(n >> 1)
+                    assert self.mref[n & 1] == n, f"reference of item {self.mref[n & 1]} read for item {n}"
+                self._write(f"S{b}", "softmax (P)")
+                self.version[f"S{b}"] = ("P", g)
                 self.b_empty[bs].arrive()
-                if not first:
-                    yield lambda: self.o_done[X].test(u - 1)
-                    self._write(f"O{X}", "softmax (rescale)")
-                self.p_ready[X].arrive()
-                first = False
-                u += 1
+                self.p_ready[b].arrive()
             # epilogue
-            if not first and not self.no_final_wait:
-                yield lambda: self.o_done[X].test(u - 1)
+            if not self.no_final_wait:
+                yield lambda: self.o_full.test(n)
             slot = 0 if self.single_xch else n & 1
             self.xch[slot][X] = n
             if self.single_xch_barrier:
@@ -304,11 +336,14 @@ class Machine:
                 self.xch_full[n & 1][X].arrive()
                 yield lambda: self.xch_full[n & 1][X ^ 1].test(n >> 1)
             assert self.xch[slot][X ^ 1] == n, f"exchange slot holds item {self.xch[slot][X ^ 1]}, read for item {n}"
-            for Y in (0, 1):
-                steps = len(range((Y - g0) & 1, T, 2))
-                if steps:
-                    assert not self.readers.get(f"O{Y}"), f"O{Y} read while a product into it is in flight"
-                    assert self.o_content[Y] == (n, steps), f"O{Y} holds {self.o_content[Y]} at the end of item {n}"
+            # this warpgroup's half of O is read over a span in which the other roles move on
+            assert "tc" not in self.readers.get("O", []), "O read while a product into it is in flight"
+            assert self.o_content == (n, T), f"O holds {self.o_content} at the end of item {n}"
+            self._start_read("O", f"epilogue{X}")
+            for _ in range(self.rng.randrange(1, 40)):  # a read of random length
+                yield lambda: True
+            assert self.o_content == (n, T), f"O changed to {self.o_content} while item {n}'s epilogue read it"
+            self._end_read("O", f"epilogue{X}")
             self.o_free.arrive()
             g0 += T
 
@@ -381,29 +416,36 @@ def test_model_catches_bias_rows_loaded_without_a_free_slot():
     assert _caught([3, 3, 3, 3, 3], 2, skip_b_empty=True) > 0
 
 
-def test_model_catches_a_single_exchange_buffer():
-    """With one-step items a warpgroup without steps reaches the next exchange while the other
-    still reads the previous one."""
-    assert _caught([0, 0, 0, 0, 0, 0], 1, single_xch=True) > 0
+def test_a_single_exchange_buffer_is_safe_with_the_shared_accumulator():
+    """Both warpgroups wait for the item's last product before the exchange, and that product
+    waits for both warpgroups' previous epilogue (o_free), so the exchange of item n + 1 cannot be
+    written before item n's has been read: one buffer would do; two are kept."""
+    assert _caught([0, 0, 0, 0, 0, 0], 1, single_xch=True) == 0
+    assert _caught([2, 0, 1, 0, 3], 1, single_xch=True) == 0
 
 
 def test_model_catches_an_epilogue_that_does_not_wait_for_the_last_product():
     assert _caught([3, 4, 1], 2, no_final_wait=True) > 0
 
 
-def test_model_catches_one_exchange_barrier_per_warpgroup():
-    """A warpgroup without steps in an item can complete a single exchange barrier twice before
-    the other warpgroup's parity wait on it runs."""
-    assert _caught([1, 0, 0, 1], 1, single_xch_barrier=True) > 0
+def test_model_catches_a_score_tile_queued_before_the_product_that_reads_its_buffer():
+    """S(g + 3) goes into the buffer that holds P(g): queued before P(g) V(g), it overwrites P."""
+    assert _caught([5, 2, 4], 2, s_before_pv=True) > 0
 
 
-def test_model_catches_q2_written_before_the_query_tile_lands():
-    assert _caught([2, 0, 3, 1], 2, spread=True, q2_no_wait=True) > 0
+def test_model_catches_a_reference_max_read_before_it_is_published():
+    assert _caught([2, 3, 1, 4], 1, no_mref_wait=True) > 0
 
 
-def test_model_catches_chunk_scores_issued_without_waiting_for_q2():
-    assert _caught([0, 1, 0, 2], 2, spread=True, mma_no_q2_wait=True) > 0
+def test_model_catches_a_first_product_that_does_not_wait_for_the_epilogue():
+    """An item's first product overwrites O: without waiting on o_free it can land while the other
+    item's epilogue still reads O."""
+    assert _caught([1, 0, 2, 1], 1, no_o_free_wait=True) > 0
 
 
-def test_model_catches_a_chunk_step_that_frees_one_of_its_two_key_tiles():
-    assert _caught([3, 0, 2], 2, spread=True, chunk_frees_one_tile=True) > 0
+def test_one_exchange_barrier_per_warpgroup_is_safe_with_the_shared_accumulator():
+    """With one accumulator the warpgroups meet at every item's last product (o_full) and at the
+    next item's first product (o_free), so a warpgroup without steps can no longer complete an
+    exchange barrier twice before the other's wait: the per-item-parity barriers are kept anyway."""
+    assert _caught([1, 0, 0, 1], 1, single_xch_barrier=True) == 0
+    assert _caught([0, 0, 2, 0, 0, 1], 1, single_xch_barrier=True) == 0
