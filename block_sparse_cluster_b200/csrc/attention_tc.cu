@@ -25,9 +25,10 @@
 // logits): a cluster column's logit gains s^2/2 sum_t q_t^2 D_{c,t}, D_c the second moment of the
 // cluster's keys about its representative.  The correction is a second contraction into the same
 // score tile: S = Q cbar^T + Q2 Dh^T, with Q2 = q o q (bf16, written into shared memory from the
-// query tile by warp 11) and Dh = (s/2) D (bf16, from the host side).  A chunk step therefore takes
+// query tile by the softmax warpgroups) and Dh = (s/2) D (bf16, from the host side).  A chunk step therefore takes
 // two key-ring tiles (the centroid chunk, then the Dh chunk), so the key ring counts tiles, not
-// steps; the query tile Q2 takes the place of one value-ring slot (two slots in this mode).
+// steps; the query tile Q2 takes the place of one value-ring slot (two slots in this mode).  The
+// softmax warpgroups write Q2 at the start of each item.
 //
 // Roles (384 threads):
 //   warps 0-3, 4-7  two softmax warpgroups X = 0, 1; warpgroup X takes the steps g with g & 1 = X
@@ -38,16 +39,20 @@
 //              accumulator O and no rescaling is ever needed; P is written back to TMEM as bf16.
 //              At the end of the item the two exchange their row sums and each normalises and
 //              stores half of the columns of O;
-//   warp 8     producer: loads Q, key tiles / centroid chunks (3-stage ring) and the softmax bias
+//   warp 8     producer: loads Q, key tiles / centroid chunks (2-stage ring) and the softmax bias
 //              rows (4-stage ring, so a slot always serves the same warpgroup);
-//   warp 9     MMA: allocates TMEM, issues tcgen05.mma S(g+1) = Q K^T ahead of O_X += P(g) V(g);
-//   warp 10    producer of value tiles / compensation chunks (2-stage ring); a warp of its own,
+//   warp 9     score issuer: allocates TMEM, issues tcgen05.mma S(g) = Q K^T into S_(g mod 3) as
+//              soon as its key tile has landed and P(g-3) V(g-3) has finished reading the buffer
+//              (in the variance-corrected mode both softmax warpgroups write Q2 at each item's start);
+//   warp 10    producer of value tiles / compensation chunks (3-stage ring); a warp of its own,
 //              since divergent lanes of one warp waiting on different barriers hold each other up;
-//   warp 11    idle (it completes the third warpgroup, whose registers go to the softmax); in the
-//              variance-corrected mode it writes Q2 for each item once the query tile has landed.
+//   warp 11    product issuer: O += P(g) V(g) once P(g) is written.  Two issuing threads keep the
+//              tensor core fed: one thread's waits on the softmax no longer hold the other's
+//              products back (issuing blocks while the tensor core's queue is full).
 // TMEM columns: S_0 [0,128), S_1 [128,256), S_2 [256,384), O [384,512).  Step g's scores go to
-// S_(g mod 3): the tensor core computes S(g+2) while the softmax of step g runs, and S(g+3) is
-// issued right after P(g) V(g), which frees its buffer (the tensor core executes in order).
+// S_(g mod 3): the tensor core computes S(g+1) and S(g+2) while the softmax of step g runs, and
+// S(g+3) waits for P(g) V(g) to complete (pv_done), since the two issuers' products are not ordered
+// with respect to each other.
 //
 // Range: P = 2^(y - m_ref) with m_ref the row max of the item's first step.  Later steps may
 // exceed it; a row whose logits exceed m_ref by more than 2^96 (in log2 units) in some step is
@@ -76,9 +81,9 @@ constexpr int kSBufs = 3;                // score buffers in TMEM (and one accum
 constexpr float kRangeLog2 = 96.0f;      // largest step max above the reference max (log2 units)
 constexpr int kThreads = 384;           // three warpgroups; warp 11 idle
 constexpr int kWarpProducer = 8;
-constexpr int kWarpMMA = 9;
+constexpr int kWarpMMA = 9;             // score issuer (and TMEM owner)
 constexpr int kWarpProducerV = 10;
-constexpr int kWarpQ2 = 11;
+constexpr int kWarpPV = 11;              // product issuer
 // Register split (setmaxnreg): the launch holds 384 x 168 registers; the softmax warpgroups grow,
 // the producer / MMA warpgroup shrinks.
 constexpr int kRegSoftmax = 232, kRegIssue = 40;
@@ -93,7 +98,8 @@ struct __align__(8) Bars {
   // s_full[g mod 6]: S(g) computed (g mod 6 fixes the buffer and the warpgroup, so each barrier
   // is waited by one warpgroup at every phase); p_ready[g mod 3]: P(g) written
   uint64_t s_full[2 * kSBufs], p_ready[kSBufs];
-  uint64_t o_full, o_free, drain;
+  uint64_t pv_done[kSBufs];              // P(g) V(g) complete: S_(g mod 3) may take S(g + 3)
+  uint64_t o_full, o_free, drain, drain_pv;
   // reference max published by the item's first step: [item parity]
   uint64_t mref_full[2];
   // (reference max, sum) published: [item parity][warpgroup].  One barrier per item parity: a
@@ -263,7 +269,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   if (tid == 0) {
     mbar_init(&bars->q_full, 1);
     mbar_init(&bars->q_empty, 1);
-    mbar_init(&bars->q2_full, 1);
+    mbar_init(&bars->q2_full, 256);
     for (int s = 0; s < kKStages; ++s) {
       mbar_init(&bars->k_full[s], 1);
       mbar_init(&bars->k_empty[s], 1);
@@ -277,7 +283,10 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       mbar_init(&bars->b_empty[s], 128);
     }
     for (int b = 0; b < 2 * kSBufs; ++b) mbar_init(&bars->s_full[b], 1);
-    for (int b = 0; b < kSBufs; ++b) mbar_init(&bars->p_ready[b], 128);
+    for (int b = 0; b < kSBufs; ++b) {
+      mbar_init(&bars->p_ready[b], 128);
+      mbar_init(&bars->pv_done[b], 1);
+    }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars->mref_full[b], 128);
       mbar_init(&bars->xch_full[b][0], 128);
@@ -286,6 +295,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     mbar_init(&bars->o_full, 1);
     mbar_init(&bars->o_free, 256);
     mbar_init(&bars->drain, 1);
+    mbar_init(&bars->drain_pv, 1);
     bars->abort = 0;
     fence_mbar_init();
   }
@@ -418,62 +428,69 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         mbar_wait_drain(&bars->v_full[gd % kVSt], (gd / kVSt) & 1);
     }
   } else if (warp == kWarpMMA) {
-    // ------------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------------ score issuer
     if (lane == 0) {
       const uint32_t idesc_qk = idesc_bf16(kBM, kBN, 0, 0);   // Q, K both K-major
-      const uint32_t idesc_pv = idesc_bf16(kBM, kD, 0, 1);    // P from TMEM, V MN-major
       const uint32_t q0 = smem_u32(sQ);
       uint32_t g = 0;
       uint32_t kt = 0;                   // key-ring tiles consumed
       int n = 0;
-      // S(gs) of step s of item `it` (the n-th of this CTA): waits for its key-ring tile(s) (and,
-      // at the item's first chunk step in the variance-corrected mode, for Q2), issues the product
-      // into S_(gs mod 3) and frees the tile(s) when it completes.
-      auto issue_s = [&](uint32_t gs, const Item& it, int s) -> bool {
-        const bool two = kSpread && !p.incl && s >= it.nsel;
-        const uint32_t t0 = kSpread ? kt : gs;   // one tile per step outside the corrected mode
-        if (!mbar_wait(&bars->k_full[t0 % kKStages], (t0 / kKStages) & 1, abort, status)) return false;
-        if (two) {
-          const uint32_t t1 = t0 + 1;
-          if (!mbar_wait(&bars->k_full[t1 % kKStages], (t1 / kKStages) & 1, abort, status)) return false;
-          if (s == it.nsel && !mbar_wait(&bars->q2_full, n & 1, abort, status)) return false;
-        }
-        tc_fence_after();
-        const uint32_t kb = smem_u32(sK + (t0 % kKStages) * kTile);
-        const uint32_t d = tmem + (gs % kSBufs) * kBN;
-#pragma unroll
-        for (int ks = 0; ks < kD / 16; ++ks) {
-          const uint32_t off = (ks >> 2) * kPanel + (ks & 3) * 32;
-          umma_ss(d, sdesc_sw128(q0 + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), idesc_qk, ks > 0);
-        }
-        if (two) {
-          // + Q2 Dh^T: the correction of the cluster logits, into the same accumulator
-          const uint32_t q2 = smem_u32(sQ2);
-          const uint32_t db = smem_u32(sK + ((t0 + 1) % kKStages) * kTile);
-#pragma unroll 1
-          for (int ks = 0; ks < kD / 16; ++ks) {
-            const uint32_t off = (ks >> 2) * kPanel + (ks & 3) * 32;
-            umma_ss(d, sdesc_sw128(q2 + off, 16, 1024), sdesc_sw128(db + off, 16, 1024), idesc_qk, 1u);
-          }
-        }
-        umma_commit(&bars->s_full[gs % (2 * kSBufs)]);
-        umma_commit(&bars->k_empty[t0 % kKStages]);
-        if (two) umma_commit(&bars->k_empty[(t0 + 1) % kKStages]);
-        if (s == it.T - 1) umma_commit(&bars->q_empty);   // the item's last read of Q (and Q2)
-        if (kSpread) kt = t0 + (two ? 2u : 1u);
-        return true;
-      };
-      const uint32_t ot = tmem + kSBufs * kBN;          // O
       bool ok = true;
       for (int k = blockIdx.x; k < p.n_items && ok; k += gridDim.x, ++n) {
         const Item it = item_at(p, k);
         if (!mbar_wait(&bars->q_full, n & 1, abort, status)) break;
-        tc_fence_after();
-        // the first kSBufs score tiles of the item: their buffers were freed by the previous
-        // item's products, issued before them
-        const int pre = min(kSBufs, it.T);
-        for (int j = 0; j < pre && ok; ++j) ok = issue_s(g + j, it, j);
-        for (int s = 0; s < it.T && ok; ++s, ++g) {
+        for (int s = 0; s < it.T; ++s, ++g) {
+          // S_(g mod 3) last held S(g - 3): its product must have read P(g - 3); every phase of
+          // pv_done[g mod 3] is waited, in order
+          if (g >= (uint32_t)kSBufs &&
+              !mbar_wait(&bars->pv_done[g % kSBufs], ((g / kSBufs) & 1) ^ 1, abort, status)) { ok = false; break; }
+          const bool two = kSpread && !p.incl && s >= it.nsel;
+          const uint32_t t0 = kSpread ? kt : g;   // one tile per step outside the corrected mode
+          if (!mbar_wait(&bars->k_full[t0 % kKStages], (t0 / kKStages) & 1, abort, status)) { ok = false; break; }
+          if (two) {
+            const uint32_t t1 = t0 + 1;
+            if (!mbar_wait(&bars->k_full[t1 % kKStages], (t1 / kKStages) & 1, abort, status)) { ok = false; break; }
+            if (s == it.nsel && !mbar_wait(&bars->q2_full, n & 1, abort, status)) { ok = false; break; }
+          }
+          tc_fence_after();
+          const uint32_t kb = smem_u32(sK + (t0 % kKStages) * kTile);
+          const uint32_t d = tmem + (g % kSBufs) * kBN;
+#pragma unroll
+          for (int ks = 0; ks < kD / 16; ++ks) {
+            const uint32_t off = (ks >> 2) * kPanel + (ks & 3) * 32;
+            umma_ss(d, sdesc_sw128(q0 + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), idesc_qk, ks > 0);
+          }
+          if (two) {
+            // + Q2 Dh^T: the correction of the cluster logits, into the same accumulator
+            const uint32_t q2 = smem_u32(sQ2);
+            const uint32_t db = smem_u32(sK + ((t0 + 1) % kKStages) * kTile);
+#pragma unroll 1
+            for (int ks = 0; ks < kD / 16; ++ks) {
+              const uint32_t off = (ks >> 2) * kPanel + (ks & 3) * 32;
+              umma_ss(d, sdesc_sw128(q2 + off, 16, 1024), sdesc_sw128(db + off, 16, 1024), idesc_qk, 1u);
+            }
+          }
+          umma_commit(&bars->s_full[g % (2 * kSBufs)]);
+          umma_commit(&bars->k_empty[t0 % kKStages]);
+          if (two) umma_commit(&bars->k_empty[(t0 + 1) % kKStages]);
+          if (s == it.T - 1) umma_commit(&bars->q_empty);   // the item's last read of Q (and Q2)
+          if (kSpread) kt = t0 + (two ? 2u : 1u);
+        }
+      }
+      umma_commit(&bars->drain);
+      mbar_wait_drain(&bars->drain, 0);
+    }
+  } else if (warp == kWarpPV) {
+    // ------------------------------------------------------------------ product issuer
+    if (lane == 0) {
+      const uint32_t idesc_pv = idesc_bf16(kBM, kD, 0, 1);    // P from TMEM, V MN-major
+      const uint32_t ot = tmem + kSBufs * kBN;                // O
+      uint32_t g = 0;
+      int n = 0;
+      bool ok = true;
+      for (int k = blockIdx.x; k < p.n_items && ok; k += gridDim.x, ++n) {
+        const Item it = item_at(p, k);
+        for (int s = 0; s < it.T; ++s, ++g) {
           const int vs = g % kVSt;
           if (!mbar_wait(&bars->p_ready[g % kSBufs], (g / kSBufs) & 1, abort, status)) { ok = false; break; }
           if (!mbar_wait(&bars->v_full[vs], (g / kVSt) & 1, abort, status)) { ok = false; break; }
@@ -489,39 +506,12 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     (s > 0 || ks > 0) ? 1u : 0u);
           }
           umma_commit(&bars->v_empty[vs]);
+          umma_commit(&bars->pv_done[g % kSBufs]);
           if (s == it.T - 1) umma_commit(&bars->o_full);
-          // S(g + 3) reuses the buffer that P(g) V(g), queued before it, reads
-          if (s + kSBufs < it.T && !issue_s(g + kSBufs, it, s + kSBufs)) { ok = false; break; }
         }
       }
-      umma_commit(&bars->drain);
-      mbar_wait_drain(&bars->drain, 0);
-    }
-  } else if (kSpread && warp == kWarpQ2) {
-    // ------------------------------------------------------------------ Q2 writer (warp 11)
-    // Once query tile n has landed, Q2 = q o q in the same swizzled layout (the square is taken
-    // elementwise, so the 128-byte swizzle carries over), published to the tensor core by a proxy
-    // fence and an arrival on q2_full.  The MMA waits for it at the item's first chunk step; the
-    // query tile of item n + 1 is loaded only after every product of item n (so every read of Q2)
-    // has completed, so Q2 is free when q_full announces the next tile.
-    int n = 0;
-    for (int k = blockIdx.x; k < p.n_items; k += gridDim.x, ++n) {
-      const bool w_ok = mbar_wait(&bars->q_full, n & 1, abort, status);
-      if (!__all_sync(0xffffffffu, w_ok)) break;
-      const uint4* src = reinterpret_cast<const uint4*>(sQ);
-      uint4* dst = reinterpret_cast<uint4*>(sQ2);
-#pragma unroll 1
-      for (int i = lane; i < kTile / 16; i += 32) {
-        uint4 v = src[i];
-        v.x = square_bf16x2(v.x);
-        v.y = square_bf16x2(v.y);
-        v.z = square_bf16x2(v.z);
-        v.w = square_bf16x2(v.w);
-        dst[i] = v;
-      }
-      fence_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->q2_full);
+      umma_commit(&bars->drain_pv);
+      mbar_wait_drain(&bars->drain_pv, 0);
     }
   } else if (warp < 8) {
     // ------------------------------------------------------------------ softmax (warps 0-7)
@@ -536,6 +526,28 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       const Item it = item_at(p, k);
       float mref = -INFINITY, l = 0.f;                       // -inf: no step of this warpgroup yet
       bool ok = true;
+      if (kSpread) {
+        // Q2 = q o q of this item in the query tile's swizzled layout (the square is elementwise, so
+        // the 128-byte swizzle carries over), written by both warpgroups once the tile has landed and
+        // published to the tensor core by a proxy fence and an arrival on q2_full.  The score
+        // issuer waits for it at the item's first chunk step; the next query tile loads only after
+        // the item's last score tile, the last reader of Q2, has completed.
+        const bool q_ok = mbar_wait(&bars->q_full, n & 1, abort, status);
+        if (!__all_sync(0xffffffffu, q_ok)) break;
+        const uint4* src = reinterpret_cast<const uint4*>(sQ);
+        uint4* dst = reinterpret_cast<uint4*>(sQ2);
+#pragma unroll 1
+        for (int i = tid; i < kTile / 16; i += 256) {
+          uint4 v = src[i];
+          v.x = square_bf16x2(v.x);
+          v.y = square_bf16x2(v.y);
+          v.z = square_bf16x2(v.z);
+          v.w = square_bf16x2(v.w);
+          dst[i] = v;
+        }
+        fence_async_smem();
+        mbar_arrive(&bars->q2_full);
+      }
       for (int s = (int)((X - g0) & 1u); s < it.T; s += 2) {
         const uint32_t g = g0 + s;
         // every phase of this warpgroup's b_full slots and s_full barriers is waited, in order

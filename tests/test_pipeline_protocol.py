@@ -24,18 +24,21 @@ bias-row rings; softmax warpgroup X taking the steps g with g & 1 == X; three
 score buffers in TMEM, step g's S (and then P, written over it) in buffer
 g mod 3, and one accumulator O shared by both warpgroups, which exponentiate
 against a reference max that the item's first step publishes to the other
-warpgroup.  The tensor core executes in issue order, so S(g + 3) is queued after
-P(g) V(g), which reads the buffer.  At the end of an item the two warpgroups
-exchange their row sums through a double-buffered shared array and each reads
-half of O.  The compensation chunks are written by an earlier kernel, so they
+warpgroup.  Two threads issue to the tensor core: the score issuer (S(g) once
+its key tile has landed and P(g - 3) V(g - 3) has completed) and the product
+issuer (P(g) V(g) once P(g) is written); each thread's products execute in its
+issue order, but nothing orders one thread's products against the other's, so
+the model keeps one in-order queue per issuer and completes them in any
+interleaving.  At the end of an item the two warpgroups exchange their row sums
+through a double-buffered shared array and each reads half of O.  The compensation chunks are written by an earlier kernel, so they
 are plain inputs here.
 
 The variance-corrected mode (spread=True) changes three things: a chunk step's
 score tile reads two key-ring tiles (the centroid chunk and the chunk of the
 scaled spread), so the key ring counts tiles, not steps; the value ring has
-two slots; and an otherwise idle warp writes the squared query tile Q2 for each
-item (after the query tile has landed), which the first chunk step of the item
-waits for.
+two slots; and both softmax warpgroups write their half of the squared query
+tile Q2 at the start of each item (after the query tile has landed), which the
+first chunk step of the item waits for.
 """
 import random
 
@@ -93,7 +96,7 @@ class Machine:
         self.q2_no_wait = q2_no_wait           # planted: Q2 written without waiting for the query tile
         self.mma_no_q2_wait = mma_no_q2_wait   # planted: chunk scores issued without waiting for Q2
         self.chunk_frees_one_tile = chunk_frees_one_tile   # planted: a chunk step frees only its first key tile
-        self.s_before_pv = s_before_pv         # planted: S(g + 3) queued before P(g) V(g)
+        self.s_before_pv = s_before_pv         # planted: S(g + 3) issued without waiting for P(g) V(g)
         self.no_mref_wait = no_mref_wait       # planted: the second warpgroup reads the reference unpublished
         self.no_o_free_wait = no_o_free_wait   # planted: an item's first product without waiting for O's readers
         self.lazy_v_wait = lazy_v_wait         # planted: value lane waits for a free slot only at chunk steps
@@ -107,12 +110,13 @@ class Machine:
         self.k_empty = [B(f"k_empty{i}", 1) for i in range(KSTAGES)]
         self.v_full = [B(f"v_full{i}", 1) for i in range(self.vstages)]
         self.v_empty = [B(f"v_empty{i}", 1) for i in range(self.vstages)]
-        self.q2_full = B("q2_full", 1)
+        self.q2_full = B("q2_full", 2)         # one arrival per softmax warpgroup
         self.b_full = [B(f"b_full{i}", 1) for i in range(BSTAGES)]
         self.b_empty = [B(f"b_empty{i}", 1) for i in range(BSTAGES)]
         self.version = {}                      # buffer -> step whose tile it holds
         self.s_full = [B(f"s_full{i}", 1) for i in range(2 * SBUFS)]   # [g mod 6]
         self.p_ready = [B(f"p_ready{i}", 1) for i in range(SBUFS)]     # [g mod 3]
+        self.pv_done = [B(f"pv_done{i}", 1) for i in range(SBUFS)]     # [g mod 3]
         self.o_full = B("o_full", 1)
         self.o_free = B("o_free", 2)           # one arrival per warpgroup (128 threads each)
         self.mref_full = [B(f"mref_full{i}", 1) for i in range(2)]
@@ -122,7 +126,7 @@ class Machine:
         self.xch_full = [[B(f"xch_full{j}{i}", 1) for i in range(2)] for j in range(2)]
         self.xch = [[None, None], [None, None]]   # [item parity][warpgroup] -> item whose (max, sum) it holds
         self.o_content = None                  # (item, products accumulated), at execution
-        self.tc_queue = []                     # in-order tensor core: ("mma", reads, writes) / ("commit", bar)
+        self.tc_queues = {"s": [], "pv": []}   # per issuer, in order: ("mma", ...) / ("commit", bar)
         self.tma = []                          # in flight: (bar, buffer written, buffers read)
         self.readers = {}                      # resource -> units with an operation in flight on it
 
@@ -134,28 +138,35 @@ class Machine:
         self.readers[res].remove(unit)
 
     def _write(self, res, who, unit=None):
-        """A write by `unit`; the tensor core executes its own queue in issue order, so its earlier
-        operations on the same buffer are not a hazard for its later ones."""
-        busy = [u for u in self.readers.get(res, []) if not (unit == "tc" and u == "tc")]
+        """A write by `unit`; an issuer's products execute in its issue order, so its earlier
+        operations on the same buffer are not a hazard for its later ones (the other issuer's are)."""
+        busy = [u for u in self.readers.get(res, []) if not (unit is not None and unit.startswith("tc") and u == unit)]
         assert not busy, f"{who} overwrites {res} while {busy} use it"
 
     # ---- asynchronous units
-    def tc_issue_mma(self, reads, writes, expect=None, produce=None, on_exec=None):
-        """Queue a product.  expect: {buffer: version it must hold when the product executes};
-        produce: {buffer: version it holds afterwards}; on_exec: a callback run at execution."""
+    def tc_issue_mma(self, q, reads, writes, expect=None, produce=None, on_exec=None):
+        """Queue a product on issuer q's queue.  expect: {buffer: version it must hold when the
+        product executes}; produce: {buffer: version it holds afterwards}; on_exec: a callback run
+        at execution."""
         for w in writes:
-            self._write(w, "tensor core", unit="tc")
+            self._write(w, "tensor core", unit=f"tc{q}")
         for r in reads + writes:     # the destination is busy until the MMA completes
-            self._start_read(r, "tc")
-        self.tc_queue.append(("mma", (reads + writes, expect or {}, produce or {}, on_exec)))
+            self._start_read(r, f"tc{q}")
+        self.tc_queues[q].append(("mma", (reads + writes, expect or {}, produce or {}, on_exec)))
 
-    def tc_commit(self, bar):
-        self.tc_queue.append(("commit", bar))
+    def tc_commit(self, q, bar):
+        self.tc_queues[q].append(("commit", bar))
+
+    @property
+    def tc_busy(self):
+        return any(self.tc_queues.values())
 
     def step_units(self):
         progressed = False
-        if self.tc_queue and self.rng.random() < 0.5:
-            kind, x = self.tc_queue.pop(0)
+        live = [q for q, v in self.tc_queues.items() if v]
+        if live and self.rng.random() < 0.5:
+            q = self.rng.choice(live)
+            kind, x = self.tc_queues[q].pop(0)
             if kind == "mma":
                 bufs, expect, produce, on_exec = x
                 for b, v in expect.items():
@@ -165,7 +176,7 @@ class Machine:
                 if on_exec:
                     on_exec()
                 for r in bufs:
-                    self._end_read(r, "tc")
+                    self._end_read(r, f"tc{q}")
             else:
                 x.arrive()
             progressed = True
@@ -232,25 +243,17 @@ class Machine:
                 self.tma_load(self.v_full[vs], f"V{vs}", g)
                 g += 1
 
-    def q2_writer(self):
-        """Warp 11 in the variance-corrected mode: Q2 = Q o Q (generic stores) once Q has landed."""
-        for n, nsel in enumerate(self.items):
-            if not self.q2_no_wait:
-                yield lambda: self.q_full.test(n)
-            assert "tma" not in self.readers.get("Q", []), "Q read by the Q2 writer before it landed"
-            self.holds("Q", n)
-            self._write("Q2", "Q2 writer")
-            self.version["Q2"] = n
-            self.q2_full.arrive()
-
-    def mma(self):
+    def s_issuer(self):
         g = 0
         kt = 0                                  # key-ring tiles consumed
         for n, nsel in enumerate(self.items):
             T = nsel + self.nchunk
-
-            def issue_s(s, gs):
-                nonlocal kt
+            yield lambda: self.q_full.test(n)
+            self.holds("Q", n)
+            for s in range(T):
+                b = g % SBUFS
+                if g >= SBUFS and not self.s_before_pv:
+                    yield lambda: self.pv_done[b].test(g // SBUFS - 1)
                 reads = ["Q"]
                 for _ in range(self.tiles_of(s, nsel)):
                     t = kt
@@ -261,25 +264,23 @@ class Machine:
                 if self.tiles_of(s, nsel) == 2:
                     if s == nsel and not self.mma_no_q2_wait:
                         yield lambda: self.q2_full.test(n)
-                    self.holds("Q2", n)
-                    reads.append("Q2")
-                b = gs % SBUFS
-                self.tc_issue_mma(reads, [f"S{b}"], produce={f"S{b}": ("S", gs)})
-                self.tc_commit(self.s_full[gs % (2 * SBUFS)])
+                    for h in (0, 1):
+                        self.holds(f"Q2h{h}", n)
+                        reads.append(f"Q2h{h}")
+                self.tc_issue_mma("s", reads, [f"S{b}"], produce={f"S{b}": ("S", g)})
+                self.tc_commit("s", self.s_full[g % (2 * SBUFS)])
                 freed = reads[1:2] if self.chunk_frees_one_tile else [r for r in reads if r.startswith("K")]
                 for r in freed:
-                    self.tc_commit(self.k_empty[int(r[1:])])
+                    self.tc_commit("s", self.k_empty[int(r[1:])])
                 if s == T - 1:
-                    self.tc_commit(self.q_empty)
+                    self.tc_commit("s", self.q_empty)
+                g += 1
 
-            yield lambda: self.q_full.test(n)
-            self.holds("Q", n)
-            pending = []                        # S issues postponed by the planted order
-            for j in range(min(SBUFS, T)):
-                yield from issue_s(j, g + j)
+    def pv_issuer(self):
+        g = 0
+        for n, nsel in enumerate(self.items):
+            T = nsel + self.nchunk
             for s in range(T):
-                if self.s_before_pv and s + SBUFS < T:
-                    yield from issue_s(s + SBUFS, g + SBUFS)
                 vs = g % self.vstages
                 yield lambda: self.p_ready[g % SBUFS].test(g // SBUFS)
                 yield lambda: self.v_full[vs].test(g // self.vstages)
@@ -289,19 +290,27 @@ class Machine:
 
                 def count(n=n, s=s):
                     self.o_content = (n, 1) if s == 0 else (n, self.o_content[1] + 1)
-                self.tc_issue_mma([f"S{g % SBUFS}", f"V{vs}"], ["O"], expect={f"S{g % SBUFS}": ("P", g)},
+                self.tc_issue_mma("pv", [f"S{g % SBUFS}", f"V{vs}"], ["O"], expect={f"S{g % SBUFS}": ("P", g)},
                                   on_exec=count)
-                self.tc_commit(self.v_empty[vs])
+                self.tc_commit("pv", self.v_empty[vs])
+                self.tc_commit("pv", self.pv_done[g % SBUFS])
                 if s == T - 1:
-                    self.tc_commit(self.o_full)
-                if not self.s_before_pv and s + SBUFS < T:
-                    yield from issue_s(s + SBUFS, g + SBUFS)
+                    self.tc_commit("pv", self.o_full)
                 g += 1
 
     def softmax(self, X):
         g0 = 0
         for n, nsel in enumerate(self.items):
             T = nsel + self.nchunk
+            if self.spread:
+                # this warpgroup's half of Q2 = Q o Q (generic stores) once Q has landed
+                if not self.q2_no_wait:
+                    yield lambda: self.q_full.test(n)
+                assert "tma" not in self.readers.get("Q", []), "Q read by the Q2 writer before it landed"
+                self.holds("Q", n)
+                self._write(f"Q2h{X}", "Q2 writer")
+                self.version[f"Q2h{X}"] = n
+                self.q2_full.arrive()
             steps = list(range((X - g0) & 1, T, 2))
             for s in steps:
                 g = g0 + s
@@ -337,7 +346,7 @@ class Machine:
                 yield lambda: self.xch_full[n & 1][X ^ 1].test(n >> 1)
             assert self.xch[slot][X ^ 1] == n, f"exchange slot holds item {self.xch[slot][X ^ 1]}, read for item {n}"
             # this warpgroup's half of O is read over a span in which the other roles move on
-            assert "tc" not in self.readers.get("O", []), "O read while a product into it is in flight"
+            assert "tcpv" not in self.readers.get("O", []), "O read while a product into it is in flight"
             assert self.o_content == (n, T), f"O holds {self.o_content} at the end of item {n}"
             self._start_read("O", f"epilogue{X}")
             for _ in range(self.rng.randrange(1, 40)):  # a read of random length
@@ -348,13 +357,12 @@ class Machine:
             g0 += T
 
     def run(self, max_iters=200000):
-        roles = [self.producer(), self.producer_v(), self.mma(), self.softmax(0), self.softmax(1)]
-        if self.spread:
-            roles.append(self.q2_writer())
+        roles = [self.producer(), self.producer_v(), self.s_issuer(), self.pv_issuer(), self.softmax(0),
+                 self.softmax(1)]
         waits = [None] * len(roles)
         done = [False] * len(roles)
         for _ in range(max_iters):
-            if all(done) and not self.tc_queue and not self.tma:
+            if all(done) and not self.tc_busy and not self.tma:
                 return True
             order = list(range(len(roles)))
             self.rng.shuffle(order)
@@ -373,7 +381,7 @@ class Machine:
                 if self.rng.random() < 0.5:
                     break
             progressed = self.step_units() or progressed
-            if not progressed and not self.tc_queue and not self.tma:
+            if not progressed and not self.tc_busy and not self.tma:
                 raise AssertionError("deadlock: no role can progress")
         raise AssertionError("did not finish")
 
@@ -428,8 +436,9 @@ def test_model_catches_an_epilogue_that_does_not_wait_for_the_last_product():
     assert _caught([3, 4, 1], 2, no_final_wait=True) > 0
 
 
-def test_model_catches_a_score_tile_queued_before_the_product_that_reads_its_buffer():
-    """S(g + 3) goes into the buffer that holds P(g): queued before P(g) V(g), it overwrites P."""
+def test_model_catches_a_score_tile_issued_before_the_product_that_reads_its_buffer_completes():
+    """S(g + 3) goes into the buffer that holds P(g); the two issuers' products are not ordered, so
+    without waiting for P(g) V(g) to complete it can overwrite P(g) first."""
     assert _caught([5, 2, 4], 2, s_before_pv=True) > 0
 
 
