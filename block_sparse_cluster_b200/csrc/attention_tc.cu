@@ -355,13 +355,17 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
               if (pi > 0.f) w = -__log2f(pi);
               else ncol = 0;               // a block that is never included: left out
             }
-            bars->bflag[bs] = (ncol == kBN && !p.incl) ? 1 : 0;
-            float4* bb = reinterpret_cast<float4*>(sBias + bs * kBN);
+            const bool full = ncol == kBN && !p.incl && p.scale_log2 > 0.f;
+            bars->bflag[bs] = full ? 1 : 0;
+            if (!full) {
+              // (a full block's row would be all zero: the softmax does not read it)
+              float4* bb = reinterpret_cast<float4*>(sBias + bs * kBN);
 #pragma unroll 4
-            for (int c4 = 0; c4 < kBN / 4; ++c4) {
-              const int c = 4 * c4;
-              bb[c4] = make_float4(c < ncol ? w : -INFINITY, c + 1 < ncol ? w : -INFINITY,
-                                   c + 2 < ncol ? w : -INFINITY, c + 3 < ncol ? w : -INFINITY);
+              for (int c4 = 0; c4 < kBN / 4; ++c4) {
+                const int c = 4 * c4;
+                bb[c4] = make_float4(c < ncol ? w : -INFINITY, c + 1 < ncol ? w : -INFINITY,
+                                     c + 2 < ncol ? w : -INFINITY, c + 3 < ncol ? w : -INFINITY);
+              }
             }
             mbar_arrive(&bars->b_full[bs]);
           } else {
