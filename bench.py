@@ -360,8 +360,7 @@ def run_spread(args):
     split = {name: sum(e[i].elapsed_time(e[i + 1]) for e in evs) / args.steps
              for i, name in enumerate(("reassign", "cluster_spread", "attention_spread"))}
     print(json.dumps({
-        "metric": "effective TFLOP/s & ms/call of reassign + cluster spread + variance-corrected attention "
-                  "(CUDA-core path)",
+        "metric": "effective TFLOP/s & ms/call of reassign + cluster spread + variance-corrected attention",
         "value": eff / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms, "steps": args.steps,
         "warmup": args.warmup, "higher_is_better": True, "dtype": {"bf16": "bf16", "f32": "f32"}[w.dtype],
         "data": "synthetic", "breakdown_ms": split, "effective_flop_per_step": eff,
