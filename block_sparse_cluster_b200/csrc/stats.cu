@@ -176,23 +176,57 @@ __global__ void __launch_bounds__(128) cluster_spread_kernel(const T* __restrict
 #pragma unroll
   for (int i = 0; i < NS; ++i) acc[i] = 0.f;
   const size_t hb = (size_t)bh * nB;
-  for (int j = 0; j < nB; ++j) {
-    if (st.seg_idx[(hb + j) * C + c] == 0xFF) continue;      // warp-uniform
-    const int k0 = j * block;
-    const int nk = min(block, N - k0);
-    for (int kb = 0; kb < nk; kb += 32) {
-      const int kk = kb + lane;
-      const bool mine = kk < nk && st.assign[(size_t)bh * N + k0 + kk] == c;
-      unsigned msk = __ballot_sync(0xffffffffu, mine);
-      while (msk) {
-        const int b = __ffs(msk) - 1;
-        msk &= msk - 1u;
-        float kv[NS];
-        load_vec(K + ((size_t)bh * N + k0 + kb + b) * D + lane * NS, kv, NS);
+  const int32_t* arow = st.assign + (size_t)bh * N;
+  const T* krow = K + (size_t)bh * N * D + lane * NS;
+  // Blocks are looked up 32 at a time (lane u: block j0 + u); in each block holding the cluster,
+  // its keys are found from the block's assignments (four independent loads) and their rows are
+  // loaded up to eight at a time, then added in key order: the order of a plain walk over the
+  // blocks and their keys.
+  constexpr int kRows = 8;
+  for (int j0 = 0; j0 < nB; j0 += 32) {
+    const int jl = j0 + lane;
+    unsigned pm = __ballot_sync(0xffffffffu, jl < nB && st.seg_idx[(hb + jl) * C + c] != 0xFF);
+    while (pm) {
+      const int j = j0 + __ffs(pm) - 1;
+      pm &= pm - 1u;
+      const int k0 = j * block;
+      const int nk = min(block, N - k0);
+      unsigned km[4];
 #pragma unroll
-        for (int i = 0; i < NS; ++i) {
-          const float dv = kv[i] - cb[i];
-          acc[i] = fmaf(dv, dv, acc[i]);
+      for (int q = 0; q < 4; ++q) {
+        const int kk = 32 * q + lane;
+        km[q] = __ballot_sync(0xffffffffu, kk < nk && arow[k0 + kk] == c);
+      }
+      // the cluster's keys of the block, in index order: keys 0-63 in lo, 64-127 in hi
+      unsigned long long lo = (unsigned long long)km[0] | ((unsigned long long)km[1] << 32);
+      unsigned long long hi = (unsigned long long)km[2] | ((unsigned long long)km[3] << 32);
+      while (lo | hi) {
+        int idx[kRows];
+#pragma unroll
+        for (int r = 0; r < kRows; ++r) {
+          int k = -1;
+          if (lo) {
+            k = __ffsll((long long)lo) - 1;
+            lo &= lo - 1ull;
+          } else if (hi) {
+            k = 64 + __ffsll((long long)hi) - 1;
+            hi &= hi - 1ull;
+          }
+          idx[r] = k;
+        }
+        float kv[kRows][NS];
+#pragma unroll
+        for (int r = 0; r < kRows; ++r)
+          if (idx[r] >= 0) load_vec(krow + (size_t)(k0 + idx[r]) * D, kv[r], NS);
+#pragma unroll
+        for (int r = 0; r < kRows; ++r) {
+          if (idx[r] >= 0) {
+#pragma unroll
+            for (int i = 0; i < NS; ++i) {
+              const float dv = kv[r][i] - cb[i];
+              acc[i] = fmaf(dv, dv, acc[i]);
+            }
+          }
         }
       }
     }
