@@ -89,6 +89,7 @@ constexpr int kWarpPV = 11;              // product issuer
 constexpr int kRegSoftmax = 232, kRegIssue = 40;
 static_assert(128 * (2 * kRegSoftmax + kRegIssue) <= kThreads * 168, "register split above the launch");
 static_assert(kBStages % 2 == 0, "a bias slot must always serve the same softmax warpgroup");
+static_assert(kVStages == kSBufs, "a value tile lands on the P-ready barrier of its score buffer");
 constexpr int kChunkBytes = kTile + kBN * 4;   // compensation chunk: vbar^U rows, then log2 n^U
 
 struct __align__(8) Bars {
@@ -284,7 +285,9 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     }
     for (int b = 0; b < 2 * kSBufs; ++b) mbar_init(&bars->s_full[b], 1);
     for (int b = 0; b < kSBufs; ++b) {
-      mbar_init(&bars->p_ready[b], 128);
+      // outside the variance-corrected mode the value tile of step g lands on p_ready[g mod 3]
+      // too: the value producer's arrival (with its bytes) joins the softmax warpgroup's 128
+      mbar_init(&bars->p_ready[b], kSpread ? 128 : 129);
       mbar_init(&bars->pv_done[b], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -413,23 +416,29 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           const int vs = g % kVSt;
           if (!mbar_wait(&bars->v_empty[vs], ((g / kVSt) & 1) ^ 1, abort, status)) { ok = false; break; }
           uint8_t* dv = sV + vs * kTile;
+          // Outside the variance-corrected mode the tile lands on p_ready[g mod 3] (the ring and the
+          // score buffers have the same three slots, and the slot is free only once P(g-3) V(g-3)
+          // has completed, so that barrier is in step g's phase), and the product issuer waits on
+          // one barrier for both P(g) and V(g).
+          uint64_t* landed = kSpread ? &bars->v_full[vs] : &bars->p_ready[g % kSBufs];
           if (s < it.nsel || p.incl) {
             bool valid;
             const int j = block_of(p, it, s, &valid);
-            mbar_expect_tx(&bars->v_full[vs], kTile);
-            tma_load_3d(dv, &tm_v, &bars->v_full[vs], 0, j * kBN, it.bh);
-            tma_load_3d(dv + kPanel, &tm_v, &bars->v_full[vs], 64, j * kBN, it.bh);
+            mbar_expect_tx(landed, kTile);
+            tma_load_3d(dv, &tm_v, landed, 0, j * kBN, it.bh);
+            tma_load_3d(dv + kPanel, &tm_v, landed, 64, j * kBN, it.bh);
           } else {
             const int z = (it.bh * p.nB + it.i) * p.nchunk + (s - it.nsel);
-            mbar_expect_tx(&bars->v_full[vs], kTile);
-            tma_load_3d(dv, &tm_p, &bars->v_full[vs], 0, 0, z);
-            tma_load_3d(dv + kPanel, &tm_p, &bars->v_full[vs], 64, 0, z);
+            mbar_expect_tx(landed, kTile);
+            tma_load_3d(dv, &tm_p, landed, 0, 0, z);
+            tma_load_3d(dv + kPanel, &tm_p, landed, 64, 0, z);
           }
         }
         if (!ok) break;
       }
       for (uint32_t gd = g >= kVSt ? g - kVSt : 0; gd < g; ++gd)
-        mbar_wait_drain(&bars->v_full[gd % kVSt], (gd / kVSt) & 1);
+        mbar_wait_drain(kSpread ? &bars->v_full[gd % kVSt] : &bars->p_ready[gd % kSBufs],
+                        (gd / kVSt) & 1);
     }
   } else if (warp == kWarpMMA) {
     // ------------------------------------------------------------------ score issuer
@@ -497,7 +506,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         for (int s = 0; s < it.T; ++s, ++g) {
           const int vs = g % kVSt;
           if (!mbar_wait(&bars->p_ready[g % kSBufs], (g / kSBufs) & 1, abort, status)) { ok = false; break; }
-          if (!mbar_wait(&bars->v_full[vs], (g / kVSt) & 1, abort, status)) { ok = false; break; }
+          if (kSpread && !mbar_wait(&bars->v_full[vs], (g / kVSt) & 1, abort, status)) { ok = false; break; }
           if (s == 0 && !mbar_wait(&bars->o_free, (n & 1) ^ 1, abort, status)) { ok = false; break; }
           tc_fence_after();
           const uint32_t vb = smem_u32(sV + vs * kTile);

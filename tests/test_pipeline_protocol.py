@@ -20,7 +20,9 @@ interleavings, and checks that
 
 It mirrors the step structure of attention_tc.cu: per work item, one step per
 selected block followed by one step per 128-cluster chunk; key, value and
-bias-row rings; softmax warpgroup X taking the steps g with g & 1 == X; three
+bias-row rings (outside the variance-corrected mode a value tile lands on the
+P-ready barrier of its score buffer, so one wait covers both); softmax warpgroup
+X taking the steps g with g & 1 == X; three
 score buffers in TMEM, step g's S (and then P, written over it) in buffer
 g mod 3, and one accumulator O shared by both warpgroups, which exponentiate
 against a reference max that the item's first step publishes to the other
@@ -115,7 +117,8 @@ class Machine:
         self.b_empty = [B(f"b_empty{i}", 1) for i in range(BSTAGES)]
         self.version = {}                      # buffer -> step whose tile it holds
         self.s_full = [B(f"s_full{i}", 1) for i in range(2 * SBUFS)]   # [g mod 6]
-        self.p_ready = [B(f"p_ready{i}", 1) for i in range(SBUFS)]     # [g mod 3]
+        # [g mod 3]; outside the variance-corrected mode the value tile of step g lands on it too
+        self.p_ready = [B(f"p_ready{i}", 1 if spread else 2) for i in range(SBUFS)]
         self.pv_done = [B(f"pv_done{i}", 1) for i in range(SBUFS)]     # [g mod 3]
         self.o_full = B("o_full", 1)
         self.o_free = B("o_free", 2)           # one arrival per warpgroup (128 threads each)
@@ -239,8 +242,9 @@ class Machine:
                 vs = g % self.vstages
                 if not self.lazy_v_wait or s >= nsel:
                     yield lambda: self.v_empty[vs].test(g // self.vstages - 1)
-                self.v_full[vs].expect_tx(1)
-                self.tma_load(self.v_full[vs], f"V{vs}", g)
+                landed = self.v_full[vs] if self.spread else self.p_ready[g % SBUFS]
+                landed.expect_tx(1)
+                self.tma_load(landed, f"V{vs}", g)
                 g += 1
 
     def s_issuer(self):
@@ -283,7 +287,8 @@ class Machine:
             for s in range(T):
                 vs = g % self.vstages
                 yield lambda: self.p_ready[g % SBUFS].test(g // SBUFS)
-                yield lambda: self.v_full[vs].test(g // self.vstages)
+                if self.spread:
+                    yield lambda: self.v_full[vs].test(g // self.vstages)
                 if s == 0 and not self.no_o_free_wait:
                     yield lambda: self.o_free.test(n - 1)
                 self.holds(f"V{vs}", g)
