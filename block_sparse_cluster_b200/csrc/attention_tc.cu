@@ -288,7 +288,10 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       // outside the variance-corrected mode the value tile of step g lands on p_ready[g mod 3]
       // too: the value producer's arrival (with its bytes) joins the softmax warpgroup's 128
       mbar_init(&bars->p_ready[b], kSpread ? 128 : 129);
-      mbar_init(&bars->pv_done[b], 1);
+      // outside the variance-corrected mode the key tile of step g lands on pv_done[g mod 3] too
+      // (the commit of P(g-3) V(g-3) and the key producer's arrival with the tile's bytes); the
+      // first phase of each stands for a product before the first step
+      mbar_init(&bars->pv_done[b], kSpread ? 1 : 2);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars->mref_full[b], 128);
@@ -298,6 +301,8 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     mbar_init(&bars->o_full, 1);
     mbar_init(&bars->o_free, 256);
     mbar_init(&bars->drain, 1);
+    if (!kSpread)
+      for (int b = 0; b < kSBufs; ++b) mbar_arrive(&bars->pv_done[b]);
     mbar_init(&bars->drain_pv, 1);
     bars->abort = 0;
     fence_mbar_init();
@@ -342,12 +347,16 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           if (!mbar_wait(&bars->k_empty[ks], ((kt / kKStages) & 1) ^ 1, abort, status)) { ok = false; break; }
           uint8_t* dk = sK + ks * kTile;
           ++kt;
+          // Outside the variance-corrected mode the tile lands on pv_done[g mod 3]: a key slot is free
+          // only once S(g-2) has completed, so P(g-6) V(g-6) has (S(g-3) waited for it) and that
+          // barrier is in step g's phase; the score issuer then waits on one barrier for both.
+          uint64_t* klanded = kSpread ? &bars->k_full[ks] : &bars->pv_done[g % kSBufs];
           if (s < it.nsel || p.incl) {
             bool valid;
             const int j = block_of(p, it, s, &valid);
-            mbar_expect_tx(&bars->k_full[ks], kTile);
-            tma_load_3d(dk, &tm_k, &bars->k_full[ks], 0, j * kBN, it.bh);
-            tma_load_3d(dk + kPanel, &tm_k, &bars->k_full[ks], 64, j * kBN, it.bh);
+            mbar_expect_tx(klanded, kTile);
+            tma_load_3d(dk, &tm_k, klanded, 0, j * kBN, it.bh);
+            tma_load_3d(dk + kPanel, &tm_k, klanded, 64, j * kBN, it.bh);
             // bias row of a key block: 0 for its keys, -inf past the end of a short last block
             // (generic stores, published to the softmax by the arrive on b_full)
             if (!mbar_wait(&bars->b_empty[bs], ((g / kBStages) & 1) ^ 1, abort, status)) { ok = false; break; }
@@ -373,9 +382,9 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             mbar_arrive(&bars->b_full[bs]);
           } else {
             const int c = s - it.nsel;
-            mbar_expect_tx(&bars->k_full[ks], kTile);
-            tma_load_3d(dk, &tm_c, &bars->k_full[ks], 0, c * kBN, it.bh);
-            tma_load_3d(dk + kPanel, &tm_c, &bars->k_full[ks], 64, c * kBN, it.bh);
+            mbar_expect_tx(klanded, kTile);
+            tma_load_3d(dk, &tm_c, klanded, 0, c * kBN, it.bh);
+            tma_load_3d(dk + kPanel, &tm_c, klanded, 64, c * kBN, it.bh);
             if (kSpread) {
               // the chunk's rows of Dh, into the next key-ring slot
               const int kd = kt % kKStages;
@@ -398,7 +407,8 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       // otherwise the consumers have waited for every load)
       if (nq > 0) mbar_wait_drain(&bars->q_full, (nq - 1) & 1);
       for (uint32_t gd = kt >= kKStages ? kt - kKStages : 0; gd < kt; ++gd)
-        mbar_wait_drain(&bars->k_full[gd % kKStages], (gd / kKStages) & 1);
+        mbar_wait_drain(kSpread ? &bars->k_full[gd % kKStages] : &bars->pv_done[gd % kSBufs],
+                        kSpread ? (gd / kKStages) & 1 : (gd / kSBufs) & 1);
       for (uint32_t gd = g >= kBStages ? g - kBStages : 0; gd < g; ++gd)
         mbar_wait_drain(&bars->b_full[gd % kBStages], (gd / kBStages) & 1);
     }
@@ -455,11 +465,21 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         for (int s = 0; s < it.T; ++s, ++g) {
           // S_(g mod 3) last held S(g - 3): its product must have read P(g - 3); every phase of
           // pv_done[g mod 3] is waited, in order
-          if (g >= (uint32_t)kSBufs &&
-              !mbar_wait(&bars->pv_done[g % kSBufs], ((g / kSBufs) & 1) ^ 1, abort, status)) { ok = false; break; }
+          // (outside the variance-corrected mode the same barrier also says that the key tile of
+          // step g has landed; its first phase stands for a product before the first step)
+          if (!kSpread) {
+            if (!mbar_wait(&bars->pv_done[g % kSBufs], (g / kSBufs) & 1, abort, status)) { ok = false; break; }
+          } else if (g >= (uint32_t)kSBufs &&
+                     !mbar_wait(&bars->pv_done[g % kSBufs], ((g / kSBufs) & 1) ^ 1, abort, status)) {
+            ok = false;
+            break;
+          }
           const bool two = kSpread && !p.incl && s >= it.nsel;
           const uint32_t t0 = kSpread ? kt : g;   // one tile per step outside the corrected mode
-          if (!mbar_wait(&bars->k_full[t0 % kKStages], (t0 / kKStages) & 1, abort, status)) { ok = false; break; }
+          if (kSpread && !mbar_wait(&bars->k_full[t0 % kKStages], (t0 / kKStages) & 1, abort, status)) {
+            ok = false;
+            break;
+          }
           if (two) {
             const uint32_t t1 = t0 + 1;
             if (!mbar_wait(&bars->k_full[t1 % kKStages], (t1 / kKStages) & 1, abort, status)) { ok = false; break; }
