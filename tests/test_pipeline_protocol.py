@@ -89,7 +89,7 @@ class Machine:
     def __init__(self, items, nchunk, rng, lazy_v_wait=False, skip_b_empty=False, single_xch=False,
                  no_final_wait=False, single_xch_barrier=False, spread=False, q2_no_wait=False,
                  mma_no_q2_wait=False, chunk_frees_one_tile=False, s_before_pv=False, no_mref_wait=False,
-                 no_o_free_wait=False):
+                 no_o_free_wait=False, key_on_own_barrier=False):
         self.items = items                     # list of nsel per item of one CTA
         self.nchunk = nchunk
         self.rng = rng
@@ -101,6 +101,7 @@ class Machine:
         self.s_before_pv = s_before_pv         # planted: S(g + 3) issued without waiting for P(g) V(g)
         self.no_mref_wait = no_mref_wait       # planted: the second warpgroup reads the reference unpublished
         self.no_o_free_wait = no_o_free_wait   # planted: an item's first product without waiting for O's readers
+        self.key_on_own_barrier = key_on_own_barrier   # planted: key tiles land on k_full, not waited
         self.lazy_v_wait = lazy_v_wait         # planted: value lane waits for a free slot only at chunk steps
         self.skip_b_empty = skip_b_empty       # planted: bias rows loaded without waiting for a free slot
         self.single_xch = single_xch           # planted: one (max, sum) exchange buffer for all items
@@ -121,7 +122,7 @@ class Machine:
         self.p_ready = [B(f"p_ready{i}", 1 if spread else 2) for i in range(SBUFS)]
         # [g mod 3]; outside the variance-corrected mode the key tile of step g lands on it too,
         # and its first phase stands for a product before the first step
-        self.pv_done = [B(f"pv_done{i}", 1 if spread else 2) for i in range(SBUFS)]
+        self.pv_done = [B(f"pv_done{i}", 1 if spread or key_on_own_barrier else 2) for i in range(SBUFS)]
         if not spread:
             for b in self.pv_done:
                 b.arrive()
@@ -158,6 +159,8 @@ class Machine:
         at execution."""
         for w in writes:
             self._write(w, "tensor core", unit=f"tc{q}")
+        for r in reads:
+            assert "tma" not in self.readers.get(r, []), f"a product reads {r} while its copy is in flight"
         for r in reads + writes:     # the destination is busy until the MMA completes
             self._start_read(r, f"tc{q}")
         self.tc_queues[q].append(("mma", (reads + writes, expect or {}, produce or {}, on_exec)))
@@ -227,7 +230,7 @@ class Machine:
                 for _ in range(self.tiles_of(s, nsel)):
                     ks = kt % KSTAGES
                     yield lambda: self.k_empty[ks].test(kt // KSTAGES - 1)
-                    landed = self.k_full[ks] if self.spread else self.pv_done[g % SBUFS]
+                    landed = self.k_full[ks] if self.spread or self.key_on_own_barrier else self.pv_done[g % SBUFS]
                     landed.expect_tx(1)
                     self.tma_load(landed, f"K{ks}", kt)
                     kt += 1
@@ -474,3 +477,9 @@ def test_one_exchange_barrier_per_warpgroup_is_safe_with_the_shared_accumulator(
     exchange barrier twice before the other's wait: the per-item-parity barriers are kept anyway."""
     assert _caught([1, 0, 0, 1], 1, single_xch_barrier=True) == 0
     assert _caught([0, 0, 2, 0, 0, 1], 1, single_xch_barrier=True) == 0
+
+
+def test_model_catches_a_key_tile_that_lands_on_a_barrier_the_score_issuer_does_not_wait():
+    """Outside the variance-corrected mode the score issuer waits only on pv_done, which the key
+    tile's bytes must complete; a tile landing on its own barrier is read while it is in flight."""
+    assert _caught([4, 3, 5], 2, key_on_own_barrier=True) > 0
