@@ -37,19 +37,31 @@ ATT_SRC = os.path.join(ROOT, "block_sparse_cluster_b200", "csrc", "attention_tc.
 ATT_PROFILE = os.path.join(ROOT, "profiles", "attention_tc_kernel_wan14b.md")
 
 
+def source_code_sha1(path: str) -> str:
+    """sha1 of a CUDA source with its comments and blank space removed: an edit of the comments
+    alone leaves it unchanged, any change of the code changes it."""
+    import hashlib
+    import re
+    text = open(path, encoding="utf-8").read()
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    text = re.sub(r"\s+", " ", text).strip()
+    return hashlib.sha1(text.encode()).hexdigest()
+
+
 def attention_traffic(w) -> "float | None":
     """DRAM bytes (read + write) per launch of attention_tc_kernel from the committed ncu summary,
-    whose record line names the workload and the sha1 of the kernel source it was captured from:
-    null for another workload or once the source has changed since the capture."""
-    import hashlib
+    whose record line names the workload and the code hash (comments aside) of the kernel source
+    it was captured from: null for another workload or once the code has changed since the
+    capture."""
     import re
     try:
         text = open(ATT_PROFILE).read()
-        sha = hashlib.sha1(open(ATT_SRC, "rb").read()).hexdigest()
+        sha = source_code_sha1(ATT_SRC)
     except OSError:
         return None
     m = re.search(r"traffic record: workload=(\w+) heads=(\d+) bytes_per_launch=([0-9.e+]+) "
-                  r"attention_tc\.cu sha1=([0-9a-f]{40})", text)
+                  r"attention_tc\.cu code-sha1=([0-9a-f]{40})", text)
     if not m or m.group(1) != w.name or int(m.group(2)) != w.H or m.group(4) != sha:
         return None
     return float(m.group(3))

@@ -25,10 +25,11 @@
 // logits): a cluster column's logit gains s^2/2 sum_t q_t^2 D_{c,t}, D_c the second moment of the
 // cluster's keys about its representative.  The correction is a second contraction into the same
 // score tile: S = Q cbar^T + Q2 Dh^T, with Q2 = q o q (bf16, written into shared memory from the
-// query tile by the softmax warpgroups) and Dh = (s/2) D (bf16, from the host side).  A chunk step therefore takes
-// two key-ring tiles (the centroid chunk, then the Dh chunk), so the key ring counts tiles, not
-// steps; the query tile Q2 takes the place of one value-ring slot (two slots in this mode).  The
-// softmax warpgroups write Q2 at the start of each item.
+// query tile by the softmax warpgroups at the start of each item) and Dh = (s/2) D (bf16, from the
+// host side).  A chunk step therefore takes two key-ring tiles (the centroid chunk, then the Dh
+// chunk), so the key ring counts tiles, not steps; the query tile Q2 takes the place of one
+// value-ring slot (two slots in this mode), and the key and value tiles land on barriers of their
+// own.
 //
 // Roles (384 threads):
 //   warps 0-3, 4-7  two softmax warpgroups X = 0, 1; warpgroup X takes the steps g with g & 1 = X
@@ -42,13 +43,17 @@
 //   warp 8     producer: loads Q, key tiles / centroid chunks (2-stage ring) and the softmax bias
 //              rows (4-stage ring, so a slot always serves the same warpgroup);
 //   warp 9     score issuer: allocates TMEM, issues tcgen05.mma S(g) = Q K^T into S_(g mod 3) as
-//              soon as its key tile has landed and P(g-3) V(g-3) has finished reading the buffer
-//              (in the variance-corrected mode both softmax warpgroups write Q2 at each item's start);
+//              soon as its key tile has landed and P(g-3) V(g-3) has finished reading the buffer;
 //   warp 10    producer of value tiles / compensation chunks (3-stage ring); a warp of its own,
 //              since divergent lanes of one warp waiting on different barriers hold each other up;
-//   warp 11    product issuer: O += P(g) V(g) once P(g) is written.  Two issuing threads keep the
-//              tensor core fed: one thread's waits on the softmax no longer hold the other's
-//              products back (issuing blocks while the tensor core's queue is full).
+//   warp 11    product issuer: O += P(g) V(g) once P(g) is written and V(g) has landed.  Two
+//              issuing threads keep the tensor core fed: one thread's waits on the softmax no
+//              longer hold the other's products back (issuing blocks while the tensor core's queue
+//              is full).
+// Outside the variance-corrected mode a tile lands on the barrier its consumer waits on anyway,
+// since every barrier operation costs a few hundred cycles here: the value tile of step g on
+// p_ready[g mod 3] (beside the softmax's arrivals) and the key tile of step g on pv_done[g mod 3]
+// (beside the commit of P(g-3) V(g-3)); the rings' slot rules put both in step g's phase.
 // TMEM columns: S_0 [0,128), S_1 [128,256), S_2 [256,384), O [384,512).  Step g's scores go to
 // S_(g mod 3): the tensor core computes S(g+1) and S(g+2) while the softmax of step g runs, and
 // S(g+3) waits for P(g) V(g) to complete (pv_done), since the two issuers' products are not ordered

@@ -99,3 +99,16 @@ def test_split_heads_partition_the_workload_with_gloo():
     for r, heads, _, _, ksum, cnt in got:
         assert abs(ksum - full.K[:, heads].sum().item()) < 1e-3 * max(1.0, abs(ksum))
         assert cnt == full.kv_cnt[:, heads].sum().item()
+
+
+def test_traffic_record_follows_the_kernel_code_not_its_comments(tmp_path):
+    """The bench line's attention traffic comes from a committed capture whose record names a hash
+    of the kernel's code: a comment edit keeps it, a code edit changes it."""
+    import bench
+    src = tmp_path / "k.cu"
+    src.write_text("// header\nint f(int x) {  /* body */\n  return x + 1;  // one\n}\n")
+    h0 = bench.source_code_sha1(str(src))
+    src.write_text("// another header\n\nint f(int x) { /* other words */ return x + 1; }\n")
+    assert bench.source_code_sha1(str(src)) == h0
+    src.write_text("int f(int x) { return x + 2; }\n")
+    assert bench.source_code_sha1(str(src)) != h0
