@@ -23,11 +23,13 @@
  * - Calls are asynchronous on the given stream (NULL = legacy default
  *   stream).  Argument checks are synchronous: a call that returns an error
  *   code launched nothing.  Problems found on the device (an out-of-range or
- *   unsorted block index, a bounded wait that gave up) are recorded in a
- *   status word inside the workspace; da_device_status() reports them.
+ *   unsorted block index, a bounded wait that gave up, logits beyond the
+ *   attention kernel's range) are recorded in a status word inside the
+ *   workspace; da_device_status() reports them.
  * - Supported sizes: d in {64, 128}; block in {64, 128}; C a multiple of 32,
  *   32 <= C <= 1024; N >= 1.  The bf16 tensor-core path needs d = 128 and
- *   block = 128; fp32 runs d in {64, 128}, block in {64, 128}.
+ *   block = 128; other bf16 sizes and fp32 run on the CUDA cores in fp32
+ *   arithmetic.
  */
 #ifndef DA_H
 #define DA_H
@@ -158,7 +160,10 @@ DA_API da_status da_mask_prepare(const da_dims* dims, const da_block_mask* mask,
  * runs over both kinds of logits with fp32 accumulation; O = [B,H,N,d] in
  * dims.dtype; lse (nullable) = [B,H,N] fp32 natural-log sum of exponentials.
  * scale <= 0 selects 1/sqrt(d).  stats must come from da_reassign on the
- * same K, V, centroids.
+ * same K, V, centroids.  On the tensor cores every row's exponentials are
+ * taken against the row max of its q-block's first step; a row whose logits
+ * in a later step exceed that max by more than 2^96 (log2 units) sets
+ * DA_ERR_RANGE in the status word, its output then unreliable.
  */
 DA_API da_status da_attention(const da_dims* dims, const void* Q, const void* K, const void* V,
                        const da_block_mask* mask, const void* centroids,
