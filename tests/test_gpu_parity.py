@@ -233,6 +233,30 @@ def test_malformed_plan_is_reported_without_fault():
     assert eng.status() == da.STATUS_NAMES.index("DA_ERR_DEVICE_INDEX")
 
 
+def test_logits_far_above_the_first_steps_max_are_reported():
+    """The tensor-core kernel exponentiates every step of a row against the row max of its
+    q-block's first step.  Queries 30 e_1 against a first block of zero keys (logits 0) and a second
+    block of keys 30 e_1 (about 115 in log2 units) exceed that reference by more than 2^96: the
+    call reports DA_ERR_RANGE through the status word, and an ordinary step after it reports
+    nothing."""
+    import dataclasses
+    import block_sparse_cluster_b200 as da
+    w = W.scaled(W.WORKLOADS["wan13b"], H=1, T=1)      # bf16, d = block = 128, 13 blocks
+    inp = W.make_inputs(w, seed=16)
+    Q = torch.zeros_like(inp.Q)
+    Q[..., 0] = 30.0
+    K = torch.zeros_like(inp.K)
+    K[0, 0, w.block:2 * w.block, 0] = 30.0
+    far = dataclasses.replace(inp, Q=Q, K=K)
+    ki = torch.empty(w.B, w.H, w.nB, 2, dtype=torch.int32)
+    ki[..., 0], ki[..., 1] = 0, 1
+    kc = torch.full_like(inp.kv_cnt, 2)
+    eng, _, _ = P.run_gpu(far, kv_idx=ki, kv_cnt=kc)
+    assert eng.status() == da.STATUS_NAMES.index("DA_ERR_RANGE")
+    eng, _, _ = P.run_gpu(inp)
+    assert eng.status() == 0
+
+
 def test_plans_longer_than_one_staging_tile():
     """Rows with more selected blocks than the compensation pre-pass stages at a time (256): every
     block but every fifth (270), every block (338, dense), and all but the first 10 and last 20
