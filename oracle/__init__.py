@@ -307,12 +307,11 @@ def sse(K, centroids, assign) -> float:
     return float(((Kf - Cf[a]) ** 2).sum())
 
 
-def lloyd_step(K, centroids) -> Tuple[np.ndarray, np.ndarray]:
-    """One Lloyd iteration: assign every key to its nearest centroid (reassign, reading R1), then
-    move each centroid to the mean of its keys; a centroid without keys stays where it is.
-    Returns (new centroids float64 [C, d], assignment int64 [N])."""
+def lloyd_update(K, centroids, assign) -> np.ndarray:
+    """The update half of a Lloyd iteration for a given assignment: each centroid moves to the
+    mean of its keys; a centroid without keys stays where it is.  Returns float64 [C, d]."""
     Kf, Cf = _f64(K), _f64(centroids)
-    a, _ = reassign(Kf, Cf)
+    a = _i64(assign)
     C = Cf.shape[0]
     n = np.bincount(a, minlength=C)
     S = np.zeros_like(Cf)
@@ -320,7 +319,15 @@ def lloyd_step(K, centroids) -> Tuple[np.ndarray, np.ndarray]:
     new = Cf.copy()
     live = n > 0
     new[live] = S[live] / n[live][:, None]
-    return new, a
+    return new
+
+
+def lloyd_step(K, centroids) -> Tuple[np.ndarray, np.ndarray]:
+    """One Lloyd iteration: assign every key to its nearest centroid (reassign, reading R1), then
+    move each centroid to the mean of its keys (lloyd_update).
+    Returns (new centroids float64 [C, d], assignment int64 [N])."""
+    a, _ = reassign(_f64(K), _f64(centroids))
+    return lloyd_update(K, centroids, a), a
 
 
 def kmeans(K, init, iters: int) -> Tuple[np.ndarray, np.ndarray]:

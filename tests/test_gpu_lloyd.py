@@ -33,13 +33,8 @@ def test_one_lloyd_step_matches_oracle(name):
         for h in range(w.H):
             a_gpu = eng.stats.assign[b, h].cpu().numpy().astype(np.int64)
             P.check_assignment(inp, b, h, a_gpu)
-            # the update given the GPU's assignment: mean of the keys of each cluster
-            Kf = inp.K[b, h].double().numpy()
-            n = np.bincount(a_gpu, minlength=w.C)
-            S = np.zeros((w.C, w.d))
-            np.add.at(S, a_gpu, Kf)
-            ref = inp.centroids[b, h].double().numpy().copy()
-            ref[n > 0] = S[n > 0] / n[n > 0][:, None]
+            # the oracle's update given the GPU's assignment: mean of the keys of each cluster
+            ref = oracle.lloyd_update(inp.K[b, h], inp.centroids[b, h], a_gpu)
             got = cent[b, h].double().cpu().numpy()
             tol = (2.0 ** -8) * np.abs(ref) + 1e-6 if bf16 else 1e-5 * np.abs(ref) + 1e-6
             assert (np.abs(got - ref) <= tol).all(), f"head {h}: {np.abs(got - ref).max()}"
