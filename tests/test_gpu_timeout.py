@@ -3,10 +3,11 @@
 The test build of the library (libda_fault.so: the same sources with DA_FAULT_INJECT) withholds
 one plain software arrival in the fused attention kernel: the second softmax warpgroup of CTA 0
 does not signal that its probabilities of step 5 are written.  Nothing else changes, so no copy or
-product is left in flight.  The MMA issuer waiting for that arrival gives up after the library's
-wait limit (2 s), records DA_ERR_TIMEOUT in the workspace status word and makes the CTA's other
-roles leave (the producers drain their copies first).  The GPU context stays usable: the regular
-library then runs a step on the same process and matches the oracle.
+product is left in flight.  The product issuer waiting for that arrival gives up after the
+library's wait limit (2 s), records DA_ERR_TIMEOUT in the workspace status word and makes the
+CTA's other roles leave (the producers drain their copies first, each drain wait bounded too).
+The GPU context stays usable: the regular library then runs a step on the same process and
+matches the oracle.
 """
 import ctypes
 import os
